@@ -1,0 +1,428 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test ties one oracle function to a closed form, a published table or
+value, a library routine on the special case it reduces to, or brute force,
+chosen so that a plausible mistake (a dropped term, a wrong sign, an
+off-by-one index, a transposed operand) fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy import integrate
+from scipy.stats import norm
+
+from oracle import turboquant_oracle as o
+
+
+# ---------------------------------------------------------------- codebook
+# Mean squared error of the optimal 2/4/8/16-level quantizer of N(0,1).
+# 1 bit: 1 - 2/pi in closed form.  2..4 bits: the values quoted with the
+# method (0.1175, 0.03455, 0.009497), which are Max's 1960 table values; the
+# table's 16-level figure is 0.04% below the exact optimum (0.0095010, found
+# here by closed form and by quadrature), so the tolerance is the printed
+# precision of the table (5e-4 relative).
+DISTORTION = {1: 0.3634, 2: 0.1175, 3: 0.03455, 4: 0.009497}
+
+# Max (1960) / Jayant & Noll: positive half of the optimal Gaussian quantizer.
+MAX_CENTROIDS = {
+    2: [0.4528, 1.510],
+    3: [0.2451, 0.7560, 1.344, 2.152],
+    4: [0.1284, 0.3881, 0.6568, 0.9424, 1.256, 1.618, 2.069, 2.733],
+}
+MAX_THRESHOLDS = {
+    2: [0.0, 0.9816],
+    3: [0.0, 0.5006, 1.050, 1.748],
+    4: [0.0, 0.2582, 0.5224, 0.7996, 1.099, 1.437, 1.844, 2.401],
+}
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_lloyd_max_distortion_matches_published(bits):
+    c = o.lloyd_max_normal(bits)
+    d = o.lloyd_max_distortion(c)
+    assert abs(d - DISTORTION[bits]) / DISTORTION[bits] < 5e-4
+
+
+def test_one_bit_closed_form():
+    c = o.lloyd_max_normal(1)
+    assert np.allclose(c, [-math.sqrt(2 / math.pi), math.sqrt(2 / math.pi)], atol=1e-13)
+    assert abs(o.lloyd_max_distortion(c) - (1 - 2 / math.pi)) < 1e-13
+
+
+def _table_tol(v):
+    """1.5 units of the last of four printed significant digits (half a unit
+    of rounding plus one unit of error in the 1960 hand computation)."""
+    v = abs(v)
+    return 1e-12 if v == 0 else 1.5 * 10.0 ** (math.floor(math.log10(v)) - 3)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_lloyd_max_matches_max_1960_table(bits):
+    c = o.lloyd_max_normal(bits)
+    t = o.thresholds_of(c)
+    for got, want in zip(c[len(c) // 2:], MAX_CENTROIDS[bits]):
+        assert abs(got - want) <= _table_tol(want)
+    for got, want in zip(t[len(t) // 2:], MAX_THRESHOLDS[bits]):
+        assert abs(got - want) <= _table_tol(want)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_centroid_and_nearest_neighbour_conditions_by_quadrature(bits):
+    """Each centroid is its cell's conditional mean (checked by numerical
+    integration, not by the closed form the iteration uses), the codebook is
+    antisymmetric, and the closed-form distortion equals the integral."""
+    c = o.lloyd_max_normal(bits)
+    assert np.array_equal(c, -c[::-1])
+    t = o.thresholds_of(c)
+    edges = np.concatenate(([-np.inf], t, [np.inf]))
+    total = 0.0
+    for j, cj in enumerate(c):
+        mass = integrate.quad(norm.pdf, edges[j], edges[j + 1], epsabs=1e-15)[0]
+        mean = integrate.quad(lambda x: x * norm.pdf(x), edges[j], edges[j + 1], epsabs=1e-15)[0] / mass
+        assert abs(mean - cj) < 1e-10
+        total += integrate.quad(lambda x: (x - cj) ** 2 * norm.pdf(x), edges[j], edges[j + 1],
+                                epsabs=1e-15, epsrel=1e-13)[0]
+    assert abs(total - o.lloyd_max_distortion(c)) < 1e-12
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_distortion_monte_carlo(bits):
+    rng = np.random.default_rng(7 + bits)
+    x = rng.standard_normal(1_000_000)
+    c = o.lloyd_max_normal(bits)
+    t = o.thresholds_of(c)
+    err = (x - c[np.sum(x[:, None] > t[None, :], axis=1)]) ** 2
+    d = o.lloyd_max_distortion(c)
+    assert abs(err.mean() - d) < 5 * err.std() / math.sqrt(x.size)
+
+
+def test_codebook_scaling_and_fp32():
+    d = 128
+    for bits in (2, 3, 4):
+        c, t = o.codebook(bits, d)
+        assert np.array_equal(c, c.astype(np.float32).astype(np.float64))
+        assert np.array_equal(t, t.astype(np.float32).astype(np.float64))
+        assert np.allclose(c * math.sqrt(d), o.lloyd_max_normal(bits), rtol=1e-6)
+        assert np.all(np.diff(c) > 0) and np.all((t > c[:-1]) & (t < c[1:]))
+        assert t[len(t) // 2] == 0.0
+
+
+# ------------------------------------------------------------------- random
+def test_splitmix64_published_values():
+    # First outputs of the reference SplitMix64 for seeds 0 and 1234567.
+    assert o.splitmix64_output(0, 1) == 0xE220A8397B1DCDAF
+    assert [o.splitmix64_output(1234567, i) for i in (1, 2, 3)] == [
+        6457827717110365317, 3203168211198807973, 9817491932198370423]
+
+
+def test_splitmix64_counter_form_equals_sequential_generator():
+    seed = 987654321
+    state = seed
+    for n in range(1, 200):
+        state = (state + o.SPLITMIX_GAMMA) & ((1 << 64) - 1)
+        z = state
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & ((1 << 64) - 1)
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & ((1 << 64) - 1)
+        assert o.splitmix64_output(seed, n) == z ^ (z >> 31)
+
+
+def test_gaussian_stream_moments_and_independence():
+    g0 = o.gaussian_stream(42, o.STREAM_PI, 200_000)
+    g1 = o.gaussian_stream(42, o.STREAM_S, 200_000)
+    for g in (g0, g1):
+        assert abs(g.mean()) < 5 / math.sqrt(g.size)
+        assert abs(g.var() - 1) < 5 * math.sqrt(2 / g.size)
+        assert abs(np.mean(g ** 4) - 3) < 0.05
+    assert abs(np.corrcoef(g0, g1)[0, 1]) < 5 / math.sqrt(g0.size)
+    assert abs(np.corrcoef(g0[:-1], g0[1:])[0, 1]) < 5 / math.sqrt(g0.size)
+    assert np.array_equal(g0[:10], o.gaussian_stream(42, o.STREAM_PI, 10))
+
+
+# ----------------------------------------------------------------- rounding
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    import torch
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(100_000).astype(np.float32).astype(np.float64) * 0.1
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(o.round_to_bf16(x), ref)
+    # exact ties go to the even neighbour
+    assert o.round_to_bf16(1 + 2 ** -8) == 1.0
+    assert o.round_to_bf16(1 + 3 * 2 ** -8) == 1 + 2 ** -6
+
+
+def test_fp16_rounding_matches_numpy_and_saturates():
+    rng = np.random.default_rng(4)
+    x = np.exp(rng.uniform(-20, 11, 100_000)).astype(np.float32).astype(np.float64)
+    x = x[x < 65504]
+    ref = x.astype(np.float32).astype(np.float16).astype(np.float64)
+    assert np.array_equal(o.round_to_fp16_sat(x), ref)
+    assert o.round_to_fp16_sat(1 + 2 ** -11) == 1.0
+    assert o.round_to_fp16_sat(1 + 3 * 2 ** -11) == 1 + 2 ** -9
+    assert o.round_to_fp16_sat(70000.0) == 65504.0
+    assert o.round_to_fp16_sat(1e9) == 65504.0
+    assert o.round_to_fp16_sat(2 ** -25) == 0.0            # tie below the smallest subnormal
+    assert o.round_to_fp16_sat(3 * 2 ** -25) == 2 ** -23
+
+
+# ---------------------------------------------------------------- rotation
+@pytest.mark.parametrize("d,seed", [(128, 42), (64, 7), (16, 1)])
+def test_rotation_is_signed_qr_of_the_seeded_gaussian(d, seed):
+    q = o.rotation_exact(d, seed)
+    g = o.gaussian_stream(seed, o.STREAM_PI, d * d).reshape(d, d)
+    assert np.abs(q.T @ q - np.eye(d)).max() < 1e-12
+    r = q.T @ g                                   # must be R of G = Q R
+    assert np.abs(np.tril(r, -1)).max() < 1e-10
+    assert np.all(np.diag(r) > 0)
+    x = np.random.default_rng(seed).standard_normal((10, d))
+    assert np.allclose(np.linalg.norm(x @ q.T, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+
+
+def test_rotation_bf16_is_near_orthogonal():
+    pi = o.rotation_bf16(128, 42)
+    assert np.array_equal(pi, o.round_to_bf16(pi))
+    err = np.abs(pi.T @ pi - np.eye(128)).max()
+    assert 0 < err < 3e-3
+
+
+def test_rotation_haar_statistics():
+    # Entries of a Haar orthogonal matrix have mean 0 and variance 1/d.
+    d = 64
+    vals = np.concatenate([o.rotation_exact(d, s).ravel() for s in range(1, 6)])
+    assert abs(vals.mean()) < 5 / math.sqrt(vals.size) / math.sqrt(d)
+    assert abs(vals.var() * d - 1) < 0.02
+
+
+def test_qjl_matrix_is_fp32_gaussian():
+    s = o.qjl_matrix(128, 42)
+    assert np.array_equal(s, s.astype(np.float32).astype(np.float64))
+    assert abs(s.mean()) < 0.03 and abs(s.var() - 1) < 0.03
+    assert not np.allclose(s, o.gaussian_stream(42, o.STREAM_PI, 128 * 128).reshape(128, 128))
+
+
+# ---------------------------------------------------------------- quantize
+def _random_bf16_rows(n, d, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return o.round_to_bf16(rng.standard_normal((n, d)) * scale)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantize_picks_nearest_centroid(bits):
+    d = 128
+    pi = o.rotation_bf16(d, 42)
+    c, t = o.codebook(bits, d)
+    x = _random_bf16_rows(2000, d, bits)
+    qz = o.quantize(x, pi, c, t)
+    # brute force: y from an independent formula, nearest centroid by argmin
+    y = (pi @ x.T).T / np.linalg.norm(x, axis=1)[:, None]
+    assert np.allclose(y, qz.y, atol=1e-13)
+    nearest = np.argmin(np.abs(y[:, :, None] - c[None, None, :]), axis=2)
+    # ties are impossible to hit except within fp32 rounding of a midpoint
+    gap = np.min(np.abs(y[:, :, None] - t[None, None, :]), axis=2)
+    ok = (nearest == qz.codes) | (gap < 1e-7)
+    assert ok.all()
+    assert np.array_equal(qz.norm, o.round_to_fp16_sat(np.linalg.norm(x, axis=1)))
+
+
+def test_quantize_zero_vector_and_threshold_tie():
+    d = 128
+    pi = o.rotation_bf16(d, 42)
+    for bits in (2, 3, 4):
+        c, t = o.codebook(bits, d)
+        qz = o.quantize(np.zeros((1, d)), pi, c, t, s_matrix=o.qjl_matrix(d, 42))
+        assert np.all(qz.codes == (1 << (bits - 1)) - 1)
+        assert qz.norm[0] == 0.0
+    # a coordinate exactly on a threshold goes to the lower cell
+    # (x = e_0 has norm exactly 1 and diag(t_5, 1, 1, 1) puts y_0 exactly on t_5)
+    c, t = o.codebook(3, 4)
+    qz = o.quantize(np.array([[1.0, 0.0, 0.0, 0.0]]), np.diag([t[5], 1.0, 1.0, 1.0]), c, t)
+    assert qz.y[0, 0] == t[5] and qz.codes[0, 0] == 5
+    qz = o.quantize(np.array([[1.0, 0.0, 0.0, 0.0]]), np.diag([np.nextafter(t[5], 1), 1.0, 1.0, 1.0]), c, t)
+    assert qz.codes[0, 0] == 6
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantize_distortion_on_unit_vectors(bits):
+    """E||u - Pi^T c[code]||^2 over random unit vectors ~= D_b (Gaussian law
+    approximation of the rotated coordinates; a few percent at d = 128)."""
+    d = 128
+    pi = o.rotation_bf16(d, 11)
+    c, t = o.codebook(bits, d)
+    rng = np.random.default_rng(bits)
+    u = rng.standard_normal((20000, d))
+    u /= np.linalg.norm(u, axis=1)[:, None]
+    qz = o.quantize(u, pi, c, t)
+    recon = c[qz.codes] @ pi
+    mse = np.mean(np.sum((u - recon) ** 2, axis=1))
+    assert abs(mse / DISTORTION[bits] - 1) < 0.04
+
+
+# ----------------------------------------------------------------- packing
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_roundtrip_and_size(bits):
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 1 << bits, size=(500, 128))
+    packed = o.pack_codes(codes, bits)
+    assert packed.shape == (500, 128 * bits // 8)
+    assert np.array_equal(o.unpack_codes(packed, bits, 128), codes)
+    pos = o.code_bit_position(bits, 128)
+    assert np.array_equal(np.sort(pos.ravel()), np.arange(128 * bits))
+
+
+def test_pack_bit_positions_worked_examples():
+    # 2 bits, LSB first: code 3 at coordinate 5 sets bits 10,11 -> byte 1 = 0b00001100
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 5] = 3
+    assert o.pack_codes(codes, 2)[0, 1] == 0b00001100
+    # 4 bits: code 9 at coordinate 3 -> byte 1 high nibble = 9
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 3] = 9
+    assert o.pack_codes(codes, 4)[0, 1] == 0x90
+    # 3 bits: coordinate 10 (word 1, nibble 2) code 5 -> word 1 = 0x500 -> byte 5 = 0x05
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 10] = 5
+    p = o.pack_codes(codes, 3)[0]
+    assert p[5] == 0x05 and p.sum() == 5
+    # 3 bits: coordinate 25 (spare column 1) code 0b101 -> bit 7 of words 0 and 2
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 25] = 0b101
+    p = o.pack_codes(codes, 3)[0]
+    assert p[0] == 0x80 and p[8] == 0x80 and p.sum() == 0x100
+    # 3 bits, second group starts at byte 12
+    codes = np.zeros((1, 128), dtype=np.int64)
+    codes[0, 33] = 7
+    p = o.pack_codes(codes, 3)[0]
+    assert p[12] == 0x70 and p.sum() == 0x70
+    # QJL signs: bit m at position m
+    s = np.zeros((1, 128), dtype=np.int64)
+    s[0, 9] = 1
+    assert o.pack_signs(s)[0, 1] == 0x02
+
+
+# --------------------------------------------------------------------- QJL
+def test_qjl_estimator_is_unbiased_with_predicted_variance():
+    """Over independent Gaussian S, the mean of the estimate equals <q, r>
+    and its variance equals ((pi/2)|q|^2|r|^2 - <q,r>^2)/d."""
+    d = 128
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal(d)
+    r = 0.3 * q / np.linalg.norm(q) + rng.standard_normal(d) * 0.02
+    trials = 12000
+    est = np.empty(trials)
+    for b0 in range(0, trials, 1000):
+        s = rng.standard_normal((1000, d, d))
+        qt = s @ q
+        sg = (s @ r >= 0).astype(np.int64)
+        for k in range(1000):
+            est[b0 + k] = o.qjl_inner_product(qt[k][None, :], sg[k][None, :],
+                                              np.array([np.linalg.norm(r)]), d)[0, 0]
+    exact = q @ r
+    var_pred = ((math.pi / 2) * (q @ q) * (r @ r) - exact ** 2) / d
+    assert abs(est.mean() - exact) < 4 * math.sqrt(var_pred / trials)
+    assert abs(est.var() / var_pred - 1) < 0.05
+
+
+def test_qjl_sign_of_zero_projection_is_plus():
+    # reading: (S r)_m == 0 stores bit 1 (+1); an all-zero S makes every projection 0
+    p = o.Params(128, 3, 3, False, 42)
+    qz = o.quantize(_random_bf16_rows(5, 128, 1), p.pi, p.ck, p.tk, s_matrix=np.zeros((128, 128)))
+    assert np.all(qz.qjl_signs == 1)
+
+
+def test_qjl_quantize_fields():
+    d = 128
+    p = o.Params(d, 2, 2, True, 42)
+    x = _random_bf16_rows(300, d, 9)
+    qz = o.quantize(x, p.pi, p.ck, p.tk, s_matrix=p.s)
+    r = qz.y - p.ck[qz.codes]
+    assert np.allclose(qz.qjl_proj, r @ p.s.T)
+    assert np.array_equal(qz.qjl_signs, (r @ p.s.T >= 0).astype(np.int64))
+    assert np.array_equal(qz.qjl_gamma, o.round_to_fp16_sat(np.linalg.norm(r, axis=1)))
+
+
+# ------------------------------------------------------------------ decode
+def _decode_case(d, t_len, g, bits_k, bits_v, qjl, seed):
+    p = o.Params(d, bits_k, bits_v, qjl, seed)
+    rng = np.random.default_rng(seed)
+    k = o.round_to_bf16(rng.standard_normal((t_len, d)) * rng.lognormal(0, 0.5, (t_len, 1)))
+    v = o.round_to_bf16(rng.standard_normal((t_len, d)))
+    q = rng.standard_normal((g, d))
+    qk = o.quantize(k, p.pi, p.ck, p.tk, s_matrix=p.s)
+    qv = o.quantize(v, p.pi, p.cv, p.tv)
+    return p, q, k, v, qk, qv
+
+
+@pytest.mark.parametrize("qjl", [False, True])
+@pytest.mark.parametrize("bits", [(2, 2), (3, 3), (4, 2)])
+def test_decode_equals_attention_over_explicit_dequantization(bits, qjl):
+    """The rotated-space decode equals plain attention over the vectors
+    reconstructed in the original space: k~ = n Pi^T (c[code] + QJL residual
+    estimate), v~ = n Pi^T c[code] (identity <Pi q, c> = <q, Pi^T c>)."""
+    d = 64
+    p, q, k, v, qk, qv = _decode_case(d, 37, 3, bits[0], bits[1], qjl, 3)
+    scale = 1 / math.sqrt(d)
+    o_dec, lse_dec, _ = o.decode_attention(
+        q, p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, scale,
+        s_matrix=p.s, qjl_signs=qk.qjl_signs, qjl_gamma=qk.qjl_gamma)
+    k_rec = o.dequantize(p.pi, p.ck, qk.codes, qk.norm)
+    if qjl:
+        pm = 2.0 * qk.qjl_signs - 1.0
+        resid_rot = math.sqrt(math.pi / 2) / d * qk.qjl_gamma[:, None] * (pm @ p.s)
+        k_rec = k_rec + qk.norm[:, None] * (resid_rot @ p.pi)
+    v_rec = o.dequantize(p.pi, p.cv, qv.codes, qv.norm)
+    o_ref, lse_ref = o.exact_attention(q, k_rec, v_rec, scale)
+    assert np.allclose(o_dec, o_ref, rtol=1e-11, atol=1e-12)
+    assert np.allclose(lse_dec, lse_ref, rtol=1e-12)
+
+
+def test_decode_single_token_and_equal_scores():
+    d = 32
+    p, q, k, v, qk, qv = _decode_case(d, 1, 2, 3, 3, False, 4)
+    o1, _, _ = o.decode_attention(q, p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, 0.1)
+    assert np.allclose(o1, np.repeat(o.dequantize(p.pi, p.cv, qv.codes, qv.norm), 2, axis=0))
+    # all keys zero -> uniform weights -> mean of the reconstructed values
+    p, q, k, v, qk, qv = _decode_case(d, 9, 2, 3, 3, False, 5)
+    zeros = o.quantize(np.zeros((9, d)), p.pi, p.ck, p.tk)
+    o2, lse, _ = o.decode_attention(q, p.pi, p.ck, zeros.codes, zeros.norm, p.cv, qv.codes, qv.norm, 0.1)
+    assert np.allclose(o2, o.dequantize(p.pi, p.cv, qv.codes, qv.norm).mean(axis=0)[None, :])
+    assert np.allclose(lse, math.log(9))
+
+
+def test_compressed_attention_converges_to_exact_with_bits():
+    """More bits -> attention over the compressed cache approaches attention
+    over the original vectors; error falls roughly as 2^-b."""
+    d = 64
+    rng = np.random.default_rng(8)
+    k = o.round_to_bf16(rng.standard_normal((200, d)))
+    v = o.round_to_bf16(rng.standard_normal((200, d)))
+    q = rng.standard_normal((4, d)) * 2
+    pi = o.rotation_bf16(d, 42)
+    o_ex, _ = o.exact_attention(q, k, v, 1 / math.sqrt(d))
+    errs = []
+    for bits in (2, 3, 4, 5, 6):
+        c, t = o.codebook(bits, d)
+        qk = o.quantize(k, pi, c, t)
+        qv = o.quantize(v, pi, c, t)
+        ob, _, _ = o.decode_attention(q, pi, c, qk.codes, qk.norm, c, qv.codes, qv.norm, 1 / math.sqrt(d))
+        errs.append(np.abs(ob - o_ex).max() / np.abs(o_ex).max())
+    assert all(a > b for a, b in zip(errs, errs[1:]))
+    assert errs[-1] < 0.05 and errs[0] / errs[-1] > 6
+
+
+def test_exact_attention_definition():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((3, 8))
+    k = rng.standard_normal((5, 8))
+    v = rng.standard_normal((5, 8))
+    o_ref, lse = o.exact_attention(q, k, v, 0.5)
+    for g in range(3):
+        s = [0.5 * sum(q[g, i] * k[j, i] for i in range(8)) for j in range(5)]
+        w = [math.exp(x) for x in s]
+        for i in range(8):
+            assert abs(o_ref[g, i] - sum(w[j] * v[j, i] for j in range(5)) / sum(w)) < 1e-12
+        assert abs(lse[g] - math.log(sum(w))) < 1e-12
+
+
+def test_cosine_similarity():
+    assert o.cosine_similarity([1, 0], [2, 0]) == pytest.approx(1.0)
+    assert o.cosine_similarity([1, 0], [0, 3]) == pytest.approx(0.0)
