@@ -1,0 +1,380 @@
+"""Benchmark of the TurboQuant hot path on B200 (one JSON line on rank 0).
+
+Workload (default ``llama8b``): one Llama-3-8B-shaped layer, 8 KV / 32 query
+heads, d = 128, 32768 cached tokens, batch 1, 3-bit K and V (no QJL).  The
+prefill is quantized once into R cache replicas; a *step* is one decode step
+of the whole hot path: quantize-on-append of one new token (8 KV heads, K and
+V) followed by decode attention of the 32 query heads over the packed cache.
+Step i uses replica i % R, so consecutive steps read disjoint memory and the
+step-to-step working set (R x 26 MB) exceeds the 126 MB L2.
+
+``value``  decode-attention effective GB/s: packed K/V bytes the step reads
+           (codes + fp16 norms) / device time per step (CUDA graph of the K
+           timed steps, CUDA events, max over ranks).
+``e2e``    the same metric when every step goes through the C ABI eagerly
+           with pinned host buffers: H2D of the token's K/V and of q, the two
+           calls, D2H of the output.
+``roofline`` the decode call alone, timed with events around each call inside
+           the timed region; algorithmic bytes = packed bytes per call.
+``quantize_*`` prefill quantize of 32768 tokens (input 128 MB > L2): tokens/s,
+           GB/s (bf16 read + packed write) and roofline fraction.
+``cpu_baseline`` the CPU oracle on a bounded sample of the same decode step.
+
+``--impl reference`` times the CPU oracle on the host instead (the reference
+arm: the method has no other implementation to run).  Multi-GPU: one process
+per GPU under torchrun; every rank runs its own replica of the workload
+(the path has no cross-GPU exchange), ``value`` sums the ranks' bytes over
+the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn over packed KV: effective GB/s (% HBM peak); quantize tokens/s"
+WORKLOAD_DESC = ("llama8b: Llama-3-8B-shaped single layer, 8 KV / 32 query heads (GQA 4), d=128, "
+                 "32768 cached tokens, batch 1, bf16 K/V ~ N(0,I) x LogNormal(0,0.5) per (token, head), "
+                 "3-bit K and V (turbo3, no QJL); step = append-quantize 1 token + decode attention")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_cpu_oracle_decode(n_heads_sample: int = 8, seq_len: int = 32768, seed: int = 1002):
+    """The CPU oracle on a bounded sample of the llama8b decode step: unpack
+    the packed codes of `n_heads_sample` KV heads and run the oracle's decode
+    attention for their query heads.  Returns (GB/s-equivalent, seconds,
+    threads used, description)."""
+    import numpy as np
+    from oracle import turboquant_oracle as o
+    from kv_cache_vector_12_b200 import workloads as wl
+    w = wl.WORKLOADS["llama8b"]
+    p = o.Params(w.d, w.bits_k, w.bits_v, False, w.pi_seed)
+    gen = wl.generator("cpu", seed)
+    k, v = wl.kv_tokens(w, seq_len, gen, "cpu")
+    q = wl.queries(w, 1, gen, "cpu").double().numpy()[0]
+    packed = []
+    for h in range(n_heads_sample):
+        qk = o.quantize(k[:, h].double().numpy(), p.pi, p.ck, p.tk)
+        qv = o.quantize(v[:, h].double().numpy(), p.pi, p.cv, p.tv)
+        packed.append((o.pack_codes(qk.codes, w.bits_k), qk.norm, o.pack_codes(qv.codes, w.bits_v), qv.norm))
+    t0 = time.perf_counter()
+    for h, (pk, nk, pv, nv) in enumerate(packed):
+        ck = o.unpack_codes(pk, w.bits_k, w.d)
+        cv = o.unpack_codes(pv, w.bits_v, w.d)
+        o.decode_attention(q[h * w.group:(h + 1) * w.group], p.pi, p.ck, ck, nk, p.cv, cv, nv,
+                           1 / math.sqrt(w.d))
+    dt = time.perf_counter() - t0
+    nbytes = n_heads_sample * seq_len * (w.d * (w.bits_k + w.bits_v) // 8 + 4)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = f"oracle unpack + decode of {n_heads_sample} KV heads x {seq_len} tokens (llama8b decode step, numpy fp64)"
+    return nbytes / dt / 1e9, dt, threads, desc
+
+
+def reference_arm(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    n_heads_sample = 1
+    vals = []
+    for i in range(args.warmup + args.steps):
+        gbs, dt, threads, desc = run_cpu_oracle_decode(n_heads_sample=n_heads_sample, seed=1002 + i % 3)
+        if i >= args.warmup:
+            vals.append((gbs, dt))
+    total_bytes = sum(g * d for g, d in vals)
+    total_t = sum(d for _, d in vals)
+    value = total_bytes / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(vals),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD_DESC, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--replicas", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    from kv_cache_vector_12_b200 import tq
+    from kv_cache_vector_12_b200 import workloads as wl
+    w = wl.WORKLOADS["llama8b"]
+    T, H, HQ, D = w.seq_len, w.n_kv_heads, w.n_q_heads, w.d
+    R = args.replicas
+    n_steps_total = args.warmup + args.steps
+    cap = int(math.ceil((T + n_steps_total + 1) / 64) * 64)
+    ctx = tq.Context(D, w.bits_k, w.bits_v, 0, w.pi_seed)
+    caches = [tq.Cache(ctx, 1, H, cap, device=dev) for _ in range(R)]
+    gen = wl.generator(dev, w.seed + 7919 * rank)
+
+    # ---- prefill quantize (also the quantize measurement) ----
+    k_pre, v_pre = wl.kv_tokens(w, T, gen, dev)
+    seq0 = torch.zeros(T, dtype=torch.int32, device=dev)
+    pos0 = torch.arange(T, dtype=torch.int32, device=dev)
+    for c in caches:
+        tq.quantize(ctx, c, k_pre, v_pre, seq0, pos0)
+    torch.cuda.synchronize()
+    qreps = 10
+    qe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * qreps)]
+    for i in range(qreps):
+        qe[2 * i].record()
+        tq.quantize(ctx, caches[i % R], k_pre, v_pre, seq0, pos0)
+        qe[2 * i + 1].record()
+    torch.cuda.synchronize()
+    q_ms = statistics.median(qe[2 * i].elapsed_time(qe[2 * i + 1]) for i in range(qreps))
+    ctx.check_device_errors()
+
+    # ---- per-step inputs, resident on the device ----
+    k_new, v_new = wl.kv_tokens(w, n_steps_total, gen, dev)           # [steps, H, D]
+    q_all = wl.queries(w, n_steps_total, gen, dev)                     # [steps, HQ, D]
+    pos_steps = torch.empty(n_steps_total, dtype=torch.int32, device=dev)
+    lens_steps = torch.empty(n_steps_total, dtype=torch.int32, device=dev)
+    for i in range(n_steps_total):
+        p = T + i // R
+        pos_steps[i] = p
+        lens_steps[i] = p + 1
+    out = torch.empty(n_steps_total, 1, HQ, D, device=dev)
+    lse = torch.empty(n_steps_total, 1, HQ, device=dev)
+    max_len = cap
+    wsb = tq.alloc_workspace(ctx, 1, HQ, max_len, device=dev)
+    zero_seq = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(i):
+        c = caches[i % R]
+        tq.quantize(ctx, c, k_new[i:i + 1], v_new[i:i + 1], zero_seq, pos_steps[i:i + 1])
+        tq.decode_attention(ctx, c, q_all[i:i + 1], lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+
+    bytes_per_token = H * (D * (w.bits_k + w.bits_v) // 8 + 4)
+    step_bytes = [int(lens_steps[i]) * bytes_per_token for i in range(n_steps_total)]
+
+    # graphs of the warm-up and timed steps
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n_steps_total):       # eager pass before capture
+            step(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm):
+        for i in range(args.warmup):
+            step(i)
+    with torch.cuda.graph(g_timed):
+        for i in range(args.warmup, n_steps_total):
+            step(i)
+    g_warm.replay()
+    torch.cuda.synchronize()
+    ctx.check_device_errors()
+
+    sampler = ClockSampler(local)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    g_timed.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms_total = ev0.elapsed_time(ev1)
+    # decode call alone, events around each call (same stream), same steps
+    de = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    for j, i in enumerate(range(args.warmup, n_steps_total)):
+        c = caches[i % R]
+        tq.quantize(ctx, c, k_new[i:i + 1], v_new[i:i + 1], zero_seq, pos_steps[i:i + 1])
+        de[2 * j].record()
+        tq.decode_attention(ctx, c, q_all[i:i + 1], lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+        de[2 * j + 1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    dec_ms = [de[2 * j].elapsed_time(de[2 * j + 1]) for j in range(args.steps)]
+    ctx.check_device_errors()
+
+    # ---- end to end through the C ABI with pinned host buffers (eager) ----
+    k_h = k_new.cpu().pin_memory()
+    v_h = v_new.cpu().pin_memory()
+    q_h = q_all.cpu().pin_memory()
+    out_h = torch.empty(1, HQ, D).pin_memory()
+    k_d = torch.empty(1, H, D, dtype=torch.bfloat16, device=dev)
+    v_d = torch.empty_like(k_d)
+    q_d = torch.empty(1, HQ, D, dtype=torch.bfloat16, device=dev)
+    h2d = k_d.numel() * 2 * 2 + q_d.numel() * 2
+    d2h = out_h.numel() * 4
+
+    def e2e_step(i):
+        c = caches[i % R]
+        k_d.copy_(k_h[i:i + 1], non_blocking=True)
+        v_d.copy_(v_h[i:i + 1], non_blocking=True)
+        q_d.copy_(q_h[i:i + 1], non_blocking=True)
+        tq.quantize(ctx, c, k_d, v_d, zero_seq, pos_steps[i:i + 1])
+        tq.decode_attention(ctx, c, q_d, lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+        out_h.copy_(out[i], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.warmup, n_steps_total):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    timed_bytes = sum(step_bytes[args.warmup:])
+    if ws > 1:
+        t = torch.tensor([ms_total, e2e_ms, statistics.mean(dec_ms), q_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total, e2e_ms, dec_mean, q_ms = t.tolist()
+    else:
+        dec_mean = statistics.mean(dec_ms)
+    peak, peak_kind = measured_peaks()
+    value = ws * timed_bytes / (ms_total * 1e-3) / 1e9
+    e2e_val = ws * timed_bytes / (e2e_ms * 1e-3) / 1e9
+    dec_achieved = (timed_bytes / args.steps) / (dec_mean * 1e-3) / 1e9
+    q_tokens = T / (q_ms * 1e-3)
+    q_bytes = T * H * (2 * D * 2 + D * (w.bits_k + w.bits_v) // 8 + 4)
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+
+    if rank != 0:
+        if ws > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return 0
+    cpu = None
+    if not args.no_cpu_baseline:
+        gbs, dt, threads, desc = run_cpu_oracle_decode(n_heads_sample=8)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
+                   f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
+                     "frac": dec_achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "kernel": "tq_decode_attention call (rotate_q + split-K attention + merge)",
+                     "algorithmic_bytes_per_call": timed_bytes / args.steps},
+        "quantize": {"tokens_per_s": q_tokens, "GBps": q_gbs, "frac": q_gbs / peak, "ms": q_ms,
+                     "tokens": T, "bytes": q_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        del g_warm, g_timed
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,191 @@
+/*
+ * tq.h - TurboQuant KV-cache compression on NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The method (ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み";
+ * qxai.app, "Tether QVACのTurboQuant実装"): every K/V head vector is split
+ * into its L2 norm and its direction; the direction is rotated by a seeded
+ * random orthogonal matrix Pi, each rotated coordinate is quantized on its own
+ * with the Lloyd-Max quantizer of its (near-Gaussian) law, and no per-block
+ * scale or centroid is stored ("ステップ1: PolarQuant").  An optional second
+ * stage keeps one sign bit per coordinate of S r, the Gaussian projection of
+ * the stage-1 residual r, plus ||r||, which makes inner products unbiased
+ * ("ステップ2: QJL").  Decode attention reads the packed cache directly.
+ *
+ * Conventions for every call below
+ *  - All pointers named "device" are CUDA device pointers on the current
+ *    device; "host" pointers are ordinary host memory.  The caller owns every
+ *    buffer; the library never frees, keeps or allocates caller memory.
+ *  - Compute calls (tq_quantize, tq_decode_attention) are asynchronous on the
+ *    given stream (a cudaStream_t passed as void*; NULL = legacy default
+ *    stream), allocate nothing, never synchronise and never read device data
+ *    on the host.
+ *  - On any non-TQ_OK status nothing has been launched (argument errors) or a
+ *    CUDA call failed (TQ_ERR_CUDA); tq_last_error() returns a thread-local
+ *    message.  Device-side range errors (a seq_idx, pos or seq_len outside the
+ *    cache) skip the offending token or sequence and set a sticky flag that
+ *    tq_check_device_errors() reports.
+ *  - Head dimension d = 128.  bits_k, bits_v in {2, 3, 4}.  qjl in {0, 1}
+ *    (applies to K only).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_ctx tq_ctx; /* opaque: Pi, Pi^T, S, codebooks on one device */
+
+typedef enum tq_status {
+  TQ_OK = 0,
+  TQ_ERR_INVALID = 1,     /* bad argument; nothing launched */
+  TQ_ERR_CUDA = 2,        /* a CUDA runtime call failed */
+  TQ_ERR_NOMEM = 3,       /* device allocation in tq_create failed */
+  TQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (e.g. d != 128) */
+  TQ_ERR_DEVICE = 5       /* a kernel recorded a device-side range error */
+} tq_status;
+
+typedef enum tq_dtype { TQ_BF16 = 0, TQ_F32 = 1 } tq_dtype;
+
+/* Plane indices of tq_layout(). */
+enum {
+  TQ_PLANE_CODES_K = 0,
+  TQ_PLANE_NORM_K = 1,
+  TQ_PLANE_QJL_BITS = 2,
+  TQ_PLANE_QJL_NORM = 3,
+  TQ_PLANE_CODES_V = 4,
+  TQ_PLANE_NORM_V = 5
+};
+
+/*
+ * The packed cache of one attention layer: six planes of caller-owned device
+ * memory, each laid out [n_seqs][n_kv_heads][capacity][bytes_per_token_head]
+ * (so the tokens of one (sequence, KV head) are contiguous).
+ *  codes_k  d*bits_k/8 bytes per vector.  2 and 4 bits: LSB-first stream,
+ *           code i at bits [i*b, i*b+b).  3 bits: groups of 32 coordinates in
+ *           three little-endian 32-bit words w0..w2; local coordinate l < 24
+ *           occupies bits [4(l%8), 4(l%8)+3) of word l/8, and bit k of the
+ *           code of l >= 24 is bit 4(l-24)+3 of word k.  A code is the index
+ *           of its centroid in ascending order.
+ *  norm_k   ||k|| as IEEE fp16 bits (round to nearest even, saturating).
+ *  qjl_bits d/8 bytes, bit m = [(S r)_m >= 0], LSB first (NULL if qjl == 0).
+ *  qjl_norm ||r|| as fp16 bits (NULL if qjl == 0).
+ *  codes_v, norm_v as codes_k, norm_k with bits_v.
+ * capacity must be a positive multiple of 64; every plane pointer 16-byte
+ * aligned.
+ */
+typedef struct tq_cache {
+  uint8_t *codes_k;
+  uint16_t *norm_k;
+  uint8_t *qjl_bits;
+  uint16_t *qjl_norm;
+  uint8_t *codes_v;
+  uint16_t *norm_v;
+  int32_t capacity;
+  int32_t n_seqs;
+  int32_t n_kv_heads;
+} tq_cache;
+
+/*
+ * Create a context on the current CUDA device.  Pi is the QR factor of a
+ * d x d Gaussian (SplitMix64 counters 1.. from `seed`, Box-Muller), columns
+ * signed so that R has a positive diagonal, rounded to bf16 (the "random
+ * orthogonal matrix" of "ステップ1: PolarQuant").  The codebook of b bits is
+ * the Lloyd-Max quantizer of N(0,1) scaled by 1/sqrt(d) ("Lloyd-Max量子化";
+ * the N(0,1/d) law is the "ガウス分布に近い" coordinate law) in fp32, with
+ * fp32 midpoints as thresholds.  With qjl, S is a second d x d Gaussian from
+ * counters 2^32+1.. (fp32).  Allocates and uploads the parameters
+ * (synchronous); the only call that allocates device memory.
+ * Errors: TQ_ERR_INVALID (null out, bits outside {2,3,4}, qjl outside {0,1}),
+ * TQ_ERR_UNSUPPORTED (d != 128), TQ_ERR_NOMEM, TQ_ERR_CUDA.
+ */
+tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v,
+                    int32_t qjl, uint64_t seed);
+
+/* Free the context's device memory.  NULL is a no-op. */
+void tq_destroy(tq_ctx *ctx);
+
+/* Bytes per (token, KV head) of each plane, indexed by TQ_PLANE_* (0 for the
+ * QJL planes when qjl == 0).  Host array of 6. */
+tq_status tq_layout(const tq_ctx *ctx, size_t bytes_per_token_head[6]);
+
+/*
+ * Copy the method's parameters to host memory (any pointer may be NULL):
+ * pi [d*d] row-major (z = Pi x), values exactly representable in bf16;
+ * s [d*d] row-major (NULL result if qjl == 0); centroids_* [2^bits]
+ * ascending; thresholds_* [2^bits - 1].
+ */
+tq_status tq_get_params(const tq_ctx *ctx, float *pi, float *s,
+                        float *centroids_k, float *thresholds_k,
+                        float *centroids_v, float *thresholds_v);
+
+/*
+ * The same parameters computed on the host only (no CUDA call): what
+ * tq_create(d, bits_k, bits_v, qjl, seed) would upload.  Same output layout
+ * as tq_get_params; s is left untouched when qjl == 0.
+ */
+tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v,
+                         int32_t qjl, uint64_t seed, float *pi, float *s,
+                         float *centroids_k, float *thresholds_k,
+                         float *centroids_v, float *thresholds_v);
+
+/*
+ * Quantize-on-append ("ステップ1" and, with qjl, "ステップ2"): for each of
+ * n_tok tokens t and KV head h, k[t][h][:] and v[t][h][:] (device, bf16,
+ * contiguous [n_tok][n_kv_heads][d]) are normed, rotated by Pi, quantized,
+ * packed and written at position pos[t] of sequence seq_idx[t] (device int32
+ * arrays of n_tok).  Rows whose (seq_idx, pos) falls outside the cache are
+ * skipped and flagged.  Tokens may arrive in any order; two tokens with the
+ * same (seq_idx, pos) race.  n_tok == 0 is a no-op.
+ */
+tq_status tq_quantize(tq_ctx *ctx, const tq_cache *cache, const void *k,
+                      const void *v, const int32_t *seq_idx,
+                      const int32_t *pos, int32_t n_tok, void *stream);
+
+/* Device workspace (bytes) that tq_decode_attention needs for this shape. */
+size_t tq_workspace_bytes(const tq_ctx *ctx, int32_t n_seqs,
+                          int32_t n_q_heads, int32_t max_seq_len);
+
+/*
+ * Decode attention over the packed cache: for every sequence s and query
+ * head g (KV head g / (n_q_heads / n_kv_heads)),
+ *   q_hat = Pi q, q_tilde = S q_hat,
+ *   score_j = scale * ||k_j|| * (q_hat . c_K[code_j]
+ *             + [qjl] sqrt(pi/2)/d * ||r_j|| * sum_m q_tilde_m (2 s_jm - 1)),
+ *   o = Pi^T sum_j softmax(score)_j ||v_j|| c_V[codeV_j]
+ * over the positions [0, seq_lens[s]).  q: device [n_seqs][n_q_heads][d] of
+ * q_dtype (TQ_BF16 or TQ_F32).  seq_lens: device int32 [n_seqs], each at most
+ * max_seq_len (a host bound used to size the grid; <= capacity).
+ * scale <= 0 means 1/sqrt(d).  out: device fp32 [n_seqs][n_q_heads][d].
+ * lse: device fp32 [n_seqs][n_q_heads] log-sum-exp of the scores, or NULL.
+ * A sequence of length 0 yields out = 0 and lse = -inf.  workspace: device,
+ * at least tq_workspace_bytes(ctx, n_seqs, n_q_heads, max_seq_len) bytes,
+ * 256-byte aligned; its contents need no initialisation.
+ */
+tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache,
+                              const void *q, int32_t q_dtype,
+                              int32_t n_q_heads, const int32_t *seq_lens,
+                              int32_t max_seq_len, float scale, float *out,
+                              float *lse, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronise `stream`, then report and clear the context's sticky
+ * device-side error flags: TQ_OK, or TQ_ERR_DEVICE with a message naming the
+ * flags (bit 0: token outside the cache in tq_quantize; bit 1: seq_len
+ * outside [0, max_seq_len] in tq_decode_attention; bit 2: a bounded wait in a
+ * kernel expired).
+ */
+tq_status tq_check_device_errors(tq_ctx *ctx, void *stream);
+
+/* Thread-local message describing the last non-TQ_OK status ("" if none). */
+const char *tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

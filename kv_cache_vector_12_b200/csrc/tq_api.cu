@@ -1,0 +1,310 @@
+// C ABI of the TurboQuant library: context lifetime, argument validation and
+// the dispatch of the compute calls to their kernels.  Validation happens
+// entirely on the host, before anything is launched; device-side range
+// problems are recorded in a sticky flag word instead of faulting.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "tq_internal.h"
+
+struct tq_ctx {
+  int device;
+  int d, bits_k, bits_v, qjl;
+  uint64_t seed;
+  std::vector<uint16_t> pi_bits;  // host copies of the uploaded parameters
+  std::vector<float> s, ck, tk, cv, tv;
+  void *dev_block;                // one allocation holding every device parameter
+  tq::DeviceParams dp;
+};
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+tq_status fail(tq_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+tq_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+tq_status check_params(int d, int bits_k, int bits_v, int qjl) {
+  if (bits_k < 2 || bits_k > 4 || bits_v < 2 || bits_v > 4)
+    return fail(TQ_ERR_INVALID, "bits_k=%d bits_v=%d: each must be 2, 3 or 4", bits_k, bits_v);
+  if (qjl != 0 && qjl != 1) return fail(TQ_ERR_INVALID, "qjl=%d must be 0 or 1", qjl);
+  if (d != tq::kHeadDim) return fail(TQ_ERR_UNSUPPORTED, "d=%d: only d=128 is implemented", d);
+  return TQ_OK;
+}
+
+tq_status check_cache(const tq_ctx *ctx, const tq_cache *c) {
+  if (!c) return fail(TQ_ERR_INVALID, "cache is NULL");
+  if (c->capacity <= 0 || c->capacity % 64 != 0)
+    return fail(TQ_ERR_INVALID, "capacity=%d must be a positive multiple of 64", c->capacity);
+  if (c->n_seqs <= 0 || c->n_kv_heads <= 0)
+    return fail(TQ_ERR_INVALID, "n_seqs=%d n_kv_heads=%d must be positive", c->n_seqs, c->n_kv_heads);
+  const void *planes[6] = {c->codes_k, c->norm_k, c->qjl_bits, c->qjl_norm, c->codes_v, c->norm_v};
+  for (int i = 0; i < 6; ++i) {
+    const bool needed = (i != 2 && i != 3) || ctx->qjl;
+    if (needed && !planes[i]) return fail(TQ_ERR_INVALID, "cache plane %d is NULL", i);
+    if (planes[i] && !aligned16(planes[i]))
+      return fail(TQ_ERR_INVALID, "cache plane %d is not 16-byte aligned", i);
+  }
+  return TQ_OK;
+}
+
+}  // namespace
+
+namespace tq {
+
+DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len) {
+  // Enough (sequence, KV head, split) work items to fill 148 SMs several
+  // times over, with splits of at least 256 tokens.
+  const long units = (long)n_seqs * n_kv_heads;
+  const long target_items = 148L * 8;
+  long per_unit = (target_items + units - 1) / units;
+  long chunk = per_unit > 0 ? ((long)max_seq_len + per_unit - 1) / per_unit : max_seq_len;
+  if (chunk < 256) chunk = 256;
+  chunk = (chunk + 63) / 64 * 64;
+  DecodeSplit s;
+  s.chunk = (int)chunk;
+  s.n_splits = max_seq_len > 0 ? (int)(((long)max_seq_len + chunk - 1) / chunk) : 1;
+  if (s.n_splits < 1) s.n_splits = 1;
+  return s;
+}
+
+DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, int qjl, DecodeSplit split) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t rows = (size_t)n_seqs * n_q_heads;
+  DecodeWorkspace w;
+  w.q_hat = 0;
+  w.q_tilde = up(rows * kHeadDim * sizeof(float));
+  w.partials = w.q_tilde + (qjl ? up(rows * kHeadDim * sizeof(float)) : 0);
+  w.total = w.partials + up(rows * (size_t)split.n_splits * (kHeadDim + 2) * sizeof(float));
+  return w;
+}
+
+}  // namespace tq
+
+extern "C" {
+
+const char *tq_last_error(void) { return g_last_error; }
+
+tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl, uint64_t seed,
+                         float *pi, float *s, float *centroids_k, float *thresholds_k,
+                         float *centroids_v, float *thresholds_v) {
+  tq_status st = check_params(d, bits_k, bits_v, qjl);
+  if (st != TQ_OK) return st;
+  if (pi) {
+    std::vector<uint16_t> bits((size_t)d * d);
+    tq::rotation_bf16(d, seed, bits.data());
+    for (size_t i = 0; i < bits.size(); ++i) pi[i] = tq::bf16_bits_to_float(bits[i]);
+  }
+  if (s && qjl) tq::qjl_matrix(d, seed, s);
+  float c[tq::kMaxLevels], t[tq::kMaxLevels];
+  if (centroids_k || thresholds_k) {
+    tq::codebook(bits_k, d, c, t);
+    if (centroids_k) std::memcpy(centroids_k, c, sizeof(float) << bits_k);
+    if (thresholds_k) std::memcpy(thresholds_k, t, sizeof(float) * ((1 << bits_k) - 1));
+  }
+  if (centroids_v || thresholds_v) {
+    tq::codebook(bits_v, d, c, t);
+    if (centroids_v) std::memcpy(centroids_v, c, sizeof(float) << bits_v);
+    if (thresholds_v) std::memcpy(thresholds_v, t, sizeof(float) * ((1 << bits_v) - 1));
+  }
+  return TQ_OK;
+}
+
+tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
+                    uint64_t seed) {
+  if (!out) return fail(TQ_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  tq_status st = check_params(d, bits_k, bits_v, qjl);
+  if (st != TQ_OK) return st;
+
+  tq_ctx *ctx = new tq_ctx();
+  ctx->d = d;
+  ctx->bits_k = bits_k;
+  ctx->bits_v = bits_v;
+  ctx->qjl = qjl;
+  ctx->seed = seed;
+  ctx->dev_block = nullptr;
+  ctx->pi_bits.resize((size_t)d * d);
+  tq::rotation_bf16(d, seed, ctx->pi_bits.data());
+  ctx->ck.assign(tq::kMaxLevels, 0.f);
+  ctx->tk.assign(tq::kMaxLevels, 0.f);
+  ctx->cv.assign(tq::kMaxLevels, 0.f);
+  ctx->tv.assign(tq::kMaxLevels, 0.f);
+  tq::codebook(bits_k, d, ctx->ck.data(), ctx->tk.data());
+  tq::codebook(bits_v, d, ctx->cv.data(), ctx->tv.data());
+  if (qjl) {
+    ctx->s.resize((size_t)d * d);
+    tq::qjl_matrix(d, seed, ctx->s.data());
+  }
+
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e != cudaSuccess) {
+    delete ctx;
+    return cuda_fail(e, "cudaGetDevice");
+  }
+  // One block: pi | pit | s | st | codebooks | error word.
+  const size_t dd = (size_t)d * d;
+  const size_t off_pi = 0, off_pit = off_pi + dd * 2, off_s = off_pit + dd * 2;
+  const size_t off_st = off_s + dd * 4, off_cb = off_st + dd * 4;
+  const size_t off_err = off_cb + 4 * tq::kMaxLevels * 4, total = off_err + 256;
+  e = cudaMalloc(&ctx->dev_block, total);
+  if (e != cudaSuccess) {
+    delete ctx;
+    return fail(TQ_ERR_NOMEM, "cudaMalloc(%zu): %s", total, cudaGetErrorString(e));
+  }
+  std::vector<char> h(total, 0);
+  std::memcpy(h.data() + off_pi, ctx->pi_bits.data(), dd * 2);
+  uint16_t *pit = (uint16_t *)(h.data() + off_pit);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) pit[(size_t)j * d + i] = ctx->pi_bits[(size_t)i * d + j];
+  if (qjl) {
+    std::memcpy(h.data() + off_s, ctx->s.data(), dd * 4);
+    float *st_h = (float *)(h.data() + off_st);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) st_h[(size_t)j * d + i] = ctx->s[(size_t)i * d + j];
+  }
+  float *cb = (float *)(h.data() + off_cb);
+  std::memcpy(cb + 0 * tq::kMaxLevels, ctx->ck.data(), tq::kMaxLevels * 4);
+  std::memcpy(cb + 1 * tq::kMaxLevels, ctx->tk.data(), tq::kMaxLevels * 4);
+  std::memcpy(cb + 2 * tq::kMaxLevels, ctx->cv.data(), tq::kMaxLevels * 4);
+  std::memcpy(cb + 3 * tq::kMaxLevels, ctx->tv.data(), tq::kMaxLevels * 4);
+  e = cudaMemcpy(ctx->dev_block, h.data(), total, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(ctx->dev_block);
+    delete ctx;
+    return cuda_fail(e, "cudaMemcpy(params)");
+  }
+  char *base = (char *)ctx->dev_block;
+  ctx->dp.pi = (const uint16_t *)(base + off_pi);
+  ctx->dp.pit = (const uint16_t *)(base + off_pit);
+  ctx->dp.s = (const float *)(base + off_s);
+  ctx->dp.st = (const float *)(base + off_st);
+  ctx->dp.cb = (const float *)(base + off_cb);
+  ctx->dp.err = (unsigned *)(base + off_err);
+  ctx->dp.bits_k = bits_k;
+  ctx->dp.bits_v = bits_v;
+  ctx->dp.qjl = qjl;
+  *out = ctx;
+  return TQ_OK;
+}
+
+void tq_destroy(tq_ctx *ctx) {
+  if (!ctx) return;
+  if (ctx->dev_block) cudaFree(ctx->dev_block);
+  delete ctx;
+}
+
+tq_status tq_layout(const tq_ctx *ctx, size_t b[6]) {
+  if (!ctx || !b) return fail(TQ_ERR_INVALID, "ctx or output is NULL");
+  b[TQ_PLANE_CODES_K] = (size_t)tq::code_bytes(ctx->bits_k);
+  b[TQ_PLANE_NORM_K] = 2;
+  b[TQ_PLANE_QJL_BITS] = ctx->qjl ? tq::kHeadDim / 8 : 0;
+  b[TQ_PLANE_QJL_NORM] = ctx->qjl ? 2 : 0;
+  b[TQ_PLANE_CODES_V] = (size_t)tq::code_bytes(ctx->bits_v);
+  b[TQ_PLANE_NORM_V] = 2;
+  return TQ_OK;
+}
+
+tq_status tq_get_params(const tq_ctx *ctx, float *pi, float *s, float *centroids_k,
+                        float *thresholds_k, float *centroids_v, float *thresholds_v) {
+  if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
+  const size_t dd = (size_t)ctx->d * ctx->d;
+  if (pi)
+    for (size_t i = 0; i < dd; ++i) pi[i] = tq::bf16_bits_to_float(ctx->pi_bits[i]);
+  if (s && ctx->qjl) std::memcpy(s, ctx->s.data(), dd * 4);
+  if (centroids_k) std::memcpy(centroids_k, ctx->ck.data(), sizeof(float) << ctx->bits_k);
+  if (thresholds_k) std::memcpy(thresholds_k, ctx->tk.data(), sizeof(float) * ((1 << ctx->bits_k) - 1));
+  if (centroids_v) std::memcpy(centroids_v, ctx->cv.data(), sizeof(float) << ctx->bits_v);
+  if (thresholds_v) std::memcpy(thresholds_v, ctx->tv.data(), sizeof(float) * ((1 << ctx->bits_v) - 1));
+  return TQ_OK;
+}
+
+tq_status tq_quantize(tq_ctx *ctx, const tq_cache *cache, const void *k, const void *v,
+                      const int32_t *seq_idx, const int32_t *pos, int32_t n_tok, void *stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
+  tq_status st = check_cache(ctx, cache);
+  if (st != TQ_OK) return st;
+  if (n_tok < 0) return fail(TQ_ERR_INVALID, "n_tok=%d is negative", n_tok);
+  if (n_tok == 0) return TQ_OK;
+  if (!k || !v || !seq_idx || !pos) return fail(TQ_ERR_INVALID, "k, v, seq_idx and pos must be non-NULL");
+  if (!aligned16(k) || !aligned16(v)) return fail(TQ_ERR_INVALID, "k and v must be 16-byte aligned");
+  if (((uintptr_t)seq_idx & 3u) || ((uintptr_t)pos & 3u))
+    return fail(TQ_ERR_INVALID, "seq_idx and pos must be 4-byte aligned");
+  const int e = tq::launch_quantize(ctx->dp, *cache, k, v, seq_idx, pos, n_tok, stream);
+  if (e != 0) return cuda_fail((cudaError_t)e, "tq_quantize launch");
+  return TQ_OK;
+}
+
+size_t tq_workspace_bytes(const tq_ctx *ctx, int32_t n_seqs, int32_t n_q_heads, int32_t max_seq_len) {
+  if (!ctx || n_seqs <= 0 || n_q_heads <= 0 || max_seq_len < 0) return 0;
+  // The split depends on n_kv_heads only through the item count; size for the
+  // worst case (one KV head per query head).
+  const tq::DecodeSplit sp = tq::decode_split(n_seqs, 1, max_seq_len);
+  return tq::decode_workspace(n_seqs, n_q_heads, ctx->qjl, sp).total;
+}
+
+tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q, int32_t q_dtype,
+                              int32_t n_q_heads, const int32_t *seq_lens, int32_t max_seq_len,
+                              float scale, float *out, float *lse, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
+  tq_status st = check_cache(ctx, cache);
+  if (st != TQ_OK) return st;
+  if (!q || !seq_lens || !out || !workspace)
+    return fail(TQ_ERR_INVALID, "q, seq_lens, out and workspace must be non-NULL");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID, "q_dtype=%d", q_dtype);
+  if (n_q_heads <= 0 || n_q_heads % cache->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "n_q_heads=%d must be a positive multiple of n_kv_heads=%d",
+                n_q_heads, cache->n_kv_heads);
+  if (n_q_heads / cache->n_kv_heads > 16)
+    return fail(TQ_ERR_UNSUPPORTED, "query heads per KV head = %d > 16", n_q_heads / cache->n_kv_heads);
+  if (max_seq_len < 0 || max_seq_len > cache->capacity)
+    return fail(TQ_ERR_INVALID, "max_seq_len=%d outside [0, capacity=%d]", max_seq_len, cache->capacity);
+  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u) || ((uintptr_t)seq_lens & 3u) ||
+      (lse && ((uintptr_t)lse & 3u)))
+    return fail(TQ_ERR_INVALID, "misaligned q/out (16 B), workspace (256 B) or seq_lens/lse (4 B)");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
+  const tq::DecodeSplit sp = tq::decode_split(cache->n_seqs, cache->n_kv_heads, max_seq_len);
+  const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, ctx->qjl, sp);
+  if (workspace_bytes < ws.total)
+    return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, ws.total);
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)ctx->d);
+  const int e = tq::launch_decode(ctx->dp, *cache, q, q_dtype, n_q_heads, seq_lens, max_seq_len, scale,
+                                  out, lse, (char *)workspace, sp, ws, stream);
+  if (e != 0) return cuda_fail((cudaError_t)e, "tq_decode_attention launch");
+  return TQ_OK;
+}
+
+tq_status tq_check_device_errors(tq_ctx *ctx, void *stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned flags = 0;
+  e = cudaMemcpy(&flags, ctx->dp.err, sizeof flags, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error flags");
+  if (!flags) return TQ_OK;
+  e = cudaMemset(ctx->dp.err, 0, sizeof flags);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error flags");
+  return fail(TQ_ERR_DEVICE, "device error flags 0x%x%s%s%s", flags,
+              (flags & tq::kErrTokenRange) ? " [token outside cache]" : "",
+              (flags & tq::kErrSeqLen) ? " [seq_len outside range]" : "",
+              (flags & tq::kErrWaitExpired) ? " [bounded wait expired]" : "");
+}
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+// Host-side construction of the method's fixed parameters: the rotation Pi,
+// the QJL projection S and the Lloyd-Max codebooks.
+//
+// Rotation: "ランダムな直交行列を掛けて「回転」" (ai-accelerate.xyz TurboQuant
+// explainer, "ステップ1: PolarQuant").  Pi is the Q factor of a seeded
+// Gaussian matrix, made unique by a positive diagonal of R, then rounded to
+// bf16: the bf16 matrix is the one both quantize and decode use.
+//
+// Codebook: "各次元を独立に最適なスカラー量子化（Lloyd-Max量子化）" (same
+// section).  Lloyd's iteration on N(0,1), scaled by 1/sqrt(d) for the
+// N(0,1/d) law of a rotated unit vector's coordinates.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+// SplitMix64 (Steele, Lea & Flood 2014) read as a counter-based generator:
+// output n (n >= 1) of the generator seeded with `seed` is the variant-13
+// finaliser applied to seed + n * 0x9E3779B97F4A7C15.
+static inline uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ULL;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+// `count` standard normals of stream `stream` (Pi: 0, S: 1).  Box-Muller on
+// 53-bit uniforms: pair p uses counters base+2p+1 (u1 in (0,1]) and
+// base+2p+2 (u2 in [0,1)); element e is component e%2 of pair e/2.
+void gaussian_stream(uint64_t seed, uint32_t stream, size_t count, double *out) {
+  const uint64_t base = (uint64_t)stream << 32;
+  const double inv53 = 1.0 / 9007199254740992.0;
+  const double two_pi = 2.0 * M_PI;
+  for (size_t p = 0; 2 * p < count; ++p) {
+    const uint64_t a = splitmix64_at(seed, base + 2 * p + 1);
+    const uint64_t b = splitmix64_at(seed, base + 2 * p + 2);
+    const double u1 = (double)((a >> 11) + 1) * inv53;
+    const double u2 = (double)(b >> 11) * inv53;
+    const double r = std::sqrt(-2.0 * std::log(u1));
+    const double theta = two_pi * u2;
+    out[2 * p] = r * std::cos(theta);
+    if (2 * p + 1 < count) out[2 * p + 1] = r * std::sin(theta);
+  }
+}
+
+// Round a double to the nearest bfloat16 (ties to even) by clearing the 45
+// low mantissa bits of the double with carry; returns the bf16 bit pattern.
+uint16_t double_to_bf16_bits(double x) {
+  uint64_t u;
+  std::memcpy(&u, &x, 8);
+  const uint64_t drop = 45;
+  const uint64_t lsb = (u >> drop) & 1u;
+  u += ((uint64_t)1 << (drop - 1)) - 1 + lsb;
+  u &= ~(((uint64_t)1 << drop) - 1);
+  double r;
+  std::memcpy(&r, &u, 8);
+  const float f = (float)r;  // exact: 8 significant bits in fp32's range
+  uint32_t fb;
+  std::memcpy(&fb, &f, 4);
+  return (uint16_t)(fb >> 16);
+}
+
+float bf16_bits_to_float(uint16_t h) {
+  const uint32_t fb = (uint32_t)h << 16;
+  float f;
+  std::memcpy(&f, &fb, 4);
+  return f;
+}
+
+// Householder QR of the n x n row-major matrix a (overwritten).  Returns Q
+// (row-major) with every column multiplied by the sign of R's diagonal entry,
+// i.e. the unique Q whose R has a positive diagonal.
+static std::vector<double> signed_householder_q(std::vector<double> a, int n) {
+  std::vector<std::vector<double>> vs(n);
+  std::vector<double> rdiag(n);
+  for (int k = 0; k < n; ++k) {
+    double norm2 = 0.0;
+    for (int i = k; i < n; ++i) norm2 += a[(size_t)i * n + k] * a[(size_t)i * n + k];
+    const double norm = std::sqrt(norm2);
+    const double x0 = a[(size_t)k * n + k];
+    const double alpha = x0 >= 0.0 ? -norm : norm;  // R_kk
+    std::vector<double> v(n - k);
+    for (int i = k; i < n; ++i) v[i - k] = a[(size_t)i * n + k];
+    v[0] -= alpha;
+    double vn2 = 0.0;
+    for (double e : v) vn2 += e * e;
+    if (vn2 > 0.0) {
+      const double inv = 1.0 / std::sqrt(vn2);
+      for (double &e : v) e *= inv;
+      for (int j = k; j < n; ++j) {  // A[k:, k:] -= 2 v (v^T A[k:, k:])
+        double dot = 0.0;
+        for (int i = k; i < n; ++i) dot += v[i - k] * a[(size_t)i * n + j];
+        for (int i = k; i < n; ++i) a[(size_t)i * n + j] -= 2.0 * v[i - k] * dot;
+      }
+    }
+    rdiag[k] = vn2 > 0.0 ? alpha : x0;
+    vs[k] = std::move(v);
+  }
+  // Q = H_0 H_1 ... H_{n-1}: apply the reflections to I from the last one.
+  std::vector<double> q((size_t)n * n, 0.0);
+  for (int i = 0; i < n; ++i) q[(size_t)i * n + i] = 1.0;
+  for (int k = n - 1; k >= 0; --k) {
+    const std::vector<double> &v = vs[k];
+    double vn2 = 0.0;
+    for (double e : v) vn2 += e * e;
+    if (vn2 == 0.0) continue;
+    for (int j = 0; j < n; ++j) {
+      double dot = 0.0;
+      for (int i = k; i < n; ++i) dot += v[i - k] * q[(size_t)i * n + j];
+      for (int i = k; i < n; ++i) q[(size_t)i * n + j] -= 2.0 * v[i - k] * dot;
+    }
+  }
+  for (int j = 0; j < n; ++j)
+    if (rdiag[j] < 0.0)
+      for (int i = 0; i < n; ++i) q[(size_t)i * n + j] = -q[(size_t)i * n + j];
+  return q;
+}
+
+void rotation_bf16(int d, uint64_t seed, uint16_t *pi_bits) {
+  std::vector<double> g((size_t)d * d);
+  gaussian_stream(seed, 0, g.size(), g.data());
+  const std::vector<double> q = signed_householder_q(std::move(g), d);
+  for (size_t i = 0; i < q.size(); ++i) pi_bits[i] = double_to_bf16_bits(q[i]);
+}
+
+void qjl_matrix(int d, uint64_t seed, float *s) {
+  std::vector<double> g((size_t)d * d);
+  gaussian_stream(seed, 1, g.size(), g.data());
+  for (size_t i = 0; i < g.size(); ++i) s[i] = (float)g[i];
+}
+
+// Standard normal density and the probability of (a, b], computed on the
+// side of zero that avoids cancellation.
+static double npdf(double x) {
+  return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) * 0.3989422804014327;
+}
+static double nmass(double a, double b) {
+  if (a >= 0.0) return 0.5 * std::erfc(a * M_SQRT1_2) - 0.5 * std::erfc(b * M_SQRT1_2);
+  return 0.5 * std::erfc(-b * M_SQRT1_2) - 0.5 * std::erfc(-a * M_SQRT1_2);
+}
+
+// Lloyd-Max centroids of N(0,1) with 2^bits levels, ascending.  Starts from
+// evenly spaced centroids on [-2, 2] and alternates the two optimality
+// conditions (thresholds at midpoints, centroids at conditional means) until
+// no centroid moves by more than 1e-15; then symmetrises exactly.
+void lloyd_max_gaussian(int bits, double *c) {
+  const int L = 1 << bits;
+  for (int j = 0; j < L; ++j) c[j] = -2.0 + 4.0 * (j + 0.5) / L;
+  std::vector<double> t(L + 1), nc(L);
+  for (int it = 0; it < 2000000; ++it) {
+    t[0] = -INFINITY;
+    t[L] = INFINITY;
+    for (int j = 1; j < L; ++j) t[j] = 0.5 * (c[j - 1] + c[j]);
+    double move = 0.0;
+    for (int j = 0; j < L; ++j) {
+      nc[j] = (npdf(t[j]) - npdf(t[j + 1])) / nmass(t[j], t[j + 1]);
+      move = std::fmax(move, std::fabs(nc[j] - c[j]));
+    }
+    for (int j = 0; j < L; ++j) c[j] = nc[j];
+    if (move <= 1e-15) break;
+  }
+  for (int j = 0; j < L / 2; ++j) {
+    const double m = 0.5 * (c[L - 1 - j] - c[j]);
+    c[j] = -m;
+    c[L - 1 - j] = m;
+  }
+}
+
+void codebook(int bits, int d, float *centroids, float *thresholds) {
+  const int L = 1 << bits;
+  std::vector<double> c(L);
+  lloyd_max_gaussian(bits, c.data());
+  const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
+  for (int j = 0; j < L; ++j) centroids[j] = (float)(c[j] * inv_sqrt_d);
+  for (int j = 0; j + 1 < L; ++j)
+    thresholds[j] = (float)(0.5 * ((double)centroids[j] + (double)centroids[j + 1]));
+}
+
+}  // namespace tq

@@ -1,0 +1,294 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs, at sizes that span several tiles and a ragged tail."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import turboquant_oracle as o
+from tests import parity_helpers as ph
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+SETTINGS = [(3, 3, 0), (2, 2, 0), (4, 4, 0), (2, 4, 1), (4, 2, 1), (3, 3, 1)]
+
+
+@pytest.fixture(scope="module")
+def tq(cuda_device):
+    from kv_cache_vector_12_b200 import tq as tqmod
+    return tqmod
+
+
+_PARAMS = {}
+
+
+def oracle_params(bits_k, bits_v, qjl, seed=42):
+    key = (bits_k, bits_v, qjl, seed)
+    if key not in _PARAMS:
+        _PARAMS[key] = o.Params(D, bits_k, bits_v, bool(qjl), seed)
+    return _PARAMS[key]
+
+
+def make_rows(n, h, seed, lognormal=True):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(n, h, D, generator=g)
+    if lognormal:
+        x = x * torch.exp(0.5 * torch.randn(n, h, 1, generator=g))
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl", SETTINGS)
+def test_device_params_match_oracle(tq, bits_k, bits_v, qjl):
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
+    p = ctx.params()
+    ref = oracle_params(bits_k, bits_v, qjl)
+    assert np.array_equal(p["pi"].double().numpy(), ref.pi)
+    assert np.array_equal(p["centroids_k"].double().numpy(), ref.ck)
+    assert np.array_equal(p["thresholds_v"].double().numpy(), ref.tv)
+    if qjl:
+        assert np.array_equal(p["s"].double().numpy(), ref.s)
+
+
+def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0):
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
+    ref = oracle_params(bits_k, bits_v, qjl)
+    k = make_rows(n_tok, n_heads, seed)
+    v = make_rows(n_tok, n_heads, seed + 1)
+    if zero_rows:
+        k[:zero_rows] = 0
+        v[:zero_rows] = 0
+    g = torch.Generator().manual_seed(seed + 2)
+    seq_idx = torch.randint(0, n_seqs, (n_tok,), generator=g, dtype=torch.int32)
+    pos = torch.empty(n_tok, dtype=torch.int32)
+    for s in range(n_seqs):  # distinct positions per sequence, in shuffled order
+        sel = (seq_idx == s).nonzero().flatten()
+        pos[sel] = torch.randperm(len(sel), generator=g).to(torch.int32) + 3
+    cap = int(math.ceil((n_tok + 3 + 1) / 64) * 64)
+    cache = tq.Cache(ctx, n_seqs, n_heads, cap)
+    dev = "cuda"
+    tq.quantize(ctx, cache, k.to(dev), v.to(dev), seq_idx.to(dev), pos.to(dev))
+    ctx.check_device_errors()
+    planes = {n: (t.cpu().numpy() if t is not None else None) for n, t in cache.planes.items()}
+    si, ps = seq_idx.numpy(), pos.numpy()
+    written = np.zeros((n_seqs, n_heads, cap), dtype=bool)
+    for t in range(n_tok):
+        written[si[t], :, ps[t]] = True
+    for name, arr in planes.items():   # untouched slots stay zero
+        if arr is not None:
+            assert not np.any(arr[~written]), name
+
+    def rows(name):
+        return np.stack([planes[name][si[t], h, ps[t]] for t in range(n_tok) for h in range(n_heads)])
+
+    stats = {}
+    for which, x, c, t, bits in (("k", k, ref.ck, ref.tk, bits_k), ("v", v, ref.cv, ref.tv, bits_v)):
+        xr = x.double().numpy().reshape(-1, D)
+        qz = o.quantize(xr, ref.pi, c, t, s_matrix=ref.s if (qjl and which == "k") else None)
+        cc = ph.compare_codes(rows("codes_" + which), qz, bits, t)
+        assert cc["outside_window"] == 0, cc
+        nn = ph.compare_fp16(rows("norm_" + which), qz.norm)
+        assert nn["worse"] == 0, nn
+        stats[which] = cc
+        if qjl and which == "k":
+            sc = ph.compare_signs(rows("qjl_bits"), qz, skip_vectors=cc["vec_mismatch"])
+            assert sc["outside_window"] == 0, sc
+            gg = ph.compare_fp16(rows("qjl_norm"), qz.qjl_gamma)
+            assert gg["worse"] == 0, gg
+    return stats
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl", SETTINGS)
+@pytest.mark.parametrize("n_tok,n_heads", [(1, 1), (7, 3), (127, 1), (128, 2), (129, 1), (1000, 8)])
+def test_quantize_parity(tq, n_tok, n_heads, bits_k, bits_v, qjl):
+    _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed=n_tok * 31 + n_heads)
+
+
+def test_quantize_zero_vectors(tq):
+    _quantize_and_compare(tq, 40, 2, 3, 3, 1, seed=5, zero_rows=9)
+
+
+def test_quantize_mismatch_rate_at_scale(tq):
+    total = mism = 0
+    for bits in (2, 3, 4):
+        st = _quantize_and_compare(tq, 4096, 8, bits, bits, 0, seed=77 + bits, n_seqs=1)
+        for s in st.values():
+            total += s["n"]
+            mism += s["mismatch"]
+    assert mism / total <= ph.MAX_MISMATCH_RATE, (mism, total)
+
+
+def test_quantize_out_of_range_tokens_are_flagged_not_written(tq):
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    cache = tq.Cache(ctx, 1, 2, 64)
+    k = make_rows(3, 2, 1).cuda()
+    seq_idx = torch.tensor([0, 1, 0], dtype=torch.int32, device="cuda")   # seq 1 does not exist
+    pos = torch.tensor([0, 0, 64], dtype=torch.int32, device="cuda")      # pos 64 >= capacity
+    tq.quantize(ctx, cache, k, k, seq_idx, pos)
+    with pytest.raises(tq.TQError) as ei:
+        ctx.check_device_errors()
+    assert ei.value.status == tq.TQ_ERR_DEVICE
+    assert int(cache.planes["norm_k"][0, :, 0].ne(0).sum()) == 2      # the valid token landed
+    assert int(cache.planes["norm_k"][0, :, 1:].ne(0).sum()) == 0
+    ctx.check_device_errors()                                          # flags were cleared
+
+
+# ------------------------------------------------------------------ decode
+def _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, kind="lognormal"):
+    """Quantize seeded K/V with the oracle; returns per-(seq, head) fields and
+    the packed planes laid out like the device cache."""
+    n_seqs = len(lens)
+    cap = max(64, int(math.ceil(max(lens) / 64) * 64))
+    per = {}
+    planes = {
+        "codes_k": np.zeros((n_seqs, n_heads, cap, D * bits_k // 8), np.uint8),
+        "norm_k": np.zeros((n_seqs, n_heads, cap), np.uint16),
+        "codes_v": np.zeros((n_seqs, n_heads, cap, D * bits_v // 8), np.uint8),
+        "norm_v": np.zeros((n_seqs, n_heads, cap), np.uint16),
+        "qjl_bits": np.zeros((n_seqs, n_heads, cap, D // 8), np.uint8) if qjl else None,
+        "qjl_norm": np.zeros((n_seqs, n_heads, cap), np.uint16) if qjl else None,
+    }
+    for s, n in enumerate(lens):
+        if n == 0:
+            continue
+        k = make_rows(n, n_heads, seed + 10 * s, lognormal=(kind == "lognormal")).double().numpy()
+        v = make_rows(n, n_heads, seed + 10 * s + 1, lognormal=False).double().numpy()
+        for h in range(n_heads):
+            qk = o.quantize(k[:, h], ref.pi, ref.ck, ref.tk, s_matrix=ref.s if qjl else None)
+            qv = o.quantize(v[:, h], ref.pi, ref.cv, ref.tv)
+            per[(s, h)] = (qk, qv)
+            planes["codes_k"][s, h, :n] = o.pack_codes(qk.codes, bits_k)
+            planes["codes_v"][s, h, :n] = o.pack_codes(qv.codes, bits_v)
+            planes["norm_k"][s, h, :n] = qk.norm.astype(np.float16).view(np.uint16)
+            planes["norm_v"][s, h, :n] = qv.norm.astype(np.float16).view(np.uint16)
+            if qjl:
+                planes["qjl_bits"][s, h, :n] = o.pack_signs(qk.qjl_signs)
+                planes["qjl_norm"][s, h, :n] = qk.qjl_gamma.astype(np.float16).view(np.uint16)
+    return per, planes, cap
+
+
+def _upload(tq, ctx, planes, n_seqs, n_heads, cap):
+    cache = tq.Cache(ctx, n_seqs, n_heads, cap)
+    for name, arr in planes.items():
+        if arr is not None:
+            t = torch.from_numpy(arr.view(np.int16) if arr.dtype == np.uint16 else arr)
+            cache.planes[name].copy_(t)
+    return cache
+
+
+def _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed, q_dtype=torch.float32,
+                        scale=0.0, max_seq_len=None):
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
+    ref = oracle_params(bits_k, bits_v, qjl)
+    per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed)
+    cache = _upload(tq, ctx, planes, len(lens), n_heads, cap)
+    n_q = n_heads * group
+    g = torch.Generator().manual_seed(seed + 99)
+    q = torch.randn(len(lens), n_q, D, generator=g).to(q_dtype)
+    max_len = max(lens) if max_seq_len is None else max_seq_len
+    out = torch.full((len(lens), n_q, D), float("nan"), device="cuda")
+    lse = torch.full((len(lens), n_q), float("nan"), device="cuda")
+    ws = tq.alloc_workspace(ctx, len(lens), n_q, max_len)
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    tq.decode_attention(ctx, cache, q.cuda(), seq_lens, max_len, out, lse, ws, scale=scale)
+    ctx.check_device_errors()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    sc = scale if scale > 0 else 1 / math.sqrt(D)
+    worst = 0.0
+    qd = q.double().numpy()
+    for s, n in enumerate(lens):
+        for h in range(n_heads):
+            rows = slice(h * group, (h + 1) * group)
+            if n == 0:
+                assert np.all(out[s, rows] == 0) and np.all(np.isneginf(lse[s, rows]))
+                continue
+            qk, qv = per[(s, h)]
+            o_ref, lse_ref, scores = o.decode_attention(
+                qd[s, rows], ref.pi, ref.ck, qk.codes, qk.norm, ref.cv, qv.codes, qv.norm, sc,
+                s_matrix=ref.s if qjl else None, qjl_signs=qk.qjl_signs if qjl else None,
+                qjl_gamma=qk.qjl_gamma if qjl else None)
+            ok, w = ph.attention_ok(out[s, rows], o_ref, lse[s, rows], lse_ref,
+                                    np.abs(scores).max(axis=1))
+            worst = max(worst, w)
+            assert ok, (s, h, w)
+    return worst
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl", SETTINGS)
+@pytest.mark.parametrize("lens,n_heads,group", [([1], 1, 1), ([7, 129], 2, 4), ([128], 1, 7),
+                                                ([1000, 0, 513], 2, 8), ([2500], 1, 16)])
+def test_decode_parity_on_oracle_packed_cache(tq, lens, n_heads, group, bits_k, bits_v, qjl):
+    _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed=sum(lens) + group)
+
+
+def test_decode_bf16_queries_explicit_scale_and_loose_bound(tq):
+    _decode_and_compare(tq, [300, 77], 2, 4, 3, 3, 0, seed=3, q_dtype=torch.bfloat16, scale=0.05,
+                        max_seq_len=640)
+
+
+def test_decode_long_sequence_many_splits(tq):
+    _decode_and_compare(tq, [20000], 1, 8, 3, 3, 0, seed=11)
+
+
+def test_decode_seq_len_above_bound_is_flagged(tq):
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    cache = tq.Cache(ctx, 1, 1, 128)
+    q = torch.randn(1, 1, D, device="cuda")
+    out = torch.empty(1, 1, D, device="cuda")
+    ws = tq.alloc_workspace(ctx, 1, 1, 64)
+    tq.decode_attention(ctx, cache, q, torch.tensor([100], dtype=torch.int32, device="cuda"), 64, out, None, ws)
+    with pytest.raises(tq.TQError):
+        ctx.check_device_errors()
+
+
+def test_decode_rejects_bad_arguments(tq):
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    cache = tq.Cache(ctx, 1, 2, 128)
+    q = torch.randn(1, 3, D, device="cuda")        # 3 query heads over 2 KV heads
+    out = torch.empty(1, 3, D, device="cuda")
+    ws = tq.alloc_workspace(ctx, 1, 3, 64)
+    lens = torch.tensor([10], dtype=torch.int32, device="cuda")
+    with pytest.raises(tq.TQError) as ei:
+        tq.decode_attention(ctx, cache, q, lens, 64, out, None, ws)
+    assert ei.value.status == tq.TQ_ERR_INVALID
+    q = torch.randn(1, 2, D, device="cuda")
+    with pytest.raises(tq.TQError):                  # max_seq_len above capacity
+        tq.decode_attention(ctx, cache, q, lens, 256, out, None, ws)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tq.TQError):                  # workspace too small
+        tq.decode_attention(ctx, cache, q, lens, 64, out, None, small)
+
+
+# -------------------------------------------------------------- end to end
+def test_end_to_end_tiny_against_oracle_and_exact_attention(tq):
+    """GPU quantize + GPU decode vs the oracle's quantize + decode on the tiny
+    workload (fp32 inputs rounded to bf16), plus the quality figure."""
+    from kv_cache_vector_12_b200 import workloads as wl
+    w = wl.WORKLOADS["tiny"]
+    gen = wl.generator("cpu", w.seed)
+    k32, v32 = wl.kv_tokens(w, w.seq_len, gen, "cpu", dtype=torch.float32)
+    q32 = wl.queries(w, 1, gen, "cpu", dtype=torch.float32)
+    k, v = k32.to(torch.bfloat16), v32.to(torch.bfloat16)
+    ctx = tq.Context(D, w.bits_k, w.bits_v, 0, w.pi_seed)
+    cache = tq.Cache(ctx, 1, 1, 1024)
+    idx = torch.zeros(w.seq_len, dtype=torch.int32, device="cuda")
+    pos = torch.arange(w.seq_len, dtype=torch.int32, device="cuda")
+    tq.quantize(ctx, cache, k.cuda(), v.cuda(), idx, pos)
+    out = torch.empty(1, 1, D, device="cuda")
+    lse = torch.empty(1, 1, device="cuda")
+    ws = tq.alloc_workspace(ctx, 1, 1, w.seq_len)
+    tq.decode_attention(ctx, cache, q32.cuda(), torch.tensor([w.seq_len], dtype=torch.int32, device="cuda"),
+                        w.seq_len, out, lse, ws)
+    ctx.check_device_errors()
+    ref = oracle_params(3, 3, 0)
+    qk = o.quantize(k[:, 0].double().numpy(), ref.pi, ref.ck, ref.tk)
+    qv = o.quantize(v[:, 0].double().numpy(), ref.pi, ref.cv, ref.tv)
+    o_ref, lse_ref, scores = o.decode_attention(q32[0].double().numpy(), ref.pi, ref.ck, qk.codes, qk.norm,
+                                                ref.cv, qv.codes, qv.norm, 1 / math.sqrt(D))
+    ok, worst = ph.attention_ok(out[0].cpu().numpy(), o_ref, lse[0].cpu().numpy(), lse_ref,
+                                np.abs(scores).max(axis=1))
+    assert ok, worst
+    o_exact, _ = o.exact_attention(q32[0].double().numpy(), k32[:, 0].double().numpy(),
+                                   v32[:, 0].double().numpy(), 1 / math.sqrt(D))
+    assert o.cosine_similarity(out[0].cpu().numpy(), o_exact) > 0.9

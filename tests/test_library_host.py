@@ -1,0 +1,83 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every entry point
+declared in include/tq.h, rejects bad arguments before touching CUDA, and its
+host-side parameters (Pi, S, codebooks) equal the oracle's, which computes
+them independently."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import turboquant_oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from kv_cache_vector_12_b200 import build
+    build.build()
+    from kv_cache_vector_12_b200 import tq as tqmod
+    return tqmod
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(tq_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(tq):
+    names = _declared_functions()
+    assert "tq_create" in names and "tq_decode_attention" in names
+    for n in names:
+        assert hasattr(tq.lib, n), n
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl,seed", [(3, 3, 0, 42), (2, 4, 1, 42), (4, 2, 1, 7), (3, 2, 0, 12345)])
+def test_host_params_equal_oracle(tq, bits_k, bits_v, qjl, seed):
+    lib_p = tq.host_params(128, bits_k, bits_v, qjl, seed)
+    ref = o.Params(128, bits_k, bits_v, bool(qjl), seed)
+    assert np.array_equal(lib_p["pi"].double().numpy(), ref.pi)
+    assert np.array_equal(lib_p["centroids_k"].double().numpy(), ref.ck)
+    assert np.array_equal(lib_p["thresholds_k"].double().numpy(), ref.tk)
+    assert np.array_equal(lib_p["centroids_v"].double().numpy(), ref.cv)
+    assert np.array_equal(lib_p["thresholds_v"].double().numpy(), ref.tv)
+    if qjl:
+        assert np.array_equal(lib_p["s"].double().numpy(), ref.s)
+
+
+def test_invalid_arguments_fail_before_cuda(tq):
+    lib = tq.lib
+    f = ctypes.POINTER(ctypes.c_float)()
+    assert lib.tq_host_params(128, 5, 3, 0, 1, f, f, f, f, f, f) == tq.TQ_ERR_INVALID
+    assert b"bits" in lib.tq_last_error()
+    assert lib.tq_host_params(128, 3, 3, 2, 1, f, f, f, f, f, f) == tq.TQ_ERR_INVALID
+    h = ctypes.c_void_p()
+    assert lib.tq_create(ctypes.byref(h), 64, 3, 3, 0, 1) == tq.TQ_ERR_UNSUPPORTED
+    assert lib.tq_create(None, 128, 3, 3, 0, 1) == tq.TQ_ERR_INVALID
+    assert lib.tq_quantize(None, None, None, None, None, None, 0, None) == tq.TQ_ERR_INVALID
+    assert lib.tq_decode_attention(None, None, None, 0, 1, None, 1, 0.0, None, None, None, 0, None) == \
+        tq.TQ_ERR_INVALID
+    assert lib.tq_layout(None, None) == tq.TQ_ERR_INVALID
+    assert lib.tq_workspace_bytes(None, 1, 1, 1) == 0
+    lib.tq_destroy(None)
+
+
+def test_binding_has_no_fallback_when_library_missing(tmp_path):
+    """Importing the binding from a package copy without libtq.so must raise."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "kv_cache_vector_12_b200"
+    pkg.mkdir()
+    for fn in ("__init__.py", "tq.py"):
+        shutil.copy(os.path.join(ROOT, "kv_cache_vector_12_b200", fn), pkg / fn)
+    r = subprocess.run([sys.executable, "-c", "import kv_cache_vector_12_b200.tq"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libtq.so" in r.stderr
