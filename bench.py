@@ -116,59 +116,83 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def run_cpu_oracle_decode(n_heads_sample: int = 8, seq_len: int = 32768, seed: int = 1002):
-    """The CPU oracle on a bounded sample of the llama8b decode step: unpack
-    the packed codes of `n_heads_sample` KV heads and run the oracle's decode
-    attention for their query heads.  Returns (GB/s-equivalent, seconds,
-    threads used, description)."""
-    import numpy as np
-    from oracle import turboquant_oracle as o
-    from kv_cache_vector_12_b200 import workloads as wl
-    w = wl.WORKLOADS["llama8b"]
-    p = o.Params(w.d, w.bits_k, w.bits_v, False, w.pi_seed)
-    gen = wl.generator("cpu", seed)
-    k, v = wl.kv_tokens(w, seq_len, gen, "cpu")
-    q = wl.queries(w, 1, gen, "cpu").double().numpy()[0]
-    packed = []
-    for h in range(n_heads_sample):
-        qk = o.quantize(k[:, h].double().numpy(), p.pi, p.ck, p.tk)
-        qv = o.quantize(v[:, h].double().numpy(), p.pi, p.cv, p.tv)
-        packed.append((o.pack_codes(qk.codes, w.bits_k), qk.norm, o.pack_codes(qv.codes, w.bits_v), qv.norm))
-    t0 = time.perf_counter()
-    for h, (pk, nk, pv, nv) in enumerate(packed):
-        ck = o.unpack_codes(pk, w.bits_k, w.d)
-        cv = o.unpack_codes(pv, w.bits_v, w.d)
-        o.decode_attention(q[h * w.group:(h + 1) * w.group], p.pi, p.ck, ck, nk, p.cv, cv, nv,
-                           1 / math.sqrt(w.d))
-    dt = time.perf_counter() - t0
-    nbytes = n_heads_sample * seq_len * (w.d * (w.bits_k + w.bits_v) // 8 + 4)
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = os.cpu_count() or 1
-    desc = f"oracle unpack + decode of {n_heads_sample} KV heads x {seq_len} tokens (llama8b decode step, numpy fp64)"
-    return nbytes / dt / 1e9, dt, threads, desc
+class OracleDecodeSample:
+    """The CPU oracle on a bounded sample of the llama8b decode step: the
+    packed codes of `n_heads` KV heads (quantized once by the oracle, untimed),
+    then per step: unpack them and run the oracle's decode attention for the
+    heads' query heads."""
+
+    def __init__(self, n_heads: int = 8, seq_len: int = 32768, seed: int = 1002):
+        from oracle import turboquant_oracle as o
+        from kv_cache_vector_12_b200 import workloads as wl
+        self.o = o
+        self.w = w = wl.WORKLOADS["llama8b"]
+        self.p = p = o.Params(w.d, w.bits_k, w.bits_v, False, w.pi_seed)
+        gen = wl.generator("cpu", seed)
+        k, v = wl.kv_tokens(w, seq_len, gen, "cpu")
+        self.q = wl.queries(w, 1, gen, "cpu").double().numpy()[0]
+        k_new, v_new = wl.kv_tokens(w, 1, gen, "cpu")
+        self.new_rows = [(k_new[:, h].double().numpy(), v_new[:, h].double().numpy()) for h in range(n_heads)]
+        self.packed = []
+        for h in range(n_heads):
+            qk = o.quantize(k[:, h].double().numpy(), p.pi, p.ck, p.tk)
+            qv = o.quantize(v[:, h].double().numpy(), p.pi, p.cv, p.tv)
+            self.packed.append((o.pack_codes(qk.codes, w.bits_k), qk.norm,
+                                o.pack_codes(qv.codes, w.bits_v), qv.norm))
+        self.step_bytes = n_heads * seq_len * (w.d * (w.bits_k + w.bits_v) // 8 + 4)
+        self.desc = (f"oracle append-quantize of 1 token + unpack + decode attention of {n_heads} KV heads x "
+                     f"{seq_len} tokens (llama8b decode step, numpy fp64)")
+
+    def step(self) -> float:
+        o, w, p = self.o, self.w, self.p
+        t0 = time.perf_counter()
+        for h, (pk, nk, pv, nv) in enumerate(self.packed):
+            kn, vn = self.new_rows[h]                      # append-quantize of the step's token
+            o.pack_codes(o.quantize(kn, p.pi, p.ck, p.tk).codes, w.bits_k)
+            o.pack_codes(o.quantize(vn, p.pi, p.cv, p.tv).codes, w.bits_v)
+            ck = o.unpack_codes(pk, w.bits_k, w.d)
+            cv = o.unpack_codes(pv, w.bits_v, w.d)
+            o.decode_attention(self.q[h * w.group:(h + 1) * w.group], p.pi, p.ck, ck, nk, p.cv, cv, nv,
+                               1 / math.sqrt(w.d))
+        return time.perf_counter() - t0
+
+    @staticmethod
+    def threads() -> int:
+        try:
+            from threadpoolctl import threadpool_info
+            return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        except Exception:
+            return os.cpu_count() or 1
+
+
+def cpu_baseline(min_seconds: float = 10.0) -> dict:
+    smp = OracleDecodeSample(n_heads=8)
+    total, reps = 0.0, 0
+    while total < min_seconds:
+        total += smp.step()
+        reps += 1
+    return {"value": reps * smp.step_bytes / total / 1e9, "unit": "GB/s", "cores": smp.threads(),
+            "kind": "oracle", "sample": f"{smp.desc}, {reps} steps", "seconds": total}
 
 
 def reference_arm(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    n_heads_sample = 1
-    vals = []
+    smp = OracleDecodeSample(n_heads=1)
+    times = []
     for i in range(args.warmup + args.steps):
-        gbs, dt, threads, desc = run_cpu_oracle_decode(n_heads_sample=n_heads_sample, seed=1002 + i % 3)
+        dt = smp.step()
         if i >= args.warmup:
-            vals.append((gbs, dt))
-    total_bytes = sum(g * d for g, d in vals)
-    total_t = sum(d for _, d in vals)
-    value = total_bytes / total_t
+            times.append(dt)
+    total_t = sum(times)
+    value = len(times) * smp.step_bytes / total_t / 1e9
+    desc = smp.desc + " per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(vals),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD_DESC, "sample": desc},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": smp.threads(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -345,11 +369,7 @@ def main(argv=None) -> int:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return 0
-    cpu = None
-    if not args.no_cpu_baseline:
-        gbs, dt, threads, desc = run_cpu_oracle_decode(n_heads_sample=8)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "seconds": dt}
+    cpu = None if args.no_cpu_baseline else cpu_baseline()
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,

@@ -135,11 +135,11 @@ def test_quantize_out_of_range_tokens_are_flagged_not_written(tq):
 
 
 # ------------------------------------------------------------------ decode
-def _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, kind="lognormal"):
+def _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, kind="lognormal", min_cap=0):
     """Quantize seeded K/V with the oracle; returns per-(seq, head) fields and
     the packed planes laid out like the device cache."""
     n_seqs = len(lens)
-    cap = max(64, int(math.ceil(max(lens) / 64) * 64))
+    cap = max(64, int(math.ceil(max(max(lens), min_cap) / 64) * 64))
     per = {}
     planes = {
         "codes_k": np.zeros((n_seqs, n_heads, cap, D * bits_k // 8), np.uint8),
@@ -181,7 +181,7 @@ def _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed, q_d
                         scale=0.0, max_seq_len=None):
     ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
     ref = oracle_params(bits_k, bits_v, qjl)
-    per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed)
+    per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, min_cap=max_seq_len or 0)
     cache = _upload(tq, ctx, planes, len(lens), n_heads, cap)
     n_q = n_heads * group
     g = torch.Generator().manual_seed(seed + 99)
