@@ -26,8 +26,10 @@ so every formula below is the plainest reading of the prose, listed as such):
 Readings where the pages are silent (each also listed in the design notes):
 
 * coordinate law N(0, 1/d); codebook = Lloyd-Max centroids of N(0,1) / sqrt(d),
-  rounded to fp32; thresholds = fp32 midpoints of adjacent fp32 centroids;
-  code = #{j : t_j < y}  (a value equal to a threshold goes to the lower cell).
+  rounded to fp16 (the precision of the stored norms; it changes the
+  distortion by < 1e-5 relative); thresholds = exact midpoints of adjacent
+  centroids (representable in fp32); code = #{j : t_j < y}  (a value equal to
+  a threshold goes to the lower cell).
 * every head vector x (bf16) is split into n = ||x||_2 and direction x/n;
   y = (Pi x)/n with Pi the bf16-rounded rotation; n = 0 gives y = 0.
 * n is stored as fp16 (round to nearest even, saturating at 65504).
@@ -221,12 +223,11 @@ def lloyd_max_distortion(centroids) -> float:
 
 
 def codebook(bits: int, d: int):
-    """The method's codebook for N(0, 1/d): (centroids, thresholds), both fp32
-    values held in float64.  Centroids are the N(0,1) Lloyd-Max centroids
-    divided by sqrt(d); thresholds are the fp32-rounded midpoints of adjacent
-    fp32 centroids."""
-    c = round_to_fp32(lloyd_max_normal(bits) / math.sqrt(d))
-    t = round_to_fp32(0.5 * (c[:-1] + c[1:]))
+    """The method's codebook for N(0, 1/d): (centroids, thresholds) as float64.
+    Centroids are the N(0,1) Lloyd-Max centroids divided by sqrt(d), rounded
+    to fp16; thresholds are the exact midpoints of adjacent centroids."""
+    c = round_to_fp16_sat(lloyd_max_normal(bits) / math.sqrt(d))
+    t = 0.5 * (c[:-1] + c[1:])
     return c, t
 
 

@@ -97,15 +97,19 @@ def test_distortion_monte_carlo(bits):
     assert abs(err.mean() - d) < 5 * err.std() / math.sqrt(x.size)
 
 
-def test_codebook_scaling_and_fp32():
+def test_codebook_fp16_scaling():
     d = 128
     for bits in (2, 3, 4):
         c, t = o.codebook(bits, d)
-        assert np.array_equal(c, c.astype(np.float32).astype(np.float64))
-        assert np.array_equal(t, t.astype(np.float32).astype(np.float64))
-        assert np.allclose(c * math.sqrt(d), o.lloyd_max_normal(bits), rtol=1e-6)
+        assert np.array_equal(c, c.astype(np.float16).astype(np.float64))     # fp16 centroids
+        assert np.array_equal(t, t.astype(np.float32).astype(np.float64))     # midpoints fit fp32
+        assert np.array_equal(2 * t, c[:-1] + c[1:])
+        assert np.allclose(c * math.sqrt(d), o.lloyd_max_normal(bits), rtol=2 ** -11)
         assert np.all(np.diff(c) > 0) and np.all((t > c[:-1]) & (t < c[1:]))
-        assert t[len(t) // 2] == 0.0
+        assert t[len(t) // 2] == 0.0 and np.array_equal(c, -c[::-1])
+        # rounding the centroids to fp16 moves the N(0,1) distortion by < 1e-5 relative
+        dist = o.lloyd_max_distortion(c * math.sqrt(d))
+        assert abs(dist / o.lloyd_max_distortion(o.lloyd_max_normal(bits)) - 1) < 1e-5
 
 
 # ------------------------------------------------------------------- random
