@@ -24,6 +24,49 @@ struct tq_ctx {
 
 namespace {
 
+// fp16 bit pattern of a float that is exactly representable in fp16's normal
+// range (every centroid is).
+uint16_t exact_half_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) == 0) return (uint16_t)(u >> 16);
+  const uint32_t sign = (u >> 16) & 0x8000u;
+  const int exp = (int)((u >> 23) & 0xff) - 127 + 15;
+  return (uint16_t)(sign | ((uint32_t)exp << 10) | ((u & 0x7fffffu) >> 13));
+}
+
+// Byte tables of the decode kernel's lookups (see tq_internal.h).
+bool build_luts(const float *ck, int bits_k, const float *cv, int bits_v, tq::Lut &lk, tq::Lut &lv) {
+  std::memset(&lk, 0, sizeof lk);
+  std::memset(&lv, 0, sizeof lv);
+  for (int e = 0; e < (1 << bits_k); ++e) {
+    const double scaled = std::ldexp((double)ck[e], tq::kKFixedShift);
+    const long v = std::lrint(scaled);
+    if ((double)v != scaled || v > 32767 || v < -32767) return false;  // not exact 16-bit fixed point
+    lk.lo[e / 4] |= (uint32_t)(v & 0xff) << (8 * (e % 4));
+    lk.hi[e / 4] |= (uint32_t)((v >> 8) & 0xff) << (8 * (e % 4));
+  }
+  for (int e = 0; e < (1 << bits_v); ++e) {
+    const uint16_t hb = exact_half_bits(cv[e]);
+    lv.lo[e / 4] |= (uint32_t)(hb & 0xff) << (8 * (e % 4));
+    lv.hi[e / 4] |= (uint32_t)(hb >> 8) << (8 * (e % 4));
+  }
+  return true;
+}
+
+bool is_permutation(const uint8_t *p) {
+  bool seen[tq::kHeadDim] = {};
+  for (int i = 0; i < tq::kHeadDim; ++i) {
+    if (p[i] >= tq::kHeadDim || seen[p[i]]) return false;
+    seen[p[i]] = true;
+  }
+  return true;
+}
+
+}  // namespace
+
+namespace {
+
 thread_local char g_last_error[512] = "";
 
 tq_status fail(tq_status st, const char *fmt, ...) {
@@ -68,29 +111,46 @@ tq_status check_cache(const tq_ctx *ctx, const tq_cache *c) {
 
 namespace tq {
 
-DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len) {
-  // Enough (sequence, KV head, split) work items to fill 148 SMs several
-  // times over, with splits of at least 256 tokens.
-  const long units = (long)n_seqs * n_kv_heads;
-  const long target_items = 148L * 8;
-  long per_unit = (target_items + units - 1) / units;
-  long chunk = per_unit > 0 ? ((long)max_seq_len + per_unit - 1) / per_unit : max_seq_len;
-  if (chunk < 256) chunk = 256;
-  chunk = (chunk + 63) / 64 * 64;
-  DecodeSplit s;
-  s.chunk = (int)chunk;
-  s.n_splits = max_seq_len > 0 ? (int)(((long)max_seq_len + chunk - 1) / chunk) : 1;
-  if (s.n_splits < 1) s.n_splits = 1;
-  return s;
+static int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
 }
 
-DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, int qjl, DecodeSplit split) {
+// Splits of the sequence axis: about one full wave of resident CTAs
+// (SMs x CTAs per SM) over the (sequence, KV head) units, at least 8 splits
+// per unit when the units alone fill less than four waves (so ragged batches
+// balance), and at least 256 tokens per split.
+DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm) {
+  if (ctas_per_sm > 4) ctas_per_sm = 4;
+  if (ctas_per_sm < 1) ctas_per_sm = 1;
+  const long units = (long)n_seqs * n_kv_heads;
+  const long slots = (long)sm_count() * ctas_per_sm;
+  long n = slots / units;
+  const long balance = (4 * slots + units - 1) / units;
+  if (n < (balance < 8 ? balance : 8)) n = balance < 8 ? balance : 8;
+  if (n < 1) n = 1;
+  long chunk = ((long)max_seq_len + n - 1) / n;
+  if (chunk < 256) chunk = 256;
+  chunk = (chunk + 63) / 64 * 64;
+  DecodeSplit sp;
+  sp.chunk = (int)chunk;
+  sp.n_splits = max_seq_len > 0 ? (int)(((long)max_seq_len + chunk - 1) / chunk) : 1;
+  return sp;
+}
+
+DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t rows = (size_t)n_seqs * n_q_heads;
   DecodeWorkspace w;
-  w.q_hat = 0;
-  w.q_tilde = up(rows * kHeadDim * sizeof(float));
-  w.partials = w.q_tilde + (qjl ? up(rows * kHeadDim * sizeof(float)) : 0);
+  w.q8 = 0;
+  w.qscale = up(rows * 4 * kHeadDim);
+  w.partials = w.qscale + up(rows * 4 * sizeof(float));
   w.total = w.partials + up(rows * (size_t)split.n_splits * (kHeadDim + 2) * sizeof(float));
   return w;
 }
@@ -158,11 +218,21 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     delete ctx;
     return cuda_fail(e, "cudaGetDevice");
   }
-  // One block: pi | pit | s | st | codebooks | error word.
+  uint8_t kperm[tq::kHeadDim], vperm[tq::kHeadDim], jperm[tq::kHeadDim];
+  tq::kperm_of(bits_k, kperm);
+  tq::vperm_of(bits_v, vperm);
+  tq::jperm_of(jperm);
+  if (!is_permutation(kperm) || !is_permutation(vperm) || !is_permutation(jperm) ||
+      !build_luts(ctx->ck.data(), bits_k, ctx->cv.data(), bits_v, ctx->dp.lut_k, ctx->dp.lut_v)) {
+    delete ctx;
+    return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
+  }
+  // One block: pi | pit | piv | s | st | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
-  const size_t off_pi = 0, off_pit = off_pi + dd * 2, off_s = off_pit + dd * 2;
+  const size_t off_pi = 0, off_pit = off_pi + dd * 2, off_piv = off_pit + dd * 2, off_s = off_piv + dd * 2;
   const size_t off_st = off_s + dd * 4, off_cb = off_st + dd * 4;
-  const size_t off_err = off_cb + 4 * tq::kMaxLevels * 4, total = off_err + 256;
+  const size_t off_kperm = off_cb + 4 * tq::kMaxLevels * 4, off_jperm = off_kperm + 256;
+  const size_t off_err = off_jperm + 256, total = off_err + 256;
   e = cudaMalloc(&ctx->dev_block, total);
   if (e != cudaSuccess) {
     delete ctx;
@@ -179,6 +249,11 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < d; ++j) st_h[(size_t)j * d + i] = ctx->s[(size_t)i * d + j];
   }
+  uint16_t *piv = (uint16_t *)(h.data() + off_piv);
+  for (int k = 0; k < d; ++k)
+    for (int i = 0; i < d; ++i) piv[(size_t)k * d + i] = ctx->pi_bits[(size_t)vperm[k] * d + i];
+  std::memcpy(h.data() + off_kperm, kperm, tq::kHeadDim);
+  std::memcpy(h.data() + off_jperm, jperm, tq::kHeadDim);
   float *cb = (float *)(h.data() + off_cb);
   std::memcpy(cb + 0 * tq::kMaxLevels, ctx->ck.data(), tq::kMaxLevels * 4);
   std::memcpy(cb + 1 * tq::kMaxLevels, ctx->tk.data(), tq::kMaxLevels * 4);
@@ -197,9 +272,15 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->dp.st = (const float *)(base + off_st);
   ctx->dp.cb = (const float *)(base + off_cb);
   ctx->dp.err = (unsigned *)(base + off_err);
+  ctx->dp.piv = (const uint16_t *)(base + off_piv);
+  ctx->dp.kperm = (const uint8_t *)(base + off_kperm);
+  ctx->dp.jperm = (const uint8_t *)(base + off_jperm);
   ctx->dp.bits_k = bits_k;
   ctx->dp.bits_v = bits_v;
   ctx->dp.qjl = qjl;
+  // resolve the decode kernels' occupancy now, outside any stream capture
+  tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8);
+  tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16);
   *out = ctx;
   return TQ_OK;
 }
@@ -253,10 +334,10 @@ tq_status tq_quantize(tq_ctx *ctx, const tq_cache *cache, const void *k, const v
 
 size_t tq_workspace_bytes(const tq_ctx *ctx, int32_t n_seqs, int32_t n_q_heads, int32_t max_seq_len) {
   if (!ctx || n_seqs <= 0 || n_q_heads <= 0 || max_seq_len < 0) return 0;
-  // The split depends on n_kv_heads only through the item count; size for the
-  // worst case (one KV head per query head).
-  const tq::DecodeSplit sp = tq::decode_split(n_seqs, 1, max_seq_len);
-  return tq::decode_workspace(n_seqs, n_q_heads, ctx->qjl, sp).total;
+  // The split count falls as the (sequence, KV head) units grow and rises with
+  // CTAs per SM; one KV head and the largest occupancy bound it from above.
+  const tq::DecodeSplit sp = tq::decode_split(n_seqs, 1, max_seq_len, 4);
+  return tq::decode_workspace(n_seqs, n_q_heads, sp).total;
 }
 
 tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q, int32_t q_dtype,
@@ -280,8 +361,10 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
       (lse && ((uintptr_t)lse & 3u)))
     return fail(TQ_ERR_INVALID, "misaligned q/out (16 B), workspace (256 B) or seq_lens/lse (4 B)");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
-  const tq::DecodeSplit sp = tq::decode_split(cache->n_seqs, cache->n_kv_heads, max_seq_len);
-  const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, ctx->qjl, sp);
+  const int group = n_q_heads / cache->n_kv_heads;
+  const int ctas = tq::decode_ctas_per_sm(ctx->bits_k, ctx->bits_v, ctx->qjl, group);
+  const tq::DecodeSplit sp = tq::decode_split(cache->n_seqs, cache->n_kv_heads, max_seq_len, ctas);
+  const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, sp);
   if (workspace_bytes < ws.total)
     return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, ws.total);
   if (scale <= 0.f) scale = 1.0f / std::sqrt((float)ctx->d);

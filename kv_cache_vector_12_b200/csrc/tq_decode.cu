@@ -1,0 +1,778 @@
+// Decode attention over the packed TurboQuant cache, sm_100a.
+//
+// The method reads K and V straight from their codes ("TurboQuantの仕組み",
+// ai-accelerate.xyz explainer: rotate once, per-coordinate Lloyd-Max codes,
+// optional 1-bit QJL residual signs).  Per (sequence, KV head, split of the
+// sequence) one CTA streams the split's packed codes and norms into a shared
+// memory ring with TMA bulk copies (one producer warp, mbarrier pipeline with
+// bounded waits) while four consumer warps each take 16 tokens of every
+// 64-token stage:
+//
+//   scores  S[tok][head] = q_hat . c_K[code]   int8 tensor cores (mma m16n8k32):
+//           K centroids are exact 16-bit fixed-point integers (c * 2^17), split
+//           into hi/lo bytes by two byte-permute lookups per 4 codes; q_hat is
+//           16-bit fixed point (hi/lo bytes), so the dot product is exact up to
+//           q_hat's rounding.  QJL signs become 0/-1 bytes (sign-replicating
+//           byte permute) against q_tilde in the same int8 MMA.
+//   softmax online per warp and query head (exp2), masked past seq_len.
+//   values  O^T[coord][head] += V~^T[coord][tok] P[tok][head]   fp16 tensor
+//           cores (mma m16n8k16): fp16 centroids looked up by byte permutes,
+//           P transposed into the B fragment with movmatrix.
+//
+// The coordinate order inside the MMA fragments is a fixed permutation of the
+// head dimension chosen so that every code is expanded where it is loaded; the
+// host computes the permutations (tq_api.cu) and rotate_q writes q_hat in the
+// K order, merge applies Pi^T with rows in the V order.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kStageTokens = 16 * kConsumerWarps;  // 64
+constexpr int kStages = 6;
+constexpr unsigned kWaitLimit = 1u << 22;           // bounded mbarrier waits
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of the barrier; false if the bounded wait expired.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (unsigned i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <bool ASigned, bool BSigned>
+__device__ __forceinline__ void mma_i8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  if constexpr (ASigned && BSigned)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else if constexpr (ASigned && !BSigned)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else if constexpr (!ASigned && BSigned)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// ------------------------------------------------------- code expansion
+// A selector holds four codes in the low three (or four) bits of the nibbles
+// of its low 16 bits.  lookup() returns the low bytes and the high bytes of
+// the four table entries (one byte per code).
+template <int B>
+__device__ __forceinline__ void lookup(const Lut &t, uint32_t sel, uint32_t &lo, uint32_t &hi) {
+  if constexpr (B <= 3) {
+    lo = prmt(t.lo[0], t.lo[1], sel);
+    hi = prmt(t.hi[0], t.hi[1], sel);
+  } else {
+    const uint32_t s7 = sel & 0x7777u;
+    // byte n of m is 0xFF when nibble n of sel has its top bit set
+    const uint32_t m = prmt(sel << 4, sel, 0xD9C8u);
+    const uint32_t l0 = prmt(t.lo[0], t.lo[1], s7), l1 = prmt(t.lo[2], t.lo[3], s7);
+    const uint32_t h0 = prmt(t.hi[0], t.hi[1], s7), h1 = prmt(t.hi[2], t.hi[3], s7);
+    lo = (l1 & m) | (l0 & ~m);
+    hi = (h1 & m) | (h0 & ~m);
+  }
+}
+
+// Spare-column codes of the 3-bit layout: bit k of each code is the top bit
+// of the same nibble of word k.
+__device__ __forceinline__ uint32_t spare3(uint32_t w0, uint32_t w1, uint32_t w2) {
+  return ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
+}
+
+// Selector sigma (0..7) of the 32 K codes a thread owns for one token
+// (the words of its 32-coordinate group).  Code order: see kperm on the host.
+template <int B>
+__device__ __forceinline__ uint32_t k_selector(const uint32_t (&w)[B], int sigma) {
+  if constexpr (B == 3) {
+    const int k = sigma >> 1;
+    const uint32_t x = k < 3 ? (w[k < 3 ? k : 0] & 0x77777777u) : spare3(w[0], w[1], w[2]);
+    return (sigma & 1) ? x >> 16 : x;
+  } else if constexpr (B == 2) {
+    const int wd = sigma >> 2, par = (sigma >> 1) & 1;
+    const uint32_t x = (w[wd] >> (2 * par)) & 0x33333333u;
+    return (sigma & 1) ? x >> 16 : x;
+  } else {
+    const uint32_t x = w[sigma >> 1];
+    return (sigma & 1) ? x >> 16 : x;
+  }
+}
+
+// fp16 pairs (token A, token B) for two coordinates from one V selector whose
+// nibbles are [A.x, A.y, B.x, B.y].
+template <int B>
+__device__ __forceinline__ void v_pairs(const Lut &t, uint32_t sel, uint32_t &px, uint32_t &py) {
+  uint32_t lo, hi;
+  lookup<B>(t, sel, lo, hi);
+  px = prmt(lo, hi, 0x6240u);
+  py = prmt(lo, hi, 0x7351u);
+}
+
+// -------------------------------------------------------- shared layout
+template <int BK, int BV, bool QJL>
+struct Stage {
+  static constexpr int kc = 0;                                   // K codes
+  static constexpr int vc = kc + kStageTokens * D * BK / 8;      // V codes
+  static constexpr int jb = vc + kStageTokens * D * BV / 8;      // QJL sign bits
+  static constexpr int kn = jb + (QJL ? kStageTokens * D / 8 : 0);
+  static constexpr int vn = kn + kStageTokens * 2;
+  static constexpr int jg = vn + kStageTokens * 2;
+  static constexpr int bytes = jg + (QJL ? kStageTokens * 2 : 0);
+};
+
+struct DecodeArgs {
+  DeviceParams p;
+  tq_cache c;
+  int n_q_heads, max_seq_len, chunk, n_splits;
+  const int32_t *seq_lens;
+  const uint8_t *q8;      // [rows][4][128] bytes: q_hat hi, lo; q_tilde hi, lo (K / QJL fragment order)
+  const float *qscale;    // [rows][4]: score factor, QJL factor, sum of q_tilde ints, unused
+  float *partials;        // [rows][n_splits][2 + D]
+};
+
+template <int BK, int BV, bool QJL, int NT>
+__global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(const DecodeArgs a) {
+  using St = Stage<BK, BV, QJL>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ int abort_flag;
+  __shared__ float sm_m[kConsumerWarps][8 * NT], sm_l[kConsumerWarps][8 * NT];
+
+  const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.n_q_heads / a.c.n_kv_heads;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int len = a.seq_lens[s];
+  if (len < 0 || len > a.max_seq_len) {
+    if (tid == 0 && split == 0 && h == 0) atomicOr(a.p.err, kErrSeqLen);
+    len = len < 0 ? 0 : a.max_seq_len;
+  }
+  const int t0 = split * a.chunk;
+  if (t0 >= len) return;  // this split holds no tokens; merge skips it
+  const int t1 = min(len, t0 + a.chunk);
+  const int n_stage = (t1 - t0 + kStageTokens - 1) / kStageTokens;
+  const long base = ((long)s * a.c.n_kv_heads + h) * a.c.capacity;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), kConsumerWarps);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one elected lane issues the bulk copies
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < n_stage; ++it) {
+        const int slot = it % kStages;
+        if (it >= kStages && !mbar_wait(smem_u32(&empty_bar[slot]), ((it / kStages) - 1) & 1)) {
+          atomicOr(a.p.err, kErrWaitExpired);
+          abort_flag = 1;
+          break;
+        }
+        if (*(volatile int *)&abort_flag) break;
+        unsigned char *st = smem + slot * St::bytes;
+        const uint32_t bar = smem_u32(&full_bar[slot]);
+        const long tok = base + t0 + (long)it * kStageTokens;
+        mbar_arrive_expect_tx(bar, St::bytes);
+        bulk_g2s(smem_u32(st + St::kc), a.c.codes_k + tok * (D * BK / 8), kStageTokens * D * BK / 8, bar);
+        bulk_g2s(smem_u32(st + St::vc), a.c.codes_v + tok * (D * BV / 8), kStageTokens * D * BV / 8, bar);
+        bulk_g2s(smem_u32(st + St::kn), a.c.norm_k + tok, kStageTokens * 2, bar);
+        bulk_g2s(smem_u32(st + St::vn), a.c.norm_v + tok, kStageTokens * 2, bar);
+        if constexpr (QJL) {
+          bulk_g2s(smem_u32(st + St::jb), a.c.qjl_bits + tok * (D / 8), kStageTokens * D / 8, bar);
+          bulk_g2s(smem_u32(st + St::jg), a.c.qjl_norm + tok, kStageTokens * 2, bar);
+        }
+        issued = it + 1;
+      }
+      // never leave the CTA with copies in flight: wait (bounded) for the
+      // last stages issued if the consumers stopped early
+      if (*(volatile int *)&abort_flag) {
+        for (int it = max(0, issued - kStages); it < issued; ++it)
+          mbar_wait(smem_u32(&full_bar[it % kStages]), (it / kStages) & 1);
+      }
+    }
+  } else {
+    // ---------------- consumers
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // rotate_q's q8 / qscale are complete
+    const int r = lane >> 2, q = lane & 3;
+    // q fragments (int8, K fragment order) of this thread's head r in every n-tile
+    uint32_t qh[NT][4][2], ql[NT][4][2], jh[NT][QJL ? 4 : 1][2], jl[NT][QJL ? 4 : 1][2];
+    float fq[NT][2], fj[NT][2], jsum[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = 8 * nt + r;
+      const bool live = g < G;
+      const uint8_t *qb = a.q8 + ((long)s * a.n_q_heads + h * G + (live ? g : 0)) * 4 * D;
+#pragma unroll
+      for (int st = 0; st < 4; ++st)
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int off = 32 * st + 16 * sl + 4 * q;
+          qh[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + off) : 0u;
+          ql[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + D + off) : 0u;
+          if constexpr (QJL) {
+            jh[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + 2 * D + off) : 0u;
+            jl[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + 3 * D + off) : 0u;
+          }
+        }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int gg = 8 * nt + 2 * q + e;
+        const float *f = a.qscale + ((long)s * a.n_q_heads + h * G + (gg < G ? gg : 0)) * 4;
+        fq[nt][e] = gg < G ? f[0] : 0.f;
+        fj[nt][e] = gg < G ? f[1] : 0.f;
+        jsum[nt][e] = gg < G ? f[2] : 0.f;
+      }
+    }
+    const Lut lk = a.p.lut_k, lv = a.p.lut_v;
+
+    float m_run[NT][2], l_run[NT][2], acc[NT][8][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        m_run[nt][e] = -INFINITY;
+        l_run[nt][e] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+    }
+
+    for (int it = 0; it < n_stage; ++it) {
+      const int slot = it % kStages;
+      if (!mbar_wait(smem_u32(&full_bar[slot]), (it / kStages) & 1)) {
+        atomicOr(a.p.err, kErrWaitExpired);
+        abort_flag = 1;
+        break;
+      }
+      const unsigned char *st = smem + slot * St::bytes;
+      const int tok0 = t0 + it * kStageTokens + 16 * warp;  // first token of this warp's tile
+      if (tok0 < t1) {
+        const int wt = 16 * warp;                            // tile row offset inside the stage
+        // ---------------- scores: int8 MMA over 4 k-steps of 32
+        int chh[NT][4], cmid[NT][4], cll[NT][4], cjh[NT][4], cjl[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) chh[nt][e] = cmid[nt][e] = cll[nt][e] = cjh[nt][e] = cjl[nt][e] = 0;
+        uint32_t wk0[BK], wk1[BK];
+        const unsigned char *kr0 = st + St::kc + (wt + r) * (D * BK / 8) + q * 4 * BK;
+        const unsigned char *kr1 = kr0 + 8 * (D * BK / 8);
+#pragma unroll
+        for (int i = 0; i < BK; ++i) {
+          wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
+          wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
+        }
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t alo[4], ahi[4];
+          lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks), alo[0], ahi[0]);
+          lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks), alo[1], ahi[1]);
+          lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks + 1), alo[2], ahi[2]);
+          lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks + 1), alo[3], ahi[3]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_i8<true, true>(chh[nt], ahi[0], ahi[1], ahi[2], ahi[3], qh[nt][ks][0], qh[nt][ks][1]);
+            mma_i8<true, false>(cmid[nt], ahi[0], ahi[1], ahi[2], ahi[3], ql[nt][ks][0], ql[nt][ks][1]);
+            mma_i8<false, true>(cmid[nt], alo[0], alo[1], alo[2], alo[3], qh[nt][ks][0], qh[nt][ks][1]);
+            mma_i8<false, false>(cll[nt], alo[0], alo[1], alo[2], alo[3], ql[nt][ks][0], ql[nt][ks][1]);
+          }
+        }
+        if constexpr (QJL) {
+          const uint32_t w0 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + r) * (D / 8))[q];
+          const uint32_t w1 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + r + 8) * (D / 8))[q];
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            // bytes 0x00 / 0xFF (= -bit) for bits j, j+8, j+16, j+24 with j = 2 ks + slot
+            const int j0 = 2 * ks, j1 = 2 * ks + 1;
+            const uint32_t a0 = prmt(w0 << (7 - j0), 0u, 0xBA98u), a1 = prmt(w1 << (7 - j0), 0u, 0xBA98u);
+            const uint32_t a2 = prmt(w0 << (7 - j1), 0u, 0xBA98u), a3 = prmt(w1 << (7 - j1), 0u, 0xBA98u);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_i8<true, true>(cjh[nt], a0, a1, a2, a3, jh[nt][ks][0], jh[nt][ks][1]);
+              mma_i8<true, false>(cjl[nt], a0, a1, a2, a3, jl[nt][ks][0], jl[nt][ks][1]);
+            }
+          }
+        }
+        // ---------------- scores -> online softmax
+        const __half *kn = reinterpret_cast<const __half *>(st + St::kn) + wt;
+        const __half *vn = reinterpret_cast<const __half *>(st + St::vn) + wt;
+        const float nk0 = __half2float(kn[r]), nk1 = __half2float(kn[r + 8]);
+        const float nv0 = __half2float(vn[r]), nv1 = __half2float(vn[r + 8]);
+        float gm0 = 0.f, gm1 = 0.f;
+        if constexpr (QJL) {
+          const __half *jg = reinterpret_cast<const __half *>(st + St::jg) + wt;
+          gm0 = __half2float(jg[r]);
+          gm1 = __half2float(jg[r + 8]);
+        }
+        const bool ok0 = tok0 + r < t1, ok1 = tok0 + r + 8 < t1;
+        uint32_t pb[NT][2];
+        bool rescale = false;
+        float alpha[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float sc[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int hd = e & 1;
+            const float dot = fmaf(65536.f, (float)chh[nt][e], fmaf(256.f, (float)cmid[nt][e], (float)cll[nt][e]));
+            float v = dot * fq[nt][hd];
+            if constexpr (QJL) {
+              const float dj = fmaf(256.f, (float)cjh[nt][e], (float)cjl[nt][e]);
+              v = fmaf((e < 2 ? gm0 : gm1) * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
+            }
+            v *= (e < 2 ? nk0 : nk1);
+            sc[e] = (e < 2 ? ok0 : ok1) ? v : -INFINITY;
+          }
+#pragma unroll
+          for (int hd = 0; hd < 2; ++hd) {
+            float mx = fmaxf(sc[hd], sc[hd + 2]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mn = fmaxf(m_run[nt][hd], mx);
+            const float al = mn == -INFINITY ? 1.f : exp2f(m_run[nt][hd] - mn);
+            alpha[nt][hd] = al;
+            rescale |= al != 1.f;
+            m_run[nt][hd] = mn;
+            const float p0 = mn == -INFINITY ? 0.f : exp2f(sc[hd] - mn);
+            const float p1 = mn == -INFINITY ? 0.f : exp2f(sc[hd + 2] - mn);
+            l_run[nt][hd] = fmaf(l_run[nt][hd], al, p0 + p1);
+            sc[hd] = ok0 ? p0 * nv0 : 0.f;
+            sc[hd + 2] = ok1 ? p1 * nv1 : 0.f;
+          }
+          pb[nt][0] = movmatrix_trans(pack_half2(sc[0], sc[1]));
+          pb[nt][1] = movmatrix_trans(pack_half2(sc[2], sc[3]));
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              acc[nt][mt][0] *= alpha[nt][0];
+              acc[nt][mt][1] *= alpha[nt][1];
+              acc[nt][mt][2] *= alpha[nt][0];
+              acc[nt][mt][3] *= alpha[nt][1];
+            }
+        }
+        // ---------------- values: fp16 MMA, 8 m-tiles of 16 coordinates
+        // tokens (2q, 2q+1) and (2q+8, 2q+9) of the tile; unit r of 16 coordinates
+        const unsigned char *vt = st + St::vc + (wt + 2 * q) * (D * BV / 8);
+        constexpr int VB = D * BV / 8;
+        if constexpr (BV == 3) {
+          const int gofs = 12 * (r >> 1);
+          const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
+          uint32_t ya[3], yb[3];
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt + gofs)[k];
+            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k];
+            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k];
+            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k];
+            ya[k] = prmt(A0, B0, gs);
+            yb[k] = prmt(A1, B1, gs);
+          }
+          const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+            const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t a0, a1, a2, a3;
+              v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
+              v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma_f16(acc[nt][2 * k + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
+          }
+        } else if constexpr (BV == 2) {
+          const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
+          const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
+          const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
+          const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
+#pragma unroll
+          for (int yh = 0; yh < 2; ++yh) {
+            const uint32_t gs = yh ? 0x7362u : 0x5140u;
+            const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+            for (int par = 0; par < 2; ++par) {
+              const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a0, a1, a2, a3;
+                v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
+                v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                  mma_f16(acc[nt][4 * yh + 2 * par + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
+            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
+            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
+            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+#pragma unroll
+            for (int yh = 0; yh < 2; ++yh) {
+              const uint32_t gs = yh ? 0x7362u : 0x5140u;
+              const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a0, a1, a2, a3;
+                v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
+                v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                  mma_f16(acc[nt][4 * u + 2 * yh + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));
+      if (*(volatile int *)&abort_flag) break;
+    }
+
+    // ---------------- all consumers are past the ring: park the state in smem
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kConsumerWarps) : "memory");
+    float *so = reinterpret_cast<float *>(smem);  // [warp][8 NT heads][D], V fragment order
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int hd = 0; hd < 2; ++hd) {
+        float l = l_run[nt][hd];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (r == 0) {
+          sm_m[warp][8 * nt + 2 * q + hd] = m_run[nt][hd];
+          sm_l[warp][8 * nt + 2 * q + hd] = l;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        float *o0 = so + ((warp * 8 * NT) + 8 * nt + 2 * q) * D + 16 * mt + r;
+        o0[0] = acc[nt][mt][0];
+        o0[D] = acc[nt][mt][1];
+        o0[8] = acc[nt][mt][2];
+        o0[D + 8] = acc[nt][mt][3];
+      }
+    }
+  }
+  __syncthreads();
+  if (*(volatile int *)&abort_flag) return;
+
+  // ---------------- combine the consumer warps, write this split's partial
+  const float *so = reinterpret_cast<const float *>(smem);
+  for (int idx = tid; idx < G * D; idx += kThreads) {
+    const int g = idx / D, i = idx % D;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, sm_m[w][g]);
+    float l = 0.f, o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float f = sm_m[w][g] == -INFINITY ? 0.f : exp2f(sm_m[w][g] - mx);
+      l = fmaf(f, sm_l[w][g], l);
+      o = fmaf(f, so[(w * 8 * NT + g) * D + i], o);
+    }
+    float *dst = a.partials + (((long)s * a.n_q_heads + h * G + g) * a.n_splits + split) * (D + 2);
+    dst[2 + i] = o;
+    if (i == 0) {
+      dst[0] = mx;
+      dst[1] = l;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// rotate_q: q_hat = Pi q per (sequence, query head), as 16-bit fixed point in
+// the K fragment order (hi bytes, lo bytes); with QJL also q_tilde = S q_hat.
+// Also the per-head factors that turn the integer dot products into scores in
+// log2 units.  One CTA of 128 threads per row.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float block_max128(float v, float *red) {
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const void *q, int q_dtype, float scale,
+                                                       uint8_t *q8, float *qscale) {
+  __shared__ float s_q[D], s_qh[D];
+  __shared__ int s_int[D];
+  __shared__ float red[4];
+  __shared__ int redi[4];
+  // let the attention kernel start streaming the cache while q is rotated
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int row = blockIdx.x, tid = threadIdx.x;
+  s_q[tid] = q_dtype == TQ_F32 ? static_cast<const float *>(q)[(long)row * D + tid]
+                               : __uint_as_float((uint32_t) static_cast<const uint16_t *>(q)[(long)row * D + tid] << 16);
+  __syncthreads();
+  float qh = 0.f;
+  for (int j = 0; j < D; ++j) qh = fmaf(__uint_as_float((uint32_t)p.pit[j * D + tid] << 16), s_q[j], qh);
+  s_qh[tid] = qh;
+  const float mx = block_max128(fabsf(qh), red);
+  const float mu = mx > 0.f ? 32767.f / mx : 1.f;
+  s_int[tid] = (int)rintf(qh * mu);
+  __syncthreads();
+  uint8_t *dst = q8 + (long)row * 4 * D;
+  {
+    const int v = s_int[p.kperm[tid]];
+    dst[tid] = (uint8_t)(v >> 8);
+    dst[D + tid] = (uint8_t)(v & 0xFF);
+  }
+  const float log2e = 1.4426950408889634f;
+  float fj = 0.f, jsum = 0.f;
+  if (p.qjl) {
+    float qt = 0.f;  // (S q_hat)_tid
+    for (int i = 0; i < D; ++i) qt = fmaf(p.st[i * D + tid], s_qh[i], qt);
+    const float mt = block_max128(fabsf(qt), red);
+    const float nu = mt > 0.f ? 32767.f / mt : 1.f;
+    const int vi = (int)rintf(qt * nu);
+    __syncthreads();
+    s_int[tid] = vi;
+    int sum = vi;
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if ((tid & 31) == 0) redi[tid >> 5] = sum;
+    __syncthreads();
+    jsum = (float)(redi[0] + redi[1] + redi[2] + redi[3]);
+    const int v = s_int[p.jperm[tid]];
+    dst[2 * D + tid] = (uint8_t)(v >> 8);
+    dst[3 * D + tid] = (uint8_t)(v & 0xFF);
+    fj = scale * log2e * sqrtf(0.5f * (float)M_PI) / ((float)D * nu);
+  }
+  if (tid == 0) {
+    float *f = qscale + (long)row * 4;
+    f[0] = scale * log2e / (mu * (float)(1 << kKFixedShift));
+    f[1] = fj;
+    f[2] = jsum;
+    f[3] = 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// merge: per (sequence, query head) combine the splits (log-sum-exp in log2
+// units) and apply Pi^T: o_i = sum_k Pi[vperm(k)][i] o~_k / L.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_heads, const int32_t *seq_lens,
+                                                    int max_seq_len, int chunk, int n_splits,
+                                                    const float *partials, float *out, float *lse) {
+  __shared__ float s_ot[D];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int s = row / n_q_heads;
+  int len = seq_lens[s];
+  len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
+  const int used = (len + chunk - 1) / chunk;
+  const float *src = partials + (long)row * n_splits * (D + 2);
+  float mm = -INFINITY;
+  for (int sp = 0; sp < used; ++sp) mm = fmaxf(mm, src[sp * (D + 2)]);
+  float ll = 0.f, oo = 0.f;
+  for (int sp = 0; sp < used; ++sp) {
+    const float ms = src[sp * (D + 2)];
+    if (ms == -INFINITY) continue;
+    const float f = exp2f(ms - mm);
+    ll = fmaf(f, src[sp * (D + 2) + 1], ll);
+    oo = fmaf(f, src[sp * (D + 2) + 2 + tid], oo);
+  }
+  s_ot[tid] = ll > 0.f ? oo / ll : 0.f;
+  __syncthreads();
+  float acc = 0.f;
+  for (int k = 0; k < D; ++k) acc = fmaf(__uint_as_float((uint32_t)p.piv[k * D + tid] << 16), s_ot[k], acc);
+  out[(long)row * D + tid] = acc;
+  if (lse && tid == 0) lse[row] = ll > 0.f ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
+}
+
+template <int BK, int BV, bool QJL, int NT>
+constexpr int decode_smem_bytes() {
+  const int ring = kStages * Stage<BK, BV, QJL>::bytes;
+  const int park = kConsumerWarps * 8 * NT * D * 4;
+  return ring > park ? ring : park;
+}
+
+using DecodeFn = void (*)(const DecodeArgs);
+
+template <int BK, int BV, bool QJL, int NT>
+DecodeFn pick_nt() {
+  return decode_mma_kernel<BK, BV, QJL, NT>;
+}
+
+struct Variant {
+  DecodeFn fn;
+  int smem;
+};
+
+template <int BK, int BV, bool QJL>
+Variant variant_q(int nt) {
+  if (nt == 1) return {decode_mma_kernel<BK, BV, QJL, 1>, decode_smem_bytes<BK, BV, QJL, 1>()};
+  return {decode_mma_kernel<BK, BV, QJL, 2>, decode_smem_bytes<BK, BV, QJL, 2>()};
+}
+
+template <int BK, int BV>
+Variant variant_v(bool qjl, int nt) {
+  return qjl ? variant_q<BK, BV, true>(nt) : variant_q<BK, BV, false>(nt);
+}
+
+template <int BK>
+Variant variant_k(int bv, bool qjl, int nt) {
+  switch (bv) {
+    case 2: return variant_v<BK, 2>(qjl, nt);
+    case 3: return variant_v<BK, 3>(qjl, nt);
+    default: return variant_v<BK, 4>(qjl, nt);
+  }
+}
+
+Variant variant(int bk, int bv, bool qjl, int nt) {
+  switch (bk) {
+    case 2: return variant_k<2>(bv, qjl, nt);
+    case 3: return variant_k<3>(bv, qjl, nt);
+    default: return variant_k<4>(bv, qjl, nt);
+  }
+}
+
+}  // namespace
+
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group) {
+  static int cache[5][5][2][3] = {};
+  const int nt = group > 8 ? 2 : 1;
+  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt];
+  if (c == 0) {
+    const Variant v = variant(bits_k, bits_v, qjl != 0, nt);
+    cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, v.fn, kThreads, v.smem) != cudaSuccess || n < 1) n = 1;
+    c = n;
+  }
+  return c;
+}
+
+int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype, int n_q_heads,
+                  const int32_t *seq_lens, int max_seq_len, float scale, float *out, float *lse,
+                  char *workspace, const DecodeSplit &split, const DecodeWorkspace &ws, void *stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  const int rows = c.n_seqs * n_q_heads;
+  const int group = n_q_heads / c.n_kv_heads;
+  uint8_t *q8 = reinterpret_cast<uint8_t *>(workspace + ws.q8);
+  float *qscale = reinterpret_cast<float *>(workspace + ws.qscale);
+  float *partials = reinterpret_cast<float *>(workspace + ws.partials);
+
+  rotate_q_kernel<<<rows, 128, 0, st>>>(p, q, q_dtype, scale, q8, qscale);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return (int)e;
+
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+
+  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1);
+  DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q8, qscale, partials};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(split.n_splits, c.n_kv_heads, c.n_seqs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = v.smem;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, v.fn, args);
+  if (e != cudaSuccess) return (int)e;
+
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3(rows);
+  mcfg.blockDim = dim3(128);
+  mcfg.stream = st;
+  mcfg.attrs = pdl;
+  mcfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&mcfg, merge_kernel, p, n_q_heads, seq_lens, max_seq_len, split.chunk, split.n_splits,
+                         (const float *)partials, out, lse);
+  return (int)e;
+}
+
+}  // namespace tq

@@ -29,6 +29,15 @@ void codebook(int bits, int d, float *centroids, float *thresholds);
 // Bytes of one packed vector of codes.
 inline int code_bytes(int bits) { return kHeadDim * bits / 8; }
 
+// Byte tables for the byte-permute lookups of the decode kernel: lo[i] packs
+// the low bytes of entries 4i..4i+3, hi[i] their high bytes.  K entries are
+// the centroids as 16-bit fixed point (c * 2^kKFixedShift); V entries are the
+// fp16 bit patterns of the centroids.
+struct Lut {
+  uint32_t lo[4], hi[4];
+};
+constexpr int kKFixedShift = 17;
+
 // Device-resident parameters of one context (all pointers device memory).
 struct DeviceParams {
   const uint16_t *pi;     // Pi  [d][d] bf16 bits, row-major (z = Pi x)
@@ -37,23 +46,34 @@ struct DeviceParams {
   const float *st;        // S^T [d][d] fp32 (qjl only)
   const float *cb;        // [4][16]: centroids_k, thresholds_k, centroids_v, thresholds_v
   unsigned *err;          // sticky error flags
+  const uint8_t *kperm;   // [d] K fragment order -> coordinate
+  const uint8_t *jperm;   // [d] QJL fragment order -> projection index
+  const uint16_t *piv;    // [d][d] bf16: row k is row vperm[k] of Pi (V fragment order)
+  Lut lut_k, lut_v;
   int bits_k, bits_v, qjl;
 };
+
+// Fragment orders of the decode kernel (host, tq_api.cu).
+void kperm_of(int bits, uint8_t *perm);
+void vperm_of(int bits, uint8_t *perm);
+void jperm_of(uint8_t *perm);
 
 // Split of the sequence axis used by decode attention.
 struct DecodeSplit {
   int chunk;     // tokens per split (multiple of 64)
   int n_splits;  // ceil(max_seq_len / chunk), at least 1
 };
-DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len);
+DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm);
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group);
 
-// Workspace layout of decode attention (byte offsets, 256-aligned).
+// Workspace layout of decode attention (byte offsets, 256-aligned):
+// q8 [rows][4][d] bytes, qscale [rows][4] floats, partials [rows][splits][d+2].
 struct DecodeWorkspace {
-  size_t q_hat, q_tilde, partials, total;
+  size_t q8, qscale, partials, total;
 };
-DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, int qjl, DecodeSplit split);
+DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split);
 
-// --- launches (tq_kernels.cu); return cudaGetLastError() as int ---
+// --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
 int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype,
