@@ -44,9 +44,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn over packed KV: effective GB/s (% HBM peak); quantize tokens/s"
-WORKLOAD_DESC = ("llama8b: Llama-3-8B-shaped single layer, 8 KV / 32 query heads (GQA 4), d=128, "
-                 "32768 cached tokens, batch 1, bf16 K/V ~ N(0,I) x LogNormal(0,0.5) per (token, head), "
-                 "3-bit K and V (turbo3, no QJL); step = append-quantize 1 token + decode attention")
+WORKLOAD_DESCS = {
+    "llama8b": ("llama8b: Llama-3-8B-shaped single layer, 8 KV / 32 query heads (GQA 4), d=128, "
+                "32768 cached tokens, batch 1, bf16 K/V ~ N(0,I) x LogNormal(0,0.5) per (token, head), "
+                "3-bit K and V (turbo3, no QJL); step = append-quantize 1 token + decode attention"),
+    "llama70b": ("llama70b: 70B-shaped long context, 8 KV / 64 query heads (GQA 8), d=128, 131072 cached "
+                 "tokens, batch 4, bf16 K/V ~ N(0,1) with 10 (head, channel) outliers x20, 3-bit K and V; "
+                 "step = append-quantize 1 token per sequence + batched decode attention"),
+}
+WORKLOAD_DESC = WORKLOAD_DESCS["llama8b"]
 
 
 def measured_peaks():
@@ -205,7 +211,8 @@ def main(argv=None) -> int:
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
-    ap.add_argument("--replicas", type=int, default=10)
+    ap.add_argument("--replicas", type=int, default=0, help="cache replicas (default: enough to exceed L2)")
+    ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOAD_DESCS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -223,54 +230,60 @@ def main(argv=None) -> int:
 
     from kv_cache_vector_12_b200 import tq
     from kv_cache_vector_12_b200 import workloads as wl
-    w = wl.WORKLOADS["llama8b"]
-    T, H, HQ, D = w.seq_len, w.n_kv_heads, w.n_q_heads, w.d
-    R = args.replicas
+    w = wl.WORKLOADS[args.workload]
+    T, H, HQ, D, B = w.seq_len, w.n_kv_heads, w.n_q_heads, w.d, w.n_seqs
+    bytes_per_token = H * (D * (w.bits_k + w.bits_v) // 8 + 4)
+    R = args.replicas or max(1, math.ceil(2 * 126e6 / (B * T * bytes_per_token)))
     n_steps_total = args.warmup + args.steps
     cap = int(math.ceil((T + n_steps_total + 1) / 64) * 64)
     ctx = tq.Context(D, w.bits_k, w.bits_v, 0, w.pi_seed)
-    caches = [tq.Cache(ctx, 1, H, cap, device=dev) for _ in range(R)]
+    caches = [tq.Cache(ctx, B, H, cap, device=dev) for _ in range(R)]
     gen = wl.generator(dev, w.seed + 7919 * rank)
+    outl = wl.outlier_scale(w, dev, w.seed) if args.workload == "llama70b" else None
 
-    # ---- prefill quantize (also the quantize measurement) ----
-    k_pre, v_pre = wl.kv_tokens(w, T, gen, dev)
-    seq0 = torch.zeros(T, dtype=torch.int32, device=dev)
+    # ---- prefill quantize (also the quantize measurement: the first sequence) ----
     pos0 = torch.arange(T, dtype=torch.int32, device=dev)
-    for c in caches:
-        tq.quantize(ctx, c, k_pre, v_pre, seq0, pos0)
+    q_ms = None
+    for b in range(B):
+        k_pre, v_pre = wl.kv_tokens(w, T, gen, dev, outlier_mask=outl)
+        seqb = torch.full((T,), b, dtype=torch.int32, device=dev)
+        for c in caches:
+            tq.quantize(ctx, c, k_pre, v_pre, seqb, pos0)
+        if b == 0:
+            torch.cuda.synchronize()
+            qreps = 10
+            qe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * qreps)]
+            for i in range(qreps):
+                qe[2 * i].record()
+                tq.quantize(ctx, caches[i % R], k_pre, v_pre, seqb, pos0)
+                qe[2 * i + 1].record()
+            torch.cuda.synchronize()
+            q_ms = statistics.median(qe[2 * i].elapsed_time(qe[2 * i + 1]) for i in range(qreps))
+        del k_pre, v_pre
     torch.cuda.synchronize()
-    qreps = 10
-    qe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * qreps)]
-    for i in range(qreps):
-        qe[2 * i].record()
-        tq.quantize(ctx, caches[i % R], k_pre, v_pre, seq0, pos0)
-        qe[2 * i + 1].record()
-    torch.cuda.synchronize()
-    q_ms = statistics.median(qe[2 * i].elapsed_time(qe[2 * i + 1]) for i in range(qreps))
     ctx.check_device_errors()
 
     # ---- per-step inputs, resident on the device ----
-    k_new, v_new = wl.kv_tokens(w, n_steps_total, gen, dev)           # [steps, H, D]
-    q_all = wl.queries(w, n_steps_total, gen, dev)                     # [steps, HQ, D]
-    pos_steps = torch.empty(n_steps_total, dtype=torch.int32, device=dev)
-    lens_steps = torch.empty(n_steps_total, dtype=torch.int32, device=dev)
+    k_new, v_new = wl.kv_tokens(w, n_steps_total * B, gen, dev, outlier_mask=outl)   # [steps*B, H, D]
+    q_all = wl.queries(w, n_steps_total * B, gen, dev).view(n_steps_total, B, HQ, D)
+    pos_steps = torch.empty(n_steps_total, B, dtype=torch.int32, device=dev)
+    lens_steps = torch.empty(n_steps_total, B, dtype=torch.int32, device=dev)
     for i in range(n_steps_total):
         p = T + i // R
         pos_steps[i] = p
         lens_steps[i] = p + 1
-    out = torch.empty(n_steps_total, 1, HQ, D, device=dev)
-    lse = torch.empty(n_steps_total, 1, HQ, device=dev)
+    out = torch.empty(n_steps_total, B, HQ, D, device=dev)
+    lse = torch.empty(n_steps_total, B, HQ, device=dev)
     max_len = cap
-    wsb = tq.alloc_workspace(ctx, 1, HQ, max_len, device=dev)
-    zero_seq = torch.zeros(1, dtype=torch.int32, device=dev)
+    wsb = tq.alloc_workspace(ctx, B, HQ, max_len, device=dev)
+    seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
 
     def step(i):
         c = caches[i % R]
-        tq.quantize(ctx, c, k_new[i:i + 1], v_new[i:i + 1], zero_seq, pos_steps[i:i + 1])
-        tq.decode_attention(ctx, c, q_all[i:i + 1], lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+        tq.quantize(ctx, c, k_new[i * B:(i + 1) * B], v_new[i * B:(i + 1) * B], seq_ids, pos_steps[i])
+        tq.decode_attention(ctx, c, q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
 
-    bytes_per_token = H * (D * (w.bits_k + w.bits_v) // 8 + 4)
-    step_bytes = [int(lens_steps[i]) * bytes_per_token for i in range(n_steps_total)]
+    step_bytes = [int(lens_steps[i].sum()) * bytes_per_token for i in range(n_steps_total)]
 
     # graphs of the warm-up and timed steps
     s = torch.cuda.Stream(device=dev)
@@ -307,9 +320,9 @@ def main(argv=None) -> int:
     de = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
     for j, i in enumerate(range(args.warmup, n_steps_total)):
         c = caches[i % R]
-        tq.quantize(ctx, c, k_new[i:i + 1], v_new[i:i + 1], zero_seq, pos_steps[i:i + 1])
+        tq.quantize(ctx, c, k_new[i * B:(i + 1) * B], v_new[i * B:(i + 1) * B], seq_ids, pos_steps[i])
         de[2 * j].record()
-        tq.decode_attention(ctx, c, q_all[i:i + 1], lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+        tq.decode_attention(ctx, c, q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
         de[2 * j + 1].record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -320,20 +333,20 @@ def main(argv=None) -> int:
     k_h = k_new.cpu().pin_memory()
     v_h = v_new.cpu().pin_memory()
     q_h = q_all.cpu().pin_memory()
-    out_h = torch.empty(1, HQ, D).pin_memory()
-    k_d = torch.empty(1, H, D, dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty(B, HQ, D).pin_memory()
+    k_d = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
     v_d = torch.empty_like(k_d)
-    q_d = torch.empty(1, HQ, D, dtype=torch.bfloat16, device=dev)
+    q_d = torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)
     h2d = k_d.numel() * 2 * 2 + q_d.numel() * 2
     d2h = out_h.numel() * 4
 
     def e2e_step(i):
         c = caches[i % R]
-        k_d.copy_(k_h[i:i + 1], non_blocking=True)
-        v_d.copy_(v_h[i:i + 1], non_blocking=True)
-        q_d.copy_(q_h[i:i + 1], non_blocking=True)
-        tq.quantize(ctx, c, k_d, v_d, zero_seq, pos_steps[i:i + 1])
-        tq.decode_attention(ctx, c, q_d, lens_steps[i:i + 1], max_len, out[i], lse[i], wsb)
+        k_d.copy_(k_h[i * B:(i + 1) * B], non_blocking=True)
+        v_d.copy_(v_h[i * B:(i + 1) * B], non_blocking=True)
+        q_d.copy_(q_h[i], non_blocking=True)
+        tq.quantize(ctx, c, k_d, v_d, seq_ids, pos_steps[i])
+        tq.decode_attention(ctx, c, q_d, lens_steps[i], max_len, out[i], lse[i], wsb)
         out_h.copy_(out[i], non_blocking=True)
 
     for i in range(args.warmup):
@@ -374,7 +387,7 @@ def main(argv=None) -> int:
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
+        "config": {"workload": WORKLOAD_DESCS[args.workload], "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
                    f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
