@@ -173,6 +173,29 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache,
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Allocation-free decode attention (no counterpart in the method's sources;
+ * it is a deployment variant of tq_decode_attention).  For callers that cannot
+ * allocate device memory while they decode: code inside CUDA graph stream
+ * capture, engines restricted to their own memory pool, latency-critical
+ * loops that cannot absorb cudaMalloc's implicit synchronisation.  Same
+ * arguments and results as tq_decode_attention, minus the workspace: the
+ * workspace is a static device array of TQ_NOALLOC_SCRATCH_BYTES built into
+ * the library (held by every GPU that loads it until exit).  Calls that need
+ * more than that (see tq_workspace_bytes) fail with TQ_ERR_INVALID and launch
+ * nothing.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array, so calls whose kernels overlap on the GPU
+ * (other streams, other threads) race; it allocates nothing itself.
+ */
+#define TQ_NOALLOC_SCRATCH_BYTES (8 * 1024 * 1024)
+tq_status tq_decode_attention_noalloc(tq_ctx *ctx, const tq_cache *cache,
+                                      const void *q, int32_t q_dtype,
+                                      int32_t n_q_heads,
+                                      const int32_t *seq_lens,
+                                      int32_t max_seq_len, float scale,
+                                      float *out, float *lse, void *stream);
+
+/*
  * Synchronise `stream`, then report and clear the context's sticky
  * device-side error flags: TQ_OK, or TQ_ERR_DEVICE with a message naming the
  * flags (bit 0: token outside the cache in tq_quantize; bit 1: seq_len

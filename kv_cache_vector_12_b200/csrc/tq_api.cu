@@ -144,6 +144,14 @@ DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_p
   return sp;
 }
 
+tq_status report_error(tq_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
 DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t rows = (size_t)n_seqs * n_q_heads;

@@ -73,6 +73,9 @@ struct DecodeWorkspace {
 };
 DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split);
 
+// Record a message for tq_last_error() and return `st` (tq_api.cu).
+tq_status report_error(tq_status st, const char *fmt, ...);
+
 // --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);

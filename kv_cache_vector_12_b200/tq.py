@@ -50,6 +50,9 @@ lib.tq_workspace_bytes.restype = ctypes.c_size_t
 lib.tq_decode_attention.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp, _i32,
                                     ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.tq_decode_attention.restype = ctypes.c_int
+lib.tq_decode_attention_noalloc.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp, _i32,
+                                            ctypes.c_float, _vp, _vp, _vp]
+lib.tq_decode_attention_noalloc.restype = ctypes.c_int
 lib.tq_check_device_errors.argtypes = [_vp, _vp]
 lib.tq_check_device_errors.restype = ctypes.c_int
 lib.tq_last_error.argtypes = []
@@ -187,6 +190,18 @@ def decode_attention(ctx: Context, cache: Cache, q: torch.Tensor, seq_lens: torc
                                    _ptr(seq_lens), max_seq_len, scale, _ptr(out), _ptr(lse),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)))
+
+
+def decode_attention_noalloc(ctx: Context, cache: Cache, q: torch.Tensor, seq_lens: torch.Tensor,
+                             max_seq_len: int, out: torch.Tensor, lse: torch.Tensor | None,
+                             scale: float = 0.0, stream=None) -> None:
+    """tq_decode_attention_noalloc: decode attention without a caller workspace,
+    for callers that cannot allocate device memory (the library's static
+    scratch is used instead; concurrent calls on the GPU race on it)."""
+    q_dtype = TQ_F32 if q.dtype == torch.float32 else TQ_BF16
+    _check(lib.tq_decode_attention_noalloc(ctx.handle, ctypes.byref(cache.struct), _ptr(q), q_dtype, q.shape[1],
+                                           _ptr(seq_lens), max_seq_len, scale, _ptr(out), _ptr(lse),
+                                           _stream(stream)))
 
 
 def alloc_workspace(ctx: Context, n_seqs: int, n_q_heads: int, max_seq_len: int, device="cuda") -> torch.Tensor:
