@@ -95,8 +95,8 @@ typedef struct tq_cache {
  * signed so that R has a positive diagonal, rounded to bf16 (the "random
  * orthogonal matrix" of "ステップ1: PolarQuant").  The codebook of b bits is
  * the Lloyd-Max quantizer of N(0,1) scaled by 1/sqrt(d) ("Lloyd-Max量子化";
- * the N(0,1/d) law is the "ガウス分布に近い" coordinate law) in fp32, with
- * fp32 midpoints as thresholds.  With qjl, S is a second d x d Gaussian from
+ * the N(0,1/d) law is the "ガウス分布に近い" coordinate law), its centroids
+ * rounded to fp16 and the exact midpoints (fp32) as thresholds.  With qjl, S is a second d x d Gaussian from
  * counters 2^32+1.. (fp32).  Allocates and uploads the parameters
  * (synchronous); the only call that allocates device memory.
  * Errors: TQ_ERR_INVALID (null out, bits outside {2,3,4}, qjl outside {0,1}),

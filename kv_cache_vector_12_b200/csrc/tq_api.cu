@@ -235,7 +235,7 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
-  // One block: pi | pit | piv | s | st | codebooks | kperm | jperm | error word.
+  // One block: pi | pit | pivt | s | st | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
   const size_t off_pi = 0, off_pit = off_pi + dd * 2, off_piv = off_pit + dd * 2, off_s = off_piv + dd * 2;
   const size_t off_st = off_s + dd * 4, off_cb = off_st + dd * 4;
@@ -257,9 +257,9 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < d; ++j) st_h[(size_t)j * d + i] = ctx->s[(size_t)i * d + j];
   }
-  uint16_t *piv = (uint16_t *)(h.data() + off_piv);
-  for (int k = 0; k < d; ++k)
-    for (int i = 0; i < d; ++i) piv[(size_t)k * d + i] = ctx->pi_bits[(size_t)vperm[k] * d + i];
+  uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
+  for (int i = 0; i < d; ++i)
+    for (int k = 0; k < d; ++k) pivt[(size_t)i * d + k] = ctx->pi_bits[(size_t)vperm[k] * d + i];
   std::memcpy(h.data() + off_kperm, kperm, tq::kHeadDim);
   std::memcpy(h.data() + off_jperm, jperm, tq::kHeadDim);
   float *cb = (float *)(h.data() + off_cb);
@@ -280,7 +280,7 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->dp.st = (const float *)(base + off_st);
   ctx->dp.cb = (const float *)(base + off_cb);
   ctx->dp.err = (unsigned *)(base + off_err);
-  ctx->dp.piv = (const uint16_t *)(base + off_piv);
+  ctx->dp.pivt = (const uint16_t *)(base + off_piv);
   ctx->dp.kperm = (const uint8_t *)(base + off_kperm);
   ctx->dp.jperm = (const uint8_t *)(base + off_jperm);
   ctx->dp.bits_k = bits_k;

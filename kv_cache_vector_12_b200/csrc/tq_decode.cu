@@ -584,6 +584,42 @@ __device__ __forceinline__ float block_max128(float v, float *red) {
   return r;
 }
 
+// Dot product of a bf16 row (128 entries, 16-byte aligned) with a vector in
+// shared memory: 16 independent 16-byte loads, four partial sums.
+__device__ __forceinline__ float dot_bf16_row(const uint16_t *row, const float *x) {
+  uint4 w[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) w[c] = reinterpret_cast<const uint4 *>(row)[c];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 8 * c + 2 * e;
+      acc[e] = fmaf(__uint_as_float(u[e] << 16), x[j], acc[e]);
+      acc[e] = fmaf(__uint_as_float(u[e] & 0xffff0000u), x[j + 1], acc[e]);
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Same for an fp32 row.
+__device__ __forceinline__ float dot_f32_row(const float *row, const float *x) {
+  float4 w[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = reinterpret_cast<const float4 *>(row)[c];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    acc[0] = fmaf(w[c].x, x[4 * c], acc[0]);
+    acc[1] = fmaf(w[c].y, x[4 * c + 1], acc[1]);
+    acc[2] = fmaf(w[c].z, x[4 * c + 2], acc[2]);
+    acc[3] = fmaf(w[c].w, x[4 * c + 3], acc[3]);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const void *q, int q_dtype, float scale,
                                                        uint8_t *q8, float *qscale) {
   __shared__ float s_q[D], s_qh[D];
@@ -596,8 +632,7 @@ __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const voi
   s_q[tid] = q_dtype == TQ_F32 ? static_cast<const float *>(q)[(long)row * D + tid]
                                : __uint_as_float((uint32_t) static_cast<const uint16_t *>(q)[(long)row * D + tid] << 16);
   __syncthreads();
-  float qh = 0.f;
-  for (int j = 0; j < D; ++j) qh = fmaf(__uint_as_float((uint32_t)p.pit[j * D + tid] << 16), s_q[j], qh);
+  const float qh = dot_bf16_row(p.pi + tid * D, s_q);  // (Pi q)_tid
   s_qh[tid] = qh;
   const float mx = block_max128(fabsf(qh), red);
   const float mu = mx > 0.f ? 32767.f / mx : 1.f;
@@ -612,8 +647,7 @@ __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const voi
   const float log2e = 1.4426950408889634f;
   float fj = 0.f, jsum = 0.f;
   if (p.qjl) {
-    float qt = 0.f;  // (S q_hat)_tid
-    for (int i = 0; i < D; ++i) qt = fmaf(p.st[i * D + tid], s_qh[i], qt);
+    const float qt = dot_f32_row(p.s + tid * D, s_qh);  // (S q_hat)_tid
     const float mt = block_max128(fabsf(qt), red);
     const float nu = mt > 0.f ? 32767.f / mt : 1.f;
     const int vi = (int)rintf(qt * nu);
@@ -642,32 +676,53 @@ __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const voi
 // merge: per (sequence, query head) combine the splits (log-sum-exp in log2
 // units) and apply Pi^T: o_i = sum_k Pi[vperm(k)][i] o~_k / L.
 // ---------------------------------------------------------------------------
+constexpr int kMergeMaxSplits = 1024;
+
 __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_heads, const int32_t *seq_lens,
                                                     int max_seq_len, int chunk, int n_splits,
                                                     const float *partials, float *out, float *lse) {
   __shared__ float s_ot[D];
+  __shared__ float s_w[kMergeMaxSplits];
+  __shared__ float red[4];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x, tid = threadIdx.x;
   const int s = row / n_q_heads;
   int len = seq_lens[s];
   len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
-  const int used = (len + chunk - 1) / chunk;
+  const int used = min((len + chunk - 1) / chunk, kMergeMaxSplits);
   const float *src = partials + (long)row * n_splits * (D + 2);
-  float mm = -INFINITY;
-  for (int sp = 0; sp < used; ++sp) mm = fmaxf(mm, src[sp * (D + 2)]);
+  // split maxima (log2 units) in parallel, then the weights 2^(m_s - M)
+  float mloc = -INFINITY;
+  for (int sp = tid; sp < used; sp += 128) {
+    const float m = src[sp * (D + 2)];
+    s_w[sp] = m;
+    mloc = fmaxf(mloc, m);
+  }
+  const float mm = block_max128(mloc, red);
+  for (int sp = tid; sp < used; sp += 128) s_w[sp] = s_w[sp] == -INFINITY ? 0.f : exp2f(s_w[sp] - mm);
+  __syncthreads();
   float ll = 0.f, oo = 0.f;
-  for (int sp = 0; sp < used; ++sp) {
-    const float ms = src[sp * (D + 2)];
-    if (ms == -INFINITY) continue;
-    const float f = exp2f(ms - mm);
-    ll = fmaf(f, src[sp * (D + 2) + 1], ll);
-    oo = fmaf(f, src[sp * (D + 2) + 2 + tid], oo);
+  int sp = 0;
+  for (; sp + 4 <= used; sp += 4) {
+    float l4[4], o4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      l4[e] = src[(sp + e) * (D + 2) + 1];
+      o4[e] = src[(sp + e) * (D + 2) + 2 + tid];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ll = fmaf(s_w[sp + e], l4[e], ll);
+      oo = fmaf(s_w[sp + e], o4[e], oo);
+    }
+  }
+  for (; sp < used; ++sp) {
+    ll = fmaf(s_w[sp], src[sp * (D + 2) + 1], ll);
+    oo = fmaf(s_w[sp], src[sp * (D + 2) + 2 + tid], oo);
   }
   s_ot[tid] = ll > 0.f ? oo / ll : 0.f;
   __syncthreads();
-  float acc = 0.f;
-  for (int k = 0; k < D; ++k) acc = fmaf(__uint_as_float((uint32_t)p.piv[k * D + tid] << 16), s_ot[k], acc);
-  out[(long)row * D + tid] = acc;
+  out[(long)row * D + tid] = dot_bf16_row(p.pivt + tid * D, s_ot);
   if (lse && tid == 0) lse[row] = ll > 0.f ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
 }
 

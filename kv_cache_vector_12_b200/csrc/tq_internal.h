@@ -48,7 +48,7 @@ struct DeviceParams {
   unsigned *err;          // sticky error flags
   const uint8_t *kperm;   // [d] K fragment order -> coordinate
   const uint8_t *jperm;   // [d] QJL fragment order -> projection index
-  const uint16_t *piv;    // [d][d] bf16: row k is row vperm[k] of Pi (V fragment order)
+  const uint16_t *pivt;   // [d][d] bf16: pivt[i][k] = Pi[vperm[k]][i] (Pi^T, columns in V fragment order)
   Lut lut_k, lut_v;
   int bits_k, bits_v, qjl;
 };
@@ -79,6 +79,8 @@ tq_status report_error(tq_status st, const char *fmt, ...);
 // --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
+int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
+                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream);
 int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype,
                   int n_q_heads, const int32_t *seq_lens, int max_seq_len, float scale,
                   float *out, float *lse, char *workspace, const DecodeSplit &split,

@@ -25,10 +25,6 @@ __device__ __forceinline__ uint16_t f32_to_f16_bits_sat(float x) {
   return __half_as_ushort(__float2half_rn(fminf(x, 65504.f)));
 }
 
-__device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {
-  return __half2float(__ushort_as_half(h));
-}
-
 // Bit position of bit k of coordinate i's code inside a packed vector (the
 // layout documented in tq.h).
 __device__ __forceinline__ int code_bit_pos(int bits, int i, int k) {
@@ -36,15 +32,6 @@ __device__ __forceinline__ int code_bit_pos(int bits, int i, int k) {
   const int g = i >> 5, l = i & 31;
   if (l < 24) return 96 * g + 32 * (l >> 3) + 4 * (l & 7) + k;
   return 96 * g + 32 * k + 4 * (l - 24) + 3;
-}
-
-__device__ __forceinline__ int read_code(const uint8_t *vec, int bits, int i) {
-  int c = 0;
-  for (int k = 0; k < bits; ++k) {
-    const int p = code_bit_pos(bits, i, k);
-    c |= ((vec[p >> 3] >> (p & 7)) & 1) << k;
-  }
-  return c;
 }
 
 // ---------------------------------------------------------------------------
@@ -140,10 +127,15 @@ __global__ void __launch_bounds__(128) quantize_kernel(DeviceParams p, tq_cache 
 
 }  // namespace
 
+// MSE-only rows (all of V; K without QJL) go through the tensor-core kernel;
+// K rows with the QJL stage use quantize_kernel (grid.y = 1 selects K only).
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream) {
+  const bool k_on_tc = !p.qjl;
+  const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, stream);
+  if (e != 0 || k_on_tc) return e;
   const long rows = (long)n_tok * c.n_kv_heads;
-  dim3 grid((unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta), 2);
+  dim3 grid((unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta), 1);
   quantize_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
                                                           seq_idx, pos, n_tok);
   return (int)cudaGetLastError();

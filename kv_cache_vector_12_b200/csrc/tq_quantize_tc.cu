@@ -1,0 +1,438 @@
+// Quantize-on-append on the 5th-generation tensor cores (sm_100a).
+//
+// "ステップ1: PolarQuant" (ai-accelerate.xyz TurboQuant explainer): every
+// head vector x is rotated by the random orthogonal matrix Pi and each rotated
+// coordinate is quantized with the Lloyd-Max codebook.  Here the rotation of
+// a tile of 128 head vectors is one 128x128x128 bf16 GEMM, z = X Pi^T:
+//
+//   producer warp   TMA (cp.async.bulk.tensor, 128-byte swizzle) loads each
+//                   128-row tile of K or V into a 4-deep shared-memory ring;
+//                   Pi stays resident in shared memory for the CTA's lifetime.
+//   MMA warp        one thread issues 8 tcgen05.mma (kind::f16, bf16 inputs,
+//                   fp32 accumulation in tensor memory) per tile and commits
+//                   to mbarriers.
+//   3 epilogue      warpgroups, one TMEM accumulator each; every thread owns
+//   warpgroups      one row (vector): ||x|| from the shared-memory tile,
+//                   z from TMEM (tcgen05.ld 32x32b), codes against the
+//                   thresholds scaled by ||x||, bit-packing into the cache
+//                   layout, 16-byte stores, fp16 norm.
+//
+// The kernel is persistent (one CTA per SM, tiles strided by the grid).  Every
+// mbarrier wait is bounded; on expiry the kernel flags the error, stops, waits
+// for its copies and MMAs in flight (bounded) and releases its tensor memory.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kTileRows = 128;
+constexpr int kRingStages = 4;
+constexpr int kEpiGroups = 3;
+constexpr int kQThreads = 32 * (2 + 4 * kEpiGroups);
+constexpr int kTileBytes = kTileRows * D * 2;     // 32 KB: two 128x64 bf16 boxes
+constexpr int kBoxBytes = kTileBytes / 2;
+constexpr unsigned kTmemCols = 512;               // 3 accumulators of 128 columns
+constexpr unsigned kSpinLimit = 1u << 22;
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void bar_init(uint32_t b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(n));
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint32_t b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(ok)
+               : "r"(b), "r"(parity)
+               : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity) {
+  for (unsigned i = 0; i < kSpinLimit; ++i)
+    if (bar_try(b, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (start address and offsets in 16-byte units).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = 128, M = 128.
+constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                   tmem_d),
+               "l"(a), "l"(b), "r"(kInstrDesc), "r"(accumulate)
+               : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct QuantTcArgs {
+  DeviceParams p;
+  tq_cache c;
+  const int32_t *seq_idx;
+  const int32_t *pos;
+  int n_rows;       // n_tok * n_kv_heads rows per matrix
+  int tiles_k;      // tiles of K handled here (0 when K goes elsewhere)
+  int tiles_v;
+};
+
+// Code of one rotated coordinate: #{j : T_j < z} with T_j = t_j ||x||,
+// evaluated as sign + count of the positive thresholds below |z| (the
+// codebook is symmetric, t_{half-1} = 0).  z = 0 (also a zero vector) gives
+// half - 1.
+template <int B>
+__device__ __forceinline__ uint32_t code_of(float z, const float (&tp)[(1 << (B - 1)) - 1]) {
+  constexpr int half = 1 << (B - 1);
+  const float a = fabsf(z);
+  int m = 0;
+#pragma unroll
+  for (int j = 0; j < half - 1; ++j) m += a > tp[j] ? 1 : 0;
+  return (uint32_t)(z > 0.f ? half + m : half - 1 - m);
+}
+
+// Pack the 32 codes of coordinate group g into words w[g*B .. g*B+B) of the
+// cache layout (LSB-first for 2 and 4 bits; nibble + spare-column layout for 3).
+template <int B>
+__device__ __forceinline__ void pack_group(const uint32_t (&cd)[32], uint32_t *w) {
+  if constexpr (B == 3) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x |= cd[8 * k + j] << (4 * j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x |= ((cd[24 + j] >> k) & 1u) << (4 * j + 3);
+      w[k] = x;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < B; ++k) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int j = 0; j < 32 / B; ++j) x |= cd[(32 / B) * k + j] << (B * j);
+      w[k] = x;
+    }
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], float n, uint32_t tmem_row,
+                                             uint32_t (&words)[4 * B]) {
+  constexpr int half = 1 << (B - 1);
+  float tp[half - 1];
+#pragma unroll
+  for (int j = 0; j < half - 1; ++j) tp[j] = thr[half + j] * n;  // positive thresholds, scaled
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float z[32];
+    tmem_ld32(tmem_row + 32 * g, z);
+    uint32_t cd[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cd[i] = code_of<B>(z[i], tp);
+    pack_group<B>(cd, words + g * B);
+  }
+}
+
+__global__ void __launch_bounds__(kQThreads, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                       const __grid_constant__ CUtensorMap map_pi, const QuantTcArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned region: Pi (32 KB) then the ring
+  unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char *pi_tile = smem;
+  unsigned char *ring = smem + kTileBytes;
+  __shared__ __align__(8) uint64_t full_bar[kRingStages], empty_bar[kRingStages];
+  __shared__ __align__(8) uint64_t tfull_bar[kEpiGroups], tempty_bar[kEpiGroups], pi_bar;
+  __shared__ uint32_t tmem_base_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = a.tiles_k + a.tiles_v;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingStages; ++i) {
+      bar_init(smem_addr(&full_bar[i]), 1);
+      bar_init(smem_addr(&empty_bar[i]), 1 + 4);  // MMA commit + the 4 norm-reading warps
+    }
+    for (int g = 0; g < kEpiGroups; ++g) {
+      bar_init(smem_addr(&tfull_bar[g]), 1);
+      bar_init(smem_addr(&tempty_bar[g]), 4);
+    }
+    bar_init(smem_addr(&pi_bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // the MMA warp owns the tensor memory
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer (TMA)
+    if (lane == 0) {
+      const uint32_t pb = smem_addr(&pi_bar);
+      bar_expect_tx(pb, kTileBytes);
+      tma_load_2d(smem_addr(pi_tile), &map_pi, 0, 0, pb);
+      tma_load_2d(smem_addr(pi_tile + kBoxBytes), &map_pi, 64, 0, pb);
+      int i = 0, issued = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+        const int slot = i % kRingStages;
+        if (i >= kRingStages && !bar_wait(smem_addr(&empty_bar[slot]), ((i / kRingStages) - 1) & 1)) {
+          atomicOr(a.p.err, kErrWaitExpired);
+          abort_flag = 1;
+          break;
+        }
+        if (*(volatile int *)&abort_flag) break;
+        const bool is_k = t < a.tiles_k;
+        const CUtensorMap *map = is_k ? &map_k : &map_v;
+        const int row0 = (is_k ? t : t - a.tiles_k) * kTileRows;
+        const uint32_t fb = smem_addr(&full_bar[slot]);
+        unsigned char *st = ring + slot * kTileBytes;
+        bar_expect_tx(fb, kTileBytes);
+        tma_load_2d(smem_addr(st), map, 0, row0, fb);
+        tma_load_2d(smem_addr(st + kBoxBytes), map, 64, row0, fb);
+        issued = i + 1;
+      }
+      bar_wait(pb, 0);
+      if (*(volatile int *)&abort_flag)  // drain: never leave copies in flight
+        for (int k = (issued > kRingStages ? issued - kRingStages : 0); k < issued; ++k)
+          bar_wait(smem_addr(&full_bar[k % kRingStages]), (k / kRingStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = bar_wait(smem_addr(&pi_bar), 0);
+      int i = 0;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++i) {
+        const int slot = i % kRingStages, acc = i % kEpiGroups;
+        ok = bar_wait(smem_addr(&full_bar[slot]), (i / kRingStages) & 1);
+        if (ok && i >= kEpiGroups) ok = bar_wait(smem_addr(&tempty_bar[acc]), ((i / kEpiGroups) - 1) & 1);
+        if (!ok || *(volatile int *)&abort_flag) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_addr(ring + slot * kTileBytes), b0 = smem_addr(pi_tile);
+        const uint32_t d = tmem_base + acc * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;  // 16 bf16 along K per MMA
+          tc_mma(d, sw128_desc(a0 + off), sw128_desc(b0 + off), kk > 0);
+        }
+        tc_commit(smem_addr(&tfull_bar[acc]));
+        tc_commit(smem_addr(&empty_bar[slot]));
+      }
+      if (!ok) {
+        atomicOr(a.p.err, kErrWaitExpired);
+        abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue warpgroups
+    const int g = (warp - 2) / 4;
+    const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
+    const int r = 32 * quarter + lane;             // the row this thread owns
+    for (int j = 0, t = blockIdx.x + g * gridDim.x; t < n_tiles; ++j, t += kEpiGroups * gridDim.x) {
+      const int i = g + j * kEpiGroups;            // tile sequence number within this CTA
+      const int slot = i % kRingStages;
+      if (!bar_wait(smem_addr(&full_bar[slot]), (i / kRingStages) & 1)) {
+        atomicOr(a.p.err, kErrWaitExpired);
+        abort_flag = 1;
+        break;
+      }
+      // ||x|| from the swizzled tile (the order of the 16-byte chunks is
+      // irrelevant to a sum of squares); bf16 squares are exact in fp32
+      const unsigned char *st = ring + slot * kTileBytes;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int box = 0; box < 2; ++box)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 u = *reinterpret_cast<const uint4 *>(st + box * kBoxBytes + r * 128 + ch * 16);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
+            s0 = fmaf(lo, lo, s0);
+            s1 = fmaf(hi, hi, s1);
+          }
+        }
+      const float nrm = sqrtf(s0 + s1);
+      __syncwarp();
+      if (lane == 0) bar_arrive(smem_addr(&empty_bar[slot]));
+
+      const bool is_k = t < a.tiles_k;
+      const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
+      if (!bar_wait(smem_addr(&tfull_bar[g]), j & 1)) {
+        atomicOr(a.p.err, kErrWaitExpired);
+        abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int bits = is_k ? a.p.bits_k : a.p.bits_v;
+      const float *thr = a.p.cb + (is_k ? 1 : 3) * kMaxLevels;
+      float tl[kMaxLevels];
+#pragma unroll
+      for (int e = 0; e < kMaxLevels; ++e) tl[e] = thr[e];
+      const uint32_t trow = tmem_base + g * 128 + ((uint32_t)(32 * quarter) << 16);
+      uint32_t words[16];
+      if (bits == 2) {
+        uint32_t w[8];
+        epilogue_row<2>(tl, nrm, trow, w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) words[e] = w[e];
+      } else if (bits == 3) {
+        uint32_t w[12];
+        epilogue_row<3>(tl, nrm, trow, w);
+#pragma unroll
+        for (int e = 0; e < 12; ++e) words[e] = w[e];
+      } else {
+        uint32_t w[16];
+        epilogue_row<4>(tl, nrm, trow, w);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) words[e] = w[e];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(smem_addr(&tempty_bar[g]));
+
+      if (row < a.n_rows) {
+        const int tok = row / a.c.n_kv_heads, h = row % a.c.n_kv_heads;
+        const int s = a.seq_idx[tok], ps = a.pos[tok];
+        if (s >= 0 && s < a.c.n_seqs && ps >= 0 && ps < a.c.capacity) {
+          const long slot_i = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + ps;
+          uint4 *dst = reinterpret_cast<uint4 *>((is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(16 * bits));
+          for (int q = 0; q < bits; ++q)
+            dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+          (is_k ? a.c.norm_k : a.c.norm_v)[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
+        } else if (h == 0 && is_k) {
+          atomicOr(a.p.err, kErrTokenRange);
+        }
+      }
+      if (*(volatile int *)&abort_flag) break;
+    }
+  }
+
+  // release tensor memory once every MMA and every tcgen05.ld is finished
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][128] bf16 matrix, boxes of 128 rows x 64
+// columns (128 bytes) with the 128-byte swizzle the MMA descriptors expect.
+bool make_row_map(CUtensorMap *m, const void *base, long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTileRows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+constexpr int kQuantTcSmem = 1024 + kTileBytes * (1 + kRingStages);
+
+int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
+                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream) {
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+    cudaFuncSetAttribute(quantize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
+  }
+  const long rows = (long)n_tok * c.n_kv_heads;
+  CUtensorMap mk, mv, mp;
+  std::memset(&mk, 0, sizeof mk);
+  if (!make_row_map(&mv, v, rows) || !make_row_map(&mp, p.pi, D) || (include_k && !make_row_map(&mk, k, rows)))
+    return (int)cudaErrorInvalidValue;
+  if (!include_k) mk = mv;
+  QuantTcArgs args{p, c, seq_idx, pos, (int)rows, 0, 0};
+  const int tiles = (int)((rows + kTileRows - 1) / kTileRows);
+  args.tiles_k = include_k ? tiles : 0;
+  args.tiles_v = tiles;
+  const int total = args.tiles_k + args.tiles_v;
+  const int grid = total < n_sm ? total : n_sm;
+  quantize_tc_kernel<<<grid, kQThreads, kQuantTcSmem, (cudaStream_t)stream>>>(mk, mv, mp, args);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace tq
