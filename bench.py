@@ -213,6 +213,8 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--replicas", type=int, default=0, help="cache replicas (default: enough to exceed L2)")
     ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOAD_DESCS))
+    ap.add_argument("--breakdown", action="store_true",
+                    help="also time each call kind alone (append quantize, decode) and add it to the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -329,6 +331,30 @@ def main(argv=None) -> int:
     dec_ms = [de[2 * j].elapsed_time(de[2 * j + 1]) for j in range(args.steps)]
     ctx.check_device_errors()
 
+    breakdown = None
+    if args.breakdown:
+        def timed(fn, reps=50):
+            for _ in range(5):
+                fn()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record()
+            for _ in range(reps):
+                fn()
+            ev[1].record()
+            torch.cuda.synchronize()
+            return ev[0].elapsed_time(ev[1]) * 1e3 / reps
+        i_last = n_steps_total - 1
+        c_last = caches[i_last % R]
+        breakdown = {
+            "append_quantize_us": timed(lambda: tq.quantize(ctx, c_last, k_new[i_last * B:(i_last + 1) * B],
+                                                            v_new[i_last * B:(i_last + 1) * B], seq_ids,
+                                                            pos_steps[i_last])),
+            "decode_call_us": timed(lambda: tq.decode_attention(ctx, c_last, q_all[i_last], lens_steps[i_last],
+                                                                max_len, out[i_last], lse[i_last], wsb)),
+            "note": "eager calls back to back on one cache (warm L2), events on the stream",
+        }
+        torch.cuda.synchronize()
+
     # ---- end to end through the C ABI with pinned host buffers (eager) ----
     k_h = k_new.cpu().pin_memory()
     v_h = v_new.cpu().pin_memory()
@@ -399,6 +425,7 @@ def main(argv=None) -> int:
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * args.steps,
+        "breakdown": breakdown,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -182,6 +182,7 @@ __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], flo
   }
 }
 
+template <int BK, int BV>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                        const __grid_constant__ CUtensorMap map_pi, const QuantTcArgs a) {
@@ -284,23 +285,47 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int g = (warp - 2) / 4;
     const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
     const int r = 32 * quarter + lane;             // the row this thread owns
+    // thresholds of both codebooks, once
+    float tk[kMaxLevels], tv[kMaxLevels];
+#pragma unroll
+    for (int e = 0; e < kMaxLevels; ++e) {
+      tk[e] = a.p.cb[1 * kMaxLevels + e];
+      tv[e] = a.p.cb[3 * kMaxLevels + e];
+    }
     for (int j = 0, t = blockIdx.x + g * gridDim.x; t < n_tiles; ++j, t += kEpiGroups * gridDim.x) {
       const int i = g + j * kEpiGroups;            // tile sequence number within this CTA
       const int slot = i % kRingStages;
+      const bool is_k = t < a.tiles_k;
+      const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
+      // destination of this row, fetched early (used after the codes)
+      long slot_i = -1;
+      int tok_h = 0;
+      if (row < a.n_rows) {
+        const int tok = row / a.c.n_kv_heads;
+        tok_h = row - tok * a.c.n_kv_heads;
+        const int s = a.seq_idx[tok], ps = a.pos[tok];
+        if (s >= 0 && s < a.c.n_seqs && ps >= 0 && ps < a.c.capacity)
+          slot_i = ((long)s * a.c.n_kv_heads + tok_h) * a.c.capacity + ps;
+        else if (tok_h == 0 && is_k)
+          atomicOr(a.p.err, kErrTokenRange);
+      }
       if (!bar_wait(smem_addr(&full_bar[slot]), (i / kRingStages) & 1)) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
         break;
       }
-      // ||x|| from the swizzled tile (the order of the 16-byte chunks is
-      // irrelevant to a sum of squares); bf16 squares are exact in fp32
+      // ||x|| from the swizzled tile.  Row r's 128-byte segment holds its 16-byte
+      // chunks permuted by r % 8; reading chunk c ^ (r % 8) keeps a warp's loads
+      // conflict-free, and the order does not matter to a sum of squares.  bf16
+      // squares are exact in fp32.
       const unsigned char *st = ring + slot * kTileBytes;
       float s0 = 0.f, s1 = 0.f;
 #pragma unroll
       for (int box = 0; box < 2; ++box)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(st + box * kBoxBytes + r * 128 + ch * 16);
+          const uint4 u =
+              *reinterpret_cast<const uint4 *>(st + box * kBoxBytes + r * 128 + ((ch ^ (r & 7)) * 16));
           const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -313,53 +338,36 @@ __global__ void __launch_bounds__(kQThreads, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(smem_addr(&empty_bar[slot]));
 
-      const bool is_k = t < a.tiles_k;
-      const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
       if (!bar_wait(smem_addr(&tfull_bar[g]), j & 1)) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int bits = is_k ? a.p.bits_k : a.p.bits_v;
-      const float *thr = a.p.cb + (is_k ? 1 : 3) * kMaxLevels;
-      float tl[kMaxLevels];
-#pragma unroll
-      for (int e = 0; e < kMaxLevels; ++e) tl[e] = thr[e];
       const uint32_t trow = tmem_base + g * 128 + ((uint32_t)(32 * quarter) << 16);
       uint32_t words[16];
-      if (bits == 2) {
-        uint32_t w[8];
-        epilogue_row<2>(tl, nrm, trow, w);
+      if (is_k) {
+        uint32_t w[4 * BK];
+        epilogue_row<BK>(tk, nrm, trow, w);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) words[e] = w[e];
-      } else if (bits == 3) {
-        uint32_t w[12];
-        epilogue_row<3>(tl, nrm, trow, w);
-#pragma unroll
-        for (int e = 0; e < 12; ++e) words[e] = w[e];
+        for (int e = 0; e < 4 * BK; ++e) words[e] = w[e];
       } else {
-        uint32_t w[16];
-        epilogue_row<4>(tl, nrm, trow, w);
+        uint32_t w[4 * BV];
+        epilogue_row<BV>(tv, nrm, trow, w);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) words[e] = w[e];
+        for (int e = 0; e < 4 * BV; ++e) words[e] = w[e];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(smem_addr(&tempty_bar[g]));
 
-      if (row < a.n_rows) {
-        const int tok = row / a.c.n_kv_heads, h = row % a.c.n_kv_heads;
-        const int s = a.seq_idx[tok], ps = a.pos[tok];
-        if (s >= 0 && s < a.c.n_seqs && ps >= 0 && ps < a.c.capacity) {
-          const long slot_i = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + ps;
-          uint4 *dst = reinterpret_cast<uint4 *>((is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(16 * bits));
-          for (int q = 0; q < bits; ++q)
-            dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-          (is_k ? a.c.norm_k : a.c.norm_v)[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
-        } else if (h == 0 && is_k) {
-          atomicOr(a.p.err, kErrTokenRange);
-        }
+      if (slot_i >= 0) {
+        const int bits = is_k ? BK : BV;
+        uint4 *dst = reinterpret_cast<uint4 *>((is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(16 * bits));
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < bits) dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+        (is_k ? a.c.norm_k : a.c.norm_v)[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
       }
       if (*(volatile int *)&abort_flag) break;
     }
@@ -406,18 +414,33 @@ bool make_row_map(CUtensorMap *m, const void *base, long rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
 constexpr int kQuantTcSmem = 1024 + kTileBytes * (1 + kRingStages);
+
+using QuantTcFn = void (*)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
+                           const __grid_constant__ CUtensorMap, const QuantTcArgs);
+
+template <int BK>
+QuantTcFn pick_bv(int bv) {
+  return bv == 2 ? quantize_tc_kernel<BK, 2> : bv == 3 ? quantize_tc_kernel<BK, 3> : quantize_tc_kernel<BK, 4>;
+}
+
+QuantTcFn pick(int bk, int bv) { return bk == 2 ? pick_bv<2>(bv) : bk == 3 ? pick_bv<3>(bv) : pick_bv<4>(bv); }
+
+}  // namespace
 
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream) {
   static int n_sm = 0;
+  static bool configured[5][5] = {};
   if (n_sm == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
-    cudaFuncSetAttribute(quantize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
+  }
+  const QuantTcFn fn = pick(p.bits_k, p.bits_v);
+  if (!configured[p.bits_k][p.bits_v]) {
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
+    configured[p.bits_k][p.bits_v] = true;
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   CUtensorMap mk, mv, mp;
@@ -431,7 +454,7 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
   args.tiles_v = tiles;
   const int total = args.tiles_k + args.tiles_v;
   const int grid = total < n_sm ? total : n_sm;
-  quantize_tc_kernel<<<grid, kQThreads, kQuantTcSmem, (cudaStream_t)stream>>>(mk, mv, mp, args);
+  fn<<<grid, kQThreads, kQuantTcSmem, (cudaStream_t)stream>>>(mk, mv, mp, args);
   return (int)cudaGetLastError();
 }
 
