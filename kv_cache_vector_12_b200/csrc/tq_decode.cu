@@ -34,11 +34,11 @@ namespace tq {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = 8;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStageTokens = 16 * kConsumerWarps;  // 64
-constexpr int kStages = 6;
-constexpr unsigned kWaitLimit = 1u << 22;           // bounded mbarrier waits
+constexpr int kStageTokens = 16 * kConsumerWarps;  // 128
+constexpr int kStages = 5;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ PTX
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
@@ -73,11 +73,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of the barrier; false if the bounded wait expired.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of the barrier; false once 2 s have passed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (unsigned i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -203,7 +213,8 @@ struct DecodeArgs {
 };
 
 template <int BK, int BV, bool QJL, int NT>
-__global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(const DecodeArgs a) {
+__global__ void __maxnreg__(112) decode_mma_kernel(const DecodeArgs a) {
+  static_assert(kStageTokens % 64 == 0, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
@@ -249,15 +260,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(const DecodeArg
         if (*(volatile int *)&abort_flag) break;
         unsigned char *st = smem + slot * St::bytes;
         const uint32_t bar = smem_u32(&full_bar[slot]);
-        const long tok = base + t0 + (long)it * kStageTokens;
-        mbar_arrive_expect_tx(bar, St::bytes);
-        bulk_g2s(smem_u32(st + St::kc), a.c.codes_k + tok * (D * BK / 8), kStageTokens * D * BK / 8, bar);
-        bulk_g2s(smem_u32(st + St::vc), a.c.codes_v + tok * (D * BV / 8), kStageTokens * D * BV / 8, bar);
-        bulk_g2s(smem_u32(st + St::kn), a.c.norm_k + tok, kStageTokens * 2, bar);
-        bulk_g2s(smem_u32(st + St::vn), a.c.norm_v + tok, kStageTokens * 2, bar);
+        const int first = t0 + it * kStageTokens;  // multiple of 64, below the capacity
+        // a stage never reads past the capacity (a multiple of 64, not of 128)
+        const uint32_t n = (uint32_t)min(kStageTokens, a.c.capacity - first);
+        const long tok = base + first;
+        const uint32_t bytes = n * (D * BK / 8 + D * BV / 8 + 4 + (QJL ? D / 8 + 2 : 0));
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(smem_u32(st + St::kc), a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8), bar);
+        bulk_g2s(smem_u32(st + St::vc), a.c.codes_v + tok * (D * BV / 8), n * (D * BV / 8), bar);
+        bulk_g2s(smem_u32(st + St::kn), a.c.norm_k + tok, n * 2, bar);
+        bulk_g2s(smem_u32(st + St::vn), a.c.norm_v + tok, n * 2, bar);
         if constexpr (QJL) {
-          bulk_g2s(smem_u32(st + St::jb), a.c.qjl_bits + tok * (D / 8), kStageTokens * D / 8, bar);
-          bulk_g2s(smem_u32(st + St::jg), a.c.qjl_norm + tok, kStageTokens * 2, bar);
+          bulk_g2s(smem_u32(st + St::jb), a.c.qjl_bits + tok * (D / 8), n * (D / 8), bar);
+          bulk_g2s(smem_u32(st + St::jg), a.c.qjl_norm + tok, n * 2, bar);
         }
         issued = it + 1;
       }
@@ -782,6 +797,7 @@ int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group) {
   if (c == 0) {
     const Variant v = variant(bits_k, bits_v, qjl != 0, nt);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
+    cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, v.fn, kThreads, v.smem) != cudaSuccess || n < 1) n = 1;
     c = n;
