@@ -34,10 +34,10 @@ namespace tq {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStageTokens = 16 * kConsumerWarps;  // 128
-constexpr int kStages = 5;
+constexpr int kStageTokens = 16 * kConsumerWarps;  // 64
+constexpr int kStages = 6;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ PTX
@@ -213,7 +213,7 @@ struct DecodeArgs {
 };
 
 template <int BK, int BV, bool QJL, int NT>
-__global__ void __maxnreg__(112) decode_mma_kernel(const DecodeArgs a) {
+__global__ void __maxnreg__(96) decode_mma_kernel(const DecodeArgs a) {
   static_assert(kStageTokens % 64 == 0, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
   extern __shared__ __align__(128) unsigned char smem[];

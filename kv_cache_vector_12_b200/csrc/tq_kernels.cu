@@ -1,5 +1,6 @@
-// TurboQuant quantize-on-append kernel for sm_100a: norm, rotation by Pi,
-// Lloyd-Max codes, bit-pack, optional QJL residual signs.
+// TurboQuant quantize-on-append for sm_100a, small batches and QJL rows:
+// norm, rotation by Pi, Lloyd-Max codes, bit-pack, optional QJL residual
+// signs; and the dispatch between this kernel and the tensor-core kernel.
 //
 // The method: ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み"
 // (rotation + per-coordinate Lloyd-Max, then the 1-bit QJL residual
@@ -35,109 +36,132 @@ __device__ __forceinline__ int code_bit_pos(int bits, int i, int k) {
 }
 
 // ---------------------------------------------------------------------------
-// quantize: one CTA (128 threads = one thread per coordinate) per chunk of
-// rows; Pi^T staged in shared memory once per CTA.
+// quantize, one CTA per head vector (small batches, and K rows with QJL):
+// thread i owns coordinate i.  z_i = (Pi x)_i from row i of Pi (16-byte loads,
+// L2-resident), ||x|| by a block reduction (fp32 over exact bf16 squares), the
+// code against the thresholds scaled by ||x||, packing by warp OR-reductions
+// (one warp = one 32-coordinate group of the layout).  With QJL:
+// r = z/||x|| - c[code], ||r||, (S r)_m from row m of S, one sign ballot per
+// warp.  grid = (rows, 2): y = 0 for K, 1 for V.
 // ---------------------------------------------------------------------------
-constexpr int kQuantRowsPerCta = 64;
+__device__ __forceinline__ float row_dot_bf16(const uint16_t *row, const float *x) {
+  uint4 w[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) w[c] = reinterpret_cast<const uint4 *>(row)[c];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[e] = fmaf(__uint_as_float(u[e] << 16), x[8 * c + 2 * e], acc[e]);
+      acc[e] = fmaf(__uint_as_float(u[e] & 0xffff0000u), x[8 * c + 2 * e + 1], acc[e]);
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
 
-__global__ void __launch_bounds__(128) quantize_kernel(DeviceParams p, tq_cache c,
-                                                       const uint16_t *__restrict__ k_in,
-                                                       const uint16_t *__restrict__ v_in,
-                                                       const int32_t *__restrict__ seq_idx,
-                                                       const int32_t *__restrict__ pos, int n_tok) {
-  __shared__ uint16_t s_pit[D * D];
-  __shared__ float s_x[D];
-  __shared__ float s_r[D];
-  __shared__ double s_red[4];
-  __shared__ float s_redf[4];
+__device__ __forceinline__ float row_dot_f32(const float *row, const float *x) {
+  float4 w[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = reinterpret_cast<const float4 *>(row)[c];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    acc[0] = fmaf(w[c].x, x[4 * c], acc[0]);
+    acc[1] = fmaf(w[c].y, x[4 * c + 1], acc[1]);
+    acc[2] = fmaf(w[c].z, x[4 * c + 2], acc[2]);
+    acc[3] = fmaf(w[c].w, x[4 * c + 3], acc[3]);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
 
+__device__ __forceinline__ float block_sum128(float v, float *red) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const float r = (red[0] + red[1]) + (red[2] + red[3]);
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_cache c,
+                                                           const uint16_t *__restrict__ k_in,
+                                                           const uint16_t *__restrict__ v_in,
+                                                           const int32_t *__restrict__ seq_idx,
+                                                           const int32_t *__restrict__ pos) {
+  __shared__ float s_x[D], s_r[D];
+  __shared__ float red[4];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool is_v = blockIdx.y == 1;
   const int bits = is_v ? p.bits_v : p.bits_k;
   const bool qjl = !is_v && p.qjl;
-  const float *cent = p.cb + (is_v ? 2 : 0) * kMaxLevels;
+  const long row = blockIdx.x;
+  const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
+  const int s = seq_idx[t], ps = pos[t];
+  if (!(s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity)) {
+    if (tid == 0 && !is_v) atomicOr(p.err, kErrTokenRange);
+    return;
+  }
+  const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * D + tid]);
+  s_x[tid] = x;
+  const float n = sqrtf(block_sum128(x * x, red));  // also orders s_x
+  const float z = row_dot_bf16(p.pi + tid * D, s_x);
   const float *thr = p.cb + (is_v ? 3 : 1) * kMaxLevels;
-  const int levels = 1 << bits;
-  const uint16_t *x_in = is_v ? v_in : k_in;
-  uint8_t *codes_plane = is_v ? c.codes_v : c.codes_k;
-  uint16_t *norm_plane = is_v ? c.norm_v : c.norm_k;
-  const int cbytes = D * bits / 8;
+  const int half = 1 << (bits - 1);
+  const float a = fabsf(z);
+  int m = 0;
+  for (int j = 0; j < half - 1; ++j) m += a > thr[half + j] * n ? 1 : 0;
+  const int code = z > 0.f ? half + m : half - 1 - m;
 
-  for (int e = tid; e < D * D; e += 128) s_pit[e] = p.pit[e];
-  __syncthreads();
-
-  const long n_rows = (long)n_tok * c.n_kv_heads;
-  const long row0 = (long)blockIdx.x * kQuantRowsPerCta;
-  for (long row = row0; row < row0 + kQuantRowsPerCta && row < n_rows; ++row) {
-    const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
-    const int s = seq_idx[t], ps = pos[t];
-    const bool ok = s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity;
-    if (!ok) {
-      if (tid == 0 && !is_v) atomicOr(p.err, kErrTokenRange);
-      continue;
+  const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
+  uint32_t *dst = reinterpret_cast<uint32_t *>((is_v ? c.codes_v : c.codes_k) + slot * (D * bits / 8));
+  for (int wd = 0; wd < bits; ++wd) {  // warp w owns words w*bits .. w*bits+bits-1
+    uint32_t contrib = 0;
+    for (int kb = 0; kb < bits; ++kb) {
+      const int pbit = code_bit_pos(bits, tid, kb) - 32 * bits * warp;
+      if ((pbit >> 5) == wd) contrib |= (uint32_t)((code >> kb) & 1) << (pbit & 31);
     }
-    const float x = bf16_bits_to_f32(x_in[row * D + tid]);
-    s_x[tid] = x;
-    // ||x||^2 in fp64: every square of a bf16 value is exact.
-    double sq = (double)x * (double)x;
-    for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) s_red[warp] = sq;
-    __syncthreads();
-    const double n64 = sqrt(s_red[0] + s_red[1] + s_red[2] + s_red[3]);
-    float z = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < D; ++j) z = fmaf(bf16_bits_to_f32(s_pit[j * D + tid]), s_x[j], z);
-    const float n = (float)n64;
+    const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
+    if (lane == 0) dst[warp * bits + wd] = word;
+  }
+  if (tid == 0) (is_v ? c.norm_v : c.norm_k)[slot] = f32_to_f16_bits_sat(n);
+
+  if (qjl) {
+    const float *cent = p.cb;  // K centroids
     const float y = n > 0.f ? z / n : 0.f;
-    int code = 0;
-    for (int j = 0; j < levels - 1; ++j) code += thr[j] < y ? 1 : 0;
-
-    const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
-    // pack: warp w owns coordinates 32w..32w+31 (one group for 3 bits)
-    uint8_t *dst = codes_plane + slot * cbytes;
-    const int words = bits;  // 32 coordinates * bits / 32 bits per word
-    for (int wd = 0; wd < words; ++wd) {
-      uint32_t contrib = 0;
-      for (int kb = 0; kb < bits; ++kb) {
-        const int pbit = code_bit_pos(bits, tid, kb) - 32 * bits * warp;  // within this warp's words
-        if ((pbit >> 5) == wd) contrib |= (uint32_t)((code >> kb) & 1) << (pbit & 31);
-      }
-      const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
-      if (lane == 0) reinterpret_cast<uint32_t *>(dst)[warp * words + wd] = word;
-    }
-    if (tid == 0) norm_plane[slot] = __half_as_ushort(__double2half(fmin(n64, 65504.0)));
-
-    if (qjl) {
-      const float r = y - cent[code];
-      s_r[tid] = r;
-      float r2 = r * r;
-      for (int o = 16; o; o >>= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, o);
-      if (lane == 0) s_redf[warp] = r2;
-      __syncthreads();
-      const float gamma = sqrtf(s_redf[0] + s_redf[1] + s_redf[2] + s_redf[3]);
-      float proj = 0.f;  // (S r)_tid
-      for (int i = 0; i < D; ++i) proj = fmaf(p.st[i * D + tid], s_r[i], proj);
-      const uint32_t sb = __ballot_sync(0xffffffffu, proj >= 0.f);
-      if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (D / 8))[warp] = sb;
-      if (tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(gamma);
-    }
-    __syncthreads();
+    const float r = y - cent[code];
+    s_r[tid] = r;
+    const float gamma = sqrtf(block_sum128(r * r, red));
+    const float proj = row_dot_f32(p.s + tid * D, s_r);  // (S r)_tid
+    const uint32_t sb = __ballot_sync(0xffffffffu, proj >= 0.f);
+    if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (D / 8))[warp] = sb;
+    if (tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(gamma);
   }
 }
 
 }  // namespace
 
-// MSE-only rows (all of V; K without QJL) go through the tensor-core kernel;
-// K rows with the QJL stage use quantize_kernel (grid.y = 1 selects K only).
+// Batches of up to kRowKernelMaxRows rows per matrix (decode-time appends) use
+// the one-CTA-per-row kernel; larger batches use the tensor-core kernel for
+// every MSE-only matrix (all of V, K without QJL) and the row kernel for K
+// rows with QJL.
+constexpr long kRowKernelMaxRows = 1024;
+
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream) {
+  const long rows = (long)n_tok * c.n_kv_heads;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows <= kRowKernelMaxRows) {
+    quantize_row_kernel<<<dim3((unsigned)rows, 2), 128, 0, st>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
+                                                               seq_idx, pos);
+    return (int)cudaGetLastError();
+  }
   const bool k_on_tc = !p.qjl;
   const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, stream);
   if (e != 0 || k_on_tc) return e;
-  const long rows = (long)n_tok * c.n_kv_heads;
-  dim3 grid((unsigned)((rows + kQuantRowsPerCta - 1) / kQuantRowsPerCta), 1);
-  quantize_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
-                                                          seq_idx, pos, n_tok);
+  quantize_row_kernel<<<dim3((unsigned)rows, 1), 128, 0, st>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
+                                                             seq_idx, pos);
   return (int)cudaGetLastError();
 }
 
