@@ -36,8 +36,9 @@ namespace {
 constexpr int D = kHeadDim;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStageTokens = 16 * kConsumerWarps;  // 64
-constexpr int kStages = 6;
+constexpr int kWarpTokens = 32;                            // tokens per consumer warp per stage
+constexpr int kStageTokens = kWarpTokens * kConsumerWarps;  // 128
+constexpr int kStages = 4;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ PTX
@@ -213,8 +214,8 @@ struct DecodeArgs {
 };
 
 template <int BK, int BV, bool QJL, int NT>
-__global__ void __maxnreg__(96) decode_mma_kernel(const DecodeArgs a) {
-  static_assert(kStageTokens % 64 == 0, "stages start on 64-token boundaries");
+__global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
+  static_assert(kStageTokens % 64 == 0 && kWarpTokens == 32, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
@@ -340,103 +341,120 @@ __global__ void __maxnreg__(96) decode_mma_kernel(const DecodeArgs a) {
         break;
       }
       const unsigned char *st = smem + slot * St::bytes;
-      const int tok0 = t0 + it * kStageTokens + 16 * warp;  // first token of this warp's tile
+      const int tok0 = t0 + it * kStageTokens + kWarpTokens * warp;  // first token of this warp's tile
       if (tok0 < t1) {
-        const int wt = 16 * warp;                            // tile row offset inside the stage
-        // ---------------- scores: int8 MMA over 4 k-steps of 32
-        int chh[NT][4], cmid[NT][4], cll[NT][4], cjh[NT][4], cjl[NT][4];
+        const int wt = kWarpTokens * warp;                             // tile row offset inside the stage
+        // ---------------- scores: int8 MMA, two 16-token row blocks, 4 k-steps of 32
+        int chh[2][NT][4], cmid[2][NT][4], cll[2][NT][4], cjh[2][NT][4], cjl[2][NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) chh[nt][e] = cmid[nt][e] = cll[nt][e] = cjh[nt][e] = cjl[nt][e] = 0;
-        uint32_t wk0[BK], wk1[BK];
-        const unsigned char *kr0 = st + St::kc + (wt + r) * (D * BK / 8) + q * 4 * BK;
-        const unsigned char *kr1 = kr0 + 8 * (D * BK / 8);
+          for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < BK; ++i) {
-          wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
-          wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
-        }
+            for (int e = 0; e < 4; ++e) chh[rb][nt][e] = cmid[rb][nt][e] = cll[rb][nt][e] = cjh[rb][nt][e] = cjl[rb][nt][e] = 0;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t alo[4], ahi[4];
-          lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks), alo[0], ahi[0]);
-          lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks), alo[1], ahi[1]);
-          lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks + 1), alo[2], ahi[2]);
-          lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks + 1), alo[3], ahi[3]);
+        for (int rb = 0; rb < 2; ++rb) {
+          uint32_t wk0[BK], wk1[BK];
+          const unsigned char *kr0 = st + St::kc + (wt + 16 * rb + r) * (D * BK / 8) + q * 4 * BK;
+          const unsigned char *kr1 = kr0 + 8 * (D * BK / 8);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_i8<true, true>(chh[nt], ahi[0], ahi[1], ahi[2], ahi[3], qh[nt][ks][0], qh[nt][ks][1]);
-            mma_i8<true, false>(cmid[nt], ahi[0], ahi[1], ahi[2], ahi[3], ql[nt][ks][0], ql[nt][ks][1]);
-            mma_i8<false, true>(cmid[nt], alo[0], alo[1], alo[2], alo[3], qh[nt][ks][0], qh[nt][ks][1]);
-            mma_i8<false, false>(cll[nt], alo[0], alo[1], alo[2], alo[3], ql[nt][ks][0], ql[nt][ks][1]);
+          for (int i = 0; i < BK; ++i) {
+            wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
+            wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
           }
-        }
-        if constexpr (QJL) {
-          const uint32_t w0 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + r) * (D / 8))[q];
-          const uint32_t w1 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + r + 8) * (D / 8))[q];
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            // bytes 0x00 / 0xFF (= -bit) for bits j, j+8, j+16, j+24 with j = 2 ks + slot
-            const int j0 = 2 * ks, j1 = 2 * ks + 1;
-            const uint32_t a0 = prmt(w0 << (7 - j0), 0u, 0xBA98u), a1 = prmt(w1 << (7 - j0), 0u, 0xBA98u);
-            const uint32_t a2 = prmt(w0 << (7 - j1), 0u, 0xBA98u), a3 = prmt(w1 << (7 - j1), 0u, 0xBA98u);
+            uint32_t alo[4], ahi[4];
+            lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks), alo[0], ahi[0]);
+            lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks), alo[1], ahi[1]);
+            lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks + 1), alo[2], ahi[2]);
+            lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks + 1), alo[3], ahi[3]);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              mma_i8<true, true>(cjh[nt], a0, a1, a2, a3, jh[nt][ks][0], jh[nt][ks][1]);
-              mma_i8<true, false>(cjl[nt], a0, a1, a2, a3, jl[nt][ks][0], jl[nt][ks][1]);
+              mma_i8<true, true>(chh[rb][nt], ahi[0], ahi[1], ahi[2], ahi[3], qh[nt][ks][0], qh[nt][ks][1]);
+              mma_i8<true, false>(cmid[rb][nt], ahi[0], ahi[1], ahi[2], ahi[3], ql[nt][ks][0], ql[nt][ks][1]);
+              mma_i8<false, true>(cmid[rb][nt], alo[0], alo[1], alo[2], alo[3], qh[nt][ks][0], qh[nt][ks][1]);
+              mma_i8<false, false>(cll[rb][nt], alo[0], alo[1], alo[2], alo[3], ql[nt][ks][0], ql[nt][ks][1]);
+            }
+          }
+          if constexpr (QJL) {
+            const uint32_t w0 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + 16 * rb + r) * (D / 8))[q];
+            const uint32_t w1 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + 16 * rb + r + 8) * (D / 8))[q];
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              // bytes 0x00 / 0xFF (= -bit) for bits j, j+8, j+16, j+24 with j = 2 ks + slot
+              const int j0 = 2 * ks, j1 = 2 * ks + 1;
+              const uint32_t a0 = prmt(w0 << (7 - j0), 0u, 0xBA98u), a1 = prmt(w1 << (7 - j0), 0u, 0xBA98u);
+              const uint32_t a2 = prmt(w0 << (7 - j1), 0u, 0xBA98u), a3 = prmt(w1 << (7 - j1), 0u, 0xBA98u);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                mma_i8<true, true>(cjh[rb][nt], a0, a1, a2, a3, jh[nt][ks][0], jh[nt][ks][1]);
+                mma_i8<true, false>(cjl[rb][nt], a0, a1, a2, a3, jl[nt][ks][0], jl[nt][ks][1]);
+              }
             }
           }
         }
-        // ---------------- scores -> online softmax
+        // ---------------- scores -> online softmax over the 32 tokens
+        // this thread's tokens: wt + 16 rb + r + 8 hf  (rb, hf in {0, 1})
         const __half *kn = reinterpret_cast<const __half *>(st + St::kn) + wt;
         const __half *vn = reinterpret_cast<const __half *>(st + St::vn) + wt;
-        const float nk0 = __half2float(kn[r]), nk1 = __half2float(kn[r + 8]);
-        const float nv0 = __half2float(vn[r]), nv1 = __half2float(vn[r + 8]);
-        float gm0 = 0.f, gm1 = 0.f;
-        if constexpr (QJL) {
-          const __half *jg = reinterpret_cast<const __half *>(st + St::jg) + wt;
-          gm0 = __half2float(jg[r]);
-          gm1 = __half2float(jg[r + 8]);
+        float nk[4], nv[4], gm[4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tt = 16 * (u >> 1) + r + 8 * (u & 1);
+          nk[u] = __half2float(kn[tt]);
+          nv[u] = __half2float(vn[tt]);
+          ok[u] = tok0 + tt < t1;
+          gm[u] = 0.f;
+          if constexpr (QJL) gm[u] = __half2float(reinterpret_cast<const __half *>(st + St::jg)[wt + tt]);
         }
-        const bool ok0 = tok0 + r < t1, ok1 = tok0 + r + 8 < t1;
-        uint32_t pb[NT][2];
+        uint32_t pb[2][NT][2];
         bool rescale = false;
         float alpha[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float sc[4];
+          float sc[4][2];  // [token u][head hd]
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int hd = e & 1;
-            const float dot = fmaf(65536.f, (float)chh[nt][e], fmaf(256.f, (float)cmid[nt][e], (float)cll[nt][e]));
-            float v = dot * fq[nt][hd];
-            if constexpr (QJL) {
-              const float dj = fmaf(256.f, (float)cjh[nt][e], (float)cjl[nt][e]);
-              v = fmaf((e < 2 ? gm0 : gm1) * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+              const int rb = u >> 1, e = 2 * (u & 1) + hd;
+              // 65536 hh + 256 mid + ll = 256 (256 hh + mid) + ll; 256 hh + mid fits int32
+              const int hm = (chh[rb][nt][e] << 8) + cmid[rb][nt][e];
+              float v = fmaf(256.f, (float)hm, (float)cll[rb][nt][e]) * fq[nt][hd];
+              if constexpr (QJL) {
+                const float dj = fmaf(256.f, (float)cjh[rb][nt][e], (float)cjl[rb][nt][e]);
+                v = fmaf(gm[u] * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
+              }
+              sc[u][hd] = ok[u] ? v * nk[u] : -INFINITY;
             }
-            v *= (e < 2 ? nk0 : nk1);
-            sc[e] = (e < 2 ? ok0 : ok1) ? v : -INFINITY;
-          }
 #pragma unroll
           for (int hd = 0; hd < 2; ++hd) {
-            float mx = fmaxf(sc[hd], sc[hd + 2]);
+            float mx = fmaxf(fmaxf(sc[0][hd], sc[1][hd]), fmaxf(sc[2][hd], sc[3][hd]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             const float mn = fmaxf(m_run[nt][hd], mx);
-            const float al = mn == -INFINITY ? 1.f : exp2f(m_run[nt][hd] - mn);
+            const bool none = mn == -INFINITY;
+            const float al = none ? 1.f : exp2f(m_run[nt][hd] - mn);
             alpha[nt][hd] = al;
             rescale |= al != 1.f;
             m_run[nt][hd] = mn;
-            const float p0 = mn == -INFINITY ? 0.f : exp2f(sc[hd] - mn);
-            const float p1 = mn == -INFINITY ? 0.f : exp2f(sc[hd + 2] - mn);
-            l_run[nt][hd] = fmaf(l_run[nt][hd], al, p0 + p1);
-            sc[hd] = ok0 ? p0 * nv0 : 0.f;
-            sc[hd + 2] = ok1 ? p1 * nv1 : 0.f;
+            float lsum = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float pv = none ? 0.f : exp2f(sc[u][hd] - mn);
+              lsum += pv;
+              sc[u][hd] = ok[u] ? pv * nv[u] : 0.f;
+            }
+            l_run[nt][hd] = fmaf(l_run[nt][hd], al, lsum);
           }
-          pb[nt][0] = movmatrix_trans(pack_half2(sc[0], sc[1]));
-          pb[nt][1] = movmatrix_trans(pack_half2(sc[2], sc[3]));
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb) {
+            pb[rb][nt][0] = movmatrix_trans(pack_half2(sc[2 * rb][0], sc[2 * rb][1]));
+            pb[rb][nt][1] = movmatrix_trans(pack_half2(sc[2 * rb + 1][0], sc[2 * rb + 1][1]));
+          }
         }
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -449,79 +467,83 @@ __global__ void __maxnreg__(96) decode_mma_kernel(const DecodeArgs a) {
               acc[nt][mt][3] *= alpha[nt][1];
             }
         }
-        // ---------------- values: fp16 MMA, 8 m-tiles of 16 coordinates
-        // tokens (2q, 2q+1) and (2q+8, 2q+9) of the tile; unit r of 16 coordinates
-        const unsigned char *vt = st + St::vc + (wt + 2 * q) * (D * BV / 8);
+        // ---------------- values: fp16 MMA, k-step rb covers tokens 16 rb .. 16 rb + 15;
+        // tokens (2q, 2q+1) and (2q+8, 2q+9) of each k-step, unit r of 16 coordinates
         constexpr int VB = D * BV / 8;
-        if constexpr (BV == 3) {
-          const int gofs = 12 * (r >> 1);
-          const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
-          uint32_t ya[3], yb[3];
 #pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt + gofs)[k];
-            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k];
-            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k];
-            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k];
-            ya[k] = prmt(A0, B0, gs);
-            yb[k] = prmt(A1, B1, gs);
-          }
-          const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+        for (int rb = 0; rb < 2; ++rb) {
+          const unsigned char *vt = st + St::vc + (wt + 16 * rb + 2 * q) * VB;
+          if constexpr (BV == 3) {
+            const int gofs = 12 * (r >> 1);
+            const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
+            uint32_t ya[3], yb[3];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
-            const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              uint32_t a0, a1, a2, a3;
-              v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
-              v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_f16(acc[nt][2 * k + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            for (int k = 0; k < 3; ++k) {
+              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt + gofs)[k];
+              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k];
+              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k];
+              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k];
+              ya[k] = prmt(A0, B0, gs);
+              yb[k] = prmt(A1, B1, gs);
             }
-          }
-        } else if constexpr (BV == 2) {
-          const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
-          const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
-          const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
-          const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
+            const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
 #pragma unroll
-          for (int yh = 0; yh < 2; ++yh) {
-            const uint32_t gs = yh ? 0x7362u : 0x5140u;
-            const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
-#pragma unroll
-            for (int par = 0; par < 2; ++par) {
-              const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+              const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
                 uint32_t a0, a1, a2, a3;
-                v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
-                v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+                v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
+                v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                  mma_f16(acc[nt][4 * yh + 2 * par + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                  mma_f16(acc[nt][2 * k + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
               }
             }
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
-            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
-            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
-            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+          } else if constexpr (BV == 2) {
+            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
+            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
+            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
+            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
 #pragma unroll
             for (int yh = 0; yh < 2; ++yh) {
               const uint32_t gs = yh ? 0x7362u : 0x5140u;
               const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
 #pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                uint32_t a0, a1, a2, a3;
-                v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
-                v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+              for (int par = 0; par < 2; ++par) {
+                const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                  mma_f16(acc[nt][4 * u + 2 * yh + hh], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                for (int hh = 0; hh < 2; ++hh) {
+                  uint32_t a0, a1, a2, a3;
+                  v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
+                  v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(acc[nt][4 * yh + 2 * par + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
+              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
+              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
+              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+#pragma unroll
+              for (int yh = 0; yh < 2; ++yh) {
+                const uint32_t gs = yh ? 0x7362u : 0x5140u;
+                const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  uint32_t a0, a1, a2, a3;
+                  v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
+                  v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(acc[nt][4 * u + 2 * yh + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                }
               }
             }
           }
