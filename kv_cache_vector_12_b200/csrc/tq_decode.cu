@@ -132,6 +132,14 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// 2^x with the hardware approximation (relative error ~2^-22; flushes
+// subnormal results to zero, which only affects weights below 2^-126).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&h);
@@ -399,15 +407,15 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
         const __half *kn = reinterpret_cast<const __half *>(st + St::kn) + wt;
         const __half *vn = reinterpret_cast<const __half *>(st + St::vn) + wt;
         float nk[4], nv[4], gm[4];
-        bool ok[4];
+        const bool partial = tok0 + kWarpTokens > t1;  // only the last tile of a split is ragged
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int tt = 16 * (u >> 1) + r + 8 * (u & 1);
           nk[u] = __half2float(kn[tt]);
           nv[u] = __half2float(vn[tt]);
-          ok[u] = tok0 + tt < t1;
           gm[u] = 0.f;
           if constexpr (QJL) gm[u] = __half2float(reinterpret_cast<const __half *>(st + St::jg)[wt + tt]);
+          if (partial && tok0 + tt >= t1) nk[u] = nv[u] = gm[u] = __int_as_float(0x7fc00000);  // NaN marks "masked"
         }
         uint32_t pb[2][NT][2];
         bool rescale = false;
@@ -427,8 +435,15 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
                 const float dj = fmaf(256.f, (float)cjh[rb][nt][e], (float)cjl[rb][nt][e]);
                 v = fmaf(gm[u] * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
               }
-              sc[u][hd] = ok[u] ? v * nk[u] : -INFINITY;
+              sc[u][hd] = v * nk[u];
             }
+          if (partial) {  // masked tokens carry NaN norms: their scores become -inf, their weights 0
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int hd = 0; hd < 2; ++hd)
+                if (isnan(nv[u])) sc[u][hd] = -INFINITY;
+          }
 #pragma unroll
           for (int hd = 0; hd < 2; ++hd) {
             float mx = fmaxf(fmaxf(sc[0][hd], sc[1][hd]), fmaxf(sc[2][hd], sc[3][hd]));
@@ -436,17 +451,23 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             const float mn = fmaxf(m_run[nt][hd], mx);
-            const bool none = mn == -INFINITY;
-            const float al = none ? 1.f : exp2f(m_run[nt][hd] - mn);
+            // a finite reference keeps exp2(-inf - ref) = 0 when nothing is unmasked yet
+            const float ref = fmaxf(mn, -3.0e38f);
+            const float al = fast_exp2(m_run[nt][hd] - ref);
             alpha[nt][hd] = al;
             rescale |= al != 1.f;
             m_run[nt][hd] = mn;
             float lsum = 0.f;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const float pv = none ? 0.f : exp2f(sc[u][hd] - mn);
+              const float pv = fast_exp2(sc[u][hd] - ref);
               lsum += pv;
-              sc[u][hd] = ok[u] ? pv * nv[u] : 0.f;
+              sc[u][hd] = pv * nv[u];
+            }
+            if (partial) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (isnan(nv[u])) sc[u][hd] = 0.f;
             }
             l_run[nt][hd] = fmaf(l_run[nt][hd], al, lsum);
           }
