@@ -11,7 +11,7 @@
 //   MMA warp        one thread issues 8 tcgen05.mma (kind::f16, bf16 inputs,
 //                   fp32 accumulation in tensor memory) per tile and commits
 //                   to mbarriers.
-//   3 epilogue      warpgroups, one TMEM accumulator each; every thread owns
+//   4 epilogue      warpgroups, one TMEM accumulator each; every thread owns
 //   warpgroups      one row (vector): ||x|| from the shared-memory tile,
 //                   z from TMEM (tcgen05.ld 32x32b), codes against the
 //                   thresholds scaled by ||x||, bit-packing into the cache
@@ -35,11 +35,11 @@ namespace {
 constexpr int D = kHeadDim;
 constexpr int kTileRows = 128;
 constexpr int kRingStages = 4;
-constexpr int kEpiGroups = 3;
+constexpr int kEpiGroups = 4;
 constexpr int kQThreads = 32 * (2 + 4 * kEpiGroups);
 constexpr int kTileBytes = kTileRows * D * 2;     // 32 KB: two 128x64 bf16 boxes
 constexpr int kBoxBytes = kTileBytes / 2;
-constexpr unsigned kTmemCols = 512;               // 3 accumulators of 128 columns
+constexpr unsigned kTmemCols = 512;               // 4 accumulators of 128 columns
 constexpr unsigned kSpinLimit = 1u << 22;
 
 // ------------------------------------------------------------------ PTX
