@@ -684,7 +684,10 @@ __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const voi
   __shared__ int s_int[D];
   __shared__ float red[4];
   __shared__ int redi[4];
-  // let the attention kernel start streaming the cache while q is rotated
+  // launched as a programmatic dependent: q (and the cache the attention
+  // kernel streams) are final once the previous kernel has completed; only
+  // then may the attention kernel start streaming the cache while q is rotated
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int row = blockIdx.x, tid = threadIdx.x;
   s_q[tid] = q_dtype == TQ_F32 ? static_cast<const float *>(q)[(long)row * D + tid]
@@ -858,13 +861,18 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   float *qscale = reinterpret_cast<float *>(workspace + ws.qscale);
   float *partials = reinterpret_cast<float *>(workspace + ws.partials);
 
-  rotate_q_kernel<<<rows, 128, 0, st>>>(p, q, q_dtype, scale, q8, qscale);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return (int)e;
-
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
+
+  cudaLaunchConfig_t rcfg = {};
+  rcfg.gridDim = dim3(rows);
+  rcfg.blockDim = dim3(128);
+  rcfg.stream = st;
+  rcfg.attrs = pdl;
+  rcfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&rcfg, rotate_q_kernel, p, q, q_dtype, scale, q8, qscale);
+  if (e != cudaSuccess) return (int)e;
 
   const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1);
   DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q8, qscale, partials};

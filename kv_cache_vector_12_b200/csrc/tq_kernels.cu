@@ -92,6 +92,10 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
                                                            const int32_t *__restrict__ pos) {
   __shared__ float s_x[D], s_r[D];
   __shared__ float red[4];
+  // launched as a programmatic dependent: nothing is read before the
+  // previous kernel in the stream has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool is_v = blockIdx.y == 1;
   const int bits = is_v ? p.bits_v : p.bits_k;
@@ -152,17 +156,24 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream) {
   const long rows = (long)n_tok * c.n_kv_heads;
   cudaStream_t st = (cudaStream_t)stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  const uint16_t *kk = (const uint16_t *)k, *vv = (const uint16_t *)v;
   if (rows <= kRowKernelMaxRows) {
-    quantize_row_kernel<<<dim3((unsigned)rows, 2), 128, 0, st>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
-                                                               seq_idx, pos);
-    return (int)cudaGetLastError();
+    cfg.gridDim = dim3((unsigned)rows, 2);
+    return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel, p, c, kk, vv, seq_idx, pos);
   }
   const bool k_on_tc = !p.qjl;
   const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, stream);
   if (e != 0 || k_on_tc) return e;
-  quantize_row_kernel<<<dim3((unsigned)rows, 1), 128, 0, st>>>(p, c, (const uint16_t *)k, (const uint16_t *)v,
-                                                             seq_idx, pos);
-  return (int)cudaGetLastError();
+  cfg.gridDim = dim3((unsigned)rows, 1);
+  return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel, p, c, kk, vv, seq_idx, pos);
 }
 
 }  // namespace tq

@@ -222,14 +222,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_slot;
+  if (warp == 0 && lane == 0) {  // Pi belongs to the context: no earlier kernel writes it
+    const uint32_t pb = smem_addr(&pi_bar);
+    bar_expect_tx(pb, kTileBytes);
+    tma_load_2d(smem_addr(pi_tile), &map_pi, 0, 0, pb);
+    tma_load_2d(smem_addr(pi_tile + kBoxBytes), &map_pi, 64, 0, pb);
+  }
+  // launched as a programmatic dependent: inputs and the cache are touched
+  // only once the previous kernel in the stream has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------ producer (TMA)
     if (lane == 0) {
       const uint32_t pb = smem_addr(&pi_bar);
-      bar_expect_tx(pb, kTileBytes);
-      tma_load_2d(smem_addr(pi_tile), &map_pi, 0, 0, pb);
-      tma_load_2d(smem_addr(pi_tile + kBoxBytes), &map_pi, 64, 0, pb);
       int i = 0, issued = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
         const int slot = i % kRingStages;
@@ -454,8 +461,17 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
   args.tiles_v = tiles;
   const int total = args.tiles_k + args.tiles_v;
   const int grid = total < n_sm ? total : n_sm;
-  fn<<<grid, kQThreads, kQuantTcSmem, (cudaStream_t)stream>>>(mk, mv, mp, args);
-  return (int)cudaGetLastError();
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = kQuantTcSmem;
+  cfg.stream = (cudaStream_t)stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return (int)cudaLaunchKernelEx(&cfg, fn, mk, mv, mp, args);
 }
 
 }  // namespace tq
