@@ -14,8 +14,9 @@ step-to-step working set (R x 26 MB) exceeds the 126 MB L2.
 ``e2e``    the same metric when every step goes through the C ABI eagerly
            with pinned host buffers: H2D of the token's K/V and of q, the two
            calls, D2H of the output.
-``roofline`` the decode call alone, timed with events around each call inside
-           the timed region; algorithmic bytes = packed bytes per call.
+``roofline`` the decode calls of the timed steps alone (same replicas and
+           lengths) as one CUDA graph, events around its replay; algorithmic
+           bytes = packed bytes per call.
 ``quantize_*`` prefill quantize of 32768 tokens (input 128 MB > L2): tokens/s,
            GB/s (bf16 read + packed write) and roofline fraction.
 ``cpu_baseline`` the CPU oracle on a bounded sample of the same decode step.
@@ -295,7 +296,7 @@ def main(argv=None) -> int:
             step(i)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
-    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_warm, g_timed, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_warm):
         for i in range(args.warmup):
             step(i)
@@ -318,17 +319,21 @@ def main(argv=None) -> int:
     ev1.record()
     torch.cuda.synchronize()
     ms_total = ev0.elapsed_time(ev1)
-    # decode call alone, events around each call (same stream), same steps
-    de = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
-    for j, i in enumerate(range(args.warmup, n_steps_total)):
-        c = caches[i % R]
-        tq.quantize(ctx, c, k_new[i * B:(i + 1) * B], v_new[i * B:(i + 1) * B], seq_ids, pos_steps[i])
-        de[2 * j].record()
-        tq.decode_attention(ctx, c, q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
-        de[2 * j + 1].record()
+    # decode calls alone: the timed steps' decode calls (same replicas, same
+    # lengths, their tokens already appended) as one CUDA graph, events around
+    # its replay on the launching stream
+    with torch.cuda.graph(g_dec):
+        for i in range(args.warmup, n_steps_total):
+            tq.decode_attention(ctx, caches[i % R], q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
+    g_dec.replay()
+    torch.cuda.synchronize()
+    ed0, ed1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ed0.record()
+    g_dec.replay()
+    ed1.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    dec_ms = [de[2 * j].elapsed_time(de[2 * j + 1]) for j in range(args.steps)]
+    dec_ms = [ed0.elapsed_time(ed1) / args.steps]
     ctx.check_device_errors()
 
     breakdown = None
@@ -361,7 +366,11 @@ def main(argv=None) -> int:
                                                             pos_steps[i_last])),
             "decode_call_us": timed(lambda: tq.decode_attention(ctx, c_last, q_all[i_last], lens_steps[i_last],
                                                                 max_len, out[i_last], lse[i_last], wsb)),
-            "note": "CUDA graph of 20 calls on one cache (warm L2), events around the replays",
+            "step_us": timed(lambda: (tq.quantize(ctx, c_last, k_new[i_last * B:(i_last + 1) * B],
+                                                  v_new[i_last * B:(i_last + 1) * B], seq_ids, pos_steps[i_last]),
+                                      tq.decode_attention(ctx, c_last, q_all[i_last], lens_steps[i_last], max_len,
+                                                          out[i_last], lse[i_last], wsb))),
+            "note": "CUDA graph of 20 calls (or steps) on one cache (warm L2), events around the replays",
         }
         torch.cuda.synchronize()
 
@@ -441,7 +450,7 @@ def main(argv=None) -> int:
     print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.barrier()
-        del g_warm, g_timed
+        del g_warm, g_timed, g_dec
         torch.distributed.destroy_process_group()
     return 0
 

@@ -159,7 +159,7 @@ DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split) {
   w.q8 = 0;
   w.qscale = up(rows * 4 * kHeadDim);
   w.partials = w.qscale + up(rows * 4 * sizeof(float));
-  w.total = w.partials + up(rows * (size_t)split.n_splits * (kHeadDim + 2) * sizeof(float));
+  w.total = w.partials + up(rows * (size_t)split.n_splits * kPartialFloats * sizeof(float));
   return w;
 }
 

@@ -64,12 +64,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One suspending test of phase `parity`: a thread whose phase is not complete
+// sleeps until it completes or kSuspendNs pass, instead of spinning (a spinning
+// producer would take issue slots from the consumer warps of its SM).
+constexpr uint32_t kSuspendNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -85,8 +89,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (;;) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (global_ns() - t0 > kWaitNs) return false;
   }
 }
@@ -618,8 +621,8 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
       l = fmaf(f, sm_l[w][g], l);
       o = fmaf(f, so[(w * 8 * NT + g) * D + i], o);
     }
-    float *dst = a.partials + (((long)s * a.n_q_heads + h * G + g) * a.n_splits + split) * (D + 2);
-    dst[2 + i] = o;
+    float *dst = a.partials + (((long)s * a.n_q_heads + h * G + g) * a.n_splits + split) * kPartialFloats;
+    dst[4 + i] = o;
     if (i == 0) {
       dst[0] = mx;
       dst[1] = l;
@@ -642,12 +645,15 @@ __device__ __forceinline__ float block_max128(float v, float *red) {
   return r;
 }
 
-// Dot product of a bf16 row (128 entries, 16-byte aligned) with a vector in
-// shared memory: 16 independent 16-byte loads, four partial sums.
-__device__ __forceinline__ float dot_bf16_row(const uint16_t *row, const float *x) {
-  uint4 w[16];
+// A bf16 row of 128 entries (16-byte aligned) as 16 independent 16-byte loads.
+__device__ __forceinline__ void load_bf16_row(const uint16_t *row, uint4 (&w)[16]) {
 #pragma unroll
   for (int c = 0; c < 16; ++c) w[c] = reinterpret_cast<const uint4 *>(row)[c];
+}
+
+// Dot product of a loaded bf16 row with a vector in shared memory, four
+// partial sums.
+__device__ __forceinline__ float dot_bf16_row(const uint4 (&w)[16], const float *x) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
@@ -684,16 +690,18 @@ __global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const voi
   __shared__ int s_int[D];
   __shared__ float red[4];
   __shared__ int redi[4];
+  const int row = blockIdx.x, tid = threadIdx.x;
+  uint4 pw[16];
+  load_bf16_row(p.pi + tid * D, pw);  // parameters: independent of the previous kernel
   // launched as a programmatic dependent: q (and the cache the attention
   // kernel streams) are final once the previous kernel has completed; only
   // then may the attention kernel start streaming the cache while q is rotated
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int row = blockIdx.x, tid = threadIdx.x;
   s_q[tid] = q_dtype == TQ_F32 ? static_cast<const float *>(q)[(long)row * D + tid]
                                : __uint_as_float((uint32_t) static_cast<const uint16_t *>(q)[(long)row * D + tid] << 16);
   __syncthreads();
-  const float qh = dot_bf16_row(p.pi + tid * D, s_q);  // (Pi q)_tid
+  const float qh = dot_bf16_row(pw, s_q);  // (Pi q)_tid
   s_qh[tid] = qh;
   const float mx = block_max128(fabsf(qh), red);
   const float mu = mx > 0.f ? 32767.f / mx : 1.f;
@@ -744,46 +752,69 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
                                                     const float *partials, float *out, float *lse) {
   __shared__ float s_ot[D];
   __shared__ float s_w[kMergeMaxSplits];
+  __shared__ __align__(16) float s_acc[4][D];
   __shared__ float red[4];
+  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this thread's row of Pi^T does not depend on the attention kernel: load it
+  // before waiting for that kernel to complete
+  uint4 pw[16];
+  load_bf16_row(p.pivt + tid * D, pw);
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int row = blockIdx.x, tid = threadIdx.x;
   const int s = row / n_q_heads;
   int len = seq_lens[s];
   len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
   const int used = min((len + chunk - 1) / chunk, kMergeMaxSplits);
-  const float *src = partials + (long)row * n_splits * (D + 2);
+  const float *src = partials + (long)row * n_splits * kPartialFloats;
   // split maxima (log2 units) in parallel, then the weights 2^(m_s - M)
   float mloc = -INFINITY;
   for (int sp = tid; sp < used; sp += 128) {
-    const float m = src[sp * (D + 2)];
+    const float m = src[sp * kPartialFloats];
     s_w[sp] = m;
     mloc = fmaxf(mloc, m);
   }
   const float mm = block_max128(mloc, red);
-  for (int sp = tid; sp < used; sp += 128) s_w[sp] = s_w[sp] == -INFINITY ? 0.f : exp2f(s_w[sp] - mm);
+  float lpart = 0.f;
+  for (int sp = tid; sp < used; sp += 128) {
+    const float w = s_w[sp] == -INFINITY ? 0.f : exp2f(s_w[sp] - mm);
+    s_w[sp] = w;
+    lpart = fmaf(w, src[sp * kPartialFloats + 1], lpart);
+  }
   __syncthreads();
-  float ll = 0.f, oo = 0.f;
-  int sp = 0;
-  for (; sp + 4 <= used; sp += 4) {
-    float l4[4], o4[4];
+  // warp w takes splits w, w + 4, ...; lane j the outputs 4 j .. 4 j + 3.
+  // Four splits per round keep four independent 16-byte loads in flight.
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int sp = warp;
+  for (; sp + 12 < used; sp += 16) {
+    float4 o4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o4[e] = reinterpret_cast<const float4 *>(src + (sp + 4 * e) * kPartialFloats + 4)[lane];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      l4[e] = src[(sp + e) * (D + 2) + 1];
-      o4[e] = src[(sp + e) * (D + 2) + 2 + tid];
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      ll = fmaf(s_w[sp + e], l4[e], ll);
-      oo = fmaf(s_w[sp + e], o4[e], oo);
+      const float w = s_w[sp + 4 * e];
+      acc.x = fmaf(w, o4[e].x, acc.x);
+      acc.y = fmaf(w, o4[e].y, acc.y);
+      acc.z = fmaf(w, o4[e].z, acc.z);
+      acc.w = fmaf(w, o4[e].w, acc.w);
     }
   }
-  for (; sp < used; ++sp) {
-    ll = fmaf(s_w[sp], src[sp * (D + 2) + 1], ll);
-    oo = fmaf(s_w[sp], src[sp * (D + 2) + 2 + tid], oo);
+  for (; sp < used; sp += 4) {
+    const float4 o4 = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
+    const float w = s_w[sp];
+    acc.x = fmaf(w, o4.x, acc.x);
+    acc.y = fmaf(w, o4.y, acc.y);
+    acc.z = fmaf(w, o4.z, acc.z);
+    acc.w = fmaf(w, o4.w, acc.w);
   }
+  reinterpret_cast<float4 *>(s_acc[warp])[lane] = acc;
+  for (int o = 16; o; o >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, o);
+  if (lane == 0) red[warp] = lpart;
+  __syncthreads();
+  const float ll = (red[0] + red[1]) + (red[2] + red[3]);
+  const float oo = (s_acc[0][tid] + s_acc[1][tid]) + (s_acc[2][tid] + s_acc[3][tid]);
   s_ot[tid] = ll > 0.f ? oo / ll : 0.f;
   __syncthreads();
-  out[(long)row * D + tid] = dot_bf16_row(p.pivt + tid * D, s_ot);
+  // o_i = sum_k Pi^T[i][k] o~_k with Pi^T's columns in the V fragment order
+  out[(long)row * D + tid] = dot_bf16_row(pw, s_ot);
   if (lse && tid == 0) lse[row] = ll > 0.f ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
 }
 

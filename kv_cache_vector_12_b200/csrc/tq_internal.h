@@ -67,7 +67,9 @@ DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_p
 int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group);
 
 // Workspace layout of decode attention (byte offsets, 256-aligned):
-// q8 [rows][4][d] bytes, qscale [rows][4] floats, partials [rows][splits][d+2].
+// q8 [rows][4][d] bytes, qscale [rows][4] floats, partials [rows][splits][d+4]
+// (a partial is m, l, two unused floats, then the d outputs: 16-byte aligned).
+constexpr int kPartialFloats = kHeadDim + 4;
 struct DecodeWorkspace {
   size_t q8, qscale, partials, total;
 };

@@ -44,10 +44,7 @@ __device__ __forceinline__ int code_bit_pos(int bits, int i, int k) {
 // r = z/||x|| - c[code], ||r||, (S r)_m from row m of S, one sign ballot per
 // warp.  grid = (rows, 2): y = 0 for K, 1 for V.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float row_dot_bf16(const uint16_t *row, const float *x) {
-  uint4 w[16];
-#pragma unroll
-  for (int c = 0; c < 16; ++c) w[c] = reinterpret_cast<const uint4 *>(row)[c];
+__device__ __forceinline__ float row_dot_bf16(const uint4 (&w)[16], const float *x) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
@@ -92,11 +89,16 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
                                                            const int32_t *__restrict__ pos) {
   __shared__ float s_x[D], s_r[D];
   __shared__ float red[4];
-  // launched as a programmatic dependent: nothing is read before the
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // row tid of Pi is a parameter, written long before: load it while the
+  // previous kernel finishes
+  uint4 pw[16];
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) pw[ch] = reinterpret_cast<const uint4 *>(p.pi + tid * D)[ch];
+  // launched as a programmatic dependent: no input is read before the
   // previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool is_v = blockIdx.y == 1;
   const int bits = is_v ? p.bits_v : p.bits_k;
   const bool qjl = !is_v && p.qjl;
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * D + tid]);
   s_x[tid] = x;
   const float n = sqrtf(block_sum128(x * x, red));  // also orders s_x
-  const float z = row_dot_bf16(p.pi + tid * D, s_x);
+  const float z = row_dot_bf16(pw, s_x);
   const float *thr = p.cb + (is_v ? 3 : 1) * kMaxLevels;
   const int half = 1 << (bits - 1);
   const float a = fabsf(z);

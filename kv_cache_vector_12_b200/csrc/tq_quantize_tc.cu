@@ -40,7 +40,8 @@ constexpr int kQThreads = 32 * (2 + 4 * kEpiGroups);
 constexpr int kTileBytes = kTileRows * D * 2;     // 32 KB: two 128x64 bf16 boxes
 constexpr int kBoxBytes = kTileBytes / 2;
 constexpr unsigned kTmemCols = 512;               // 4 accumulators of 128 columns
-constexpr unsigned kSpinLimit = 1u << 22;
+constexpr uint32_t kSuspendNs = 1000000;                 // longest sleep of one barrier test: 1 ms
+constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded barrier waits: 2 s
 
 // ------------------------------------------------------------------ PTX
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -55,18 +56,29 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t b, uint32_t bytes) {
 __device__ __forceinline__ void bar_arrive(uint32_t b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
 }
+// A suspending test: the thread sleeps until the phase completes or
+// kSuspendNs pass, so waiting warps leave the issue slots to working ones.
 __device__ __forceinline__ bool bar_try(uint32_t b, uint32_t parity) {
   uint32_t ok;
-  asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+  asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
                : "=r"(ok)
-               : "r"(b), "r"(parity)
+               : "r"(b), "r"(parity), "r"(kSuspendNs)
                : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity`; false once kWaitNs have passed.
 __device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity) {
-  for (unsigned i = 0; i < kSpinLimit; ++i)
+  if (bar_try(b, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
     if (bar_try(b, parity)) return true;
-  return false;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -98,6 +110,20 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -125,41 +151,62 @@ struct QuantTcArgs {
   int tiles_v;
 };
 
+// All ones when a > b, else 0.
+__device__ __forceinline__ int gt_mask(float a, float b) { return -(int)(a > b); }
+
 // Code of one rotated coordinate: #{j : T_j < z} with T_j = t_j ||x||,
 // evaluated as sign + count of the positive thresholds below |z| (the
-// codebook is symmetric, t_{half-1} = 0).  z = 0 (also a zero vector) gives
-// half - 1.
+// codebook is symmetric, t_{half-1} = 0): with m = #{j : tp_j < |z|} and
+// sn = -1 for z > 0 (else 0), half - 1 - (m ^ sn) is half + m for z > 0 and
+// half - 1 - m otherwise.  z = 0 (also a zero vector) gives half - 1.
 template <int B>
 __device__ __forceinline__ uint32_t code_of(float z, const float (&tp)[(1 << (B - 1)) - 1]) {
   constexpr int half = 1 << (B - 1);
   const float a = fabsf(z);
-  int m = 0;
+  int neg_m = 0;
 #pragma unroll
-  for (int j = 0; j < half - 1; ++j) m += a > tp[j] ? 1 : 0;
-  return (uint32_t)(z > 0.f ? half + m : half - 1 - m);
+  for (int j = 0; j < half - 1; ++j) neg_m += gt_mask(a, tp[j]);
+  return (uint32_t)((half - 1) - ((-neg_m) ^ gt_mask(z, 0.f)));
 }
 
-// Pack the 32 codes of coordinate group g into words w[g*B .. g*B+B) of the
-// cache layout (LSB-first for 2 and 4 bits; nibble + spare-column layout for 3).
+// Codes of coordinates 16 c .. 16 c + 15 packed into the words of the cache
+// layout as they are computed: LSB-first for 2 and 4 bits; for 3 bits, in
+// each 32-coordinate group nibble l % 8 of word l / 8 (l < 24), and the eight
+// spare-column codes gathered into the nibbles of one word whose bit k of
+// every nibble then moves to bit 3 of word k.
 template <int B>
-__device__ __forceinline__ void pack_group(const uint32_t (&cd)[32], uint32_t *w) {
+__device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const float (&tp)[(1 << (B - 1)) - 1],
+                                           uint32_t (&w)[4 * B]) {
   if constexpr (B == 3) {
+    const int g = c >> 1;
+    if ((c & 1) == 0) {
+      uint32_t x0 = 0u, x1 = 0u;
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      uint32_t x = 0;
+      for (int j = 0; j < 8; ++j) {
+        x0 |= code_of<3>(z[j], tp) << (4 * j);
+        x1 |= code_of<3>(z[8 + j], tp) << (4 * j);
+      }
+      w[3 * g] = x0;
+      w[3 * g + 1] = x1;
+    } else {
+      uint32_t x2 = 0u, sp = 0u;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x |= cd[8 * k + j] << (4 * j);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x |= ((cd[24 + j] >> k) & 1u) << (4 * j + 3);
-      w[k] = x;
+      for (int j = 0; j < 8; ++j) {
+        x2 |= code_of<3>(z[j], tp) << (4 * j);
+        sp |= code_of<3>(z[8 + j], tp) << (4 * j);
+      }
+      w[3 * g] |= (sp << 3) & 0x88888888u;
+      w[3 * g + 1] |= (sp << 2) & 0x88888888u;
+      w[3 * g + 2] = x2 | ((sp << 1) & 0x88888888u);
     }
   } else {
+    constexpr int per = 32 / B;  // codes per word
 #pragma unroll
-    for (int k = 0; k < B; ++k) {
-      uint32_t x = 0;
+    for (int k = 0; k < 16 / per; ++k) {
+      uint32_t x = 0u;
 #pragma unroll
-      for (int j = 0; j < 32 / B; ++j) x |= cd[(32 / B) * k + j] << (B * j);
-      w[k] = x;
+      for (int j = 0; j < per; ++j) x |= code_of<B>(z[per * k + j], tp) << (B * j);
+      w[(16 / per) * c + k] = x;
     }
   }
 }
@@ -172,13 +219,10 @@ __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], flo
 #pragma unroll
   for (int j = 0; j < half - 1; ++j) tp[j] = thr[half + j] * n;  // positive thresholds, scaled
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float z[32];
-    tmem_ld32(tmem_row + 32 * g, z);
-    uint32_t cd[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) cd[i] = code_of<B>(z[i], tp);
-    pack_group<B>(cd, words + g * B);
+  for (int c = 0; c < 8; ++c) {
+    float z[16];
+    tmem_ld16(tmem_row + 16 * c, z);
+    code_chunk<B>(c, z, tp, words);
   }
 }
 
