@@ -5,9 +5,13 @@
 // optional 1-bit QJL residual signs).  Per (sequence, KV head, split of the
 // sequence) one CTA streams the split's packed codes and norms into a shared
 // memory ring with TMA bulk copies (one producer warp, mbarrier pipeline with
-// bounded waits) while four consumer warps each take 16 tokens of every
-// 64-token stage:
+// bounded waits) while four consumer warps each take 32 tokens of every
+// 128-token stage.  Before the first stage arrives the consumers rotate the
+// KV head's queries themselves:
 //
+//   q_hat   Pi q for the G query heads on the tensor cores (mma m16n8k16
+//           bf16, fp32 q as an exact hi + lo pair), then 16-bit fixed point;
+//           with QJL also q_tilde = S q_hat (fp32).
 //   scores  S[tok][head] = q_hat . c_K[code]   int8 tensor cores (mma m16n8k32):
 //           K centroids are exact 16-bit fixed-point integers (c * 2^17), split
 //           into hi/lo bytes by two byte-permute lookups per 4 codes; q_hat is
@@ -21,8 +25,10 @@
 //
 // The coordinate order inside the MMA fragments is a fixed permutation of the
 // head dimension chosen so that every code is expanded where it is loaded; the
-// host computes the permutations (tq_api.cu) and rotate_q writes q_hat in the
-// K order, merge applies Pi^T with rows in the V order.
+// host computes the permutations (tq_fragments.cpp) and stores Pi's rows in
+// the K order (so q_hat comes out of its MMA already in that order) and S in
+// the QJL and K orders; merge applies Pi^T with rows in the V order.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -129,6 +135,30 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// x0, x1 as bf16 pairs hi + lo (x0 in the low halves): hi = bf16(x), lo =
+// bf16(x - hi), so x - hi - lo is below 2^-16 |x|.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __low2float(h), x1 - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Barrier of the four consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(32 * kConsumerWarps) : "memory");
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi / 2), the QJL constant's numerator
+
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -219,24 +249,49 @@ struct DecodeArgs {
   tq_cache c;
   int n_q_heads, max_seq_len, chunk, n_splits;
   const int32_t *seq_lens;
-  const uint8_t *q8;      // [rows][4][128] bytes: q_hat hi, lo; q_tilde hi, lo (K / QJL fragment order)
-  const float *qscale;    // [rows][4]: score factor, QJL factor, sum of q_tilde ints, unused
-  float *partials;        // [rows][n_splits][2 + D]
+  const void *q;          // [n_seqs][n_q_heads][d], fp32 or bf16 (q_dtype)
+  int q_dtype;
+  float scale;
+  float *partials;        // [rows][n_splits][d + 4]
 };
 
 template <int BK, int BV, bool QJL, int NT>
 __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
   static_assert(kStageTokens % 64 == 0 && kWarpTokens == 32, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
+  constexpr int kRows = 8 * NT;  // query-head rows of the score MMAs
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ int abort_flag;
-  __shared__ float sm_m[kConsumerWarps][8 * NT], sm_l[kConsumerWarps][8 * NT];
+  __shared__ float sm_m[kConsumerWarps][kRows], sm_l[kConsumerWarps][kRows];
+  __shared__ __align__(16) uint8_t s_q8[kRows][QJL ? 4 : 2][D];  // q_hat hi, lo; q_tilde hi, lo (fragment orders)
+  __shared__ __align__(16) float s_qf[QJL ? kRows : 1][D];       // q_hat, fp32, K order (QJL input)
+  __shared__ float s_qs[kRows][4];                                // score factor, QJL factor, sum of q_tilde ints
+  __shared__ float s_red[kConsumerWarps][kRows];
 
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, q = lane & 3;
   const int G = a.n_q_heads / a.c.n_kv_heads;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // B fragments of Pi (rows in the K fragment order) for this consumer warp's
+  // 32 output positions: parameters, loaded before waiting for the previous
+  // kernel in the stream
+  uint32_t bfr[4][8][2];
+  if (warp < kConsumerWarps) {
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[((warp * 4 + nt) * 4 + j) * 32 + lane];
+        bfr[nt][2 * j][0] = v.x;
+        bfr[nt][2 * j][1] = v.y;
+        bfr[nt][2 * j + 1][0] = v.z;
+        bfr[nt][2 * j + 1][1] = v.w;
+      }
+  }
+  // launched as a programmatic dependent: the cache, q and seq_lens are final
+  // once the previous kernel in the stream has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = a.seq_lens[s];
   if (len < 0 || len > a.max_seq_len) {
     if (tid == 0 && split == 0 && h == 0) atomicOr(a.p.err, kErrSeqLen);
@@ -297,35 +352,160 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
     }
   } else {
     // ---------------- consumers
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // rotate_q's q8 / qscale are complete
-    const int r = lane >> 2, q = lane & 3;
+    // q_hat = Pi q for this KV head's query heads on the tensor cores: mma
+    // m16n8k16 bf16 with the heads as rows and the K fragment positions as
+    // columns (Pi's rows are stored in that order), fp32 q split into a bf16
+    // hi + lo pair so every product is exact and the sums are fp32.  Warp w
+    // computes positions 32 w .. 32 w + 31.
+    {
+      const long qrow0 = (long)s * a.n_q_heads + (long)h * G;
+      const bool f32 = a.q_dtype == TQ_F32;
+      float c[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t ahi[4], alo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // a0: row r; a1: row r + 8; a2, a3: the same rows, columns + 8
+          const int row = r + 8 * (e & 1), col = 16 * ks + 8 * (e >> 1) + 2 * q;
+          float x0 = 0.f, x1 = 0.f;
+          if (row < G) {
+            if (f32) {
+              const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(a.q) + (qrow0 + row) * D + col);
+              x0 = v.x;
+              x1 = v.y;
+            } else {
+              const uint32_t v = *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.q) + (qrow0 + row) * D + col);
+              x0 = __uint_as_float(v << 16);
+              x1 = __uint_as_float(v & 0xffff0000u);
+            }
+          }
+          split_bf16x2(x0, x1, ahi[e], alo[e]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          mma_bf16(c[nt], ahi[0], ahi[1], ahi[2], ahi[3], bfr[nt][ks][0], bfr[nt][ks][1]);
+          if (f32) mma_bf16(c[nt], alo[0], alo[1], alo[2], alo[3], bfr[nt][ks][0], bfr[nt][ks][1]);
+        }
+      }
+      // per head: mu = 32767 / max |q_hat|, q_hat as 16-bit fixed point (hi, lo bytes)
+      float mx0 = 0.f, mx1 = 0.f;  // rows r, r + 8
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        mx0 = fmaxf(mx0, fmaxf(fabsf(c[nt][0]), fabsf(c[nt][1])));
+        mx1 = fmaxf(mx1, fmaxf(fabsf(c[nt][2]), fabsf(c[nt][3])));
+      }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (q == 0) {
+        s_red[warp][r] = mx0;
+        if constexpr (kRows > 8) s_red[warp][r + 8] = mx1;
+      }
+      consumer_sync();
+      float mu[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (kRows <= 8 && e == 1) break;
+        const int row = r + 8 * e;
+        const float m = fmaxf(fmaxf(s_red[0][row], s_red[1][row]), fmaxf(s_red[2][row], s_red[3][row]));
+        mu[e] = m > 0.f ? 32767.f / m : 1.f;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int kap = 32 * warp + 8 * nt + 2 * q;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (kRows <= 8 && e == 1) break;
+          const int row = r + 8 * e;
+          const int v0 = (int)rintf(c[nt][2 * e] * mu[e]), v1 = (int)rintf(c[nt][2 * e + 1] * mu[e]);
+          *reinterpret_cast<uint16_t *>(&s_q8[row][0][kap]) = (uint16_t)(((v0 >> 8) & 0xFF) | (((v1 >> 8) & 0xFF) << 8));
+          *reinterpret_cast<uint16_t *>(&s_q8[row][1][kap]) = (uint16_t)((v0 & 0xFF) | ((v1 & 0xFF) << 8));
+          if constexpr (QJL) *reinterpret_cast<float2 *>(&s_qf[row][kap]) = make_float2(c[nt][2 * e], c[nt][2 * e + 1]);
+        }
+      }
+      if (warp == 0 && q == 0) {
+        s_qs[r][0] = a.scale * kLog2e / (mu[0] * (float)(1 << kKFixedShift));
+        if constexpr (kRows > 8) s_qs[r + 8][0] = a.scale * kLog2e / (mu[1] * (float)(1 << kKFixedShift));
+      }
+      if constexpr (QJL) {
+        // q_tilde = S q_hat: position tid (QJL fragment order) of every head,
+        // from row tid of S permuted into the QJL (rows) and K (columns) orders
+        consumer_sync();
+        float qt[kRows];
+#pragma unroll
+        for (int g = 0; g < kRows; ++g) qt[g] = 0.f;
+        const float4 *srow = reinterpret_cast<const float4 *>(a.p.sjk + tid * D);
+#pragma unroll 4
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+          const float4 w4 = srow[c4];
+#pragma unroll
+          for (int g = 0; g < kRows; ++g) {
+            const float4 x = *reinterpret_cast<const float4 *>(&s_qf[g][4 * c4]);
+            qt[g] = fmaf(w4.x, x.x, fmaf(w4.y, x.y, fmaf(w4.z, x.z, fmaf(w4.w, x.w, qt[g]))));
+          }
+        }
+        // nu = 32767 / max |q_tilde| per head, then the ints and their sum
+#pragma unroll
+        for (int g = 0; g < kRows; ++g) {
+          float m = fabsf(qt[g]);
+#pragma unroll
+          for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) s_red[warp][g] = m;
+        }
+        consumer_sync();
+        float nu[kRows];
+#pragma unroll
+        for (int g = 0; g < kRows; ++g) {
+          const float m = fmaxf(fmaxf(s_red[0][g], s_red[1][g]), fmaxf(s_red[2][g], s_red[3][g]));
+          nu[g] = m > 0.f ? 32767.f / m : 1.f;
+          if (tid == g) s_qs[g][1] = a.scale * kLog2e * kSqrtHalfPi / ((float)D * nu[g]);
+        }
+        consumer_sync();  // s_red is reused for the sums
+#pragma unroll
+        for (int g = 0; g < kRows; ++g) {
+          const int vi = (int)rintf(qt[g] * nu[g]);
+          s_q8[g][2][tid] = (uint8_t)(vi >> 8);
+          s_q8[g][3][tid] = (uint8_t)(vi & 0xFF);
+          int sum = vi;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          if (lane == 0) s_red[warp][g] = (float)sum;  // |sum| < 2^22: exact
+        }
+        consumer_sync();
+        if (tid < kRows) s_qs[tid][2] = (s_red[0][tid] + s_red[1][tid]) + (s_red[2][tid] + s_red[3][tid]);
+      }
+      consumer_sync();
+    }
     // q fragments (int8, K fragment order) of this thread's head r in every n-tile
     uint32_t qh[NT][4][2], ql[NT][4][2], jh[NT][QJL ? 4 : 1][2], jl[NT][QJL ? 4 : 1][2];
     float fq[NT][2], fj[NT][2], jsum[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int g = 8 * nt + r;
-      const bool live = g < G;
-      const uint8_t *qb = a.q8 + ((long)s * a.n_q_heads + h * G + (live ? g : 0)) * 4 * D;
+      const uint8_t *qb = &s_q8[8 * nt + r][0][0];
 #pragma unroll
       for (int st = 0; st < 4; ++st)
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
           const int off = 32 * st + 16 * sl + 4 * q;
-          qh[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + off) : 0u;
-          ql[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + D + off) : 0u;
+          qh[nt][st][sl] = *reinterpret_cast<const uint32_t *>(qb + off);
+          ql[nt][st][sl] = *reinterpret_cast<const uint32_t *>(qb + D + off);
           if constexpr (QJL) {
-            jh[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + 2 * D + off) : 0u;
-            jl[nt][st][sl] = live ? *reinterpret_cast<const uint32_t *>(qb + 3 * D + off) : 0u;
+            jh[nt][st][sl] = *reinterpret_cast<const uint32_t *>(qb + 2 * D + off);
+            jl[nt][st][sl] = *reinterpret_cast<const uint32_t *>(qb + 3 * D + off);
           }
         }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int gg = 8 * nt + 2 * q + e;
-        const float *f = a.qscale + ((long)s * a.n_q_heads + h * G + (gg < G ? gg : 0)) * 4;
-        fq[nt][e] = gg < G ? f[0] : 0.f;
-        fj[nt][e] = gg < G ? f[1] : 0.f;
-        jsum[nt][e] = gg < G ? f[2] : 0.f;
+        const int gg = 8 * nt + 2 * q + e;  // heads past G have zero q and zero factors
+        fq[nt][e] = gg < G ? s_qs[gg][0] : 0.f;
+        fj[nt][e] = gg < G && QJL ? s_qs[gg][1] : 0.f;
+        jsum[nt][e] = gg < G && QJL ? s_qs[gg][2] : 0.f;
       }
     }
     const Lut lk = a.p.lut_k, lv = a.p.lut_v;
@@ -579,7 +759,7 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
     }
 
     // ---------------- all consumers are past the ring: park the state in smem
-    asm volatile("bar.sync 1, %0;" ::"r"(32 * kConsumerWarps) : "memory");
+    consumer_sync();
     float *so = reinterpret_cast<float *>(smem);  // [warp][8 NT heads][D], V fragment order
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -605,6 +785,8 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
     }
   }
   __syncthreads();
+  // the merge kernel may start launching once every CTA is here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (*(volatile int *)&abort_flag) return;
 
   // ---------------- combine the consumer warps, write this split's partial
@@ -631,10 +813,8 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// rotate_q: q_hat = Pi q per (sequence, query head), as 16-bit fixed point in
-// the K fragment order (hi bytes, lo bytes); with QJL also q_tilde = S q_hat.
-// Also the per-head factors that turn the integer dot products into scores in
-// log2 units.  One CTA of 128 threads per row.
+// merge: per (sequence, query head) combine the splits (log-sum-exp in log2
+// units) and apply Pi^T.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float block_max128(float v, float *red) {
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -668,79 +848,6 @@ __device__ __forceinline__ float dot_bf16_row(const uint4 (&w)[16], const float 
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-// Same for an fp32 row.
-__device__ __forceinline__ float dot_f32_row(const float *row, const float *x) {
-  float4 w[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) w[c] = reinterpret_cast<const float4 *>(row)[c];
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    acc[0] = fmaf(w[c].x, x[4 * c], acc[0]);
-    acc[1] = fmaf(w[c].y, x[4 * c + 1], acc[1]);
-    acc[2] = fmaf(w[c].z, x[4 * c + 2], acc[2]);
-    acc[3] = fmaf(w[c].w, x[4 * c + 3], acc[3]);
-  }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
-__global__ void __launch_bounds__(128) rotate_q_kernel(DeviceParams p, const void *q, int q_dtype, float scale,
-                                                       uint8_t *q8, float *qscale) {
-  __shared__ float s_q[D], s_qh[D];
-  __shared__ int s_int[D];
-  __shared__ float red[4];
-  __shared__ int redi[4];
-  const int row = blockIdx.x, tid = threadIdx.x;
-  uint4 pw[16];
-  load_bf16_row(p.pi + tid * D, pw);  // parameters: independent of the previous kernel
-  // launched as a programmatic dependent: q (and the cache the attention
-  // kernel streams) are final once the previous kernel has completed; only
-  // then may the attention kernel start streaming the cache while q is rotated
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  s_q[tid] = q_dtype == TQ_F32 ? static_cast<const float *>(q)[(long)row * D + tid]
-                               : __uint_as_float((uint32_t) static_cast<const uint16_t *>(q)[(long)row * D + tid] << 16);
-  __syncthreads();
-  const float qh = dot_bf16_row(pw, s_q);  // (Pi q)_tid
-  s_qh[tid] = qh;
-  const float mx = block_max128(fabsf(qh), red);
-  const float mu = mx > 0.f ? 32767.f / mx : 1.f;
-  s_int[tid] = (int)rintf(qh * mu);
-  __syncthreads();
-  uint8_t *dst = q8 + (long)row * 4 * D;
-  {
-    const int v = s_int[p.kperm[tid]];
-    dst[tid] = (uint8_t)(v >> 8);
-    dst[D + tid] = (uint8_t)(v & 0xFF);
-  }
-  const float log2e = 1.4426950408889634f;
-  float fj = 0.f, jsum = 0.f;
-  if (p.qjl) {
-    const float qt = dot_f32_row(p.s + tid * D, s_qh);  // (S q_hat)_tid
-    const float mt = block_max128(fabsf(qt), red);
-    const float nu = mt > 0.f ? 32767.f / mt : 1.f;
-    const int vi = (int)rintf(qt * nu);
-    __syncthreads();
-    s_int[tid] = vi;
-    int sum = vi;
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if ((tid & 31) == 0) redi[tid >> 5] = sum;
-    __syncthreads();
-    jsum = (float)(redi[0] + redi[1] + redi[2] + redi[3]);
-    const int v = s_int[p.jperm[tid]];
-    dst[2 * D + tid] = (uint8_t)(v >> 8);
-    dst[3 * D + tid] = (uint8_t)(v & 0xFF);
-    fj = scale * log2e * sqrtf(0.5f * (float)M_PI) / ((float)D * nu);
-  }
-  if (tid == 0) {
-    float *f = qscale + (long)row * 4;
-    f[0] = scale * log2e / (mu * (float)(1 << kKFixedShift));
-    f[1] = fj;
-    f[2] = jsum;
-    f[3] = 0.f;
-  }
-}
-
 // ---------------------------------------------------------------------------
 // merge: per (sequence, query head) combine the splits (log-sum-exp in log2
 // units) and apply Pi^T: o_i = sum_k Pi[vperm(k)][i] o~_k / L.
@@ -751,7 +858,7 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
                                                     int max_seq_len, int chunk, int n_splits,
                                                     const float *partials, float *out, float *lse) {
   __shared__ float s_ot[D];
-  __shared__ float s_w[kMergeMaxSplits];
+  __shared__ float s_w[kMergeMaxSplits], s_l[kMergeMaxSplits];
   __shared__ __align__(16) float s_acc[4][D];
   __shared__ float red[4];
   const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -760,50 +867,60 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
   uint4 pw[16];
   load_bf16_row(p.pivt + tid * D, pw);
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next kernel in the stream (an append, the next decode) may launch and
+  // load its parameters now; it waits for this grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int s = row / n_q_heads;
+  const float *src = partials + (long)row * n_splits * kPartialFloats;
+  // One round of loads: the sequence length, and warp w's outputs of splits
+  // w, w + 4, ... (lane j: outputs 4 j .. 4 j + 3) of every allocated split,
+  // requested before any of them is used; splits past the used ones are
+  // ignored below (their slots may hold anything).
+  constexpr int kOPerWarp = 16;  // splits per warp held in registers
+  float4 o4[kOPerWarp];
+#pragma unroll
+  for (int e = 0; e < kOPerWarp; ++e) {
+    const int sp = warp + 4 * e;
+    if (sp < n_splits) o4[e] = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
+  }
   int len = seq_lens[s];
   len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
   const int used = min((len + chunk - 1) / chunk, kMergeMaxSplits);
-  const float *src = partials + (long)row * n_splits * kPartialFloats;
-  // split maxima (log2 units) in parallel, then the weights 2^(m_s - M)
   float mloc = -INFINITY;
   for (int sp = tid; sp < used; sp += 128) {
-    const float m = src[sp * kPartialFloats];
-    s_w[sp] = m;
-    mloc = fmaxf(mloc, m);
+    const float2 ml = *reinterpret_cast<const float2 *>(src + sp * kPartialFloats);
+    s_w[sp] = ml.x;
+    s_l[sp] = ml.y;
+    mloc = fmaxf(mloc, ml.x);
   }
-  const float mm = block_max128(mloc, red);
+  const float mm = block_max128(mloc, red);  // split maxima in log2 units
   float lpart = 0.f;
   for (int sp = tid; sp < used; sp += 128) {
     const float w = s_w[sp] == -INFINITY ? 0.f : exp2f(s_w[sp] - mm);
     s_w[sp] = w;
-    lpart = fmaf(w, src[sp * kPartialFloats + 1], lpart);
+    lpart = fmaf(w, s_l[sp], lpart);
   }
   __syncthreads();
-  // warp w takes splits w, w + 4, ...; lane j the outputs 4 j .. 4 j + 3.
-  // Four splits per round keep four independent 16-byte loads in flight.
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int sp = warp;
-  for (; sp + 12 < used; sp += 16) {
-    float4 o4[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o4[e] = reinterpret_cast<const float4 *>(src + (sp + 4 * e) * kPartialFloats + 4)[lane];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float w = s_w[sp + 4 * e];
+  for (int e = 0; e < kOPerWarp; ++e) {
+    const int sp = warp + 4 * e;
+    if (sp < used) {
+      const float w = s_w[sp];
       acc.x = fmaf(w, o4[e].x, acc.x);
       acc.y = fmaf(w, o4[e].y, acc.y);
       acc.z = fmaf(w, o4[e].z, acc.z);
       acc.w = fmaf(w, o4[e].w, acc.w);
     }
   }
-  for (; sp < used; sp += 4) {
-    const float4 o4 = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
+  // splits beyond 4 * kOPerWarp (long sequences with short splits)
+  for (int sp = warp + 4 * kOPerWarp; sp < used; sp += 4) {
+    const float4 v = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
     const float w = s_w[sp];
-    acc.x = fmaf(w, o4.x, acc.x);
-    acc.y = fmaf(w, o4.y, acc.y);
-    acc.z = fmaf(w, o4.z, acc.z);
-    acc.w = fmaf(w, o4.w, acc.w);
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
   }
   reinterpret_cast<float4 *>(s_acc[warp])[lane] = acc;
   for (int o = 16; o; o >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, o);
@@ -888,25 +1005,14 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   cudaStream_t st = (cudaStream_t)stream;
   const int rows = c.n_seqs * n_q_heads;
   const int group = n_q_heads / c.n_kv_heads;
-  uint8_t *q8 = reinterpret_cast<uint8_t *>(workspace + ws.q8);
-  float *qscale = reinterpret_cast<float *>(workspace + ws.qscale);
   float *partials = reinterpret_cast<float *>(workspace + ws.partials);
 
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
-  cudaLaunchConfig_t rcfg = {};
-  rcfg.gridDim = dim3(rows);
-  rcfg.blockDim = dim3(128);
-  rcfg.stream = st;
-  rcfg.attrs = pdl;
-  rcfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&rcfg, rotate_q_kernel, p, q, q_dtype, scale, q8, qscale);
-  if (e != cudaSuccess) return (int)e;
-
   const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1);
-  DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q8, qscale, partials};
+  DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q, q_dtype, scale, partials};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(split.n_splits, c.n_kv_heads, c.n_seqs);
   cfg.blockDim = dim3(kThreads);
@@ -914,7 +1020,7 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   cfg.stream = st;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, v.fn, args);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, v.fn, args);
   if (e != cudaSuccess) return (int)e;
 
   cudaLaunchConfig_t mcfg = {};

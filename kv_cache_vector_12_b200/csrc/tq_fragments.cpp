@@ -3,9 +3,10 @@
 // The decode kernel expands the codes a thread loads straight into its MMA
 // fragments, so the head dimension appears inside a fragment in an order set
 // by the bit layout.  These functions give, for each position of the logical
-// (fragment) order, the coordinate of the head vector it holds.  rotate_q
-// writes q_hat (and q_tilde) in the K (and QJL) order; the inverse rotation
-// in merge reads Pi's rows in the V order.  Each is a permutation of 0..127.
+// (fragment) order, the coordinate of the head vector it holds.  The decode
+// kernel computes q_hat (and q_tilde) in the K (and QJL) order from Pi (and
+// S) stored with permuted rows; the inverse rotation in merge reads Pi's rows
+// in the V order.  Each is a permutation of 0..127.
 #include <cstdint>
 
 #include "tq_internal.h"

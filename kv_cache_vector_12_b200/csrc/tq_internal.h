@@ -41,9 +41,10 @@ constexpr int kKFixedShift = 17;
 // Device-resident parameters of one context (all pointers device memory).
 struct DeviceParams {
   const uint16_t *pi;     // Pi  [d][d] bf16 bits, row-major (z = Pi x)
-  const uint16_t *pit;    // Pi^T [d][d] bf16 bits
+  const uint32_t *pikf;   // Pi with rows in K fragment order, as the decode kernel's bf16 MMA B fragments:
+                          // [warp 4][n-tile 4][chunk 4][lane 32][4 words] (16-byte aligned; see tq_api.cu)
   const float *s;         // S   [d][d] fp32 (qjl only)
-  const float *st;        // S^T [d][d] fp32 (qjl only)
+  const float *sjk;       // [d][d] fp32: sjk[kappa][kappa'] = S[jperm[kappa]][kperm[kappa']] (qjl only)
   const float *cb;        // [4][16]: centroids_k, thresholds_k, centroids_v, thresholds_v
   unsigned *err;          // sticky error flags
   const uint8_t *kperm;   // [d] K fragment order -> coordinate
@@ -66,12 +67,12 @@ struct DecodeSplit {
 DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm);
 int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group);
 
-// Workspace layout of decode attention (byte offsets, 256-aligned):
-// q8 [rows][4][d] bytes, qscale [rows][4] floats, partials [rows][splits][d+4]
-// (a partial is m, l, two unused floats, then the d outputs: 16-byte aligned).
+// Workspace layout of decode attention (byte offsets, 256-aligned): the split
+// partials [rows][splits][d+4] (m, l, two unused floats, then the d outputs,
+// so every output block is 16-byte aligned).
 constexpr int kPartialFloats = kHeadDim + 4;
 struct DecodeWorkspace {
-  size_t q8, qscale, partials, total;
+  size_t partials, total;
 };
 DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split);
 

@@ -124,23 +124,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 struct QuantTcArgs {
   DeviceParams p;
   tq_cache c;
@@ -154,60 +137,59 @@ struct QuantTcArgs {
 // All ones when a > b, else 0.
 __device__ __forceinline__ int gt_mask(float a, float b) { return -(int)(a > b); }
 
-// Code of one rotated coordinate: #{j : T_j < z} with T_j = t_j ||x||,
-// evaluated as sign + count of the positive thresholds below |z| (the
-// codebook is symmetric, t_{half-1} = 0): with m = #{j : tp_j < |z|} and
-// sn = -1 for z > 0 (else 0), half - 1 - (m ^ sn) is half + m for z > 0 and
-// half - 1 - m otherwise.  z = 0 (also a zero vector) gives half - 1.
+// Code of one rotated coordinate, #{j : T_j < z} with T_j = t_j ||x||,
+// returned as its offset from half - 1.  The codebook is symmetric
+// (t_{half-1} = 0), so with mn = -#{j : tp_j < |z|} (tp: the positive
+// thresholds) and sn = -1 for z > 0 (else 0), the offset (mn ^ sn) - 2 sn is
+// m + 1 for z > 0 and -m otherwise.  z = 0 (also a zero vector) gives 0.
 template <int B>
-__device__ __forceinline__ uint32_t code_of(float z, const float (&tp)[(1 << (B - 1)) - 1]) {
+__device__ __forceinline__ int code_offset(float z, const float (&tp)[(1 << (B - 1)) - 1]) {
   constexpr int half = 1 << (B - 1);
   const float a = fabsf(z);
-  int neg_m = 0;
+  int mn = 0;
 #pragma unroll
-  for (int j = 0; j < half - 1; ++j) neg_m += gt_mask(a, tp[j]);
-  return (uint32_t)((half - 1) - ((-neg_m) ^ gt_mask(z, 0.f)));
+  for (int j = 0; j < half - 1; ++j) mn += gt_mask(a, tp[j]);
+  const int sn = gt_mask(z, 0.f);
+  return (mn ^ sn) - 2 * sn;
+}
+
+// Word of `n` codes of `bits` bits each (LSB first) from their offsets: the
+// offsets are summed at their positions and half - 1 is added to every field
+// at once (arithmetic modulo 2^32, so borrows between fields cancel exactly).
+template <int B, int n, int bits>
+__device__ __forceinline__ uint32_t pack_offsets(const float *z, const float (&tp)[(1 << (B - 1)) - 1]) {
+  constexpr uint32_t half_m1 = (1u << (B - 1)) - 1;
+  uint32_t ones = 0, x = 0;
+#pragma unroll
+  for (int j = 0; j < n; ++j) ones |= 1u << (bits * j);
+#pragma unroll
+  for (int j = 0; j < n; ++j) x += (uint32_t)code_offset<B>(z[j], tp) * (1u << (bits * j));
+  return x + half_m1 * ones;
 }
 
 // Codes of coordinates 16 c .. 16 c + 15 packed into the words of the cache
-// layout as they are computed: LSB-first for 2 and 4 bits; for 3 bits, in
-// each 32-coordinate group nibble l % 8 of word l / 8 (l < 24), and the eight
-// spare-column codes gathered into the nibbles of one word whose bit k of
-// every nibble then moves to bit 3 of word k.
+// layout: LSB-first for 2 and 4 bits; for 3 bits, in each 32-coordinate group
+// nibble l % 8 of word l / 8 (l < 24), and the eight spare-column codes
+// gathered into the nibbles of one word whose bit k of every nibble then
+// moves to bit 3 of word k.
 template <int B>
 __device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const float (&tp)[(1 << (B - 1)) - 1],
                                            uint32_t (&w)[4 * B]) {
   if constexpr (B == 3) {
     const int g = c >> 1;
     if ((c & 1) == 0) {
-      uint32_t x0 = 0u, x1 = 0u;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        x0 |= code_of<3>(z[j], tp) << (4 * j);
-        x1 |= code_of<3>(z[8 + j], tp) << (4 * j);
-      }
-      w[3 * g] = x0;
-      w[3 * g + 1] = x1;
+      w[3 * g] = pack_offsets<3, 8, 4>(z, tp);
+      w[3 * g + 1] = pack_offsets<3, 8, 4>(z + 8, tp);
     } else {
-      uint32_t x2 = 0u, sp = 0u;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        x2 |= code_of<3>(z[j], tp) << (4 * j);
-        sp |= code_of<3>(z[8 + j], tp) << (4 * j);
-      }
+      const uint32_t sp = pack_offsets<3, 8, 4>(z + 8, tp);
       w[3 * g] |= (sp << 3) & 0x88888888u;
       w[3 * g + 1] |= (sp << 2) & 0x88888888u;
-      w[3 * g + 2] = x2 | ((sp << 1) & 0x88888888u);
+      w[3 * g + 2] = pack_offsets<3, 8, 4>(z, tp) | ((sp << 1) & 0x88888888u);
     }
   } else {
     constexpr int per = 32 / B;  // codes per word
 #pragma unroll
-    for (int k = 0; k < 16 / per; ++k) {
-      uint32_t x = 0u;
-#pragma unroll
-      for (int j = 0; j < per; ++j) x |= code_of<B>(z[per * k + j], tp) << (B * j);
-      w[(16 / per) * c + k] = x;
-    }
+    for (int k = 0; k < 16 / per; ++k) w[(16 / per) * c + k] = pack_offsets<B, per, B>(z + per * k, tp);
   }
 }
 

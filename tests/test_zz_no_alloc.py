@@ -77,7 +77,7 @@ def test_noalloc_matches_workspace_path_on_two_calls_in_a_row(tq):
 
 def test_noalloc_rejects_workspace_beyond_static_scratch(tq):
     ctx = tq.Context(D, 3, 3, 0, 42)
-    n_seqs, n_q = 128, 128          # 16384 query rows: their q fragments alone exceed the scratch
+    n_seqs, n_q = 128, 128          # 16384 query rows: one 528-byte partial each exceeds the scratch
     cache = tq.Cache(ctx, n_seqs, 8, 64)
     max_len = 64
     need = tq.workspace_bytes(ctx, n_seqs, n_q, max_len)
