@@ -52,6 +52,13 @@ WORKLOAD_DESCS = {
     "llama70b": ("llama70b: 70B-shaped long context, 8 KV / 64 query heads (GQA 8), d=128, 131072 cached "
                  "tokens, batch 4, bf16 K/V ~ N(0,1) with 10 (head, channel) outliers x20, 3-bit K and V; "
                  "step = append-quantize 1 token per sequence + batched decode attention"),
+    "tiny": ("tiny: 1 KV head, 1 query head, d=128, 1024 cached tokens, K, V, q iid N(0,1) (bf16 at the "
+             "boundary), 3-bit K and V; step = append-quantize 1 token + decode attention"),
+    "qwen": ("qwen: Qwen-like anisotropic norms, 4 KV / 28 query heads (GQA 7), d=128, 16384 cached tokens, "
+             "K norms U[172,778], V norms U[2,4], directions uniform on the sphere, q on the unit sphere; "
+             "step = append-quantize 1 token + decode attention"),
+    "serving": ("serving: 32 sequences, lengths uniform on [1024, 65536] (seeded), 8 KV / 32 query heads, "
+                "d=128, bf16 N(0,1); step = append-quantize 1 token per sequence + ragged batched decode"),
 }
 WORKLOAD_DESC = WORKLOAD_DESCS["llama8b"]
 
@@ -229,6 +236,9 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--replicas", type=int, default=0, help="cache replicas (default: enough to exceed L2)")
     ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOAD_DESCS))
+    ap.add_argument("--bits", type=int, nargs=2, metavar=("K", "V"), default=None,
+                    help="code bits of K and V (default: the workload's)")
+    ap.add_argument("--qjl", type=int, choices=[0, 1], default=None, help="1-bit QJL on K (default: the workload's)")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each call kind alone (append quantize, decode) and add it to the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -249,22 +259,27 @@ def main(argv=None) -> int:
     from kv_cache_vector_12_b200 import tq
     from kv_cache_vector_12_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
-    T, H, HQ, D, B = w.seq_len, w.n_kv_heads, w.n_q_heads, w.d, w.n_seqs
-    bytes_per_token = H * (D * (w.bits_k + w.bits_v) // 8 + 4)
-    R = args.replicas or max(1, math.ceil(2 * 126e6 / (B * T * bytes_per_token)))
+    bits_k, bits_v = args.bits if args.bits else (w.bits_k, w.bits_v)
+    qjl = w.qjl if args.qjl is None else bool(args.qjl)
+    H, HQ, D, B = w.n_kv_heads, w.n_q_heads, w.d, w.n_seqs
+    lens0 = wl.serving_lengths(w, w.seed) if args.workload == "serving" else [w.seq_len] * B
+    T = lens0[0]                       # the quantize measurement uses the first sequence's prefill
+    bytes_per_token = H * (D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
+    R = args.replicas or max(1, math.ceil(2 * 126e6 / (sum(lens0) * bytes_per_token)))
     n_steps_total = args.warmup + args.steps
-    cap = int(math.ceil((T + n_steps_total + 1) / 64) * 64)
-    ctx = tq.Context(D, w.bits_k, w.bits_v, 0, w.pi_seed)
+    cap = int(math.ceil((max(lens0) + n_steps_total + 1) / 64) * 64)
+    ctx = tq.Context(D, bits_k, bits_v, int(qjl), w.pi_seed)
     caches = [tq.Cache(ctx, B, H, cap, device=dev) for _ in range(R)]
     gen = wl.generator(dev, w.seed + 7919 * rank)
     outl = wl.outlier_scale(w, dev, w.seed) if args.workload == "llama70b" else None
 
     # ---- prefill quantize (also the quantize measurement: the first sequence) ----
-    pos0 = torch.arange(T, dtype=torch.int32, device=dev)
     q_ms = None
     for b in range(B):
-        k_pre, v_pre = wl.kv_tokens(w, T, gen, dev, outlier_mask=outl)
-        seqb = torch.full((T,), b, dtype=torch.int32, device=dev)
+        n_b = lens0[b]
+        pos0 = torch.arange(n_b, dtype=torch.int32, device=dev)
+        k_pre, v_pre = wl.kv_tokens(w, n_b, gen, dev, outlier_mask=outl)
+        seqb = torch.full((n_b,), b, dtype=torch.int32, device=dev)
         for c in caches:
             tq.quantize(ctx, c, k_pre, v_pre, seqb, pos0)
         if b == 0:
@@ -286,10 +301,10 @@ def main(argv=None) -> int:
     q_all = wl.queries(w, n_steps_total * B, gen, dev).view(n_steps_total, B, HQ, D)
     pos_steps = torch.empty(n_steps_total, B, dtype=torch.int32, device=dev)
     lens_steps = torch.empty(n_steps_total, B, dtype=torch.int32, device=dev)
+    lens_t = torch.tensor(lens0, dtype=torch.int32, device=dev)
     for i in range(n_steps_total):
-        p = T + i // R
-        pos_steps[i] = p
-        lens_steps[i] = p + 1
+        pos_steps[i] = lens_t + i // R
+        lens_steps[i] = lens_t + i // R + 1
     out = torch.empty(n_steps_total, B, HQ, D, device=dev)
     lse = torch.empty(n_steps_total, B, HQ, device=dev)
     max_len = cap
@@ -429,7 +444,7 @@ def main(argv=None) -> int:
     e2e_val = job_gbps(ws, timed_bytes, e2e_ms)
     dec_achieved = (timed_bytes / args.steps) / (dec_mean * 1e-3) / 1e9
     q_tokens = T / (q_ms * 1e-3)
-    q_bytes = T * H * (2 * D * 2 + D * (w.bits_k + w.bits_v) // 8 + 4)
+    q_bytes = T * H * (2 * D * 2 + D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
     q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
 
     if rank != 0:
@@ -442,7 +457,8 @@ def main(argv=None) -> int:
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESCS[args.workload], "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
+        "config": {"workload": WORKLOAD_DESCS[args.workload], "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl,
+                   "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
                    f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
