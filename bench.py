@@ -63,6 +63,13 @@ WORKLOAD_DESCS = {
 WORKLOAD_DESC = WORKLOAD_DESCS["llama8b"]
 
 
+# DRAM bytes per attention-kernel launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from one ncu capture of the default command, keyed by
+# (workload, bits_k, bits_v, qjl); null elsewhere.  Re-captured whenever the
+# kernel changes.
+MEASURED_TRAFFIC = {("llama8b", 3, 3, False): 26351360.0}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -462,7 +469,9 @@ def main(argv=None) -> int:
                    f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
-                     "frac": dec_achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "frac": dec_achieved / peak,
+                     "traffic": MEASURED_TRAFFIC.get((args.workload, bits_k, bits_v, qjl)),
+                     "traffic_kernel": "decode_mma_kernel", "peak_source": peak_kind,
                      "kernel": "tq_decode_attention call (split-K attention with q rotation + merge)",
                      "algorithmic_bytes_per_call": timed_bytes / args.steps},
         "quantize": {"tokens_per_s": q_tokens, "GBps": q_gbs, "frac": q_gbs / peak, "ms": q_ms,
