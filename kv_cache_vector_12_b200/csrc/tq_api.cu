@@ -152,6 +152,17 @@ tq_status report_error(tq_status st, const char *fmt, ...) {
   return st;
 }
 
+void mma_b_fragments(const uint16_t *m_bits, uint32_t *out) {
+  for (int nt = 0; nt < 16; ++nt)
+    for (int j = 0; j < 4; ++j)
+      for (int lane = 0; lane < 32; ++lane)
+        for (int e = 0; e < 4; ++e) {
+          const int ks = (4 * j + e) / 2, b = (4 * j + e) % 2;
+          const uint16_t *src = m_bits + (size_t)(8 * nt + lane / 4) * kHeadDim + 16 * ks + 8 * b + 2 * (lane % 4);
+          out[((nt * 4 + j) * 32 + lane) * 4 + e] = (uint32_t)src[0] | ((uint32_t)src[1] << 16);
+        }
+}
+
 DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t rows = (size_t)n_seqs * n_q_heads;
@@ -233,10 +244,11 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
-  // One block: pi | pik | pivt | s | sjk | codebooks | kperm | jperm | error word.
+  // One block: pi | pik | pivt | pif | s | sjk | sf | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
-  const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_s = off_piv + dd * 2;
-  const size_t off_sjk = off_s + dd * 4, off_cb = off_sjk + dd * 4;
+  const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_pif = off_piv + dd * 2;
+  const size_t off_s = off_pif + dd * 2;
+  const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_cb = off_sf + 3 * dd * 2;
   const size_t off_kperm = off_cb + 4 * tq::kMaxLevels * 4, off_jperm = off_kperm + 256;
   const size_t off_err = off_jperm + 256, total = off_err + 256;
   e = cudaMalloc(&ctx->dev_block, total);
@@ -247,28 +259,30 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   std::vector<char> h(total, 0);
   std::memcpy(h.data() + off_pi, ctx->pi_bits.data(), dd * 2);
   // Pi with its rows in the K fragment order (q_hat = Pi q then comes out of
-  // the MMA in that order), laid out as the B fragments of mma m16n8k16 so
-  // that each thread of the decode kernel loads its 64 bytes per n-tile with
-  // four fully coalesced 16-byte loads: 32-bit word 4 j + e of lane
-  // (r = lane / 4, qq = lane % 4) in (warp w, n-tile nt) holds the bf16 pair
-  // at row kappa = 32 w + 8 nt + r, columns 16 ks + 8 b + 2 qq (+1), with
-  // ks = (4 j + e) / 2 and b = (4 j + e) % 2.
-  uint32_t *pikf = (uint32_t *)(h.data() + off_pik);
-  for (int w = 0; w < 4; ++w)
-    for (int nt = 0; nt < 4; ++nt)
-      for (int j = 0; j < 4; ++j)
-        for (int lane = 0; lane < 32; ++lane)
-          for (int e = 0; e < 4; ++e) {
-            const int kap = 32 * w + 8 * nt + lane / 4, ks = (4 * j + e) / 2, b = (4 * j + e) % 2;
-            const int col = 16 * ks + 8 * b + 2 * (lane % 4);
-            const uint16_t *src = ctx->pi_bits.data() + (size_t)kperm[kap] * d + col;
-            pikf[(((w * 4 + nt) * 4 + j) * 32 + lane) * 4 + e] = (uint32_t)src[0] | ((uint32_t)src[1] << 16);
-          }
+  // the decode kernel's MMA in that order), as B fragments: consumer warp w
+  // reads n-tiles 4 w .. 4 w + 3.
+  {
+    std::vector<uint16_t> pik(dd);
+    for (int kap = 0; kap < d; ++kap)
+      std::memcpy(pik.data() + (size_t)kap * d, ctx->pi_bits.data() + (size_t)kperm[kap] * d, (size_t)d * 2);
+    tq::mma_b_fragments(pik.data(), (uint32_t *)(h.data() + off_pik));
+  }
+  tq::mma_b_fragments(ctx->pi_bits.data(), (uint32_t *)(h.data() + off_pif));
   if (qjl) {
     std::memcpy(h.data() + off_s, ctx->s.data(), dd * 4);
     float *sjk = (float *)(h.data() + off_sjk);
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < d; ++j) sjk[(size_t)i * d + j] = ctx->s[(size_t)jperm[i] * d + kperm[j]];
+    // S = hi + mid + lo with three bf16 parts (exact: 24 significant bits)
+    std::vector<uint16_t> part(dd);
+    std::vector<double> rest(ctx->s.begin(), ctx->s.end());
+    for (int k = 0; k < 3; ++k) {
+      for (size_t i = 0; i < dd; ++i) {
+        part[i] = tq::double_to_bf16_bits(rest[i]);
+        rest[i] -= (double)tq::bf16_bits_to_float(part[i]);
+      }
+      tq::mma_b_fragments(part.data(), (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
+    }
   }
   uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
   for (int i = 0; i < d; ++i)
@@ -291,6 +305,8 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->dp.pikf = (const uint32_t *)(base + off_pik);
   ctx->dp.s = (const float *)(base + off_s);
   ctx->dp.sjk = (const float *)(base + off_sjk);
+  ctx->dp.pif = (const uint32_t *)(base + off_pif);
+  ctx->dp.sf = (const uint32_t *)(base + off_sf);
   ctx->dp.cb = (const float *)(base + off_cb);
   ctx->dp.err = (unsigned *)(base + off_err);
   ctx->dp.pivt = (const uint16_t *)(base + off_piv);

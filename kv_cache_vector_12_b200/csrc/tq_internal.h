@@ -45,6 +45,9 @@ struct DeviceParams {
                           // [warp 4][n-tile 4][chunk 4][lane 32][4 words] (16-byte aligned; see tq_api.cu)
   const float *s;         // S   [d][d] fp32 (qjl only)
   const float *sjk;       // [d][d] fp32: sjk[kappa][kappa'] = S[jperm[kappa]][kperm[kappa']] (qjl only)
+  const uint32_t *pif;    // Pi (natural row order) as bf16 MMA B fragments [n-tile 16][chunk 4][lane 32][4 words]
+  const uint32_t *sf;     // S split into three bf16 parts (S = hi + mid + lo), each as B fragments like pif:
+                          // [part 3][n-tile 16][chunk 4][lane 32][4 words] (qjl only)
   const float *cb;        // [4][16]: centroids_k, thresholds_k, centroids_v, thresholds_v
   unsigned *err;          // sticky error flags
   const uint8_t *kperm;   // [d] K fragment order -> coordinate
@@ -84,6 +87,15 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream);
+int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
+                        const int32_t *pos, int n_tok, void *stream);
+
+// B fragments of mma m16n8k16 for a 128 x 128 row-major bf16 matrix M (the
+// product is X M^T): 32-bit word 4 j + e of lane (r = lane / 4, qq = lane % 4)
+// in n-tile nt holds the pair M[8 nt + r][16 ks + 8 b + 2 qq (+1)] with
+// ks = (4 j + e) / 2 and b = (4 j + e) % 2, so a thread loads an n-tile's
+// fragments with four coalesced 16-byte loads (tq_api.cu).
+void mma_b_fragments(const uint16_t *m_bits, uint32_t *out);
 int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype,
                   int n_q_heads, const int32_t *seq_lens, int max_seq_len, float scale,
                   float *out, float *lse, char *workspace, const DecodeSplit &split,

@@ -149,9 +149,9 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
 }  // namespace
 
 // Batches of up to kRowKernelMaxRows rows per matrix (decode-time appends) use
-// the one-CTA-per-row kernel; larger batches use the tensor-core kernel for
-// every MSE-only matrix (all of V, K without QJL) and the row kernel for K
-// rows with QJL.
+// the one-CTA-per-row kernel; larger batches use the tcgen05 kernel for every
+// MSE-only matrix (all of V, K without QJL) and the tiled QJL kernel
+// (tq_quantize_qjl.cu) for K with QJL.
 constexpr long kRowKernelMaxRows = 1024;
 
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
@@ -174,8 +174,7 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
   const bool k_on_tc = !p.qjl;
   const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, stream);
   if (e != 0 || k_on_tc) return e;
-  cfg.gridDim = dim3((unsigned)rows, 1);
-  return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel, p, c, kk, vv, seq_idx, pos);
+  return launch_quantize_qjl(p, c, k, seq_idx, pos, n_tok, stream);
 }
 
 }  // namespace tq

@@ -100,13 +100,17 @@ def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=
 
 
 @pytest.mark.parametrize("bits_k,bits_v,qjl", SETTINGS)
-@pytest.mark.parametrize("n_tok,n_heads", [(1, 1), (7, 3), (127, 1), (128, 2), (129, 1), (1000, 8)])
+@pytest.mark.parametrize("n_tok,n_heads", [(1, 1), (7, 3), (127, 1), (128, 2), (129, 1), (1000, 8), (1031, 3)])
 def test_quantize_parity(tq, n_tok, n_heads, bits_k, bits_v, qjl):
+    # up to 1024 rows per matrix: the one-CTA-per-row kernel; above: the
+    # tcgen05 tile kernel, and the tiled QJL kernel for K with QJL (1031 x 3
+    # rows leave a partial last tile in both)
     _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed=n_tok * 31 + n_heads)
 
 
-def test_quantize_zero_vectors(tq):
-    _quantize_and_compare(tq, 40, 2, 3, 3, 1, seed=5, zero_rows=9)
+@pytest.mark.parametrize("n_tok", [40, 700])   # row kernel; tile kernels
+def test_quantize_zero_vectors(tq, n_tok):
+    _quantize_and_compare(tq, n_tok, 2, 3, 3, 1, seed=5, zero_rows=9)
 
 
 def test_quantize_mismatch_rate_at_scale(tq):
@@ -132,6 +136,31 @@ def test_quantize_out_of_range_tokens_are_flagged_not_written(tq):
     assert int(cache.planes["norm_k"][0, :, 0].ne(0).sum()) == 2      # the valid token landed
     assert int(cache.planes["norm_k"][0, :, 1:].ne(0).sum()) == 0
     ctx.check_device_errors()                                          # flags were cleared
+
+
+@pytest.mark.parametrize("qjl", [0, 1])
+def test_quantize_tile_kernels_flag_out_of_range_tokens(tq, qjl):
+    """Batches above the row kernel's limit: tokens with a bad sequence or
+    position are flagged and skipped, every other token lands."""
+    ctx = tq.Context(D, 3, 3, qjl, 42)
+    n_tok, n_heads = 600, 2                                            # 1200 rows per matrix
+    cache = tq.Cache(ctx, 2, n_heads, 640)
+    k = make_rows(n_tok, n_heads, 11).cuda()
+    seq_idx = torch.zeros(n_tok, dtype=torch.int32)
+    pos = torch.arange(n_tok, dtype=torch.int32)
+    seq_idx[5], pos[17], pos[599] = 2, 640, -1                         # no sequence 2; pos outside [0, 640)
+    tq.quantize(ctx, cache, k, k, seq_idx.cuda(), pos.cuda())
+    with pytest.raises(tq.TQError) as ei:
+        ctx.check_device_errors()
+    assert ei.value.status == tq.TQ_ERR_DEVICE
+    landed = cache.planes["norm_k"][0].ne(0).cpu()
+    expect = torch.zeros(n_heads, 640, dtype=torch.bool)
+    good = [t for t in range(n_tok) if t not in (5, 17, 599)]
+    expect[:, torch.tensor(good)] = True
+    assert torch.equal(landed, expect)
+    assert int(cache.planes["norm_v"][1].ne(0).sum()) == 0
+    if qjl:
+        assert torch.equal(cache.planes["qjl_norm"][0].ne(0).cpu(), expect)
 
 
 # ------------------------------------------------------------------ decode
