@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
                                                                     const int32_t *__restrict__ seq_idx,
                                                                     const int32_t *__restrict__ pos, int n_rows) {
   constexpr int half = 1 << (BK - 1);
-  __shared__ __align__(16) uint8_t s_code[kRows][D];
+  __shared__ __align__(16) uint8_t s_code[kRows][D + 4];  // rows padded by one bank
   __shared__ float s_cent[1 << BK];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = lane >> 2, q = lane & 3;
   // parameters (written long before) first, then wait for the previous kernel
@@ -125,21 +125,23 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
   }
   const float nrm[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
 
-  // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8
+  // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8.
+  // The n-tiles are the inner loop, so consecutive MMAs feed 16 independent
+  // accumulators.
   float z[16][4];
   const uint4 *pif = reinterpret_cast<const uint4 *>(p.pif);
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int e = 0; e < 4; ++e) z[nt][e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
       const uint4 v = pif[(nt * 4 + j) * 32 + lane];
-      mma_bf16(acc, a[2 * j], v.x, v.y);
-      mma_bf16(acc, a[2 * j + 1], v.z, v.w);
+      mma_bf16(z[nt], a[2 * j], v.x, v.y);
+      mma_bf16(z[nt], a[2 * j + 1], v.z, v.w);
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) z[nt][e] = acc[e];
-  }
 
   // ---- codes (to shared memory), residuals r = y - c[code], ||r||^2
   float tp[2][half - 1];
@@ -152,15 +154,19 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int hr = e >> 1;  // 0: row r, 1: row r + 8
-      const float zz = z[nt][e];
-      const int code = code_of<BK>(zz, tp[hr]);
-      s_code[16 * warp + r + 8 * hr][8 * nt + 2 * q + (e & 1)] = (uint8_t)code;
-      const float y = nrm[hr] > 0.f ? zz / nrm[hr] : 0.f;
-      const float res = y - s_cent[code];
-      z[nt][e] = res;
-      gg[hr] = fmaf(res, res, gg[hr]);
+    for (int hr = 0; hr < 2; ++hr) {  // 0: row r, 1: row r + 8; columns 8 nt + 2 q and + 1
+      int code[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float zz = z[nt][2 * hr + u];
+        code[u] = code_of<BK>(zz, tp[hr]);
+        const float y = nrm[hr] > 0.f ? zz / nrm[hr] : 0.f;
+        const float res = y - s_cent[code[u]];
+        z[nt][2 * hr + u] = res;
+        gg[hr] = fmaf(res, res, gg[hr]);
+      }
+      *reinterpret_cast<uint16_t *>(&s_code[16 * warp + r + 8 * hr][8 * nt + 2 * q]) =
+          (uint16_t)(code[0] | (code[1] << 8));
     }
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -180,32 +186,43 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
   }
   const uint4 *sfh = reinterpret_cast<const uint4 *>(p.sf);
   const uint4 *sfm = sfh + kFragWords / 4, *sfl = sfm + kFragWords / 4;
+  // projection m = 8 nt + 2 q (+1) is bit m of the row; a projection of exactly
+  // 0 stores 1.  Two halves of 8 n-tiles: 8 independent accumulators between
+  // consecutive MMAs.
   uint32_t sb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};  // sign bits of rows r, r + 8 (LSB first)
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int hf = 0; hf < 2; ++hf) {
+    float acc[8][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int f = (nt * 4 + j) * 32 + lane;
-      const uint4 h = sfh[f], m = sfm[f], l = sfl[f];
+    for (int t = 0; t < 8; ++t)
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {  // k-steps 2 j and 2 j + 1
-        const int ks = 2 * j + u;
-        const uint32_t hb0 = u ? h.z : h.x, hb1 = u ? h.w : h.y;
-        const uint32_t mb0 = u ? m.z : m.x, mb1 = u ? m.w : m.y;
-        const uint32_t lb0 = u ? l.z : l.x, lb1 = u ? l.w : l.y;
-        mma_bf16(acc, ah[ks], hb0, hb1);
-        mma_bf16(acc, ah[ks], mb0, mb1);
-        mma_bf16(acc, am[ks], hb0, hb1);
-        mma_bf16(acc, ah[ks], lb0, lb1);
-        mma_bf16(acc, al[ks], hb0, hb1);
-        mma_bf16(acc, am[ks], mb0, mb1);
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int f = ((8 * hf + t) * 4 + j) * 32 + lane;
+        const uint4 h = sfh[f], m = sfm[f], l = sfl[f];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {  // k-steps 2 j and 2 j + 1
+          const int ks = 2 * j + u;
+          const uint32_t hb0 = u ? h.z : h.x, hb1 = u ? h.w : h.y;
+          const uint32_t mb0 = u ? m.z : m.x, mb1 = u ? m.w : m.y;
+          const uint32_t lb0 = u ? l.z : l.x, lb1 = u ? l.w : l.y;
+          mma_bf16(acc[t], ah[ks], hb0, hb1);
+          mma_bf16(acc[t], ah[ks], mb0, mb1);
+          mma_bf16(acc[t], am[ks], hb0, hb1);
+          mma_bf16(acc[t], ah[ks], lb0, lb1);
+          mma_bf16(acc[t], al[ks], hb0, hb1);
+          mma_bf16(acc[t], am[ks], mb0, mb1);
+        }
       }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int nt = 8 * hf + t, sh = 8 * (nt & 3) + 2 * q;
+      sb[0][nt >> 2] |= ((acc[t][0] >= 0.f ? 1u : 0u) | (acc[t][1] >= 0.f ? 2u : 0u)) << sh;
+      sb[1][nt >> 2] |= ((acc[t][2] >= 0.f ? 1u : 0u) | (acc[t][3] >= 0.f ? 2u : 0u)) << sh;
     }
-    // projection m = 8 nt + 2 q (+1): bit m of the row, a projection of exactly 0 stores 1
-    const int sh = 8 * (nt & 3) + 2 * q;
-    sb[0][nt >> 2] |= ((acc[0] >= 0.f ? 1u : 0u) | (acc[1] >= 0.f ? 2u : 0u)) << sh;
-    sb[1][nt >> 2] |= ((acc[2] >= 0.f ? 1u : 0u) | (acc[3] >= 0.f ? 2u : 0u)) << sh;
   }
 #pragma unroll
   for (int e = 0; e < 2; ++e)

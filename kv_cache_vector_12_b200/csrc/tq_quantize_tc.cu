@@ -330,18 +330,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int slot = i % kRingStages;
       const bool is_k = t < a.tiles_k;
       const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
-      // destination of this row, fetched early (used after the codes)
-      long slot_i = -1;
-      int tok_h = 0;
-      if (row < a.n_rows) {
-        const int tok = row / a.c.n_kv_heads;
-        tok_h = row - tok * a.c.n_kv_heads;
-        const int s = a.seq_idx[tok], ps = a.pos[tok];
-        if (s >= 0 && s < a.c.n_seqs && ps >= 0 && ps < a.c.capacity)
-          slot_i = ((long)s * a.c.n_kv_heads + tok_h) * a.c.capacity + ps;
-        else if (tok_h == 0 && is_k)
-          atomicOr(a.p.err, kErrTokenRange);
-      }
+      // destination of this row: loaded now, checked after the codes, so the
+      // loads' latency overlaps the barrier waits and the epilogue
+      const bool live = row < a.n_rows;
+      const int tok = live ? row / a.c.n_kv_heads : 0;
+      const int tok_h = live ? row - tok * a.c.n_kv_heads : 0;
+      const int s_dst = a.seq_idx[tok], p_dst = a.pos[tok];
       if (!bar_wait(smem_addr(&full_bar[slot]), (i / kRingStages) & 1)) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
@@ -394,6 +388,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(smem_addr(&tempty_bar[g]));
 
+      long slot_i = -1;
+      if (live) {
+        if (s_dst >= 0 && s_dst < a.c.n_seqs && p_dst >= 0 && p_dst < a.c.capacity)
+          slot_i = ((long)s_dst * a.c.n_kv_heads + tok_h) * a.c.capacity + p_dst;
+        else if (tok_h == 0 && is_k)
+          atomicOr(a.p.err, kErrTokenRange);
+      }
       if (slot_i >= 0) {
         const int bits = is_k ? BK : BV;
         uint4 *dst = reinterpret_cast<uint4 *>((is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(16 * bits));
