@@ -45,6 +45,7 @@ constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr int kWarpTokens = 32;                            // tokens per consumer warp per stage
 constexpr int kStageTokens = kWarpTokens * kConsumerWarps;  // 128
 constexpr int kStages = 4;
+constexpr int kPrefetchTokens = kStages * kStageTokens;  // L2 prefetch before the dependency wait
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ PTX
@@ -98,6 +99,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     if (global_ns() - t0 > kWaitNs) return false;
   }
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -288,6 +294,27 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
         bfr[nt][2 * j + 1][0] = v.z;
         bfr[nt][2 * j + 1][1] = v.w;
       }
+  }
+  // While the previous kernel (typically the append) still runs, warm L2 with
+  // the first stages this CTA will stream.  A prefetch only moves lines into
+  // L2, the point of coherence, so whatever the previous kernel writes there
+  // is what the copies read after the wait; lengths are not known yet, so the
+  // split's whole range (below the length bound and the capacity) is fetched.
+  if (warp == kConsumerWarps && lane == 0) {
+    const int first = split * a.chunk;
+    const int last = min(min(first + a.chunk, a.max_seq_len), min(first + kPrefetchTokens, a.c.capacity));
+    if (first < last) {
+      const long tok = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + first;
+      const uint32_t n = (uint32_t)(last - first);
+      prefetch_l2(a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8));
+      prefetch_l2(a.c.codes_v + tok * (D * BV / 8), n * (D * BV / 8));
+      prefetch_l2(a.c.norm_k + tok, (n * 2 + 15) & ~15u);
+      prefetch_l2(a.c.norm_v + tok, (n * 2 + 15) & ~15u);
+      if constexpr (QJL) {
+        prefetch_l2(a.c.qjl_bits + tok * (D / 8), n * (D / 8));
+        prefetch_l2(a.c.qjl_norm + tok, (n * 2 + 15) & ~15u);
+      }
+    }
   }
   // launched as a programmatic dependent: the cache, q and seq_lens are final
   // once the previous kernel in the stream has completed
