@@ -301,6 +301,12 @@ __global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
   // is what the copies read after the wait; lengths are not known yet, so the
   // split's whole range (below the length bound and the capacity) is fetched.
   if (warp == kConsumerWarps && lane == 0) {
+    // this KV head's query rows and the sequence length (read right after the wait)
+    const size_t qbytes = (size_t)G * D * (a.q_dtype == TQ_F32 ? 4 : 2);
+    prefetch_l2(static_cast<const char *>(a.q) + ((size_t)s * a.n_q_heads + (size_t)h * G) * D *
+                                                     (a.q_dtype == TQ_F32 ? 4 : 2),
+                (uint32_t)qbytes);
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.seq_lens + s));
     const int first = split * a.chunk;
     const int last = min(min(first + a.chunk, a.max_seq_len), min(first + kPrefetchTokens, a.c.capacity));
     if (first < last) {

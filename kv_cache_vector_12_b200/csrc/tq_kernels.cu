@@ -95,6 +95,15 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   uint4 pw[16];
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch) pw[ch] = reinterpret_cast<const uint4 *>(p.pi + tid * D)[ch];
+  // warm L2 with this row's inputs (a prefetch only moves lines into L2, the
+  // point of coherence, so it may run before the previous kernel is done)
+  if (tid == 0) {
+    const long row = blockIdx.x;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"((blockIdx.y == 1 ? v_in : k_in) + row * D));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"((blockIdx.y == 1 ? v_in : k_in) + row * D + 64));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(seq_idx + row / c.n_kv_heads));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(pos + row / c.n_kv_heads));
+  }
   // launched as a programmatic dependent: no input is read before the
   // previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
