@@ -121,7 +121,9 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * D + tid]);
   s_x[tid] = x;
   const float n = sqrtf(block_sum128(x * x, red));  // also orders s_x
-  const float z = row_dot_bf16(pw, s_x);
+  // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
+  const bool live = n > 0x1p-25f;
+  const float z = live ? row_dot_bf16(pw, s_x) : 0.f;
   const float *thr = p.cb + (is_v ? 3 : 1) * kMaxLevels;
   const int half = 1 << (bits - 1);
   const float a = fabsf(z);
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
 
   if (qjl) {
     const float *cent = p.cb;  // K centroids
-    const float y = n > 0.f ? z / n : 0.f;
+    const float y = live ? z / n : 0.f;
     const float r = y - cent[code];
     s_r[tid] = r;
     const float gamma = sqrtf(block_sum128(r * r, red));

@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
     ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], 2);
   }
   const float nrm[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
+  // a vector whose stored fp16 norm is zero (||x|| <= 2^-25) is the zero vector
+  const bool live[2] = {nrm[0] > 0x1p-25f, nrm[1] > 0x1p-25f};
 
   // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8.
   // The n-tiles are the inner loop, so consecutive MMAs feed 16 independent
@@ -158,9 +160,9 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
       int code[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const float zz = z[nt][2 * hr + u];
+        const float zz = live[hr] ? z[nt][2 * hr + u] : 0.f;
         code[u] = code_of<BK>(zz, tp[hr]);
-        const float y = nrm[hr] > 0.f ? zz / nrm[hr] : 0.f;
+        const float y = live[hr] ? zz / nrm[hr] : 0.f;
         const float res = y - s_cent[code[u]];
         z[nt][2 * hr + u] = res;
         gg[hr] = fmaf(res, res, gg[hr]);

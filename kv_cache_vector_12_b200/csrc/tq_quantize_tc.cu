@@ -134,37 +134,67 @@ struct QuantTcArgs {
   int tiles_v;
 };
 
-// All ones when a > b, else 0.
-__device__ __forceinline__ int gt_mask(float a, float b) { return -(int)(a > b); }
-
-// Code of one rotated coordinate, #{j : T_j < z} with T_j = t_j ||x||,
-// returned as its offset from half - 1.  The codebook is symmetric
-// (t_{half-1} = 0), so with mn = -#{j : tp_j < |z|} (tp: the positive
-// thresholds) and sn = -1 for z > 0 (else 0), the offset (mn ^ sn) - 2 sn is
-// m + 1 for z > 0 and -m otherwise.  z = 0 (also a zero vector) gives 0.
-template <int B>
-__device__ __forceinline__ int code_offset(float z, const float (&tp)[(1 << (B - 1)) - 1]) {
-  constexpr int half = 1 << (B - 1);
-  const float a = fabsf(z);
-  int mn = 0;
-#pragma unroll
-  for (int j = 0; j < half - 1; ++j) mn += gt_mask(a, tp[j]);
-  const int sn = gt_mask(z, 0.f);
-  return (mn ^ sn) - 2 * sn;
+// 1 when a b + c > 0 (exact product and sum, one rounding), else 0 when the
+// result rounds to at most 0; values in (0, 1) only for exact results below 1.
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float d;
+  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
-// Word of `n` codes of `bits` bits each (LSB first) from their offsets: the
-// offsets are summed at their positions and half - 1 is added to every field
-// at once (arithmetic modulo 2^32, so borrows between fields cancel exactly).
+// Per-row constants of the code computation.  A row whose stored fp16 norm is
+// zero (||x|| <= 2^-25) is the zero vector (y = 0): sc = zc = 0.  Otherwise
+// sc = 2^64 / ||x|| (at most 2^89), zc = 2^127, and nt_j = -t_j 2^64 for the
+// positive unit thresholds t_j.  [|z| / ||x|| > t_j] is fma_sat(|z|, sc, nt_j):
+// the exact value |z| sc - t_j 2^64 is either <= 0 or at least t_j 2^16 > 1 (a
+// product of two floats differs from a float by at least 2^-48 of it unless
+// equal), so the saturated result is exactly 0 or 1; the comparison differs
+// from |z| > t_j ||x|| only by the rounding of 2^64 / ||x||.
+template <int B>
+struct CodeConsts {
+  float sc, zc, nt[(1 << (B - 1)) - 1];
+};
+
+// Offset from half - 1 of the code #{j : T_j < z} of one rotated coordinate,
+// exactly, as a float on the FMA pipe: m = #{j : t_j < |z| / ||x||},
+// p = [z > 0] (z zc 2^127 saturates to 1 for every positive float when
+// zc = 2^127, and to 0 otherwise), offset = p (2 m + 1) - m, i.e. m + 1 for
+// z > 0, -m otherwise.
+template <int B>
+__device__ __forceinline__ float code_offset_f(float z, const CodeConsts<B> &k) {
+  constexpr int half = 1 << (B - 1);
+  const float a = fabsf(z);
+  float m = fma_sat(a, k.sc, k.nt[0]);
+#pragma unroll
+  for (int j = 1; j < half - 1; ++j) m += fma_sat(a, k.sc, k.nt[j]);
+  const float p = mul_sat(z * k.zc, 0x1p127f);
+  return fmaf(p, fmaf(m, 2.f, 1.f), -m);
+}
+
+// 16 bits of codes (n codes of `bits` bits, LSB first): their offsets summed
+// at their positions in a float (exact: |sum| < 2^16), then half - 1 added to
+// every field and the integer read out of the mantissa of 2^23 + sum.
 template <int B, int n, int bits>
-__device__ __forceinline__ uint32_t pack_offsets(const float *z, const float (&tp)[(1 << (B - 1)) - 1]) {
-  constexpr uint32_t half_m1 = (1u << (B - 1)) - 1;
-  uint32_t ones = 0, x = 0;
+__device__ __forceinline__ uint32_t pack16(const float *z, const CodeConsts<B> &k) {
+  constexpr int half_m1 = (1 << (B - 1)) - 1;
+  float acc = 0.f;
 #pragma unroll
-  for (int j = 0; j < n; ++j) ones |= 1u << (bits * j);
+  for (int j = 0; j < n; ++j) acc = fmaf(code_offset_f<B>(z[j], k), (float)(1 << (bits * j)), acc);
+  int ones = 0;
 #pragma unroll
-  for (int j = 0; j < n; ++j) x += (uint32_t)code_offset<B>(z[j], tp) * (1u << (bits * j));
-  return x + half_m1 * ones;
+  for (int j = 0; j < n; ++j) ones += 1 << (bits * j);
+  return __float_as_uint(acc + (8388608.f + (float)(half_m1 * ones))) & 0xFFFFu;
+}
+
+__device__ __forceinline__ uint32_t join16(uint32_t lo, uint32_t hi) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(d) : "r"(lo), "r"(hi));
+  return d;
 }
 
 // Codes of coordinates 16 c .. 16 c + 15 packed into the words of the cache
@@ -173,23 +203,25 @@ __device__ __forceinline__ uint32_t pack_offsets(const float *z, const float (&t
 // gathered into the nibbles of one word whose bit k of every nibble then
 // moves to bit 3 of word k.
 template <int B>
-__device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const float (&tp)[(1 << (B - 1)) - 1],
+__device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const CodeConsts<B> &k,
                                            uint32_t (&w)[4 * B]) {
   if constexpr (B == 3) {
     const int g = c >> 1;
+    const uint32_t x0 = join16(pack16<3, 4, 4>(z, k), pack16<3, 4, 4>(z + 4, k));
+    const uint32_t x1 = join16(pack16<3, 4, 4>(z + 8, k), pack16<3, 4, 4>(z + 12, k));
     if ((c & 1) == 0) {
-      w[3 * g] = pack_offsets<3, 8, 4>(z, tp);
-      w[3 * g + 1] = pack_offsets<3, 8, 4>(z + 8, tp);
+      w[3 * g] = x0;
+      w[3 * g + 1] = x1;
     } else {
-      const uint32_t sp = pack_offsets<3, 8, 4>(z + 8, tp);
-      w[3 * g] |= (sp << 3) & 0x88888888u;
-      w[3 * g + 1] |= (sp << 2) & 0x88888888u;
-      w[3 * g + 2] = pack_offsets<3, 8, 4>(z, tp) | ((sp << 1) & 0x88888888u);
+      w[3 * g] |= (x1 << 3) & 0x88888888u;
+      w[3 * g + 1] |= (x1 << 2) & 0x88888888u;
+      w[3 * g + 2] = x0 | ((x1 << 1) & 0x88888888u);
     }
+  } else if constexpr (B == 2) {
+    w[c] = join16(pack16<2, 8, 2>(z, k), pack16<2, 8, 2>(z + 8, k));
   } else {
-    constexpr int per = 32 / B;  // codes per word
-#pragma unroll
-    for (int k = 0; k < 16 / per; ++k) w[(16 / per) * c + k] = pack_offsets<B, per, B>(z + per * k, tp);
+    w[2 * c] = join16(pack16<4, 4, 4>(z, k), pack16<4, 4, 4>(z + 4, k));
+    w[2 * c + 1] = join16(pack16<4, 4, 4>(z + 8, k), pack16<4, 4, 4>(z + 12, k));
   }
 }
 
@@ -197,14 +229,17 @@ template <int B>
 __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], float n, uint32_t tmem_row,
                                              uint32_t (&words)[4 * B]) {
   constexpr int half = 1 << (B - 1);
-  float tp[half - 1];
+  CodeConsts<B> k;
+  const bool live = n > 0x1p-25f;  // stored fp16 norm nonzero
+  k.sc = live ? 0x1p64f / n : 0.f;
+  k.zc = live ? 0x1p127f : 0.f;
 #pragma unroll
-  for (int j = 0; j < half - 1; ++j) tp[j] = thr[half + j] * n;  // positive thresholds, scaled
+  for (int j = 0; j < half - 1; ++j) k.nt[j] = -thr[half + j] * 0x1p64f;  // positive thresholds x -2^64
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     float z[16];
     tmem_ld16(tmem_row + 16 * c, z);
-    code_chunk<B>(c, z, tp, words);
+    code_chunk<B>(c, z, k, words);
   }
 }
 
@@ -373,7 +408,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tc_fence_after();
       const uint32_t trow = tmem_base + g * 128 + ((uint32_t)(32 * quarter) << 16);
       uint32_t words[16];
-      if (is_k) {
+      if constexpr (BK == BV) {  // one copy of the epilogue code for K and V tiles
+        float thr[kMaxLevels];
+#pragma unroll
+        for (int e = 0; e < kMaxLevels; ++e) thr[e] = is_k ? tk[e] : tv[e];
+        uint32_t w[4 * BK];
+        epilogue_row<BK>(thr, nrm, trow, w);
+#pragma unroll
+        for (int e = 0; e < 4 * BK; ++e) words[e] = w[e];
+      } else if (is_k) {
         uint32_t w[4 * BK];
         epilogue_row<BK>(tk, nrm, trow, w);
 #pragma unroll

@@ -31,7 +31,8 @@ Readings where the pages are silent (each also listed in the design notes):
   centroids (representable in fp32); code = #{j : t_j < y}  (a value equal to
   a threshold goes to the lower cell).
 * every head vector x (bf16) is split into n = ||x||_2 and direction x/n;
-  y = (Pi x)/n with Pi the bf16-rounded rotation; n = 0 gives y = 0.
+  y = (Pi x)/n with Pi the bf16-rounded rotation; a vector whose stored fp16
+  norm is zero (n <= 2^-25) gives y = 0, as n = 0 does.
 * n is stored as fp16 (round to nearest even, saturating at 65504).
 * QJL (K only, optional): r = y - c[code] in rotated, unit-direction units,
   gamma = ||r|| stored as fp16, sign bit s_m = [(S r)_m >= 0] for the d rows
@@ -316,8 +317,11 @@ class Quantized:
 def quantize(x, pi, centroids, thresholds, s_matrix=None, chunk: int = 8192) -> Quantized:
     """Quantize rows of x ([N, d], the exact bf16 values as float64).
 
-    n = ||x||;  y = (Pi x) / n  (y = 0 when n = 0);  code_i = #{j : t_j < y_i};
-    stored norm = fp16(n).  With ``s_matrix``: r = y - c[code], gamma = ||r||
+    n = ||x||;  y = (Pi x) / n;  code_i = #{j : t_j < y_i};  stored norm =
+    fp16(n).  A vector whose stored norm is zero (n <= 2^-25, below half the
+    smallest fp16 subnormal) is stored as the zero vector: y = 0 (codes
+    2^(b-1) - 1), since its reconstruction fp16(n) Pi^T c[code] is zero
+    whatever the codes.  With ``s_matrix``: r = y - c[code], gamma = ||r||
     (stored as fp16), sign bit m = [(S r)_m >= 0].
     """
     x = np.asarray(x, dtype=np.float64)
@@ -327,16 +331,18 @@ def quantize(x, pi, centroids, thresholds, s_matrix=None, chunk: int = 8192) -> 
     codes = np.empty(x.shape, dtype=np.int64)
     ys = np.empty(x.shape, dtype=np.float64)
     norms = np.sqrt(np.sum(x * x, axis=1))
+    stored = round_to_fp16_sat(norms)
     for s0 in range(0, n_rows, chunk):
         xb = x[s0:s0 + chunk]
         nb = norms[s0:s0 + chunk]
+        live = stored[s0:s0 + chunk] > 0.0
         z = xb @ pi.T
-        safe = np.where(nb > 0.0, nb, 1.0)
-        y = np.where(nb[:, None] > 0.0, z / safe[:, None], 0.0)
+        safe = np.where(live, nb, 1.0)
+        y = np.where(live[:, None], z / safe[:, None], 0.0)
         ys[s0:s0 + chunk] = y
         # code = number of thresholds strictly below y
         codes[s0:s0 + chunk] = np.sum(y[:, :, None] > t[None, None, :], axis=2)
-    out = Quantized(codes, round_to_fp16_sat(norms), ys)
+    out = Quantized(codes, stored, ys)
     if s_matrix is not None:
         r = ys - c[codes]
         gamma = np.sqrt(np.sum(r * r, axis=1))

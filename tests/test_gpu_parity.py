@@ -51,7 +51,9 @@ def test_device_params_match_oracle(tq, bits_k, bits_v, qjl):
         assert np.array_equal(p["s"].double().numpy(), ref.s)
 
 
-def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0):
+def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0, scaled_rows=()):
+    """scaled_rows: (first token, last token, exponent) ranges whose rows are
+    multiplied by 2^exponent (exact in bf16)."""
     ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
     ref = oracle_params(bits_k, bits_v, qjl)
     k = make_rows(n_tok, n_heads, seed)
@@ -59,6 +61,9 @@ def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=
     if zero_rows:
         k[:zero_rows] = 0
         v[:zero_rows] = 0
+    for t0, t1, e in scaled_rows:
+        k[t0:t1] *= 2.0 ** e
+        v[t0:t1] *= 2.0 ** e
     g = torch.Generator().manual_seed(seed + 2)
     seq_idx = torch.randint(0, n_seqs, (n_tok,), generator=g, dtype=torch.int32)
     pos = torch.empty(n_tok, dtype=torch.int32)
@@ -111,6 +116,14 @@ def test_quantize_parity(tq, n_tok, n_heads, bits_k, bits_v, qjl):
 @pytest.mark.parametrize("n_tok", [40, 700])   # row kernel; tile kernels
 def test_quantize_zero_vectors(tq, n_tok):
     _quantize_and_compare(tq, n_tok, 2, 3, 3, 1, seed=5, zero_rows=9)
+
+
+@pytest.mark.parametrize("n_tok,bits,qjl", [(40, 3, 1), (700, 3, 1), (700, 2, 0), (700, 4, 0)])
+def test_quantize_tiny_and_small_norms(tq, n_tok, bits, qjl):
+    """Rows scaled by 2^-32 (stored fp16 norm 0: the zero vector) and by 2^-20
+    (fp16 subnormal norm: ordinary codes) through the row kernel (40 tokens)
+    and the tile kernels (700 tokens x 2 heads)."""
+    _quantize_and_compare(tq, n_tok, 2, bits, bits, qjl, seed=13, scaled_rows=((3, 9, -32), (9, 15, -20)))
 
 
 def test_quantize_mismatch_rate_at_scale(tq):

@@ -245,6 +245,32 @@ def test_quantize_zero_vector_and_threshold_tie():
     assert qz.codes[0, 0] == 6
 
 
+def test_quantize_codes_are_scale_invariant_until_the_stored_norm_vanishes():
+    """y = (Pi x)/||x|| does not depend on the scale of x, so exact power-of-two
+    scalings of x keep every code and QJL sign while the fp16 norm is nonzero
+    (fp16 subnormals reach down to 2^-24); once ||x|| <= 2^-25 the stored norm
+    is 0 and the vector is stored as the zero vector."""
+    d = 128
+    pi = o.rotation_bf16(d, 42)
+    s = o.qjl_matrix(d, 42)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((64, d))
+    x /= np.linalg.norm(x, axis=1)[:, None]
+    for bits in (2, 3, 4):
+        c, t = o.codebook(bits, d)
+        ref = o.quantize(x, pi, c, t, s_matrix=s)
+        for e in (-24, -10, 0, 10):            # stored norm 2^e > 0
+            q = o.quantize(x * 2.0 ** e, pi, c, t, s_matrix=s)
+            assert np.array_equal(q.codes, ref.codes) and np.array_equal(q.qjl_signs, ref.qjl_signs)
+            assert np.all(q.norm == 2.0 ** e)
+        for e in (-26, -40):                   # stored norm rounds to 0
+            q = o.quantize(x * 2.0 ** e, pi, c, t, s_matrix=s)
+            zero = o.quantize(np.zeros((1, d)), pi, c, t, s_matrix=s)
+            assert np.all(q.norm == 0.0)
+            assert np.all(q.codes == (1 << (bits - 1)) - 1)
+            assert np.array_equal(q.qjl_signs, np.repeat(zero.qjl_signs, len(x), axis=0))
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_quantize_distortion_on_unit_vectors(bits):
     """E||u - Pi^T c[code]||^2 over random unit vectors ~= D_b (Gaussian law
