@@ -90,3 +90,32 @@ def test_noalloc_rejects_workspace_beyond_static_scratch(tq):
     assert b"static scratch" in tq.lib.tq_last_error()
     torch.cuda.synchronize()
     assert bool((out == 7.0).all()) and bool((lse == 7.0).all())   # nothing was launched
+
+
+def test_noalloc_inside_cuda_graph_capture(tq):
+    """The point of the entry point: captured in a CUDA graph (no allocation,
+    no synchronisation inside the call), then replayed on new queries."""
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    n_heads, group = 2, 4
+    lens_all = [2500, 900]
+    cache, cap = _filled_cache(tq, ctx, lens_all, n_heads, seed=31)
+    seq_lens = torch.tensor(lens_all, dtype=torch.int32, device="cuda")
+    q = torch.zeros(len(lens_all), n_heads * group, D, device="cuda")
+    out = torch.empty(len(lens_all), n_heads * group, D, device="cuda")
+    lse = torch.empty(len(lens_all), n_heads * group, device="cuda")
+    assert _noalloc(tq, ctx, cache, q, seq_lens, cap, out, lse) == tq.TQ_OK   # first call outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        assert _noalloc(tq, ctx, cache, q, seq_lens, cap, out, lse) == tq.TQ_OK
+    g = torch.Generator().manual_seed(32)
+    ws = tq.alloc_workspace(ctx, len(lens_all), n_heads * group, cap)
+    for _ in range(2):
+        q.copy_(torch.randn(q.shape, generator=g))
+        graph.replay()
+        torch.cuda.synchronize()
+        out_ref = torch.empty_like(out)
+        lse_ref = torch.empty_like(lse)
+        tq.decode_attention(ctx, cache, q, seq_lens, cap, out_ref, lse_ref, ws)
+        ctx.check_device_errors()
+        _agree(out, lse, out_ref, lse_ref)
