@@ -349,8 +349,18 @@ def main(argv=None) -> int:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
+    # keep the GPU busy up to the timed region (clocks at their loaded level,
+    # and the clock sampler sees load): about 50 ms of warm-up replays, then
+    # the timed replay is queued behind them with no idle gap
+    wb0, wb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wb0.record()
+    g_warm.replay()
+    wb1.record()
+    torch.cuda.synchronize()
+    n_burst = max(1, min(2000, int(50.0 / max(wb0.elapsed_time(wb1), 1e-3))))
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(n_burst):
+        g_warm.replay()
     ev0.record()
     g_timed.replay()
     ev1.record()
