@@ -439,12 +439,33 @@ def main(argv=None) -> int:
     h2d = step_in
     d2h = out_h.numel() * 4
 
+    # A host application's loop: the C ABI called directly with its
+    # arguments prepared once, and the two copies as plain asynchronous
+    # driver copies on the same stream (one host-to-device, one back).
+    import ctypes
+    cu = ctypes.CDLL("libcuda.so.1")
+    cu.cuMemcpyHtoDAsync_v2.argtypes = [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    cu.cuMemcpyDtoHAsync_v2.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_void_p]
+    stream = torch.cuda.current_stream().cuda_stream
+    cache_refs = [ctypes.byref(c.struct) for c in caches]
+    in_ptrs = [host_in[i].data_ptr() for i in range(n_steps_total)]
+    pos_ptrs = [pos_steps[i].data_ptr() for i in range(n_steps_total)]
+    len_ptrs = [lens_steps[i].data_ptr() for i in range(n_steps_total)]
+    out_ptrs = [out[i].data_ptr() for i in range(n_steps_total)]
+    lse_ptrs = [lse[i].data_ptr() for i in range(n_steps_total)]
+    dev_ptr, k_ptr, v_ptr, q_ptr = dev_in.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), q_d.data_ptr()
+    seq_ptr, out_h_ptr, ws_ptr, ws_len = seq_ids.data_ptr(), out_h.data_ptr(), wsb.data_ptr(), wsb.numel()
+    handle, n_out = ctx.handle, out_h.numel() * 4
+
     def e2e_step(i):
-        c = caches[i % R]
-        dev_in.copy_(host_in[i], non_blocking=True)
-        tq.quantize(ctx, c, k_d, v_d, seq_ids, pos_steps[i])
-        tq.decode_attention(ctx, c, q_d, lens_steps[i], max_len, out[i], lse[i], wsb)
-        out_h.copy_(out[i], non_blocking=True)
+        c = cache_refs[i % R]
+        e = cu.cuMemcpyHtoDAsync_v2(dev_ptr, in_ptrs[i], step_in, stream)
+        e |= tq.lib.tq_quantize(handle, c, k_ptr, v_ptr, seq_ptr, pos_ptrs[i], B, stream)
+        e |= tq.lib.tq_decode_attention(handle, c, q_ptr, tq.TQ_BF16, HQ, len_ptrs[i], max_len, 0.0, out_ptrs[i],
+                                        lse_ptrs[i], ws_ptr, ws_len, stream)
+        e |= cu.cuMemcpyDtoHAsync_v2(out_h_ptr, out_ptrs[i], n_out, stream)
+        if e:
+            raise RuntimeError(f"e2e step {i} failed: {tq.lib.tq_last_error()}")
 
     for i in range(args.warmup):
         e2e_step(i)
