@@ -141,7 +141,30 @@ DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_p
   DecodeSplit sp;
   sp.chunk = (int)chunk;
   sp.n_splits = max_seq_len > 0 ? (int)(((long)max_seq_len + chunk - 1) / chunk) : 1;
+  sp.long_splits = false;
   return sp;
+}
+
+// The attention kernel has two register budgets.  With 128 registers (3 CTAs
+// per SM) twelve consumer warps per SM hide more latency; with 168 (2 CTAs per
+// SM, where the code needs more than 128) each CTA is longer and fewer CTAs
+// pay the per-CTA prologue.  Measured on the 3/3-bit kernel, the 3-CTA budget
+// wins when the split grid fills at least two waves (a batch of many
+// sequences) or a split streams at least kLongSplitTokens tokens; the 2-CTA
+// budget wins for one wave of short splits (one or a few sequences).
+constexpr int kLongSplitTokens = 8192;
+
+// The split is planned for the 3-CTA budget first; a call that meets neither
+// condition runs the 2-CTA budget instead, re-split for that occupancy.
+DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len) {
+  const int ctas = decode_ctas_per_sm(bits_k, bits_v, qjl, group, true);
+  DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len, ctas);
+  const long grid = (long)sp.n_splits * n_seqs * n_kv_heads;
+  if (grid >= 2L * sm_count() * ctas || sp.chunk >= kLongSplitTokens) {
+    sp.long_splits = true;
+    return sp;
+  }
+  return decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group, false));
 }
 
 tq_status report_error(tq_status st, const char *fmt, ...) {
@@ -316,8 +339,10 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->dp.bits_v = bits_v;
   ctx->dp.qjl = qjl;
   // resolve the decode kernels' occupancy now, outside any stream capture
-  tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8);
-  tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16);
+  for (const bool long_splits : {false, true}) {
+    tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8, long_splits);
+    tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16, long_splits);
+  }
   *out = ctx;
   return TQ_OK;
 }
@@ -399,8 +424,8 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
     return fail(TQ_ERR_INVALID, "misaligned q/out (16 B), workspace (256 B) or seq_lens/lse (4 B)");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
   const int group = n_q_heads / cache->n_kv_heads;
-  const int ctas = tq::decode_ctas_per_sm(ctx->bits_k, ctx->bits_v, ctx->qjl, group);
-  const tq::DecodeSplit sp = tq::decode_split(cache->n_seqs, cache->n_kv_heads, max_seq_len, ctas);
+  const tq::DecodeSplit sp =
+      tq::plan_decode(ctx->bits_k, ctx->bits_v, ctx->qjl, group, cache->n_seqs, cache->n_kv_heads, max_seq_len);
   const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, sp);
   if (workspace_bytes < ws.total)
     return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, ws.total);

@@ -261,8 +261,13 @@ struct DecodeArgs {
   float *partials;        // [rows][n_splits][d + 4]
 };
 
-template <int BK, int BV, bool QJL, int NT>
-__global__ void __maxnreg__(128) decode_mma_kernel(const DecodeArgs a) {
+// Two register budgets of the same kernel, chosen per call from the split
+// length (tq_api.cu): CTAS = 2 (168 registers) for short splits, where fewer
+// CTAs amortise the per-CTA prologue and each warp has room for more
+// independent work; CTAS = 3 (128 registers) for long splits, where twelve
+// consumer warps per SM hide more latency in the steady state.
+template <int BK, int BV, bool QJL, int NT, int CTAS>
+__global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const DecodeArgs a) {
   static_assert(kStageTokens % 64 == 0 && kWarpTokens == 32, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
   constexpr int kRows = 8 * NT;  // query-head rows of the score MMAs
@@ -916,11 +921,20 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
     const int sp = warp + 4 * e;
     if (sp < n_splits) o4[e] = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
   }
+  // and thread t's (m, l) pair of split t, so that the pairs of the first 128
+  // splits do not wait for the sequence length
+  float2 ml0 = make_float2(-INFINITY, 0.f);
+  if (tid < n_splits) ml0 = *reinterpret_cast<const float2 *>(src + tid * kPartialFloats);
   int len = seq_lens[s];
   len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
   const int used = min((len + chunk - 1) / chunk, kMergeMaxSplits);
   float mloc = -INFINITY;
-  for (int sp = tid; sp < used; sp += 128) {
+  if (tid < used) {
+    s_w[tid] = ml0.x;
+    s_l[tid] = ml0.y;
+    mloc = ml0.x;
+  }
+  for (int sp = tid + 128; sp < used; sp += 128) {
     const float2 ml = *reinterpret_cast<const float2 *>(src + sp * kPartialFloats);
     s_w[sp] = ml.x;
     s_l[sp] = ml.y;
@@ -977,52 +991,52 @@ constexpr int decode_smem_bytes() {
 
 using DecodeFn = void (*)(const DecodeArgs);
 
-template <int BK, int BV, bool QJL, int NT>
-DecodeFn pick_nt() {
-  return decode_mma_kernel<BK, BV, QJL, NT>;
-}
-
 struct Variant {
   DecodeFn fn;
   int smem;
 };
 
+template <int BK, int BV, bool QJL, int NT>
+Variant variant_c(bool long_splits) {
+  if (long_splits) return {decode_mma_kernel<BK, BV, QJL, NT, 3>, decode_smem_bytes<BK, BV, QJL, NT>()};
+  return {decode_mma_kernel<BK, BV, QJL, NT, 2>, decode_smem_bytes<BK, BV, QJL, NT>()};
+}
+
 template <int BK, int BV, bool QJL>
-Variant variant_q(int nt) {
-  if (nt == 1) return {decode_mma_kernel<BK, BV, QJL, 1>, decode_smem_bytes<BK, BV, QJL, 1>()};
-  return {decode_mma_kernel<BK, BV, QJL, 2>, decode_smem_bytes<BK, BV, QJL, 2>()};
+Variant variant_q(int nt, bool long_splits) {
+  return nt == 1 ? variant_c<BK, BV, QJL, 1>(long_splits) : variant_c<BK, BV, QJL, 2>(long_splits);
 }
 
 template <int BK, int BV>
-Variant variant_v(bool qjl, int nt) {
-  return qjl ? variant_q<BK, BV, true>(nt) : variant_q<BK, BV, false>(nt);
+Variant variant_v(bool qjl, int nt, bool long_splits) {
+  return qjl ? variant_q<BK, BV, true>(nt, long_splits) : variant_q<BK, BV, false>(nt, long_splits);
 }
 
 template <int BK>
-Variant variant_k(int bv, bool qjl, int nt) {
+Variant variant_k(int bv, bool qjl, int nt, bool long_splits) {
   switch (bv) {
-    case 2: return variant_v<BK, 2>(qjl, nt);
-    case 3: return variant_v<BK, 3>(qjl, nt);
-    default: return variant_v<BK, 4>(qjl, nt);
+    case 2: return variant_v<BK, 2>(qjl, nt, long_splits);
+    case 3: return variant_v<BK, 3>(qjl, nt, long_splits);
+    default: return variant_v<BK, 4>(qjl, nt, long_splits);
   }
 }
 
-Variant variant(int bk, int bv, bool qjl, int nt) {
+Variant variant(int bk, int bv, bool qjl, int nt, bool long_splits) {
   switch (bk) {
-    case 2: return variant_k<2>(bv, qjl, nt);
-    case 3: return variant_k<3>(bv, qjl, nt);
-    default: return variant_k<4>(bv, qjl, nt);
+    case 2: return variant_k<2>(bv, qjl, nt, long_splits);
+    case 3: return variant_k<3>(bv, qjl, nt, long_splits);
+    default: return variant_k<4>(bv, qjl, nt, long_splits);
   }
 }
 
 }  // namespace
 
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group) {
-  static int cache[5][5][2][3] = {};
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits) {
+  static int cache[5][5][2][3][2] = {};
   const int nt = group > 8 ? 2 : 1;
-  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt];
+  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt][long_splits ? 1 : 0];
   if (c == 0) {
-    const Variant v = variant(bits_k, bits_v, qjl != 0, nt);
+    const Variant v = variant(bits_k, bits_v, qjl != 0, nt, long_splits);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int n = 0;
@@ -1044,7 +1058,7 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
-  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1);
+  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1, split.long_splits);
   DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q, q_dtype, scale, partials};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(split.n_splits, c.n_kv_heads, c.n_seqs);

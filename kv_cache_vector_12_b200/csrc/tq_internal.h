@@ -64,11 +64,16 @@ void jperm_of(uint8_t *perm);
 
 // Split of the sequence axis used by decode attention.
 struct DecodeSplit {
-  int chunk;     // tokens per split (multiple of 64)
-  int n_splits;  // ceil(max_seq_len / chunk), at least 1
+  int chunk;         // tokens per split (multiple of 64)
+  int n_splits;      // ceil(max_seq_len / chunk), at least 1
+  bool long_splits;  // run the 3-CTA-per-SM register budget of the attention kernel
 };
 DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm);
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group);
+// CTAs per SM of the attention kernel for these bit widths and query heads per
+// KV head, with the long-split (128-register) or short-split (168) budget.
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits);
+// The split and register budget of one decode call (tq_api.cu).
+DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len);
 
 // Workspace layout of decode attention (byte offsets, 256-aligned): the split
 // partials [rows][splits][d+4] (m, l, two unused floats, then the d outputs,
