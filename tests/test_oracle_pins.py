@@ -6,6 +6,7 @@ chosen so that a plausible mistake (a dropped term, a wrong sign, an
 off-by-one index, a transposed operand) fails at least one of them.
 """
 import math
+from pathlib import Path
 
 import numpy as np
 import pytest
@@ -15,26 +16,31 @@ from scipy.stats import norm
 from oracle import turboquant_oracle as o
 
 
-# ---------------------------------------------------------------- codebook
-# Mean squared error of the optimal 2/4/8/16-level quantizer of N(0,1).
-# 1 bit: 1 - 2/pi in closed form.  2..4 bits: the values quoted with the
-# method (0.1175, 0.03455, 0.009497), which are Max's 1960 table values; the
-# table's 16-level figure is 0.04% below the exact optimum (0.0095010, found
-# here by closed form and by quadrature), so the tolerance is the printed
-# precision of the table (5e-4 relative).
-DISTORTION = {1: 0.3634, 2: 0.1175, 3: 0.03455, 4: 0.009497}
+GOLDEN = Path(__file__).parent / "golden"
 
-# Max (1960) / Jayant & Noll: positive half of the optimal Gaussian quantizer.
-MAX_CENTROIDS = {
-    2: [0.4528, 1.510],
-    3: [0.2451, 0.7560, 1.344, 2.152],
-    4: [0.1284, 0.3881, 0.6568, 0.9424, 1.256, 1.618, 2.069, 2.733],
-}
-MAX_THRESHOLDS = {
-    2: [0.0, 0.9816],
-    3: [0.0, 0.5006, 1.050, 1.748],
-    4: [0.0, 0.2582, 0.5224, 0.7996, 1.099, 1.437, 1.844, 2.401],
-}
+
+def _records(name):
+    """Non-comment lines of a golden fixture, split on whitespace."""
+    return [ln.split() for ln in (GOLDEN / name).read_text().splitlines() if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------- codebook
+# Max's 1960 table of the optimal Gaussian quantizer (golden fixture, with its
+# citation): mean squared error of the 2/4/8/16-level quantizer of N(0,1) and
+# the positive halves of its levels and thresholds.  The table's 16-level
+# error is 0.04% below the exact optimum (0.0095010, found here by closed form
+# and by quadrature), so the distortion tolerance is the printed precision of
+# the table (5e-4 relative).
+_MAX = _records("max1960_gaussian_quantizer.txt")
+DISTORTION = {int(r[0]): float(r[2]) for r in _MAX if r[1] == "distortion"}
+MAX_CENTROIDS = {int(r[0]): [float(v) for v in r[2:]] for r in _MAX if r[1] == "centroids"}
+MAX_THRESHOLDS = {int(r[0]): [float(v) for v in r[2:]] for r in _MAX if r[1] == "thresholds"}
+
+
+def test_golden_max_table_is_complete():
+    assert sorted(DISTORTION) == [1, 2, 3, 4]
+    for bits in (2, 3, 4):
+        assert len(MAX_CENTROIDS[bits]) == len(MAX_THRESHOLDS[bits]) == 2 ** (bits - 1)
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
@@ -114,10 +120,11 @@ def test_codebook_fp16_scaling():
 
 # ------------------------------------------------------------------- random
 def test_splitmix64_published_values():
-    # First outputs of the reference SplitMix64 for seeds 0 and 1234567.
-    assert o.splitmix64_output(0, 1) == 0xE220A8397B1DCDAF
-    assert [o.splitmix64_output(1234567, i) for i in (1, 2, 3)] == [
-        6457827717110365317, 3203168211198807973, 9817491932198370423]
+    # First outputs of the reference SplitMix64 (golden fixture, with its citation).
+    rec = _records("splitmix64_outputs.txt")
+    assert len(rec) == 4
+    for seed, n, want in rec:
+        assert o.splitmix64_output(int(seed), int(n)) == int(want)
 
 
 def test_splitmix64_counter_form_equals_sequential_generator():
