@@ -147,6 +147,37 @@ __device__ __forceinline__ float mul_sat(float a, float b) {
   return d;
 }
 
+// Two fp32 lanes in one 64-bit register pair: add, multiply and fused
+// multiply-add of both lanes in one instruction (f32x2, sm_100), round to
+// nearest like their scalar forms.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 // Per-row constants of the code computation.  A row whose stored fp16 norm is
 // zero (||x|| <= 2^-25) is the zero vector (y = 0): sc = zc = 0.  Otherwise
 // sc = 2^64 / ||x|| (at most 2^89), zc = 2^127, and nt_j = -t_j 2^64 for the
@@ -160,35 +191,44 @@ struct CodeConsts {
   float sc, zc, nt[(1 << (B - 1)) - 1];
 };
 
-// Offset from half - 1 of the code #{j : T_j < z} of one rotated coordinate,
-// exactly, as a float on the FMA pipe: m = #{j : t_j < |z| / ||x||},
-// p = [z > 0] (z zc 2^127 saturates to 1 for every positive float when
-// zc = 2^127, and to 0 otherwise), offset = p (2 m + 1) - m, i.e. m + 1 for
-// z > 0, -m otherwise.
+// Offsets from half - 1 of the codes #{j : T_j < z} of two rotated
+// coordinates, exactly, as floats on the FMA pipe: m = #{j : t_j < |z| / ||x||}
+// from one saturating test per positive threshold (per lane: the paired form
+// has no saturation), p = [z > 0] (z zc 2^127 saturates to 1 for every
+// positive float when zc = 2^127, and to 0 otherwise), and the offset
+// m (2 p - 1) + p, i.e. m + 1 for z > 0, -m otherwise; the sums and products
+// after the tests run on both lanes at once.
 template <int B>
-__device__ __forceinline__ float code_offset_f(float z, const CodeConsts<B> &k) {
+__device__ __forceinline__ float2 code_offset_f2(float z0, float z1, const CodeConsts<B> &k) {
   constexpr int half = 1 << (B - 1);
-  const float a = fabsf(z);
-  float m = fma_sat(a, k.sc, k.nt[0]);
+  const float a0 = fabsf(z0), a1 = fabsf(z1);
+  float2 m = make_float2(fma_sat(a0, k.sc, k.nt[0]), fma_sat(a1, k.sc, k.nt[0]));
 #pragma unroll
-  for (int j = 1; j < half - 1; ++j) m += fma_sat(a, k.sc, k.nt[j]);
-  const float p = mul_sat(z * k.zc, 0x1p127f);
-  return fmaf(p, fmaf(m, 2.f, 1.f), -m);
+  for (int j = 1; j < half - 1; ++j)
+    m = add2(m, make_float2(fma_sat(a0, k.sc, k.nt[j]), fma_sat(a1, k.sc, k.nt[j])));
+  const float2 s = mul2(make_float2(z0, z1), make_float2(k.zc, k.zc));
+  const float2 p = make_float2(mul_sat(s.x, 0x1p127f), mul_sat(s.y, 0x1p127f));
+  const float2 q = fma2(p, make_float2(2.f, 2.f), make_float2(-1.f, -1.f));
+  return fma2(m, q, p);
 }
 
 // 16 bits of codes (n codes of `bits` bits, LSB first): their offsets summed
-// at their positions in a float (exact: |sum| < 2^16), then half - 1 added to
-// every field and the integer read out of the mantissa of 2^23 + sum.
+// at their positions (even and odd codes in the two lanes, the even lane
+// starting from 2^23 + (half - 1) in every field), the lanes added, and the
+// integer read out of the mantissa.  Every partial sum is an integer below
+// 2^24, so all of it is exact.
 template <int B, int n, int bits>
 __device__ __forceinline__ uint32_t pack16(const float *z, const CodeConsts<B> &k) {
   constexpr int half_m1 = (1 << (B - 1)) - 1;
-  float acc = 0.f;
-#pragma unroll
-  for (int j = 0; j < n; ++j) acc = fmaf(code_offset_f<B>(z[j], k), (float)(1 << (bits * j)), acc);
   int ones = 0;
 #pragma unroll
   for (int j = 0; j < n; ++j) ones += 1 << (bits * j);
-  return __float_as_uint(acc + (8388608.f + (float)(half_m1 * ones))) & 0xFFFFu;
+  float2 acc = make_float2(8388608.f + (float)(half_m1 * ones), 0.f);
+#pragma unroll
+  for (int j = 0; j < n; j += 2)
+    acc = fma2(code_offset_f2<B>(z[j], z[j + 1], k),
+               make_float2((float)(1 << (bits * j)), (float)(1 << (bits * (j + 1)))), acc);
+  return __float_as_uint(acc.x + acc.y) & 0xFFFFu;
 }
 
 __device__ __forceinline__ uint32_t join16(uint32_t lo, uint32_t hi) {
@@ -381,7 +421,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // conflict-free, and the order does not matter to a sum of squares.  bf16
       // squares are exact in fp32.
       const unsigned char *st = ring + slot * kTileBytes;
-      float s0 = 0.f, s1 = 0.f;
+      float2 ss = make_float2(0.f, 0.f);  // sums of the squares of the low and the high halves
 #pragma unroll
       for (int box = 0; box < 2; ++box)
 #pragma unroll
@@ -391,12 +431,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
-            s0 = fmaf(lo, lo, s0);
-            s1 = fmaf(hi, hi, s1);
+            const float2 x = make_float2(__uint_as_float(w4[e] << 16), __uint_as_float(w4[e] & 0xffff0000u));
+            ss = fma2(x, x, ss);
           }
         }
-      const float nrm = sqrtf(s0 + s1);
+      const float nrm = sqrtf(ss.x + ss.y);
       __syncwarp();
       if (lane == 0) bar_arrive(smem_addr(&empty_bar[slot]));
 
