@@ -213,6 +213,11 @@ tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
   }
   if (s && qjl) tq::qjl_matrix(d, seed, s);
   float c[tq::kMaxLevels], t[tq::kMaxLevels];
+  for (const int b : {bits_k, bits_v}) {
+    tq::codebook(b, d, c, t);
+    if (!tq::threshold_search_exact(b, t))
+      return fail(TQ_ERR_UNSUPPORTED, "%d-bit thresholds: the quantize search is not exact in fp32", b);
+  }
   if (centroids_k || thresholds_k) {
     tq::codebook(bits_k, d, c, t);
     if (centroids_k) std::memcpy(centroids_k, c, sizeof(float) << bits_k);
@@ -248,6 +253,10 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->tv.assign(tq::kMaxLevels, 0.f);
   tq::codebook(bits_k, d, ctx->ck.data(), ctx->tk.data());
   tq::codebook(bits_v, d, ctx->cv.data(), ctx->tv.data());
+  if (!tq::threshold_search_exact(bits_k, ctx->tk.data()) || !tq::threshold_search_exact(bits_v, ctx->tv.data())) {
+    delete ctx;
+    return fail(TQ_ERR_UNSUPPORTED, "thresholds: the quantize search is not exact in fp32");
+  }
   if (qjl) {
     ctx->s.resize((size_t)d * d);
     tq::qjl_matrix(d, seed, ctx->s.data());

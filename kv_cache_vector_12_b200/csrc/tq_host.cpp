@@ -198,4 +198,31 @@ void codebook(int bits, int d, float *centroids, float *thresholds) {
     thresholds[j] = (float)(0.5 * ((double)centroids[j] + (double)centroids[j + 1]));
 }
 
+// The quantize kernel finds m = #{j : t_j < |y|} over the positive thresholds
+// by binary search, selecting each level's threshold (scaled by -2^64) with
+// fp32 fused multiply-adds from differences of the scaled thresholds.  That
+// is exact only if every difference and every selection is exact in fp32;
+// this replays the kernel's arithmetic for every path of the search.
+bool threshold_search_exact(int bits, const float *thresholds) {
+  const int half = 1 << (bits - 1);
+  float nt[kMaxLevels / 2];
+  for (int j = 0; j < half - 1; ++j) nt[j] = -thresholds[half + j] * 0x1p64f;
+  if (bits == 2) return true;
+  if (bits == 3) {
+    const float d20 = nt[2] - nt[0];
+    return std::fma(0.f, d20, nt[0]) == nt[0] && std::fma(1.f, d20, nt[0]) == nt[2];
+  }
+  if (bits != 4) return false;
+  const float d51 = nt[5] - nt[1], d40 = nt[4] - nt[0], d20 = nt[2] - nt[0];
+  const float ddd = (nt[6] - nt[4]) - d20;
+  for (int b2 = 0; b2 < 2; ++b2) {
+    if (std::fma((float)b2, d51, nt[1]) != nt[b2 ? 5 : 1]) return false;
+    const float base = std::fma((float)b2, d40, nt[0]);
+    const float step = std::fma((float)b2, ddd, d20);
+    for (int b1 = 0; b1 < 2; ++b1)
+      if (std::fma((float)b1, step, base) != nt[4 * b2 + 2 * b1]) return false;
+  }
+  return true;
+}
+
 }  // namespace tq

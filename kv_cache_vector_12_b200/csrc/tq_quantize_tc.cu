@@ -147,18 +147,9 @@ __device__ __forceinline__ float mul_sat(float a, float b) {
   return d;
 }
 
-// Two fp32 lanes in one 64-bit register pair: add, multiply and fused
-// multiply-add of both lanes in one instruction (f32x2, sm_100), round to
-// nearest like their scalar forms.
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  float2 d;
-  asm("{.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
+// Two fp32 lanes in one 64-bit register pair: multiply and fused multiply-add
+// of both lanes in one instruction (f32x2, sm_100), round to nearest like
+// their scalar forms.
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   float2 d;
   asm("{.reg .b64 ra, rb, rd;\n\t"
@@ -186,26 +177,67 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // product of two floats differs from a float by at least 2^-48 of it unless
 // equal), so the saturated result is exactly 0 or 1; the comparison differs
 // from |z| > t_j ||x|| only by the rounding of 2^64 / ||x||.
+//
+// m = #{j : t_j < |z| / ||x||} is found by binary search over the sorted nt_j,
+// one saturating test per level, the next level's threshold selected with
+// fused multiply-adds by the bits found so far (sel = b D + base).  The
+// differences D (below) are exact in fp32 for the codebooks in use, so every
+// selection yields one of the nt_j exactly; the host checks this for each
+// codebook before a context is created (threshold_search_exact).
+//   3 bits (t0 < t1 < t2): b1 = [> t1]; b0 = [> (b1 ? t2 : t0)]; m = 2 b1 + b0.
+//   4 bits (t0 .. t6):     b2 = [> t3]; b1 = [> (b2 ? t5 : t1)];
+//                          b0 = [> t(4 b2 + 2 b1)]; m = 4 b2 + 2 b1 + b0.
 template <int B>
 struct CodeConsts {
   float sc, zc, nt[(1 << (B - 1)) - 1];
+  float d20;                  // 3 bits: nt2 - nt0
+  float d51, d40, d20b, ddd;  // 4 bits: nt5 - nt1, nt4 - nt0, nt2 - nt0, (nt6 - nt4) - (nt2 - nt0)
 };
+
+template <int B>
+__device__ __forceinline__ void search_consts(CodeConsts<B> &k) {
+  if constexpr (B == 3) {
+    k.d20 = k.nt[2] - k.nt[0];
+  } else if constexpr (B == 4) {
+    k.d51 = k.nt[5] - k.nt[1];
+    k.d40 = k.nt[4] - k.nt[0];
+    k.d20b = k.nt[2] - k.nt[0];
+    k.ddd = (k.nt[6] - k.nt[4]) - k.d20b;
+  }
+}
+
+// m for two coordinates (|z| in a0, a1).
+template <int B>
+__device__ __forceinline__ float2 threshold_count2(float a0, float a1, const CodeConsts<B> &k) {
+  if constexpr (B == 2) {
+    return make_float2(fma_sat(a0, k.sc, k.nt[0]), fma_sat(a1, k.sc, k.nt[0]));
+  } else if constexpr (B == 3) {
+    const float2 b1 = make_float2(fma_sat(a0, k.sc, k.nt[1]), fma_sat(a1, k.sc, k.nt[1]));
+    const float2 sel = fma2(b1, make_float2(k.d20, k.d20), make_float2(k.nt[0], k.nt[0]));
+    const float2 b0 = make_float2(fma_sat(a0, k.sc, sel.x), fma_sat(a1, k.sc, sel.y));
+    return fma2(b1, make_float2(2.f, 2.f), b0);
+  } else {
+    const float2 b2 = make_float2(fma_sat(a0, k.sc, k.nt[3]), fma_sat(a1, k.sc, k.nt[3]));
+    const float2 sel1 = fma2(b2, make_float2(k.d51, k.d51), make_float2(k.nt[1], k.nt[1]));
+    const float2 b1 = make_float2(fma_sat(a0, k.sc, sel1.x), fma_sat(a1, k.sc, sel1.y));
+    const float2 base = fma2(b2, make_float2(k.d40, k.d40), make_float2(k.nt[0], k.nt[0]));
+    const float2 step = fma2(b2, make_float2(k.ddd, k.ddd), make_float2(k.d20b, k.d20b));
+    const float2 sel0 = fma2(b1, step, base);
+    const float2 b0 = make_float2(fma_sat(a0, k.sc, sel0.x), fma_sat(a1, k.sc, sel0.y));
+    return fma2(b2, make_float2(4.f, 4.f), fma2(b1, make_float2(2.f, 2.f), b0));
+  }
+}
 
 // Offsets from half - 1 of the codes #{j : T_j < z} of two rotated
 // coordinates, exactly, as floats on the FMA pipe: m = #{j : t_j < |z| / ||x||}
-// from one saturating test per positive threshold (per lane: the paired form
+// (threshold_count2; the saturating tests run per lane, as the paired form
 // has no saturation), p = [z > 0] (z zc 2^127 saturates to 1 for every
 // positive float when zc = 2^127, and to 0 otherwise), and the offset
 // m (2 p - 1) + p, i.e. m + 1 for z > 0, -m otherwise; the sums and products
 // after the tests run on both lanes at once.
 template <int B>
 __device__ __forceinline__ float2 code_offset_f2(float z0, float z1, const CodeConsts<B> &k) {
-  constexpr int half = 1 << (B - 1);
-  const float a0 = fabsf(z0), a1 = fabsf(z1);
-  float2 m = make_float2(fma_sat(a0, k.sc, k.nt[0]), fma_sat(a1, k.sc, k.nt[0]));
-#pragma unroll
-  for (int j = 1; j < half - 1; ++j)
-    m = add2(m, make_float2(fma_sat(a0, k.sc, k.nt[j]), fma_sat(a1, k.sc, k.nt[j])));
+  const float2 m = threshold_count2<B>(fabsf(z0), fabsf(z1), k);
   const float2 s = mul2(make_float2(z0, z1), make_float2(k.zc, k.zc));
   const float2 p = make_float2(mul_sat(s.x, 0x1p127f), mul_sat(s.y, 0x1p127f));
   const float2 q = fma2(p, make_float2(2.f, 2.f), make_float2(-1.f, -1.f));
@@ -275,6 +307,7 @@ __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], flo
   k.zc = live ? 0x1p127f : 0.f;
 #pragma unroll
   for (int j = 0; j < half - 1; ++j) k.nt[j] = -thr[half + j] * 0x1p64f;  // positive thresholds x -2^64
+  search_consts<B>(k);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     float z[16];
