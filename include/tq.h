@@ -100,7 +100,10 @@ typedef struct tq_cache {
  * counters 2^32+1.. (fp32).  Allocates and uploads the parameters
  * (synchronous); the only call that allocates device memory.
  * Errors: TQ_ERR_INVALID (null out, bits outside {2,3,4}, qjl outside {0,1}),
- * TQ_ERR_UNSUPPORTED (d != 128), TQ_ERR_NOMEM, TQ_ERR_CUDA.
+ * TQ_ERR_UNSUPPORTED (d != 128, or a codebook whose thresholds the quantize
+ * kernel's binary search could not select exactly in fp32; the host checks
+ * this, and it holds for every codebook of d = 128), TQ_ERR_NOMEM,
+ * TQ_ERR_CUDA.
  */
 tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v,
                     int32_t qjl, uint64_t seed);
@@ -125,7 +128,8 @@ tq_status tq_get_params(const tq_ctx *ctx, float *pi, float *s,
 /*
  * The same parameters computed on the host only (no CUDA call): what
  * tq_create(d, bits_k, bits_v, qjl, seed) would upload.  Same output layout
- * as tq_get_params; s is left untouched when qjl == 0.
+ * as tq_get_params; s is left untouched when qjl == 0.  Errors: those of
+ * tq_create's host checks (TQ_ERR_INVALID, TQ_ERR_UNSUPPORTED).
  */
 tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v,
                          int32_t qjl, uint64_t seed, float *pi, float *s,
