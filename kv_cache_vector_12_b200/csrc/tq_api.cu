@@ -4,6 +4,7 @@
 // problems are recorded in a sticky flag word instead of faulting.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -280,7 +281,7 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   const size_t dd = (size_t)d * d;
   const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_pif = off_piv + dd * 2;
   const size_t off_s = off_pif + dd * 2;
-  const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_cb = off_sf + 3 * dd * 2;
+  const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_cb = off_sf + 2 * dd * 2;
   const size_t off_kperm = off_cb + 4 * tq::kMaxLevels * 4, off_jperm = off_kperm + 256;
   const size_t off_err = off_jperm + 256, total = off_err + 256;
   e = cudaMalloc(&ctx->dev_block, total);
@@ -305,13 +306,20 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
     float *sjk = (float *)(h.data() + off_sjk);
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < d; ++j) sjk[(size_t)i * d + j] = ctx->s[(size_t)jperm[i] * d + kperm[j]];
-    // S = hi + mid + lo with three bf16 parts (exact: 24 significant bits)
+    // S 2^sigma = hi + lo with two fp16 parts (22 significant bits; only the
+    // signs of S r are kept, so the power-of-two scale is free).  sigma puts
+    // the largest entry at or below 2^15: hi never overflows, and lo stays in
+    // fp16's normal range for every entry above 2^-(sigma - 3).
+    double smax = 0.0;
+    for (size_t i = 0; i < dd; ++i) smax = std::max(smax, (double)std::fabs(ctx->s[i]));
+    const int sigma = smax > 0.0 ? (int)std::floor(std::log2(32768.0 / smax)) : 0;
     std::vector<uint16_t> part(dd);
-    std::vector<double> rest(ctx->s.begin(), ctx->s.end());
-    for (int k = 0; k < 3; ++k) {
+    std::vector<double> rest(dd);
+    for (size_t i = 0; i < dd; ++i) rest[i] = std::ldexp((double)ctx->s[i], sigma);
+    for (int k = 0; k < 2; ++k) {
       for (size_t i = 0; i < dd; ++i) {
-        part[i] = tq::double_to_bf16_bits(rest[i]);
-        rest[i] -= (double)tq::bf16_bits_to_float(part[i]);
+        part[i] = tq::double_to_half_bits(rest[i]);
+        rest[i] -= tq::half_bits_to_double(part[i]);
       }
       tq::mma_b_fragments(part.data(), (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
     }

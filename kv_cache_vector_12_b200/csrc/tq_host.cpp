@@ -51,6 +51,31 @@ void gaussian_stream(uint64_t seed, uint32_t stream, size_t count, double *out) 
 
 // Round a double to the nearest bfloat16 (ties to even) by clearing the 45
 // low mantissa bits of the double with carry; returns the bf16 bit pattern.
+// IEEE half bits of a double, rounded to nearest even, subnormals included;
+// magnitudes from 65520 up become infinity.
+uint16_t double_to_half_bits(double x) {
+  const uint16_t sign = std::signbit(x) ? 0x8000u : 0u;
+  const double a = std::fabs(x);
+  if (!(a < 65520.0)) return (uint16_t)(sign | 0x7C00u);
+  if (a < 0x1p-14) return (uint16_t)(sign | (uint16_t)std::nearbyint(a * 0x1p24));  // 1024 is the smallest normal
+  int e;
+  const double f = std::frexp(a, &e);         // a = f 2^e, f in [0.5, 1)
+  double m = std::nearbyint(f * 2048.0);      // 11 significant bits, 1024 .. 2048
+  if (m == 2048.0) {
+    m = 1024.0;
+    ++e;
+  }
+  const int biased = e - 1 + 15;
+  if (biased >= 31) return (uint16_t)(sign | 0x7C00u);
+  return (uint16_t)(sign | (biased << 10) | ((int)m - 1024));
+}
+
+double half_bits_to_double(uint16_t h) {
+  const int e = (h >> 10) & 0x1F, m = h & 0x3FF;
+  const double v = e == 0 ? std::ldexp((double)m, -24) : std::ldexp((double)(m + 1024), e - 25);
+  return (h & 0x8000u) ? -v : v;
+}
+
 uint16_t double_to_bf16_bits(double x) {
   uint64_t u;
   std::memcpy(&u, &x, 8);

@@ -21,6 +21,8 @@ constexpr unsigned kErrWaitExpired = 4u;
 void gaussian_stream(uint64_t seed, uint32_t stream, size_t count, double *out);
 uint16_t double_to_bf16_bits(double x);
 float bf16_bits_to_float(uint16_t h);
+uint16_t double_to_half_bits(double x);  // round to nearest even, subnormals kept
+double half_bits_to_double(uint16_t h);  // finite halves
 void rotation_bf16(int d, uint64_t seed, uint16_t *pi_bits);
 void qjl_matrix(int d, uint64_t seed, float *s);
 void lloyd_max_gaussian(int bits, double *c);
@@ -49,8 +51,8 @@ struct DeviceParams {
   const float *s;         // S   [d][d] fp32 (qjl only)
   const float *sjk;       // [d][d] fp32: sjk[kappa][kappa'] = S[jperm[kappa]][kperm[kappa']] (qjl only)
   const uint32_t *pif;    // Pi (natural row order) as bf16 MMA B fragments [n-tile 16][chunk 4][lane 32][4 words]
-  const uint32_t *sf;     // S split into three bf16 parts (S = hi + mid + lo), each as B fragments like pif:
-                          // [part 3][n-tile 16][chunk 4][lane 32][4 words] (qjl only)
+  const uint32_t *sf;     // S 2^sigma split into two fp16 parts (hi + lo), each as B fragments like pif:
+                          // [part 2][n-tile 16][chunk 4][lane 32][4 words] (qjl only; sigma chosen on the host)
   const float *cb;        // [4][16]: centroids_k, thresholds_k, centroids_v, thresholds_v
   unsigned *err;          // sticky error flags
   const uint8_t *kperm;   // [d] K fragment order -> coordinate

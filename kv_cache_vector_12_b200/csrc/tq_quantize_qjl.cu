@@ -14,11 +14,13 @@
 //   codes, y = z / ||x||, r = y - c[code], ||r||;
 //   S r            the residual goes from the accumulator fragments straight
 //                  into the A fragments of the second product (the k-steps
-//                  are the accumulators' column pairs); r and S are each split
-//                  into three bf16 parts (24 significant bits), and the six
-//                  products that matter give S r to fp32 precision, so its
-//                  signs agree with an fp32 dot product wherever |S r| is
-//                  above the rounding level;
+//                  are the accumulators' column pairs); r 2^14 and S 2^sigma
+//                  are each split into two fp16 parts (22 significant bits;
+//                  the power-of-two scales keep the low parts out of fp16's
+//                  subnormal range and do not change a sign), and the three
+//                  products hi hi, hi lo, lo hi give S r to within about
+//                  2^-21 of |S| |r|, so its signs agree with an fp32 dot
+//                  product wherever |S r| is above that level;
 //   store          packed codes, fp16 ||x||, sign bits (LSB first), fp16 ||r||.
 // Pi and S are read as coalesced B-fragment tables (built on the host),
 // 128 KB per 64 rows from L2, instead of 96 KB per row.
@@ -42,17 +44,26 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<const uint32_t *>(&v); }
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
-// x0, x1 (x0 in the low halves) as three bf16 pairs hi + mid + lo.
-__device__ __forceinline__ void split3(float x0, float x1, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  const float r0 = x0 - __low2float(h), r1 = x1 - __high2float(h);
-  const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(r0 - __low2float(m), r1 - __high2float(m));
-  hi = bf16x2_bits(h);
-  mid = bf16x2_bits(m);
-  lo = bf16x2_bits(l);
+__device__ __forceinline__ uint32_t half2_bits(__half2 v) { return *reinterpret_cast<const uint32_t *>(&v); }
+
+// Residuals r0, r1 (r0 in the low halves), scaled by 2^14, as two fp16 pairs
+// hi + lo.  |r| is below 1.3 (a coordinate of a unit direction minus a
+// centroid), so r 2^14 stays below fp16's largest finite value; hi + lo
+// differs from r 2^14 by at most 2^-22 |r| 2^14 + 2^-24 (lo's rounding, in
+// the normal or the subnormal range).
+constexpr float kResidualScale = 0x1p14f;
+__device__ __forceinline__ void split2(float r0, float r1, uint32_t &hi, uint32_t &lo) {
+  const float x0 = r0 * kResidualScale, x1 = r1 * kResidualScale;
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const __half2 l = __floats2half2_rn(x0 - __low2float(h), x1 - __high2float(h));
+  hi = half2_bits(h);
+  lo = half2_bits(l);
 }
 
 // Code #{j : T_j < z} of one coordinate against the positive thresholds tp
@@ -84,8 +95,10 @@ __device__ __forceinline__ uint32_t pack_word(const uint8_t *cd, int k) {
   return x;
 }
 
+// Four CTAs (16 warps) per SM: the register cap of 128 costs about 100 bytes
+// of spills and gains 9-23 % over three CTAs at 152 registers.
 template <int BK>
-__global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams p, tq_cache c,
+__global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DeviceParams p, tq_cache c,
                                                                     const uint16_t *__restrict__ k_in,
                                                                     const int32_t *__restrict__ seq_idx,
                                                                     const int32_t *__restrict__ pos, int n_rows) {
@@ -178,16 +191,16 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
 
   // ---- S r: A fragments of k-step j are the residual accumulators of
   // n-tiles 2 j (columns 16 j + 2 q ..) and 2 j + 1 (columns 16 j + 8 + 2 q ..)
-  uint32_t ah[8][4], am[8][4], al[8][4];
+  uint32_t ah[8][4], al[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    split3(z[2 * j][0], z[2 * j][1], ah[j][0], am[j][0], al[j][0]);
-    split3(z[2 * j][2], z[2 * j][3], ah[j][1], am[j][1], al[j][1]);
-    split3(z[2 * j + 1][0], z[2 * j + 1][1], ah[j][2], am[j][2], al[j][2]);
-    split3(z[2 * j + 1][2], z[2 * j + 1][3], ah[j][3], am[j][3], al[j][3]);
+    split2(z[2 * j][0], z[2 * j][1], ah[j][0], al[j][0]);
+    split2(z[2 * j][2], z[2 * j][3], ah[j][1], al[j][1]);
+    split2(z[2 * j + 1][0], z[2 * j + 1][1], ah[j][2], al[j][2]);
+    split2(z[2 * j + 1][2], z[2 * j + 1][3], ah[j][3], al[j][3]);
   }
   const uint4 *sfh = reinterpret_cast<const uint4 *>(p.sf);
-  const uint4 *sfm = sfh + kFragWords / 4, *sfl = sfm + kFragWords / 4;
+  const uint4 *sfl = sfh + kFragWords / 4;
   // projection m = 8 nt + 2 q (+1) is bit m of the row; a projection of exactly
   // 0 stores 1.  Two halves of 8 n-tiles: 8 independent accumulators between
   // consecutive MMAs.
@@ -204,19 +217,15 @@ __global__ void __launch_bounds__(32 * kWarps) quantize_qjl_kernel(DeviceParams 
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const int f = ((8 * hf + t) * 4 + j) * 32 + lane;
-        const uint4 h = sfh[f], m = sfm[f], l = sfl[f];
+        const uint4 h = sfh[f], l = sfl[f];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {  // k-steps 2 j and 2 j + 1
           const int ks = 2 * j + u;
           const uint32_t hb0 = u ? h.z : h.x, hb1 = u ? h.w : h.y;
-          const uint32_t mb0 = u ? m.z : m.x, mb1 = u ? m.w : m.y;
           const uint32_t lb0 = u ? l.z : l.x, lb1 = u ? l.w : l.y;
-          mma_bf16(acc[t], ah[ks], hb0, hb1);
-          mma_bf16(acc[t], ah[ks], mb0, mb1);
-          mma_bf16(acc[t], am[ks], hb0, hb1);
-          mma_bf16(acc[t], ah[ks], lb0, lb1);
-          mma_bf16(acc[t], al[ks], hb0, hb1);
-          mma_bf16(acc[t], am[ks], mb0, mb1);
+          mma_f16(acc[t], ah[ks], hb0, hb1);
+          mma_f16(acc[t], ah[ks], lb0, lb1);
+          mma_f16(acc[t], al[ks], hb0, hb1);
         }
       }
 #pragma unroll
