@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DevicePara
   const float nrm[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
   // a vector whose stored fp16 norm is zero (||x|| <= 2^-25) is the zero vector
   const bool live[2] = {nrm[0] > 0x1p-25f, nrm[1] > 0x1p-25f};
+  const float inv[2] = {live[0] ? 1.f / nrm[0] : 0.f, live[1] ? 1.f / nrm[1] : 0.f};
 
   // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8.
   // The n-tiles are the inner loop, so consecutive MMAs feed 16 independent
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DevicePara
       for (int u = 0; u < 2; ++u) {
         const float zz = live[hr] ? z[nt][2 * hr + u] : 0.f;
         code[u] = code_of<BK>(zz, tp[hr]);
-        const float y = live[hr] ? zz / nrm[hr] : 0.f;
+        const float y = zz * inv[hr];  // within an ulp of z / ||x||; only r and ||r|| use it
         const float res = y - s_cent[code[u]];
         z[nt][2 * hr + u] = res;
         gg[hr] = fmaf(res, res, gg[hr]);
