@@ -95,10 +95,12 @@ __device__ __forceinline__ uint32_t pack_word(const uint8_t *cd, int k) {
   return x;
 }
 
-// Four CTAs (16 warps) per SM: the register cap of 128 costs about 100 bytes
-// of spills and gains 9-23 % over three CTAs at 152 registers.
+// Persistent: each CTA stages the Pi and S fragment tables (96 KB) in shared
+// memory once, then takes 64-row tiles strided over the grid; two CTAs per SM.
+constexpr int kTabVec = kFragWords / 4;           // 16-byte vectors of one fragment table
+constexpr int kTabBytes = 3 * kTabVec * 16;       // Pi, S hi, S lo
 template <int BK>
-__global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DeviceParams p, tq_cache c,
+__global__ void __launch_bounds__(32 * kWarps, 2) quantize_qjl_kernel(DeviceParams p, tq_cache c,
                                                                     const uint16_t *__restrict__ k_in,
                                                                     const int32_t *__restrict__ seq_idx,
                                                                     const int32_t *__restrict__ pos, int n_rows) {
@@ -106,166 +108,176 @@ __global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DevicePara
   __shared__ __align__(16) uint8_t s_code[kRows][D + 4];  // rows padded by one bank
   __shared__ float s_cent[1 << BK];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = lane >> 2, q = lane & 3;
+  extern __shared__ __align__(16) uint4 s_tab[];             // [Pi | S hi | S lo] fragment tables
   // parameters (written long before) first, then wait for the previous kernel
   if (tid < (1 << BK)) s_cent[tid] = p.cb[tid];
   float thr[half - 1];
 #pragma unroll
   for (int j = 0; j < half - 1; ++j) thr[j] = p.cb[kMaxLevels + half + j];
+  {
+    const uint4 *gp = reinterpret_cast<const uint4 *>(p.pif), *gs = reinterpret_cast<const uint4 *>(p.sf);
+    for (int i = tid; i < kTabVec; i += 32 * kWarps) s_tab[i] = gp[i];
+    for (int i = tid; i < 2 * kTabVec; i += 32 * kWarps) s_tab[kTabVec + i] = gs[i];
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
 
-  const long row0 = (long)blockIdx.x * kRows + 16 * warp;
-  const long rows[2] = {row0 + r, row0 + r + 8};
-  // ---- X fragments (a0: row r, a1: row r + 8, a2 / a3: the same rows, columns + 8) and ||x||^2
-  uint32_t a[8][4];
-  float ss[2] = {0.f, 0.f};
+  const int n_tiles = (n_rows + kRows - 1) / kRows;
+  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const long row0 = (long)tile * kRows + 16 * warp;
+    const long rows[2] = {row0 + r, row0 + r + 8};
+    // ---- X fragments (a0: row r, a1: row r + 8, a2 / a3: the same rows, columns + 8) and ||x||^2
+    uint32_t a[8][4];
+    float ss[2] = {0.f, 0.f};
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks)
+    for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const long row = rows[e & 1];
-      const int col = 16 * ks + 8 * (e >> 1) + 2 * q;
-      const uint32_t w = row < n_rows ? *reinterpret_cast<const uint32_t *>(k_in + row * D + col) : 0u;
-      a[ks][e] = w;
-      const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
-      ss[e & 1] = fmaf(lo, lo, fmaf(hi, hi, ss[e & 1]));  // bf16 squares are exact in fp32
-    }
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], 1);
-    ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], 2);
-  }
-  const float nrm[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
-  // a vector whose stored fp16 norm is zero (||x|| <= 2^-25) is the zero vector
-  const bool live[2] = {nrm[0] > 0x1p-25f, nrm[1] > 0x1p-25f};
-  const float inv[2] = {live[0] ? 1.f / nrm[0] : 0.f, live[1] ? 1.f / nrm[1] : 0.f};
-
-  // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8.
-  // The n-tiles are the inner loop, so consecutive MMAs feed 16 independent
-  // accumulators.
-  float z[16][4];
-  const uint4 *pif = reinterpret_cast<const uint4 *>(p.pif);
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) z[nt][e] = 0.f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const uint4 v = pif[(nt * 4 + j) * 32 + lane];
-      mma_bf16(z[nt], a[2 * j], v.x, v.y);
-      mma_bf16(z[nt], a[2 * j + 1], v.z, v.w);
-    }
-
-  // ---- codes (to shared memory), residuals r = y - c[code], ||r||^2
-  float tp[2][half - 1];
-#pragma unroll
-  for (int j = 0; j < half - 1; ++j) {
-    tp[0][j] = thr[j] * nrm[0];
-    tp[1][j] = thr[j] * nrm[1];
-  }
-  float gg[2] = {0.f, 0.f};
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {  // 0: row r, 1: row r + 8; columns 8 nt + 2 q and + 1
-      int code[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float zz = live[hr] ? z[nt][2 * hr + u] : 0.f;
-        code[u] = code_of<BK>(zz, tp[hr]);
-        const float y = zz * inv[hr];  // within an ulp of z / ||x||; only r and ||r|| use it
-        const float res = y - s_cent[code[u]];
-        z[nt][2 * hr + u] = res;
-        gg[hr] = fmaf(res, res, gg[hr]);
+      for (int e = 0; e < 4; ++e) {
+        const long row = rows[e & 1];
+        const int col = 16 * ks + 8 * (e >> 1) + 2 * q;
+        const uint32_t w = row < n_rows ? *reinterpret_cast<const uint32_t *>(k_in + row * D + col) : 0u;
+        a[ks][e] = w;
+        const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+        ss[e & 1] = fmaf(lo, lo, fmaf(hi, hi, ss[e & 1]));  // bf16 squares are exact in fp32
       }
-      *reinterpret_cast<uint16_t *>(&s_code[16 * warp + r + 8 * hr][8 * nt + 2 * q]) =
-          (uint16_t)(code[0] | (code[1] << 8));
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], 1);
+      ss[e] += __shfl_xor_sync(0xffffffffu, ss[e], 2);
     }
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    gg[e] += __shfl_xor_sync(0xffffffffu, gg[e], 1);
-    gg[e] += __shfl_xor_sync(0xffffffffu, gg[e], 2);
-  }
+    const float nrm[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
+    // a vector whose stored fp16 norm is zero (||x|| <= 2^-25) is the zero vector
+    const bool live[2] = {nrm[0] > 0x1p-25f, nrm[1] > 0x1p-25f};
+    const float inv[2] = {live[0] ? 1.f / nrm[0] : 0.f, live[1] ? 1.f / nrm[1] : 0.f};
 
-  // ---- S r: A fragments of k-step j are the residual accumulators of
-  // n-tiles 2 j (columns 16 j + 2 q ..) and 2 j + 1 (columns 16 j + 8 + 2 q ..)
-  uint32_t ah[8][4], al[8][4];
+    // ---- z = X Pi^T: z[nt][0..1] = row r, columns 8 nt + 2 q (+1); [2..3] = row r + 8.
+    // The n-tiles are the inner loop, so consecutive MMAs feed 16 independent
+    // accumulators.
+    float z[16][4];
+    const uint4 *pif = s_tab;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    split2(z[2 * j][0], z[2 * j][1], ah[j][0], al[j][0]);
-    split2(z[2 * j][2], z[2 * j][3], ah[j][1], al[j][1]);
-    split2(z[2 * j + 1][0], z[2 * j + 1][1], ah[j][2], al[j][2]);
-    split2(z[2 * j + 1][2], z[2 * j + 1][3], ah[j][3], al[j][3]);
-  }
-  const uint4 *sfh = reinterpret_cast<const uint4 *>(p.sf);
-  const uint4 *sfl = sfh + kFragWords / 4;
-  // projection m = 8 nt + 2 q (+1) is bit m of the row; a projection of exactly
-  // 0 stores 1.  Two halves of 8 n-tiles: 8 independent accumulators between
-  // consecutive MMAs.
-  uint32_t sb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};  // sign bits of rows r, r + 8 (LSB first)
+    for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    float acc[8][4];
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+      for (int e = 0; e < 4; ++e) z[nt][e] = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int f = ((8 * hf + t) * 4 + j) * 32 + lane;
-        const uint4 h = sfh[f], l = sfl[f];
+      for (int nt = 0; nt < 16; ++nt) {
+        const uint4 v = pif[(nt * 4 + j) * 32 + lane];
+        mma_bf16(z[nt], a[2 * j], v.x, v.y);
+        mma_bf16(z[nt], a[2 * j + 1], v.z, v.w);
+      }
+
+    // ---- codes (to shared memory), residuals r = y - c[code], ||r||^2
+    float tp[2][half - 1];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {  // k-steps 2 j and 2 j + 1
-          const int ks = 2 * j + u;
-          const uint32_t hb0 = u ? h.z : h.x, hb1 = u ? h.w : h.y;
-          const uint32_t lb0 = u ? l.z : l.x, lb1 = u ? l.w : l.y;
-          mma_f16(acc[t], ah[ks], hb0, hb1);
-          mma_f16(acc[t], ah[ks], lb0, lb1);
-          mma_f16(acc[t], al[ks], hb0, hb1);
+    for (int j = 0; j < half - 1; ++j) {
+      tp[0][j] = thr[j] * nrm[0];
+      tp[1][j] = thr[j] * nrm[1];
+    }
+    float gg[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {  // 0: row r, 1: row r + 8; columns 8 nt + 2 q and + 1
+        int code[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float zz = live[hr] ? z[nt][2 * hr + u] : 0.f;
+          code[u] = code_of<BK>(zz, tp[hr]);
+          const float y = zz * inv[hr];  // within an ulp of z / ||x||; only r and ||r|| use it
+          const float res = y - s_cent[code[u]];
+          z[nt][2 * hr + u] = res;
+          gg[hr] = fmaf(res, res, gg[hr]);
         }
+        *reinterpret_cast<uint16_t *>(&s_code[16 * warp + r + 8 * hr][8 * nt + 2 * q]) =
+            (uint16_t)(code[0] | (code[1] << 8));
       }
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int nt = 8 * hf + t, sh = 8 * (nt & 3) + 2 * q;
-      sb[0][nt >> 2] |= ((acc[t][0] >= 0.f ? 1u : 0u) | (acc[t][1] >= 0.f ? 2u : 0u)) << sh;
-      sb[1][nt >> 2] |= ((acc[t][2] >= 0.f ? 1u : 0u) | (acc[t][3] >= 0.f ? 2u : 0u)) << sh;
+    for (int e = 0; e < 2; ++e) {
+      gg[e] += __shfl_xor_sync(0xffffffffu, gg[e], 1);
+      gg[e] += __shfl_xor_sync(0xffffffffu, gg[e], 2);
     }
-  }
-#pragma unroll
-  for (int e = 0; e < 2; ++e)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      sb[e][w] |= __shfl_xor_sync(0xffffffffu, sb[e][w], 1);
-      sb[e][w] |= __shfl_xor_sync(0xffffffffu, sb[e][w], 2);
-    }
-  __syncwarp();  // this warp's code rows are complete
 
-  // ---- stores: thread q of a quad packs code group q of its two rows
+    // ---- S r: A fragments of k-step j are the residual accumulators of
+    // n-tiles 2 j (columns 16 j + 2 q ..) and 2 j + 1 (columns 16 j + 8 + 2 q ..)
+    uint32_t ah[8][4], al[8][4];
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const long row = rows[e];
-    if (row >= n_rows) continue;
-    const int tok = (int)(row / c.n_kv_heads), h = (int)(row - (long)tok * c.n_kv_heads);
-    const int s = seq_idx[tok], ps = pos[tok];
-    if (!(s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity)) {
-      if (q == 0 && h == 0) atomicOr(p.err, kErrTokenRange);
-      continue;
+    for (int j = 0; j < 8; ++j) {
+      split2(z[2 * j][0], z[2 * j][1], ah[j][0], al[j][0]);
+      split2(z[2 * j][2], z[2 * j][3], ah[j][1], al[j][1]);
+      split2(z[2 * j + 1][0], z[2 * j + 1][1], ah[j][2], al[j][2]);
+      split2(z[2 * j + 1][2], z[2 * j + 1][3], ah[j][3], al[j][3]);
     }
-    const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
-    const uint8_t *cd = &s_code[16 * warp + r + 8 * e][32 * q];
-    uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + slot * (D * BK / 8)) + BK * q;
+    const uint4 *sfh = s_tab + kTabVec;
+    const uint4 *sfl = sfh + kTabVec;
+    // projection m = 8 nt + 2 q (+1) is bit m of the row; a projection of exactly
+    // 0 stores 1.  Two halves of 8 n-tiles: 8 independent accumulators between
+    // consecutive MMAs.
+    uint32_t sb[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};  // sign bits of rows r, r + 8 (LSB first)
 #pragma unroll
-    for (int k = 0; k < BK; ++k) dst[k] = pack_word<BK>(cd, k);
-    if (q == 0) {
-      reinterpret_cast<uint4 *>(c.qjl_bits + slot * (D / 8))[0] = make_uint4(sb[e][0], sb[e][1], sb[e][2], sb[e][3]);
-      c.norm_k[slot] = __half_as_ushort(__float2half_rn(fminf(nrm[e], 65504.f)));
-      c.qjl_norm[slot] = __half_as_ushort(__float2half_rn(fminf(sqrtf(gg[e]), 65504.f)));
+    for (int hf = 0; hf < 2; ++hf) {
+      float acc[8][4];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int f = ((8 * hf + t) * 4 + j) * 32 + lane;
+          const uint4 h = sfh[f], l = sfl[f];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {  // k-steps 2 j and 2 j + 1
+            const int ks = 2 * j + u;
+            const uint32_t hb0 = u ? h.z : h.x, hb1 = u ? h.w : h.y;
+            const uint32_t lb0 = u ? l.z : l.x, lb1 = u ? l.w : l.y;
+            mma_f16(acc[t], ah[ks], hb0, hb1);
+            mma_f16(acc[t], ah[ks], lb0, lb1);
+            mma_f16(acc[t], al[ks], hb0, hb1);
+          }
+        }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int nt = 8 * hf + t, sh = 8 * (nt & 3) + 2 * q;
+        sb[0][nt >> 2] |= ((acc[t][0] >= 0.f ? 1u : 0u) | (acc[t][1] >= 0.f ? 2u : 0u)) << sh;
+        sb[1][nt >> 2] |= ((acc[t][2] >= 0.f ? 1u : 0u) | (acc[t][3] >= 0.f ? 2u : 0u)) << sh;
+      }
     }
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        sb[e][w] |= __shfl_xor_sync(0xffffffffu, sb[e][w], 1);
+        sb[e][w] |= __shfl_xor_sync(0xffffffffu, sb[e][w], 2);
+      }
+    __syncwarp();  // this warp's code rows are complete
+
+    // ---- stores: thread q of a quad packs code group q of its two rows
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const long row = rows[e];
+      if (row >= n_rows) continue;
+      const int tok = (int)(row / c.n_kv_heads), h = (int)(row - (long)tok * c.n_kv_heads);
+      const int s = seq_idx[tok], ps = pos[tok];
+      if (!(s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity)) {
+        if (q == 0 && h == 0) atomicOr(p.err, kErrTokenRange);
+        continue;
+      }
+      const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
+      const uint8_t *cd = &s_code[16 * warp + r + 8 * e][32 * q];
+      uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + slot * (D * BK / 8)) + BK * q;
+#pragma unroll
+      for (int k = 0; k < BK; ++k) dst[k] = pack_word<BK>(cd, k);
+      if (q == 0) {
+        reinterpret_cast<uint4 *>(c.qjl_bits + slot * (D / 8))[0] = make_uint4(sb[e][0], sb[e][1], sb[e][2], sb[e][3]);
+        c.norm_k[slot] = __half_as_ushort(__float2half_rn(fminf(nrm[e], 65504.f)));
+        c.qjl_norm[slot] = __half_as_ushort(__float2half_rn(fminf(sqrtf(gg[e]), 65504.f)));
+      }
+    }
+    __syncwarp();  // this warp's code rows are read before the next tile writes them
   }
 }
 
@@ -273,22 +285,33 @@ __global__ void __launch_bounds__(32 * kWarps, 4) quantize_qjl_kernel(DevicePara
 
 int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                         const int32_t *pos, int n_tok, void *stream) {
+  using Fn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, int);
+  const Fn fn = p.bits_k == 2 ? quantize_qjl_kernel<2> : p.bits_k == 3 ? quantize_qjl_kernel<3> : quantize_qjl_kernel<4>;
+  static int slots[5] = {};  // resident CTAs on the device, per bit width
+  int &n_slots = slots[p.bits_k];
+  if (n_slots == 0) {
+    int dev = 0, n_sm = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kTabBytes);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 32 * kWarps, kTabBytes) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    n_slots = n_sm * per_sm;
+  }
   const long rows = (long)n_tok * c.n_kv_heads;
+  const long tiles = (rows + kRows - 1) / kRows;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((rows + kRows - 1) / kRows));
+  cfg.gridDim = dim3((unsigned)(tiles < n_slots ? tiles : n_slots));
   cfg.blockDim = dim3(32 * kWarps);
+  cfg.dynamicSmemBytes = kTabBytes;
   cfg.stream = (cudaStream_t)stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  const uint16_t *kk = static_cast<const uint16_t *>(k);
-  switch (p.bits_k) {
-    case 2: return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_kernel<2>, p, c, kk, seq_idx, pos, (int)rows);
-    case 3: return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_kernel<3>, p, c, kk, seq_idx, pos, (int)rows);
-    default: return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_kernel<4>, p, c, kk, seq_idx, pos, (int)rows);
-  }
+  return (int)cudaLaunchKernelEx(&cfg, fn, p, c, static_cast<const uint16_t *>(k), seq_idx, pos, (int)rows);
 }
 
 }  // namespace tq
