@@ -50,6 +50,21 @@ typedef enum tq_status {
 
 typedef enum tq_dtype { TQ_BF16 = 0, TQ_F32 = 1 } tq_dtype;
 
+/*
+ * Coordinate law the Lloyd-Max codebook is optimised for.  After the random
+ * rotation every coordinate of a unit direction follows one fixed law, which
+ * the method describes as close to Gaussian ("ステップ1: PolarQuant",
+ * ai-accelerate.xyz TurboQuant explainer).
+ *  TQ_LAW_GAUSSIAN  N(0, 1/d): Lloyd-Max centroids of N(0,1) / sqrt(d) (the
+ *                   default, and what tq_create uses).
+ *  TQ_LAW_SPHERE    the exact law of one coordinate of a uniform unit vector
+ *                   in R^d, density (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on
+ *                   (-1, 1), of which N(0, 1/d) is the large-d limit.
+ * Either way the centroids are rounded to fp16 and the thresholds are the
+ * exact midpoints; the kernels, layouts and the decode are the same.
+ */
+typedef enum tq_law { TQ_LAW_GAUSSIAN = 0, TQ_LAW_SPHERE = 1 } tq_law;
+
 /* Plane indices of tq_layout(). */
 enum {
   TQ_PLANE_CODES_K = 0,
@@ -108,6 +123,14 @@ typedef struct tq_cache {
 tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v,
                     int32_t qjl, uint64_t seed);
 
+/*
+ * tq_create with the codebook's coordinate law chosen (tq_law); law =
+ * TQ_LAW_GAUSSIAN is tq_create.  Errors: those of tq_create, and
+ * TQ_ERR_INVALID for a law outside tq_law.
+ */
+tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v,
+                       int32_t qjl, uint64_t seed, int32_t law);
+
 /* Free the context's device memory.  NULL is a no-op. */
 void tq_destroy(tq_ctx *ctx);
 
@@ -135,6 +158,13 @@ tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v,
                          int32_t qjl, uint64_t seed, float *pi, float *s,
                          float *centroids_k, float *thresholds_k,
                          float *centroids_v, float *thresholds_v);
+
+/* tq_host_params for tq_create_ex(d, bits_k, bits_v, qjl, seed, law). */
+tq_status tq_host_params_ex(int32_t d, int32_t bits_k, int32_t bits_v,
+                            int32_t qjl, uint64_t seed, int32_t law,
+                            float *pi, float *s,
+                            float *centroids_k, float *thresholds_k,
+                            float *centroids_v, float *thresholds_v);
 
 /*
  * Quantize-on-append ("ステップ1" and, with qjl, "ステップ2"): for each of

@@ -15,7 +15,7 @@
 
 struct tq_ctx {
   int device;
-  int d, bits_k, bits_v, qjl;
+  int d, bits_k, bits_v, qjl, law;
   uint64_t seed;
   std::vector<uint16_t> pi_bits;  // host copies of the uploaded parameters
   std::vector<float> s, ck, tk, cv, tv;
@@ -84,7 +84,9 @@ tq_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-tq_status check_params(int d, int bits_k, int bits_v, int qjl) {
+tq_status check_params(int d, int bits_k, int bits_v, int qjl, int law) {
+  if (law != TQ_LAW_GAUSSIAN && law != TQ_LAW_SPHERE)
+    return fail(TQ_ERR_INVALID, "law=%d must be TQ_LAW_GAUSSIAN (0) or TQ_LAW_SPHERE (1)", law);
   if (bits_k < 2 || bits_k > 4 || bits_v < 2 || bits_v > 4)
     return fail(TQ_ERR_INVALID, "bits_k=%d bits_v=%d: each must be 2, 3 or 4", bits_k, bits_v);
   if (qjl != 0 && qjl != 1) return fail(TQ_ERR_INVALID, "qjl=%d must be 0 or 1", qjl);
@@ -205,7 +207,14 @@ const char *tq_last_error(void) { return g_last_error; }
 tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl, uint64_t seed,
                          float *pi, float *s, float *centroids_k, float *thresholds_k,
                          float *centroids_v, float *thresholds_v) {
-  tq_status st = check_params(d, bits_k, bits_v, qjl);
+  return tq_host_params_ex(d, bits_k, bits_v, qjl, seed, TQ_LAW_GAUSSIAN, pi, s, centroids_k, thresholds_k,
+                           centroids_v, thresholds_v);
+}
+
+tq_status tq_host_params_ex(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl, uint64_t seed, int32_t law,
+                            float *pi, float *s, float *centroids_k, float *thresholds_k,
+                            float *centroids_v, float *thresholds_v) {
+  tq_status st = check_params(d, bits_k, bits_v, qjl, law);
   if (st != TQ_OK) return st;
   if (pi) {
     std::vector<uint16_t> bits((size_t)d * d);
@@ -215,17 +224,17 @@ tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
   if (s && qjl) tq::qjl_matrix(d, seed, s);
   float c[tq::kMaxLevels], t[tq::kMaxLevels];
   for (const int b : {bits_k, bits_v}) {
-    tq::codebook(b, d, c, t);
+    tq::codebook(b, d, law, c, t);
     if (!tq::threshold_search_exact(b, t))
       return fail(TQ_ERR_UNSUPPORTED, "%d-bit thresholds: the quantize search is not exact in fp32", b);
   }
   if (centroids_k || thresholds_k) {
-    tq::codebook(bits_k, d, c, t);
+    tq::codebook(bits_k, d, law, c, t);
     if (centroids_k) std::memcpy(centroids_k, c, sizeof(float) << bits_k);
     if (thresholds_k) std::memcpy(thresholds_k, t, sizeof(float) * ((1 << bits_k) - 1));
   }
   if (centroids_v || thresholds_v) {
-    tq::codebook(bits_v, d, c, t);
+    tq::codebook(bits_v, d, law, c, t);
     if (centroids_v) std::memcpy(centroids_v, c, sizeof(float) << bits_v);
     if (thresholds_v) std::memcpy(thresholds_v, t, sizeof(float) * ((1 << bits_v) - 1));
   }
@@ -234,9 +243,14 @@ tq_status tq_host_params(int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
 
 tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
                     uint64_t seed) {
+  return tq_create_ex(out, d, bits_k, bits_v, qjl, seed, TQ_LAW_GAUSSIAN);
+}
+
+tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int32_t qjl,
+                       uint64_t seed, int32_t law) {
   if (!out) return fail(TQ_ERR_INVALID, "out is NULL");
   *out = nullptr;
-  tq_status st = check_params(d, bits_k, bits_v, qjl);
+  tq_status st = check_params(d, bits_k, bits_v, qjl, law);
   if (st != TQ_OK) return st;
 
   tq_ctx *ctx = new tq_ctx();
@@ -244,6 +258,7 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->bits_k = bits_k;
   ctx->bits_v = bits_v;
   ctx->qjl = qjl;
+  ctx->law = law;
   ctx->seed = seed;
   ctx->dev_block = nullptr;
   ctx->pi_bits.resize((size_t)d * d);
@@ -252,8 +267,8 @@ tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, int
   ctx->tk.assign(tq::kMaxLevels, 0.f);
   ctx->cv.assign(tq::kMaxLevels, 0.f);
   ctx->tv.assign(tq::kMaxLevels, 0.f);
-  tq::codebook(bits_k, d, ctx->ck.data(), ctx->tk.data());
-  tq::codebook(bits_v, d, ctx->cv.data(), ctx->tv.data());
+  tq::codebook(bits_k, d, law, ctx->ck.data(), ctx->tk.data());
+  tq::codebook(bits_v, d, law, ctx->cv.data(), ctx->tv.data());
   if (!tq::threshold_search_exact(bits_k, ctx->tk.data()) || !tq::threshold_search_exact(bits_v, ctx->tv.data())) {
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "thresholds: the quantize search is not exact in fp32");

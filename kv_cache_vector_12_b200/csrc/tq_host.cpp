@@ -211,14 +211,102 @@ double round_to_half(double x) {
   return r;
 }
 
-// Codebook of `bits` bits for N(0, 1/d): Lloyd-Max centroids / sqrt(d)
-// rounded to fp16 (exact as fp32), thresholds at the exact midpoints.
-void codebook(int bits, int d, float *centroids, float *thresholds) {
+// Regularised incomplete beta function I_x(a, b), from its continued
+// fraction (DLMF 8.17.22) evaluated by the modified Lentz method, on the side
+// of (a + 1) / (a + b + 2) where the fraction converges fast
+// (I_x(a, b) = 1 - I_{1-x}(b, a) on the other side).
+static double incomplete_beta(double a, double b, double x) {
+  if (x <= 0.0) return 0.0;
+  if (x >= 1.0) return 1.0;
+  if (x > (a + 1.0) / (a + b + 2.0)) return 1.0 - incomplete_beta(b, a, 1.0 - x);
+  const double tiny = 1e-300;
+  const double log_front = a * std::log(x) + b * std::log1p(-x) -
+                           (std::lgamma(a) + std::lgamma(b) - std::lgamma(a + b));
+  // 1 / (1 + e1 / (1 + e2 / (1 + ...))) with
+  //   e_{2m+1} = -(a + m)(a + b + m) x / ((a + 2m)(a + 2m + 1)),
+  //   e_{2m}   =  m (b - m) x / ((a + 2m - 1)(a + 2m)).
+  double num = -(a + b) * x / (a + 1.0);  // e_1
+  double dd = 1.0 + num;
+  if (std::fabs(dd) < tiny) dd = tiny;
+  dd = 1.0 / dd;
+  double cc = 1.0, f = dd;
+  for (int m = 1; m < 10000; ++m) {
+    for (int odd = 0; odd < 2; ++odd) {
+      num = odd ? -(a + m) * (a + b + m) * x / ((a + 2.0 * m) * (a + 2.0 * m + 1.0))
+                : m * (b - m) * x / ((a + 2.0 * m - 1.0) * (a + 2.0 * m));
+      dd = 1.0 + num * dd;
+      if (std::fabs(dd) < tiny) dd = tiny;
+      cc = 1.0 + num / cc;
+      if (std::fabs(cc) < tiny) cc = tiny;
+      dd = 1.0 / dd;
+      f *= dd * cc;
+      if (odd && std::fabs(dd * cc - 1.0) < 1e-16) return std::exp(log_front) * f / a;
+    }
+  }
+  return std::exp(log_front) * f / a;
+}
+
+// The coordinate X of a uniform unit vector in R^d has the density
+// (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on (-1, 1): (X + 1) / 2 is
+// Beta(h, h) with h = (d - 1) / 2.  Mass of (lo, hi], on the side of zero
+// that avoids cancellation.
+static double sphere_mass(double lo, double hi, int d) {
+  const double h = 0.5 * (d - 1);
+  if (lo >= 0.0) return incomplete_beta(h, h, 0.5 * (1.0 - lo)) - incomplete_beta(h, h, 0.5 * (1.0 - hi));
+  return incomplete_beta(h, h, 0.5 * (1.0 + hi)) - incomplete_beta(h, h, 0.5 * (1.0 + lo));
+}
+
+// int_lo^hi x f(x) dx = ((1 - lo^2)^h - (1 - hi^2)^h) / (2 h B(1/2, h)).
+static double sphere_first_moment(double lo, double hi, int d) {
+  const double h = 0.5 * (d - 1);
+  const double beta_half_h = std::exp(std::lgamma(0.5) + std::lgamma(h) - std::lgamma(h + 0.5));
+  return (std::pow(1.0 - lo * lo, h) - std::pow(1.0 - hi * hi, h)) / (2.0 * h * beta_half_h);
+}
+
+// Lloyd-Max centroids of that law with 2^bits levels, ascending.  Starts from
+// the N(0, 1/d) centroids (its large-d limit) and alternates the two
+// optimality conditions until no centroid moves by more than 1e-15; then
+// symmetrises exactly.
+void lloyd_max_sphere(int bits, int d, double *c) {
+  const int L = 1 << bits;
+  lloyd_max_gaussian(bits, c);
+  const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
+  for (int j = 0; j < L; ++j) c[j] = std::fmax(-0.999, std::fmin(0.999, c[j] * inv_sqrt_d));
+  std::vector<double> t(L + 1), nc(L);
+  for (int it = 0; it < 2000000; ++it) {
+    t[0] = -1.0;
+    t[L] = 1.0;
+    for (int j = 1; j < L; ++j) t[j] = 0.5 * (c[j - 1] + c[j]);
+    double move = 0.0;
+    for (int j = 0; j < L; ++j) {
+      nc[j] = sphere_first_moment(t[j], t[j + 1], d) / sphere_mass(t[j], t[j + 1], d);
+      move = std::fmax(move, std::fabs(nc[j] - c[j]));
+    }
+    for (int j = 0; j < L; ++j) c[j] = nc[j];
+    if (move <= 1e-15) break;
+  }
+  for (int j = 0; j < L / 2; ++j) {
+    const double m = 0.5 * (c[L - 1 - j] - c[j]);
+    c[j] = -m;
+    c[L - 1 - j] = m;
+  }
+}
+
+// Codebook of `bits` bits, rounded to fp16 (exact as fp32), thresholds at the
+// exact midpoints.  TQ_LAW_GAUSSIAN: Lloyd-Max centroids of N(0,1) / sqrt(d),
+// for the N(0, 1/d) law; TQ_LAW_SPHERE: Lloyd-Max centroids of the exact
+// coordinate law of a unit vector in R^d.
+void codebook(int bits, int d, int law, float *centroids, float *thresholds) {
   const int L = 1 << bits;
   std::vector<double> c(L);
-  lloyd_max_gaussian(bits, c.data());
-  const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
-  for (int j = 0; j < L; ++j) centroids[j] = (float)round_to_half(c[j] * inv_sqrt_d);
+  if (law == TQ_LAW_SPHERE) {
+    lloyd_max_sphere(bits, d, c.data());
+  } else {
+    lloyd_max_gaussian(bits, c.data());
+    const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
+    for (int j = 0; j < L; ++j) c[j] *= inv_sqrt_d;
+  }
+  for (int j = 0; j < L; ++j) centroids[j] = (float)round_to_half(c[j]);
   for (int j = 0; j + 1 < L; ++j)
     thresholds[j] = (float)(0.5 * ((double)centroids[j] + (double)centroids[j + 1]));
 }

@@ -26,7 +26,8 @@ double half_bits_to_double(uint16_t h);  // finite halves
 void rotation_bf16(int d, uint64_t seed, uint16_t *pi_bits);
 void qjl_matrix(int d, uint64_t seed, float *s);
 void lloyd_max_gaussian(int bits, double *c);
-void codebook(int bits, int d, float *centroids, float *thresholds);
+void lloyd_max_sphere(int bits, int d, double *c);
+void codebook(int bits, int d, int law, float *centroids, float *thresholds);
 // Whether the quantize kernel's binary search over these thresholds selects
 // every threshold exactly in fp32 (tq_host.cpp).
 bool threshold_search_exact(int bits, const float *thresholds);

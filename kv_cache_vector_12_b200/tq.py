@@ -20,6 +20,8 @@ lib = ctypes.CDLL(_LIB_PATH)
 
 TQ_OK, TQ_ERR_INVALID, TQ_ERR_CUDA, TQ_ERR_NOMEM, TQ_ERR_UNSUPPORTED, TQ_ERR_DEVICE = range(6)
 TQ_BF16, TQ_F32 = 0, 1
+TQ_LAW_GAUSSIAN, TQ_LAW_SPHERE = 0, 1
+LAWS = {"gaussian": TQ_LAW_GAUSSIAN, "sphere": TQ_LAW_SPHERE}
 PLANES = ("codes_k", "norm_k", "qjl_bits", "qjl_norm", "codes_v", "norm_v")
 
 _vp = ctypes.c_void_p
@@ -35,6 +37,8 @@ class tq_cache(ctypes.Structure):
 
 lib.tq_create.argtypes = [ctypes.POINTER(_vp), _i32, _i32, _i32, _i32, ctypes.c_uint64]
 lib.tq_create.restype = ctypes.c_int
+lib.tq_create_ex.argtypes = [ctypes.POINTER(_vp), _i32, _i32, _i32, _i32, ctypes.c_uint64, _i32]
+lib.tq_create_ex.restype = ctypes.c_int
 lib.tq_destroy.argtypes = [_vp]
 lib.tq_destroy.restype = None
 lib.tq_layout.argtypes = [_vp, ctypes.POINTER(ctypes.c_size_t)]
@@ -43,6 +47,8 @@ lib.tq_get_params.argtypes = [_vp, _fp, _fp, _fp, _fp, _fp, _fp]
 lib.tq_get_params.restype = ctypes.c_int
 lib.tq_host_params.argtypes = [_i32, _i32, _i32, _i32, ctypes.c_uint64, _fp, _fp, _fp, _fp, _fp, _fp]
 lib.tq_host_params.restype = ctypes.c_int
+lib.tq_host_params_ex.argtypes = [_i32, _i32, _i32, _i32, ctypes.c_uint64, _i32, _fp, _fp, _fp, _fp, _fp, _fp]
+lib.tq_host_params_ex.restype = ctypes.c_int
 lib.tq_quantize.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _vp, _vp, _vp, _i32, _vp]
 lib.tq_quantize.restype = ctypes.c_int
 lib.tq_workspace_bytes.argtypes = [_vp, _i32, _i32, _i32]
@@ -90,14 +96,18 @@ def _fbuf(t: torch.Tensor | None):
     return None if t is None else ctypes.cast(t.data_ptr(), _fp)
 
 
-def host_params(d: int, bits_k: int, bits_v: int, qjl: int, seed: int) -> dict:
-    """tq_host_params: the parameters tq_create would upload (CPU only)."""
+def _law(law) -> int:
+    return LAWS[law] if isinstance(law, str) else int(law)
+
+
+def host_params(d: int, bits_k: int, bits_v: int, qjl: int, seed: int, law="gaussian") -> dict:
+    """tq_host_params_ex: the parameters tq_create_ex would upload (CPU only)."""
     out = {"pi": torch.empty(d * d), "s": torch.empty(d * d) if qjl else None,
            "centroids_k": torch.empty(1 << bits_k), "thresholds_k": torch.empty((1 << bits_k) - 1),
            "centroids_v": torch.empty(1 << bits_v), "thresholds_v": torch.empty((1 << bits_v) - 1)}
-    _check(lib.tq_host_params(d, bits_k, bits_v, qjl, seed, _fbuf(out["pi"]), _fbuf(out["s"]),
-                              _fbuf(out["centroids_k"]), _fbuf(out["thresholds_k"]),
-                              _fbuf(out["centroids_v"]), _fbuf(out["thresholds_v"])))
+    _check(lib.tq_host_params_ex(d, bits_k, bits_v, qjl, seed, _law(law), _fbuf(out["pi"]), _fbuf(out["s"]),
+                                 _fbuf(out["centroids_k"]), _fbuf(out["thresholds_k"]),
+                                 _fbuf(out["centroids_v"]), _fbuf(out["thresholds_v"])))
     out["pi"] = out["pi"].view(d, d)
     if qjl:
         out["s"] = out["s"].view(d, d)
@@ -105,13 +115,16 @@ def host_params(d: int, bits_k: int, bits_v: int, qjl: int, seed: int) -> dict:
 
 
 class Context:
-    """Owns one tq_ctx (tq_create / tq_destroy)."""
+    """Owns one tq_ctx (tq_create_ex / tq_destroy); law "gaussian" (the
+    default, as tq_create) or "sphere" (tq_law)."""
 
-    def __init__(self, d: int = 128, bits_k: int = 3, bits_v: int = 3, qjl: int = 0, seed: int = 42):
+    def __init__(self, d: int = 128, bits_k: int = 3, bits_v: int = 3, qjl: int = 0, seed: int = 42,
+                 law="gaussian"):
         h = _vp()
-        _check(lib.tq_create(ctypes.byref(h), d, bits_k, bits_v, int(qjl), seed))
+        _check(lib.tq_create_ex(ctypes.byref(h), d, bits_k, bits_v, int(qjl), seed, _law(law)))
         self.handle = h
         self.d, self.bits_k, self.bits_v, self.qjl, self.seed = d, bits_k, bits_v, int(qjl), seed
+        self.law = law
 
     def close(self) -> None:
         if self.handle:

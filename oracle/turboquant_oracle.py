@@ -223,11 +223,95 @@ def lloyd_max_distortion(centroids) -> float:
     return float(np.sum(per_cell))
 
 
-def codebook(bits: int, d: int):
-    """The method's codebook for N(0, 1/d): (centroids, thresholds) as float64.
-    Centroids are the N(0,1) Lloyd-Max centroids divided by sqrt(d), rounded
-    to fp16; thresholds are the exact midpoints of adjacent centroids."""
-    c = round_to_fp16_sat(lloyd_max_normal(bits) / math.sqrt(d))
+# --------------------------------------------------------------------------
+# Lloyd-Max scalar quantizer for the exact coordinate law of a unit vector
+# --------------------------------------------------------------------------
+# A coordinate X of a uniformly distributed unit vector in R^d has the density
+# f(x) = (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on (-1, 1), i.e. (X + 1)/2 is
+# Beta(a, a) with a = (d-1)/2; N(0, 1/d) is its large-d limit.  This is the
+# law the rotation makes every coordinate follow exactly (the pages call it
+# close to Gaussian); quantizing against it is the exact-law variant of the
+# codebook.
+def _sphere_mass(lo, hi, d: int):
+    """P(lo < X <= hi) for the coordinate law, taking the tail that avoids
+    cancellation."""
+    from scipy.special import betainc
+    a = 0.5 * (d - 1)
+    lo = np.asarray(lo, dtype=np.float64)
+    hi = np.asarray(hi, dtype=np.float64)
+    upper = betainc(a, a, 0.5 * (1.0 - lo)) - betainc(a, a, 0.5 * (1.0 - hi))
+    lower = betainc(a, a, 0.5 * (1.0 + hi)) - betainc(a, a, 0.5 * (1.0 + lo))
+    return np.where(lo >= 0.0, upper, lower)
+
+
+def _sphere_first_moment(lo, hi, d: int):
+    """int_lo^hi x f(x) dx = ((1 - lo^2)^a - (1 - hi^2)^a) / (2 a B(1/2, a)),
+    a = (d-1)/2, since d/dx (1 - x^2)^a = -2 a x (1 - x^2)^(a-1)."""
+    from scipy.special import beta
+    a = 0.5 * (d - 1)
+    lo = np.asarray(lo, dtype=np.float64)
+    hi = np.asarray(hi, dtype=np.float64)
+    return ((1.0 - lo * lo) ** a - (1.0 - hi * hi) ** a) / (2.0 * a * beta(0.5, a))
+
+
+def lloyd_max_sphere(bits: int, d: int, tol: float = 1e-15, max_iter: int = 2000000):
+    """Lloyd-Max centroids (ascending, float64) of the coordinate law of a
+    uniform unit vector in R^d, for 2**bits levels.
+
+    The same two optimality conditions as for N(0,1): thresholds at midpoints,
+    centroids at the conditional means int x f / int f of their cells.  Starts
+    from equiprobable cells; stops when no centroid moves by more than
+    ``tol``; symmetrised exactly.
+    """
+    from scipy.special import betaincinv
+    levels = 1 << bits
+    a = 0.5 * (d - 1)
+    t = 2.0 * betaincinv(a, a, np.arange(1, levels) / levels) - 1.0
+    c = None
+    for _ in range(max_iter):
+        lo = np.concatenate(([-1.0], t))
+        hi = np.concatenate((t, [1.0]))
+        c_new = _sphere_first_moment(lo, hi, d) / _sphere_mass(lo, hi, d)
+        t = 0.5 * (c_new[:-1] + c_new[1:])
+        if c is not None and np.max(np.abs(c_new - c)) <= tol:
+            c = c_new
+            break
+        c = c_new
+    return 0.5 * (c - c[::-1])
+
+
+def sphere_distortion(centroids, d: int) -> float:
+    """Mean squared error of the quantizer on the coordinate law, in closed
+    form: per cell, int (x - c)^2 f = M2 - 2 c M1 + c^2 P, where the second
+    moment uses x^2 (1 - x^2)^(a-1) = (1 - x^2)^(a-1) - (1 - x^2)^a, i.e.
+    M2 = P_d - (d-1)/d P_(d+2) with P_d the cell's mass under dimension d."""
+    c = np.asarray(centroids, dtype=np.float64)
+    t = thresholds_of(c)
+    lo = np.concatenate(([-1.0], t))
+    hi = np.concatenate((t, [1.0]))
+    mass = _sphere_mass(lo, hi, d)
+    m1 = _sphere_first_moment(lo, hi, d)
+    m2 = mass - (d - 1) / d * _sphere_mass(lo, hi, d + 2)
+    return float(np.sum(m2 - 2.0 * c * m1 + c * c * mass))
+
+
+LAW_GAUSSIAN, LAW_SPHERE = "gaussian", "sphere"
+
+
+def codebook(bits: int, d: int, law: str = LAW_GAUSSIAN):
+    """The method's codebook: (centroids, thresholds) as float64.
+
+    law "gaussian" (the reading the build defaults to): the N(0,1) Lloyd-Max
+    centroids divided by sqrt(d), for the N(0, 1/d) law.  law "sphere": the
+    Lloyd-Max centroids of the exact coordinate law of a unit vector in R^d.
+    Centroids are rounded to fp16; thresholds are the exact midpoints of
+    adjacent centroids."""
+    if law == LAW_GAUSSIAN:
+        c = round_to_fp16_sat(lloyd_max_normal(bits) / math.sqrt(d))
+    elif law == LAW_SPHERE:
+        c = round_to_fp16_sat(lloyd_max_sphere(bits, d))
+    else:
+        raise ValueError(f"unknown codebook law {law!r}")
     t = 0.5 * (c[:-1] + c[1:])
     return c, t
 
@@ -417,9 +501,10 @@ class Params:
     """Everything tq_create(d, bits_k, bits_v, qjl, seed) fixes, computed here
     independently of the library."""
 
-    def __init__(self, d: int, bits_k: int, bits_v: int, qjl: bool, seed: int):
+    def __init__(self, d: int, bits_k: int, bits_v: int, qjl: bool, seed: int, law: str = LAW_GAUSSIAN):
         self.d, self.bits_k, self.bits_v, self.qjl, self.seed = d, bits_k, bits_v, bool(qjl), seed
+        self.law = law
         self.pi = rotation_bf16(d, seed)
-        self.ck, self.tk = codebook(bits_k, d)
-        self.cv, self.tv = codebook(bits_v, d)
+        self.ck, self.tk = codebook(bits_k, d, law)
+        self.cv, self.tv = codebook(bits_v, d, law)
         self.s = qjl_matrix(d, seed) if qjl else None

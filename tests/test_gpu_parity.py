@@ -24,10 +24,10 @@ def tq(cuda_device):
 _PARAMS = {}
 
 
-def oracle_params(bits_k, bits_v, qjl, seed=42):
-    key = (bits_k, bits_v, qjl, seed)
+def oracle_params(bits_k, bits_v, qjl, seed=42, law=o.LAW_GAUSSIAN):
+    key = (bits_k, bits_v, qjl, seed, law)
     if key not in _PARAMS:
-        _PARAMS[key] = o.Params(D, bits_k, bits_v, bool(qjl), seed)
+        _PARAMS[key] = o.Params(D, bits_k, bits_v, bool(qjl), seed, law)
     return _PARAMS[key]
 
 
@@ -51,11 +51,12 @@ def test_device_params_match_oracle(tq, bits_k, bits_v, qjl):
         assert np.array_equal(p["s"].double().numpy(), ref.s)
 
 
-def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0, scaled_rows=()):
+def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0, scaled_rows=(),
+                          law=o.LAW_GAUSSIAN):
     """scaled_rows: (first token, last token, exponent) ranges whose rows are
     multiplied by 2^exponent (exact in bf16)."""
-    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
-    ref = oracle_params(bits_k, bits_v, qjl)
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42, law=law)
+    ref = oracle_params(bits_k, bits_v, qjl, law=law)
     k = make_rows(n_tok, n_heads, seed)
     v = make_rows(n_tok, n_heads, seed + 1)
     if zero_rows:
@@ -220,9 +221,9 @@ def _upload(tq, ctx, planes, n_seqs, n_heads, cap):
 
 
 def _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed, q_dtype=torch.float32,
-                        scale=0.0, max_seq_len=None):
-    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
-    ref = oracle_params(bits_k, bits_v, qjl)
+                        scale=0.0, max_seq_len=None, law=o.LAW_GAUSSIAN):
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42, law=law)
+    ref = oracle_params(bits_k, bits_v, qjl, law=law)
     per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, min_cap=max_seq_len or 0)
     cache = _upload(tq, ctx, planes, len(lens), n_heads, cap)
     n_q = n_heads * group
@@ -267,6 +268,27 @@ def test_decode_parity_on_oracle_packed_cache(tq, lens, n_heads, group, bits_k, 
 def test_decode_bf16_queries_explicit_scale_and_loose_bound(tq):
     _decode_and_compare(tq, [300, 77], 2, 4, 3, 3, 0, seed=3, q_dtype=torch.bfloat16, scale=0.05,
                         max_seq_len=640)
+
+
+# The exact-law (sphere) codebook: same kernels, different tables.
+@pytest.mark.parametrize("bits_k,bits_v,qjl", [(3, 3, 0), (2, 4, 1), (4, 2, 0)])
+@pytest.mark.parametrize("n_tok,n_heads", [(129, 2), (1031, 3)])
+def test_quantize_parity_sphere_codebook(tq, n_tok, n_heads, bits_k, bits_v, qjl):
+    _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed=n_tok * 17 + n_heads, law=o.LAW_SPHERE)
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl", [(3, 3, 0), (2, 4, 1), (4, 4, 1)])
+def test_decode_parity_sphere_codebook(tq, bits_k, bits_v, qjl):
+    _decode_and_compare(tq, [1000, 0, 513], 2, 8, bits_k, bits_v, qjl, seed=21, law=o.LAW_SPHERE)
+
+
+def test_sphere_device_params_match_oracle(tq):
+    for bits in (2, 3, 4):
+        ctx = tq.Context(D, bits, bits, 0, 42, law="sphere")
+        p = ctx.params()
+        ref = oracle_params(bits, bits, 0, law=o.LAW_SPHERE)
+        assert np.array_equal(p["centroids_k"].double().numpy(), ref.ck)
+        assert np.array_equal(p["thresholds_v"].double().numpy(), ref.tv)
 
 
 def test_decode_long_sequence_many_splits(tq):

@@ -118,6 +118,87 @@ def test_codebook_fp16_scaling():
         assert abs(dist / o.lloyd_max_distortion(o.lloyd_max_normal(bits)) - 1) < 1e-5
 
 
+# ------------------------------------------- codebook for the exact law (sphere)
+# One coordinate of a uniform unit vector in R^d has the density
+# (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on (-1, 1).  The pins below use plain
+# quadrature of that density, closed forms of special cases, the large-d
+# limit and sampled unit vectors: none of them uses the incomplete beta
+# function the oracle's iteration uses.
+def _sphere_pdf(d):
+    from scipy.special import gammaln
+    logc = gammaln(0.5 * d) - gammaln(0.5) - gammaln(0.5 * (d - 1))   # 1 / B(1/2, (d-1)/2)
+    return lambda x: math.exp(logc + 0.5 * (d - 3) * math.log1p(-x * x)) if abs(x) < 1 else 0.0
+
+
+def test_sphere_density_normalised_and_d3_is_uniform():
+    for d in (3, 16, 128):
+        f = _sphere_pdf(d)
+        assert abs(integrate.quad(f, -1, 1, epsabs=1e-14, points=[0.0])[0] - 1) < 1e-10
+    # d = 3: the coordinate is uniform on [-1, 1] (Archimedes), so the optimal
+    # L-level quantizer has equal cells: c_j = -1 + (2 j + 1) / L and MSE 1 / (3 L^2)
+    for bits in (1, 2, 3, 4):
+        levels = 1 << bits
+        c = o.lloyd_max_sphere(bits, 3)
+        assert np.allclose(c, -1 + (2 * np.arange(levels) + 1) / levels, atol=1e-12)
+        assert abs(o.sphere_distortion(c, 3) - 1 / (3 * levels ** 2)) < 1e-12
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_sphere_centroid_and_nearest_neighbour_conditions_by_quadrature(bits):
+    d = 128
+    f = _sphere_pdf(d)
+    c = o.lloyd_max_sphere(bits, d)
+    assert np.array_equal(c, -c[::-1]) and np.all(np.diff(c) > 0)
+    t = o.thresholds_of(c)
+    edges = np.concatenate(([-1.0], t, [1.0]))
+    total = 0.0
+    for j, cj in enumerate(c):
+        lo, hi = edges[j], edges[j + 1]
+        mass = integrate.quad(f, lo, hi, epsabs=1e-15, epsrel=1e-13, limit=200)[0]
+        mean = integrate.quad(lambda x: x * f(x), lo, hi, epsabs=1e-15, epsrel=1e-13, limit=200)[0] / mass
+        assert abs(mean - cj) < 1e-11
+        total += integrate.quad(lambda x: (x - cj) ** 2 * f(x), lo, hi, epsabs=1e-16, epsrel=1e-12, limit=200)[0]
+    assert abs(total - o.sphere_distortion(c, d)) < 1e-13
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_sphere_codebook_tends_to_the_gaussian_one(bits):
+    """N(0, 1/d) is the large-d limit of the coordinate law: sqrt(d) times the
+    exact-law centroids approach the N(0,1) ones at rate 1/d."""
+    g = o.lloyd_max_normal(bits)
+    gaps = [np.max(np.abs(o.lloyd_max_sphere(bits, d) * math.sqrt(d) - g)) for d in (128, 1024)]
+    assert gaps[1] < 0.01
+    assert 6 < gaps[0] / gaps[1] < 10   # about 1024 / 128 = 8
+
+
+def test_sphere_codebook_on_sampled_unit_vectors():
+    """On the coordinates of sampled unit vectors, the closed-form MSE of a
+    codebook under the exact law matches the sampled MSE (checked for the
+    exact-law codebook and for the N(0, 1/d) one), and the exact-law codebook
+    has the lower closed-form MSE (it is the optimum for that law)."""
+    d, bits = 128, 3
+    rng = np.random.default_rng(2024)
+    x = rng.standard_normal((20000, d))
+    y = (x / np.linalg.norm(x, axis=1, keepdims=True)).ravel()
+    cs = o.lloyd_max_sphere(bits, d)
+    cg = o.lloyd_max_normal(bits) / math.sqrt(d)
+    for c in (cs, cg):
+        t = o.thresholds_of(c)
+        e = (y - c[np.searchsorted(t, y, side="left")]) ** 2
+        assert abs(e.mean() - o.sphere_distortion(c, d)) < 5 * e.std() / math.sqrt(y.size)
+    assert o.sphere_distortion(cs, d) < o.sphere_distortion(cg, d)
+
+
+def test_codebook_laws():
+    for bits in (2, 3, 4):
+        c, t = o.codebook(bits, 128, o.LAW_SPHERE)
+        assert np.array_equal(c, c.astype(np.float16).astype(np.float64))
+        assert np.array_equal(2 * t, c[:-1] + c[1:])
+        assert np.allclose(c, o.lloyd_max_sphere(bits, 128), rtol=2 ** -11)
+    with pytest.raises(ValueError):
+        o.codebook(3, 128, "cauchy")
+
+
 # ------------------------------------------------------------------- random
 def test_splitmix64_published_values():
     # First outputs of the reference SplitMix64 (golden fixture, with its citation).
