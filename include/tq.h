@@ -107,12 +107,13 @@ typedef struct tq_cache {
 /*
  * Create a context on the current CUDA device.  Pi is the QR factor of a
  * d x d Gaussian (SplitMix64 counters 1.. from `seed`, Box-Muller), columns
- * signed so that R has a positive diagonal, rounded to bf16 (the "random
- * orthogonal matrix" of "ステップ1: PolarQuant").  The codebook of b bits is
- * the Lloyd-Max quantizer of N(0,1) scaled by 1/sqrt(d) ("Lloyd-Max量子化";
- * the N(0,1/d) law is the "ガウス分布に近い" coordinate law), its centroids
- * rounded to fp16 and the exact midpoints (fp32) as thresholds.  With qjl, S is a second d x d Gaussian from
- * counters 2^32+1.. (fp32).  Allocates and uploads the parameters
+ * signed so that R has a positive diagonal, rounded to bf16 (the random
+ * orthogonal matrix of section "ステップ1: PolarQuant").  The codebook of b
+ * bits is the Lloyd-Max quantizer of N(0,1) scaled by 1/sqrt(d) (the same
+ * section's optimal scalar quantizer, for the N(0,1/d) reading of its
+ * near-Gaussian coordinate law), its centroids rounded to fp16 and the exact
+ * midpoints (fp32) as thresholds.  With qjl, S is a second d x d Gaussian
+ * from counters 2^32+1.. (fp32).  Allocates and uploads the parameters
  * (synchronous); the only call that allocates device memory.
  * Errors: TQ_ERR_INVALID (null out, bits outside {2,3,4}, qjl outside {0,1}),
  * TQ_ERR_UNSUPPORTED (d != 128, or a codebook whose thresholds the quantize

@@ -1,16 +1,18 @@
 // Host-side construction of the method's fixed parameters: the rotation Pi,
 // the QJL projection S and the Lloyd-Max codebooks.
 //
-// Rotation: "ランダムな直交行列を掛けて「回転」" (ai-accelerate.xyz TurboQuant
-// explainer, "ステップ1: PolarQuant").  Pi is the Q factor of a seeded
-// Gaussian matrix, made unique by a positive diagonal of R, then rounded to
-// bf16: the bf16 matrix is the one both quantize and decode use.
+// Rotation: the first step of the method multiplies every vector by a random
+// orthogonal matrix (ai-accelerate.xyz TurboQuant explainer, section
+// "ステップ1: PolarQuant").  Pi is the Q factor of a seeded Gaussian matrix,
+// made unique by a positive diagonal of R, then rounded to bf16: the bf16
+// matrix is the one both quantize and decode use.
 //
-// Codebook: "各次元を独立に最適なスカラー量子化（Lloyd-Max量子化）" (same
-// section).  Lloyd's iteration on N(0,1), scaled by 1/sqrt(d) for the
-// N(0,1/d) law of a rotated unit vector's coordinates, held in fp16 (the
-// pages fix no precision; fp16 costs < 1e-5 of the distortion and makes every
-// centroid an exact tensor-core operand).
+// Codebook: the same section quantizes each coordinate on its own with the
+// optimal (Lloyd-Max) scalar quantizer.  Lloyd's iteration on N(0,1), scaled
+// by 1/sqrt(d) for the N(0,1/d) law of a rotated unit vector's coordinates
+// (or, as a variant, on the exact law of one coordinate of a unit vector),
+// held in fp16 (the pages fix no precision; fp16 costs < 1e-5 of the
+// distortion and makes every centroid an exact tensor-core operand).
 #include <cmath>
 #include <cstdint>
 #include <cstring>
