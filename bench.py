@@ -248,6 +248,8 @@ def main(argv=None) -> int:
     ap.add_argument("--qjl", type=int, choices=[0, 1], default=None, help="1-bit QJL on K (default: the workload's)")
     ap.add_argument("--law", choices=["gaussian", "sphere"], default="gaussian",
                     help="coordinate law of the codebook (tq_law): N(0,1/d) or the exact unit-vector law")
+    ap.add_argument("--paged", type=int, default=0, metavar="BLOCK",
+                    help="paged cache with BLOCK tokens per block (a multiple of 64) and a shuffled block table")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each call kind alone (append quantize, decode) and add it to the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -278,7 +280,19 @@ def main(argv=None) -> int:
     n_steps_total = args.warmup + args.steps
     cap = int(math.ceil((max(lens0) + n_steps_total + 1) / 64) * 64)
     ctx = tq.Context(D, bits_k, bits_v, int(qjl), w.pi_seed, law=args.law)
-    caches = [tq.Cache(ctx, B, H, cap, device=dev) for _ in range(R)]
+    if args.paged:
+        if args.paged % 64:
+            raise SystemExit("--paged: the block size must be a multiple of 64")
+        cap = int(math.ceil(cap / args.paged) * args.paged)
+        per_seq = cap // args.paged
+        tgen = torch.Generator().manual_seed(w.seed + 31)
+
+        def paged_cache():
+            table = torch.randperm(B * per_seq, generator=tgen).to(torch.int32).view(B, per_seq)
+            return tq.PagedCache(ctx, B, H, cap, args.paged, n_blocks=B * per_seq, block_table=table, device=dev)
+        caches = [paged_cache() for _ in range(R)]
+    else:
+        caches = [tq.Cache(ctx, B, H, cap, device=dev) for _ in range(R)]
     gen = wl.generator(dev, w.seed + 7919 * rank)
     outl = wl.outlier_scale(w, dev, w.seed) if args.workload == "llama70b" else None
 
@@ -503,7 +517,7 @@ def main(argv=None) -> int:
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESCS[args.workload], "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl,
-                   "codebook": args.law,
+                   "codebook": args.law, "cache_layout": f"paged, {args.paged}-token blocks" if args.paged else "contiguous",
                    "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
                    f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
                    "parallelism": f"replicas x{ws}"},

@@ -91,6 +91,19 @@ enum {
  *  codes_v, norm_v as codes_k, norm_k with bits_v.
  * capacity must be a positive multiple of 64; every plane pointer 16-byte
  * aligned.
+ *
+ * Paged layout (block_table != NULL), as serving engines keep their KV
+ * caches: the planes hold n_blocks physical blocks of block_size tokens,
+ * laid out [n_blocks][n_kv_heads][block_size][bytes_per_token_head], and
+ * block_table (device int32, [n_seqs][capacity / block_size], 4-byte
+ * aligned) maps logical block j of sequence s to its physical block.
+ * Position p of sequence s is token p % block_size of physical block
+ * block_table[s][p / block_size].  capacity (the logical length per
+ * sequence) must be a multiple of block_size, and block_size a positive
+ * multiple of 64.  Entries outside [0, n_blocks) are device-side range
+ * errors: quantize skips the token, decode reads block 0 instead, and both
+ * set the token-range flag that tq_check_device_errors reports.  With
+ * block_table == NULL, block_size and n_blocks are ignored.
  */
 typedef struct tq_cache {
   uint8_t *codes_k;
@@ -102,6 +115,9 @@ typedef struct tq_cache {
   int32_t capacity;
   int32_t n_seqs;
   int32_t n_kv_heads;
+  const int32_t *block_table;
+  int32_t block_size;
+  int32_t n_blocks;
 } tq_cache;
 
 /*

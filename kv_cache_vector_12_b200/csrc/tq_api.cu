@@ -107,6 +107,14 @@ tq_status check_cache(const tq_ctx *ctx, const tq_cache *c) {
     if (planes[i] && !aligned16(planes[i]))
       return fail(TQ_ERR_INVALID, "cache plane %d is not 16-byte aligned", i);
   }
+  if (c->block_table) {  // paged layout
+    if (((uintptr_t)c->block_table & 3u) != 0) return fail(TQ_ERR_INVALID, "block_table must be 4-byte aligned");
+    if (c->block_size <= 0 || c->block_size % 64 != 0)
+      return fail(TQ_ERR_INVALID, "block_size=%d must be a positive multiple of 64", c->block_size);
+    if (c->capacity % c->block_size != 0)
+      return fail(TQ_ERR_INVALID, "capacity=%d must be a multiple of block_size=%d", c->capacity, c->block_size);
+    if (c->n_blocks <= 0) return fail(TQ_ERR_INVALID, "n_blocks=%d must be positive", c->n_blocks);
+  }
   return TQ_OK;
 }
 
@@ -159,15 +167,22 @@ constexpr int kLongSplitTokens = 8192;
 
 // The split is planned for the 3-CTA budget first; a call that meets neither
 // condition runs the 2-CTA budget instead, re-split for that occupancy.
-DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len) {
-  const int ctas = decode_ctas_per_sm(bits_k, bits_v, qjl, group, true);
+DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len,
+                        bool paged) {
+  if (paged) {  // the paged build has the 3-CTA budget only
+    DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group,
+                                                                                      true, true));
+    sp.long_splits = true;
+    return sp;
+  }
+  const int ctas = decode_ctas_per_sm(bits_k, bits_v, qjl, group, true, false);
   DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len, ctas);
   const long grid = (long)sp.n_splits * n_seqs * n_kv_heads;
   if (grid >= 2L * sm_count() * ctas || sp.chunk >= kLongSplitTokens) {
     sp.long_splits = true;
     return sp;
   }
-  return decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group, false));
+  return decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group, false, false));
 }
 
 tq_status report_error(tq_status st, const char *fmt, ...) {
@@ -371,10 +386,11 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->dp.bits_v = bits_v;
   ctx->dp.qjl = qjl;
   // resolve the decode kernels' occupancy now, outside any stream capture
-  for (const bool long_splits : {false, true}) {
-    tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8, long_splits);
-    tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16, long_splits);
-  }
+  for (const bool long_splits : {false, true})
+    for (const bool paged : {false, true}) {
+      tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8, long_splits, paged);
+      tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16, long_splits, paged);
+    }
   *out = ctx;
   return TQ_OK;
 }
@@ -456,8 +472,8 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
     return fail(TQ_ERR_INVALID, "misaligned q/out (16 B), workspace (256 B) or seq_lens/lse (4 B)");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
   const int group = n_q_heads / cache->n_kv_heads;
-  const tq::DecodeSplit sp =
-      tq::plan_decode(ctx->bits_k, ctx->bits_v, ctx->qjl, group, cache->n_seqs, cache->n_kv_heads, max_seq_len);
+  const tq::DecodeSplit sp = tq::plan_decode(ctx->bits_k, ctx->bits_v, ctx->qjl, group, cache->n_seqs,
+                                             cache->n_kv_heads, max_seq_len, cache->block_table != nullptr);
   const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, sp);
   if (workspace_bytes < ws.total)
     return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, ws.total);

@@ -266,7 +266,11 @@ struct DecodeArgs {
 // CTAs amortise the per-CTA prologue and each warp has room for more
 // independent work; CTAS = 3 (128 registers) for long splits, where twelve
 // consumer warps per SM hide more latency in the steady state.
-template <int BK, int BV, bool QJL, int NT, int CTAS>
+//
+// PAGED selects the paged cache layout (the stage copies follow the block
+// table); it is its own instantiation so that the contiguous kernels keep
+// their code and register allocation.
+template <int BK, int BV, bool QJL, int NT, int CTAS, bool PAGED>
 __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const DecodeArgs a) {
   static_assert(kStageTokens % 64 == 0 && kWarpTokens == 32, "stages start on 64-token boundaries");
   using St = Stage<BK, BV, QJL>;
@@ -314,7 +318,8 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     asm volatile("prefetch.global.L2 [%0];" ::"l"(a.seq_lens + s));
     const int first = split * a.chunk;
     const int last = min(min(first + a.chunk, a.max_seq_len), min(first + kPrefetchTokens, a.c.capacity));
-    if (first < last) {
+    // (contiguous layout only: a paged cache's block table is not read before the wait)
+    if (!PAGED && first < last) {
       const long tok = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + first;
       const uint32_t n = (uint32_t)(last - first);
       prefetch_l2(a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8));
@@ -368,16 +373,43 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         const int first = t0 + it * kStageTokens;  // multiple of 64, below the capacity
         // a stage never reads past the capacity (a multiple of 64, not of 128)
         const uint32_t n = (uint32_t)min(kStageTokens, a.c.capacity - first);
-        const long tok = base + first;
         const uint32_t bytes = n * (D * BK / 8 + D * BV / 8 + 4 + (QJL ? D / 8 + 2 : 0));
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(smem_u32(st + St::kc), a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8), bar);
-        bulk_g2s(smem_u32(st + St::vc), a.c.codes_v + tok * (D * BV / 8), n * (D * BV / 8), bar);
-        bulk_g2s(smem_u32(st + St::kn), a.c.norm_k + tok, n * 2, bar);
-        bulk_g2s(smem_u32(st + St::vn), a.c.norm_v + tok, n * 2, bar);
-        if constexpr (QJL) {
-          bulk_g2s(smem_u32(st + St::jb), a.c.qjl_bits + tok * (D / 8), n * (D / 8), bar);
-          bulk_g2s(smem_u32(st + St::jg), a.c.qjl_norm + tok, n * 2, bar);
+        if constexpr (!PAGED) {
+          const long tok = base + first;
+          bulk_g2s(smem_u32(st + St::kc), a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8), bar);
+          bulk_g2s(smem_u32(st + St::vc), a.c.codes_v + tok * (D * BV / 8), n * (D * BV / 8), bar);
+          bulk_g2s(smem_u32(st + St::kn), a.c.norm_k + tok, n * 2, bar);
+          bulk_g2s(smem_u32(st + St::vn), a.c.norm_v + tok, n * 2, bar);
+          if constexpr (QJL) {
+            bulk_g2s(smem_u32(st + St::jb), a.c.qjl_bits + tok * (D / 8), n * (D / 8), bar);
+            bulk_g2s(smem_u32(st + St::jg), a.c.qjl_norm + tok, n * 2, bar);
+          }
+        } else {
+          // the stage in runs of consecutive slots, one per block it touches
+          // (block sizes are multiples of 64, so every run is too and every
+          // copy stays 16-byte aligned at both ends)
+          for (uint32_t done = 0; done < n;) {
+            const int p = first + (int)done, j = p / a.c.block_size, off = p - j * a.c.block_size;
+            const uint32_t run = min(n - done, (uint32_t)(a.c.block_size - off));
+            int blk = a.c.block_table[(long)s * (a.c.capacity / a.c.block_size) + j];
+            if (blk < 0 || blk >= a.c.n_blocks) {  // flagged; a valid block is read in its place
+              atomicOr(a.p.err, kErrTokenRange);
+              blk = 0;
+            }
+            const long tok = ((long)blk * a.c.n_kv_heads + h) * a.c.block_size + off;
+            bulk_g2s(smem_u32(st + St::kc + done * (D * BK / 8)), a.c.codes_k + tok * (D * BK / 8),
+                     run * (D * BK / 8), bar);
+            bulk_g2s(smem_u32(st + St::vc + done * (D * BV / 8)), a.c.codes_v + tok * (D * BV / 8),
+                     run * (D * BV / 8), bar);
+            bulk_g2s(smem_u32(st + St::kn + done * 2), a.c.norm_k + tok, run * 2, bar);
+            bulk_g2s(smem_u32(st + St::vn + done * 2), a.c.norm_v + tok, run * 2, bar);
+            if constexpr (QJL) {
+              bulk_g2s(smem_u32(st + St::jb + done * (D / 8)), a.c.qjl_bits + tok * (D / 8), run * (D / 8), bar);
+              bulk_g2s(smem_u32(st + St::jg + done * 2), a.c.qjl_norm + tok, run * 2, bar);
+            }
+            done += run;
+          }
         }
         issued = it + 1;
       }
@@ -996,47 +1028,57 @@ struct Variant {
   int smem;
 };
 
+// Budgets: kShort (2 CTAs per SM), kLong (3 CTAs per SM) on the contiguous
+// layout; kPaged, the paged layout, which always runs the 3-CTA budget (its
+// callers decode batches of many sequences).
+enum Build { kShort = 0, kLong = 1, kPaged = 2 };
+
 template <int BK, int BV, bool QJL, int NT>
-Variant variant_c(bool long_splits) {
-  if (long_splits) return {decode_mma_kernel<BK, BV, QJL, NT, 3>, decode_smem_bytes<BK, BV, QJL, NT>()};
-  return {decode_mma_kernel<BK, BV, QJL, NT, 2>, decode_smem_bytes<BK, BV, QJL, NT>()};
+Variant variant_c(int build) {
+  constexpr int smem = decode_smem_bytes<BK, BV, QJL, NT>();
+  if (build == kPaged) return {decode_mma_kernel<BK, BV, QJL, NT, 3, true>, smem};
+  if (build == kLong) return {decode_mma_kernel<BK, BV, QJL, NT, 3, false>, smem};
+  return {decode_mma_kernel<BK, BV, QJL, NT, 2, false>, smem};
 }
 
 template <int BK, int BV, bool QJL>
-Variant variant_q(int nt, bool long_splits) {
-  return nt == 1 ? variant_c<BK, BV, QJL, 1>(long_splits) : variant_c<BK, BV, QJL, 2>(long_splits);
+Variant variant_q(int nt, int build) {
+  return nt == 1 ? variant_c<BK, BV, QJL, 1>(build) : variant_c<BK, BV, QJL, 2>(build);
 }
 
 template <int BK, int BV>
-Variant variant_v(bool qjl, int nt, bool long_splits) {
-  return qjl ? variant_q<BK, BV, true>(nt, long_splits) : variant_q<BK, BV, false>(nt, long_splits);
+Variant variant_v(bool qjl, int nt, int build) {
+  return qjl ? variant_q<BK, BV, true>(nt, build) : variant_q<BK, BV, false>(nt, build);
 }
 
 template <int BK>
-Variant variant_k(int bv, bool qjl, int nt, bool long_splits) {
+Variant variant_k(int bv, bool qjl, int nt, int build) {
   switch (bv) {
-    case 2: return variant_v<BK, 2>(qjl, nt, long_splits);
-    case 3: return variant_v<BK, 3>(qjl, nt, long_splits);
-    default: return variant_v<BK, 4>(qjl, nt, long_splits);
+    case 2: return variant_v<BK, 2>(qjl, nt, build);
+    case 3: return variant_v<BK, 3>(qjl, nt, build);
+    default: return variant_v<BK, 4>(qjl, nt, build);
   }
 }
 
-Variant variant(int bk, int bv, bool qjl, int nt, bool long_splits) {
+Variant variant(int bk, int bv, bool qjl, int nt, int build) {
   switch (bk) {
-    case 2: return variant_k<2>(bv, qjl, nt, long_splits);
-    case 3: return variant_k<3>(bv, qjl, nt, long_splits);
-    default: return variant_k<4>(bv, qjl, nt, long_splits);
+    case 2: return variant_k<2>(bv, qjl, nt, build);
+    case 3: return variant_k<3>(bv, qjl, nt, build);
+    default: return variant_k<4>(bv, qjl, nt, build);
   }
 }
+
+int build_of(bool long_splits, bool paged) { return paged ? kPaged : long_splits ? kLong : kShort; }
 
 }  // namespace
 
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits) {
-  static int cache[5][5][2][3][2] = {};
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged) {
+  static int cache[5][5][2][3][3] = {};
   const int nt = group > 8 ? 2 : 1;
-  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt][long_splits ? 1 : 0];
+  const int build = build_of(long_splits, paged);
+  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt][build];
   if (c == 0) {
-    const Variant v = variant(bits_k, bits_v, qjl != 0, nt, long_splits);
+    const Variant v = variant(bits_k, bits_v, qjl != 0, nt, build);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int n = 0;
@@ -1058,7 +1100,8 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
-  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1, split.long_splits);
+  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1,
+                            build_of(split.long_splits, c.block_table != nullptr));
   DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q, q_dtype, scale, partials};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(split.n_splits, c.n_kv_heads, c.n_seqs);

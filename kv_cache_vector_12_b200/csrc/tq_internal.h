@@ -76,10 +76,12 @@ struct DecodeSplit {
 };
 DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm);
 // CTAs per SM of the attention kernel for these bit widths and query heads per
-// KV head, with the long-split (128-register) or short-split (168) budget.
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits);
+// KV head, with the long-split (128-register) or short-split (168) budget, or
+// the paged-layout build (128 registers).
+int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged);
 // The split and register budget of one decode call (tq_api.cu).
-DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len);
+DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len,
+                        bool paged);
 
 // Workspace layout of decode attention (byte offsets, 256-aligned): the split
 // partials [rows][splits][d+4] (m, l, two unused floats, then the d outputs,

@@ -11,6 +11,7 @@
 
 #include <cmath>
 
+#include "tq_cache_slot.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -113,8 +114,8 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   const bool qjl = !is_v && p.qjl;
   const long row = blockIdx.x;
   const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
-  const int s = seq_idx[t], ps = pos[t];
-  if (!(s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity)) {
+  const long slot = cache_slot(c, seq_idx[t], h, pos[t]);
+  if (slot < 0) {
     if (tid == 0 && !is_v) atomicOr(p.err, kErrTokenRange);
     return;
   }
@@ -131,7 +132,6 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   for (int j = 0; j < half - 1; ++j) m += a > thr[half + j] * n ? 1 : 0;
   const int code = z > 0.f ? half + m : half - 1 - m;
 
-  const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
   uint32_t *dst = reinterpret_cast<uint32_t *>((is_v ? c.codes_v : c.codes_k) + slot * (D * bits / 8));
   for (int wd = 0; wd < bits; ++wd) {  // warp w owns words w*bits .. w*bits+bits-1
     uint32_t contrib = 0;

@@ -28,6 +28,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "tq_cache_slot.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -261,12 +262,11 @@ __global__ void __launch_bounds__(32 * kWarps, 2) quantize_qjl_kernel(DevicePara
       const long row = rows[e];
       if (row >= n_rows) continue;
       const int tok = (int)(row / c.n_kv_heads), h = (int)(row - (long)tok * c.n_kv_heads);
-      const int s = seq_idx[tok], ps = pos[tok];
-      if (!(s >= 0 && s < c.n_seqs && ps >= 0 && ps < c.capacity)) {
+      const long slot = cache_slot(c, seq_idx[tok], h, pos[tok]);
+      if (slot < 0) {
         if (q == 0 && h == 0) atomicOr(p.err, kErrTokenRange);
         continue;
       }
-      const long slot = ((long)s * c.n_kv_heads + h) * c.capacity + ps;
       const uint8_t *cd = &s_code[16 * warp + r + 8 * e][32 * q];
       uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + slot * (D * BK / 8)) + BK * q;
 #pragma unroll

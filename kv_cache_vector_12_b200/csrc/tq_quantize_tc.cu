@@ -27,6 +27,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "tq_cache_slot.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -505,10 +506,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
       long slot_i = -1;
       if (live) {
-        if (s_dst >= 0 && s_dst < a.c.n_seqs && p_dst >= 0 && p_dst < a.c.capacity)
-          slot_i = ((long)s_dst * a.c.n_kv_heads + tok_h) * a.c.capacity + p_dst;
-        else if (tok_h == 0 && is_k)
-          atomicOr(a.p.err, kErrTokenRange);
+        slot_i = cache_slot(a.c, s_dst, tok_h, p_dst);
+        if (slot_i < 0 && tok_h == 0 && is_k) atomicOr(a.p.err, kErrTokenRange);
       }
       if (slot_i >= 0) {
         const int bits = is_k ? BK : BV;

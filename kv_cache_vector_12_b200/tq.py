@@ -32,7 +32,7 @@ _fp = ctypes.POINTER(ctypes.c_float)
 class tq_cache(ctypes.Structure):
     _fields_ = [("codes_k", _vp), ("norm_k", _vp), ("qjl_bits", _vp), ("qjl_norm", _vp),
                 ("codes_v", _vp), ("norm_v", _vp), ("capacity", _i32), ("n_seqs", _i32),
-                ("n_kv_heads", _i32)]
+                ("n_kv_heads", _i32), ("block_table", _vp), ("block_size", _i32), ("n_blocks", _i32)]
 
 
 lib.tq_create.argtypes = [ctypes.POINTER(_vp), _i32, _i32, _i32, _i32, ctypes.c_uint64]
@@ -175,7 +175,41 @@ class Cache:
             dtype = torch.uint8 if nbytes > 2 else torch.int16
             self.planes[name] = torch.zeros(shape, dtype=dtype, device=device)
         self.n_seqs, self.n_kv_heads, self.capacity = n_seqs, n_kv_heads, capacity
-        self.struct = tq_cache(*[_ptr(self.planes[n]) for n in PLANES], capacity, n_seqs, n_kv_heads)
+        self.struct = tq_cache(*[_ptr(self.planes[n]) for n in PLANES], capacity, n_seqs, n_kv_heads, None, 0, 0)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.planes.values() if t is not None)
+
+
+class PagedCache:
+    """Device planes of one layer's packed cache in the paged layout:
+    n_blocks physical blocks of block_size tokens ([n_blocks][n_kv_heads]
+    [block_size][bytes] per plane) and a block table (device int32
+    [n_seqs][capacity / block_size]) mapping each sequence's logical blocks
+    to physical ones.  `block_table` may be given; by default sequence s owns
+    physical blocks s * per_seq ... in order."""
+
+    def __init__(self, ctx: Context, n_seqs: int, n_kv_heads: int, capacity: int, block_size: int,
+                 n_blocks: int | None = None, block_table: torch.Tensor | None = None, device="cuda"):
+        per_seq = capacity // block_size
+        if n_blocks is None:
+            n_blocks = n_seqs * per_seq
+        if block_table is None:
+            block_table = torch.arange(n_seqs * per_seq, dtype=torch.int32).view(n_seqs, per_seq)
+        self.block_table = block_table.to(device=device, dtype=torch.int32).contiguous()
+        sizes = ctx.layout()
+        self.planes = {}
+        for name, nbytes in zip(PLANES, sizes):
+            if nbytes == 0:
+                self.planes[name] = None
+                continue
+            shape = (n_blocks, n_kv_heads, block_size, nbytes) if nbytes > 2 else (n_blocks, n_kv_heads, block_size)
+            dtype = torch.uint8 if nbytes > 2 else torch.int16
+            self.planes[name] = torch.zeros(shape, dtype=dtype, device=device)
+        self.n_seqs, self.n_kv_heads, self.capacity = n_seqs, n_kv_heads, capacity
+        self.block_size, self.n_blocks = block_size, n_blocks
+        self.struct = tq_cache(*[_ptr(self.planes[n]) for n in PLANES], capacity, n_seqs, n_kv_heads,
+                               self.block_table.data_ptr(), block_size, n_blocks)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in self.planes.values() if t is not None)

@@ -52,7 +52,7 @@ def test_device_params_match_oracle(tq, bits_k, bits_v, qjl):
 
 
 def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=2, zero_rows=0, scaled_rows=(),
-                          law=o.LAW_GAUSSIAN):
+                          law=o.LAW_GAUSSIAN, paged_block=0):
     """scaled_rows: (first token, last token, exponent) ranges whose rows are
     multiplied by 2^exponent (exact in bf16)."""
     ctx = tq.Context(D, bits_k, bits_v, qjl, 42, law=law)
@@ -72,11 +72,18 @@ def _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed, n_seqs=
         sel = (seq_idx == s).nonzero().flatten()
         pos[sel] = torch.randperm(len(sel), generator=g).to(torch.int32) + 3
     cap = int(math.ceil((n_tok + 3 + 1) / 64) * 64)
-    cache = tq.Cache(ctx, n_seqs, n_heads, cap)
+    if paged_block:
+        cap = int(math.ceil(cap / paged_block) * paged_block)
+        table, n_blocks = _block_table(n_seqs, cap // paged_block, seed)
+        cache = tq.PagedCache(ctx, n_seqs, n_heads, cap, paged_block, n_blocks=n_blocks, block_table=table)
+    else:
+        cache = tq.Cache(ctx, n_seqs, n_heads, cap)
     dev = "cuda"
     tq.quantize(ctx, cache, k.to(dev), v.to(dev), seq_idx.to(dev), pos.to(dev))
     ctx.check_device_errors()
     planes = {n: (t.cpu().numpy() if t is not None else None) for n, t in cache.planes.items()}
+    if paged_block:
+        planes = _to_logical(planes, table, paged_block)
     si, ps = seq_idx.numpy(), pos.numpy()
     written = np.zeros((n_seqs, n_heads, cap), dtype=bool)
     for t in range(n_tok):
@@ -211,21 +218,64 @@ def _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, kind="lognormal
     return per, planes, cap
 
 
-def _upload(tq, ctx, planes, n_seqs, n_heads, cap):
-    cache = tq.Cache(ctx, n_seqs, n_heads, cap)
+def _block_table(n_seqs, per_seq, seed, spare=3):
+    """A shuffled block table: the sequences' logical blocks spread over
+    n_seqs * per_seq + spare physical blocks in a seeded random order."""
+    g = torch.Generator().manual_seed(seed)
+    n_blocks = n_seqs * per_seq + spare
+    return torch.randperm(n_blocks, generator=g)[:n_seqs * per_seq].to(torch.int32).view(n_seqs, per_seq), n_blocks
+
+
+def _to_logical(planes, table, block_size):
+    """Gather paged planes [n_blocks][H][block_size][...] into the logical
+    layout [n_seqs][H][capacity][...] through the block table."""
+    table = table.cpu().numpy()
+    out = {}
     for name, arr in planes.items():
-        if arr is not None:
-            t = torch.from_numpy(arr.view(np.int16) if arr.dtype == np.uint16 else arr)
-            cache.planes[name].copy_(t)
+        if arr is None:
+            out[name] = None
+            continue
+        blocks = arr[table]                                  # [n_seqs][per_seq][H][bs][...]
+        blocks = np.moveaxis(blocks, 2, 1)                   # [n_seqs][H][per_seq][bs][...]
+        out[name] = blocks.reshape(blocks.shape[0], blocks.shape[1], -1, *blocks.shape[4:])
+    return out
+
+
+def _upload(tq, ctx, planes, n_seqs, n_heads, cap, paged=None):
+    """paged: (block_size, seed) stores the planes in a paged cache whose
+    block table is shuffled."""
+    if paged is None:
+        cache = tq.Cache(ctx, n_seqs, n_heads, cap)
+        for name, arr in planes.items():
+            if arr is not None:
+                t = torch.from_numpy(arr.view(np.int16) if arr.dtype == np.uint16 else arr)
+                cache.planes[name].copy_(t)
+        return cache
+    bs, seed = paged
+    table, n_blocks = _block_table(n_seqs, cap // bs, seed)
+    cache = tq.PagedCache(ctx, n_seqs, n_heads, cap, bs, n_blocks=n_blocks, block_table=table)
+    tab = table.numpy()
+    for name, arr in planes.items():
+        if arr is None:
+            continue
+        a = arr.view(np.int16) if arr.dtype == np.uint16 else arr
+        phys = np.zeros((n_blocks,) + (n_heads, bs) + a.shape[3:], dtype=a.dtype)
+        for si in range(n_seqs):
+            for j in range(cap // bs):
+                phys[tab[si, j]] = a[si, :, j * bs:(j + 1) * bs]
+        cache.planes[name].copy_(torch.from_numpy(phys))
     return cache
 
 
 def _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed, q_dtype=torch.float32,
-                        scale=0.0, max_seq_len=None, law=o.LAW_GAUSSIAN):
+                        scale=0.0, max_seq_len=None, law=o.LAW_GAUSSIAN, paged_block=0):
     ctx = tq.Context(D, bits_k, bits_v, qjl, 42, law=law)
     ref = oracle_params(bits_k, bits_v, qjl, law=law)
-    per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, min_cap=max_seq_len or 0)
-    cache = _upload(tq, ctx, planes, len(lens), n_heads, cap)
+    min_cap = max(max_seq_len or 0, max(lens))
+    if paged_block:  # the logical capacity is a whole number of blocks
+        min_cap = int(math.ceil(max(min_cap, 1) / paged_block) * paged_block)
+    per, planes, cap = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed, min_cap=min_cap)
+    cache = _upload(tq, ctx, planes, len(lens), n_heads, cap, paged=(paged_block, seed) if paged_block else None)
     n_q = n_heads * group
     g = torch.Generator().manual_seed(seed + 99)
     q = torch.randn(len(lens), n_q, D, generator=g).to(q_dtype)
@@ -289,6 +339,53 @@ def test_sphere_device_params_match_oracle(tq):
         ref = oracle_params(bits, bits, 0, law=o.LAW_SPHERE)
         assert np.array_equal(p["centroids_k"].double().numpy(), ref.ck)
         assert np.array_equal(p["thresholds_v"].double().numpy(), ref.tv)
+
+
+# The paged layout: physical blocks in shuffled order behind a block table.
+@pytest.mark.parametrize("bits_k,bits_v,qjl", [(3, 3, 0), (2, 4, 1)])
+@pytest.mark.parametrize("n_tok,n_heads,block", [(129, 2, 64), (1031, 3, 128), (700, 2, 192)])
+def test_quantize_parity_paged(tq, n_tok, n_heads, block, bits_k, bits_v, qjl):
+    _quantize_and_compare(tq, n_tok, n_heads, bits_k, bits_v, qjl, seed=n_tok + block, paged_block=block)
+
+
+@pytest.mark.parametrize("bits_k,bits_v,qjl", [(3, 3, 0), (4, 2, 1)])
+@pytest.mark.parametrize("lens,n_heads,group,block", [([1000, 0, 513], 2, 8, 64), ([2500, 77], 1, 4, 128),
+                                                      ([20000], 1, 8, 256)])
+def test_decode_parity_paged(tq, lens, n_heads, group, block, bits_k, bits_v, qjl):
+    _decode_and_compare(tq, lens, n_heads, group, bits_k, bits_v, qjl, seed=sum(lens) + block, paged_block=block)
+
+
+def test_paged_block_table_out_of_range_is_flagged(tq):
+    """A block-table entry outside [0, n_blocks): quantize skips the token and
+    decode reads block 0 instead; both set the token-range flag."""
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    table = torch.tensor([[1, -1], [0, 5]], dtype=torch.int32)
+    cache = tq.PagedCache(ctx, 2, 1, 128, 64, n_blocks=2, block_table=table)
+    k = make_rows(2, 1, 3).cuda()
+    tq.quantize(ctx, cache, k, k, torch.tensor([0, 1], dtype=torch.int32, device="cuda"),
+                torch.tensor([70, 70], dtype=torch.int32, device="cuda"))   # logical block 1 of both: invalid
+    with pytest.raises(tq.TQError):
+        ctx.check_device_errors()
+    assert not torch.any(cache.planes["codes_k"]) and not torch.any(cache.planes["norm_k"])
+    out = torch.empty(2, 1, D, device="cuda")
+    ws = tq.alloc_workspace(ctx, 2, 1, 128)
+    tq.decode_attention(ctx, cache, torch.randn(2, 1, D, device="cuda"),
+                        torch.tensor([100, 100], dtype=torch.int32, device="cuda"), 128, out, None, ws)
+    with pytest.raises(tq.TQError):
+        ctx.check_device_errors()
+    assert torch.all(torch.isfinite(out))
+
+
+def test_paged_cache_argument_checks(tq):
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    k = torch.zeros(1, 1, D, dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for bs, cap in ((96, 192), (128, 192)):   # block size not a multiple of 64; capacity not a multiple of it
+        cache = tq.PagedCache(ctx, 1, 1, cap, bs, n_blocks=4,
+                              block_table=torch.zeros(1, max(1, cap // bs), dtype=torch.int32))
+        with pytest.raises(tq.TQError) as ei:
+            tq.quantize(ctx, cache, k, k, idx, idx)
+        assert ei.value.status == tq.TQ_ERR_INVALID
 
 
 def test_decode_long_sequence_many_splits(tq):
