@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -122,13 +123,16 @@ tq_status check_cache(const tq_ctx *ctx, const tq_cache *c) {
 
 namespace tq {
 
+// Cached once per process (atomically: calls may come from several threads).
 static int sm_count() {
-  static int n = 0;
+  static std::atomic<int> cached{0};
+  int n = cached.load(std::memory_order_relaxed);
   if (n == 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
+    cached.store(n, std::memory_order_relaxed);
   }
   return n;
 }

@@ -32,6 +32,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 
 #include "tq_internal.h"
@@ -1073,10 +1074,12 @@ int build_of(bool long_splits, bool paged) { return paged ? kPaged : long_splits
 }  // namespace
 
 int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged) {
-  static int cache[5][5][2][3][3] = {};
+  // cached per variant; atomically, as calls may come from several threads
+  static std::atomic<int> cache[5][5][2][3][3];
   const int nt = group > 8 ? 2 : 1;
   const int build = build_of(long_splits, paged);
-  int &c = cache[bits_k][bits_v][qjl ? 1 : 0][nt][build];
+  std::atomic<int> &slot = cache[bits_k][bits_v][qjl ? 1 : 0][nt][build];
+  int c = slot.load(std::memory_order_relaxed);
   if (c == 0) {
     const Variant v = variant(bits_k, bits_v, qjl != 0, nt, build);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
@@ -1084,6 +1087,7 @@ int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_spl
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, v.fn, kThreads, v.smem) != cudaSuccess || n < 1) n = 1;
     c = n;
+    slot.store(c, std::memory_order_relaxed);
   }
   return c;
 }

@@ -24,6 +24,8 @@
 //   store          packed codes, fp16 ||x||, sign bits (LSB first), fp16 ||r||.
 // Pi and S are read as coalesced B-fragment tables (built on the host),
 // 128 KB per 64 rows from L2, instead of 96 KB per row.
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -287,8 +289,10 @@ int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k,
                         const int32_t *pos, int n_tok, void *stream) {
   using Fn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, int);
   const Fn fn = p.bits_k == 2 ? quantize_qjl_kernel<2> : p.bits_k == 3 ? quantize_qjl_kernel<3> : quantize_qjl_kernel<4>;
-  static int slots[5] = {};  // resident CTAs on the device, per bit width
-  int &n_slots = slots[p.bits_k];
+  // resident CTAs on the device, per bit width; cached atomically, as calls
+  // may come from several threads
+  static std::atomic<int> slots[5];
+  int n_slots = slots[p.bits_k].load(std::memory_order_relaxed);
   if (n_slots == 0) {
     int dev = 0, n_sm = 0, per_sm = 0;
     cudaGetDevice(&dev);
@@ -298,6 +302,7 @@ int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k,
         per_sm < 1)
       per_sm = 1;
     n_slots = n_sm * per_sm;
+    slots[p.bits_k].store(n_slots, std::memory_order_relaxed);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   const long tiles = (rows + kRows - 1) / kRows;

@@ -24,6 +24,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -578,17 +579,20 @@ QuantTcFn pick(int bk, int bv) { return bk == 2 ? pick_bv<2>(bv) : bk == 3 ? pic
 
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream) {
-  static int n_sm = 0;
-  static bool configured[5][5] = {};
+  // cached atomically, as calls may come from several threads
+  static std::atomic<int> cached_sm{0};
+  static std::atomic<bool> configured[5][5];
+  int n_sm = cached_sm.load(std::memory_order_relaxed);
   if (n_sm == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+    cached_sm.store(n_sm, std::memory_order_relaxed);
   }
   const QuantTcFn fn = pick(p.bits_k, p.bits_v);
-  if (!configured[p.bits_k][p.bits_v]) {
+  if (!configured[p.bits_k][p.bits_v].load(std::memory_order_acquire)) {
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
-    configured[p.bits_k][p.bits_v] = true;
+    configured[p.bits_k][p.bits_v].store(true, std::memory_order_release);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   CUtensorMap mk, mv, mp;

@@ -53,6 +53,27 @@ def test_host_params_equal_oracle(tq, bits_k, bits_v, qjl, seed, law):
         assert np.array_equal(lib_p["s"].double().numpy(), ref.s)
 
 
+def test_cache_struct_layout_matches_header(tq, tmp_path):
+    """The binding's tq_cache mirrors include/tq.h field for field: a C
+    program compiled against the header prints sizeof and every offsetof."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in tq.tq_cache._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"tq.h\"\nint main(void) {\n"
+                   + "".join(f'  printf("%zu\\n", offsetof(tq_cache, {f}));\n' for f in fields)
+                   + '  printf("%zu\\n", sizeof(tq_cache));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    # the header's CUDA-free part only: tq.h includes nothing from CUDA
+    subprocess.run([cc, "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [getattr(tq.tq_cache, f).offset for f in fields] + [ctypes.sizeof(tq.tq_cache)]
+    assert got == want
+
+
 def test_invalid_arguments_fail_before_cuda(tq):
     lib = tq.lib
     f = ctypes.POINTER(ctypes.c_float)()
