@@ -227,7 +227,8 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD_DESC, "sample": desc},
+            "data": "synthetic", "config": {"workload": WORKLOAD_DESC, "bits_k": 3, "bits_v": 3, "qjl": False,
+                                            "codebook": "gaussian", "sample": desc},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": smp.threads(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
