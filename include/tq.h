@@ -188,8 +188,9 @@ tq_status tq_host_params_ex(int32_t d, int32_t bits_k, int32_t bits_v,
  * n_tok tokens t and KV head h, k[t][h][:] and v[t][h][:] (device, bf16,
  * contiguous [n_tok][n_kv_heads][d]) are normed, rotated by Pi, quantized,
  * packed and written at position pos[t] of sequence seq_idx[t] (device int32
- * arrays of n_tok).  Rows whose (seq_idx, pos) falls outside the cache are
- * skipped and flagged.  Tokens may arrive in any order; two tokens with the
+ * arrays of n_tok).  Rows whose (seq_idx, pos) falls outside the cache, or
+ * whose block-table entry is out of range in a paged cache, are skipped and
+ * flagged.  Tokens may arrive in any order; two tokens with the
  * same (seq_idx, pos) race.  n_tok == 0 is a no-op.
  */
 tq_status tq_quantize(tq_ctx *ctx, const tq_cache *cache, const void *k,
@@ -249,9 +250,10 @@ tq_status tq_decode_attention_noalloc(tq_ctx *ctx, const tq_cache *cache,
 /*
  * Synchronise `stream`, then report and clear the context's sticky
  * device-side error flags: TQ_OK, or TQ_ERR_DEVICE with a message naming the
- * flags (bit 0: token outside the cache in tq_quantize; bit 1: seq_len
- * outside [0, max_seq_len] in tq_decode_attention; bit 2: a bounded wait in a
- * kernel expired).
+ * flags (bit 0: a token outside the cache in tq_quantize, or a paged
+ * cache's block-table entry outside [0, n_blocks) in either call; bit 1:
+ * seq_len outside [0, max_seq_len] in tq_decode_attention; bit 2: a bounded
+ * wait in a kernel expired).
  */
 tq_status tq_check_device_errors(tq_ctx *ctx, void *stream);
 
