@@ -1,24 +1,35 @@
 """Benchmark of the TurboQuant hot path on B200 (one JSON line on rank 0).
 
-Workload (default ``llama8b``): one Llama-3-8B-shaped layer, 8 KV / 32 query
-heads, d = 128, 32768 cached tokens, batch 1, 3-bit K and V (no QJL).  The
+Workload (default ``serving``, the largest single-GPU configuration): 32
+decode sequences with seeded lengths uniform on [1024, 65536], 8 KV / 32
+query heads, d = 128, bf16 K/V ~ N(0,1), 3-bit K and V (no QJL).  The
 prefill is quantized once into R cache replicas; a *step* is one decode step
-of the whole hot path: quantize-on-append of one new token (8 KV heads, K and
-V) followed by decode attention of the 32 query heads over the packed cache.
-Step i uses replica i % R, so consecutive steps read disjoint memory and the
-step-to-step working set (R x 26 MB) exceeds the 126 MB L2.
+of the whole hot path: quantize-on-append of one new token per sequence (8 KV
+heads, K and V) followed by the ragged batched decode attention of the 32
+query heads over the packed cache.  Step i uses replica i % R; R is chosen so
+the replicas exceed twice the 126 MB L2 (one replica of ~0.85 GB for
+serving), so every step reads its cache cold.  ``--workload`` selects the
+other configurations (llama8b, llama70b, qwen, tiny).
 
 ``value``  decode-attention effective GB/s: packed K/V bytes the step reads
-           (codes + fp16 norms) / device time per step (CUDA graph of the K
-           timed steps, CUDA events, max over ranks).
+           (codes + fp16 norms) / device time per step.  The K timed steps
+           are one CUDA graph; it is replayed back to back for at least
+           200 ms, each replay bracketed by CUDA events, and the median replay
+           time is the time of K steps (max over ranks).
 ``e2e``    the same metric when every step goes through the C ABI eagerly
-           with pinned host buffers: H2D of the token's K/V and of q, the two
+           with pinned host buffers: H2D of the tokens' K/V and of q, the two
            calls, D2H of the output.
 ``roofline`` the decode calls of the timed steps alone (same replicas and
-           lengths) as one CUDA graph, events around its replay; algorithmic
+           lengths) as one CUDA graph, replayed the same way; algorithmic
            bytes = packed bytes per call.
-``quantize_*`` prefill quantize of 32768 tokens (input 128 MB > L2): tokens/s,
-           GB/s (bf16 read + packed write) and roofline fraction.
+``quantize`` the whole prefill of the batch (every sequence's tokens, one
+           call; inputs far larger than L2): tokens/s, GB/s (bf16 read +
+           packed write) and roofline fraction.
+``quality`` compressed vs exact (fp64, over the bf16 inputs) attention of a
+           sampled (sequence, KV head): cosine similarity of the outputs,
+           bias and RMS of the per-token score error relative to the RMS of
+           the exact scores, and the cosine similarity of reconstructed V
+           vectors, all read from the library's own kernels.
 ``cpu_baseline`` the CPU oracle on a bounded sample of the same decode step.
 
 ``--impl reference`` times the CPU oracle on the host instead (the reference
@@ -60,7 +71,7 @@ WORKLOAD_DESCS = {
     "serving": ("serving: 32 sequences, lengths uniform on [1024, 65536] (seeded), 8 KV / 32 query heads, "
                 "d=128, bf16 N(0,1); step = append-quantize 1 token per sequence + ragged batched decode"),
 }
-WORKLOAD_DESC = WORKLOAD_DESCS["llama8b"]
+DEFAULT_WORKLOAD = "serving"
 
 
 # DRAM bytes per attention-kernel launch (dram__bytes_read.sum +
@@ -153,43 +164,51 @@ class ClockSampler:
 
 
 class OracleDecodeSample:
-    """The CPU oracle on a bounded sample of the llama8b decode step: the
-    packed codes of `n_heads` KV heads (quantized once by the oracle, untimed),
-    then per step: unpack them and run the oracle's decode attention for the
-    heads' query heads."""
+    """The CPU oracle on a bounded sample of one decode step of a workload:
+    the first sequence's cache for `n_heads` KV heads (quantized once by the
+    oracle, untimed), then per step: append-quantize of the step's token,
+    unpack of the codes and the oracle's decode attention for the heads'
+    query heads."""
 
-    def __init__(self, n_heads: int = 8, seq_len: int = 32768, seed: int = 1002):
+    def __init__(self, workload: str, bits_k: int, bits_v: int, qjl: bool, n_heads: int = 8):
         from oracle import turboquant_oracle as o
         from kv_cache_vector_12_b200 import workloads as wl
         self.o = o
-        self.w = w = wl.WORKLOADS["llama8b"]
-        self.p = p = o.Params(w.d, w.bits_k, w.bits_v, False, w.pi_seed)
-        gen = wl.generator("cpu", seed)
-        k, v = wl.kv_tokens(w, seq_len, gen, "cpu")
+        self.w = w = wl.WORKLOADS[workload]
+        self.bits_k, self.bits_v, self.qjl = bits_k, bits_v, qjl
+        self.p = p = o.Params(w.d, bits_k, bits_v, qjl, w.pi_seed)
+        n_heads = min(n_heads, w.n_kv_heads)
+        seq_len = wl.serving_lengths(w, w.seed)[0] if workload == "serving" else w.seq_len
+        gen = wl.generator("cpu", w.seed)
+        outl = wl.outlier_scale(w, "cpu", w.seed) if workload == "llama70b" else None
+        k, v = wl.kv_tokens(w, seq_len, gen, "cpu", outlier_mask=outl)
         self.q = wl.queries(w, 1, gen, "cpu").double().numpy()[0]
-        k_new, v_new = wl.kv_tokens(w, 1, gen, "cpu")
+        k_new, v_new = wl.kv_tokens(w, 1, gen, "cpu", outlier_mask=outl)
         self.new_rows = [(k_new[:, h].double().numpy(), v_new[:, h].double().numpy()) for h in range(n_heads)]
         self.packed = []
         for h in range(n_heads):
-            qk = o.quantize(k[:, h].double().numpy(), p.pi, p.ck, p.tk)
+            qk = o.quantize(k[:, h].double().numpy(), p.pi, p.ck, p.tk, s_matrix=p.s if qjl else None)
             qv = o.quantize(v[:, h].double().numpy(), p.pi, p.cv, p.tv)
-            self.packed.append((o.pack_codes(qk.codes, w.bits_k), qk.norm,
-                                o.pack_codes(qv.codes, w.bits_v), qv.norm))
-        self.step_bytes = n_heads * seq_len * (w.d * (w.bits_k + w.bits_v) // 8 + 4)
+            self.packed.append((o.pack_codes(qk.codes, bits_k), qk.norm, o.pack_codes(qv.codes, bits_v), qv.norm,
+                                o.pack_signs(qk.qjl_signs) if qjl else None, qk.qjl_gamma if qjl else None))
+        self.step_bytes = n_heads * seq_len * (w.d * (bits_k + bits_v) // 8 + 4 + (w.d // 8 + 2 if qjl else 0))
         self.desc = (f"oracle append-quantize of 1 token + unpack + decode attention of {n_heads} KV heads x "
-                     f"{seq_len} tokens (llama8b decode step, numpy fp64)")
+                     f"{seq_len} tokens ({workload} decode step, first sequence, {bits_k}/{bits_v} bits"
+                     f"{' + QJL' if qjl else ''}, numpy fp64)")
 
     def step(self) -> float:
         o, w, p = self.o, self.w, self.p
+        s_mat = p.s if self.qjl else None
         t0 = time.perf_counter()
-        for h, (pk, nk, pv, nv) in enumerate(self.packed):
+        for h, (pk, nk, pv, nv, pj, gj) in enumerate(self.packed):
             kn, vn = self.new_rows[h]                      # append-quantize of the step's token
-            o.pack_codes(o.quantize(kn, p.pi, p.ck, p.tk).codes, w.bits_k)
-            o.pack_codes(o.quantize(vn, p.pi, p.cv, p.tv).codes, w.bits_v)
-            ck = o.unpack_codes(pk, w.bits_k, w.d)
-            cv = o.unpack_codes(pv, w.bits_v, w.d)
+            o.pack_codes(o.quantize(kn, p.pi, p.ck, p.tk, s_matrix=s_mat).codes, self.bits_k)
+            o.pack_codes(o.quantize(vn, p.pi, p.cv, p.tv).codes, self.bits_v)
+            ck = o.unpack_codes(pk, self.bits_k, w.d)
+            cv = o.unpack_codes(pv, self.bits_v, w.d)
+            signs = o.unpack_signs(pj, w.d) if self.qjl else None
             o.decode_attention(self.q[h * w.group:(h + 1) * w.group], p.pi, p.ck, ck, nk, p.cv, cv, nv,
-                               1 / math.sqrt(w.d))
+                               1 / math.sqrt(w.d), s_matrix=s_mat, qjl_signs=signs, qjl_gamma=gj)
         return time.perf_counter() - t0
 
     @staticmethod
@@ -201,8 +220,8 @@ class OracleDecodeSample:
             return os.cpu_count() or 1
 
 
-def cpu_baseline(min_seconds: float = 10.0) -> dict:
-    smp = OracleDecodeSample(n_heads=8)
+def cpu_baseline(workload: str, bits_k: int, bits_v: int, qjl: bool, min_seconds: float = 10.0) -> dict:
+    smp = OracleDecodeSample(workload, bits_k, bits_v, qjl, n_heads=8)
     total, reps = 0.0, 0
     while total < min_seconds:
         total += smp.step()
@@ -211,11 +230,20 @@ def cpu_baseline(min_seconds: float = 10.0) -> dict:
             "kind": "oracle", "sample": f"{smp.desc}, {reps} steps", "seconds": total}
 
 
+def resolve_setting(args):
+    from kv_cache_vector_12_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    bits_k, bits_v = args.bits if args.bits else (w.bits_k, w.bits_v)
+    qjl = w.qjl if args.qjl is None else bool(args.qjl)
+    return w, bits_k, bits_v, qjl
+
+
 def reference_arm(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    smp = OracleDecodeSample(n_heads=1)
+    w, bits_k, bits_v, qjl = resolve_setting(args)
+    smp = OracleDecodeSample(args.workload, bits_k, bits_v, qjl, n_heads=1)
     times = []
     for i in range(args.warmup + args.steps):
         dt = smp.step()
@@ -227,13 +255,68 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD_DESC, "bits_k": 3, "bits_v": 3, "qjl": False,
-                                            "codebook": "gaussian", "sample": desc},
+            "data": "synthetic", "config": {"workload": WORKLOAD_DESCS[args.workload], "bits_k": bits_k,
+                                            "bits_v": bits_v, "qjl": qjl, "codebook": args.law, "sample": desc},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": smp.threads(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def quality_report(tq, ctx, cache, lens0, q_first, k_s0, v_s0, group, n_tokens=4096) -> dict:
+    """Compressed vs exact attention on a sampled (sequence 0, KV head 0),
+    every compressed figure read from the library's kernels.
+
+    * attn_cos_sim: cosine similarity of the decode outputs of KV head 0's
+      query heads over sequence 0 (its prefill length) with fp64 softmax
+      attention over the bf16 K/V rows that were quantized (mean and min over
+      the query heads).
+    * score_bias_rel / score_rms_rel: the per-token score error (inner-product
+      error times the softmax scale) of the first `n_tokens` tokens: a batch
+      of one-token sequences, quantized by the library, whose decode returns
+      each token's score as the log-sum-exp; bias and RMS of s_tq - s_exact,
+      relative to the RMS of the exact scores.
+    * v_cos_sim: the same one-token decodes return the reconstructed V
+      vectors (o = Pi^T ||v|| c_V[codes]); mean cosine similarity with the
+      original rows, the figure the pages quote per V bit width."""
+    dev = q_first.device
+    D = q_first.shape[-1]
+    scale = 1.0 / math.sqrt(D)
+    B, HQ = q_first.shape[0], q_first.shape[1]
+    out = torch.empty(B, HQ, D, device=dev)
+    ws = tq.alloc_workspace(ctx, B, HQ, max(lens0), device=dev)
+    tq.decode_attention(ctx, cache, q_first, torch.tensor(lens0, dtype=torch.int32, device=dev), max(lens0), out,
+                        None, ws)
+    q0 = q_first[0, :group].double().cpu()                         # [G, d]
+    k0, v0 = k_s0.double(), v_s0.double()                          # [T, d]
+    s_ex = scale * (q0 @ k0.T)
+    o_ex = torch.softmax(s_ex, dim=1) @ v0
+    o_tq = out[0, :group].double().cpu()
+    cos = torch.nn.functional.cosine_similarity(o_tq, o_ex, dim=1)
+
+    n = min(n_tokens, k_s0.shape[0])
+    one = tq.Cache(ctx, n, 1, 64, device=dev)
+    idx = torch.arange(n, dtype=torch.int32, device=dev)
+    tq.quantize(ctx, one, k_s0[:n, None].to(dev).contiguous(), v_s0[:n, None].to(dev).contiguous(), idx, idx * 0)
+    q_rep = q_first[0, :group].float()[None].expand(n, group, D).contiguous()
+    out1 = torch.empty(n, group, D, device=dev)
+    lse1 = torch.empty(n, group, device=dev)
+    ws1 = tq.alloc_workspace(ctx, n, group, 1, device=dev)
+    tq.decode_attention(ctx, one, q_rep, torch.ones(n, dtype=torch.int32, device=dev), 1, out1, lse1, ws1)
+    ctx.check_device_errors()
+    s_tq = lse1.double().cpu().T                                   # [G, n]
+    err = s_tq - s_ex[:, :n]
+    rms_ex = float(s_ex[:, :n].pow(2).mean().sqrt())
+    v_hat = out1[:, 0].double().cpu()
+    v_cos = torch.nn.functional.cosine_similarity(v_hat, v0[:n], dim=1)
+    return {"sample": f"sequence 0, KV head 0 ({k_s0.shape[0]} tokens, {group} query heads); scores and V "
+                      f"vectors of its first {n} tokens",
+            "attn_cos_sim": float(cos.mean()), "attn_cos_sim_min": float(cos.min()),
+            "score_bias_rel": float(err.mean()) / rms_ex, "score_rms_rel": float(err.pow(2).mean().sqrt()) / rms_ex,
+            "v_cos_sim": float(v_cos.mean()),
+            "pages_v_cos_sim": {"2-bit V": 0.94, "4-bit V": 0.997},
+            "reference": "exact softmax attention in fp64 over the bf16 K/V rows"}
 
 
 def main(argv=None) -> int:
@@ -243,7 +326,7 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--replicas", type=int, default=0, help="cache replicas (default: enough to exceed L2)")
-    ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOAD_DESCS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOAD_DESCS))
     ap.add_argument("--bits", type=int, nargs=2, metavar=("K", "V"), default=None,
                     help="code bits of K and V (default: the workload's)")
     ap.add_argument("--qjl", type=int, choices=[0, 1], default=None, help="1-bit QJL on K (default: the workload's)")
@@ -270,12 +353,9 @@ def main(argv=None) -> int:
 
     from kv_cache_vector_12_b200 import tq
     from kv_cache_vector_12_b200 import workloads as wl
-    w = wl.WORKLOADS[args.workload]
-    bits_k, bits_v = args.bits if args.bits else (w.bits_k, w.bits_v)
-    qjl = w.qjl if args.qjl is None else bool(args.qjl)
+    w, bits_k, bits_v, qjl = resolve_setting(args)
     H, HQ, D, B = w.n_kv_heads, w.n_q_heads, w.d, w.n_seqs
     lens0 = wl.serving_lengths(w, w.seed) if args.workload == "serving" else [w.seq_len] * B
-    T = lens0[0]                       # the quantize measurement uses the first sequence's prefill
     bytes_per_token = H * (D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
     R = args.replicas or max(1, math.ceil(2 * 126e6 / (sum(lens0) * bytes_per_token)))
     n_steps_total = args.warmup + args.steps
@@ -297,26 +377,36 @@ def main(argv=None) -> int:
     gen = wl.generator(dev, w.seed + 7919 * rank)
     outl = wl.outlier_scale(w, dev, w.seed) if args.workload == "llama70b" else None
 
-    # ---- prefill quantize (also the quantize measurement: the first sequence) ----
-    q_ms = None
-    for b in range(B):
-        n_b = lens0[b]
-        pos0 = torch.arange(n_b, dtype=torch.int32, device=dev)
-        k_pre, v_pre = wl.kv_tokens(w, n_b, gen, dev, outlier_mask=outl)
-        seqb = torch.full((n_b,), b, dtype=torch.int32, device=dev)
-        for c in caches:
-            tq.quantize(ctx, c, k_pre, v_pre, seqb, pos0)
-        if b == 0:
-            torch.cuda.synchronize()
-            qreps = 10
-            qe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * qreps)]
-            for i in range(qreps):
-                qe[2 * i].record()
-                tq.quantize(ctx, caches[i % R], k_pre, v_pre, seqb, pos0)
-                qe[2 * i + 1].record()
-            torch.cuda.synchronize()
-            q_ms = statistics.median(qe[2 * i].elapsed_time(qe[2 * i + 1]) for i in range(qreps))
-        del k_pre, v_pre
+    # ---- prefill: every sequence's tokens in one quantize call per replica;
+    # the same call, repeated, is the quantize measurement (inputs of
+    # sum(lens) x H x d bf16 for K and V, far larger than L2) ----
+    n_pre = sum(lens0)
+    k_pre = torch.empty(n_pre, H, D, dtype=torch.bfloat16, device=dev)
+    v_pre = torch.empty_like(k_pre)
+    seq_pre = torch.empty(n_pre, dtype=torch.int32, device=dev)
+    pos_pre = torch.empty(n_pre, dtype=torch.int32, device=dev)
+    off = 0
+    for b, n_b in enumerate(lens0):
+        k_b, v_b = wl.kv_tokens(w, n_b, gen, dev, outlier_mask=outl)
+        k_pre[off:off + n_b], v_pre[off:off + n_b] = k_b, v_b
+        seq_pre[off:off + n_b] = b
+        pos_pre[off:off + n_b] = torch.arange(n_b, dtype=torch.int32, device=dev)
+        off += n_b
+        del k_b, v_b
+    # the sampled (sequence 0, KV head 0) of the quality report, kept on the host
+    k_s0, v_s0 = k_pre[:lens0[0], 0].cpu(), v_pre[:lens0[0], 0].cpu()
+    for c in caches:
+        tq.quantize(ctx, c, k_pre, v_pre, seq_pre, pos_pre)
+    torch.cuda.synchronize()
+    qreps = 10
+    qe = [torch.cuda.Event(enable_timing=True) for _ in range(2 * qreps)]
+    for i in range(qreps):
+        qe[2 * i].record()
+        tq.quantize(ctx, caches[i % R], k_pre, v_pre, seq_pre, pos_pre)
+        qe[2 * i + 1].record()
+    torch.cuda.synchronize()
+    q_ms = statistics.median(qe[2 * i].elapsed_time(qe[2 * i + 1]) for i in range(qreps))
+    del k_pre, v_pre, seq_pre, pos_pre
     torch.cuda.synchronize()
     ctx.check_device_errors()
 
@@ -361,6 +451,33 @@ def main(argv=None) -> int:
     torch.cuda.synchronize()
     ctx.check_device_errors()
 
+    def replay_median(graph, min_ms=200.0):
+        """Median device time (ms) of one replay of `graph`: replays queued
+        back to back, each bracketed by CUDA events on the launching stream,
+        for at least `min_ms` in total (three at least)."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        n = max(3, min(1000, int(math.ceil(min_ms / max(e0.elapsed_time(e1), 1e-3)))))
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+        for j in range(n):
+            evs[2 * j].record()
+            graph.replay()
+            evs[2 * j + 1].record()
+        torch.cuda.synchronize()
+        times = [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(n)]
+        return statistics.median(times), n
+
+    # decode calls alone: the timed steps' decode calls (same replicas, same
+    # lengths, their tokens already appended) as one CUDA graph
+    with torch.cuda.graph(g_dec):
+        for i in range(args.warmup, n_steps_total):
+            tq.decode_attention(ctx, caches[i % R], q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
+    g_dec.replay()
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(local)
     if ws > 1:
         torch.distributed.barrier()
@@ -368,37 +485,21 @@ def main(argv=None) -> int:
     sampler.start()
     # keep the GPU busy up to the timed region (clocks at their loaded level,
     # and the clock sampler sees load): about 50 ms of warm-up replays, then
-    # the timed replay is queued behind them with no idle gap
+    # the timed replays are queued behind them with no idle gap
     wb0, wb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wb0.record()
     g_warm.replay()
     wb1.record()
     torch.cuda.synchronize()
     n_burst = max(1, min(2000, int(50.0 / max(wb0.elapsed_time(wb1), 1e-3))))
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(n_burst):
         g_warm.replay()
-    ev0.record()
-    g_timed.replay()
-    ev1.record()
-    torch.cuda.synchronize()
-    ms_total = ev0.elapsed_time(ev1)
-    # decode calls alone: the timed steps' decode calls (same replicas, same
-    # lengths, their tokens already appended) as one CUDA graph, events around
-    # its replay on the launching stream
-    with torch.cuda.graph(g_dec):
-        for i in range(args.warmup, n_steps_total):
-            tq.decode_attention(ctx, caches[i % R], q_all[i], lens_steps[i], max_len, out[i], lse[i], wsb)
-    g_dec.replay()
-    torch.cuda.synchronize()
-    ed0, ed1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ed0.record()
-    g_dec.replay()
-    ed1.record()
-    torch.cuda.synchronize()
+    ms_total, n_replays = replay_median(g_timed)
+    dec_total, _ = replay_median(g_dec)
     clocks = sampler.stop()
-    dec_ms = [ed0.elapsed_time(ed1) / args.steps]
+    dec_ms = [dec_total / args.steps]
     ctx.check_device_errors()
+    quality = quality_report(tq, ctx, caches[0], lens0, q_all[args.warmup], k_s0, v_s0, w.group)
 
     breakdown = None
     if args.breakdown:
@@ -503,8 +604,8 @@ def main(argv=None) -> int:
     value = job_gbps(ws, timed_bytes, ms_total)
     e2e_val = job_gbps(ws, timed_bytes, e2e_ms)
     dec_achieved = (timed_bytes / args.steps) / (dec_mean * 1e-3) / 1e9
-    q_tokens = T / (q_ms * 1e-3)
-    q_bytes = T * H * (2 * D * 2 + D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
+    q_tokens = n_pre / (q_ms * 1e-3)
+    q_bytes = n_pre * H * (2 * D * 2 + D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
     q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
 
     if rank != 0:
@@ -512,7 +613,7 @@ def main(argv=None) -> int:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return 0
-    cpu = None if args.no_cpu_baseline else cpu_baseline()
+    cpu = None if args.no_cpu_baseline else cpu_baseline(args.workload, bits_k, bits_v, qjl)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
@@ -520,7 +621,8 @@ def main(argv=None) -> int:
         "config": {"workload": WORKLOAD_DESCS[args.workload], "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl,
                    "codebook": args.law, "cache_layout": f"paged, {args.paged}-token blocks" if args.paged else "contiguous",
                    "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
-                   f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": "CUDA graph of the timed steps",
+                   f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": f"CUDA graph of the {args.steps} timed steps, replayed back to back "
+                   f"{n_replays} times (>= 200 ms); median replay",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
                      "frac": dec_achieved / peak,
@@ -529,7 +631,10 @@ def main(argv=None) -> int:
                      "kernel": "tq_decode_attention call (split-K attention with q rotation + merge)",
                      "algorithmic_bytes_per_call": timed_bytes / args.steps},
         "quantize": {"tokens_per_s": q_tokens, "GBps": q_gbs, "frac": q_gbs / peak, "ms": q_ms,
-                     "tokens": T, "bytes": q_bytes},
+                     "tokens": n_pre, "bytes": q_bytes,
+                     "call": f"one tq_quantize of the whole prefill ({B} sequences, {n_pre} tokens x {H} KV heads), "
+                             "median of 10"},
+        "quality": quality,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,

@@ -15,6 +15,11 @@
  *  - All pointers named "device" are CUDA device pointers on the current
  *    device; "host" pointers are ordinary host memory.  The caller owns every
  *    buffer; the library never frees, keeps or allocates caller memory.
+ *  - A context belongs to the device that was current when it was created.
+ *    The compute calls (tq_quantize, tq_decode_attention,
+ *    tq_decode_attention_noalloc) check that this device is current and
+ *    return TQ_ERR_INVALID, launching nothing, when it is not.  One process
+ *    may hold contexts on several devices.
  *  - Compute calls (tq_quantize, tq_decode_attention) are asynchronous on the
  *    given stream (a cudaStream_t passed as void*; NULL = legacy default
  *    stream), allocate nothing, never synchronise and never read device data
@@ -100,10 +105,15 @@ enum {
  * Position p of sequence s is token p % block_size of physical block
  * block_table[s][p / block_size].  capacity (the logical length per
  * sequence) must be a multiple of block_size, and block_size a positive
- * multiple of 64.  Entries outside [0, n_blocks) are device-side range
- * errors: quantize skips the token, decode reads block 0 instead, and both
- * set the token-range flag that tq_check_device_errors reports.  With
- * block_table == NULL, block_size and n_blocks are ignored.
+ * multiple of 64.  Only the entries a call needs are read: quantize reads
+ * the entry of each position it writes, decode the entries of the blocks
+ * that hold positions below each sequence's length.  Entries past a
+ * sequence's length may therefore hold anything (an engine's -1 for an
+ * unassigned block, say).  An entry that is read and lies outside
+ * [0, n_blocks) is a device-side range error: quantize skips the token,
+ * decode reads block 0 instead, and both set the token-range flag that
+ * tq_check_device_errors reports.  With block_table == NULL, block_size and
+ * n_blocks are ignored.
  */
 typedef struct tq_cache {
   uint8_t *codes_k;

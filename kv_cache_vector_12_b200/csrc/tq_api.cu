@@ -123,16 +123,30 @@ tq_status check_cache(const tq_ctx *ctx, const tq_cache *c) {
 
 namespace tq {
 
-// Cached once per process (atomically: calls may come from several threads).
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  return dev;
+}
+
+tq_status check_context_device(const tq_ctx *ctx) {
+  int cur = -1;
+  const cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != ctx->device)
+    return fail(TQ_ERR_INVALID, "the current CUDA device is %d but the context was created on device %d", cur,
+                ctx->device);
+  return TQ_OK;
+}
+
+// Cached once per device (atomically: calls may come from several threads).
 static int sm_count() {
-  static std::atomic<int> cached{0};
-  int n = cached.load(std::memory_order_relaxed);
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  int n = cached[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    cached.store(n, std::memory_order_relaxed);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -433,7 +447,9 @@ tq_status tq_get_params(const tq_ctx *ctx, float *pi, float *s, float *centroids
 tq_status tq_quantize(tq_ctx *ctx, const tq_cache *cache, const void *k, const void *v,
                       const int32_t *seq_idx, const int32_t *pos, int32_t n_tok, void *stream) {
   if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
-  tq_status st = check_cache(ctx, cache);
+  tq_status st = tq::check_context_device(ctx);
+  if (st != TQ_OK) return st;
+  st = check_cache(ctx, cache);
   if (st != TQ_OK) return st;
   if (n_tok < 0) return fail(TQ_ERR_INVALID, "n_tok=%d is negative", n_tok);
   if (n_tok == 0) return TQ_OK;
@@ -459,7 +475,9 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
                               float scale, float *out, float *lse, void *workspace,
                               size_t workspace_bytes, void *stream) {
   if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
-  tq_status st = check_cache(ctx, cache);
+  tq_status st = tq::check_context_device(ctx);
+  if (st != TQ_OK) return st;
+  st = check_cache(ctx, cache);
   if (st != TQ_OK) return st;
   if (!q || !seq_lens || !out || !workspace)
     return fail(TQ_ERR_INVALID, "q, seq_lens, out and workspace must be non-NULL");

@@ -371,9 +371,12 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         if (*(volatile int *)&abort_flag) break;
         unsigned char *st = smem + slot * St::bytes;
         const uint32_t bar = smem_u32(&full_bar[slot]);
-        const int first = t0 + it * kStageTokens;  // multiple of 64, below the capacity
-        // a stage never reads past the capacity (a multiple of 64, not of 128)
-        const uint32_t n = (uint32_t)min(kStageTokens, a.c.capacity - first);
+        const int first = t0 + it * kStageTokens;  // multiple of 64, below the split's end t1
+        // a stage copies its tokens below t1 rounded up to a multiple of 64:
+        // never past the capacity (a multiple of 64 at or above t1), and in a
+        // paged cache never from a block that holds no position below t1, so
+        // the table entries of blocks past the length are not read
+        const uint32_t n = (uint32_t)min(kStageTokens, (t1 - first + 63) & ~63);
         const uint32_t bytes = n * (D * BK / 8 + D * BV / 8 + 4 + (QJL ? D / 8 + 2 : 0));
         mbar_arrive_expect_tx(bar, bytes);
         if constexpr (!PAGED) {
@@ -1075,10 +1078,11 @@ int build_of(bool long_splits, bool paged) { return paged ? kPaged : long_splits
 
 int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged) {
   // cached per variant; atomically, as calls may come from several threads
-  static std::atomic<int> cache[5][5][2][3][3];
+  // (per device: the attribute and the occupancy query apply to the current one)
+  static std::atomic<int> cache[kMaxDevices][3][3][2][2][3];
   const int nt = group > 8 ? 2 : 1;
   const int build = build_of(long_splits, paged);
-  std::atomic<int> &slot = cache[bits_k][bits_v][qjl ? 1 : 0][nt][build];
+  std::atomic<int> &slot = cache[current_device()][bits_k - 2][bits_v - 2][qjl ? 1 : 0][nt - 1][build];
   int c = slot.load(std::memory_order_relaxed);
   if (c == 0) {
     const Variant v = variant(bits_k, bits_v, qjl != 0, nt, build);

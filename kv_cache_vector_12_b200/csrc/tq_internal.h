@@ -95,6 +95,17 @@ DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split);
 // Record a message for tq_last_error() and return `st` (tq_api.cu).
 tq_status report_error(tq_status st, const char *fmt, ...);
 
+// TQ_OK when the current CUDA device is the one the context was created on;
+// otherwise TQ_ERR_INVALID (or TQ_ERR_CUDA) with a message (tq_api.cu).
+tq_status check_context_device(const tq_ctx *ctx);
+
+// Host-side caches of per-device facts (SM count, kernel attributes,
+// occupancy) are indexed by the device ordinal: cudaFuncSetAttribute and the
+// occupancy queries apply to the current device only.
+constexpr int kMaxDevices = 64;
+// The current device's ordinal, clamped into [0, kMaxDevices).
+int current_device();
+
 // --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);

@@ -30,7 +30,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ_NOALLOC_SCRA
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using tq::kMaxDevices;
 std::mutex g_scratch_mutex;
 void *g_scratch_address[kMaxDevices];
 
@@ -41,6 +41,10 @@ extern "C" tq_status tq_decode_attention_noalloc(tq_ctx *ctx, const tq_cache *ca
                                                  int32_t max_seq_len, float scale, float *out, float *lse,
                                                  void *stream) {
   if (!ctx || !cache) return tq::report_error(TQ_ERR_INVALID, "ctx and cache must be non-NULL");
+  // the scratch address below is looked up on the current device: it must be
+  // the context's, or the kernels would mix two GPUs' memory
+  const tq_status st = tq::check_context_device(ctx);
+  if (st != TQ_OK) return st;
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return tq::report_error(TQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));

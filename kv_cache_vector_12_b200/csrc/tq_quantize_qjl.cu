@@ -289,20 +289,21 @@ int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k,
                         const int32_t *pos, int n_tok, void *stream) {
   using Fn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, int);
   const Fn fn = p.bits_k == 2 ? quantize_qjl_kernel<2> : p.bits_k == 3 ? quantize_qjl_kernel<3> : quantize_qjl_kernel<4>;
-  // resident CTAs on the device, per bit width; cached atomically, as calls
-  // may come from several threads
-  static std::atomic<int> slots[5];
-  int n_slots = slots[p.bits_k].load(std::memory_order_relaxed);
+  // resident CTAs on the device, per bit width; cached per device (the
+  // attribute and the occupancy query apply to the current device) and
+  // atomically, as calls may come from several threads
+  static std::atomic<int> slots[kMaxDevices][3];
+  const int dev = current_device();
+  int n_slots = slots[dev][p.bits_k - 2].load(std::memory_order_relaxed);
   if (n_slots == 0) {
-    int dev = 0, n_sm = 0, per_sm = 0;
-    cudaGetDevice(&dev);
+    int n_sm = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kTabBytes);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 32 * kWarps, kTabBytes) != cudaSuccess ||
         per_sm < 1)
       per_sm = 1;
     n_slots = n_sm * per_sm;
-    slots[p.bits_k].store(n_slots, std::memory_order_relaxed);
+    slots[dev][p.bits_k - 2].store(n_slots, std::memory_order_relaxed);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   const long tiles = (rows + kRows - 1) / kRows;

@@ -579,20 +579,21 @@ QuantTcFn pick(int bk, int bv) { return bk == 2 ? pick_bv<2>(bv) : bk == 3 ? pic
 
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream) {
-  // cached atomically, as calls may come from several threads
-  static std::atomic<int> cached_sm{0};
-  static std::atomic<bool> configured[5][5];
-  int n_sm = cached_sm.load(std::memory_order_relaxed);
+  // cached per device (the attribute applies to the current device), and
+  // atomically, as calls may come from several threads
+  static std::atomic<int> cached_sm[kMaxDevices];
+  static std::atomic<bool> configured[kMaxDevices][3][3];
+  const int dev = current_device();
+  int n_sm = cached_sm[dev].load(std::memory_order_relaxed);
   if (n_sm == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
-    cached_sm.store(n_sm, std::memory_order_relaxed);
+    cached_sm[dev].store(n_sm, std::memory_order_relaxed);
   }
   const QuantTcFn fn = pick(p.bits_k, p.bits_v);
-  if (!configured[p.bits_k][p.bits_v].load(std::memory_order_acquire)) {
+  std::atomic<bool> &done = configured[dev][p.bits_k - 2][p.bits_v - 2];
+  if (!done.load(std::memory_order_acquire)) {
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
-    configured[p.bits_k][p.bits_v].store(true, std::memory_order_release);
+    done.store(true, std::memory_order_release);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   CUtensorMap mk, mv, mp;

@@ -376,6 +376,76 @@ def test_paged_block_table_out_of_range_is_flagged(tq):
     assert torch.all(torch.isfinite(out))
 
 
+@pytest.mark.parametrize("lens,block", [([60, 130, 1], 64), ([250, 3], 128)])
+def test_decode_paged_unassigned_blocks_past_length(tq, lens, block):
+    """Table entries of blocks that hold no position below a sequence's length
+    are never read: an engine may leave them -1, and decode neither flags them
+    nor reads through them."""
+    bits_k, bits_v, qjl, n_heads, group = 3, 3, 0, 2, 4
+    ctx = tq.Context(D, bits_k, bits_v, qjl, 42)
+    ref = oracle_params(bits_k, bits_v, qjl)
+    cap = 4 * block
+    per, planes, _ = _oracle_cache(ref, lens, n_heads, bits_k, bits_v, qjl, seed=17, min_cap=cap)
+    per_seq = cap // block
+    table = torch.full((len(lens), per_seq), -1, dtype=torch.int32)
+    n_blocks, nxt = len(lens) * per_seq, 0
+    for s, n in enumerate(lens):
+        for j in range((n + block - 1) // block):   # blocks holding a position below the length
+            table[s, j] = nxt
+            nxt += 1
+    cache = tq.PagedCache(ctx, len(lens), n_heads, cap, block, n_blocks=n_blocks, block_table=table)
+    tab = table.numpy()
+    for name, arr in planes.items():
+        if arr is None:
+            continue
+        a = arr.view(np.int16) if arr.dtype == np.uint16 else arr
+        phys = np.zeros((n_blocks, n_heads, block) + a.shape[3:], dtype=a.dtype)
+        for s in range(len(lens)):
+            for j in range(per_seq):
+                if tab[s, j] >= 0:
+                    phys[tab[s, j]] = a[s, :, j * block:(j + 1) * block]
+        cache.planes[name].copy_(torch.from_numpy(phys))
+    n_q = n_heads * group
+    q = torch.randn(len(lens), n_q, D, generator=torch.Generator().manual_seed(5))
+    out = torch.empty(len(lens), n_q, D, device="cuda")
+    lse = torch.empty(len(lens), n_q, device="cuda")
+    ws = tq.alloc_workspace(ctx, len(lens), n_q, cap)
+    tq.decode_attention(ctx, cache, q.cuda(), torch.tensor(lens, dtype=torch.int32, device="cuda"), cap, out, lse,
+                        ws)
+    ctx.check_device_errors()                       # no range flag for the -1 entries past the lengths
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for s in range(len(lens)):
+        for h in range(n_heads):
+            qk, qv = per[(s, h)]
+            rows = slice(h * group, (h + 1) * group)
+            o_ref, lse_ref, scores = o.decode_attention(q[s, rows].double().numpy(), ref.pi, ref.ck, qk.codes,
+                                                        qk.norm, ref.cv, qv.codes, qv.norm, 1 / math.sqrt(D))
+            ok, w = ph.attention_ok(out[s, rows], o_ref, lse[s, rows], lse_ref, np.abs(scores).max(axis=1))
+            assert ok, (s, h, w)
+
+
+def test_calls_on_another_device_are_rejected(tq):
+    """A context belongs to the device it was created on; compute calls made
+    while another device is current return TQ_ERR_INVALID and launch nothing."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two CUDA devices")
+    ctx = tq.Context(D, 3, 3, 0, 42)
+    cache = tq.Cache(ctx, 1, 1, 64)
+    k = torch.zeros(1, 1, D, dtype=torch.bfloat16, device="cuda:0")
+    idx = torch.zeros(1, dtype=torch.int32, device="cuda:0")
+    out = torch.empty(1, 1, D, device="cuda:0")
+    ws = tq.alloc_workspace(ctx, 1, 1, 64)
+    with torch.cuda.device(1):
+        for call in (lambda: tq.quantize(ctx, cache, k, k, idx, idx),
+                     lambda: tq.decode_attention(ctx, cache, torch.zeros(1, 1, D, device="cuda:0"), idx + 1, 64,
+                                                 out, None, ws),
+                     lambda: tq.decode_attention_noalloc(ctx, cache, torch.zeros(1, 1, D, device="cuda:0"),
+                                                         idx + 1, 64, out, None)):
+            with pytest.raises(tq.TQError) as ei:
+                call()
+            assert ei.value.status == tq.TQ_ERR_INVALID
+
+
 def test_paged_cache_argument_checks(tq):
     ctx = tq.Context(D, 3, 3, 0, 42)
     k = torch.zeros(1, 1, D, dtype=torch.bfloat16, device="cuda")
