@@ -45,6 +45,11 @@ Readings where the pages are silent (each also listed in the design notes):
 * decode: q_hat = Pi q, q_tilde = S q_hat, score
   s_j = scale * n_j * (q_hat . c_K[code_j] + QJL term), softmax over j,
   o_tilde = sum_j p_j nV_j c_V[codeV_j] in rotated space, o = Pi^T o_tilde.
+* prefill (prompt processing, whose cost over a compressed cache qxai.app's
+  "Tether QVACのTurboQuant実装", fifth paragraph, singles out): the chunk's
+  tokens are quantized into the cache first, then the query at position p
+  attends over the cached positions [0, p] (causal), each query exactly as
+  the decode above over that prefix.
 
 Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
 against closed forms, textbook values and brute force (no function is
@@ -475,6 +480,28 @@ def decode_attention(q, pi, centroids_k, codes_k, norm_k, centroids_v, codes_v, 
     o_tilde = (p * np.asarray(norm_v)[None, :]) @ np.asarray(centroids_v)[codes_v]
     o = (o_tilde / l[:, None]) @ pi          # row form of Pi^T o_tilde
     return o, m + np.log(l), scores
+
+
+def prefill_attention(q, q_pos, pi, centroids_k, codes_k, norm_k, centroids_v, codes_v, norm_v, scale,
+                      s_matrix=None, qjl_signs=None, qjl_gamma=None):
+    """Causal attention of a chunk of queries over one (sequence, KV head)'s
+    packed cache: the query at position q_pos[t] attends over the cached
+    positions [0, q_pos[t]], exactly as decode_attention over that prefix.
+
+    q [n, G, d] float64; q_pos [n] (each below the cached length); codes_*,
+    norm_*, qjl_* as decode_attention, over the whole cached sequence.
+    Returns (o [n, G, d], lse [n, G]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    o = np.empty(q.shape)
+    lse = np.empty(q.shape[:2])
+    for t, p in enumerate(np.asarray(q_pos, dtype=np.int64)):
+        n = int(p) + 1
+        o[t], lse[t], _ = decode_attention(
+            q[t], pi, centroids_k, codes_k[:n], norm_k[:n], centroids_v, codes_v[:n], norm_v[:n], scale,
+            s_matrix=s_matrix, qjl_signs=None if qjl_signs is None else qjl_signs[:n],
+            qjl_gamma=None if qjl_gamma is None else qjl_gamma[:n])
+    return o, lse
 
 
 def exact_attention(q, k, v, scale):

@@ -544,3 +544,52 @@ def test_exact_attention_definition():
 def test_cosine_similarity():
     assert o.cosine_similarity([1, 0], [2, 0]) == pytest.approx(1.0)
     assert o.cosine_similarity([1, 0], [0, 3]) == pytest.approx(0.0)
+
+
+# ----------------------------------------------------------------- prefill
+@pytest.mark.parametrize("qjl", [False, True])
+def test_prefill_is_causal_attention_over_explicit_dequantization(qjl):
+    """Every query of a prefill chunk equals plain causal softmax attention
+    over the vectors reconstructed in the original space (QJL residual
+    included), with the mask written out as a full score matrix: query t at
+    position p sees keys 0..p and nothing after."""
+    d, t_len, g = 32, 29, 2
+    p, _, k, v, qk, qv = _decode_case(d, t_len, g, 3, 2, qjl, 8)
+    rng = np.random.default_rng(81)
+    q_pos = np.array([3, 10, 11, 20, 28])                    # a chunk of positions inside the cache
+    q = rng.standard_normal((len(q_pos), g, d))
+    scale = 1 / math.sqrt(d)
+    o_pre, lse_pre = o.prefill_attention(q, q_pos, p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, scale,
+                                         s_matrix=p.s, qjl_signs=qk.qjl_signs, qjl_gamma=qk.qjl_gamma)
+    k_rec = o.dequantize(p.pi, p.ck, qk.codes, qk.norm)
+    if qjl:
+        pm = 2.0 * qk.qjl_signs - 1.0
+        k_rec = k_rec + qk.norm[:, None] * ((math.sqrt(math.pi / 2) / d * qk.qjl_gamma[:, None] * (pm @ p.s)) @ p.pi)
+    v_rec = o.dequantize(p.pi, p.cv, qv.codes, qv.norm)
+    for t, pos in enumerate(q_pos):
+        s_full = scale * q[t] @ k_rec.T                      # [g, t_len]
+        s_full[:, np.arange(t_len) > pos] = -np.inf           # causal mask
+        w = np.exp(s_full - s_full.max(axis=1, keepdims=True))
+        o_ref = (w @ v_rec) / w.sum(axis=1, keepdims=True)
+        lse_ref = s_full.max(axis=1) + np.log(w.sum(axis=1))
+        assert np.allclose(o_pre[t], o_ref, rtol=1e-11, atol=1e-12)
+        assert np.allclose(lse_pre[t], lse_ref, rtol=1e-12)
+
+
+def test_prefill_ignores_tokens_after_each_query():
+    """Causality: changing the cached tokens after a query's position leaves
+    that query's output unchanged, and the first position attends to itself
+    alone."""
+    d = 32
+    p, _, k, v, qk, qv = _decode_case(d, 16, 3, 2, 4, False, 9)
+    q = np.random.default_rng(4).standard_normal((3, 3, d))
+    q_pos = np.array([0, 7, 15])
+    args = (p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, 0.2)
+    o1, l1 = o.prefill_attention(q, q_pos, *args)
+    codes_k2, codes_v2 = qk.codes.copy(), qv.codes.copy()
+    codes_k2[8:] = (codes_k2[8:] + 1) % 4
+    codes_v2[8:] = (codes_v2[8:] + 5) % 16
+    o2, l2 = o.prefill_attention(q, q_pos, p.pi, p.ck, codes_k2, qk.norm, p.cv, codes_v2, qv.norm, 0.2)
+    assert np.array_equal(o1[:2], o2[:2]) and np.array_equal(l1[:2], l2[:2])
+    assert not np.allclose(o1[2], o2[2])
+    assert np.allclose(o1[0], np.repeat(o.dequantize(p.pi, p.cv, qv.codes[:1], qv.norm[:1]), 3, axis=0))
