@@ -90,6 +90,18 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s) for a kernel timed alone: the measured
+    burst figure, else the fallback measurement of this GPU type."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        if "bf16_tflops" in p:
+            return float(p["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -319,6 +331,39 @@ def quality_report(tq, ctx, cache, lens0, q_first, k_s0, v_s0, group, n_tokens=4
             "reference": "exact softmax attention in fp64 over the bf16 K/V rows"}
 
 
+def prefill_report(tq, ctx, cache, q_all, n_tok, n_q_heads, reps=3) -> dict:
+    """Causal prefill attention of the first n_tok positions of sequence 0 of
+    `cache` (every position a query; the cache holds the quantized prompt), as
+    one tq_prefill_attention call: median device time of `reps` calls (CUDA
+    events on the launching stream).  Logical flops per (query, key, query
+    head) = 4 d (2 d for the score, 2 d for the value accumulation)."""
+    dev = q_all.device
+    D = q_all.shape[-1]
+    B = cache.n_seqs
+    cu = torch.tensor([0] + [n_tok] * B, dtype=torch.int32, device=dev)   # only sequence 0 has queries
+    lens = torch.full((B,), n_tok, dtype=torch.int32, device=dev)
+    out = torch.empty(n_tok, n_q_heads, D, device=dev)
+    lse = torch.empty(n_tok, n_q_heads, device=dev)
+    tq.prefill_attention(ctx, cache, q_all, cu, lens, n_tok, n_tok, out, lse)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    for i in range(reps):
+        evs[2 * i].record()
+        tq.prefill_attention(ctx, cache, q_all, cu, lens, n_tok, n_tok, out, lse)
+        evs[2 * i + 1].record()
+    torch.cuda.synchronize()
+    ctx.check_device_errors()
+    ms = statistics.median(evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(reps))
+    flops = n_tok * (n_tok + 1) / 2 * n_q_heads * 4 * D
+    peak, kind = measured_tensor_peak()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"tokens": n_tok, "ms": ms, "tokens_per_s": n_tok / (ms * 1e-3), "logical_TFLOPs": tflops,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "peak_source": kind},
+            "call": f"tq_prefill_attention over the first {n_tok} positions of sequence 0 (every position a "
+                    f"query, causal), median of {reps}"}
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,6 +545,10 @@ def main(argv=None) -> int:
     dec_ms = [dec_total / args.steps]
     ctx.check_device_errors()
     quality = quality_report(tq, ctx, caches[0], lens0, q_all[args.warmup], k_s0, v_s0, w.group)
+    n_prefill = min(lens0[0], 32768)
+    q_prefill = wl.queries(w, n_prefill, gen, dev)                     # [n_prefill, HQ, D]
+    prefill = prefill_report(tq, ctx, caches[0], q_prefill, n_prefill, HQ)
+    del q_prefill
 
     breakdown = None
     if args.breakdown:
@@ -635,6 +684,7 @@ def main(argv=None) -> int:
                      "call": f"one tq_quantize of the whole prefill ({B} sequences, {n_pre} tokens x {H} KV heads), "
                              "median of 10"},
         "quality": quality,
+        "prefill": prefill,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,

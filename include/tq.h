@@ -235,6 +235,36 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache,
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Causal prefill (prompt) attention over the packed cache, the step that
+ * qxai.app ("Tether QVACのTurboQuant実装", fifth paragraph) names as where a
+ * compressed cache costs the most: the prompt's K and V are first quantized
+ * into the cache with tq_quantize, then every prompt token attends over the
+ * cached positions up to and including its own, reading the packed codes
+ * exactly as tq_decode_attention does (q_hat = Pi q, the same scores,
+ * softmax, V accumulation in rotated space, o = Pi^T o_tilde).  The bf16 K/V
+ * of the prompt is not read.  The queries of sequence s are rows
+ * cu_q[s] .. cu_q[s+1]-1 of q and sit at the last n_s = cu_q[s+1] - cu_q[s]
+ * positions of the sequence, seq_lens[s] - n_s .. seq_lens[s] - 1 (a whole
+ * prompt when n_s == seq_lens[s], a chunk of one otherwise); the query at
+ * position p attends over positions [0, p].
+ *  q        device [total][n_q_heads][d] of q_dtype, total = cu_q[n_seqs].
+ *  cu_q     device int32 [n_seqs + 1], cu_q[0] = 0, non-decreasing.
+ *  seq_lens device int32 [n_seqs], each at most max_seq_len (<= capacity).
+ *  max_q    host bound on every n_s (sizes the grid); max_seq_len likewise.
+ *  out      device fp32 [total][n_q_heads][d]; lse device fp32
+ *           [total][n_q_heads] or NULL.
+ * No workspace.  A sequence whose n_s or seq_lens is out of range gets no
+ * output and sets the seq_len flag of tq_check_device_errors.  Query heads
+ * per KV head at most 16.
+ */
+tq_status tq_prefill_attention(tq_ctx *ctx, const tq_cache *cache,
+                               const void *q, int32_t q_dtype,
+                               int32_t n_q_heads, const int32_t *cu_q,
+                               const int32_t *seq_lens, int32_t max_q,
+                               int32_t max_seq_len, float scale, float *out,
+                               float *lse, void *stream);
+
+/*
  * Allocation-free decode attention (no counterpart in the method's sources;
  * it is a deployment variant of tq_decode_attention).  For callers that cannot
  * allocate device memory while they decode: code inside CUDA graph stream

@@ -294,6 +294,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->law = law;
   ctx->seed = seed;
   ctx->dev_block = nullptr;
+  ctx->dp.s_shift = 0;
   ctx->pi_bits.resize((size_t)d * d);
   tq::rotation_bf16(d, seed, ctx->pi_bits.data());
   ctx->ck.assign(tq::kMaxLevels, 0.f);
@@ -361,6 +362,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     double smax = 0.0;
     for (size_t i = 0; i < dd; ++i) smax = std::max(smax, (double)std::fabs(ctx->s[i]));
     const int sigma = smax > 0.0 ? (int)std::floor(std::log2(32768.0 / smax)) : 0;
+    ctx->dp.s_shift = sigma;
     std::vector<uint16_t> part(dd);
     std::vector<double> rest(dd);
     for (size_t i = 0; i < dd; ++i) rest[i] = std::ldexp((double)ctx->s[i], sigma);
@@ -503,6 +505,37 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
   const int e = tq::launch_decode(ctx->dp, *cache, q, q_dtype, n_q_heads, seq_lens, max_seq_len, scale,
                                   out, lse, (char *)workspace, sp, ws, stream);
   if (e != 0) return cuda_fail((cudaError_t)e, "tq_decode_attention launch");
+  return TQ_OK;
+}
+
+tq_status tq_prefill_attention(tq_ctx *ctx, const tq_cache *cache, const void *q, int32_t q_dtype,
+                               int32_t n_q_heads, const int32_t *cu_q, const int32_t *seq_lens, int32_t max_q,
+                               int32_t max_seq_len, float scale, float *out, float *lse, void *stream) {
+  if (!ctx) return fail(TQ_ERR_INVALID, "ctx is NULL");
+  tq_status st = tq::check_context_device(ctx);
+  if (st != TQ_OK) return st;
+  st = check_cache(ctx, cache);
+  if (st != TQ_OK) return st;
+  if (!q || !cu_q || !seq_lens || !out) return fail(TQ_ERR_INVALID, "q, cu_q, seq_lens and out must be non-NULL");
+  if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID, "q_dtype=%d", q_dtype);
+  if (n_q_heads <= 0 || n_q_heads % cache->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "n_q_heads=%d must be a positive multiple of n_kv_heads=%d",
+                n_q_heads, cache->n_kv_heads);
+  if (n_q_heads / cache->n_kv_heads > 16)
+    return fail(TQ_ERR_UNSUPPORTED, "query heads per KV head = %d > 16", n_q_heads / cache->n_kv_heads);
+  if (max_seq_len < 0 || max_seq_len > cache->capacity)
+    return fail(TQ_ERR_INVALID, "max_seq_len=%d outside [0, capacity=%d]", max_seq_len, cache->capacity);
+  if (max_q < 0 || max_q > max_seq_len)
+    return fail(TQ_ERR_INVALID, "max_q=%d outside [0, max_seq_len=%d]", max_q, max_seq_len);
+  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)cu_q & 3u) || ((uintptr_t)seq_lens & 3u) ||
+      (lse && ((uintptr_t)lse & 3u)))
+    return fail(TQ_ERR_INVALID, "misaligned q/out (16 B) or cu_q/seq_lens/lse (4 B)");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
+  if (max_q == 0) return TQ_OK;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)ctx->d);
+  const int e = tq::launch_prefill(ctx->dp, *cache, q, q_dtype, n_q_heads, cu_q, seq_lens, max_q, max_seq_len,
+                                   scale, out, lse, stream);
+  if (e != 0) return cuda_fail((cudaError_t)e, "tq_prefill_attention launch");
   return TQ_OK;
 }
 

@@ -61,6 +61,7 @@ struct DeviceParams {
   const uint16_t *pivt;   // [d][d] bf16: pivt[i][k] = Pi[vperm[k]][i] (Pi^T, columns in V fragment order)
   Lut lut_k, lut_v;
   int bits_k, bits_v, qjl;
+  int s_shift;            // sigma of sf: the fragment tables hold S 2^sigma (qjl only)
 };
 
 // Fragment orders of the decode kernel (host, tq_api.cu).
@@ -120,6 +121,12 @@ int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k,
 // ks = (4 j + e) / 2 and b = (4 j + e) % 2, so a thread loads an n-tile's
 // fragments with four coalesced 16-byte loads (tq_api.cu).
 void mma_b_fragments(const uint16_t *m_bits, uint32_t *out);
+// Causal prefill attention over the packed cache (tq_prefill.cu): the queries
+// of sequence s are rows cu_q[s] .. cu_q[s + 1] - 1 of q, at the last
+// cu_q[s + 1] - cu_q[s] positions below seq_lens[s].
+int launch_prefill(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype, int n_q_heads,
+                   const int32_t *cu_q, const int32_t *seq_lens, int max_q, int max_seq_len, float scale,
+                   float *out, float *lse, void *stream);
 int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype,
                   int n_q_heads, const int32_t *seq_lens, int max_seq_len, float scale,
                   float *out, float *lse, char *workspace, const DecodeSplit &split,

@@ -59,6 +59,9 @@ lib.tq_decode_attention.restype = ctypes.c_int
 lib.tq_decode_attention_noalloc.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp, _i32,
                                             ctypes.c_float, _vp, _vp, _vp]
 lib.tq_decode_attention_noalloc.restype = ctypes.c_int
+lib.tq_prefill_attention.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp, _vp, _i32, _i32,
+                                     ctypes.c_float, _vp, _vp, _vp]
+lib.tq_prefill_attention.restype = ctypes.c_int
 lib.tq_check_device_errors.argtypes = [_vp, _vp]
 lib.tq_check_device_errors.restype = ctypes.c_int
 lib.tq_last_error.argtypes = []
@@ -237,6 +240,18 @@ def decode_attention(ctx: Context, cache: Cache, q: torch.Tensor, seq_lens: torc
                                    _ptr(seq_lens), max_seq_len, scale, _ptr(out), _ptr(lse),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)))
+
+
+def prefill_attention(ctx: Context, cache: Cache, q: torch.Tensor, cu_q: torch.Tensor, seq_lens: torch.Tensor,
+                      max_q: int, max_seq_len: int, out: torch.Tensor, lse: torch.Tensor | None = None,
+                      scale: float = 0.0, stream=None) -> None:
+    """tq_prefill_attention: q [total, n_q_heads, d] bf16 or fp32, the queries of
+    sequence s being rows cu_q[s]:cu_q[s+1] (its last positions below
+    seq_lens[s], already quantized into the cache); out fp32 [total, n_q_heads, d]."""
+    q_dtype = TQ_F32 if q.dtype == torch.float32 else TQ_BF16
+    _check(lib.tq_prefill_attention(ctx.handle, ctypes.byref(cache.struct), _ptr(q), q_dtype, q.shape[1],
+                                    _ptr(cu_q), _ptr(seq_lens), max_q, max_seq_len, scale, _ptr(out), _ptr(lse),
+                                    _stream(stream)))
 
 
 def decode_attention_noalloc(ctx: Context, cache: Cache, q: torch.Tensor, seq_lens: torch.Tensor,

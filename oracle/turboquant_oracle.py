@@ -490,18 +490,21 @@ def prefill_attention(q, q_pos, pi, centroids_k, codes_k, norm_k, centroids_v, c
 
     q [n, G, d] float64; q_pos [n] (each below the cached length); codes_*,
     norm_*, qjl_* as decode_attention, over the whole cached sequence.
-    Returns (o [n, G, d], lse [n, G]).
+    Returns (o [n, G, d], lse [n, G], max_abs_score [n, G]), the last being
+    max_j |s_j| over each query's prefix.
     """
     q = np.asarray(q, dtype=np.float64)
     o = np.empty(q.shape)
     lse = np.empty(q.shape[:2])
+    smax = np.empty(q.shape[:2])
     for t, p in enumerate(np.asarray(q_pos, dtype=np.int64)):
         n = int(p) + 1
-        o[t], lse[t], _ = decode_attention(
+        o[t], lse[t], sc = decode_attention(
             q[t], pi, centroids_k, codes_k[:n], norm_k[:n], centroids_v, codes_v[:n], norm_v[:n], scale,
             s_matrix=s_matrix, qjl_signs=None if qjl_signs is None else qjl_signs[:n],
             qjl_gamma=None if qjl_gamma is None else qjl_gamma[:n])
-    return o, lse
+        smax[t] = np.abs(sc).max(axis=1)
+    return o, lse, smax
 
 
 def exact_attention(q, k, v, scale):

@@ -559,7 +559,7 @@ def test_prefill_is_causal_attention_over_explicit_dequantization(qjl):
     q_pos = np.array([3, 10, 11, 20, 28])                    # a chunk of positions inside the cache
     q = rng.standard_normal((len(q_pos), g, d))
     scale = 1 / math.sqrt(d)
-    o_pre, lse_pre = o.prefill_attention(q, q_pos, p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, scale,
+    o_pre, lse_pre, _ = o.prefill_attention(q, q_pos, p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, scale,
                                          s_matrix=p.s, qjl_signs=qk.qjl_signs, qjl_gamma=qk.qjl_gamma)
     k_rec = o.dequantize(p.pi, p.ck, qk.codes, qk.norm)
     if qjl:
@@ -585,11 +585,11 @@ def test_prefill_ignores_tokens_after_each_query():
     q = np.random.default_rng(4).standard_normal((3, 3, d))
     q_pos = np.array([0, 7, 15])
     args = (p.pi, p.ck, qk.codes, qk.norm, p.cv, qv.codes, qv.norm, 0.2)
-    o1, l1 = o.prefill_attention(q, q_pos, *args)
+    o1, l1, _ = o.prefill_attention(q, q_pos, *args)
     codes_k2, codes_v2 = qk.codes.copy(), qv.codes.copy()
     codes_k2[8:] = (codes_k2[8:] + 1) % 4
     codes_v2[8:] = (codes_v2[8:] + 5) % 16
-    o2, l2 = o.prefill_attention(q, q_pos, p.pi, p.ck, codes_k2, qk.norm, p.cv, codes_v2, qv.norm, 0.2)
+    o2, l2, _ = o.prefill_attention(q, q_pos, p.pi, p.ck, codes_k2, qk.norm, p.cv, codes_v2, qv.norm, 0.2)
     assert np.array_equal(o1[:2], o2[:2]) and np.array_equal(l1[:2], l2[:2])
     assert not np.allclose(o1[2], o2[2])
     assert np.allclose(o1[0], np.repeat(o.dequantize(p.pi, p.cv, qv.codes[:1], qv.norm[:1]), 3, axis=0))
