@@ -265,6 +265,43 @@ tq_status tq_prefill_attention(tq_ctx *ctx, const tq_cache *cache,
                                float *lse, void *stream);
 
 /*
+ * Weight quantization with the same method (ai-accelerate.xyz TurboQuant
+ * explainer, "重みの量子化にも応用できる": the algorithm applied to the
+ * weights of a linear layer).  Every row of W (device, bf16, row-major
+ * [n_out][n_in]) is cut into n_in / d blocks of d coordinates, and every
+ * block is quantized as one vector with the context's K codebook (its norm,
+ * the rotation by Pi, bits_k-bit codes; no QJL, whatever the context's qjl).
+ * The packed rows go to a tq_cache `w` of one sequence whose KV heads are the
+ * blocks and whose positions are the rows: n_seqs = 1, n_kv_heads = n_in / d,
+ * capacity >= n_out (a multiple of 64), block_table NULL; only codes_k and
+ * norm_k are used (the other planes may be NULL).  Block b of row i is at
+ * position i of KV head b, in the cache's K layout.  d must be 128 and n_in
+ * a positive multiple of it.  Asynchronous on `stream`, allocates nothing.
+ */
+tq_status tq_weight_quantize(tq_ctx *ctx, const tq_cache *w, const void *w_rows,
+                             int32_t n_out, int32_t n_in, void *stream);
+
+/* Device workspace (bytes) that tq_weight_gemm needs for n_tok rows of x. */
+size_t tq_weight_workspace_bytes(const tq_ctx *ctx, int32_t n_tok, int32_t n_in);
+
+/*
+ * y = x W~^T over weights packed by tq_weight_quantize, W~ being the rows as
+ * the method reconstructs them (each block n_b Pi^T c[codes_b]).  The product
+ * runs in rotated space and never rebuilds W~:
+ *   y[t][i] = sum_b n_ib (Pi x[t][block b]) . c[code_ib].
+ *  x         device [n_tok][n_in] of x_dtype (TQ_BF16 or TQ_F32).
+ *  y         device fp32 [n_tok][n_out] (overwritten).
+ *  workspace device, at least tq_weight_workspace_bytes(ctx, n_tok, n_in)
+ *            bytes, 256-byte aligned; contents need no initialisation.
+ * n_tok at most 65520.  Sums over blocks are fp32 and combined with atomic
+ * adds, so the last bits of y may differ between runs.
+ */
+tq_status tq_weight_gemm(tq_ctx *ctx, const tq_cache *w, int32_t n_out,
+                         int32_t n_in, const void *x, int32_t x_dtype,
+                         int32_t n_tok, float *y, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
  * Allocation-free decode attention (no counterpart in the method's sources;
  * it is a deployment variant of tq_decode_attention).  For callers that cannot
  * allocate device memory while they decode: code inside CUDA graph stream

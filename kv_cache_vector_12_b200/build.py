@@ -21,7 +21,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtq.so")
 
 SOURCES = ["tq_host.cpp", "tq_fragments.cpp", "tq_api.cu", "tq_kernels.cu", "tq_quantize_tc.cu", "tq_quantize_qjl.cu", "tq_decode.cu",
-           "tq_prefill.cu", "tq_noalloc.cu"]
+           "tq_prefill.cu", "tq_weight.cu", "tq_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           "-I" + os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]

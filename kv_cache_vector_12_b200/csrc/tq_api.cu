@@ -37,12 +37,27 @@ uint16_t exact_half_bits(float f) {
   return (uint16_t)(sign | ((uint32_t)exp << 10) | ((u & 0x7fffffu) >> 13));
 }
 
+// The largest shift k <= 17 with every K centroid c 2^k an integer in
+// [-32767, 32767] (exact 16-bit fixed point), or -1 if none from 17 down to 8.
+int k_fixed_shift(const float *ck, int bits_k) {
+  for (int k = 17; k >= 8; --k) {
+    bool ok = true;
+    for (int e = 0; e < (1 << bits_k) && ok; ++e) {
+      const double scaled = std::ldexp((double)ck[e], k);
+      ok = std::nearbyint(scaled) == scaled && std::fabs(scaled) <= 32767.0;
+    }
+    if (ok) return k;
+  }
+  return -1;
+}
+
 // Byte tables of the decode kernel's lookups (see tq_internal.h).
-bool build_luts(const float *ck, int bits_k, const float *cv, int bits_v, tq::Lut &lk, tq::Lut &lv) {
+bool build_luts(const float *ck, int bits_k, int k_shift, const float *cv, int bits_v, tq::Lut &lk, tq::Lut &lv) {
   std::memset(&lk, 0, sizeof lk);
   std::memset(&lv, 0, sizeof lv);
+  if (k_shift < 0) return false;
   for (int e = 0; e < (1 << bits_k); ++e) {
-    const double scaled = std::ldexp((double)ck[e], tq::kKFixedShift);
+    const double scaled = std::ldexp((double)ck[e], k_shift);
     const long v = std::lrint(scaled);
     if ((double)v != scaled || v > 32767 || v < -32767) return false;  // not exact 16-bit fixed point
     lk.lo[e / 4] |= (uint32_t)(v & 0xff) << (8 * (e % 4));
@@ -56,10 +71,10 @@ bool build_luts(const float *ck, int bits_k, const float *cv, int bits_v, tq::Lu
   return true;
 }
 
-bool is_permutation(const uint8_t *p) {
-  bool seen[tq::kHeadDim] = {};
-  for (int i = 0; i < tq::kHeadDim; ++i) {
-    if (p[i] >= tq::kHeadDim || seen[p[i]]) return false;
+bool is_permutation(const uint8_t *p, int d) {
+  bool seen[256] = {};
+  for (int i = 0; i < d; ++i) {
+    if (p[i] >= d || seen[p[i]]) return false;
     seen[p[i]] = true;
   }
   return true;
@@ -91,7 +106,7 @@ tq_status check_params(int d, int bits_k, int bits_v, int qjl, int law) {
   if (bits_k < 2 || bits_k > 4 || bits_v < 2 || bits_v > 4)
     return fail(TQ_ERR_INVALID, "bits_k=%d bits_v=%d: each must be 2, 3 or 4", bits_k, bits_v);
   if (qjl != 0 && qjl != 1) return fail(TQ_ERR_INVALID, "qjl=%d must be 0 or 1", qjl);
-  if (d != tq::kHeadDim) return fail(TQ_ERR_UNSUPPORTED, "d=%d: only d=128 is implemented", d);
+  if (!tq::supported_head_dim(d)) return fail(TQ_ERR_UNSUPPORTED, "d=%d: the head dimension must be 64, 128 or 256", d);
   return TQ_OK;
 }
 
@@ -185,22 +200,23 @@ constexpr int kLongSplitTokens = 8192;
 
 // The split is planned for the 3-CTA budget first; a call that meets neither
 // condition runs the 2-CTA budget instead, re-split for that occupancy.
-DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len,
-                        bool paged) {
-  if (paged) {  // the paged build has the 3-CTA budget only
-    DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group,
-                                                                                      true, true));
+DecodeSplit plan_decode(int d, int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads,
+                        int max_seq_len, bool paged) {
+  if (paged) {  // the paged build has one budget
+    DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len,
+                                  decode_ctas_per_sm(d, bits_k, bits_v, qjl, group, true, true));
     sp.long_splits = true;
     return sp;
   }
-  const int ctas = decode_ctas_per_sm(bits_k, bits_v, qjl, group, true, false);
+  const int ctas = decode_ctas_per_sm(d, bits_k, bits_v, qjl, group, true, false);
   DecodeSplit sp = decode_split(n_seqs, n_kv_heads, max_seq_len, ctas);
   const long grid = (long)sp.n_splits * n_seqs * n_kv_heads;
   if (grid >= 2L * sm_count() * ctas || sp.chunk >= kLongSplitTokens) {
     sp.long_splits = true;
     return sp;
   }
-  return decode_split(n_seqs, n_kv_heads, max_seq_len, decode_ctas_per_sm(bits_k, bits_v, qjl, group, false, false));
+  return decode_split(n_seqs, n_kv_heads, max_seq_len,
+                      decode_ctas_per_sm(d, bits_k, bits_v, qjl, group, false, false));
 }
 
 tq_status report_error(tq_status st, const char *fmt, ...) {
@@ -211,23 +227,24 @@ tq_status report_error(tq_status st, const char *fmt, ...) {
   return st;
 }
 
-void mma_b_fragments(const uint16_t *m_bits, uint32_t *out) {
-  for (int nt = 0; nt < 16; ++nt)
-    for (int j = 0; j < 4; ++j)
+void mma_b_fragments(const uint16_t *m_bits, int d, uint32_t *out) {
+  const int chunks = d / 32;
+  for (int nt = 0; nt < d / 8; ++nt)
+    for (int j = 0; j < chunks; ++j)
       for (int lane = 0; lane < 32; ++lane)
         for (int e = 0; e < 4; ++e) {
           const int ks = (4 * j + e) / 2, b = (4 * j + e) % 2;
-          const uint16_t *src = m_bits + (size_t)(8 * nt + lane / 4) * kHeadDim + 16 * ks + 8 * b + 2 * (lane % 4);
-          out[((nt * 4 + j) * 32 + lane) * 4 + e] = (uint32_t)src[0] | ((uint32_t)src[1] << 16);
+          const uint16_t *src = m_bits + (size_t)(8 * nt + lane / 4) * d + 16 * ks + 8 * b + 2 * (lane % 4);
+          out[((nt * chunks + j) * 32 + lane) * 4 + e] = (uint32_t)src[0] | ((uint32_t)src[1] << 16);
         }
 }
 
-DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split) {
+DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split, int d) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t rows = (size_t)n_seqs * n_q_heads;
   DecodeWorkspace w;
   w.partials = 0;
-  w.total = up(rows * (size_t)split.n_splits * kPartialFloats * sizeof(float));
+  w.total = up(rows * (size_t)split.n_splits * (size_t)(d + 4) * sizeof(float));
   return w;
 }
 
@@ -258,7 +275,7 @@ tq_status tq_host_params_ex(int32_t d, int32_t bits_k, int32_t bits_v, int32_t q
   float c[tq::kMaxLevels], t[tq::kMaxLevels];
   for (const int b : {bits_k, bits_v}) {
     tq::codebook(b, d, law, c, t);
-    if (!tq::threshold_search_exact(b, t))
+    if (d == tq::kHeadDim && !tq::threshold_search_exact(b, t))
       return fail(TQ_ERR_UNSUPPORTED, "%d-bit thresholds: the quantize search is not exact in fp32", b);
   }
   if (centroids_k || thresholds_k) {
@@ -303,7 +320,8 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->tv.assign(tq::kMaxLevels, 0.f);
   tq::codebook(bits_k, d, law, ctx->ck.data(), ctx->tk.data());
   tq::codebook(bits_v, d, law, ctx->cv.data(), ctx->tv.data());
-  if (!tq::threshold_search_exact(bits_k, ctx->tk.data()) || !tq::threshold_search_exact(bits_v, ctx->tv.data())) {
+  if (d == tq::kHeadDim &&
+      (!tq::threshold_search_exact(bits_k, ctx->tk.data()) || !tq::threshold_search_exact(bits_v, ctx->tv.data()))) {
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "thresholds: the quantize search is not exact in fp32");
   }
@@ -317,12 +335,13 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     delete ctx;
     return cuda_fail(e, "cudaGetDevice");
   }
-  uint8_t kperm[tq::kHeadDim], vperm[tq::kHeadDim], jperm[tq::kHeadDim];
-  tq::kperm_of(bits_k, kperm);
-  tq::vperm_of(bits_v, vperm);
-  tq::jperm_of(jperm);
-  if (!is_permutation(kperm) || !is_permutation(vperm) || !is_permutation(jperm) ||
-      !build_luts(ctx->ck.data(), bits_k, ctx->cv.data(), bits_v, ctx->dp.lut_k, ctx->dp.lut_v)) {
+  uint8_t kperm[256], vperm[256], jperm[256];
+  tq::kperm_of(bits_k, d, kperm);
+  tq::vperm_of(bits_v, d, vperm);
+  tq::jperm_of(d, jperm);
+  ctx->dp.k_shift = k_fixed_shift(ctx->ck.data(), bits_k);
+  if (!is_permutation(kperm, d) || !is_permutation(vperm, d) || !is_permutation(jperm, d) ||
+      !build_luts(ctx->ck.data(), bits_k, ctx->dp.k_shift, ctx->cv.data(), bits_v, ctx->dp.lut_k, ctx->dp.lut_v)) {
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
@@ -347,9 +366,9 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     std::vector<uint16_t> pik(dd);
     for (int kap = 0; kap < d; ++kap)
       std::memcpy(pik.data() + (size_t)kap * d, ctx->pi_bits.data() + (size_t)kperm[kap] * d, (size_t)d * 2);
-    tq::mma_b_fragments(pik.data(), (uint32_t *)(h.data() + off_pik));
+    tq::mma_b_fragments(pik.data(), d, (uint32_t *)(h.data() + off_pik));
   }
-  tq::mma_b_fragments(ctx->pi_bits.data(), (uint32_t *)(h.data() + off_pif));
+  tq::mma_b_fragments(ctx->pi_bits.data(), d, (uint32_t *)(h.data() + off_pif));
   if (qjl) {
     std::memcpy(h.data() + off_s, ctx->s.data(), dd * 4);
     float *sjk = (float *)(h.data() + off_sjk);
@@ -371,14 +390,14 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
         part[i] = tq::double_to_half_bits(rest[i]);
         rest[i] -= tq::half_bits_to_double(part[i]);
       }
-      tq::mma_b_fragments(part.data(), (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
+      tq::mma_b_fragments(part.data(), d, (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
     }
   }
   uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
   for (int i = 0; i < d; ++i)
     for (int k = 0; k < d; ++k) pivt[(size_t)i * d + k] = ctx->pi_bits[(size_t)vperm[k] * d + i];
-  std::memcpy(h.data() + off_kperm, kperm, tq::kHeadDim);
-  std::memcpy(h.data() + off_jperm, jperm, tq::kHeadDim);
+  std::memcpy(h.data() + off_kperm, kperm, (size_t)d);
+  std::memcpy(h.data() + off_jperm, jperm, (size_t)d);
   float *cb = (float *)(h.data() + off_cb);
   std::memcpy(cb + 0 * tq::kMaxLevels, ctx->ck.data(), tq::kMaxLevels * 4);
   std::memcpy(cb + 1 * tq::kMaxLevels, ctx->tk.data(), tq::kMaxLevels * 4);
@@ -402,14 +421,15 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->dp.pivt = (const uint16_t *)(base + off_piv);
   ctx->dp.kperm = (const uint8_t *)(base + off_kperm);
   ctx->dp.jperm = (const uint8_t *)(base + off_jperm);
+  ctx->dp.d = d;
   ctx->dp.bits_k = bits_k;
   ctx->dp.bits_v = bits_v;
   ctx->dp.qjl = qjl;
   // resolve the decode kernels' occupancy now, outside any stream capture
   for (const bool long_splits : {false, true})
     for (const bool paged : {false, true}) {
-      tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 8, long_splits, paged);
-      tq::decode_ctas_per_sm(bits_k, bits_v, qjl, 16, long_splits, paged);
+      tq::decode_ctas_per_sm(d, bits_k, bits_v, qjl, 8, long_splits, paged);
+      tq::decode_ctas_per_sm(d, bits_k, bits_v, qjl, 16, long_splits, paged);
     }
   *out = ctx;
   return TQ_OK;
@@ -423,11 +443,11 @@ void tq_destroy(tq_ctx *ctx) {
 
 tq_status tq_layout(const tq_ctx *ctx, size_t b[6]) {
   if (!ctx || !b) return fail(TQ_ERR_INVALID, "ctx or output is NULL");
-  b[TQ_PLANE_CODES_K] = (size_t)tq::code_bytes(ctx->bits_k);
+  b[TQ_PLANE_CODES_K] = (size_t)tq::code_bytes(ctx->bits_k, ctx->d);
   b[TQ_PLANE_NORM_K] = 2;
-  b[TQ_PLANE_QJL_BITS] = ctx->qjl ? tq::kHeadDim / 8 : 0;
+  b[TQ_PLANE_QJL_BITS] = ctx->qjl ? (size_t)ctx->d / 8 : 0;
   b[TQ_PLANE_QJL_NORM] = ctx->qjl ? 2 : 0;
-  b[TQ_PLANE_CODES_V] = (size_t)tq::code_bytes(ctx->bits_v);
+  b[TQ_PLANE_CODES_V] = (size_t)tq::code_bytes(ctx->bits_v, ctx->d);
   b[TQ_PLANE_NORM_V] = 2;
   return TQ_OK;
 }
@@ -469,7 +489,7 @@ size_t tq_workspace_bytes(const tq_ctx *ctx, int32_t n_seqs, int32_t n_q_heads, 
   // The split count falls as the (sequence, KV head) units grow and rises with
   // CTAs per SM; one KV head and the largest occupancy bound it from above.
   const tq::DecodeSplit sp = tq::decode_split(n_seqs, 1, max_seq_len, 4);
-  return tq::decode_workspace(n_seqs, n_q_heads, sp).total;
+  return tq::decode_workspace(n_seqs, n_q_heads, sp, ctx->d).total;
 }
 
 tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q, int32_t q_dtype,
@@ -496,9 +516,9 @@ tq_status tq_decode_attention(tq_ctx *ctx, const tq_cache *cache, const void *q,
     return fail(TQ_ERR_INVALID, "misaligned q/out (16 B), workspace (256 B) or seq_lens/lse (4 B)");
   if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID, "scale is not finite");
   const int group = n_q_heads / cache->n_kv_heads;
-  const tq::DecodeSplit sp = tq::plan_decode(ctx->bits_k, ctx->bits_v, ctx->qjl, group, cache->n_seqs,
+  const tq::DecodeSplit sp = tq::plan_decode(ctx->d, ctx->bits_k, ctx->bits_v, ctx->qjl, group, cache->n_seqs,
                                              cache->n_kv_heads, max_seq_len, cache->block_table != nullptr);
-  const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, sp);
+  const tq::DecodeWorkspace ws = tq::decode_workspace(cache->n_seqs, n_q_heads, sp, ctx->d);
   if (workspace_bytes < ws.total)
     return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, ws.total);
   if (scale <= 0.f) scale = 1.0f / std::sqrt((float)ctx->d);
@@ -517,6 +537,8 @@ tq_status tq_prefill_attention(tq_ctx *ctx, const tq_cache *cache, const void *q
   st = check_cache(ctx, cache);
   if (st != TQ_OK) return st;
   if (!q || !cu_q || !seq_lens || !out) return fail(TQ_ERR_INVALID, "q, cu_q, seq_lens and out must be non-NULL");
+  if (ctx->d != tq::kHeadDim)
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: prefill attention is implemented for d = 128", ctx->d);
   if (q_dtype != TQ_BF16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID, "q_dtype=%d", q_dtype);
   if (n_q_heads <= 0 || n_q_heads % cache->n_kv_heads != 0)
     return fail(TQ_ERR_INVALID, "n_q_heads=%d must be a positive multiple of n_kv_heads=%d",
@@ -536,6 +558,63 @@ tq_status tq_prefill_attention(tq_ctx *ctx, const tq_cache *cache, const void *q
   const int e = tq::launch_prefill(ctx->dp, *cache, q, q_dtype, n_q_heads, cu_q, seq_lens, max_q, max_seq_len,
                                    scale, out, lse, stream);
   if (e != 0) return cuda_fail((cudaError_t)e, "tq_prefill_attention launch");
+  return TQ_OK;
+}
+
+namespace {
+
+tq_status check_weight_args(const tq_ctx *ctx, const tq_cache *w, int32_t n_out, int32_t n_in) {
+  if (!ctx || !w) return fail(TQ_ERR_INVALID, "ctx and w must be non-NULL");
+  tq_status st = tq::check_context_device(ctx);
+  if (st != TQ_OK) return st;
+  if (ctx->d != tq::kHeadDim) return fail(TQ_ERR_UNSUPPORTED, "d=%d: weight rows are implemented for d = 128", ctx->d);
+  if (n_out <= 0 || n_in <= 0 || n_in % ctx->d != 0)
+    return fail(TQ_ERR_INVALID, "n_out=%d n_in=%d: both positive, n_in a multiple of d=%d", n_out, n_in, ctx->d);
+  if (w->n_seqs != 1 || w->n_kv_heads != n_in / ctx->d || w->block_table)
+    return fail(TQ_ERR_INVALID, "w must hold one sequence of n_in / d = %d KV heads, contiguous", n_in / ctx->d);
+  if (w->capacity < n_out || w->capacity % 64 != 0)
+    return fail(TQ_ERR_INVALID, "capacity=%d must be a multiple of 64 and at least n_out=%d", w->capacity, n_out);
+  if (!w->codes_k || !w->norm_k || !aligned16(w->codes_k) || !aligned16(w->norm_k))
+    return fail(TQ_ERR_INVALID, "codes_k and norm_k must be non-NULL and 16-byte aligned");
+  return TQ_OK;
+}
+
+}  // namespace
+
+tq_status tq_weight_quantize(tq_ctx *ctx, const tq_cache *w, const void *w_rows, int32_t n_out, int32_t n_in,
+                             void *stream) {
+  tq_status st = check_weight_args(ctx, w, n_out, n_in);
+  if (st != TQ_OK) return st;
+  if (!w_rows || !aligned16(w_rows)) return fail(TQ_ERR_INVALID, "w_rows must be non-NULL and 16-byte aligned");
+  tq::DeviceParams p = ctx->dp;
+  p.qjl = 0;  // weights keep the MSE codes only
+  const long rows = (long)n_out * (n_in / ctx->d);
+  const int e = rows <= 1024 ? tq::launch_quantize_rows_k(p, *w, w_rows, nullptr, nullptr, n_out, stream)
+                             : tq::launch_quantize_tc(p, *w, w_rows, w_rows, nullptr, nullptr, n_out, true, false,
+                                                      stream);
+  if (e != 0) return cuda_fail((cudaError_t)e, "tq_weight_quantize launch");
+  return TQ_OK;
+}
+
+size_t tq_weight_workspace_bytes(const tq_ctx *ctx, int32_t n_tok, int32_t n_in) {
+  if (!ctx || n_tok <= 0 || n_in <= 0 || n_in % ctx->d != 0) return 0;
+  return tq::weight_workspace_bytes(n_tok, n_in);
+}
+
+tq_status tq_weight_gemm(tq_ctx *ctx, const tq_cache *w, int32_t n_out, int32_t n_in, const void *x,
+                         int32_t x_dtype, int32_t n_tok, float *y, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+  tq_status st = check_weight_args(ctx, w, n_out, n_in);
+  if (st != TQ_OK) return st;
+  if (!x || !y || !workspace) return fail(TQ_ERR_INVALID, "x, y and workspace must be non-NULL");
+  if (x_dtype != TQ_BF16 && x_dtype != TQ_F32) return fail(TQ_ERR_INVALID, "x_dtype=%d", x_dtype);
+  if (n_tok <= 0 || n_tok > 65520) return fail(TQ_ERR_INVALID, "n_tok=%d outside [1, 65520]", n_tok);
+  if (((uintptr_t)x & 3u) || ((uintptr_t)y & 3u) || ((uintptr_t)workspace & 255u))
+    return fail(TQ_ERR_INVALID, "misaligned x/y (4 B) or workspace (256 B)");
+  const size_t need = tq::weight_workspace_bytes(n_tok, n_in);
+  if (workspace_bytes < need) return fail(TQ_ERR_INVALID, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
+  const int e = tq::launch_weight_gemm(ctx->dp, *w, n_out, n_in, x, x_dtype, n_tok, y, (char *)workspace, stream);
+  if (e != 0) return cuda_fail((cudaError_t)e, "tq_weight_gemm launch");
   return TQ_OK;
 }
 

@@ -47,6 +47,8 @@ constexpr int kWarpTokens = 32;                            // tokens per consume
 constexpr int kStageTokens = kWarpTokens * kConsumerWarps;  // 128
 constexpr int kStages = 4;
 constexpr int kPrefetchTokens = kStages * kStageTokens;  // L2 prefetch before the dependency wait
+// ring depth: d = 256 stages are twice as large, so two of them
+constexpr int stages_of(int dh) { return dh == 256 ? 2 : kStages; }
 
 // Barrier of the four consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumer_sync() {
@@ -64,6 +66,78 @@ struct DecodeArgs {
   float *partials;        // [rows][n_splits][d + 4]
 };
 
+// Per-thread K words and selectors of the score MMAs for head dimension DH.
+// The int8 MMA's k index kappa = 32 s + 16 slot + 4 q + i is byte i of the
+// A register (k-step s, slot) of the threads with q = lane % 4:
+//   DH = 128: thread q holds coordinate group q (32 codes, BK words) and
+//             register (s, slot) is selector 2 s + slot of that group;
+//   DH = 256: groups q and q + 4 (2 BK words); k-steps 4 H .. 4 H + 3 read
+//             group q + 4 H, selector 2 (s % 4) + slot;
+//   DH = 64:  half q % 2 of group q / 2: selectors 4 (q % 2) + 2 s + slot.
+template <int BK, int DH>
+struct KWords {
+  static constexpr int n = DH == 256 ? 2 * BK : BK;  // words loaded per token
+  // byte offset of the thread's words inside a token's code row
+  __device__ __forceinline__ static int offset(int q) {
+    if constexpr (DH == 64) return BK == 3 ? 12 * (q >> 1) : q * 2 * BK;
+    else return q * 4 * BK;
+  }
+  __device__ __forceinline__ static void load(const unsigned char *row, int q, uint32_t (&w)[n]) {
+    const uint32_t *p = reinterpret_cast<const uint32_t *>(row + offset(q));
+    if constexpr (DH == 256) {
+      const uint32_t *p2 = reinterpret_cast<const uint32_t *>(row + 16 * BK + offset(q));
+#pragma unroll
+      for (int i = 0; i < BK; ++i) {
+        w[i] = p[i];
+        w[BK + i] = p2[i];
+      }
+    } else if constexpr (DH == 64 && BK != 3) {
+#pragma unroll
+      for (int i = 0; i < BK / 2; ++i) w[i] = p[i];
+#pragma unroll
+      for (int i = BK / 2; i < BK; ++i) w[i] = 0u;
+    } else {
+#pragma unroll
+      for (int i = 0; i < BK; ++i) w[i] = p[i];
+    }
+  }
+  // selector of register (s, slot); s and slot are compile-time after unrolling
+  __device__ __forceinline__ static uint32_t sel(const uint32_t (&w)[n], int s, int slot, int q) {
+    if constexpr (DH == 128) {
+      return k_selector<BK>(w, 2 * s + slot);
+    } else if constexpr (DH == 256) {
+      uint32_t wh[BK];
+#pragma unroll
+      for (int i = 0; i < BK; ++i) wh[i] = w[(s >= 4 ? BK : 0) + i];
+      return k_selector<BK>(wh, 2 * (s & 3) + slot);
+    } else {
+      const int j = 2 * s + slot;
+      if constexpr (BK == 3) {
+        const bool odd = (q & 1) != 0;
+        const uint32_t x = j < 2 ? (odd ? w[2] & 0x77777777u : w[0] & 0x77777777u)
+                                 : (odd ? spare3(w[0], w[1], w[2]) : w[1] & 0x77777777u);
+        return (j & 1) ? x >> 16 : x;
+      } else {
+        return k_selector<BK>(w, j);
+      }
+    }
+  }
+};
+
+// The QJL sign word of register (s, slot) and the bit inside its bytes: the
+// register holds bits j, j + 8, j + 16, j + 24 of word `wd` of the token's
+// sign row (DH / 32 words).
+template <int DH>
+__device__ __forceinline__ void qjl_pick(int s, int slot, int q, int &wd, int &j) {
+  if constexpr (DH == 64) {
+    wd = q >> 1;
+    j = 4 * (q & 1) + 2 * s + slot;
+  } else {
+    wd = q + 4 * (s / 4);
+    j = 2 * (s & 3) + slot;
+  }
+}
+
 // Two register budgets of the same kernel, chosen per call from the split
 // length (tq_api.cu): CTAS = 2 (168 registers) for short splits, where fewer
 // CTAs amortise the per-CTA prologue and each warp has room for more
@@ -73,17 +147,25 @@ struct DecodeArgs {
 // PAGED selects the paged cache layout (the stage copies follow the block
 // table); it is its own instantiation so that the contiguous kernels keep
 // their code and register allocation.
-template <int BK, int BV, bool QJL, int NT, int CTAS, bool PAGED>
+template <int BK, int BV, bool QJL, int NT, int CTAS, bool PAGED, int DH>
 __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const DecodeArgs a) {
   static_assert(kStageTokens % 64 == 0 && kWarpTokens == 32, "stages start on 64-token boundaries");
-  using St = Stage<BK, BV, QJL, kStageTokens>;
+  static_assert(DH == 64 || DH == 128 || DH == 256, "head dimension");
+  using St = Stage<BK, BV, QJL, kStageTokens, DH>;
   constexpr int kRows = 8 * NT;  // query-head rows of the score MMAs
+  constexpr int KS = DH / 32;    // int8 k-steps of the scores
+  constexpr int MT = DH / 16;    // m-tiles (16 coordinates) of the values
+  constexpr int NTW = DH / 32;   // q-rotation n-tiles per consumer warp (DH / 4 positions)
+  constexpr int KR = DH / 16;    // q-rotation k-steps
+  constexpr bool kHoldPi = DH <= 128;  // Pi's fragments held in registers from before the dependency wait
+  constexpr int D = DH;                // (shadows the library-wide 128 inside this kernel)
+  constexpr int kStages = stages_of(DH);
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ int abort_flag;
   __shared__ float sm_m[kConsumerWarps][kRows], sm_l[kConsumerWarps][kRows];
-  __shared__ __align__(16) uint8_t s_q8[kRows][QJL ? 4 : 2][D];  // q_hat hi, lo; q_tilde hi, lo (fragment orders)
-  __shared__ __align__(16) float s_qf[QJL ? kRows : 1][D];       // q_hat, fp32, K order (QJL input)
+  __shared__ __align__(16) uint8_t s_q8[kRows][QJL ? 4 : 2][DH];  // q_hat hi, lo; q_tilde hi, lo (fragment orders)
+  __shared__ __align__(16) float s_qf[QJL ? kRows : 1][DH];       // q_hat, fp32, K order (QJL input)
   __shared__ float s_qs[kRows][4];                                // score factor, QJL factor, sum of q_tilde ints
   __shared__ float s_red[kConsumerWarps][kRows];
 
@@ -92,15 +174,15 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
   const int r = lane >> 2, q = lane & 3;
   const int G = a.n_q_heads / a.c.n_kv_heads;
   // B fragments of Pi (rows in the K fragment order) for this consumer warp's
-  // 32 output positions: parameters, loaded before waiting for the previous
-  // kernel in the stream
-  uint32_t bfr[4][8][2];
-  if (warp < kConsumerWarps) {
+  // DH / 4 output positions: parameters, loaded before waiting for the
+  // previous kernel in the stream (DH = 256: read during the rotation)
+  uint32_t bfr[kHoldPi ? NTW : 1][kHoldPi ? KR : 1][2];
+  if (kHoldPi && warp < kConsumerWarps) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[((warp * 4 + nt) * 4 + j) * 32 + lane];
+      for (int j = 0; j < KR / 2; ++j) {
+        const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[((warp * NTW + nt) * (KR / 2) + j) * 32 + lane];
         bfr[nt][2 * j][0] = v.x;
         bfr[nt][2 * j][1] = v.y;
         bfr[nt][2 * j + 1][0] = v.z;
@@ -114,8 +196,8 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
   // split's whole range (below the length bound and the capacity) is fetched.
   if (warp == kConsumerWarps && lane == 0) {
     // this KV head's query rows and the sequence length (read right after the wait)
-    const size_t qbytes = (size_t)G * D * (a.q_dtype == TQ_F32 ? 4 : 2);
-    prefetch_l2(static_cast<const char *>(a.q) + ((size_t)s * a.n_q_heads + (size_t)h * G) * D *
+    const size_t qbytes = (size_t)G * DH * (a.q_dtype == TQ_F32 ? 4 : 2);
+    prefetch_l2(static_cast<const char *>(a.q) + ((size_t)s * a.n_q_heads + (size_t)h * G) * DH *
                                                      (a.q_dtype == TQ_F32 ? 4 : 2),
                 (uint32_t)qbytes);
     asm volatile("prefetch.global.L2 [%0];" ::"l"(a.seq_lens + s));
@@ -125,12 +207,12 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     if (!PAGED && first < last) {
       const long tok = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + first;
       const uint32_t n = (uint32_t)(last - first);
-      prefetch_l2(a.c.codes_k + tok * (D * BK / 8), n * (D * BK / 8));
-      prefetch_l2(a.c.codes_v + tok * (D * BV / 8), n * (D * BV / 8));
+      prefetch_l2(a.c.codes_k + tok * (DH * BK / 8), n * (DH * BK / 8));
+      prefetch_l2(a.c.codes_v + tok * (DH * BV / 8), n * (DH * BV / 8));
       prefetch_l2(a.c.norm_k + tok, (n * 2 + 15) & ~15u);
       prefetch_l2(a.c.norm_v + tok, (n * 2 + 15) & ~15u);
       if constexpr (QJL) {
-        prefetch_l2(a.c.qjl_bits + tok * (D / 8), n * (D / 8));
+        prefetch_l2(a.c.qjl_bits + tok * (DH / 8), n * (DH / 8));
         prefetch_l2(a.c.qjl_norm + tok, (n * 2 + 15) & ~15u);
       }
     }
@@ -232,17 +314,17 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     // m16n8k16 bf16 with the heads as rows and the K fragment positions as
     // columns (Pi's rows are stored in that order), fp32 q split into a bf16
     // hi + lo pair so every product is exact and the sums are fp32.  Warp w
-    // computes positions 32 w .. 32 w + 31.
+    // computes positions (D / 4) w .. (D / 4) w + D / 4 - 1.
     {
       const long qrow0 = (long)s * a.n_q_heads + (long)h * G;
       const bool f32 = a.q_dtype == TQ_F32;
-      float c[4][4];
+      float c[NTW][4];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
+      for (int ks = 0; ks < KR; ++ks) {
         uint32_t ahi[4], alo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {  // a0: row r; a1: row r + 8; a2, a3: the same rows, columns + 8
@@ -262,15 +344,25 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
           split_bf16x2(x0, x1, ahi[e], alo[e]);
         }
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          mma_bf16(c[nt], ahi[0], ahi[1], ahi[2], ahi[3], bfr[nt][ks][0], bfr[nt][ks][1]);
-          if (f32) mma_bf16(c[nt], alo[0], alo[1], alo[2], alo[3], bfr[nt][ks][0], bfr[nt][ks][1]);
+        for (int nt = 0; nt < NTW; ++nt) {
+          uint32_t b0, b1;
+          if constexpr (kHoldPi) {
+            b0 = bfr[nt][ks][0];
+            b1 = bfr[nt][ks][1];
+          } else {
+            const uint2 v = reinterpret_cast<const uint2 *>(
+                a.p.pikf)[(((warp * NTW + nt) * (KR / 2) + ks / 2) * 32 + lane) * 2 + (ks & 1)];
+            b0 = v.x;
+            b1 = v.y;
+          }
+          mma_bf16(c[nt], ahi[0], ahi[1], ahi[2], ahi[3], b0, b1);
+          if (f32) mma_bf16(c[nt], alo[0], alo[1], alo[2], alo[3], b0, b1);
         }
       }
       // per head: mu = 32767 / max |q_hat|, q_hat as 16-bit fixed point (hi, lo bytes)
       float mx0 = 0.f, mx1 = 0.f;  // rows r, r + 8
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
+      for (int nt = 0; nt < NTW; ++nt) {
         mx0 = fmaxf(mx0, fmaxf(fabsf(c[nt][0]), fabsf(c[nt][1])));
         mx1 = fmaxf(mx1, fmaxf(fabsf(c[nt][2]), fabsf(c[nt][3])));
       }
@@ -293,8 +385,8 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         mu[e] = m > 0.f ? 32767.f / m : 1.f;
       }
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int kap = 32 * warp + 8 * nt + 2 * q;
+      for (int nt = 0; nt < NTW; ++nt) {
+        const int kap = (D / 4) * warp + 8 * nt + 2 * q;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           if (kRows <= 8 && e == 1) break;
@@ -306,30 +398,40 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         }
       }
       if (warp == 0 && q == 0) {
-        s_qs[r][0] = a.scale * kLog2e / (mu[0] * (float)(1 << kKFixedShift));
-        if constexpr (kRows > 8) s_qs[r + 8][0] = a.scale * kLog2e / (mu[1] * (float)(1 << kKFixedShift));
+        s_qs[r][0] = a.scale * kLog2e / (mu[0] * ldexpf(1.f, a.p.k_shift));
+        if constexpr (kRows > 8) s_qs[r + 8][0] = a.scale * kLog2e / (mu[1] * ldexpf(1.f, a.p.k_shift));
       }
       if constexpr (QJL) {
-        // q_tilde = S q_hat: position tid (QJL fragment order) of every head,
-        // from row tid of S permuted into the QJL (rows) and K (columns) orders
+        // q_tilde = S q_hat: positions tid (+ 128) (QJL fragment order) of
+        // every head, from rows of S permuted into the QJL (rows) and K
+        // (columns) orders
         consumer_sync();
-        float qt[kRows];
+        constexpr int PP = D >= 128 ? D / 128 : 1;  // positions per consumer thread
+        float qt[PP][kRows];
 #pragma unroll
-        for (int g = 0; g < kRows; ++g) qt[g] = 0.f;
-        const float4 *srow = reinterpret_cast<const float4 *>(a.p.sjk + tid * D);
+        for (int pp = 0; pp < PP; ++pp) {
+#pragma unroll
+          for (int g = 0; g < kRows; ++g) qt[pp][g] = 0.f;
+          const int pos = tid + 128 * pp;
+          if (pos < D) {
+            const float4 *srow = reinterpret_cast<const float4 *>(a.p.sjk + pos * D);
 #pragma unroll 4
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-          const float4 w4 = srow[c4];
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+              const float4 w4 = srow[c4];
 #pragma unroll
-          for (int g = 0; g < kRows; ++g) {
-            const float4 x = *reinterpret_cast<const float4 *>(&s_qf[g][4 * c4]);
-            qt[g] = fmaf(w4.x, x.x, fmaf(w4.y, x.y, fmaf(w4.z, x.z, fmaf(w4.w, x.w, qt[g]))));
+              for (int g = 0; g < kRows; ++g) {
+                const float4 x = *reinterpret_cast<const float4 *>(&s_qf[g][4 * c4]);
+                qt[pp][g] = fmaf(w4.x, x.x, fmaf(w4.y, x.y, fmaf(w4.z, x.z, fmaf(w4.w, x.w, qt[pp][g]))));
+              }
+            }
           }
         }
         // nu = 32767 / max |q_tilde| per head, then the ints and their sum
 #pragma unroll
         for (int g = 0; g < kRows; ++g) {
-          float m = fabsf(qt[g]);
+          float m = 0.f;
+#pragma unroll
+          for (int pp = 0; pp < PP; ++pp) m = fmaxf(m, fabsf(qt[pp][g]));
 #pragma unroll
           for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
           if (lane == 0) s_red[warp][g] = m;
@@ -345,13 +447,20 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         consumer_sync();  // s_red is reused for the sums
 #pragma unroll
         for (int g = 0; g < kRows; ++g) {
-          const int vi = (int)rintf(qt[g] * nu[g]);
-          s_q8[g][2][tid] = (uint8_t)(vi >> 8);
-          s_q8[g][3][tid] = (uint8_t)(vi & 0xFF);
-          int sum = vi;
+          int sum = 0;
+#pragma unroll
+          for (int pp = 0; pp < PP; ++pp) {
+            const int pos = tid + 128 * pp;
+            if (pos < D) {
+              const int vi = (int)rintf(qt[pp][g] * nu[g]);
+              s_q8[g][2][pos] = (uint8_t)(vi >> 8);
+              s_q8[g][3][pos] = (uint8_t)(vi & 0xFF);
+              sum += vi;
+            }
+          }
 #pragma unroll
           for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          if (lane == 0) s_red[warp][g] = (float)sum;  // |sum| < 2^22: exact
+          if (lane == 0) s_red[warp][g] = (float)sum;  // |sum| < 2^23: exact
         }
         consumer_sync();
         if (tid < kRows) s_qs[tid][2] = (s_red[0][tid] + s_red[1][tid]) + (s_red[2][tid] + s_red[3][tid]);
@@ -359,13 +468,13 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
       consumer_sync();
     }
     // q fragments (int8, K fragment order) of this thread's head r in every n-tile
-    uint32_t qh[NT][4][2], ql[NT][4][2], jh[NT][QJL ? 4 : 1][2], jl[NT][QJL ? 4 : 1][2];
+    uint32_t qh[NT][KS][2], ql[NT][KS][2], jh[NT][QJL ? KS : 1][2], jl[NT][QJL ? KS : 1][2];
     float fq[NT][2], fj[NT][2], jsum[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint8_t *qb = &s_q8[8 * nt + r][0][0];
 #pragma unroll
-      for (int st = 0; st < 4; ++st)
+      for (int st = 0; st < KS; ++st)
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
           const int off = 32 * st + 16 * sl + 4 * q;
@@ -386,7 +495,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     }
     const Lut lk = a.p.lut_k, lv = a.p.lut_v;
 
-    float m_run[NT][2], l_run[NT][2], acc[NT][8][4];
+    float m_run[NT][2], l_run[NT][2], acc[NT][MT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -395,7 +504,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         l_run[nt][e] = 0.f;
       }
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
     }
@@ -411,7 +520,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
       const int tok0 = t0 + it * kStageTokens + kWarpTokens * warp;  // first token of this warp's tile
       if (tok0 < t1) {
         const int wt = kWarpTokens * warp;                             // tile row offset inside the stage
-        // ---------------- scores: int8 MMA, two 16-token row blocks, 4 k-steps of 32
+        // ---------------- scores: int8 MMA, two 16-token row blocks, D / 32 k-steps of 32
         int chh[2][NT][4], cmid[2][NT][4], cll[2][NT][4], cjh[2][NT][4], cjl[2][NT][4];
 #pragma unroll
         for (int rb = 0; rb < 2; ++rb)
@@ -421,21 +530,18 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
             for (int e = 0; e < 4; ++e) chh[rb][nt][e] = cmid[rb][nt][e] = cll[rb][nt][e] = cjh[rb][nt][e] = cjl[rb][nt][e] = 0;
 #pragma unroll
         for (int rb = 0; rb < 2; ++rb) {
-          uint32_t wk0[BK], wk1[BK];
-          const unsigned char *kr0 = st + St::kc + (wt + 16 * rb + r) * (D * BK / 8) + q * 4 * BK;
-          const unsigned char *kr1 = kr0 + 8 * (D * BK / 8);
+          using KW = KWords<BK, D>;
+          uint32_t wk0[KW::n], wk1[KW::n];
+          const unsigned char *kr0 = st + St::kc + (wt + 16 * rb + r) * (D * BK / 8);
+          KW::load(kr0, q, wk0);
+          KW::load(kr0 + 8 * (D * BK / 8), q, wk1);
 #pragma unroll
-          for (int i = 0; i < BK; ++i) {
-            wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
-            wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
-          }
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
+          for (int ks = 0; ks < KS; ++ks) {
             uint32_t alo[4], ahi[4];
-            lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks), alo[0], ahi[0]);
-            lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks), alo[1], ahi[1]);
-            lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks + 1), alo[2], ahi[2]);
-            lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks + 1), alo[3], ahi[3]);
+            lookup<BK>(lk, KW::sel(wk0, ks, 0, q), alo[0], ahi[0]);
+            lookup<BK>(lk, KW::sel(wk1, ks, 0, q), alo[1], ahi[1]);
+            lookup<BK>(lk, KW::sel(wk0, ks, 1, q), alo[2], ahi[2]);
+            lookup<BK>(lk, KW::sel(wk1, ks, 1, q), alo[3], ahi[3]);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               mma_i8<true, true>(chh[rb][nt], ahi[0], ahi[1], ahi[2], ahi[3], qh[nt][ks][0], qh[nt][ks][1]);
@@ -445,14 +551,16 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
             }
           }
           if constexpr (QJL) {
-            const uint32_t w0 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + 16 * rb + r) * (D / 8))[q];
-            const uint32_t w1 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + 16 * rb + r + 8) * (D / 8))[q];
+            const uint32_t *jr0 = reinterpret_cast<const uint32_t *>(st + St::jb + (wt + 16 * rb + r) * (D / 8));
+            const uint32_t *jr1 = jr0 + 8 * (D / 32);  // token + 8 (D / 32 words per token)
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              // bytes 0x00 / 0xFF (= -bit) for bits j, j+8, j+16, j+24 with j = 2 ks + slot
-              const int j0 = 2 * ks, j1 = 2 * ks + 1;
-              const uint32_t a0 = prmt(w0 << (7 - j0), 0u, 0xBA98u), a1 = prmt(w1 << (7 - j0), 0u, 0xBA98u);
-              const uint32_t a2 = prmt(w0 << (7 - j1), 0u, 0xBA98u), a3 = prmt(w1 << (7 - j1), 0u, 0xBA98u);
+            for (int ks = 0; ks < KS; ++ks) {
+              // bytes 0x00 / 0xFF (= -bit) for bits j, j+8, j+16, j+24 of word wd
+              int wd0, j0, wd1, j1;
+              qjl_pick<D>(ks, 0, q, wd0, j0);
+              qjl_pick<D>(ks, 1, q, wd1, j1);
+              const uint32_t a0 = prmt(jr0[wd0] << (7 - j0), 0u, 0xBA98u), a1 = prmt(jr1[wd0] << (7 - j0), 0u, 0xBA98u);
+              const uint32_t a2 = prmt(jr0[wd1] << (7 - j1), 0u, 0xBA98u), a3 = prmt(jr1[wd1] << (7 - j1), 0u, 0xBA98u);
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 mma_i8<true, true>(cjh[rb][nt], a0, a1, a2, a3, jh[nt][ks][0], jh[nt][ks][1]);
@@ -540,7 +648,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
+            for (int mt = 0; mt < MT; ++mt) {
               acc[nt][mt][0] *= alpha[nt][0];
               acc[nt][mt][1] *= alpha[nt][1];
               acc[nt][mt][2] *= alpha[nt][0];
@@ -548,84 +656,148 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
             }
         }
         // ---------------- values: fp16 MMA, k-step rb covers tokens 16 rb .. 16 rb + 15;
-        // tokens (2q, 2q+1) and (2q+8, 2q+9) of each k-step, unit r of 16 coordinates
+        // tokens (2q, 2q+1) and (2q+8, 2q+9) of each k-step; per 128-coordinate
+        // half, unit r of 16 coordinates (D = 64: unit r of 8 coordinates)
         constexpr int VB = D * BV / 8;
 #pragma unroll
         for (int rb = 0; rb < 2; ++rb) {
-          const unsigned char *vt = st + St::vc + (wt + 16 * rb + 2 * q) * VB;
-          if constexpr (BV == 3) {
-            const int gofs = 12 * (r >> 1);
-            const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
-            uint32_t ya[3], yb[3];
+          const unsigned char *vt0 = st + St::vc + (wt + 16 * rb + 2 * q) * VB;
+          if constexpr (D == 64) {
+            if constexpr (BV == 3) {
+              // byte r % 4 of each word of group r / 4: codes 8 k + 2 (r % 4) (x) and + 1 (y)
+              const int gofs = 12 * (r >> 2), b = r & 3;
+              const uint32_t gs = (uint32_t)(b | ((4 + b) << 4));
+              uint32_t ya[3], yb[3];
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
-              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt + gofs)[k];
-              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k];
-              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k];
-              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k];
-              ya[k] = prmt(A0, B0, gs);
-              yb[k] = prmt(A1, B1, gs);
-            }
-            const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+              for (int k = 0; k < 3; ++k) {
+                const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt0 + gofs)[k];
+                const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt0 + VB + gofs)[k];
+                const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt0 + 8 * VB + gofs)[k];
+                const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt0 + 9 * VB + gofs)[k];
+                ya[k] = prmt(A0, B0, gs);
+                yb[k] = prmt(A1, B1, gs);
+              }
+              const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
-              const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+                const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
                 uint32_t a0, a1, a2, a3;
-                v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
-                v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
+                v_pairs<3>(lv, za, a0, a1);
+                v_pairs<3>(lv, zb, a2, a3);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                  mma_f16(acc[nt][2 * k + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                  mma_f16(acc[nt][k], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
               }
-            }
-          } else if constexpr (BV == 2) {
-            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
-            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
-            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
-            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
+            } else {
+              // 2 bits: bytes 2 (r % 2), + 1 of word r / 2; 4 bits: word r
+              const int wd = BV == 2 ? (r >> 1) : r;
+              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt0)[wd];
+              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt0 + VB)[wd];
+              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt0 + 8 * VB)[wd];
+              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt0 + 9 * VB)[wd];
 #pragma unroll
-            for (int yh = 0; yh < 2; ++yh) {
-              const uint32_t gs = yh ? 0x7362u : 0x5140u;
-              const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+              for (int yh = 0; yh < 2; ++yh) {
+                if (BV == 2 && yh == 1) break;
+                const uint32_t gs = (BV == 2 ? (r & 1) : yh) ? 0x7362u : 0x5140u;
+                const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
 #pragma unroll
-              for (int par = 0; par < 2; ++par) {
-                const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
+                for (int par = 0; par < (BV == 2 ? 2 : 1); ++par) {
+                  const uint32_t za = BV == 2 ? (ya >> (2 * par)) & 0x33333333u : ya;
+                  const uint32_t zb = BV == 2 ? (yb >> (2 * par)) & 0x33333333u : yb;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  uint32_t a0, a1, a2, a3;
-                  v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
-                  v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+                  for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a0, a1, a2, a3;
+                    v_pairs<BV>(lv, hh ? za >> 16 : za, a0, a1);
+                    v_pairs<BV>(lv, hh ? zb >> 16 : zb, a2, a3);
+                    const int mt = BV == 2 ? 2 * par + hh : 2 * yh + hh;
 #pragma unroll
-                  for (int nt = 0; nt < NT; ++nt)
-                    mma_f16(acc[nt][4 * yh + 2 * par + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                    for (int nt = 0; nt < NT; ++nt)
+                      mma_f16(acc[nt][mt], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                  }
                 }
               }
             }
           } else {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
-              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
-              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
-              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+          for (int hv = 0; hv < D / 128; ++hv) {
+            const unsigned char *vt = vt0 + hv * 16 * BV;
+            if constexpr (BV == 3) {
+              const int gofs = 12 * (r >> 1);
+              const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
+              uint32_t ya[3], yb[3];
+#pragma unroll
+              for (int k = 0; k < 3; ++k) {
+                const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt + gofs)[k];
+                const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k];
+                const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k];
+                const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k];
+                ya[k] = prmt(A0, B0, gs);
+                yb[k] = prmt(A1, B1, gs);
+              }
+              const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+                const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  uint32_t a0, a1, a2, a3;
+                  v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
+                  v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(acc[nt][8 * hv + 2 * k + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                }
+              }
+            } else if constexpr (BV == 2) {
+              const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
+              const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
+              const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
+              const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
 #pragma unroll
               for (int yh = 0; yh < 2; ++yh) {
                 const uint32_t gs = yh ? 0x7362u : 0x5140u;
                 const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  uint32_t a0, a1, a2, a3;
-                  v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
-                  v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+                for (int par = 0; par < 2; ++par) {
+                  const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
 #pragma unroll
-                  for (int nt = 0; nt < NT; ++nt)
-                    mma_f16(acc[nt][4 * u + 2 * yh + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                  for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a0, a1, a2, a3;
+                    v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
+                    v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                      mma_f16(acc[nt][8 * hv + 4 * yh + 2 * par + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                  }
+                }
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
+                const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
+                const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
+                const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+#pragma unroll
+                for (int yh = 0; yh < 2; ++yh) {
+                  const uint32_t gs = yh ? 0x7362u : 0x5140u;
+                  const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+                  for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a0, a1, a2, a3;
+                    v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
+                    v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                      mma_f16(acc[nt][8 * hv + 4 * u + 2 * yh + hh], a0, a1, a2, a3, pb[rb][nt][0], pb[rb][nt][1]);
+                  }
                 }
               }
             }
+
+          }
           }
         }
       }
@@ -651,7 +823,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         }
       }
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
+      for (int mt = 0; mt < MT; ++mt) {
         float *o0 = so + ((warp * 8 * NT) + 8 * nt + 2 * q) * D + 16 * mt + r;
         o0[0] = acc[nt][mt][0];
         o0[D] = acc[nt][mt][1];
@@ -679,7 +851,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
       l = fmaf(f, sm_l[w][g], l);
       o = fmaf(f, so[(w * 8 * NT + g) * D + i], o);
     }
-    float *dst = a.partials + (((long)s * a.n_q_heads + h * G + g) * a.n_splits + split) * kPartialFloats;
+    float *dst = a.partials + (((long)s * a.n_q_heads + h * G + g) * a.n_splits + split) * (D + 4);
     dst[4 + i] = o;
     if (i == 0) {
       dst[0] = mx;
@@ -701,19 +873,35 @@ __device__ __forceinline__ float block_max128(float v, float *red) {
   return r;
 }
 
-// A bf16 row of 128 entries (16-byte aligned) as 16 independent 16-byte loads.
-__device__ __forceinline__ void load_bf16_row(const uint16_t *row, uint4 (&w)[16]) {
+// A bf16 row of DH entries (16-byte aligned): held in registers as
+// independent 16-byte loads (DH <= 128, loaded ahead of use) or read on the
+// fly (DH = 256).
+template <int DH>
+struct Bf16Row {
+  static constexpr int kHeld = DH <= 128 ? DH / 8 : 1;
+  uint4 w[kHeld];
+  const uint16_t *row;
+  __device__ __forceinline__ void load(const uint16_t *r) {
+    row = r;
+    if constexpr (DH <= 128) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) w[c] = reinterpret_cast<const uint4 *>(row)[c];
-}
+      for (int c = 0; c < DH / 8; ++c) w[c] = reinterpret_cast<const uint4 *>(r)[c];
+    }
+  }
+  __device__ __forceinline__ uint4 get(int c) const {
+    if constexpr (DH <= 128) return w[c];
+    else return reinterpret_cast<const uint4 *>(row)[c];
+  }
+};
 
-// Dot product of a loaded bf16 row with a vector in shared memory, four
-// partial sums.
-__device__ __forceinline__ float dot_bf16_row(const uint4 (&w)[16], const float *x) {
+// Dot product of a bf16 row with a vector in shared memory, four partial sums.
+template <int DH>
+__device__ __forceinline__ float dot_bf16_row(const Bf16Row<DH> &w, const float *x) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+  for (int c = 0; c < DH / 8; ++c) {
+    const uint4 v = w.get(c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int j = 8 * c + 2 * e;
@@ -724,45 +912,65 @@ __device__ __forceinline__ float dot_bf16_row(const uint4 (&w)[16], const float 
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
+// PL consecutive floats (PL * 4-byte aligned) as vector loads.
+template <int PL>
+__device__ __forceinline__ void load_floats(const float *src, float (&v)[PL]) {
+  if constexpr (PL == 2) {
+    const float2 x = *reinterpret_cast<const float2 *>(src);
+    v[0] = x.x, v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int c = 0; c < PL / 4; ++c) {
+      const float4 x = reinterpret_cast<const float4 *>(src)[c];
+      v[4 * c] = x.x, v[4 * c + 1] = x.y, v[4 * c + 2] = x.z, v[4 * c + 3] = x.w;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // merge: per (sequence, query head) combine the splits (log-sum-exp in log2
-// units) and apply Pi^T: o_i = sum_k Pi[vperm(k)][i] o~_k / L.
+// units) and apply Pi^T: o_i = sum_k Pi[vperm(k)][i] o~_k / L.  128 threads;
+// thread t owns outputs t (and t + 128 for DH = 256).
 // ---------------------------------------------------------------------------
 constexpr int kMergeMaxSplits = 1024;
 
+template <int DH>
 __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_heads, const int32_t *seq_lens,
                                                     int max_seq_len, int chunk, int n_splits,
                                                     const float *partials, float *out, float *lse) {
-  __shared__ float s_ot[D];
+  constexpr int PF = DH + 4;                      // floats per split partial: m, l, 2 unused, DH outputs
+  constexpr int PL = DH / 32;                     // outputs per lane in the split loads
+  constexpr int kOPerWarp = DH == 256 ? 8 : 16;   // splits per warp held in registers
+  __shared__ float s_ot[DH];
   __shared__ float s_w[kMergeMaxSplits], s_l[kMergeMaxSplits];
-  __shared__ __align__(16) float s_acc[4][D];
+  __shared__ __align__(16) float s_acc[4][DH];
   __shared__ float red[4];
   const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // this thread's row of Pi^T does not depend on the attention kernel: load it
-  // before waiting for that kernel to complete
-  uint4 pw[16];
-  load_bf16_row(p.pivt + tid * D, pw);
+  // this thread's rows of Pi^T do not depend on the attention kernel: load
+  // them before waiting for that kernel to complete
+  Bf16Row<DH> pw0, pw1;
+  if (tid < DH) pw0.load(p.pivt + tid * DH);
+  if constexpr (DH == 256) pw1.load(p.pivt + (tid + 128) * DH);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // the next kernel in the stream (an append, the next decode) may launch and
   // load its parameters now; it waits for this grid before reading anything
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int s = row / n_q_heads;
-  const float *src = partials + (long)row * n_splits * kPartialFloats;
+  const float *src = partials + (long)row * n_splits * PF;
   // One round of loads: the sequence length, and warp w's outputs of splits
-  // w, w + 4, ... (lane j: outputs 4 j .. 4 j + 3) of every allocated split,
-  // requested before any of them is used; splits past the used ones are
-  // ignored below (their slots may hold anything).
-  constexpr int kOPerWarp = 16;  // splits per warp held in registers
-  float4 o4[kOPerWarp];
+  // w, w + 4, ... (lane j: outputs PL j .. PL j + PL - 1) of every allocated
+  // split, requested before any of them is used; splits past the used ones
+  // are ignored below (their slots may hold anything).
+  float ov[kOPerWarp][PL];
 #pragma unroll
   for (int e = 0; e < kOPerWarp; ++e) {
     const int sp = warp + 4 * e;
-    if (sp < n_splits) o4[e] = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
+    if (sp < n_splits) load_floats<PL>(src + sp * PF + 4 + lane * PL, ov[e]);
   }
   // and thread t's (m, l) pair of split t, so that the pairs of the first 128
   // splits do not wait for the sequence length
   float2 ml0 = make_float2(-INFINITY, 0.f);
-  if (tid < n_splits) ml0 = *reinterpret_cast<const float2 *>(src + tid * kPartialFloats);
+  if (tid < n_splits) ml0 = *reinterpret_cast<const float2 *>(src + tid * PF);
   int len = seq_lens[s];
   len = len < 0 ? 0 : (len > max_seq_len ? max_seq_len : len);
   const int used = min((len + chunk - 1) / chunk, kMergeMaxSplits);
@@ -773,7 +981,7 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
     mloc = ml0.x;
   }
   for (int sp = tid + 128; sp < used; sp += 128) {
-    const float2 ml = *reinterpret_cast<const float2 *>(src + sp * kPartialFloats);
+    const float2 ml = *reinterpret_cast<const float2 *>(src + sp * PF);
     s_w[sp] = ml.x;
     s_l[sp] = ml.y;
     mloc = fmaxf(mloc, ml.x);
@@ -786,44 +994,47 @@ __global__ void __launch_bounds__(128) merge_kernel(DeviceParams p, int n_q_head
     lpart = fmaf(w, s_l[sp], lpart);
   }
   __syncthreads();
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[PL];
+#pragma unroll
+  for (int c = 0; c < PL; ++c) acc[c] = 0.f;
 #pragma unroll
   for (int e = 0; e < kOPerWarp; ++e) {
     const int sp = warp + 4 * e;
     if (sp < used) {
       const float w = s_w[sp];
-      acc.x = fmaf(w, o4[e].x, acc.x);
-      acc.y = fmaf(w, o4[e].y, acc.y);
-      acc.z = fmaf(w, o4[e].z, acc.z);
-      acc.w = fmaf(w, o4[e].w, acc.w);
+#pragma unroll
+      for (int c = 0; c < PL; ++c) acc[c] = fmaf(w, ov[e][c], acc[c]);
     }
   }
   // splits beyond 4 * kOPerWarp (long sequences with short splits)
   for (int sp = warp + 4 * kOPerWarp; sp < used; sp += 4) {
-    const float4 v = reinterpret_cast<const float4 *>(src + sp * kPartialFloats + 4)[lane];
+    float v[PL];
+    load_floats<PL>(src + sp * PF + 4 + lane * PL, v);
     const float w = s_w[sp];
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
+#pragma unroll
+    for (int c = 0; c < PL; ++c) acc[c] = fmaf(w, v[c], acc[c]);
   }
-  reinterpret_cast<float4 *>(s_acc[warp])[lane] = acc;
+#pragma unroll
+  for (int c = 0; c < PL; ++c) s_acc[warp][lane * PL + c] = acc[c];
   for (int o = 16; o; o >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, o);
   if (lane == 0) red[warp] = lpart;
   __syncthreads();
   const float ll = (red[0] + red[1]) + (red[2] + red[3]);
-  const float oo = (s_acc[0][tid] + s_acc[1][tid]) + (s_acc[2][tid] + s_acc[3][tid]);
-  s_ot[tid] = ll > 0.f ? oo / ll : 0.f;
+  for (int i = tid; i < DH; i += 128) {
+    const float oo = (s_acc[0][i] + s_acc[1][i]) + (s_acc[2][i] + s_acc[3][i]);
+    s_ot[i] = ll > 0.f ? oo / ll : 0.f;
+  }
   __syncthreads();
   // o_i = sum_k Pi^T[i][k] o~_k with Pi^T's columns in the V fragment order
-  out[(long)row * D + tid] = dot_bf16_row(pw, s_ot);
+  if (tid < DH) out[(long)row * DH + tid] = dot_bf16_row<DH>(pw0, s_ot);
+  if constexpr (DH == 256) out[(long)row * DH + tid + 128] = dot_bf16_row<DH>(pw1, s_ot);
   if (lse && tid == 0) lse[row] = ll > 0.f ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int BK, int BV, bool QJL, int NT>
+template <int BK, int BV, bool QJL, int NT, int DH>
 constexpr int decode_smem_bytes() {
-  const int ring = kStages * Stage<BK, BV, QJL, kStageTokens>::bytes;
-  const int park = kConsumerWarps * 8 * NT * D * 4;
+  const int ring = stages_of(DH) * Stage<BK, BV, QJL, kStageTokens, DH>::bytes;
+  const int park = kConsumerWarps * 8 * NT * DH * 4;
   return ring > park ? ring : park;
 }
 
@@ -834,60 +1045,78 @@ struct Variant {
   int smem;
 };
 
-// Budgets: kShort (2 CTAs per SM), kLong (3 CTAs per SM) on the contiguous
-// layout; kPaged, the paged layout, which always runs the 3-CTA budget (its
-// callers decode batches of many sequences).
+// Budgets at d = 128: kShort (2 CTAs per SM), kLong (3 CTAs per SM) on the
+// contiguous layout; kPaged, the paged layout, which always runs the 3-CTA
+// budget (its callers decode batches of many sequences).  At d = 256 every
+// build runs the 168-register budget (twice the value accumulators), at
+// d = 64 the 128-register one; kShort and kLong are then the same kernel.
 enum Build { kShort = 0, kLong = 1, kPaged = 2 };
 
-template <int BK, int BV, bool QJL, int NT>
+template <int BK, int BV, bool QJL, int NT, int DH>
 Variant variant_c(int build) {
-  constexpr int smem = decode_smem_bytes<BK, BV, QJL, NT>();
-  if (build == kPaged) return {decode_mma_kernel<BK, BV, QJL, NT, 3, true>, smem};
-  if (build == kLong) return {decode_mma_kernel<BK, BV, QJL, NT, 3, false>, smem};
-  return {decode_mma_kernel<BK, BV, QJL, NT, 2, false>, smem};
+  constexpr int smem = decode_smem_bytes<BK, BV, QJL, NT, DH>();
+  if constexpr (DH == 128) {
+    if (build == kPaged) return {decode_mma_kernel<BK, BV, QJL, NT, 3, true, DH>, smem};
+    if (build == kLong) return {decode_mma_kernel<BK, BV, QJL, NT, 3, false, DH>, smem};
+    return {decode_mma_kernel<BK, BV, QJL, NT, 2, false, DH>, smem};
+  } else {
+    constexpr int C = DH == 256 ? 2 : 3;
+    if (build == kPaged) return {decode_mma_kernel<BK, BV, QJL, NT, C, true, DH>, smem};
+    return {decode_mma_kernel<BK, BV, QJL, NT, C, false, DH>, smem};
+  }
 }
 
-template <int BK, int BV, bool QJL>
+template <int BK, int BV, bool QJL, int DH>
 Variant variant_q(int nt, int build) {
-  return nt == 1 ? variant_c<BK, BV, QJL, 1>(build) : variant_c<BK, BV, QJL, 2>(build);
+  return nt == 1 ? variant_c<BK, BV, QJL, 1, DH>(build) : variant_c<BK, BV, QJL, 2, DH>(build);
 }
 
-template <int BK, int BV>
+template <int BK, int BV, int DH>
 Variant variant_v(bool qjl, int nt, int build) {
-  return qjl ? variant_q<BK, BV, true>(nt, build) : variant_q<BK, BV, false>(nt, build);
+  return qjl ? variant_q<BK, BV, true, DH>(nt, build) : variant_q<BK, BV, false, DH>(nt, build);
 }
 
-template <int BK>
+template <int BK, int DH>
 Variant variant_k(int bv, bool qjl, int nt, int build) {
   switch (bv) {
-    case 2: return variant_v<BK, 2>(qjl, nt, build);
-    case 3: return variant_v<BK, 3>(qjl, nt, build);
-    default: return variant_v<BK, 4>(qjl, nt, build);
+    case 2: return variant_v<BK, 2, DH>(qjl, nt, build);
+    case 3: return variant_v<BK, 3, DH>(qjl, nt, build);
+    default: return variant_v<BK, 4, DH>(qjl, nt, build);
   }
 }
 
-Variant variant(int bk, int bv, bool qjl, int nt, int build) {
+template <int DH>
+Variant variant_d(int bk, int bv, bool qjl, int nt, int build) {
   switch (bk) {
-    case 2: return variant_k<2>(bv, qjl, nt, build);
-    case 3: return variant_k<3>(bv, qjl, nt, build);
-    default: return variant_k<4>(bv, qjl, nt, build);
+    case 2: return variant_k<2, DH>(bv, qjl, nt, build);
+    case 3: return variant_k<3, DH>(bv, qjl, nt, build);
+    default: return variant_k<4, DH>(bv, qjl, nt, build);
   }
+}
+
+Variant variant(int d, int bk, int bv, bool qjl, int nt, int build) {
+  if (d == 64) return variant_d<64>(bk, bv, qjl, nt, build);
+  if (d == 256) return variant_d<256>(bk, bv, qjl, nt, build);
+  return variant_d<128>(bk, bv, qjl, nt, build);
 }
 
 int build_of(bool long_splits, bool paged) { return paged ? kPaged : long_splits ? kLong : kShort; }
 
+int dim_index(int d) { return d == 64 ? 0 : d == 128 ? 1 : 2; }
+
 }  // namespace
 
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged) {
+int decode_ctas_per_sm(int d, int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged) {
   // cached per variant; atomically, as calls may come from several threads
   // (per device: the attribute and the occupancy query apply to the current one)
-  static std::atomic<int> cache[kMaxDevices][3][3][2][2][3];
+  static std::atomic<int> cache[kMaxDevices][3][3][3][2][2][3];
   const int nt = group > 8 ? 2 : 1;
   const int build = build_of(long_splits, paged);
-  std::atomic<int> &slot = cache[current_device()][bits_k - 2][bits_v - 2][qjl ? 1 : 0][nt - 1][build];
+  std::atomic<int> &slot =
+      cache[current_device()][dim_index(d)][bits_k - 2][bits_v - 2][qjl ? 1 : 0][nt - 1][build];
   int c = slot.load(std::memory_order_relaxed);
   if (c == 0) {
-    const Variant v = variant(bits_k, bits_v, qjl != 0, nt, build);
+    const Variant v = variant(d, bits_k, bits_v, qjl != 0, nt, build);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
     cudaFuncSetAttribute(v.fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int n = 0;
@@ -910,7 +1139,7 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
-  const Variant v = variant(p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1,
+  const Variant v = variant(p.d, p.bits_k, p.bits_v, p.qjl != 0, group > 8 ? 2 : 1,
                             build_of(split.long_splits, c.block_table != nullptr));
   DecodeArgs args{p, c, n_q_heads, max_seq_len, split.chunk, split.n_splits, seq_lens, q, q_dtype, scale, partials};
   cudaLaunchConfig_t cfg = {};
@@ -929,7 +1158,8 @@ int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q
   mcfg.stream = st;
   mcfg.attrs = pdl;
   mcfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&mcfg, merge_kernel, p, n_q_heads, seq_lens, max_seq_len, split.chunk, split.n_splits,
+  const auto merge = p.d == 64 ? merge_kernel<64> : p.d == 256 ? merge_kernel<256> : merge_kernel<128>;
+  e = cudaLaunchKernelEx(&mcfg, merge, p, n_q_heads, seq_lens, max_seq_len, split.chunk, split.n_splits,
                          (const float *)partials, out, lse);
   return (int)e;
 }

@@ -9,7 +9,9 @@
 
 namespace tq {
 
-constexpr int kHeadDim = 128;
+constexpr int kHeadDim = 128;  // the head dimension of the tensor-core quantize and prefill kernels
+// Head dimensions the library takes: 64, 128, 256.
+inline bool supported_head_dim(int d) { return d == 64 || d == 128 || d == 256; }
 constexpr int kMaxLevels = 16;  // 2^4 centroids at most
 
 // Sticky device-side error flags (tq_check_device_errors).
@@ -32,17 +34,17 @@ void codebook(int bits, int d, int law, float *centroids, float *thresholds);
 // every threshold exactly in fp32 (tq_host.cpp).
 bool threshold_search_exact(int bits, const float *thresholds);
 
-// Bytes of one packed vector of codes.
-inline int code_bytes(int bits) { return kHeadDim * bits / 8; }
+// Bytes of one packed vector of d codes.
+inline int code_bytes(int bits, int d) { return d * bits / 8; }
 
 // Byte tables for the byte-permute lookups of the decode kernel: lo[i] packs
 // the low bytes of entries 4i..4i+3, hi[i] their high bytes.  K entries are
-// the centroids as 16-bit fixed point (c * 2^kKFixedShift); V entries are the
-// fp16 bit patterns of the centroids.
+// the centroids as 16-bit fixed point (c * 2^k_shift, exact; k_shift is the
+// largest shift up to 17 that keeps every entry in [-32767, 32767], 17 at
+// d = 128); V entries are the fp16 bit patterns of the centroids.
 struct Lut {
   uint32_t lo[4], hi[4];
 };
-constexpr int kKFixedShift = 17;
 
 // Device-resident parameters of one context (all pointers device memory).
 struct DeviceParams {
@@ -60,14 +62,16 @@ struct DeviceParams {
   const uint8_t *jperm;   // [d] QJL fragment order -> projection index
   const uint16_t *pivt;   // [d][d] bf16: pivt[i][k] = Pi[vperm[k]][i] (Pi^T, columns in V fragment order)
   Lut lut_k, lut_v;
-  int bits_k, bits_v, qjl;
+  int d, bits_k, bits_v, qjl;
+  int k_shift;            // K centroids are exact integers times 2^-k_shift (Lut)
   int s_shift;            // sigma of sf: the fragment tables hold S 2^sigma (qjl only)
 };
 
-// Fragment orders of the decode kernel (host, tq_api.cu).
-void kperm_of(int bits, uint8_t *perm);
-void vperm_of(int bits, uint8_t *perm);
-void jperm_of(uint8_t *perm);
+// Fragment orders of the decode kernel for head dimension d (host,
+// tq_fragments.cpp): permutations of 0 .. d - 1.
+void kperm_of(int bits, int d, uint8_t *perm);
+void vperm_of(int bits, int d, uint8_t *perm);
+void jperm_of(int d, uint8_t *perm);
 
 // Split of the sequence axis used by decode attention.
 struct DecodeSplit {
@@ -79,19 +83,18 @@ DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_p
 // CTAs per SM of the attention kernel for these bit widths and query heads per
 // KV head, with the long-split (128-register) or short-split (168) budget, or
 // the paged-layout build (128 registers).
-int decode_ctas_per_sm(int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged);
+int decode_ctas_per_sm(int d, int bits_k, int bits_v, int qjl, int group, bool long_splits, bool paged);
 // The split and register budget of one decode call (tq_api.cu).
-DecodeSplit plan_decode(int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads, int max_seq_len,
-                        bool paged);
+DecodeSplit plan_decode(int d, int bits_k, int bits_v, int qjl, int group, int n_seqs, int n_kv_heads,
+                        int max_seq_len, bool paged);
 
 // Workspace layout of decode attention (byte offsets, 256-aligned): the split
 // partials [rows][splits][d+4] (m, l, two unused floats, then the d outputs,
 // so every output block is 16-byte aligned).
-constexpr int kPartialFloats = kHeadDim + 4;
 struct DecodeWorkspace {
   size_t partials, total;
 };
-DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split);
+DecodeWorkspace decode_workspace(int n_seqs, int n_q_heads, DecodeSplit split, int d);
 
 // Record a message for tq_last_error() and return `st` (tq_api.cu).
 tq_status report_error(tq_status st, const char *fmt, ...);
@@ -110,23 +113,37 @@ int current_device();
 // --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
+// seq_idx and pos may both be null: token t then goes to position t of
+// sequence 0 (the row layout of tq_weight_quantize).  include_k / include_v
+// select the matrices quantized here.
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
-                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream);
+                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
+                       void *stream);
+// K rows only through the per-row kernel (batches of at most 1024 rows, or a
+// head dimension other than 128), the same index convention.
+int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
+                           const int32_t *pos, int n_tok, void *stream);
 int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                         const int32_t *pos, int n_tok, void *stream);
 
-// B fragments of mma m16n8k16 for a 128 x 128 row-major bf16 matrix M (the
-// product is X M^T): 32-bit word 4 j + e of lane (r = lane / 4, qq = lane % 4)
-// in n-tile nt holds the pair M[8 nt + r][16 ks + 8 b + 2 qq (+1)] with
-// ks = (4 j + e) / 2 and b = (4 j + e) % 2, so a thread loads an n-tile's
-// fragments with four coalesced 16-byte loads (tq_api.cu).
-void mma_b_fragments(const uint16_t *m_bits, uint32_t *out);
+// B fragments of mma m16n8k16 for a d x d row-major 16-bit matrix M (the
+// product is X M^T), laid out [n-tile d / 8][chunk d / 32][lane 32][4 words]:
+// word 4 j + e of lane (r = lane / 4, qq = lane % 4) in n-tile nt holds the
+// pair M[8 nt + r][16 ks + 8 b + 2 qq (+1)] with ks = (4 j + e) / 2 and
+// b = (4 j + e) % 2, so a thread loads a chunk with one coalesced 16-byte
+// load (tq_api.cu).
+void mma_b_fragments(const uint16_t *m_bits, int d, uint32_t *out);
 // Causal prefill attention over the packed cache (tq_prefill.cu): the queries
 // of sequence s are rows cu_q[s] .. cu_q[s + 1] - 1 of q, at the last
 // cu_q[s + 1] - cu_q[s] positions below seq_lens[s].
 int launch_prefill(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype, int n_q_heads,
                    const int32_t *cu_q, const int32_t *seq_lens, int max_q, int max_seq_len, float scale,
                    float *out, float *lse, void *stream);
+// Weight rows (tq_weight.cu): workspace of the product and its launch
+// (y zeroed, x rotated, the packed rows streamed).
+size_t weight_workspace_bytes(int n_tok, int n_in);
+int launch_weight_gemm(const DeviceParams &p, const tq_cache &w, int n_out, int n_in, const void *x, int x_dtype,
+                       int n_tok, float *y, char *workspace, void *stream);
 int launch_decode(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype,
                   int n_q_heads, const int32_t *seq_lens, int max_seq_len, float scale,
                   float *out, float *lse, char *workspace, const DecodeSplit &split,

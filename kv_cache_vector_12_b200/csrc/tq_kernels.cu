@@ -17,8 +17,6 @@
 namespace tq {
 namespace {
 
-constexpr int D = kHeadDim;
-
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
   return __uint_as_float((uint32_t)h << 16);
 }
@@ -37,19 +35,42 @@ __device__ __forceinline__ int code_bit_pos(int bits, int i, int k) {
 }
 
 // ---------------------------------------------------------------------------
-// quantize, one CTA per head vector (small batches, and K rows with QJL):
-// thread i owns coordinate i.  z_i = (Pi x)_i from row i of Pi (16-byte loads,
+// quantize, one CTA per head vector (small batches, K rows with QJL, and every
+// batch of a head dimension other than 128): thread i owns coordinate i of a
+// DH-dimensional vector.  z_i = (Pi x)_i from row i of Pi (16-byte loads,
 // L2-resident), ||x|| by a block reduction (fp32 over exact bf16 squares), the
 // code against the thresholds scaled by ||x||, packing by warp OR-reductions
 // (one warp = one 32-coordinate group of the layout).  With QJL:
 // r = z/||x|| - c[code], ||r||, (S r)_m from row m of S, one sign ballot per
 // warp.  grid = (rows, 2): y = 0 for K, 1 for V.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float row_dot_bf16(const uint4 (&w)[16], const float *x) {
+// Row of Pi held in registers (up to 128 coordinates: loaded before the
+// dependency wait) or read on the fly (256).
+template <int DH>
+struct PiRow {
+  static constexpr int kHeld = DH <= 128 ? DH / 8 : 1;
+  uint4 w[kHeld];
+  const uint16_t *row;
+  __device__ __forceinline__ void load(const uint16_t *r) {
+    row = r;
+    if constexpr (DH <= 128) {
+#pragma unroll
+      for (int c = 0; c < DH / 8; ++c) w[c] = reinterpret_cast<const uint4 *>(r)[c];
+    }
+  }
+  __device__ __forceinline__ uint4 get(int c) const {
+    if constexpr (DH <= 128) return w[c];
+    else return reinterpret_cast<const uint4 *>(row)[c];
+  }
+};
+
+template <int DH>
+__device__ __forceinline__ float row_dot_bf16(const PiRow<DH> &pr, const float *x) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+  for (int c = 0; c < DH / 8; ++c) {
+    const uint4 w = pr.get(c);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       acc[e] = fmaf(__uint_as_float(u[e] << 16), x[8 * c + 2 * e], acc[e]);
@@ -59,51 +80,53 @@ __device__ __forceinline__ float row_dot_bf16(const uint4 (&w)[16], const float 
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
+template <int DH>
 __device__ __forceinline__ float row_dot_f32(const float *row, const float *x) {
-  float4 w[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) w[c] = reinterpret_cast<const float4 *>(row)[c];
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    acc[0] = fmaf(w[c].x, x[4 * c], acc[0]);
-    acc[1] = fmaf(w[c].y, x[4 * c + 1], acc[1]);
-    acc[2] = fmaf(w[c].z, x[4 * c + 2], acc[2]);
-    acc[3] = fmaf(w[c].w, x[4 * c + 3], acc[3]);
+#pragma unroll 8
+  for (int c = 0; c < DH / 4; ++c) {
+    const float4 w = reinterpret_cast<const float4 *>(row)[c];
+    acc[0] = fmaf(w.x, x[4 * c], acc[0]);
+    acc[1] = fmaf(w.y, x[4 * c + 1], acc[1]);
+    acc[2] = fmaf(w.z, x[4 * c + 2], acc[2]);
+    acc[3] = fmaf(w.w, x[4 * c + 3], acc[3]);
   }
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-__device__ __forceinline__ float block_sum128(float v, float *red) {
+template <int DH>
+__device__ __forceinline__ float block_sum(float v, float *red) {
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
-  const float r = (red[0] + red[1]) + (red[2] + red[3]);
+  float r = 0.f;
+#pragma unroll
+  for (int w = 0; w < DH / 32; ++w) r += red[w];
   __syncthreads();
   return r;
 }
 
-__global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_cache c,
-                                                           const uint16_t *__restrict__ k_in,
-                                                           const uint16_t *__restrict__ v_in,
-                                                           const int32_t *__restrict__ seq_idx,
-                                                           const int32_t *__restrict__ pos) {
-  __shared__ float s_x[D], s_r[D];
-  __shared__ float red[4];
+template <int DH>
+__global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cache c,
+                                                          const uint16_t *__restrict__ k_in,
+                                                          const uint16_t *__restrict__ v_in,
+                                                          const int32_t *__restrict__ seq_idx,
+                                                          const int32_t *__restrict__ pos) {
+  __shared__ float s_x[DH], s_r[DH];
+  __shared__ float red[DH / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // row tid of Pi is a parameter, written long before: load it while the
   // previous kernel finishes
-  uint4 pw[16];
-#pragma unroll
-  for (int ch = 0; ch < 16; ++ch) pw[ch] = reinterpret_cast<const uint4 *>(p.pi + tid * D)[ch];
+  PiRow<DH> pw;
+  pw.load(p.pi + tid * DH);
   // warm L2 with this row's inputs (a prefetch only moves lines into L2, the
   // point of coherence, so it may run before the previous kernel is done)
   if (tid == 0) {
     const long row = blockIdx.x;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"((blockIdx.y == 1 ? v_in : k_in) + row * D));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"((blockIdx.y == 1 ? v_in : k_in) + row * D + 64));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(seq_idx + row / c.n_kv_heads));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(pos + row / c.n_kv_heads));
+    for (int ch = 0; ch < DH * 2; ch += 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"((blockIdx.y == 1 ? v_in : k_in) + row * DH + ch / 2));
+    if (seq_idx) asm volatile("prefetch.global.L2 [%0];" ::"l"(seq_idx + row / c.n_kv_heads));
+    if (pos) asm volatile("prefetch.global.L2 [%0];" ::"l"(pos + row / c.n_kv_heads));
   }
   // launched as a programmatic dependent: no input is read before the
   // previous kernel in the stream has completed
@@ -114,17 +137,18 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   const bool qjl = !is_v && p.qjl;
   const long row = blockIdx.x;
   const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
-  const long slot = cache_slot(c, seq_idx[t], h, pos[t]);
+  // (no index arrays: token t goes to position t of sequence 0)
+  const long slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, h, pos ? pos[t] : t);
   if (slot < 0) {
     if (tid == 0 && !is_v) atomicOr(p.err, kErrTokenRange);
     return;
   }
-  const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * D + tid]);
+  const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * DH + tid]);
   s_x[tid] = x;
-  const float n = sqrtf(block_sum128(x * x, red));  // also orders s_x
+  const float n = sqrtf(block_sum<DH>(x * x, red));  // also orders s_x
   // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
   const bool live = n > 0x1p-25f;
-  const float z = live ? row_dot_bf16(pw, s_x) : 0.f;
+  const float z = live ? row_dot_bf16<DH>(pw, s_x) : 0.f;
   const float *thr = p.cb + (is_v ? 3 : 1) * kMaxLevels;
   const int half = 1 << (bits - 1);
   const float a = fabsf(z);
@@ -132,7 +156,7 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
   for (int j = 0; j < half - 1; ++j) m += a > thr[half + j] * n ? 1 : 0;
   const int code = z > 0.f ? half + m : half - 1 - m;
 
-  uint32_t *dst = reinterpret_cast<uint32_t *>((is_v ? c.codes_v : c.codes_k) + slot * (D * bits / 8));
+  uint32_t *dst = reinterpret_cast<uint32_t *>((is_v ? c.codes_v : c.codes_k) + slot * (DH * bits / 8));
   for (int wd = 0; wd < bits; ++wd) {  // warp w owns words w*bits .. w*bits+bits-1
     uint32_t contrib = 0;
     for (int kb = 0; kb < bits; ++kb) {
@@ -149,10 +173,10 @@ __global__ void __launch_bounds__(128) quantize_row_kernel(DeviceParams p, tq_ca
     const float y = live ? z / n : 0.f;
     const float r = y - cent[code];
     s_r[tid] = r;
-    const float gamma = sqrtf(block_sum128(r * r, red));
-    const float proj = row_dot_f32(p.s + tid * D, s_r);  // (S r)_tid
+    const float gamma = sqrtf(block_sum<DH>(r * r, red));
+    const float proj = row_dot_f32<DH>(p.s + tid * DH, s_r);  // (S r)_tid
     const uint32_t sb = __ballot_sync(0xffffffffu, proj >= 0.f);
-    if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (D / 8))[warp] = sb;
+    if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp] = sb;
     if (tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(gamma);
   }
 }
@@ -178,14 +202,32 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k, *vv = (const uint16_t *)v;
+  if (p.d != kHeadDim) {  // other head dimensions: the per-row kernel for every batch
+    cfg.gridDim = dim3((unsigned)rows, 2);
+    cfg.blockDim = dim3(p.d);
+    if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, vv, seq_idx, pos);
+    return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<256>, p, c, kk, vv, seq_idx, pos);
+  }
   if (rows <= kRowKernelMaxRows) {
     cfg.gridDim = dim3((unsigned)rows, 2);
-    return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel, p, c, kk, vv, seq_idx, pos);
+    return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<kHeadDim>, p, c, kk, vv, seq_idx, pos);
   }
   const bool k_on_tc = !p.qjl;
-  const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, stream);
+  const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, true, stream);
   if (e != 0 || k_on_tc) return e;
   return launch_quantize_qjl(p, c, k, seq_idx, pos, n_tok, stream);
+}
+
+int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
+                           const int32_t *pos, int n_tok, void *stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long)n_tok * c.n_kv_heads), 1);  // y = 0: K only
+  cfg.blockDim = dim3(p.d);
+  cfg.stream = (cudaStream_t)stream;
+  const uint16_t *kk = (const uint16_t *)k;
+  if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, kk, seq_idx, pos);
+  if (p.d == 256) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<256>, p, c, kk, kk, seq_idx, pos);
+  return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<kHeadDim>, p, c, kk, kk, seq_idx, pos);
 }
 
 }  // namespace tq

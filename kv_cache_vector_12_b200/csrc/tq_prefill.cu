@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kPThreads, 2) prefill_attn_kernel(const Prefil
         s_q8[row][0][kap] = (uint8_t)((v >> 8) & 0xFF);
         s_q8[row][1][kap] = (uint8_t)(v & 0xFF);
       }
-      if (half == 0) s_qs[row][0] = a.scale * kLog2e / (mu * (float)(1 << kKFixedShift));
+      if (half == 0) s_qs[row][0] = a.scale * kLog2e / (mu * ldexpf(1.f, a.p.k_shift));
       if constexpr (QJL) {
         const float *qt = s_qt + row * D;
         float mt = 0.f;

@@ -445,7 +445,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const bool live = row < a.n_rows;
       const int tok = live ? row / a.c.n_kv_heads : 0;
       const int tok_h = live ? row - tok * a.c.n_kv_heads : 0;
-      const int s_dst = a.seq_idx[tok], p_dst = a.pos[tok];
+      // (no index arrays: token t goes to position t of sequence 0, the
+      // weight-row layout of tq_weight_quantize)
+      const int s_dst = a.seq_idx ? a.seq_idx[tok] : 0, p_dst = a.pos ? a.pos[tok] : tok;
       if (!bar_wait(smem_addr(&full_bar[slot]), (i / kRingStages) & 1)) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
@@ -578,7 +580,8 @@ QuantTcFn pick(int bk, int bv) { return bk == 2 ? pick_bv<2>(bv) : bk == 3 ? pic
 }  // namespace
 
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
-                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, void *stream) {
+                       const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
+                       void *stream) {
   // cached per device (the attribute applies to the current device), and
   // atomically, as calls may come from several threads
   static std::atomic<int> cached_sm[kMaxDevices];
@@ -598,13 +601,16 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
   const long rows = (long)n_tok * c.n_kv_heads;
   CUtensorMap mk, mv, mp;
   std::memset(&mk, 0, sizeof mk);
-  if (!make_row_map(&mv, v, rows) || !make_row_map(&mp, p.pi, D) || (include_k && !make_row_map(&mk, k, rows)))
+  std::memset(&mv, 0, sizeof mv);
+  if ((include_v && !make_row_map(&mv, v, rows)) || !make_row_map(&mp, p.pi, D) ||
+      (include_k && !make_row_map(&mk, k, rows)))
     return (int)cudaErrorInvalidValue;
   if (!include_k) mk = mv;
+  if (!include_v) mv = mk;
   QuantTcArgs args{p, c, seq_idx, pos, (int)rows, 0, 0};
   const int tiles = (int)((rows + kTileRows - 1) / kTileRows);
   args.tiles_k = include_k ? tiles : 0;
-  args.tiles_v = tiles;
+  args.tiles_v = include_v ? tiles : 0;
   const int total = args.tiles_k + args.tiles_v;
   const int grid = total < n_sm ? total : n_sm;
   cudaLaunchAttribute pdl[1];

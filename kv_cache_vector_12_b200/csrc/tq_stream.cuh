@@ -202,14 +202,15 @@ __device__ __forceinline__ void v_pairs(const Lut &t, uint32_t sel, uint32_t &px
 }
 
 // -------------------------------------------------------- shared layout
-// One stage of TOK tokens of every plane, packed back to back (every plane
-// offset a multiple of 16 bytes for TOK a multiple of 8).
-template <int BK, int BV, bool QJL, int TOK>
+// One stage of TOK tokens of every plane of DH-dimensional vectors, packed
+// back to back (every plane offset a multiple of 16 bytes for TOK a multiple
+// of 8).
+template <int BK, int BV, bool QJL, int TOK, int DH = D>
 struct Stage {
-  static constexpr int kc = 0;                          // K codes
-  static constexpr int vc = kc + TOK * D * BK / 8;      // V codes
-  static constexpr int jb = vc + TOK * D * BV / 8;      // QJL sign bits
-  static constexpr int kn = jb + (QJL ? TOK * D / 8 : 0);
+  static constexpr int kc = 0;                           // K codes
+  static constexpr int vc = kc + TOK * DH * BK / 8;      // V codes
+  static constexpr int jb = vc + TOK * DH * BV / 8;      // QJL sign bits
+  static constexpr int kn = jb + (QJL ? TOK * DH / 8 : 0);
   static constexpr int vn = kn + TOK * 2;
   static constexpr int jg = vn + TOK * 2;
   static constexpr int bytes = jg + (QJL ? TOK * 2 : 0);

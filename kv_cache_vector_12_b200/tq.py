@@ -62,6 +62,13 @@ lib.tq_decode_attention_noalloc.restype = ctypes.c_int
 lib.tq_prefill_attention.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp, _vp, _i32, _i32,
                                      ctypes.c_float, _vp, _vp, _vp]
 lib.tq_prefill_attention.restype = ctypes.c_int
+lib.tq_weight_quantize.argtypes = [_vp, ctypes.POINTER(tq_cache), _vp, _i32, _i32, _vp]
+lib.tq_weight_quantize.restype = ctypes.c_int
+lib.tq_weight_workspace_bytes.argtypes = [_vp, _i32, _i32]
+lib.tq_weight_workspace_bytes.restype = ctypes.c_size_t
+lib.tq_weight_gemm.argtypes = [_vp, ctypes.POINTER(tq_cache), _i32, _i32, _vp, _i32, _i32, _vp, _vp,
+                               ctypes.c_size_t, _vp]
+lib.tq_weight_gemm.restype = ctypes.c_int
 lib.tq_check_device_errors.argtypes = [_vp, _vp]
 lib.tq_check_device_errors.restype = ctypes.c_int
 lib.tq_last_error.argtypes = []
@@ -264,6 +271,43 @@ def decode_attention_noalloc(ctx: Context, cache: Cache, q: torch.Tensor, seq_le
     _check(lib.tq_decode_attention_noalloc(ctx.handle, ctypes.byref(cache.struct), _ptr(q), q_dtype, q.shape[1],
                                            _ptr(seq_lens), max_seq_len, scale, _ptr(out), _ptr(lse),
                                            _stream(stream)))
+
+
+class WeightCache:
+    """Packed weight rows for tq_weight_quantize / tq_weight_gemm: a cache of
+    one sequence whose KV heads are the n_in / d blocks of a row and whose
+    positions are the n_out rows (K planes only)."""
+
+    def __init__(self, ctx: Context, n_out: int, n_in: int, device="cuda"):
+        nb = n_in // ctx.d
+        cap = (n_out + 63) // 64 * 64
+        sizes = ctx.layout()
+        self.codes = torch.zeros((nb, cap, sizes[0]), dtype=torch.uint8, device=device)
+        self.norms = torch.zeros((nb, cap), dtype=torch.int16, device=device)
+        self.n_out, self.n_in, self.capacity = n_out, n_in, cap
+        self.struct = tq_cache(self.codes.data_ptr(), self.norms.data_ptr(), None, None, None, None, cap, 1, nb,
+                               None, 0, 0)
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + 2 * self.norms.numel()
+
+
+def weight_quantize(ctx: Context, wc: WeightCache, w: torch.Tensor, stream=None) -> None:
+    """tq_weight_quantize: w bf16 [n_out, n_in] contiguous."""
+    _check(lib.tq_weight_quantize(ctx.handle, ctypes.byref(wc.struct), _ptr(w), wc.n_out, wc.n_in, _stream(stream)))
+
+
+def weight_workspace_bytes(ctx: Context, n_tok: int, n_in: int) -> int:
+    return int(lib.tq_weight_workspace_bytes(ctx.handle, n_tok, n_in))
+
+
+def weight_gemm(ctx: Context, wc: WeightCache, x: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                stream=None) -> None:
+    """tq_weight_gemm: x [n_tok, n_in] bf16 or fp32; y fp32 [n_tok, n_out]."""
+    x_dtype = TQ_F32 if x.dtype == torch.float32 else TQ_BF16
+    _check(lib.tq_weight_gemm(ctx.handle, ctypes.byref(wc.struct), wc.n_out, wc.n_in, _ptr(x), x_dtype, x.shape[0],
+                              _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
 
 
 def alloc_workspace(ctx: Context, n_seqs: int, n_q_heads: int, max_seq_len: int, device="cuda") -> torch.Tensor:

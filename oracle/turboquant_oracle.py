@@ -45,6 +45,11 @@ Readings where the pages are silent (each also listed in the design notes):
 * decode: q_hat = Pi q, q_tilde = S q_hat, score
   s_j = scale * n_j * (q_hat . c_K[code_j] + QJL term), softmax over j,
   o_tilde = sum_j p_j nV_j c_V[codeV_j] in rotated space, o = Pi^T o_tilde.
+* weights (ai-accelerate.xyz explainer, "重みの量子化にも応用できる": the same
+  algorithm applied to the weights of a linear layer): every row of W is cut
+  into blocks of d coordinates, each block quantized as one vector (norm,
+  rotation, codes); y = W~ x is evaluated in rotated space,
+  y_i = sum_b n_ib (Pi x_b) . c[code_ib].
 * prefill (prompt processing, whose cost over a compressed cache qxai.app's
   "Tether QVACのTurboQuant実装", fifth paragraph, singles out): the chunk's
   tokens are quantized into the cache first, then the query at position p
@@ -505,6 +510,31 @@ def prefill_attention(q, q_pos, pi, centroids_k, codes_k, norm_k, centroids_v, c
             qjl_gamma=None if qjl_gamma is None else qjl_gamma[:n])
         smax[t] = np.abs(sc).max(axis=1)
     return o, lse, smax
+
+
+def weight_quantize(w, d, pi, centroids, thresholds) -> Quantized:
+    """Rows of W [n_out, n_in] (n_in a multiple of d) cut into n_in / d blocks of
+    d coordinates, every block quantized as one vector.  Returns the Quantized
+    fields with shapes [n_out, n_in / d, ...] (codes [n_out, n_blocks, d], norm
+    [n_out, n_blocks])."""
+    w = np.asarray(w, dtype=np.float64)
+    n_out, n_in = w.shape
+    qz = quantize(w.reshape(n_out * (n_in // d), d), pi, centroids, thresholds)
+    nb = n_in // d
+    return Quantized(qz.codes.reshape(n_out, nb, d), qz.norm.reshape(n_out, nb), qz.y.reshape(n_out, nb, d))
+
+
+def weight_gemm(x, pi, centroids, codes, norm):
+    """y = W~ x for the block-quantized rows, in rotated space:
+    y[t, i] = sum_b norm[i, b] (Pi x[t, b]) . c[codes[i, b]].
+    x [n_tok, n_in] float64; codes [n_out, n_blocks, d]; norm [n_out, n_blocks].
+    Returns y [n_tok, n_out]."""
+    x = np.asarray(x, dtype=np.float64)
+    n_out, nb, d = codes.shape
+    xb = x.reshape(x.shape[0], nb, d)
+    x_hat = np.einsum("ij,tbj->tbi", pi, xb)                 # Pi x_tb
+    c = np.asarray(centroids)[codes]                          # [n_out, nb, d]
+    return np.einsum("tbk,obk,ob->to", x_hat, c, np.asarray(norm, dtype=np.float64))
 
 
 def exact_attention(q, k, v, scale):

@@ -39,11 +39,12 @@ def test_every_declared_symbol_is_exported(tq):
         assert hasattr(tq.lib, n), n
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("law", [o.LAW_GAUSSIAN, o.LAW_SPHERE])
 @pytest.mark.parametrize("bits_k,bits_v,qjl,seed", [(3, 3, 0, 42), (2, 4, 1, 42), (4, 2, 1, 7), (3, 2, 0, 12345)])
-def test_host_params_equal_oracle(tq, bits_k, bits_v, qjl, seed, law):
-    lib_p = tq.host_params(128, bits_k, bits_v, qjl, seed, law=law)
-    ref = o.Params(128, bits_k, bits_v, bool(qjl), seed, law)
+def test_host_params_equal_oracle(tq, d, bits_k, bits_v, qjl, seed, law):
+    lib_p = tq.host_params(d, bits_k, bits_v, qjl, seed, law=law)
+    ref = o.Params(d, bits_k, bits_v, bool(qjl), seed, law)
     assert np.array_equal(lib_p["pi"].double().numpy(), ref.pi)
     assert np.array_equal(lib_p["centroids_k"].double().numpy(), ref.ck)
     assert np.array_equal(lib_p["thresholds_k"].double().numpy(), ref.tk)
@@ -84,7 +85,8 @@ def test_invalid_arguments_fail_before_cuda(tq):
     assert b"law" in lib.tq_last_error()
     assert lib.tq_create_ex(None, 128, 3, 3, 0, 1, 1) == tq.TQ_ERR_INVALID
     h = ctypes.c_void_p()
-    assert lib.tq_create(ctypes.byref(h), 64, 3, 3, 0, 1) == tq.TQ_ERR_UNSUPPORTED
+    assert lib.tq_create(ctypes.byref(h), 96, 3, 3, 0, 1) == tq.TQ_ERR_UNSUPPORTED
+    assert b"64, 128 or 256" in lib.tq_last_error()
     assert lib.tq_create(None, 128, 3, 3, 0, 1) == tq.TQ_ERR_INVALID
     assert lib.tq_quantize(None, None, None, None, None, None, 0, None) == tq.TQ_ERR_INVALID
     assert lib.tq_decode_attention(None, None, None, 0, 1, None, 1, 0.0, None, None, None, 0, None) == \
