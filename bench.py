@@ -182,11 +182,12 @@ class OracleDecodeSample:
     unpack of the codes and the oracle's decode attention for the heads'
     query heads."""
 
-    def __init__(self, workload: str, bits_k: int, bits_v: int, qjl: bool, n_heads: int = 8):
+    def __init__(self, workload: str, bits_k: int, bits_v: int, qjl: bool, n_heads: int = 8, head_dim: int = 128):
+        import dataclasses
         from oracle import turboquant_oracle as o
         from kv_cache_vector_12_b200 import workloads as wl
         self.o = o
-        self.w = w = wl.WORKLOADS[workload]
+        self.w = w = dataclasses.replace(wl.WORKLOADS[workload], d=head_dim)
         self.bits_k, self.bits_v, self.qjl = bits_k, bits_v, qjl
         self.p = p = o.Params(w.d, bits_k, bits_v, qjl, w.pi_seed)
         n_heads = min(n_heads, w.n_kv_heads)
@@ -232,8 +233,9 @@ class OracleDecodeSample:
             return os.cpu_count() or 1
 
 
-def cpu_baseline(workload: str, bits_k: int, bits_v: int, qjl: bool, min_seconds: float = 10.0) -> dict:
-    smp = OracleDecodeSample(workload, bits_k, bits_v, qjl, n_heads=8)
+def cpu_baseline(workload: str, bits_k: int, bits_v: int, qjl: bool, head_dim: int = 128,
+                 min_seconds: float = 10.0) -> dict:
+    smp = OracleDecodeSample(workload, bits_k, bits_v, qjl, n_heads=8, head_dim=head_dim)
     total, reps = 0.0, 0
     while total < min_seconds:
         total += smp.step()
@@ -243,8 +245,11 @@ def cpu_baseline(workload: str, bits_k: int, bits_v: int, qjl: bool, min_seconds
 
 
 def resolve_setting(args):
+    import dataclasses
     from kv_cache_vector_12_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
+    if args.head_dim != w.d:
+        w = dataclasses.replace(w, d=args.head_dim)
     bits_k, bits_v = args.bits if args.bits else (w.bits_k, w.bits_v)
     qjl = w.qjl if args.qjl is None else bool(args.qjl)
     return w, bits_k, bits_v, qjl
@@ -255,7 +260,7 @@ def reference_arm(args):
     if rank != 0:
         return 0
     w, bits_k, bits_v, qjl = resolve_setting(args)
-    smp = OracleDecodeSample(args.workload, bits_k, bits_v, qjl, n_heads=1)
+    smp = OracleDecodeSample(args.workload, bits_k, bits_v, qjl, n_heads=1, head_dim=w.d)
     times = []
     for i in range(args.warmup + args.steps):
         dt = smp.step()
@@ -364,6 +369,72 @@ def prefill_report(tq, ctx, cache, q_all, n_tok, n_q_heads, reps=3) -> dict:
                     f"query, causal), median of {reps}"}
 
 
+def weight_report(tq, ctx, dev, n_out=14336, n_in=4096, token_counts=(1, 16), reps=20) -> dict:
+    """Weight-quantization reuse on a Llama-3-8B-shaped MLP projection
+    (W [14336][4096], seeded N(0,1) bf16): the rows quantized block by block
+    (tq_weight_quantize) with the context's K bits, then y = x W~^T over the
+    packed rows (tq_weight_gemm) for 1 and 16 tokens; median device time of
+    `reps` calls each, beside torch's bf16 matmul of the same shape (the
+    library product it replaces).  Effective GB/s = packed weight bytes per
+    call / time."""
+    gen = torch.Generator(device=dev).manual_seed(77)
+    w = torch.randn(n_out, n_in, generator=gen, device=dev).to(torch.bfloat16)
+    wc = tq.WeightCache(ctx, n_out, n_in, device=dev)
+    tq.weight_quantize(ctx, wc, w)
+    torch.cuda.synchronize()
+    packed = wc.codes[:, :n_out].numel() + 2 * wc.norms[:, :n_out].numel()
+
+    def med(fn):
+        fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+        for i in range(reps):
+            ev[2 * i].record()
+            fn()
+            ev[2 * i + 1].record()
+        torch.cuda.synchronize()
+        return statistics.median(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(reps))
+
+    out = {"shape": [n_out, n_in], "bits": ctx.bits_k, "packed_bytes": packed, "bf16_bytes": 2 * n_out * n_in}
+    for n_tok in token_counts:
+        x = torch.randn(n_tok, n_in, generator=gen, device=dev).to(torch.bfloat16)
+        y = torch.empty(n_tok, n_out, device=dev)
+        ws = torch.empty(tq.weight_workspace_bytes(ctx, n_tok, n_in), dtype=torch.uint8, device=dev)
+        ms = med(lambda: tq.weight_gemm(ctx, wc, x, y, ws))
+        ms_ref = med(lambda: x @ w.T)
+        ref = (x.float() @ w.float().T)
+        out[f"tokens_{n_tok}"] = {"us": ms * 1e3, "GBps": packed / (ms * 1e-3) / 1e9, "bf16_matmul_us": ms_ref * 1e3,
+                                  "speedup_vs_bf16": ms_ref / ms,
+                                  "rel_error_vs_bf16": float((y - ref).norm() / ref.norm())}
+    ctx.check_device_errors()
+    return out
+
+
+def prefill_only(args) -> int:
+    """`--prefill-only N`: the prefill leg alone on one sequence of the
+    workload's shapes and value law whose N tokens are quantized and then all
+    attend causally (the command the prefill kernel's profile is taken on)."""
+    from kv_cache_vector_12_b200 import tq
+    from kv_cache_vector_12_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w, bits_k, bits_v, qjl = resolve_setting(args)
+    n = args.prefill_only
+    ctx = tq.Context(w.d, bits_k, bits_v, int(qjl), w.pi_seed, law=args.law)
+    cache = tq.Cache(ctx, 1, w.n_kv_heads, (n + 63) // 64 * 64, device=dev)
+    gen = wl.generator(dev, w.seed)
+    outl = wl.outlier_scale(w, dev, w.seed) if args.workload == "llama70b" else None
+    k, v = wl.kv_tokens(w, n, gen, dev, outlier_mask=outl)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    tq.quantize(ctx, cache, k, v, torch.zeros(n, dtype=torch.int32, device=dev), pos)
+    rep = prefill_report(tq, ctx, cache, wl.queries(w, n, gen, dev), n, w.n_q_heads, reps=max(3, args.steps))
+    print(json.dumps({"metric": "causal prefill attention over the packed cache", "value": rep["tokens_per_s"],
+                      "unit": "tokens/s", "config": {"workload": WORKLOAD_DESCS[args.workload], "tokens": n,
+                                                      "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl},
+                      "prefill": rep}), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -377,16 +448,22 @@ def main(argv=None) -> int:
     ap.add_argument("--qjl", type=int, choices=[0, 1], default=None, help="1-bit QJL on K (default: the workload's)")
     ap.add_argument("--law", choices=["gaussian", "sphere"], default="gaussian",
                     help="coordinate law of the codebook (tq_law): N(0,1/d) or the exact unit-vector law")
+    ap.add_argument("--head-dim", type=int, choices=[64, 128, 256], default=128,
+                    help="head dimension d of the workload (its other shapes unchanged)")
     ap.add_argument("--paged", type=int, default=0, metavar="BLOCK",
                     help="paged cache with BLOCK tokens per block (a multiple of 64) and a shuffled block table")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each call kind alone (append quantize, decode) and add it to the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", type=int, default=0, metavar="N",
+                    help="only the prefill-attention leg, on one sequence of N tokens of the workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.prefill_only:
+        return prefill_only(args)
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -545,10 +622,13 @@ def main(argv=None) -> int:
     dec_ms = [dec_total / args.steps]
     ctx.check_device_errors()
     quality = quality_report(tq, ctx, caches[0], lens0, q_all[args.warmup], k_s0, v_s0, w.group)
-    n_prefill = min(lens0[0], 32768)
-    q_prefill = wl.queries(w, n_prefill, gen, dev)                     # [n_prefill, HQ, D]
-    prefill = prefill_report(tq, ctx, caches[0], q_prefill, n_prefill, HQ)
-    del q_prefill
+    prefill = None
+    if D == 128:  # prefill attention is built for d = 128
+        n_prefill = min(lens0[0], 32768)
+        q_prefill = wl.queries(w, n_prefill, gen, dev)                 # [n_prefill, HQ, D]
+        prefill = prefill_report(tq, ctx, caches[0], q_prefill, n_prefill, HQ)
+        del q_prefill
+    weights = weight_report(tq, ctx, dev) if D == 128 else None
 
     breakdown = None
     if args.breakdown:
@@ -662,12 +742,13 @@ def main(argv=None) -> int:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return 0
-    cpu = None if args.no_cpu_baseline else cpu_baseline(args.workload, bits_k, bits_v, qjl)
+    cpu = None if args.no_cpu_baseline else cpu_baseline(args.workload, bits_k, bits_v, qjl, D)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESCS[args.workload], "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl,
+        "config": {"workload": WORKLOAD_DESCS[args.workload] + (f" (head dimension {D})" if D != 128 else ""),
+                   "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl, "head_dim": D,
                    "codebook": args.law, "cache_layout": f"paged, {args.paged}-token blocks" if args.paged else "contiguous",
                    "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
                    f"cache replicas of {caches[0].nbytes() / 1e6:.1f} MB", "graph": f"CUDA graph of the {args.steps} timed steps, replayed back to back "
@@ -685,6 +766,7 @@ def main(argv=None) -> int:
                              "median of 10"},
         "quality": quality,
         "prefill": prefill,
+        "weights": weights,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,

@@ -345,10 +345,10 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
-  // One block: pi | pik | pivt | pif | s | sjk | sf | codebooks | kperm | jperm | error word.
+  // One block: pi | pik | pivt | pif | pvf | s | sjk | sf | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
   const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_pif = off_piv + dd * 2;
-  const size_t off_s = off_pif + dd * 2;
+  const size_t off_pvf = off_pif + dd * 2, off_s = off_pvf + dd * 2;
   const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_cb = off_sf + 2 * dd * 2;
   const size_t off_kperm = off_cb + 4 * tq::kMaxLevels * 4, off_jperm = off_kperm + 256;
   const size_t off_err = off_jperm + 256, total = off_err + 256;
@@ -396,6 +396,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
   for (int i = 0; i < d; ++i)
     for (int k = 0; k < d; ++k) pivt[(size_t)i * d + k] = ctx->pi_bits[(size_t)vperm[k] * d + i];
+  tq::mma_b_fragments(pivt, d, (uint32_t *)(h.data() + off_pvf));
   std::memcpy(h.data() + off_kperm, kperm, (size_t)d);
   std::memcpy(h.data() + off_jperm, jperm, (size_t)d);
   float *cb = (float *)(h.data() + off_cb);
@@ -419,6 +420,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->dp.cb = (const float *)(base + off_cb);
   ctx->dp.err = (unsigned *)(base + off_err);
   ctx->dp.pivt = (const uint16_t *)(base + off_piv);
+  ctx->dp.pvf = (const uint32_t *)(base + off_pvf);
   ctx->dp.kperm = (const uint8_t *)(base + off_kperm);
   ctx->dp.jperm = (const uint8_t *)(base + off_jperm);
   ctx->dp.d = d;

@@ -61,6 +61,7 @@ struct DeviceParams {
   const uint8_t *kperm;   // [d] K fragment order -> coordinate
   const uint8_t *jperm;   // [d] QJL fragment order -> projection index
   const uint16_t *pivt;   // [d][d] bf16: pivt[i][k] = Pi[vperm[k]][i] (Pi^T, columns in V fragment order)
+  const uint32_t *pvf;    // pivt as bf16 MMA B fragments, laid out like pif (the product O pivt^T)
   Lut lut_k, lut_v;
   int d, bits_k, bits_v, qjl;
   int k_shift;            // K centroids are exact integers times 2^-k_shift (Lut)

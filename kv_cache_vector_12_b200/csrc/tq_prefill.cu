@@ -581,14 +581,17 @@ __global__ void __launch_bounds__(kPThreads, 2) prefill_attn_kernel(const Prefil
   const int rho0 = row0 & 15, rho1 = row1 & 15;
   float *o0 = pos0 >= 0 ? a.out + (qrow0 + (long)(pos0 - p0) * a.n_q_heads + rho0 % G) * D : nullptr;
   float *o1 = pos1 >= 0 ? a.out + (qrow0 + (long)(pos1 - p0) * a.n_q_heads + rho1 % G) * D : nullptr;
-#pragma unroll 1
+#pragma unroll 2
   for (int nt = 0; nt < 16; ++nt) {
-    const uint16_t *prow = a.p.pivt + (size_t)(8 * nt + r) * D;
+    // this n-tile's B fragments: four coalesced 16-byte loads (two k-steps each)
+    uint4 bf[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bf[j] = reinterpret_cast<const uint4 *>(a.p.pvf)[(nt * 4 + j) * 32 + lane];
     float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t b0 = *reinterpret_cast<const uint32_t *>(prow + 16 * ks + 2 * q);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t *>(prow + 16 * ks + 8 + 2 * q);
+      const uint4 &v = bf[ks / 2];
+      const uint32_t b0 = (ks & 1) ? v.z : v.x, b1 = (ks & 1) ? v.w : v.y;
       mma_bf16(c, ohi[ks][0], ohi[ks][1], ohi[ks][2], ohi[ks][3], b0, b1);
       mma_bf16(c, olo[ks][0], olo[ks][1], olo[ks][2], olo[ks][3], b0, b1);
     }
@@ -634,10 +637,638 @@ int smem_of(int bk, int bv, bool qjl) {
 
 }  // namespace
 
+}  // namespace tq
+
+
+// ===========================================================================
+// The tcgen05 form (contexts without QJL).  Per CTA 128 query rows (the MMA's
+// M) and, per tile of 128 keys:
+//   expand   the four consumer warps turn the keys' codes into two fp16
+//            shared-memory operands in the 128-byte-swizzled K-major layout:
+//            K~[key][kappa] (the exact fp16 K centroids, K fragment order)
+//            and V~^T[kappa_v][key] (fp16 V centroids, V fragment order);
+//   scores   one thread issues S = Q^_hi K~^T + Q^_lo K~^T (tcgen05.mma
+//            kind::f16, fp32 accumulator in tensor memory), q_hat as a
+//            two-part fp16 split scaled per row by a power of two;
+//   softmax  thread i owns row i: S from tensor memory, times the row's
+//            factor and the key norms, causal mask, online max and sum (exp2),
+//            P' = p ||v|| as fp16 into the swizzled A operand; a moved max
+//            rescales the row of O in tensor memory;
+//   values   O += P' V~ (tcgen05.mma, fp32 in tensor memory).
+// At the end o = Pi^T (O / l) is one more pair of MMAs (O as bf16 hi + lo,
+// Pi^T's rows in the V fragment order as the B operand), and the lse.
+// A producer warp streams the codes with 1-D bulk copies.  Every mbarrier
+// wait is bounded.
+// ===========================================================================
+namespace tq {
+namespace {
+
+constexpr int kTcRows = 128;                      // query rows per CTA
+constexpr int kTcKeys = 128;                      // keys per tile
+constexpr int kTcWarps = 4;
+constexpr int kTcThreads = 32 * (kTcWarps + 1);
+constexpr int kTcStages = 2;
+constexpr int kOpBytes = 128 * kHeadDim * 2;      // one 128 x 128 16-bit operand: two 128 x 64 swizzled boxes
+constexpr int kOpBox = kOpBytes / 2;
+constexpr uint32_t kTcCols = 256;                 // S at columns 0 .. 127, O at 128 .. 255
+
+template <int BK, int BV>
+struct TcLayout {
+  static constexpr int qhi = 0, qlo = kOpBytes, kt = 2 * kOpBytes, vt = 3 * kOpBytes, pt = 4 * kOpBytes;
+  static constexpr int ring = 5 * kOpBytes;
+  static constexpr int stage = Stage<BK, BV, false, kTcKeys>::bytes;
+  static constexpr int bytes = ring + kTcStages * stage + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ void tcx_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tcx_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcWarps) : "memory");
+}
+
+// Byte offset of element (row, col) of a 128 x 128 16-bit operand stored as
+// two boxes of 128 rows x 64 columns, 128-byte rows, 16-byte chunks swizzled
+// by the row within each 8-row (1024-byte) atom.
+__device__ __forceinline__ uint32_t sw_off(int row, int col) {
+  const int box = col >> 6, cc = col & 63;
+  return (uint32_t)(box * kOpBox + row * 128 + ((((cc >> 3) ^ (row & 7)) & 7) << 4) + ((cc & 7) << 1));
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart.
+__device__ __forceinline__ uint64_t swdesc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptors, kind::f16, fp32 accumulator, A and B K-major,
+// M = N = 128: fp16 inputs, and bf16 inputs.
+constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescBF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void tcx_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                   tmem_d),
+               "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+__device__ __forceinline__ void tcx_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tmem_ld16x(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st16x(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// fp16 pairs (codes 0, 1) and (codes 2, 3) of one lookup's low and high bytes.
+__device__ __forceinline__ void f16_pairs(uint32_t lo, uint32_t hi, uint32_t &p01, uint32_t &p23) {
+  p01 = prmt(lo, hi, 0x5140u);
+  p23 = prmt(lo, hi, 0x7362u);
+}
+
+template <int BK, int BV>
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const PrefillArgs a) {
+  using L = TcLayout<BK, BV>;
+  using St = Stage<BK, BV, false, kTcKeys>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages], s_bar, pv_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ int s_pos[kTcRows];
+
+  const int s = blockIdx.z, h = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = lane >> 2, q = lane & 3;
+  const int G = a.n_q_heads / a.c.n_kv_heads;
+  const int PC = kTcRows / G;                  // positions per CTA
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int blk = gridDim.x - 1 - blockIdx.x;  // the longest blocks first
+  const int q0 = a.cu_q[s], n_q = a.cu_q[s + 1] - q0;
+  const int len = a.seq_lens[s];
+  if (len < 0 || len > a.max_seq_len || n_q < 0 || n_q > len || n_q > a.max_q) {
+    if (tid == 0 && blk == 0 && h == 0) atomicOr(a.p.err, kErrSeqLen);
+    return;
+  }
+  const int first_q = blk * PC;
+  if (first_q >= n_q) return;
+  const int p0 = len - n_q;
+  const int last_q = min(n_q, first_q + PC) - 1;
+  const int kend = p0 + last_q + 1;
+  const int n_tiles = (kend + kTcKeys - 1) / kTcKeys;
+  const long base = ((long)s * a.c.n_kv_heads + h) * a.c.capacity;
+  const long qrow0 = (long)q0 * a.n_q_heads + (long)h * G;
+
+  if (tid < kTcRows) {
+    const int qi = first_q + tid / G;
+    s_pos[tid] = (tid < PC * G && qi < n_q) ? p0 + qi : -1;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), kTcWarps);
+    }
+    mbar_init(smem_u32(&s_bar), 1);
+    mbar_init(smem_u32(&pv_bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTcCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tcx_fence_before();
+  __syncthreads();
+  tcx_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t t_s = tmem, t_o = tmem + 128;
+
+  if (warp == kTcWarps) {
+    // ---------------- producer: the codes of one tile of keys per stage
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int slot = it % kTcStages;
+        if (it >= kTcStages && !mbar_wait(smem_u32(&empty_bar[slot]), ((it / kTcStages) - 1) & 1)) {
+          atomicOr(a.p.err, kErrWaitExpired);
+          abort_flag = 1;
+          break;
+        }
+        if (*(volatile int *)&abort_flag) break;
+        unsigned char *st = sm + L::ring + slot * L::stage;
+        const uint32_t bar = smem_u32(&full_bar[slot]);
+        const int first = it * kTcKeys;
+        const uint32_t n = (uint32_t)min(kTcKeys, (kend - first + 63) & ~63);
+        mbar_arrive_expect_tx(bar, n * (D * BK / 8 + D * BV / 8 + 4));
+        for (uint32_t done = 0; done < n;) {
+          long tok;
+          uint32_t run = n - done;
+          if (a.c.block_table) {
+            const int pp = first + (int)done, j = pp / a.c.block_size, off = pp - j * a.c.block_size;
+            run = min(run, (uint32_t)(a.c.block_size - off));
+            int bl = a.c.block_table[(long)s * (a.c.capacity / a.c.block_size) + j];
+            if (bl < 0 || bl >= a.c.n_blocks) {
+              atomicOr(a.p.err, kErrTokenRange);
+              bl = 0;
+            }
+            tok = ((long)bl * a.c.n_kv_heads + h) * a.c.block_size + off;
+          } else {
+            tok = base + first + done;
+          }
+          bulk_g2s(smem_u32(st + St::kc + done * (D * BK / 8)), a.c.codes_k + tok * (D * BK / 8), run * (D * BK / 8),
+                   bar);
+          bulk_g2s(smem_u32(st + St::vc + done * (D * BV / 8)), a.c.codes_v + tok * (D * BV / 8), run * (D * BV / 8),
+                   bar);
+          bulk_g2s(smem_u32(st + St::kn + done * 2), a.c.norm_k + tok, run * 2, bar);
+          bulk_g2s(smem_u32(st + St::vn + done * 2), a.c.norm_v + tok, run * 2, bar);
+          done += run;
+        }
+        issued = it + 1;
+      }
+      if (*(volatile int *)&abort_flag) {
+        for (int it = max(0, issued - kTcStages); it < issued; ++it)
+          mbar_wait(smem_u32(&full_bar[it % kTcStages]), (it / kTcStages) & 1);
+      }
+    }
+  } else {
+    // ---------------- consumers: thread tid owns query row tid
+    const int row = tid, pos = s_pos[row];
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;  // this warp's TMEM lane quarter
+    // q_hat = Pi q in the K fragment order (Pi's rows stored in that order),
+    // mma m16n8k16 bf16, fp32 q as hi + lo; warp w computes rows 32 w ..
+    // 32 w + 31 into a fp32 scratch (the V~ and P' regions, free until the
+    // first tile)
+    float *scr = reinterpret_cast<float *>(sm + L::vt);  // [128 rows][128], 64 KB over vt and pt
+    {
+      const bool f32 = a.q_dtype == TQ_F32;
+#pragma unroll 1
+      for (int mt = 0; mt < 2; ++mt) {
+        uint32_t ahi[8][4], alo[8][4];
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int rr = 32 * warp + 16 * mt + r + 8 * (e & 1), col = 16 * ks + 8 * (e >> 1) + 2 * q;
+            const int pr = s_pos[rr];
+            float x0 = 0.f, x1 = 0.f;
+            if (pr >= 0) {
+              const long qr = qrow0 + (long)(pr - p0) * a.n_q_heads + (rr % G);
+              if (f32) {
+                const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(a.q) + qr * D + col);
+                x0 = v.x;
+                x1 = v.y;
+              } else {
+                const uint32_t v =
+                    *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.q) + qr * D + col);
+                x0 = __uint_as_float(v << 16);
+                x1 = __uint_as_float(v & 0xffff0000u);
+              }
+            }
+            split_bf16x2(x0, x1, ahi[ks][e], alo[ks][e]);
+          }
+#pragma unroll 1
+        for (int nt = 0; nt < 16; ++nt) {
+          uint32_t bfr[8][2];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[(nt * 4 + j) * 32 + lane];
+            bfr[2 * j][0] = v.x, bfr[2 * j][1] = v.y, bfr[2 * j + 1][0] = v.z, bfr[2 * j + 1][1] = v.w;
+          }
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            mma_bf16(c, ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], bfr[ks][0], bfr[ks][1]);
+            mma_bf16(c, alo[ks][0], alo[ks][1], alo[ks][2], alo[ks][3], bfr[ks][0], bfr[ks][1]);
+          }
+          float *d0 = scr + (32 * warp + 16 * mt + r) * D + 8 * nt + 2 * q;
+          *reinterpret_cast<float2 *>(d0) = make_float2(c[0], c[1]);
+          *reinterpret_cast<float2 *>(d0 + 8 * D) = make_float2(c[2], c[3]);
+        }
+      }
+    }
+    __syncwarp();
+    // per row: a power-of-two scale puts max |q_hat| in [2^13, 2^14), then
+    // q_hat = hi + lo in fp16 into the swizzled A operands
+    float fq;
+    {
+      const float *qr = scr + row * D;
+      float m = 0.f;
+      for (int k = 0; k < D; ++k) m = fmaxf(m, fabsf(qr[(k + lane) & (D - 1)]));
+      int ex = 0;
+      if (m > 0.f) frexpf(m, &ex);
+      const float sc = m > 0.f ? ldexpf(1.f, 14 - ex) : 1.f;
+      fq = a.scale * kLog2e / sc;
+#pragma unroll 4
+      for (int k0 = 0; k0 < D; k0 += 8) {
+        const int k = (k0 + 8 * lane) & (D - 1);  // lane-rotated chunks spread the shared-memory banks
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_f16x2(qr[k + 2 * e] * sc, qr[k + 2 * e + 1] * sc, hi[e], lo[e]);
+        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, k)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, k)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    // the K centroids as fp16 byte tables (exact: the centroids are fp16 values)
+    Lut lkf;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lkf.lo[i] = lkf.hi[i] = 0u;
+    for (int e = 0; e < (1 << BK); ++e) {
+      const uint16_t hb = __half_as_ushort(__float2half_rn(a.p.cb[e]));
+      lkf.lo[e / 4] |= (uint32_t)(hb & 0xff) << (8 * (e % 4));
+      lkf.hi[e / 4] |= (uint32_t)(hb >> 8) << (8 * (e % 4));
+    }
+    const Lut lv = a.p.lut_v;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    tc_consumer_sync();  // the scratch is read: the first tile may overwrite it
+
+    for (int it = 0; it < n_tiles && ok; ++it) {
+      const int slot = it % kTcStages;
+      ok = mbar_wait(smem_u32(&full_bar[slot]), (it / kTcStages) & 1);
+      if (!ok) break;
+      tcx_fence_after();
+      const unsigned char *st = sm + L::ring + slot * L::stage;
+      // K~ is free (the previous scores were waited for): expand it while the
+      // previous tile's value MMAs run, then issue this tile's scores
+      // ---------------- expand: warp w takes keys 32 w .. 32 w + 31 of the tile
+#pragma unroll
+      for (int rb = 0; rb < 2; ++rb) {
+        const int k0 = 32 * warp + 16 * rb + r, k1 = k0 + 8;
+        uint32_t wk0[BK], wk1[BK];
+        const unsigned char *kr0 = st + St::kc + k0 * (D * BK / 8) + q * 4 * BK;
+        const unsigned char *kr1 = st + St::kc + k1 * (D * BK / 8) + q * 4 * BK;
+#pragma unroll
+        for (int i = 0; i < BK; ++i) {
+          wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
+          wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
+        }
+#pragma unroll
+        for (int sg = 0; sg < 8; ++sg) {
+          const int kap = 32 * (sg >> 1) + 16 * (sg & 1) + 4 * q;
+          uint32_t lo, hi, p01, p23;
+          lookup<BK>(lkf, k_selector<BK>(wk0, sg), lo, hi);
+          f16_pairs(lo, hi, p01, p23);
+          *reinterpret_cast<uint2 *>(sm + L::kt + sw_off(k0, kap)) = make_uint2(p01, p23);
+          lookup<BK>(lkf, k_selector<BK>(wk1, sg), lo, hi);
+          f16_pairs(lo, hi, p01, p23);
+          *reinterpret_cast<uint2 *>(sm + L::kt + sw_off(k1, kap)) = make_uint2(p01, p23);
+        }
+      }
+      fence_async_smem();
+      tcx_fence_before();
+      tc_consumer_sync();
+      if (tid == 0) {  // ---------------- S = Q^_hi K~^T + Q^_lo K~^T
+        tcx_fence_after();
+        const uint32_t aq = smem_u32(sm + L::qhi), al = smem_u32(sm + L::qlo), bk = smem_u32(sm + L::kt);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+          tcx_mma(t_s, swdesc(aq + off), swdesc(bk + off), kIdescF16, kk > 0);
+          tcx_mma(t_s, swdesc(al + off), swdesc(bk + off), kIdescF16, 1);
+        }
+        tcx_commit(smem_u32(&s_bar));
+      }
+      // the previous tile's value MMAs read V~ and P' and write O: wait for
+      // them, then expand V~ while this tile's scores run
+      if (it > 0) ok = mbar_wait(smem_u32(&pv_bar), (it - 1) & 1);
+      if (!ok) break;
+      tcx_fence_after();
+      // ---------------- V~^T for the same keys
+#pragma unroll
+      for (int rb = 0; rb < 2; ++rb) {
+        // V~^T: rows in the V fragment order, keys as columns (decode's A
+        // fragments: a0 = row 16 mt + r, keys 2q, 2q+1; a1 = row + 8; a2, a3:
+        // keys + 8)
+        constexpr int VB = D * BV / 8;
+        const int kb = 32 * warp + 16 * rb;  // first key of the 16-key block
+        const unsigned char *vt = st + St::vc + (kb + 2 * q) * VB;
+        auto put = [&](int mt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+          unsigned char *vb = sm + L::vt;
+          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r, kb + 2 * q)) = a0;
+          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r + 8, kb + 2 * q)) = a1;
+          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r, kb + 8 + 2 * q)) = a2;
+          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r + 8, kb + 8 + 2 * q)) = a3;
+        };
+        if constexpr (BV == 3) {
+          const int gofs = 12 * (r >> 1);
+          const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
+          uint32_t ya[3], yb[3];
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            ya[k] = prmt(reinterpret_cast<const uint32_t *>(vt + gofs)[k],
+                         reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k], gs);
+            yb[k] = prmt(reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k],
+                         reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k], gs);
+          }
+          const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+            const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t a0, a1, a2, a3;
+              v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
+              v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
+              put(2 * k + hh, a0, a1, a2, a3);
+            }
+          }
+        } else if constexpr (BV == 2) {
+          const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
+          const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
+          const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
+          const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
+#pragma unroll
+          for (int yh = 0; yh < 2; ++yh) {
+            const uint32_t gs = yh ? 0x7362u : 0x5140u;
+            const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+            for (int par = 0; par < 2; ++par) {
+              const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a0, a1, a2, a3;
+                v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
+                v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+                put(4 * yh + 2 * par + hh, a0, a1, a2, a3);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
+            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
+            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
+            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
+#pragma unroll
+            for (int yh = 0; yh < 2; ++yh) {
+              const uint32_t gs = yh ? 0x7362u : 0x5140u;
+              const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a0, a1, a2, a3;
+                v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
+                v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+                put(4 * u + 2 * yh + hh, a0, a1, a2, a3);
+              }
+            }
+          }
+        }
+      }
+      // V~ is published to the tensor cores with P' before the value MMAs
+      ok = mbar_wait(smem_u32(&s_bar), it & 1);
+      if (!ok) break;
+      tcx_fence_after();
+      // ---------------- softmax of row `row` over the tile's keys
+      const __half *kn = reinterpret_cast<const __half *>(st + St::kn);
+      const __half *vn = reinterpret_cast<const __half *>(st + St::vn);
+      const int kfirst = it * kTcKeys;
+      float sc[kTcKeys];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTcKeys / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16x(t_s + lane_off + 16 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = 16 * c + e;
+          const float x = __uint_as_float(v[e]) * fq * __half2float(kn[j]);
+          sc[j] = kfirst + j <= pos ? x : -INFINITY;
+          mx = fmaxf(mx, sc[j]);
+        }
+      }
+      const float mn = fmaxf(m_run, mx);
+      const float ref = fmaxf(mn, -3.0e38f);
+      const float al = fast_exp2(m_run - ref);
+      m_run = mn;
+      float ls = 0.f;
+#pragma unroll
+      for (int c = 0; c < kTcKeys / 8; ++c) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 8 * c + 2 * e;
+          const float pa = fast_exp2(sc[j] - ref), pb = fast_exp2(sc[j + 1] - ref);
+          ls += pa + pb;
+          pk[e] = pack_half2(sc[j] == -INFINITY ? 0.f : pa * __half2float(vn[j]),
+                             sc[j + 1] == -INFINITY ? 0.f : pb * __half2float(vn[j + 1]));
+        }
+        *reinterpret_cast<uint4 *>(sm + L::pt + sw_off(row, 8 * c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l_run = fmaf(l_run, al, ls);
+      // the norms are read: the producer may refill this stage
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));
+      // a moved maximum rescales this warp's rows of O (O is complete: the
+      // previous tile's values were waited for above)
+      if (it > 0 && __any_sync(0xffffffffu, al != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16x(t_o + lane_off + 16 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
+          tmem_st16x(t_o + lane_off + 16 * c, v);
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tcx_fence_before();
+      tc_consumer_sync();
+      if (tid == 0) {  // ---------------- O += P' V~
+        tcx_fence_after();
+        const uint32_t ap = smem_u32(sm + L::pt), bv = smem_u32(sm + L::vt);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+          tcx_mma(t_o, swdesc(ap + off), swdesc(bv + off), kIdescF16, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        tcx_commit(smem_u32(&pv_bar));
+      }
+    }
+    // ---------------- o = Pi^T (O / l): O as bf16 hi + lo (A, over the Q^
+    // operands), Pi^T with its rows in the V fragment order (B, over K~)
+    if (ok) ok = mbar_wait(smem_u32(&pv_bar), (n_tiles - 1) & 1);
+    if (ok) {
+      tcx_fence_after();
+      float l = l_run;
+      const float il = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16x(t_o + lane_off + 16 * c, v);
+        tmem_wait_ld();
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          split_bf16x2(__uint_as_float(v[2 * e]) * il, __uint_as_float(v[2 * e + 1]) * il, hi[e], lo[e]);
+        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, 16 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, 16 * c + 8)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, 16 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, 16 * c + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+      }
+      // row `row` of Pi^T (pivt[i][k] = Pi[vperm k][i]) into the B operand
+      const uint4 *prow = reinterpret_cast<const uint4 *>(a.p.pivt + (size_t)row * D);
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4 *>(sm + L::kt + sw_off(row, 8 * c)) = prow[c];
+      fence_async_smem();
+      tcx_fence_before();
+      tc_consumer_sync();
+      if (tid == 0) {
+        tcx_fence_after();
+        const uint32_t ah = smem_u32(sm + L::qhi), alo2 = smem_u32(sm + L::qlo), bp = smem_u32(sm + L::kt);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+          tcx_mma(t_s, swdesc(ah + off), swdesc(bp + off), kIdescBF16, kk > 0);
+          tcx_mma(t_s, swdesc(alo2 + off), swdesc(bp + off), kIdescBF16, 1);
+        }
+        tcx_commit(smem_u32(&s_bar));
+      }
+      ok = mbar_wait(smem_u32(&s_bar), n_tiles & 1);
+      if (ok) {
+        tcx_fence_after();
+        const int rho = row % G;
+        float *orow = pos >= 0 ? a.out + (qrow0 + (long)(pos - p0) * a.n_q_heads + rho) * D : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16x(t_s + lane_off + 16 * c, v);
+          tmem_wait_ld();
+          if (orow) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              reinterpret_cast<float4 *>(orow + 16 * c)[e] =
+                  make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                              __uint_as_float(v[4 * e + 3]));
+          }
+        }
+        if (a.lse && pos >= 0)
+          a.lse[qrow0 + (long)(pos - p0) * a.n_q_heads + rho] = (m_run + log2f(l)) * 0.6931471805599453f;
+      }
+    }
+    if (!ok) {
+      atomicOr(a.p.err, kErrWaitExpired);
+      abort_flag = 1;
+    }
+  }
+  // release the tensor memory once every MMA and tcgen05 access is finished
+  tcx_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcx_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols) : "memory");
+  }
+}
+
+}  // namespace
+}  // namespace tq
+
+namespace tq {
+namespace {
+
+using PrefillTcFn = void (*)(const PrefillArgs);
+
+template <int BK>
+PrefillTcFn pick_tc_v(int bv) {
+  return bv == 2 ? prefill_tc_kernel<BK, 2> : bv == 3 ? prefill_tc_kernel<BK, 3> : prefill_tc_kernel<BK, 4>;
+}
+
+PrefillTcFn pick_tc(int bk, int bv) { return bk == 2 ? pick_tc_v<2>(bv) : bk == 3 ? pick_tc_v<3>(bv) : pick_tc_v<4>(bv); }
+
+template <int BK>
+int tc_bytes_v(int bv) {
+  return bv == 2 ? TcLayout<BK, 2>::bytes : bv == 3 ? TcLayout<BK, 3>::bytes : TcLayout<BK, 4>::bytes;
+}
+
+int tc_bytes(int bk, int bv) { return bk == 2 ? tc_bytes_v<2>(bv) : bk == 3 ? tc_bytes_v<3>(bv) : tc_bytes_v<4>(bv); }
+
+}  // namespace
+
+// Contexts without QJL run the tcgen05 kernel (128 query rows per CTA);
+// with QJL, the mma.sync kernel (64 rows per CTA).
 int launch_prefill(const DeviceParams &p, const tq_cache &c, const void *q, int q_dtype, int n_q_heads,
                    const int32_t *cu_q, const int32_t *seq_lens, int max_q, int max_seq_len, float scale,
                    float *out, float *lse, void *stream) {
   const bool qjl = p.qjl != 0;
+  const int G = n_q_heads / c.n_kv_heads;
+  PrefillArgs args{p, c, n_q_heads, max_seq_len, max_q, cu_q, seq_lens, q, q_dtype, scale, out, lse};
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = (cudaStream_t)stream;
+  if (!qjl) {
+    const PrefillTcFn fn = pick_tc(p.bits_k, p.bits_v);
+    const int smem = tc_bytes(p.bits_k, p.bits_v);
+    static std::atomic<bool> configured_tc[kMaxDevices][3][3];
+    std::atomic<bool> &done = configured_tc[current_device()][p.bits_k - 2][p.bits_v - 2];
+    if (!done.load(std::memory_order_acquire)) {
+      const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return (int)e;
+      done.store(true, std::memory_order_release);
+    }
+    const int per_cta = kTcRows / G;
+    cfg.gridDim = dim3((unsigned)((max_q + per_cta - 1) / per_cta), c.n_kv_heads, c.n_seqs);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = smem;
+    return (int)cudaLaunchKernelEx(&cfg, fn, args);
+  }
   const PrefillFn fn = pick(p.bits_k, p.bits_v, qjl);
   const int smem = smem_of(p.bits_k, p.bits_v, qjl);
   // the dynamic shared-memory limit is set once per device and variant
@@ -648,14 +1279,10 @@ int launch_prefill(const DeviceParams &p, const tq_cache &c, const void *q, int 
     if (e != cudaSuccess) return (int)e;
     done.store(true, std::memory_order_release);
   }
-  const int G = n_q_heads / c.n_kv_heads;
   const int per_cta = kPWarps * (16 / G);
-  PrefillArgs args{p, c, n_q_heads, max_seq_len, max_q, cu_q, seq_lens, q, q_dtype, scale, out, lse};
-  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((max_q + per_cta - 1) / per_cta), c.n_kv_heads, c.n_seqs);
   cfg.blockDim = dim3(kPThreads);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = (cudaStream_t)stream;
   return (int)cudaLaunchKernelEx(&cfg, fn, args);
 }
 

@@ -13,7 +13,7 @@
 //   rotate  x_hat[b][t] = Pi x_tb per (block, token), as 16-bit fixed point
 //           (hi, lo bytes) in the decode kernel's K fragment order, with its
 //           scale factor; one CTA of d threads per (block, token).
-//   gemm    per CTA 128 weight rows x 16 tokens, over a range of blocks: the
+//   gemm    per CTA 128 weight rows x 8 or 16 tokens, over a range of blocks: the
 //           rows' codes, norms and the blocks' x_hat stream in by TMA bulk
 //           copies (one producer warp, mbarrier ring, bounded waits); four
 //           consumer warps of 32 rows compute each block's dot products on
@@ -39,13 +39,14 @@ namespace {
 constexpr int kWWarps = 4;
 constexpr int kWThreads = 32 * (kWWarps + 1);
 constexpr int kWRows = 32 * kWWarps;  // weight rows per CTA
-constexpr int kWTok = 16;             // tokens per CTA (two n-tiles of 8)
+constexpr int kWTok = 16;             // token padding of the workspace (up to two n-tiles of 8 per CTA)
 constexpr int kWStages = 4;
 
 // ------------------------------------------------------------------ rotate
-// x_hat = Pi x for one (block b, token t): thread kappa computes fragment
-// position kappa (row kperm[kappa] of Pi), then the block's scale.  Tokens at
-// or past n_tok (padding up to a multiple of 16) get zeros.
+// x_hat = Pi x for one (block b, token t < n_tok): thread kappa computes
+// fragment position kappa (row kperm[kappa] of Pi), then the block's scale.
+// The padding tokens up to a multiple of 16 are never written: the product
+// reads them but never stores their results.
 __global__ void __launch_bounds__(kHeadDim) weight_rotate_kernel(DeviceParams p, const void *x, int x_dtype,
                                                                  int n_tok, int n_in, int t_pad, uint8_t *xq,
                                                                  float *xf) {
@@ -87,13 +88,14 @@ __global__ void __launch_bounds__(kHeadDim) weight_rotate_kernel(DeviceParams p,
 }
 
 // -------------------------------------------------------------------- gemm
-template <int BK>
+template <int BK, int NT>
 struct WStage {
+  static constexpr int tok = 8 * NT;                               // tokens per CTA
   static constexpr int codes = 0;                                  // [128 rows][16 BK]
   static constexpr int norms = codes + kWRows * 16 * BK;           // [128 rows] fp16
-  static constexpr int xq = norms + kWRows * 2;                    // [16 tokens][2][128] bytes
-  static constexpr int xf = xq + kWTok * 2 * kHeadDim;             // [16 tokens] fp32
-  static constexpr int bytes = xf + kWTok * 4;
+  static constexpr int xq = norms + kWRows * 2;                    // [tok][2][128] bytes
+  static constexpr int xf = xq + tok * 2 * kHeadDim;               // [tok] fp32
+  static constexpr int bytes = xf + tok * 4;
 };
 
 struct WeightArgs {
@@ -105,9 +107,9 @@ struct WeightArgs {
   float *y;          // [n_tok][n_out], accumulated with atomic adds
 };
 
-template <int BK>
+template <int BK, int NT>
 __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs a) {
-  using St = WStage<BK>;
+  using St = WStage<BK, NT>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kWStages], empty_bar[kWStages];
   __shared__ int abort_flag;
@@ -145,12 +147,12 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
         const uint32_t bar = smem_u32(&full_bar[slot]);
         const int b = b0 + it;
         const long tok = (long)b * a.w.capacity + row0;  // sequence 0, KV head b, position row0
-        mbar_arrive_expect_tx(bar, n_rows * (16 * BK + 2) + kWTok * (2 * kHeadDim + 4));
+        mbar_arrive_expect_tx(bar, n_rows * (16 * BK + 2) + St::tok * (2 * kHeadDim + 4));
         bulk_g2s(smem_u32(st + St::codes), a.w.codes_k + tok * (16 * BK), n_rows * (16 * BK), bar);
         bulk_g2s(smem_u32(st + St::norms), a.w.norm_k + tok, n_rows * 2, bar);
-        bulk_g2s(smem_u32(st + St::xq), a.xq + ((size_t)b * a.t_pad + (size_t)tg * kWTok) * 2 * kHeadDim,
-                 kWTok * 2 * kHeadDim, bar);
-        bulk_g2s(smem_u32(st + St::xf), a.xf + (size_t)b * a.t_pad + (size_t)tg * kWTok, kWTok * 4, bar);
+        bulk_g2s(smem_u32(st + St::xq), a.xq + ((size_t)b * a.t_pad + (size_t)tg * St::tok) * 2 * kHeadDim,
+                 St::tok * 2 * kHeadDim, bar);
+        bulk_g2s(smem_u32(st + St::xf), a.xf + (size_t)b * a.t_pad + (size_t)tg * St::tok, St::tok * 4, bar);
         issued = it + 1;
       }
       if (*(volatile int *)&abort_flag) {
@@ -163,11 +165,11 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
 
   // ---------------- consumers: rows 32 warp + 16 rb + r (+ 8), tokens 8 nt + 2 q (+ 1)
   const Lut lk = a.p.lut_k;
-  float yacc[2][2][4];
+  float yacc[2][NT][4];
 #pragma unroll
   for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) yacc[rb][nt][e] = 0.f;
   for (int it = 0; it < n_stage; ++it) {
@@ -179,10 +181,10 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
     }
     const unsigned char *st = smem + slot * St::bytes;
     // B fragments of x_hat (tokens 8 nt + r), the tokens' factors and the rows' norms
-    uint32_t xh[2][4][2], xl[2][4][2];
-    float xfac[2][2];
+    uint32_t xh[NT][4][2], xl[NT][4][2];
+    float xfac[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       const uint8_t *xb = st + St::xq + (8 * nt + r) * 2 * kHeadDim;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
@@ -208,9 +210,9 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
         wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
         wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
       }
-      int chh[2][4], cmid[2][4], cll[2][4];
+      int chh[NT][4], cmid[NT][4], cll[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) chh[nt][e] = cmid[nt][e] = cll[nt][e] = 0;
 #pragma unroll
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
         lookup<BK>(lk, k_selector<BK>(wk0, 2 * ks + 1), alo[2], ahi[2]);
         lookup<BK>(lk, k_selector<BK>(wk1, 2 * ks + 1), alo[3], ahi[3]);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < NT; ++nt) {
           mma_i8<true, true>(chh[nt], ahi[0], ahi[1], ahi[2], ahi[3], xh[nt][ks][0], xh[nt][ks][1]);
           mma_i8<true, false>(cmid[nt], ahi[0], ahi[1], ahi[2], ahi[3], xl[nt][ks][0], xl[nt][ks][1]);
           mma_i8<false, true>(cmid[nt], alo[0], alo[1], alo[2], alo[3], xh[nt][ks][0], xh[nt][ks][1]);
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
       }
       const float n0 = __half2float(nrm[lr]), n1 = __half2float(nrm[lr + 8]);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int hm = (chh[nt][e] << 8) + cmid[nt][e];
@@ -246,11 +248,11 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
 #pragma unroll
   for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int row = row0 + 32 * warp + 16 * rb + r + 8 * (e >> 1);
-        const int t = tg * kWTok + 8 * nt + 2 * q + (e & 1);
+        const int t = tg * St::tok + 8 * nt + 2 * q + (e & 1);
         if (row < a.n_out && t < a.n_tok) atomicAdd(a.y + (size_t)t * a.n_out + row, yacc[rb][nt][e]);
       }
 }
@@ -285,22 +287,28 @@ int launch_weight_gemm(const DeviceParams &p, const tq_cache &w, int n_out, int 
   float *xf = reinterpret_cast<float *>(workspace + ((size_t)nb * t_pad * 2 * kHeadDim + 255) / 256 * 256);
   cudaError_t e = cudaMemsetAsync(y, 0, (size_t)n_tok * n_out * sizeof(float), st);
   if (e != cudaSuccess) return (int)e;
-  weight_rotate_kernel<<<dim3(nb, t_pad), kHeadDim, 0, st>>>(p, x, x_dtype, n_tok, n_in, t_pad, xq, xf);
+  weight_rotate_kernel<<<dim3(nb, n_tok), kHeadDim, 0, st>>>(p, x, x_dtype, n_tok, n_in, t_pad, xq, xf);
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  // split the blocks so that the grid fills about two waves of the SMs
-  const int tiles = (n_out + kWRows - 1) / kWRows, groups = t_pad / kWTok;
+  // split the blocks so that the grid fills about four CTAs per SM
+  // one n-tile of 8 tokens per CTA for up to 8 tokens, else two
+  const int nt = n_tok <= 8 ? 1 : 2;
+  const int tiles = (n_out + kWRows - 1) / kWRows, groups = (n_tok + 8 * nt - 1) / (8 * nt);
   const long units = (long)tiles * groups;
   const long want = 2L * sm_count_here() * 2;
   int splits = (int)std::max(1L, std::min<long>(nb, (want + units - 1) / units));
   const int per = (nb + splits - 1) / splits;
   splits = (nb + per - 1) / per;
-  const WeightFn fn = p.bits_k == 2 ? weight_gemm_kernel<2> : p.bits_k == 3 ? weight_gemm_kernel<3>
-                                                                            : weight_gemm_kernel<4>;
-  const int smem = kWStages * (p.bits_k == 2 ? WStage<2>::bytes : p.bits_k == 3 ? WStage<3>::bytes
-                                                                               : WStage<4>::bytes);
-  static std::atomic<bool> configured[kMaxDevices][3];
-  std::atomic<bool> &done = configured[current_device()][p.bits_k - 2];
+  const WeightFn fn = nt == 1 ? (p.bits_k == 2 ? weight_gemm_kernel<2, 1> : p.bits_k == 3 ? weight_gemm_kernel<3, 1>
+                                                                                         : weight_gemm_kernel<4, 1>)
+                              : (p.bits_k == 2 ? weight_gemm_kernel<2, 2> : p.bits_k == 3 ? weight_gemm_kernel<3, 2>
+                                                                                         : weight_gemm_kernel<4, 2>);
+  const int smem = kWStages * (nt == 1 ? (p.bits_k == 2 ? WStage<2, 1>::bytes : p.bits_k == 3 ? WStage<3, 1>::bytes
+                                                                                             : WStage<4, 1>::bytes)
+                                       : (p.bits_k == 2 ? WStage<2, 2>::bytes : p.bits_k == 3 ? WStage<3, 2>::bytes
+                                                                                             : WStage<4, 2>::bytes));
+  static std::atomic<bool> configured[kMaxDevices][3][2];
+  std::atomic<bool> &done = configured[current_device()][p.bits_k - 2][nt - 1];
   if (!done.load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return (int)e;
