@@ -455,6 +455,8 @@ def main(argv=None) -> int:
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each call kind alone (append quantize, decode) and add it to the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-seqs", type=int, default=0, metavar="N",
+                    help="keep only the workload's first N sequences (a smaller case of the same kernels, for profiling)")
     ap.add_argument("--prefill-only", type=int, default=0, metavar="N",
                     help="only the prefill-attention leg, on one sequence of N tokens of the workload")
     args = ap.parse_args(argv)
@@ -476,8 +478,12 @@ def main(argv=None) -> int:
     from kv_cache_vector_12_b200 import tq
     from kv_cache_vector_12_b200 import workloads as wl
     w, bits_k, bits_v, qjl = resolve_setting(args)
+    lens0 = wl.serving_lengths(w, w.seed) if args.workload == "serving" else [w.seq_len] * w.n_seqs
+    if args.max_seqs:
+        import dataclasses
+        lens0 = lens0[:args.max_seqs]
+        w = dataclasses.replace(w, n_seqs=len(lens0))
     H, HQ, D, B = w.n_kv_heads, w.n_q_heads, w.d, w.n_seqs
-    lens0 = wl.serving_lengths(w, w.seed) if args.workload == "serving" else [w.seq_len] * B
     bytes_per_token = H * (D * (bits_k + bits_v) // 8 + 4 + (D // 8 + 2 if qjl else 0))
     R = args.replicas or max(1, math.ceil(2 * 126e6 / (sum(lens0) * bytes_per_token)))
     n_steps_total = args.warmup + args.steps
@@ -747,7 +753,8 @@ def main(argv=None) -> int:
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESCS[args.workload] + (f" (head dimension {D})" if D != 128 else ""),
+        "config": {"workload": WORKLOAD_DESCS[args.workload] + (f" (head dimension {D})" if D != 128 else "")
+                   + (f" (first {B} sequences only)" if args.max_seqs else ""),
                    "bits_k": bits_k, "bits_v": bits_v, "qjl": qjl, "head_dim": D,
                    "codebook": args.law, "cache_layout": f"paged, {args.paged}-token blocks" if args.paged else "contiguous",
                    "replicas": R, "l2": f"inputs larger than L2: {R} rotating "
