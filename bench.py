@@ -374,8 +374,9 @@ def weight_report(tq, ctx, dev, n_out=14336, n_in=4096, token_counts=(1, 16), re
     (W [14336][4096], seeded N(0,1) bf16): the rows quantized block by block
     (tq_weight_quantize) with the context's K bits, then y = x W~^T over the
     packed rows (tq_weight_gemm) for 1 and 16 tokens; median device time of
-    `reps` calls each, beside torch's bf16 matmul of the same shape (the
-    library product it replaces).  Effective GB/s = packed weight bytes per
+    `reps` calls each (a CUDA graph of the calls, so the host's launch time is
+    not counted), beside torch's bf16 matmul of the same shape (the library
+    product it replaces).  Effective GB/s = packed weight bytes per
     call / time."""
     gen = torch.Generator(device=dev).manual_seed(77)
     w = torch.randn(n_out, n_in, generator=gen, device=dev).to(torch.bfloat16)
@@ -385,15 +386,28 @@ def weight_report(tq, ctx, dev, n_out=14336, n_in=4096, token_counts=(1, 16), re
     packed = wc.codes[:, :n_out].numel() + 2 * wc.norms[:, :n_out].numel()
 
     def med(fn):
-        fn()
-        torch.cuda.synchronize()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
-        for i in range(reps):
-            ev[2 * i].record()
+        """Device time per call: `reps` calls captured as one CUDA graph (so
+        host launch overhead is not timed), replayed 5 times; median replay."""
+        gs = torch.cuda.Stream(device=dev)
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
             fn()
+        torch.cuda.current_stream().wait_stream(gs)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for i in range(5):
+            ev[2 * i].record()
+            g.replay()
             ev[2 * i + 1].record()
         torch.cuda.synchronize()
-        return statistics.median(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(reps))
+        del g
+        return statistics.median(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(5)) / reps
 
     out = {"shape": [n_out, n_in], "bits": ctx.bits_k, "packed_bytes": packed, "bf16_bytes": 2 * n_out * n_in}
     for n_tok in token_counts:
