@@ -29,8 +29,9 @@
  *    message.  Device-side range errors (a seq_idx, pos or seq_len outside the
  *    cache) skip the offending token or sequence and set a sticky flag that
  *    tq_check_device_errors() reports.
- *  - Head dimension d = 128.  bits_k, bits_v in {2, 3, 4}.  qjl in {0, 1}
- *    (applies to K only).
+ *  - Head dimension d in {64, 128, 256} for the cache (tq_quantize,
+ *    tq_decode_attention); prefill attention and weight rows take d = 128
+ *    only.  bits_k, bits_v in {2, 3, 4}.  qjl in {0, 1} (applies to K only).
  */
 #ifndef TQ_H
 #define TQ_H
@@ -49,7 +50,7 @@ typedef enum tq_status {
   TQ_ERR_INVALID = 1,     /* bad argument; nothing launched */
   TQ_ERR_CUDA = 2,        /* a CUDA runtime call failed */
   TQ_ERR_NOMEM = 3,       /* device allocation in tq_create failed */
-  TQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (e.g. d != 128) */
+  TQ_ERR_UNSUPPORTED = 4, /* valid but not implemented (e.g. d = 96) */
   TQ_ERR_DEVICE = 5       /* a kernel recorded a device-side range error */
 } tq_status;
 
@@ -142,9 +143,9 @@ typedef struct tq_cache {
  * from counters 2^32+1.. (fp32).  Allocates and uploads the parameters
  * (synchronous); the only call that allocates device memory.
  * Errors: TQ_ERR_INVALID (null out, bits outside {2,3,4}, qjl outside {0,1}),
- * TQ_ERR_UNSUPPORTED (d != 128, or a codebook whose thresholds the quantize
- * kernel's binary search could not select exactly in fp32; the host checks
- * this, and it holds for every codebook of d = 128), TQ_ERR_NOMEM,
+ * TQ_ERR_UNSUPPORTED (d outside {64, 128, 256}, or a codebook whose
+ * thresholds the quantize kernels could not select exactly in fp32; the host
+ * checks this, and it holds for every codebook of those d), TQ_ERR_NOMEM,
  * TQ_ERR_CUDA.
  */
 tq_status tq_create(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v,

@@ -20,8 +20,14 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtq.so")
 
-SOURCES = ["tq_host.cpp", "tq_fragments.cpp", "tq_api.cu", "tq_kernels.cu", "tq_quantize_tc.cu", "tq_quantize_qjl.cu", "tq_decode.cu",
-           "tq_prefill.cu", "tq_weight.cu", "tq_noalloc.cu"]
+# (source, object name, extra flags): tq_decode_variants.cu is compiled once
+# per (head dimension, K width) slice of the attention kernel's instantiations
+SOURCES = [(s, os.path.splitext(s)[0], []) for s in
+           ["tq_host.cpp", "tq_fragments.cpp", "tq_api.cu", "tq_kernels.cu", "tq_quantize_tc.cu",
+            "tq_quantize_qjl.cu", "tq_quantize_tile.cu", "tq_decode.cu", "tq_prefill.cu", "tq_weight.cu",
+            "tq_noalloc.cu"]]
+SOURCES += [("tq_decode_variants.cu", f"tq_decode_variants_d{d}_k{bk}", [f"-DTQ_DECODE_DH={d}", f"-DTQ_DECODE_BK={bk}"])
+            for d in (64, 128, 256) for bk in (2, 3, 4)]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           "-I" + os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]
@@ -34,14 +40,15 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
-    obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+def _compile(entry, verbose: bool, ptxas_v: bool) -> str:
+    src, name, flags = entry
+    obj = os.path.join(BUILD, name + ".o")
     path = os.path.join(CSRC, src)
     deps = [path] + [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith((".h", ".cuh"))]
     deps.append(os.path.join(ROOT, "include", "tq.h"))
     if os.path.exists(obj) and all(os.path.getmtime(obj) >= os.path.getmtime(d) for d in deps) and not ptxas_v:
         return obj
-    cmd = [nvcc(), *ARCH, *COMMON, "-c", path, "-o", obj]
+    cmd = [nvcc(), *ARCH, *COMMON, *flags, "-c", path, "-o", obj]
     if ptxas_v and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
     if verbose:
@@ -56,7 +63,7 @@ def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
 
 def build(verbose: bool = False, ptxas_v: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+    with cf.ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 4)) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_v), SOURCES))
     if not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
         tmp = LIB + ".tmp"

@@ -120,6 +120,10 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                        void *stream);
+// K (is_v false) or V rows in 64-row tiles for head dimensions 64 and 256,
+// MSE codes only (tq_quantize_tile.cu).
+int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x, const int32_t *seq_idx,
+                         const int32_t *pos, int n_tok, bool is_v, void *stream);
 // K rows only through the per-row kernel (batches of at most 1024 rows, or a
 // head dimension other than 128), the same index convention.
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,

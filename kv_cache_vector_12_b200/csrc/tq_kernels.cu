@@ -202,11 +202,20 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k, *vv = (const uint16_t *)v;
-  if (p.d != kHeadDim) {  // other head dimensions: the per-row kernel for every batch
-    cfg.gridDim = dim3((unsigned)rows, 2);
-    cfg.blockDim = dim3(p.d);
-    if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, vv, seq_idx, pos);
-    return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<256>, p, c, kk, vv, seq_idx, pos);
+  if (p.d != kHeadDim) {
+    // other head dimensions: the per-row kernel for small batches, else the
+    // tile kernel for V and for K without QJL (K with QJL keeps the per-row
+    // kernel: the QJL tile kernel is specialised for d = 128)
+    if (rows <= kRowKernelMaxRows) {
+      cfg.gridDim = dim3((unsigned)rows, 2);
+      cfg.blockDim = dim3(p.d);
+      if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, vv, seq_idx, pos);
+      return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<256>, p, c, kk, vv, seq_idx, pos);
+    }
+    int e = launch_quantize_tile(p, c, v, seq_idx, pos, n_tok, true, stream);
+    if (e != 0) return e;
+    return p.qjl ? launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream)
+                 : launch_quantize_tile(p, c, k, seq_idx, pos, n_tok, false, stream);
   }
   if (rows <= kRowKernelMaxRows) {
     cfg.gridDim = dim3((unsigned)rows, 2);

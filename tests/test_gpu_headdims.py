@@ -44,12 +44,15 @@ def rows(n, h, d, seed, lognormal=True):
 
 @pytest.mark.parametrize("d", [64, 256])
 @pytest.mark.parametrize("bits_k,bits_v,qjl", SETTINGS)
-def test_quantize_parity(tq, d, bits_k, bits_v, qjl):
-    n_tok, n_heads = 300, 2
+@pytest.mark.parametrize("n_tok", [300, 700])
+def test_quantize_parity(tq, d, bits_k, bits_v, qjl, n_tok):
+    """300 tokens x 2 heads: the per-row kernel; 700 x 2 (1400 rows, a ragged
+    last tile of 56): the tile kernel (V, and K without QJL)."""
+    n_heads = 2
     ctx = tq.Context(d, bits_k, bits_v, qjl, 42)
     ref = params(d, bits_k, bits_v, qjl)
     k, v = rows(n_tok, n_heads, d, 5 + d), rows(n_tok, n_heads, d, 6 + d)
-    cache = tq.Cache(ctx, 1, n_heads, 320)
+    cache = tq.Cache(ctx, 1, n_heads, (n_tok + 63) // 64 * 64)
     pos = torch.randperm(n_tok, generator=torch.Generator().manual_seed(d)).to(torch.int32)
     tq.quantize(ctx, cache, k.cuda(), v.cuda(), torch.zeros(n_tok, dtype=torch.int32, device="cuda"), pos.cuda())
     ctx.check_device_errors()
