@@ -345,11 +345,12 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
-  // One block: pi | pik | pivt | pif | pvf | s | sjk | sf | codebooks | kperm | jperm | error word.
+  // One block: pi | pik | pivt | pif | pvf | s | sjk | sf | ssplit | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
   const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_pif = off_piv + dd * 2;
   const size_t off_pvf = off_pif + dd * 2, off_s = off_pvf + dd * 2;
-  const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_cb = off_sf + 2 * dd * 2;
+  const size_t off_sjk = off_s + dd * 4, off_sf = off_sjk + dd * 4, off_ss = off_sf + 2 * dd * 2;
+  const size_t off_cb = off_ss + 2 * dd * 2;
   const size_t off_kperm = off_cb + 4 * tq::kMaxLevels * 4, off_jperm = off_kperm + 256;
   const size_t off_err = off_jperm + 256, total = off_err + 256;
   e = cudaMalloc(&ctx->dev_block, total);
@@ -391,6 +392,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
         rest[i] -= tq::half_bits_to_double(part[i]);
       }
       tq::mma_b_fragments(part.data(), d, (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
+      std::memcpy(h.data() + off_ss + (size_t)k * dd * 2, part.data(), dd * 2);
     }
   }
   uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
@@ -417,6 +419,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->dp.sjk = (const float *)(base + off_sjk);
   ctx->dp.pif = (const uint32_t *)(base + off_pif);
   ctx->dp.sf = (const uint32_t *)(base + off_sf);
+  ctx->dp.ssplit = (const uint16_t *)(base + off_ss);
   ctx->dp.cb = (const float *)(base + off_cb);
   ctx->dp.err = (unsigned *)(base + off_err);
   ctx->dp.pivt = (const uint16_t *)(base + off_piv);

@@ -56,6 +56,7 @@ struct DeviceParams {
   const uint32_t *pif;    // Pi (natural row order) as bf16 MMA B fragments [n-tile 16][chunk 4][lane 32][4 words]
   const uint32_t *sf;     // S 2^sigma split into two fp16 parts (hi + lo), each as B fragments like pif:
                           // [part 2][n-tile 16][chunk 4][lane 32][4 words] (qjl only; sigma chosen on the host)
+  const uint16_t *ssplit; // the same two parts as plain row-major fp16 matrices [part 2][d][d] (qjl only)
   const float *cb;        // [4][16]: centroids_k, thresholds_k, centroids_v, thresholds_v
   unsigned *err;          // sticky error flags
   const uint8_t *kperm;   // [d] K fragment order -> coordinate
@@ -130,6 +131,9 @@ int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void 
                            const int32_t *pos, int n_tok, void *stream);
 int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                         const int32_t *pos, int n_tok, void *stream);
+// K with QJL on tcgen05 (d = 128), tiles of 128 rows (tq_quantize_qjl_tc.cu).
+int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
+                           const int32_t *pos, int n_tok, void *stream);
 
 // B fragments of mma m16n8k16 for a d x d row-major 16-bit matrix M (the
 // product is X M^T), laid out [n-tile d / 8][chunk d / 32][lane 32][4 words]:
