@@ -121,7 +121,7 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                        void *stream);
-// K (is_v false) or V rows in 64-row tiles for head dimensions 64 and 256,
+// K (is_v false) or V rows in 64- or 128-row tiles for head dimensions 64 and 256,
 // MSE codes only (tq_quantize_tile.cu).
 int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x, const int32_t *seq_idx,
                          const int32_t *pos, int n_tok, bool is_v, void *stream);
@@ -129,11 +129,10 @@ int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x
 // head dimension other than 128), the same index convention.
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                            const int32_t *pos, int n_tok, void *stream);
-int launch_quantize_qjl(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
-                        const int32_t *pos, int n_tok, void *stream);
-// K with QJL on tcgen05 (d = 128), tiles of 128 rows (tq_quantize_qjl_tc.cu).
-int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
-                           const int32_t *pos, int n_tok, void *stream);
+// K with QJL and V (MSE codes) on tcgen05 (d = 128), tiles of 128 rows, one
+// launch (tq_quantize_qjl_tc.cu).
+int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
+                           const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
 
 // B fragments of mma m16n8k16 for a d x d row-major 16-bit matrix M (the
 // product is X M^T), laid out [n-tile d / 8][chunk d / 32][lane 32][4 words]:

@@ -184,9 +184,9 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 }  // namespace
 
 // Batches of up to kRowKernelMaxRows rows per matrix (decode-time appends) use
-// the one-CTA-per-row kernel; larger batches use the tcgen05 kernel for every
-// MSE-only matrix (all of V, K without QJL) and the tcgen05 QJL kernel
-// (tq_quantize_qjl_tc.cu) for K with QJL.
+// the one-CTA-per-row kernel; larger batches one tcgen05 kernel for K and V:
+// the MSE kernel (tq_quantize_tc.cu) without QJL, the QJL kernel
+// (tq_quantize_qjl_tc.cu) with it.
 constexpr long kRowKernelMaxRows = 1024;
 
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
@@ -221,10 +221,8 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
     cfg.gridDim = dim3((unsigned)rows, 2);
     return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<kHeadDim>, p, c, kk, vv, seq_idx, pos);
   }
-  const bool k_on_tc = !p.qjl;
-  const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, k_on_tc, true, stream);
-  if (e != 0 || k_on_tc) return e;
-  return launch_quantize_qjl_tc(p, c, k, seq_idx, pos, n_tok, stream);
+  if (p.qjl) return launch_quantize_qjl_tc(p, c, k, v, seq_idx, pos, n_tok, stream);
+  return launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, true, true, stream);
 }
 
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,

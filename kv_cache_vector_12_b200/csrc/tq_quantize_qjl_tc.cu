@@ -1,5 +1,6 @@
-// Quantize-on-append of K with the 1-bit QJL residual stage on the
-// 5th-generation tensor cores (sm_100a).
+// Quantize-on-append with the 1-bit QJL residual stage on K, on the
+// 5th-generation tensor cores (sm_100a); V rows of the same batch (MSE codes
+// only) run in the same launch.
 //
 // The method ("ステップ2: QJL", ai-accelerate.xyz TurboQuant explainer; the
 // residual 1-bit QJL transform of "Tether QVACのTurboQuant実装", qxai.app):
@@ -7,31 +8,33 @@
 // each K vector (y = Pi x / ||x||) is projected by a Gaussian matrix S, and
 // only the signs of S r are kept, with ||r||.
 //
-// Two GEMMs per tile of 128 K rows, both on tcgen05 with fp32 accumulators in
-// tensor memory:
+// Per tile of 128 rows, on tcgen05 with fp32 accumulators in tensor memory:
 //   MMA 1   Z = X Pi^T: X by TMA (128-byte swizzle) from a 3-deep ring, Pi
 //           resident in shared memory (bf16, exact products).
-//   epilogue A (one thread per row): ||x|| from the shared-memory tile, z from
-//           tensor memory, the codes against the thresholds scaled by ||x||
-//           (the exact saturating-FMA search of the MSE kernel), the residual
-//           r 2^14 = y 2^14 - c[code] 2^14 (the centroid selected by fused
-//           multiply-adds from the search's bits, exact), ||r||^2, and r 2^14
-//           split into two fp16 parts hi + lo written back over the row's Z
-//           columns in tensor memory (hi and lo of each 16 coordinates side by
-//           side: the A operand of MMA 2).
-//   MMA 2   S r = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T with A from tensor
-//           memory and S 2^sigma = S_hi + S_lo (fp16, resident in shared
-//           memory): 22 significant bits on each side, so the signs agree with
-//           an exact dot product wherever |S r| is above about 2^-21 |S| |r|.
-//   epilogue B: the signs (bit n of the row = [(S r)_n >= 0]) from tensor
-//           memory, then the stores: packed codes, fp16 ||x||, sign bits,
-//           fp16 ||r||.
-// Two epilogue warpgroups take alternate tiles, each with its own 256 columns
-// of tensor memory (Z / R, then S r), so one group's MMAs run while the other
-// computes.  One thread issues both GEMMs, polling the barriers of both
-// stages.  Every wait is bounded; on expiry the kernel flags the error and
-// stops, after waiting (bounded) for its copies and MMAs in flight, and
-// releases its tensor memory.
+//   epilogue A (two threads per row, 64 coordinates each): ||x|| from the
+//           shared-memory tile, z from tensor memory, the codes against the
+//           thresholds scaled by ||x|| (the exact saturating-FMA search of
+//           the MSE kernel); for K also the residual r 2^14 = y 2^14 -
+//           c[code] 2^14 (the centroid selected by fused multiply-adds from
+//           the search's bits, exact), ||r||^2, and r 2^14 split into two
+//           fp16 parts hi + lo written back over the row's Z columns in
+//           tensor memory (hi and lo of each 16 coordinates side by side: the
+//           A operand of MMA 2).
+//   MMA 2   (K) S r = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T with A from
+//           tensor memory and S 2^sigma = S_hi + S_lo (fp16, resident in
+//           shared memory): 22 significant bits on each side, so the signs
+//           agree with an exact dot product wherever |S r| is above about
+//           2^-21 |S| |r|.
+//   epilogue B (K): the signs (bit n of the row = [(S r)_n >= 0]) from
+//           tensor memory; then the stores: packed codes, fp16 ||x||, and for
+//           K the sign bits and fp16 ||r||.
+// The K tiles come first in the tile order and the cheaper V tiles fill the
+// tail.  Two tile groups (each two warpgroups, one per half row) take
+// alternate tiles with 256 columns of tensor memory each (Z / R, then S r),
+// so one group's MMAs run while the other computes.  One thread issues both
+// GEMMs, polling the barriers of both stages.  Every wait is bounded; on
+// expiry the kernel flags the error and stops, after waiting (bounded) for
+// its copies and MMAs in flight, and releases its tensor memory.
 #include <atomic>
 #include <cstring>
 
@@ -43,8 +46,8 @@ namespace tq {
 namespace {
 
 constexpr int kJStages = 3;                          // X ring depth
-constexpr int kJGroups = 2;                          // epilogue warpgroups
-constexpr int kJThreads = 32 * (2 + 4 * kJGroups);   // producer, MMA issuer, epilogue
+constexpr int kJGroups = 2;                          // tile groups (two warpgroups each)
+constexpr int kJThreads = 32 * (2 + 8 * kJGroups);   // producer, MMA issuer, epilogue
 constexpr unsigned kJTmemCols = 512;                 // per group: Z / R (128 columns), S r (128)
 constexpr int kJSmem = 1024 + kTileBytes * (3 + kJStages);  // Pi, S hi, S lo, the ring
 constexpr float kRScale = 0x1p14f;  // |r| < 1.3: r 2^14 stays below fp16's largest finite value
@@ -69,6 +72,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+
 // Non-blocking test of phase `parity`.
 __device__ __forceinline__ bool bar_test(uint32_t b, uint32_t parity) {
   uint32_t ok;
@@ -84,8 +88,8 @@ struct QjlTcArgs {
   tq_cache c;
   const int32_t *seq_idx;
   const int32_t *pos;
-  int n_rows;   // n_tok * n_kv_heads K rows
-  int n_tiles;  // tiles of 128 rows
+  int n_rows;   // n_tok * n_kv_heads rows per matrix
+  int tiles_k;  // K tiles (with QJL), then as many V tiles (MSE only)
 };
 
 // Centroid magnitudes of the positive half, times 2^14, and the differences
@@ -196,8 +200,8 @@ __device__ __forceinline__ uint32_t pack16_off(const float *off) {
   return __float_as_uint(acc.x + acc.y) & 0xFFFFu;
 }
 
-// Codes of coordinates 16 c .. 16 c + 15 into the cache words (code_chunk's
-// layout).
+// Codes of coordinates 16 c .. 16 c + 15 (c counted from the first of the
+// words in w) into the cache words (code_chunk's layout).
 template <int B>
 __device__ __forceinline__ void code_chunk_off(int c, const float (&off)[16], uint32_t (&w)[4 * B]) {
   if constexpr (B == 3) {
@@ -230,10 +234,13 @@ __device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, ui
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
-template <int BK>
+// 18 warps: one of the four schedulers holds five, whose registers (at most
+// 16384 per scheduler) cap a thread at 96
+template <int BK, int BV>
 __global__ void __launch_bounds__(kJThreads, 1)
-    quantize_qjl_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_pi,
-                           const __grid_constant__ CUtensorMap map_s, const QjlTcArgs a) {
+    quantize_qjl_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                           const __grid_constant__ CUtensorMap map_pi, const __grid_constant__ CUtensorMap map_s,
+                           const QjlTcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char *pi_tile = smem;                  // Pi, bf16
@@ -242,24 +249,30 @@ __global__ void __launch_bounds__(kJThreads, 1)
   unsigned char *ring = smem + 3 * kTileBytes;
   __shared__ __align__(8) uint64_t full_bar[kJStages], empty_bar[kJStages];
   __shared__ __align__(8) uint64_t zfull[kJGroups], rfull[kJGroups], sfull[kJGroups], tfree[kJGroups];
+  __shared__ __align__(8) uint64_t rr_bar[kJGroups];  // both halves' ||r||^2 written
   __shared__ __align__(8) uint64_t const_bar, mma_done;
+  __shared__ float s_rr[kJGroups][2][2][kTileRows];  // ||r||^2 of each half row, by tile parity
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // tiles t = blockIdx.x + i gridDim.x, i = 0 .. my_tiles - 1
-  const int my_tiles = (int)blockIdx.x < a.n_tiles ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int n_tiles = 2 * a.tiles_k;
+  // tiles t = blockIdx.x + i gridDim.x, i = 0 .. my_tiles - 1; the first my_k are K tiles
+  const int bx = (int)blockIdx.x, grid = (int)gridDim.x;
+  const int my_tiles = bx < n_tiles ? (n_tiles - 1 - bx) / grid + 1 : 0;
+  const int my_k = bx < a.tiles_k ? (a.tiles_k - 1 - bx) / grid + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kJStages; ++i) {
       bar_init(smem_addr(&full_bar[i]), 1);
-      bar_init(smem_addr(&empty_bar[i]), 1 + 4);  // MMA 1 commit + the 4 norm-reading warps
+      bar_init(smem_addr(&empty_bar[i]), 1 + 8);  // MMA 1 commit + the 8 norm-reading warps
     }
     for (int g = 0; g < kJGroups; ++g) {
       bar_init(smem_addr(&zfull[g]), 1);
-      bar_init(smem_addr(&rfull[g]), 4);
+      bar_init(smem_addr(&rfull[g]), 8);
       bar_init(smem_addr(&sfull[g]), 1);
-      bar_init(smem_addr(&tfree[g]), 4);
+      bar_init(smem_addr(&tfree[g]), 8);
+      bar_init(smem_addr(&rr_bar[g]), 8);
     }
     bar_init(smem_addr(&const_bar), 1);
     bar_init(smem_addr(&mma_done), 1);
@@ -303,12 +316,15 @@ __global__ void __launch_bounds__(kJThreads, 1)
           break;
         }
         if (*(volatile int *)&abort_flag) break;
-        const int row0 = ((int)blockIdx.x + i * (int)gridDim.x) * kTileRows;
+        const int t = bx + i * grid;
+        const bool is_k = i < my_k;
+        const int row0 = (is_k ? t : t - a.tiles_k) * kTileRows;
+        const CUtensorMap *map = is_k ? &map_k : &map_v;
         const uint32_t fb = smem_addr(&full_bar[slot]);
         unsigned char *st = ring + slot * kTileBytes;
         bar_expect_tx(fb, kTileBytes);
-        tma_load_2d(smem_addr(st), &map_x, 0, row0, fb);
-        tma_load_2d(smem_addr(st + kBoxBytes), &map_x, 64, row0, fb);
+        tma_load_2d(smem_addr(st), map, 0, row0, fb);
+        tma_load_2d(smem_addr(st + kBoxBytes), map, 64, row0, fb);
         issued = i + 1;
       }
       bar_wait(smem_addr(&const_bar), 0);
@@ -319,12 +335,12 @@ __global__ void __launch_bounds__(kJThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer: MMA 1 of the
     // next tile whenever its X has landed and its group's tensor memory is
-    // free, MMA 2 of the oldest tile whose residuals are written
+    // free, MMA 2 of the oldest K tile whose residuals are written
     if (lane == 0) {
       bool ok = bar_wait(smem_addr(&const_bar), 0);
       int n1 = 0, n2 = 0;
       unsigned long long t_last = global_ns();
-      while (ok && n2 < my_tiles) {
+      while (ok && n2 < my_k) {
         if (*(volatile int *)&abort_flag) break;
         bool progress = false;
         if (n1 < my_tiles) {
@@ -370,6 +386,23 @@ __global__ void __launch_bounds__(kJThreads, 1)
           __nanosleep(32);
         }
       }
+      // the V tiles need MMA 1 only
+      for (int i = n1; ok && i < my_tiles; ++i) {
+        const int slot = i % kJStages, g = i % kJGroups;
+        ok = bar_wait(smem_addr(&full_bar[slot]), (i / kJStages) & 1);
+        if (ok && i >= kJGroups) ok = bar_wait(smem_addr(&tfree[g]), ((i / kJGroups) - 1) & 1);
+        if (!ok || *(volatile int *)&abort_flag) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_addr(ring + slot * kTileBytes), b0 = smem_addr(pi_tile);
+        const uint32_t d = tmem_base + g * 256;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          tc_mma(d, sw128_desc(a0 + off), sw128_desc(b0 + off), kk > 0);
+        }
+        tc_commit(smem_addr(&zfull[g]));
+        tc_commit(smem_addr(&empty_bar[slot]));
+      }
       if (!ok) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
@@ -379,25 +412,29 @@ __global__ void __launch_bounds__(kJThreads, 1)
       bar_wait(smem_addr(&mma_done), 0);
     }
   } else {
-    // ------------------------------------------------ epilogue warpgroups
-    const int g = (warp - 2) / 4;
+    // ------------------------------------------------ epilogue: tile group g,
+    // half h of every row (coordinates and projections 64 h .. 64 h + 63)
+    const int g = (warp - 2) / 8, h = ((warp - 2) / 4) & 1;
     const int quarter = warp & 3;       // TMEM lanes 32 quarter .. + 31
-    const int r = 32 * quarter + lane;  // the row this thread owns
-    float tk[kMaxLevels];
-#pragma unroll
-    for (int e = 0; e < kMaxLevels; ++e) tk[e] = a.p.cb[1 * kMaxLevels + e];
+    const int r = 32 * quarter + lane;  // the row this thread shares
+    constexpr int hk = 1 << (BK - 1), hv = 1 << (BV - 1);
     ResConsts<BK> rc;
     res_consts<BK>(a.p.cb, rc);
-    constexpr int half = 1 << (BK - 1);
-    CodeConsts<BK> k;
+    CodeConsts<BK> kk;
+    CodeConsts<BV> kv;
 #pragma unroll
-    for (int j = 0; j < half - 1; ++j) k.nt[j] = -tk[half + j] * 0x1p64f;  // positive thresholds x -2^64
-    search_consts<BK>(k);
-    const uint32_t tz = tmem_base + g * 256 + ((uint32_t)(32 * quarter) << 16);
+    for (int j = 0; j < hk - 1; ++j) kk.nt[j] = -a.p.cb[1 * kMaxLevels + hk + j] * 0x1p64f;  // positive thresholds x -2^64
+#pragma unroll
+    for (int j = 0; j < hv - 1; ++j) kv.nt[j] = -a.p.cb[3 * kMaxLevels + hv + j] * 0x1p64f;
+    search_consts<BK>(kk);
+    search_consts<BV>(kv);
+    const uint32_t tz = tmem_base + g * 256 + 64 * h + ((uint32_t)(32 * quarter) << 16);
 
     for (int j = 0, i = g; i < my_tiles; ++j, i += kJGroups) {
       const int slot = i % kJStages;
-      const int row = ((int)blockIdx.x + i * (int)gridDim.x) * kTileRows + r;
+      const int t = bx + i * grid;
+      const bool is_k = i < my_k;
+      const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
       // destination, loaded now and checked after the codes
       const bool in_range = row < a.n_rows;
       const int tok = in_range ? row / a.c.n_kv_heads : 0;
@@ -409,7 +446,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
         break;
       }
       // ||x|| from the swizzled tile (chunk c of row r sits at c ^ (r % 8));
-      // bf16 squares are exact in fp32
+      // bf16 squares are exact in fp32.  Both halves read the whole row.
       const unsigned char *st = ring + slot * kTileBytes;
       float2 ss = make_float2(0.f, 0.f);
 #pragma unroll
@@ -429,7 +466,6 @@ __global__ void __launch_bounds__(kJThreads, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(smem_addr(&empty_bar[slot]));
 
-      // ---- epilogue A: codes, residuals, R into tensor memory
       if (!bar_wait(smem_addr(&zfull[g]), j & 1)) {
         atomicOr(a.p.err, kErrWaitExpired);
         abort_flag = 1;
@@ -437,69 +473,119 @@ __global__ void __launch_bounds__(kJThreads, 1)
       }
       tc_fence_after();
       const bool live = nrm > 0x1p-25f;  // stored fp16 norm nonzero
-      k.sc = live ? 0x1p64f / nrm : 0.f;
-      k.zc = live ? 0x1p127f : 0.f;
-      const float rinv = live ? kRScale / nrm : 0.f;
-      uint32_t words[4 * BK];
-      float2 rr = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float z[16];
-        tmem_ld16(tz + 16 * c, z);
-        float off[16];
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float2 o2, r2;
-          code_res2<BK>(z[2 * e], z[2 * e + 1], k, rc, rinv, o2, r2);
-          off[2 * e] = o2.x;
-          off[2 * e + 1] = o2.y;
-          rr = fma2(r2, r2, rr);
-          split_f16x2(r2.x, r2.y, hi[e], lo[e]);
-        }
-        code_chunk_off<BK>(c, off, words);
-        tmem_st8(tz + 16 * c, hi);
-        tmem_st8(tz + 16 * c + 8, lo);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(smem_addr(&rfull[g]));
-
-      // ---- epilogue B: the signs of S r
-      if (!bar_wait(smem_addr(&sfull[g]), j & 1)) {
-        atomicOr(a.p.err, kErrWaitExpired);
-        abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sb[4] = {0u, 0u, 0u, 0u};  // bit n of the row = [(S r)_n >= 0], LSB first
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v[16];
-        tmem_ld16(tz + 128 + 16 * c, v);
-        uint32_t b = 0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) b |= (v[e] >= 0.f ? 1u : 0u) << e;
-        sb[c >> 1] |= b << (16 * (c & 1));
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(smem_addr(&tfree[g]));
-
       long slot_i = -1;
       if (in_range) {
         slot_i = cache_slot(a.c, s_dst, tok_h, p_dst);
-        if (slot_i < 0 && tok_h == 0) atomicOr(a.p.err, kErrTokenRange);
+        if (slot_i < 0 && tok_h == 0 && h == 0 && is_k) atomicOr(a.p.err, kErrTokenRange);
       }
-      if (slot_i >= 0) {
-        uint4 *dst = reinterpret_cast<uint4 *>(a.c.codes_k + slot_i * (long)(16 * BK));
+      if (is_k) {
+        // ---- epilogue A: codes, residuals, R into tensor memory
+        kk.sc = live ? 0x1p64f / nrm : 0.f;
+        kk.zc = live ? 0x1p127f : 0.f;
+        const float rinv = live ? kRScale / nrm : 0.f;
+        uint32_t words[4 * BK];
+        float2 rr = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < BK; ++q) dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-        reinterpret_cast<uint4 *>(a.c.qjl_bits + slot_i * 16)[0] = make_uint4(sb[0], sb[1], sb[2], sb[3]);
-        a.c.norm_k[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
-        const float gamma = sqrtf(rr.x + rr.y) * (1.f / kRScale);
-        a.c.qjl_norm[slot_i] = __half_as_ushort(__float2half_rn(fminf(gamma, 65504.f)));
+        for (int c = 0; c < 4; ++c) {
+          float z[16];
+          tmem_ld16(tz + 16 * c, z);
+          float off[16];
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float2 o2, r2;
+            code_res2<BK>(z[2 * e], z[2 * e + 1], kk, rc, rinv, o2, r2);
+            off[2 * e] = o2.x;
+            off[2 * e + 1] = o2.y;
+            rr = fma2(r2, r2, rr);
+            split_f16x2(r2.x, r2.y, hi[e], lo[e]);
+          }
+          code_chunk_off<BK>(c, off, words);
+          tmem_st8(tz + 16 * c, hi);
+          tmem_st8(tz + 16 * c + 8, lo);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(smem_addr(&rfull[g]));
+        // ||r||^2 of the row from both halves (the group's eight warps meet on
+        // rr_bar; double-buffered by tile parity, so a half never overwrites a
+        // value its partner has yet to read)
+        s_rr[g][j & 1][h][r] = rr.x + rr.y;
+        __syncwarp();
+        if (lane == 0) bar_arrive(smem_addr(&rr_bar[g]));
+        if (!bar_wait(smem_addr(&rr_bar[g]), j & 1)) {
+          atomicOr(a.p.err, kErrWaitExpired);
+          abort_flag = 1;
+          break;
+        }
+        const float rr_row = s_rr[g][j & 1][0][r] + s_rr[g][j & 1][1][r];
+
+        // ---- epilogue B: the signs of S r
+        if (!bar_wait(smem_addr(&sfull[g]), j & 1)) {  // K tiles are a prefix: j K tiles before
+          atomicOr(a.p.err, kErrWaitExpired);
+          abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sb[2] = {0u, 0u};  // bit n of the row = [(S r)_n >= 0], LSB first, n = 64 h ..
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          tmem_ld16(tz + 128 + 16 * c, v);
+          uint32_t b = 0;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) b |= (v[e] >= 0.f ? 1u : 0u) << e;
+          sb[c >> 1] |= b << (16 * (c & 1));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(smem_addr(&tfree[g]));
+
+        if (slot_i >= 0) {
+          // code groups 2 h and 2 h + 1: 8 BK bytes from byte 8 BK h of the row
+          uint32_t *dst = reinterpret_cast<uint32_t *>(a.c.codes_k + slot_i * (long)(16 * BK) + 8 * BK * h);
+          if constexpr (BK == 3) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BK / 2; ++q)
+              reinterpret_cast<uint4 *>(dst)[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+          }
+          reinterpret_cast<uint2 *>(a.c.qjl_bits + slot_i * 16)[h] = make_uint2(sb[0], sb[1]);
+          if (h == 0) {
+            a.c.norm_k[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
+            const float gamma = sqrtf(rr_row) * (1.f / kRScale);
+            a.c.qjl_norm[slot_i] = __half_as_ushort(__float2half_rn(fminf(gamma, 65504.f)));
+          }
+        }
+      } else {
+        // ---- V: codes only
+        kv.sc = live ? 0x1p64f / nrm : 0.f;
+        kv.zc = live ? 0x1p127f : 0.f;
+        uint32_t words[4 * BV];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float z[16];
+          tmem_ld16(tz + 16 * c, z);
+          code_chunk<BV>(c, z, kv, words);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(smem_addr(&tfree[g]));
+        if (slot_i >= 0) {
+          uint32_t *dst = reinterpret_cast<uint32_t *>(a.c.codes_v + slot_i * (long)(16 * BV) + 8 * BV * h);
+          if constexpr (BV == 3) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BV / 2; ++q)
+              reinterpret_cast<uint4 *>(dst)[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+          }
+          if (h == 0) a.c.norm_v[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
+        }
       }
       if (*(volatile int *)&abort_flag) break;
     }
@@ -516,38 +602,42 @@ __global__ void __launch_bounds__(kJThreads, 1)
 }
 
 using QjlTcFn = void (*)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                         const __grid_constant__ CUtensorMap, const QjlTcArgs);
+                         const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap, const QjlTcArgs);
+
+template <int BK>
+QjlTcFn pick_bv(int bv) {
+  return bv == 2 ? quantize_qjl_tc_kernel<BK, 2> : bv == 3 ? quantize_qjl_tc_kernel<BK, 3> : quantize_qjl_tc_kernel<BK, 4>;
+}
 
 }  // namespace
 
-int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
-                           const int32_t *pos, int n_tok, void *stream) {
+int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
+                           const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream) {
   // cached per device (the attribute applies to the current device), and
   // atomically, as calls may come from several threads
   static std::atomic<int> cached_sm[kMaxDevices];
-  static std::atomic<bool> configured[kMaxDevices][3];
+  static std::atomic<bool> configured[kMaxDevices][3][3];
   const int dev = current_device();
   int n_sm = cached_sm[dev].load(std::memory_order_relaxed);
   if (n_sm == 0) {
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
     cached_sm[dev].store(n_sm, std::memory_order_relaxed);
   }
-  const QjlTcFn fn = p.bits_k == 2 ? quantize_qjl_tc_kernel<2>
-                     : p.bits_k == 3 ? quantize_qjl_tc_kernel<3>
-                                     : quantize_qjl_tc_kernel<4>;
-  std::atomic<bool> &done = configured[dev][p.bits_k - 2];
+  const QjlTcFn fn = p.bits_k == 2 ? pick_bv<2>(p.bits_v) : p.bits_k == 3 ? pick_bv<3>(p.bits_v) : pick_bv<4>(p.bits_v);
+  std::atomic<bool> &done = configured[dev][p.bits_k - 2][p.bits_v - 2];
   if (!done.load(std::memory_order_acquire)) {
     const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kJSmem);
     if (e != cudaSuccess) return (int)e;
     done.store(true, std::memory_order_release);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
-  CUtensorMap mx, mp, ms;
-  if (!make_row_map(&mx, k, rows) || !make_row_map(&mp, p.pi, kHeadDim) ||
+  CUtensorMap mk, mv, mp, ms;
+  if (!make_row_map(&mk, k, rows) || !make_row_map(&mv, v, rows) || !make_row_map(&mp, p.pi, kHeadDim) ||
       !make_row_map(&ms, p.ssplit, 2 * kHeadDim, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return (int)cudaErrorInvalidValue;
   QjlTcArgs args{p, c, seq_idx, pos, (int)rows, (int)((rows + kTileRows - 1) / kTileRows)};
-  const int grid = args.n_tiles < n_sm ? args.n_tiles : n_sm;
+  const int n_tiles = 2 * args.tiles_k;
+  const int grid = n_tiles < n_sm ? n_tiles : n_sm;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -558,7 +648,7 @@ int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void 
   cfg.stream = (cudaStream_t)stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  return (int)cudaLaunchKernelEx(&cfg, fn, mx, mp, ms, args);
+  return (int)cudaLaunchKernelEx(&cfg, fn, mk, mv, mp, ms, args);
 }
 
 }  // namespace tq
