@@ -166,18 +166,26 @@ static int sm_count() {
   return n;
 }
 
-// Splits of the sequence axis: about one full wave of resident CTAs
-// (SMs x CTAs per SM) over the (sequence, KV head) units, at least 8 splits
-// per unit when the units alone fill less than four waves (so ragged batches
-// balance), and at least 256 tokens per split.
+// Splits of the sequence axis.  Start from one wave of resident CTAs (SMs x
+// CTAs per SM) spread over the (sequence, KV head) units; take at least
+// min(8, four waves / units) splits per unit, so that ragged batches balance;
+// when the units hold fewer than four slots each (batches of many sequences,
+// whose lengths the host does not see), at least min(12, six waves / units)
+// (on the 32-sequence serving batch 11 splits decode 4.5 % faster than 7);
+// and at least 256 tokens per split.
 DecodeSplit decode_split(int n_seqs, int n_kv_heads, int max_seq_len, int ctas_per_sm) {
   if (ctas_per_sm > 4) ctas_per_sm = 4;
   if (ctas_per_sm < 1) ctas_per_sm = 1;
   const long units = (long)n_seqs * n_kv_heads;
   const long slots = (long)sm_count() * ctas_per_sm;
   long n = slots / units;
+  const long per_unit = n;
   const long balance = (4 * slots + units - 1) / units;
   if (n < (balance < 8 ? balance : 8)) n = balance < 8 ? balance : 8;
+  if (per_unit < 4) {
+    const long ragged = (6 * slots + units - 1) / units;
+    if (n < (ragged < 12 ? ragged : 12)) n = ragged < 12 ? ragged : 12;
+  }
   if (n < 1) n = 1;
   long chunk = ((long)max_seq_len + n - 1) / n;
   if (chunk < 256) chunk = 256;
