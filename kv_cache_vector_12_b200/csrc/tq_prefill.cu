@@ -642,40 +642,48 @@ int smem_of(int bk, int bv, bool qjl) {
 
 // ===========================================================================
 // The tcgen05 form (contexts without QJL).  Per CTA 128 query rows (the MMA's
-// M) and, per tile of 128 keys:
-//   expand   the four consumer warps turn the keys' codes into two fp16
-//            shared-memory operands in the 128-byte-swizzled K-major layout:
+// M) and, per tile of 128 keys, four roles that overlap across tiles:
+//   expand   (warps 4-7) the keys' codes into two fp16 shared-memory operands
+//            in the 128-byte-swizzled K-major layout, double-buffered:
 //            K~[key][kappa] (the exact fp16 K centroids, K fragment order)
 //            and V~^T[kappa_v][key] (fp16 V centroids, V fragment order);
-//   scores   one thread issues S = Q^_hi K~^T + Q^_lo K~^T (tcgen05.mma
-//            kind::f16, fp32 accumulator in tensor memory), q_hat as a
-//            two-part fp16 split scaled per row by a power of two;
-//   softmax  thread i owns row i: S from tensor memory, times the row's
-//            factor and the key norms, causal mask, online max and sum (exp2),
-//            P' = p ||v|| as fp16 into the swizzled A operand; a moved max
-//            rescales the row of O in tensor memory;
-//   values   O += P' V~ (tcgen05.mma, fp32 in tensor memory).
+//   MMA      (warp 9, one thread) S = Q^_hi K~^T + Q^_lo K~^T with the
+//            two-part fp16 q_hat (scaled per row by a power of two) as the A
+//            operand in tensor memory, and O += P' V~ with P' as the A
+//            operand in tensor memory; fp32 accumulators in tensor memory;
+//            the next tile's scores are issued as soon as the softmax has
+//            read the current ones;
+//   softmax  (warps 0-3) thread i owns row i: S from tensor memory, times the
+//            row's factor and the key norms, causal mask, online max and sum
+//            (exp2), P' = p ||v|| as fp16 into tensor memory; a moved max
+//            rescales the row of O;
+//   producer (warp 8) streams the codes with 1-D bulk copies.
 // At the end o = Pi^T (O / l) is one more pair of MMAs (O as bf16 hi + lo,
 // Pi^T's rows in the V fragment order as the B operand), and the lse.
-// A producer warp streams the codes with 1-D bulk copies.  Every mbarrier
-// wait is bounded.
+// Tensor memory: S at columns 0-127, O at 128-255, q_hat hi and lo at
+// 256-319 and 320-383, P' at 384-447.  Every mbarrier wait is bounded.
 // ===========================================================================
 namespace tq {
 namespace {
 
 constexpr int kTcRows = 128;                      // query rows per CTA
 constexpr int kTcKeys = 128;                      // keys per tile
-constexpr int kTcWarps = 4;
-constexpr int kTcThreads = 32 * (kTcWarps + 1);
+constexpr int kTcSoftWarps = 4;                   // warps 0-3
+constexpr int kTcExpWarp0 = 4;                    // warps 4-7 expand
+constexpr int kTcProdWarp = 8, kTcMmaWarp = 9;
+constexpr int kTcThreads = 32 * 10;
 constexpr int kTcStages = 2;
 constexpr int kOpBytes = 128 * kHeadDim * 2;      // one 128 x 128 16-bit operand: two 128 x 64 swizzled boxes
 constexpr int kOpBox = kOpBytes / 2;
-constexpr uint32_t kTcCols = 256;                 // S at columns 0 .. 127, O at 128 .. 255
+constexpr uint32_t kTcCols = 512;
+constexpr uint32_t kTcS = 0, kTcO = 128, kTcQ = 256, kTcP = 384;  // tensor-memory columns
 
 template <int BK, int BV>
 struct TcLayout {
-  static constexpr int qhi = 0, qlo = kOpBytes, kt = 2 * kOpBytes, vt = 3 * kOpBytes, pt = 4 * kOpBytes;
-  static constexpr int ring = 5 * kOpBytes;
+  // K~ buffers 0, 1; V~ buffers 0, 1 (the prologue's fp32 q_hat scratch
+  // spans both K~ buffers; the epilogue's operands reuse K~ and V~ 0)
+  static constexpr int kt0 = 0, kt1 = kOpBytes, vt0 = 2 * kOpBytes, vt1 = 3 * kOpBytes;
+  static constexpr int ring = 4 * kOpBytes;
   static constexpr int stage = Stage<BK, BV, false, kTcKeys>::bytes;
   static constexpr int bytes = ring + kTcStages * stage + 1024;  // + alignment slack
 };
@@ -683,9 +691,6 @@ struct TcLayout {
 __device__ __forceinline__ void tcx_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tcx_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(32 * kTcWarps) : "memory");
-}
 
 // Byte offset of element (row, col) of a 128 x 128 16-bit operand stored as
 // two boxes of 128 rows x 64 columns, 128-byte rows, 16-byte chunks swizzled
@@ -706,10 +711,19 @@ __device__ __forceinline__ uint64_t swdesc(uint32_t addr) {
 constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescBF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
+// D += A B with A and B in shared memory.
 __device__ __forceinline__ void tcx_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
   asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
                    tmem_d),
                "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+// D += A B with A in tensor memory (fp16, two elements per 32-bit column)
+// and B in shared memory.
+__device__ __forceinline__ void tcx_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t accumulate) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+                   tmem_d),
+               "r"(tmem_a), "l"(b), "r"(kIdescF16), "r"(accumulate)
                : "memory");
 }
 __device__ __forceinline__ void tcx_commit(uint32_t bar) {
@@ -740,13 +754,136 @@ __device__ __forceinline__ void f16_pairs(uint32_t lo, uint32_t hi, uint32_t &p0
   p23 = prmt(lo, hi, 0x7362u);
 }
 
+// K~ and V~^T of one tile of keys (ew: the expanding warp 0-3, keys
+// 32 ew .. 32 ew + 31) into the operand buffers kt and vt.
+template <int BK, int BV>
+__device__ __forceinline__ void expand_tile(const unsigned char *st, unsigned char *kt, unsigned char *vt,
+                                            const Lut &lkf, const Lut &lv, int ew, int r, int q) {
+  using St = Stage<BK, BV, false, kTcKeys>;
+#pragma unroll
+  for (int rb = 0; rb < 2; ++rb) {
+    const int k0 = 32 * ew + 16 * rb + r, k1 = k0 + 8;
+    uint32_t wk0[BK], wk1[BK];
+    const unsigned char *kr0 = st + St::kc + k0 * (D * BK / 8) + q * 4 * BK;
+    const unsigned char *kr1 = st + St::kc + k1 * (D * BK / 8) + q * 4 * BK;
+#pragma unroll
+    for (int i = 0; i < BK; ++i) {
+      wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
+      wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
+    }
+#pragma unroll
+    for (int sg = 0; sg < 8; ++sg) {
+      const int kap = 32 * (sg >> 1) + 16 * (sg & 1) + 4 * q;
+      uint32_t lo, hi, p01, p23;
+      lookup<BK>(lkf, k_selector<BK>(wk0, sg), lo, hi);
+      f16_pairs(lo, hi, p01, p23);
+      *reinterpret_cast<uint2 *>(kt + sw_off(k0, kap)) = make_uint2(p01, p23);
+      lookup<BK>(lkf, k_selector<BK>(wk1, sg), lo, hi);
+      f16_pairs(lo, hi, p01, p23);
+      *reinterpret_cast<uint2 *>(kt + sw_off(k1, kap)) = make_uint2(p01, p23);
+    }
+  }
+#pragma unroll
+  for (int rb = 0; rb < 2; ++rb) {
+    // V~^T: rows in the V fragment order, keys as columns (decode's A
+    // fragments: a0 = row 16 mt + r, keys 2q, 2q+1; a1 = row + 8; a2, a3:
+    // keys + 8)
+    constexpr int VB = D * BV / 8;
+    const int kb = 32 * ew + 16 * rb;  // first key of the 16-key block
+    const unsigned char *vc = st + St::vc + (kb + 2 * q) * VB;
+    auto put = [&](int mt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+      *reinterpret_cast<uint32_t *>(vt + sw_off(16 * mt + r, kb + 2 * q)) = a0;
+      *reinterpret_cast<uint32_t *>(vt + sw_off(16 * mt + r + 8, kb + 2 * q)) = a1;
+      *reinterpret_cast<uint32_t *>(vt + sw_off(16 * mt + r, kb + 8 + 2 * q)) = a2;
+      *reinterpret_cast<uint32_t *>(vt + sw_off(16 * mt + r + 8, kb + 8 + 2 * q)) = a3;
+    };
+    if constexpr (BV == 3) {
+      const int gofs = 12 * (r >> 1);
+      const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
+      uint32_t ya[3], yb[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        ya[k] = prmt(reinterpret_cast<const uint32_t *>(vc + gofs)[k],
+                     reinterpret_cast<const uint32_t *>(vc + VB + gofs)[k], gs);
+        yb[k] = prmt(reinterpret_cast<const uint32_t *>(vc + 8 * VB + gofs)[k],
+                     reinterpret_cast<const uint32_t *>(vc + 9 * VB + gofs)[k], gs);
+      }
+      const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
+        const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t a0, a1, a2, a3;
+          v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
+          v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
+          put(2 * k + hh, a0, a1, a2, a3);
+        }
+      }
+    } else if constexpr (BV == 2) {
+      const uint32_t A0 = reinterpret_cast<const uint32_t *>(vc)[r];
+      const uint32_t B0 = reinterpret_cast<const uint32_t *>(vc + VB)[r];
+      const uint32_t A1 = reinterpret_cast<const uint32_t *>(vc + 8 * VB)[r];
+      const uint32_t B1 = reinterpret_cast<const uint32_t *>(vc + 9 * VB)[r];
+#pragma unroll
+      for (int yh = 0; yh < 2; ++yh) {
+        const uint32_t gs = yh ? 0x7362u : 0x5140u;
+        const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+        for (int par = 0; par < 2; ++par) {
+          const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t a0, a1, a2, a3;
+            v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
+            v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
+            put(4 * yh + 2 * par + hh, a0, a1, a2, a3);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t A0 = reinterpret_cast<const uint32_t *>(vc)[2 * r + u];
+        const uint32_t B0 = reinterpret_cast<const uint32_t *>(vc + VB)[2 * r + u];
+        const uint32_t A1 = reinterpret_cast<const uint32_t *>(vc + 8 * VB)[2 * r + u];
+        const uint32_t B1 = reinterpret_cast<const uint32_t *>(vc + 9 * VB)[2 * r + u];
+#pragma unroll
+        for (int yh = 0; yh < 2; ++yh) {
+          const uint32_t gs = yh ? 0x7362u : 0x5140u;
+          const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t a0, a1, a2, a3;
+            v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
+            v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
+            put(4 * u + 2 * yh + hh, a0, a1, a2, a3);
+          }
+        }
+      }
+    }
+  }
+}
+
+// A wait on the kernel's flag or on a barrier; false (and the error flagged,
+// the kernel told to stop) once the barrier's bounded wait expires.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, unsigned *err, int *abort_flag) {
+  if (mbar_wait(smem_u32(bar), parity)) return true;
+  atomicOr(err, kErrWaitExpired);
+  *(volatile int *)abort_flag = 1;
+  return false;
+}
+
 template <int BK, int BV>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const PrefillArgs a) {
   using L = TcLayout<BK, BV>;
   using St = Stage<BK, BV, false, kTcKeys>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages], s_bar, pv_bar;
+  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
+  __shared__ __align__(8) uint64_t kv_full[2], kv_empty[2], s_full, s_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t q_ready, scratch_free, o_ready, fin_bar, mma_done;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int s_pos[kTcRows];
@@ -771,6 +908,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   const int n_tiles = (kend + kTcKeys - 1) / kTcKeys;
   const long base = ((long)s * a.c.n_kv_heads + h) * a.c.capacity;
   const long qrow0 = (long)q0 * a.n_q_heads + (long)h * G;
+  unsigned *err = a.p.err;
 
   if (tid < kTcRows) {
     const int qi = first_q + tid / G;
@@ -779,14 +917,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   if (tid == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
-      mbar_init(smem_u32(&empty_bar[i]), kTcWarps);
+      mbar_init(smem_u32(&empty_bar[i]), 8);  // the expanding and the softmax warps
     }
-    mbar_init(smem_u32(&s_bar), 1);
-    mbar_init(smem_u32(&pv_bar), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&kv_full[b]), 4);
+      mbar_init(smem_u32(&kv_empty[b]), 1);
+    }
+    mbar_init(smem_u32(&s_full), 1);
+    mbar_init(smem_u32(&s_empty), 4);
+    mbar_init(smem_u32(&p_full), 4);
+    mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&q_ready), 4);
+    mbar_init(smem_u32(&scratch_free), 4);
+    mbar_init(smem_u32(&o_ready), 4);
+    mbar_init(smem_u32(&fin_bar), 1);
+    mbar_init(smem_u32(&mma_done), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == kTcMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
                  "r"(kTcCols)
                  : "memory");
@@ -796,20 +945,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   __syncthreads();
   tcx_fence_after();
   const uint32_t tmem = tmem_slot;
-  const uint32_t t_s = tmem, t_o = tmem + 128;
+  int *abf = &abort_flag;
 
-  if (warp == kTcWarps) {
+  if (warp == kTcProdWarp) {
     // ---------------- producer: the codes of one tile of keys per stage
     if (lane == 0) {
       int issued = 0;
       for (int it = 0; it < n_tiles; ++it) {
         const int slot = it % kTcStages;
-        if (it >= kTcStages && !mbar_wait(smem_u32(&empty_bar[slot]), ((it / kTcStages) - 1) & 1)) {
-          atomicOr(a.p.err, kErrWaitExpired);
-          abort_flag = 1;
-          break;
-        }
-        if (*(volatile int *)&abort_flag) break;
+        if (it >= kTcStages && !tc_wait(&empty_bar[slot], ((it / kTcStages) - 1) & 1, err, abf)) break;
+        if (*(volatile int *)abf) break;
         unsigned char *st = sm + L::ring + slot * L::stage;
         const uint32_t bar = smem_u32(&full_bar[slot]);
         const int first = it * kTcKeys;
@@ -823,7 +968,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
             run = min(run, (uint32_t)(a.c.block_size - off));
             int bl = a.c.block_table[(long)s * (a.c.capacity / a.c.block_size) + j];
             if (bl < 0 || bl >= a.c.n_blocks) {
-              atomicOr(a.p.err, kErrTokenRange);
+              atomicOr(err, kErrTokenRange);
               bl = 0;
             }
             tok = ((long)bl * a.c.n_kv_heads + h) * a.c.block_size + off;
@@ -840,20 +985,109 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         }
         issued = it + 1;
       }
-      if (*(volatile int *)&abort_flag) {
+      if (*(volatile int *)abf) {  // never leave copies in flight
         for (int it = max(0, issued - kTcStages); it < issued; ++it)
           mbar_wait(smem_u32(&full_bar[it % kTcStages]), (it / kTcStages) & 1);
       }
     }
+  } else if (warp == kTcMmaWarp) {
+    // ---------------- MMA issuer: S(it + 1) as soon as the softmax has read
+    // S(it), then O += P'(it) V~(it)
+    if (lane == 0) {
+      const uint32_t t_s = tmem + kTcS, t_o = tmem + kTcO, t_q = tmem + kTcQ, t_p = tmem + kTcP;
+      auto scores = [&](int it) {
+        const uint32_t bk = smem_u32(sm + ((it & 1) ? L::kt1 : L::kt0));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+          tcx_mma_ts(t_s, t_q + 8 * kk, swdesc(bk + off), kk > 0);  // q_hat hi
+          tcx_mma_ts(t_s, t_q + 64 + 8 * kk, swdesc(bk + off), 1);  // q_hat lo
+        }
+        tcx_commit(smem_u32(&s_full));
+      };
+      bool ok = tc_wait(&q_ready, 0, err, abf) && tc_wait(&kv_full[0], 0, err, abf);
+      if (ok) {
+        tcx_fence_after();
+        scores(0);
+      }
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        if (it + 1 < n_tiles) {
+          ok = tc_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1, err, abf) && tc_wait(&s_empty, it & 1, err, abf);
+          if (!ok || *(volatile int *)abf) break;
+          tcx_fence_after();
+          scores(it + 1);
+        }
+        ok = tc_wait(&p_full, it & 1, err, abf);
+        if (!ok || *(volatile int *)abf) break;
+        tcx_fence_after();
+        const uint32_t bv = smem_u32(sm + ((it & 1) ? L::vt1 : L::vt0));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+          tcx_mma_ts(t_o, t_p + 8 * kk, swdesc(bv + off), (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        tcx_commit(smem_u32(&pv_done));
+        tcx_commit(smem_u32(&kv_empty[it & 1]));
+      }
+      // o = Pi^T (O / l): A = O as bf16 hi + lo (over K~ 0 and 1), B = Pi^T's
+      // rows in the V fragment order (over V~ 0)
+      if (ok && !*(volatile int *)abf) {
+        ok = tc_wait(&o_ready, 0, err, abf);
+        if (ok) {
+          tcx_fence_after();
+          const uint32_t ah = smem_u32(sm + L::kt0), alo = smem_u32(sm + L::kt1), bp = smem_u32(sm + L::vt0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
+            tcx_mma(t_s, swdesc(ah + off), swdesc(bp + off), kIdescBF16, kk > 0);
+            tcx_mma(t_s, swdesc(alo + off), swdesc(bp + off), kIdescBF16, 1);
+          }
+          tcx_commit(smem_u32(&fin_bar));
+        }
+      }
+      // every MMA issued here has completed before the tensor memory is released
+      tcx_commit(smem_u32(&mma_done));
+      mbar_wait(smem_u32(&mma_done), 0);
+    }
+  } else if (warp >= kTcExpWarp0) {
+    // ---------------- expansion: K~ and V~ of every tile, double-buffered
+    const int ew = warp - kTcExpWarp0;
+    Lut lkf;  // the K centroids as fp16 byte tables (exact: the centroids are fp16 values)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lkf.lo[i] = lkf.hi[i] = 0u;
+    for (int e = 0; e < (1 << BK); ++e) {
+      const uint16_t hb = __half_as_ushort(__float2half_rn(a.p.cb[e]));
+      lkf.lo[e / 4] |= (uint32_t)(hb & 0xff) << (8 * (e % 4));
+      lkf.hi[e / 4] |= (uint32_t)(hb >> 8) << (8 * (e % 4));
+    }
+    const Lut lv = a.p.lut_v;
+    // the first expansion overwrites the softmax warps' q_hat scratch
+    bool ok = tc_wait(&scratch_free, 0, err, abf);
+    for (int it = 0; ok && it < n_tiles; ++it) {
+      const int slot = it % kTcStages, b = it & 1;
+      ok = tc_wait(&full_bar[slot], (it / kTcStages) & 1, err, abf);
+      if (ok && it >= 2) ok = tc_wait(&kv_empty[b], ((it >> 1) - 1) & 1, err, abf);
+      if (!ok || *(volatile int *)abf) break;
+      tcx_fence_after();
+      const unsigned char *st = sm + L::ring + slot * L::stage;
+      expand_tile<BK, BV>(st, sm + (b ? L::kt1 : L::kt0), sm + (b ? L::vt1 : L::vt0), lkf, lv, ew, r, q);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&kv_full[b]));
+        mbar_arrive(smem_u32(&empty_bar[slot]));  // the codes are read
+      }
+    }
   } else {
-    // ---------------- consumers: thread tid owns query row tid
+    // ---------------- softmax warps: thread tid owns query row tid
     const int row = tid, pos = s_pos[row];
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;  // this warp's TMEM lane quarter
+    const uint32_t t_s = tmem + kTcS + lane_off, t_o = tmem + kTcO + lane_off;
+    const uint32_t t_q = tmem + kTcQ + lane_off, t_p = tmem + kTcP + lane_off;
     // q_hat = Pi q in the K fragment order (Pi's rows stored in that order),
     // mma m16n8k16 bf16, fp32 q as hi + lo; warp w computes rows 32 w ..
-    // 32 w + 31 into a fp32 scratch (the V~ and P' regions, free until the
-    // first tile)
-    float *scr = reinterpret_cast<float *>(sm + L::vt);  // [128 rows][128], 64 KB over vt and pt
+    // 32 w + 31 into a fp32 scratch over the K~ buffers
+    float *scr = reinterpret_cast<float *>(sm + L::kt0);  // [128 rows][128], 64 KB
     {
       const bool f32 = a.q_dtype == TQ_F32;
 #pragma unroll 1
@@ -903,7 +1137,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     }
     __syncwarp();
     // per row: a power-of-two scale puts max |q_hat| in [2^13, 2^14), then
-    // q_hat = hi + lo in fp16 into the swizzled A operands
+    // q_hat = hi + lo in fp16 into tensor memory (the scores' A operand)
     float fq;
     {
       const float *qr = scr + row * D;
@@ -913,169 +1147,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       if (m > 0.f) frexpf(m, &ex);
       const float sc = m > 0.f ? ldexpf(1.f, 14 - ex) : 1.f;
       fq = a.scale * kLog2e / sc;
-#pragma unroll 4
-      for (int k0 = 0; k0 < D; k0 += 8) {
-        const int k = (k0 + 8 * lane) & (D - 1);  // lane-rotated chunks spread the shared-memory banks
-        uint32_t hi[4], lo[4];
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split_f16x2(qr[k + 2 * e] * sc, qr[k + 2 * e + 1] * sc, hi[e], lo[e]);
-        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, k)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, k)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int e = 0; e < 16; ++e) split_f16x2(qr[32 * c + 2 * e] * sc, qr[32 * c + 2 * e + 1] * sc, hi[e], lo[e]);
+        tmem_st16x(t_q + 16 * c, hi);
+        tmem_st16x(t_q + 64 + 16 * c, lo);
       }
+      tmem_wait_st();
     }
-    // the K centroids as fp16 byte tables (exact: the centroids are fp16 values)
-    Lut lkf;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) lkf.lo[i] = lkf.hi[i] = 0u;
-    for (int e = 0; e < (1 << BK); ++e) {
-      const uint16_t hb = __half_as_ushort(__float2half_rn(a.p.cb[e]));
-      lkf.lo[e / 4] |= (uint32_t)(hb & 0xff) << (8 * (e % 4));
-      lkf.hi[e / 4] |= (uint32_t)(hb >> 8) << (8 * (e % 4));
+    tcx_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(smem_u32(&q_ready));
+      mbar_arrive(smem_u32(&scratch_free));  // this warp's scratch rows are read
     }
-    const Lut lv = a.p.lut_v;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    tc_consumer_sync();  // the scratch is read: the first tile may overwrite it
-
-    for (int it = 0; it < n_tiles && ok; ++it) {
+    for (int it = 0; ok && it < n_tiles; ++it) {
       const int slot = it % kTcStages;
-      ok = mbar_wait(smem_u32(&full_bar[slot]), (it / kTcStages) & 1);
+      // the stage's key norms (its copies are complete) and S(it)
+      ok = tc_wait(&full_bar[slot], (it / kTcStages) & 1, err, abf) && tc_wait(&s_full, it & 1, err, abf);
       if (!ok) break;
       tcx_fence_after();
       const unsigned char *st = sm + L::ring + slot * L::stage;
-      // K~ is free (the previous scores were waited for): expand it while the
-      // previous tile's value MMAs run, then issue this tile's scores
-      // ---------------- expand: warp w takes keys 32 w .. 32 w + 31 of the tile
-#pragma unroll
-      for (int rb = 0; rb < 2; ++rb) {
-        const int k0 = 32 * warp + 16 * rb + r, k1 = k0 + 8;
-        uint32_t wk0[BK], wk1[BK];
-        const unsigned char *kr0 = st + St::kc + k0 * (D * BK / 8) + q * 4 * BK;
-        const unsigned char *kr1 = st + St::kc + k1 * (D * BK / 8) + q * 4 * BK;
-#pragma unroll
-        for (int i = 0; i < BK; ++i) {
-          wk0[i] = reinterpret_cast<const uint32_t *>(kr0)[i];
-          wk1[i] = reinterpret_cast<const uint32_t *>(kr1)[i];
-        }
-#pragma unroll
-        for (int sg = 0; sg < 8; ++sg) {
-          const int kap = 32 * (sg >> 1) + 16 * (sg & 1) + 4 * q;
-          uint32_t lo, hi, p01, p23;
-          lookup<BK>(lkf, k_selector<BK>(wk0, sg), lo, hi);
-          f16_pairs(lo, hi, p01, p23);
-          *reinterpret_cast<uint2 *>(sm + L::kt + sw_off(k0, kap)) = make_uint2(p01, p23);
-          lookup<BK>(lkf, k_selector<BK>(wk1, sg), lo, hi);
-          f16_pairs(lo, hi, p01, p23);
-          *reinterpret_cast<uint2 *>(sm + L::kt + sw_off(k1, kap)) = make_uint2(p01, p23);
-        }
-      }
-      fence_async_smem();
-      tcx_fence_before();
-      tc_consumer_sync();
-      if (tid == 0) {  // ---------------- S = Q^_hi K~^T + Q^_lo K~^T
-        tcx_fence_after();
-        const uint32_t aq = smem_u32(sm + L::qhi), al = smem_u32(sm + L::qlo), bk = smem_u32(sm + L::kt);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
-          tcx_mma(t_s, swdesc(aq + off), swdesc(bk + off), kIdescF16, kk > 0);
-          tcx_mma(t_s, swdesc(al + off), swdesc(bk + off), kIdescF16, 1);
-        }
-        tcx_commit(smem_u32(&s_bar));
-      }
-      // the previous tile's value MMAs read V~ and P' and write O: wait for
-      // them, then expand V~ while this tile's scores run
-      if (it > 0) ok = mbar_wait(smem_u32(&pv_bar), (it - 1) & 1);
-      if (!ok) break;
-      tcx_fence_after();
-      // ---------------- V~^T for the same keys
-#pragma unroll
-      for (int rb = 0; rb < 2; ++rb) {
-        // V~^T: rows in the V fragment order, keys as columns (decode's A
-        // fragments: a0 = row 16 mt + r, keys 2q, 2q+1; a1 = row + 8; a2, a3:
-        // keys + 8)
-        constexpr int VB = D * BV / 8;
-        const int kb = 32 * warp + 16 * rb;  // first key of the 16-key block
-        const unsigned char *vt = st + St::vc + (kb + 2 * q) * VB;
-        auto put = [&](int mt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-          unsigned char *vb = sm + L::vt;
-          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r, kb + 2 * q)) = a0;
-          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r + 8, kb + 2 * q)) = a1;
-          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r, kb + 8 + 2 * q)) = a2;
-          *reinterpret_cast<uint32_t *>(vb + sw_off(16 * mt + r + 8, kb + 8 + 2 * q)) = a3;
-        };
-        if constexpr (BV == 3) {
-          const int gofs = 12 * (r >> 1);
-          const uint32_t gs = (r & 1) ? 0x7362u : 0x5140u;
-          uint32_t ya[3], yb[3];
-#pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            ya[k] = prmt(reinterpret_cast<const uint32_t *>(vt + gofs)[k],
-                         reinterpret_cast<const uint32_t *>(vt + VB + gofs)[k], gs);
-            yb[k] = prmt(reinterpret_cast<const uint32_t *>(vt + 8 * VB + gofs)[k],
-                         reinterpret_cast<const uint32_t *>(vt + 9 * VB + gofs)[k], gs);
-          }
-          const uint32_t spa = spare3(ya[0], ya[1], ya[2]), spb = spare3(yb[0], yb[1], yb[2]);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t za = k < 3 ? (ya[k < 3 ? k : 0] & 0x77777777u) : spa;
-            const uint32_t zb = k < 3 ? (yb[k < 3 ? k : 0] & 0x77777777u) : spb;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              uint32_t a0, a1, a2, a3;
-              v_pairs<3>(lv, hh ? za >> 16 : za, a0, a1);
-              v_pairs<3>(lv, hh ? zb >> 16 : zb, a2, a3);
-              put(2 * k + hh, a0, a1, a2, a3);
-            }
-          }
-        } else if constexpr (BV == 2) {
-          const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[r];
-          const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[r];
-          const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[r];
-          const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[r];
-#pragma unroll
-          for (int yh = 0; yh < 2; ++yh) {
-            const uint32_t gs = yh ? 0x7362u : 0x5140u;
-            const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
-#pragma unroll
-            for (int par = 0; par < 2; ++par) {
-              const uint32_t za = (ya >> (2 * par)) & 0x33333333u, zb = (yb >> (2 * par)) & 0x33333333u;
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                uint32_t a0, a1, a2, a3;
-                v_pairs<2>(lv, hh ? za >> 16 : za, a0, a1);
-                v_pairs<2>(lv, hh ? zb >> 16 : zb, a2, a3);
-                put(4 * yh + 2 * par + hh, a0, a1, a2, a3);
-              }
-            }
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t A0 = reinterpret_cast<const uint32_t *>(vt)[2 * r + u];
-            const uint32_t B0 = reinterpret_cast<const uint32_t *>(vt + VB)[2 * r + u];
-            const uint32_t A1 = reinterpret_cast<const uint32_t *>(vt + 8 * VB)[2 * r + u];
-            const uint32_t B1 = reinterpret_cast<const uint32_t *>(vt + 9 * VB)[2 * r + u];
-#pragma unroll
-            for (int yh = 0; yh < 2; ++yh) {
-              const uint32_t gs = yh ? 0x7362u : 0x5140u;
-              const uint32_t ya = prmt(A0, B0, gs), yb = prmt(A1, B1, gs);
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                uint32_t a0, a1, a2, a3;
-                v_pairs<4>(lv, hh ? ya >> 16 : ya, a0, a1);
-                v_pairs<4>(lv, hh ? yb >> 16 : yb, a2, a3);
-                put(4 * u + 2 * yh + hh, a0, a1, a2, a3);
-              }
-            }
-          }
-        }
-      }
-      // V~ is published to the tensor cores with P' before the value MMAs
-      ok = mbar_wait(smem_u32(&s_bar), it & 1);
-      if (!ok) break;
-      tcx_fence_after();
-      // ---------------- softmax of row `row` over the tile's keys
       const __half *kn = reinterpret_cast<const __half *>(st + St::kn);
       const __half *vn = reinterpret_cast<const __half *>(st + St::vn);
       const int kfirst = it * kTcKeys;
@@ -1084,7 +1180,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
 #pragma unroll
       for (int c = 0; c < kTcKeys / 16; ++c) {
         uint32_t v[16];
-        tmem_ld16x(t_s + lane_off + 16 * c, v);
+        tmem_ld16x(t_s + 16 * c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -1094,96 +1190,85 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
           mx = fmaxf(mx, sc[j]);
         }
       }
+      // S is read: the next tile's scores may overwrite it
+      tcx_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_empty));
       const float mn = fmaxf(m_run, mx);
       const float ref = fmaxf(mn, -3.0e38f);
       const float al = fast_exp2(m_run - ref);
       m_run = mn;
       float ls = 0.f;
+      uint32_t pk[kTcKeys / 2];
 #pragma unroll
-      for (int c = 0; c < kTcKeys / 8; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 8 * c + 2 * e;
-          const float pa = fast_exp2(sc[j] - ref), pb = fast_exp2(sc[j + 1] - ref);
-          ls += pa + pb;
-          pk[e] = pack_half2(sc[j] == -INFINITY ? 0.f : pa * __half2float(vn[j]),
-                             sc[j + 1] == -INFINITY ? 0.f : pb * __half2float(vn[j + 1]));
-        }
-        *reinterpret_cast<uint4 *>(sm + L::pt + sw_off(row, 8 * c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < kTcKeys / 2; ++e) {
+        const int j = 2 * e;
+        const float pa = fast_exp2(sc[j] - ref), pb = fast_exp2(sc[j + 1] - ref);
+        ls += pa + pb;
+        pk[e] = pack_half2(sc[j] == -INFINITY ? 0.f : pa * __half2float(vn[j]),
+                           sc[j + 1] == -INFINITY ? 0.f : pb * __half2float(vn[j + 1]));
       }
       l_run = fmaf(l_run, al, ls);
-      // the norms are read: the producer may refill this stage
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));
-      // a moved maximum rescales this warp's rows of O (O is complete: the
-      // previous tile's values were waited for above)
-      if (it > 0 && __any_sync(0xffffffffu, al != 1.f)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t v[16];
-          tmem_ld16x(t_o + lane_off + 16 * c, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
-          tmem_st16x(t_o + lane_off + 16 * c, v);
-        }
-        tmem_wait_st();
-      }
-      fence_async_smem();
-      tcx_fence_before();
-      tc_consumer_sync();
-      if (tid == 0) {  // ---------------- O += P' V~
+      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));  // the norms are read
+      // the previous tile's value MMAs read P' and write O: wait for them,
+      // then rescale O on a moved maximum and write this tile's P'
+      if (it > 0) {
+        ok = tc_wait(&pv_done, (it - 1) & 1, err, abf);
+        if (!ok) break;
         tcx_fence_after();
-        const uint32_t ap = smem_u32(sm + L::pt), bv = smem_u32(sm + L::vt);
+        if (__any_sync(0xffffffffu, al != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t v[16];
+            tmem_ld16x(t_o + 16 * c, v);
+            tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
-          tcx_mma(t_o, swdesc(ap + off), swdesc(bv + off), kIdescF16, (it > 0 || kk > 0) ? 1u : 0u);
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
+            tmem_st16x(t_o + 16 * c, v);
+          }
         }
-        tcx_commit(smem_u32(&pv_bar));
       }
+#pragma unroll
+      for (int c = 0; c < kTcKeys / 32; ++c) {
+        uint32_t v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = pk[16 * c + e];
+        tmem_st16x(t_p + 16 * c, v);
+      }
+      tmem_wait_st();
+      tcx_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_full));
     }
-    // ---------------- o = Pi^T (O / l): O as bf16 hi + lo (A, over the Q^
-    // operands), Pi^T with its rows in the V fragment order (B, over K~)
-    if (ok) ok = mbar_wait(smem_u32(&pv_bar), (n_tiles - 1) & 1);
+    // ---------------- o = Pi^T (O / l)
+    if (ok) ok = tc_wait(&pv_done, (n_tiles - 1) & 1, err, abf);
     if (ok) {
       tcx_fence_after();
-      float l = l_run;
-      const float il = l > 0.f ? 1.f / l : 0.f;
+      const float il = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 16; ++c) {
         uint32_t v[16];
-        tmem_ld16x(t_o + lane_off + 16 * c, v);
+        tmem_ld16x(t_o + 16 * c, v);
         tmem_wait_ld();
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           split_bf16x2(__uint_as_float(v[2 * e]) * il, __uint_as_float(v[2 * e + 1]) * il, hi[e], lo[e]);
-        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, 16 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sm + L::qhi + sw_off(row, 16 * c + 8)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, 16 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4 *>(sm + L::qlo + sw_off(row, 16 * c + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, 16 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, 16 * c + 8)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, 16 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, 16 * c + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
       }
       // row `row` of Pi^T (pivt[i][k] = Pi[vperm k][i]) into the B operand
       const uint4 *prow = reinterpret_cast<const uint4 *>(a.p.pivt + (size_t)row * D);
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4 *>(sm + L::kt + sw_off(row, 8 * c)) = prow[c];
+      for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4 *>(sm + L::vt0 + sw_off(row, 8 * c)) = prow[c];
       fence_async_smem();
       tcx_fence_before();
-      tc_consumer_sync();
-      if (tid == 0) {
-        tcx_fence_after();
-        const uint32_t ah = smem_u32(sm + L::qhi), alo2 = smem_u32(sm + L::qlo), bp = smem_u32(sm + L::kt);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
-          tcx_mma(t_s, swdesc(ah + off), swdesc(bp + off), kIdescBF16, kk > 0);
-          tcx_mma(t_s, swdesc(alo2 + off), swdesc(bp + off), kIdescBF16, 1);
-        }
-        tcx_commit(smem_u32(&s_bar));
-      }
-      ok = mbar_wait(smem_u32(&s_bar), n_tiles & 1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&o_ready));
+      ok = tc_wait(&fin_bar, 0, err, abf);
       if (ok) {
         tcx_fence_after();
         const int rho = row % G;
@@ -1191,7 +1276,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           uint32_t v[16];
-          tmem_ld16x(t_s + lane_off + 16 * c, v);
+          tmem_ld16x(t_s + 16 * c, v);
           tmem_wait_ld();
           if (orow) {
 #pragma unroll
@@ -1202,18 +1287,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
           }
         }
         if (a.lse && pos >= 0)
-          a.lse[qrow0 + (long)(pos - p0) * a.n_q_heads + rho] = (m_run + log2f(l)) * 0.6931471805599453f;
+          a.lse[qrow0 + (long)(pos - p0) * a.n_q_heads + rho] = (m_run + log2f(l_run)) * 0.6931471805599453f;
       }
-    }
-    if (!ok) {
-      atomicOr(a.p.err, kErrWaitExpired);
-      abort_flag = 1;
     }
   }
   // release the tensor memory once every MMA and tcgen05 access is finished
   tcx_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kTcMmaWarp) {
     tcx_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols) : "memory");
   }
