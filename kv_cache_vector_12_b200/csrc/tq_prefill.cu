@@ -643,21 +643,24 @@ int smem_of(int bk, int bv, bool qjl) {
 // ===========================================================================
 // The tcgen05 form (contexts without QJL).  Per CTA 128 query rows (the MMA's
 // M) and, per tile of 128 keys, four roles that overlap across tiles:
-//   expand   (warps 4-7) the keys' codes into two fp16 shared-memory operands
-//            in the 128-byte-swizzled K-major layout, double-buffered:
-//            K~[key][kappa] (the exact fp16 K centroids, K fragment order)
-//            and V~^T[kappa_v][key] (fp16 V centroids, V fragment order);
-//   MMA      (warp 9, one thread) S = Q^_hi K~^T + Q^_lo K~^T with the
+//   expand   (warps 8-11) the keys' codes into two fp16 shared-memory
+//            operands in the 128-byte-swizzled K-major layout,
+//            double-buffered: K~[key][kappa] (the exact fp16 K centroids, K
+//            fragment order) and V~^T[kappa_v][key] (fp16 V centroids, V
+//            fragment order), and the key norms as fp32;
+//   MMA      (warp 13, one thread) S = Q^_hi K~^T + Q^_lo K~^T with the
 //            two-part fp16 q_hat (scaled per row by a power of two) as the A
 //            operand in tensor memory, and O += P' V~ with P' as the A
 //            operand in tensor memory; fp32 accumulators in tensor memory;
 //            the next tile's scores are issued as soon as the softmax has
 //            read the current ones;
-//   softmax  (warps 0-3) thread i owns row i: S from tensor memory, times the
-//            row's factor and the key norms, causal mask, online max and sum
-//            (exp2), P' = p ||v|| as fp16 into tensor memory; a moved max
-//            rescales the row of O;
-//   producer (warp 8) streams the codes with 1-D bulk copies.
+//   softmax  (warps 0-7) two threads per row, one per half of the keys and
+//            of the output coordinates: S from tensor memory, times the row's
+//            factor and the key norms, causal mask (on the diagonal tiles
+//            only), the tile maximum exchanged between the halves, online max
+//            and sum (exp2), P' = p ||v|| as fp16 into tensor memory; a moved
+//            max rescales the row of O;
+//   producer (warp 12) streams the codes with 1-D bulk copies.
 // At the end o = Pi^T (O / l) is one more pair of MMAs (O as bf16 hi + lo,
 // Pi^T's rows in the V fragment order as the B operand), and the lse.
 // Tensor memory: S at columns 0-127, O at 128-255, q_hat hi and lo at
@@ -668,10 +671,9 @@ namespace {
 
 constexpr int kTcRows = 128;                      // query rows per CTA
 constexpr int kTcKeys = 128;                      // keys per tile
-constexpr int kTcSoftWarps = 4;                   // warps 0-3
-constexpr int kTcExpWarp0 = 4;                    // warps 4-7 expand
-constexpr int kTcProdWarp = 8, kTcMmaWarp = 9;
-constexpr int kTcThreads = 32 * 10;
+constexpr int kTcExpWarp0 = 8;                    // warps 8-11 expand (0-7: softmax)
+constexpr int kTcProdWarp = 12, kTcMmaWarp = 13;
+constexpr int kTcThreads = 32 * 14;
 constexpr int kTcStages = 2;
 constexpr int kOpBytes = 128 * kHeadDim * 2;      // one 128 x 128 16-bit operand: two 128 x 64 swizzled boxes
 constexpr int kOpBox = kOpBytes / 2;
@@ -685,7 +687,9 @@ struct TcLayout {
   static constexpr int kt0 = 0, kt1 = kOpBytes, vt0 = 2 * kOpBytes, vt1 = 3 * kOpBytes;
   static constexpr int ring = 4 * kOpBytes;
   static constexpr int stage = Stage<BK, BV, false, kTcKeys>::bytes;
-  static constexpr int bytes = ring + kTcStages * stage + 1024;  // + alignment slack
+  // the tile's key norms as fp32, per K~ / V~ buffer: nf[buffer][k or v][key]
+  static constexpr int nf = ring + kTcStages * stage;
+  static constexpr int bytes = nf + 2 * 2 * kTcKeys * 4 + 1024;  // + alignment slack
 };
 
 __device__ __forceinline__ void tcx_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -747,6 +751,13 @@ __device__ __forceinline__ void tmem_st16x(uint32_t taddr, const uint32_t (&r)[1
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// After tmem_wait_ld: passes the loaded registers through an empty asm, so
+// that no use of them is scheduled above the wait.
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
 
 // fp16 pairs (codes 0, 1) and (codes 2, 3) of one lookup's low and high bytes.
 __device__ __forceinline__ void f16_pairs(uint32_t lo, uint32_t hi, uint32_t &p01, uint32_t &p23) {
@@ -883,7 +894,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
   __shared__ __align__(8) uint64_t kv_full[2], kv_empty[2], s_full, s_empty, p_full, pv_done;
-  __shared__ __align__(8) uint64_t q_ready, scratch_free, o_ready, fin_bar, mma_done;
+  __shared__ __align__(8) uint64_t q_ready, scratch_done, scratch_free, o_ready, fin_bar, mma_done;
+  __shared__ __align__(8) uint64_t mx_bar[2], l_bar;
+  __shared__ float s_max[2][2][kTcRows], s_l[2][kTcRows];  // the half rows' maxima (by tile parity) and sums
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int s_pos[kTcRows];
@@ -917,19 +930,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   if (tid == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
-      mbar_init(smem_u32(&empty_bar[i]), 8);  // the expanding and the softmax warps
+      mbar_init(smem_u32(&empty_bar[i]), 4);  // the expanding warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&kv_full[b]), 4);
       mbar_init(smem_u32(&kv_empty[b]), 1);
     }
     mbar_init(smem_u32(&s_full), 1);
-    mbar_init(smem_u32(&s_empty), 4);
-    mbar_init(smem_u32(&p_full), 4);
+    mbar_init(smem_u32(&s_empty), 8);  // the eight softmax warps
+    mbar_init(smem_u32(&p_full), 8);
     mbar_init(smem_u32(&pv_done), 1);
-    mbar_init(smem_u32(&q_ready), 4);
-    mbar_init(smem_u32(&scratch_free), 4);
-    mbar_init(smem_u32(&o_ready), 4);
+    mbar_init(smem_u32(&q_ready), 8);
+    mbar_init(smem_u32(&scratch_done), 8);
+    mbar_init(smem_u32(&scratch_free), 8);
+    mbar_init(smem_u32(&o_ready), 8);
+    mbar_init(smem_u32(&mx_bar[0]), 8);
+    mbar_init(smem_u32(&mx_bar[1]), 8);
+    mbar_init(smem_u32(&l_bar), 8);
     mbar_init(smem_u32(&fin_bar), 1);
     mbar_init(smem_u32(&mma_done), 1);
     abort_flag = 0;
@@ -1071,6 +1088,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       tcx_fence_after();
       const unsigned char *st = sm + L::ring + slot * L::stage;
       expand_tile<BK, BV>(st, sm + (b ? L::kt1 : L::kt0), sm + (b ? L::vt1 : L::vt0), lkf, lv, ew, r, q);
+      {  // the key norms as fp32 for the softmax warps (keys past the copied ones are masked there)
+        const int key = tid - 32 * kTcExpWarp0;
+        float *nf = reinterpret_cast<float *>(sm + L::nf) + b * 2 * kTcKeys;
+        nf[key] = __half2float(reinterpret_cast<const __half *>(st + St::kn)[key]);
+        nf[kTcKeys + key] = __half2float(reinterpret_cast<const __half *>(st + St::vn)[key]);
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -1079,67 +1102,71 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       }
     }
   } else {
-    // ---------------- softmax warps: thread tid owns query row tid
-    const int row = tid, pos = s_pos[row];
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;  // this warp's TMEM lane quarter
-    const uint32_t t_s = tmem + kTcS + lane_off, t_o = tmem + kTcO + lane_off;
-    const uint32_t t_q = tmem + kTcQ + lane_off, t_p = tmem + kTcP + lane_off;
+    // ---------------- softmax warps: row 32 (warp % 4) + lane, half
+    // h = warp / 4 of its keys (64 h .. 64 h + 63 of every tile) and of its
+    // output coordinates; the two halves of a row meet on mbarriers for the
+    // tile maximum and, at the end, for the sum
+    const int h2 = warp >> 2, quarter = warp & 3;
+    const int row = 32 * quarter + lane, pos = s_pos[row];
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;  // this warp's TMEM lane quarter
+    const uint32_t t_s = tmem + kTcS + lane_off + 64 * h2, t_o = tmem + kTcO + lane_off + 64 * h2;
+    const uint32_t t_q = tmem + kTcQ + lane_off + 32 * h2, t_p = tmem + kTcP + lane_off + 32 * h2;
     // q_hat = Pi q in the K fragment order (Pi's rows stored in that order),
-    // mma m16n8k16 bf16, fp32 q as hi + lo; warp w computes rows 32 w ..
-    // 32 w + 31 into a fp32 scratch over the K~ buffers
+    // mma m16n8k16 bf16, fp32 q as hi + lo; warp w computes rows 16 w ..
+    // 16 w + 15 into a fp32 scratch over the K~ buffers
     float *scr = reinterpret_cast<float *>(sm + L::kt0);  // [128 rows][128], 64 KB
     {
       const bool f32 = a.q_dtype == TQ_F32;
-#pragma unroll 1
-      for (int mt = 0; mt < 2; ++mt) {
-        uint32_t ahi[8][4], alo[8][4];
+      uint32_t ahi[8][4], alo[8][4];
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int rr = 32 * warp + 16 * mt + r + 8 * (e & 1), col = 16 * ks + 8 * (e >> 1) + 2 * q;
-            const int pr = s_pos[rr];
-            float x0 = 0.f, x1 = 0.f;
-            if (pr >= 0) {
-              const long qr = qrow0 + (long)(pr - p0) * a.n_q_heads + (rr % G);
-              if (f32) {
-                const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(a.q) + qr * D + col);
-                x0 = v.x;
-                x1 = v.y;
-              } else {
-                const uint32_t v =
-                    *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.q) + qr * D + col);
-                x0 = __uint_as_float(v << 16);
-                x1 = __uint_as_float(v & 0xffff0000u);
-              }
+        for (int e = 0; e < 4; ++e) {
+          const int rr = 16 * warp + r + 8 * (e & 1), col = 16 * ks + 8 * (e >> 1) + 2 * q;
+          const int pr = s_pos[rr];
+          float x0 = 0.f, x1 = 0.f;
+          if (pr >= 0) {
+            const long qr = qrow0 + (long)(pr - p0) * a.n_q_heads + (rr % G);
+            if (f32) {
+              const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(a.q) + qr * D + col);
+              x0 = v.x;
+              x1 = v.y;
+            } else {
+              const uint32_t v =
+                  *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.q) + qr * D + col);
+              x0 = __uint_as_float(v << 16);
+              x1 = __uint_as_float(v & 0xffff0000u);
             }
-            split_bf16x2(x0, x1, ahi[ks][e], alo[ks][e]);
           }
-#pragma unroll 1
-        for (int nt = 0; nt < 16; ++nt) {
-          uint32_t bfr[8][2];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[(nt * 4 + j) * 32 + lane];
-            bfr[2 * j][0] = v.x, bfr[2 * j][1] = v.y, bfr[2 * j + 1][0] = v.z, bfr[2 * j + 1][1] = v.w;
-          }
-          float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            mma_bf16(c, ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], bfr[ks][0], bfr[ks][1]);
-            mma_bf16(c, alo[ks][0], alo[ks][1], alo[ks][2], alo[ks][3], bfr[ks][0], bfr[ks][1]);
-          }
-          float *d0 = scr + (32 * warp + 16 * mt + r) * D + 8 * nt + 2 * q;
-          *reinterpret_cast<float2 *>(d0) = make_float2(c[0], c[1]);
-          *reinterpret_cast<float2 *>(d0 + 8 * D) = make_float2(c[2], c[3]);
+          split_bf16x2(x0, x1, ahi[ks][e], alo[ks][e]);
         }
+#pragma unroll 1
+      for (int nt = 0; nt < 16; ++nt) {
+        uint32_t bfr[8][2];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const uint4 v = reinterpret_cast<const uint4 *>(a.p.pikf)[(nt * 4 + jj) * 32 + lane];
+          bfr[2 * jj][0] = v.x, bfr[2 * jj][1] = v.y, bfr[2 * jj + 1][0] = v.z, bfr[2 * jj + 1][1] = v.w;
+        }
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_bf16(c, ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], bfr[ks][0], bfr[ks][1]);
+          mma_bf16(c, alo[ks][0], alo[ks][1], alo[ks][2], alo[ks][3], bfr[ks][0], bfr[ks][1]);
+        }
+        float *d0 = scr + (16 * warp + r) * D + 8 * nt + 2 * q;
+        *reinterpret_cast<float2 *>(d0) = make_float2(c[0], c[1]);
+        *reinterpret_cast<float2 *>(d0 + 8 * D) = make_float2(c[2], c[3]);
       }
     }
     __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&scratch_done));
+    bool ok = tc_wait(&scratch_done, 0, err, abf);
     // per row: a power-of-two scale puts max |q_hat| in [2^13, 2^14), then
-    // q_hat = hi + lo in fp16 into tensor memory (the scores' A operand)
-    float fq;
-    {
+    // this half's coordinates of q_hat = hi + lo in fp16 into tensor memory
+    // (the scores' A operand)
+    float fq = 0.f;
+    if (ok) {
       const float *qr = scr + row * D;
       float m = 0.f;
       for (int k = 0; k < D; ++k) m = fmaxf(m, fabsf(qr[(k + lane) & (D - 1)]));
@@ -1148,10 +1175,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       const float sc = m > 0.f ? ldexpf(1.f, 14 - ex) : 1.f;
       fq = a.scale * kLog2e / sc;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
+        const int k0 = 64 * h2 + 32 * c;
         uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) split_f16x2(qr[32 * c + 2 * e] * sc, qr[32 * c + 2 * e + 1] * sc, hi[e], lo[e]);
+        for (int e = 0; e < 16; ++e) split_f16x2(qr[k0 + 2 * e] * sc, qr[k0 + 2 * e + 1] * sc, hi[e], lo[e]);
         tmem_st16x(t_q + 16 * c, hi);
         tmem_st16x(t_q + 64 + 16 * c, lo);
       }
@@ -1161,81 +1189,102 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(smem_u32(&q_ready));
-      mbar_arrive(smem_u32(&scratch_free));  // this warp's scratch rows are read
+      mbar_arrive(smem_u32(&scratch_free));  // this thread's scratch reads are done
     }
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
+    const int min_pos = p0 + first_q;  // the CTA's first query position
     for (int it = 0; ok && it < n_tiles; ++it) {
-      const int slot = it % kTcStages;
-      // the stage's key norms (its copies are complete) and S(it)
-      ok = tc_wait(&full_bar[slot], (it / kTcStages) & 1, err, abf) && tc_wait(&s_full, it & 1, err, abf);
+      const int b = it & 1;
+      // the tile's key norms (published with K~ and V~) and S(it)
+      ok = tc_wait(&kv_full[b], (it >> 1) & 1, err, abf) && tc_wait(&s_full, it & 1, err, abf);
       if (!ok) break;
       tcx_fence_after();
-      const unsigned char *st = sm + L::ring + slot * L::stage;
-      const __half *kn = reinterpret_cast<const __half *>(st + St::kn);
-      const __half *vn = reinterpret_cast<const __half *>(st + St::vn);
-      const int kfirst = it * kTcKeys;
-      float sc[kTcKeys];
-      float mx = -INFINITY;
+      const float4 *kn4 = reinterpret_cast<const float4 *>(sm + L::nf) + b * 2 * (kTcKeys / 4) + 16 * h2;
+      const float4 *vn4 = kn4 + kTcKeys / 4;
+      const int kfirst = it * kTcKeys + 64 * h2;  // this half's first key
+      // tiles wholly below the CTA's first query position need no causal mask
+      const bool masked = it * kTcKeys + kTcKeys - 1 > min_pos;
+      // this half of the row of S: four loads in flight before one wait
+      uint32_t sv[4][16];
 #pragma unroll
-      for (int c = 0; c < kTcKeys / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16x(t_s + 16 * c, v);
-        tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tmem_ld16x(t_s + 16 * c, sv[c]);
+      tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = 16 * c + e;
-          const float x = __uint_as_float(v[e]) * fq * __half2float(kn[j]);
-          sc[j] = kfirst + j <= pos ? x : -INFINITY;
-          mx = fmaxf(mx, sc[j]);
-        }
-      }
+      for (int c = 0; c < 4; ++c) reg_fence16(sv[c]);
       // S is read: the next tile's scores may overwrite it
       tcx_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s_empty));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j4 = 0; j4 < 16; ++j4) {
+        const float4 kf = kn4[j4];
+        const float kk[4] = {kf.x, kf.y, kf.z, kf.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * j4 + e;
+          uint32_t &cell = sv[j >> 4][j & 15];
+          const float x = __uint_as_float(cell) * fq * kk[e];
+          const float y = (!masked || kfirst + j <= pos) ? x : -INFINITY;
+          cell = __float_as_uint(y);
+          mx = fmaxf(mx, y);
+        }
+      }
+      // the row's maximum from both halves (double-buffered by tile parity)
+      s_max[b][h2][row] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&mx_bar[b]));
+      ok = tc_wait(&mx_bar[b], (it >> 1) & 1, err, abf);
+      if (!ok) break;
+      mx = fmaxf(s_max[b][0][row], s_max[b][1][row]);
       const float mn = fmaxf(m_run, mx);
       const float ref = fmaxf(mn, -3.0e38f);
       const float al = fast_exp2(m_run - ref);
       m_run = mn;
-      float ls = 0.f;
-      uint32_t pk[kTcKeys / 2];
-#pragma unroll
-      for (int e = 0; e < kTcKeys / 2; ++e) {
-        const int j = 2 * e;
-        const float pa = fast_exp2(sc[j] - ref), pb = fast_exp2(sc[j + 1] - ref);
-        ls += pa + pb;
-        pk[e] = pack_half2(sc[j] == -INFINITY ? 0.f : pa * __half2float(vn[j]),
-                           sc[j + 1] == -INFINITY ? 0.f : pb * __half2float(vn[j + 1]));
-      }
-      l_run = fmaf(l_run, al, ls);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[slot]));  // the norms are read
-      // the previous tile's value MMAs read P' and write O: wait for them,
-      // then rescale O on a moved maximum and write this tile's P'
+      // the previous tile's value MMAs read P' and write O (issued after this
+      // tile's scores, so usually finished by now): wait for them, rescale
+      // this half of O on a moved maximum, then write this half of P'
       if (it > 0) {
         ok = tc_wait(&pv_done, (it - 1) & 1, err, abf);
         if (!ok) break;
         tcx_fence_after();
         if (__any_sync(0xffffffffu, al != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t v[16];
             tmem_ld16x(t_o + 16 * c, v);
             tmem_wait_ld();
+            reg_fence16(v);
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
             tmem_st16x(t_o + 16 * c, v);
           }
         }
       }
+      float ls = 0.f;
 #pragma unroll
-      for (int c = 0; c < kTcKeys / 32; ++c) {
-        uint32_t v[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = pk[16 * c + e];
-        tmem_st16x(t_p + 16 * c, v);
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 vf = vn4[8 * c + j4];
+          const float vv[4] = {vf.x, vf.y, vf.z, vf.w};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 32 * c + 4 * j4 + 2 * e;
+            const float sa = __uint_as_float(sv[j >> 4][j & 15]), sb = __uint_as_float(sv[(j + 1) >> 4][(j + 1) & 15]);
+            const float pa = fast_exp2(sa - ref), pb = fast_exp2(sb - ref);
+            ls += pa + pb;
+            // masked keys (and keys past the copied ones, whose norms are not
+            // set) contribute 0
+            pk[2 * j4 + e] = masked ? pack_half2(sa == -INFINITY ? 0.f : pa * vv[2 * e],
+                                                 sb == -INFINITY ? 0.f : pb * vv[2 * e + 1])
+                                    : pack_half2(pa * vv[2 * e], pb * vv[2 * e + 1]);
+          }
+        }
+        tmem_st16x(t_p + 16 * c, pk);
       }
+      l_run = fmaf(l_run, al, ls);
       tmem_wait_st();
       tcx_fence_before();
       __syncwarp();
@@ -1244,26 +1293,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     // ---------------- o = Pi^T (O / l)
     if (ok) ok = tc_wait(&pv_done, (n_tiles - 1) & 1, err, abf);
     if (ok) {
+      s_l[h2][row] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&l_bar));
+      ok = tc_wait(&l_bar, 0, err, abf);
+    }
+    if (ok) {
       tcx_fence_after();
-      const float il = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float l = s_l[0][row] + s_l[1][row];
+      const float il = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = 0; c < 4; ++c) {
+        const int col = 64 * h2 + 16 * c;
         uint32_t v[16];
         tmem_ld16x(t_o + 16 * c, v);
         tmem_wait_ld();
+        reg_fence16(v);
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           split_bf16x2(__uint_as_float(v[2 * e]) * il, __uint_as_float(v[2 * e + 1]) * il, hi[e], lo[e]);
-        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, 16 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, 16 * c + 8)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, 16 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, 16 * c + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, col)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(sm + L::kt0 + sw_off(row, col + 8)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, col)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4 *>(sm + L::kt1 + sw_off(row, col + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
       }
-      // row `row` of Pi^T (pivt[i][k] = Pi[vperm k][i]) into the B operand
-      const uint4 *prow = reinterpret_cast<const uint4 *>(a.p.pivt + (size_t)row * D);
+      // this half of row `row` of Pi^T (pivt[i][k] = Pi[vperm k][i]) into the B operand
+      const uint4 *prow = reinterpret_cast<const uint4 *>(a.p.pivt + (size_t)row * D + 64 * h2);
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4 *>(sm + L::vt0 + sw_off(row, 8 * c)) = prow[c];
+      for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(sm + L::vt0 + sw_off(row, 64 * h2 + 8 * c)) = prow[c];
       fence_async_smem();
       tcx_fence_before();
       __syncwarp();
@@ -1272,12 +1330,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       if (ok) {
         tcx_fence_after();
         const int rho = row % G;
-        float *orow = pos >= 0 ? a.out + (qrow0 + (long)(pos - p0) * a.n_q_heads + rho) * D : nullptr;
+        float *orow = pos >= 0 ? a.out + (qrow0 + (long)(pos - p0) * a.n_q_heads + rho) * D + 64 * h2 : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t v[16];
           tmem_ld16x(t_s + 16 * c, v);
           tmem_wait_ld();
+          reg_fence16(v);
           if (orow) {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -1286,8 +1345,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
                               __uint_as_float(v[4 * e + 3]));
           }
         }
-        if (a.lse && pos >= 0)
-          a.lse[qrow0 + (long)(pos - p0) * a.n_q_heads + rho] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+        if (a.lse && pos >= 0 && h2 == 0)
+          a.lse[qrow0 + (long)(pos - p0) * a.n_q_heads + rho] = (m_run + log2f(l)) * 0.6931471805599453f;
       }
     }
   }
