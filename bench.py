@@ -75,10 +75,11 @@ DEFAULT_WORKLOAD = "serving"
 
 
 # DRAM bytes per attention-kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from one ncu capture of the default command, keyed by
-# (workload, bits_k, bits_v, qjl); null elsewhere.  Re-captured whenever the
-# kernel changes.
-MEASURED_TRAFFIC = {("llama8b", 3, 3, False): 26352640.0}
+# dram__bytes_write.sum) from one ncu capture of a full-size launch of the
+# workload's default setting (d = 128, contiguous cache, Gaussian codebook,
+# every sequence), keyed by (workload, bits_k, bits_v, qjl); null elsewhere.
+# Re-captured whenever the kernel changes.
+MEASURED_TRAFFIC = {("serving", 3, 3, False): 809897216.0 + 5739008.0}
 
 
 def measured_peaks():
@@ -777,7 +778,9 @@ def main(argv=None) -> int:
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
                      "frac": dec_achieved / peak,
-                     "traffic": MEASURED_TRAFFIC.get((args.workload, bits_k, bits_v, qjl)),
+                     "traffic": (MEASURED_TRAFFIC.get((args.workload, bits_k, bits_v, qjl))
+                                 if D == 128 and not args.paged and not args.max_seqs and args.law == "gaussian"
+                                 else None),
                      "traffic_kernel": "decode_mma_kernel", "peak_source": peak_kind,
                      "kernel": "tq_decode_attention call (split-K attention with q rotation + merge)",
                      "algorithmic_bytes_per_call": timed_bytes / args.steps},
