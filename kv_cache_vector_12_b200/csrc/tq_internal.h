@@ -126,7 +126,7 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
 int launch_quantize_tc256(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                           const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                           void *stream);
-// K (is_v false) or V rows in 64- or 128-row tiles for head dimensions 64 and 256,
+// K (is_v false) or V rows in 64-row tiles for head dimension 64,
 // MSE codes only (tq_quantize_tile.cu).
 int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x, const int32_t *seq_idx,
                          const int32_t *pos, int n_tok, bool is_v, void *stream);

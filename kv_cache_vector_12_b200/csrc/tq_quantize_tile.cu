@@ -1,5 +1,5 @@
-// Quantize-on-append in tiles for head dimensions 64 and 256 (sm_100a): the
-// method's norm, rotation by Pi and Lloyd-Max codes ("ステップ1: PolarQuant",
+// Quantize-on-append in tiles for head dimension 64 (sm_100a): the method's
+// norm, rotation by Pi and Lloyd-Max codes ("ステップ1: PolarQuant",
 // ai-accelerate.xyz TurboQuant explainer) for the K rows without QJL and for
 // every V row, 64 vectors per CTA tile.
 //
@@ -11,11 +11,9 @@
 //                  memory;
 //   store          the packed 32-code groups of every row (thread q of a
 //                  quad packs groups q, q + 4, ...), the fp16 norm.
-// Pi's B-fragment table is copied once per CTA into shared memory (8 KB at
-// d = 64, 128 KB at d = 256, where one CTA of eight warps holds an SM; read
-// from L2 instead, the table's 8 KB per row saturated L2).  The kernel is
-// persistent: tiles are strided over the grid.  d = 128 uses the tcgen05
-// kernel instead.
+// Pi's B-fragment table (8 KB) is copied once per CTA into shared memory.
+// The kernel is persistent: tiles are strided over the grid.  d = 128 and
+// d = 256 use the tcgen05 kernels instead.
 #include <atomic>
 
 #include <cuda_bf16.h>
@@ -28,10 +26,9 @@
 namespace tq {
 namespace {
 
-// warps per CTA (16 rows each): d = 256 runs one CTA of eight per SM around
-// its 128 KB table, d = 64 several CTAs of four
+// warps per CTA (16 rows each)
 template <int DH>
-__host__ __device__ constexpr int tile_warps() { return DH == 256 ? 8 : 4; }
+__host__ __device__ constexpr int tile_warps() { return 4; }
 
 __device__ __forceinline__ void mma_bf16_t(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
@@ -189,13 +186,14 @@ TileFn pick_tile(int bits) {
 int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x, const int32_t *seq_idx,
                          const int32_t *pos, int n_tok, bool is_v, void *stream) {
   const int bits = is_v ? p.bits_v : p.bits_k;
-  const TileFn fn = p.d == 64 ? pick_tile<64>(bits) : pick_tile<256>(bits);
-  const int warps = p.d == 64 ? tile_warps<64>() : tile_warps<256>();
+  if (p.d != 64) return (int)cudaErrorInvalidValue;  // d = 64 only
+  const TileFn fn = pick_tile<64>(bits);
+  const int warps = tile_warps<64>();
   const int smem = (p.d / 8) * (p.d / 32) * 32 * 16;  // the fragment table
-  // resident CTAs on the device, cached per device, head dimension and width
-  static std::atomic<int> slots[kMaxDevices][2][3];
+  // resident CTAs on the device, cached per device and width
+  static std::atomic<int> slots[kMaxDevices][3];
   const int dev = current_device();
-  std::atomic<int> &slot = slots[dev][p.d == 64 ? 0 : 1][bits - 2];
+  std::atomic<int> &slot = slots[dev][bits - 2];
   int n_slots = slot.load(std::memory_order_relaxed);
   if (n_slots == 0) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
