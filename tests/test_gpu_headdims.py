@@ -70,6 +70,31 @@ def test_quantize_parity(tq, d, bits_k, bits_v, qjl, n_tok):
                 assert ph.compare_fp16(pl["qjl_norm"][0, h, ps], qz.qjl_gamma)["worse"] == 0
 
 
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("bits_k,bits_v,qjl", [(3, 3, 0), (2, 4, 1)])
+def test_quantize_parity_many_tiles(tq, d, bits_k, bits_v, qjl):
+    """20001 tokens x 4 heads (80004 rows per matrix): several tiles per
+    persistent CTA, so the tile kernels' rings and barrier phases wrap, and
+    the last tile is ragged (4 rows); every row is compared."""
+    n_tok, n_heads = 20001, 4
+    ctx = tq.Context(d, bits_k, bits_v, qjl, 42)
+    ref = params(d, bits_k, bits_v, qjl)
+    k, v = rows(n_tok, n_heads, d, 11 + d), rows(n_tok, n_heads, d, 12 + d)
+    cache = tq.Cache(ctx, 1, n_heads, (n_tok + 63) // 64 * 64)
+    pos = torch.arange(n_tok, dtype=torch.int32)
+    tq.quantize(ctx, cache, k.cuda(), v.cuda(), torch.zeros(n_tok, dtype=torch.int32, device="cuda"), pos.cuda())
+    ctx.check_device_errors()
+    pl = {n: (t.cpu().numpy() if t is not None else None) for n, t in cache.planes.items()}
+    for which, x, c, t, bits in (("k", k, ref.ck, ref.tk, bits_k), ("v", v, ref.cv, ref.tv, bits_v)):
+        if qjl and which == "k":
+            continue  # K with QJL runs the per-row kernel at these head dimensions (covered above)
+        for h in range(n_heads):
+            qz = o.quantize(x[:, h].double().numpy(), ref.pi, c, t)
+            cc = ph.compare_codes(pl["codes_" + which][0, h, :n_tok], qz, bits, t, d=d)
+            assert cc["outside_window"] == 0, cc
+            assert ph.compare_fp16(pl["norm_" + which][0, h, :n_tok], qz.norm)["worse"] == 0
+
+
 def _decode_and_compare(tq, d, lens, n_heads, group, bits_k, bits_v, qjl, seed, law=o.LAW_GAUSSIAN, paged=0,
                         q_dtype=torch.float32):
     ctx = tq.Context(d, bits_k, bits_v, qjl, 42, law=law)
