@@ -219,23 +219,32 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
       }
   }
   // While the previous kernel (typically the append) still runs, warm L2 with
-  // the first stages this CTA will stream.  A prefetch only moves lines into
-  // L2, the point of coherence, so whatever the previous kernel writes there
-  // is what the copies read after the wait.  The sequence length is not final
-  // yet either: its current value (a relaxed read) only bounds the prefetch,
-  // so that splits past the end fetch nothing; a stale value costs at most a
-  // useless or a missing prefetch.
+  // the first four stages this CTA will stream (below the length bound and
+  // the capacity).  A prefetch only moves lines into L2, the point of
+  // coherence, so whatever the previous kernel writes there is what the
+  // copies read after the wait.  The sequence length is not final yet.  The
+  // 2-CTA (168-register) build, which at d = 128 runs short splits of one or
+  // a few sequences (every split holds tokens, and the CTA's start is on the
+  // critical path), fetches blind.  The 3-CTA build, which runs the long
+  // splits of ragged batches, first reads the current length (a relaxed read,
+  // one more memory round trip, amortised over a long split) and bounds the
+  // prefetch by it, so that splits past their sequence's end fetch nothing; a
+  // stale value costs at most a useless or a missing prefetch.
   if (warp == kConsumerWarps && lane == 0) {
     // this KV head's query rows (read right after the wait)
     const size_t qbytes = (size_t)G * DH * (a.q_dtype == TQ_F32 ? 4 : 2);
     prefetch_l2(static_cast<const char *>(a.q) + ((size_t)s * a.n_q_heads + (size_t)h * G) * DH *
                                                      (a.q_dtype == TQ_F32 ? 4 : 2),
                 (uint32_t)qbytes);
-    int len_hint;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(len_hint) : "l"(a.seq_lens + s));
     const int first = split * a.chunk;
-    const int last = min(min(min(first + a.chunk, a.max_seq_len), len_hint),
-                         min(first + kPrefetchTokens, a.c.capacity));
+    int last = min(min(first + a.chunk, a.max_seq_len), min(first + kPrefetchTokens, a.c.capacity));
+    if constexpr (CTAS == 3) {
+      int len_hint;
+      asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(len_hint) : "l"(a.seq_lens + s));
+      last = min(last, len_hint);
+    } else {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a.seq_lens + s));
+    }
     // (contiguous layout only: a paged cache's block table is not read before the wait)
     if (!PAGED && first < last) {
       const long tok = ((long)s * a.c.n_kv_heads + h) * a.c.capacity + first;
