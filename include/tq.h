@@ -17,13 +17,13 @@
  *    buffer; the library never frees, keeps or allocates caller memory.
  *  - A context belongs to the device that was current when it was created.
  *    The compute calls (tq_quantize, tq_decode_attention,
- *    tq_decode_attention_noalloc) check that this device is current and
- *    return TQ_ERR_INVALID, launching nothing, when it is not.  One process
- *    may hold contexts on several devices.
- *  - Compute calls (tq_quantize, tq_decode_attention) are asynchronous on the
- *    given stream (a cudaStream_t passed as void*; NULL = legacy default
- *    stream), allocate nothing, never synchronise and never read device data
- *    on the host.
+ *    tq_decode_attention_noalloc, tq_prefill_attention, tq_weight_quantize,
+ *    tq_weight_gemm) check that this device is current and return
+ *    TQ_ERR_INVALID, launching nothing, when it is not.  One process may hold
+ *    contexts on several devices.
+ *  - The compute calls are asynchronous on the given stream (a cudaStream_t
+ *    passed as void*; NULL = legacy default stream), allocate nothing, never
+ *    synchronise and never read device data on the host.
  *  - On any non-TQ_OK status nothing has been launched (argument errors) or a
  *    CUDA call failed (TQ_ERR_CUDA); tq_last_error() returns a thread-local
  *    message.  Device-side range errors (a seq_idx, pos or seq_len outside the
