@@ -256,11 +256,15 @@ __global__ void __launch_bounds__(kJThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = 2 * a.tiles_k;
-  // tiles t = blockIdx.x + i gridDim.x, i = 0 .. my_tiles - 1; the first my_k are K tiles
-  const int bx = (int)blockIdx.x, grid = (int)gridDim.x;
-  const int my_tiles = bx < n_tiles ? (n_tiles - 1 - bx) / grid + 1 : 0;
+  // this CTA's tiles: first the K tiles bx + i gridDim.x, then the V tiles
+  // (gridDim.x - 1 - bx) + j gridDim.x, so that the CTAs with one K tile more
+  // than the others get one V tile less (the K tiles cost about twice as much)
+  const int bx = (int)blockIdx.x, grid = (int)gridDim.x, bv = grid - 1 - bx;
   const int my_k = bx < a.tiles_k ? (a.tiles_k - 1 - bx) / grid + 1 : 0;
+  const int my_v = bv < a.tiles_k ? (a.tiles_k - 1 - bv) / grid + 1 : 0;
+  const int my_tiles = my_k + my_v;
+  // first row (of K or V) of the CTA's i-th tile
+  auto tile_row0 = [&](int i) { return (i < my_k ? bx + i * grid : bv + (i - my_k) * grid) * kTileRows; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kJStages; ++i) {
@@ -316,9 +320,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
           break;
         }
         if (*(volatile int *)&abort_flag) break;
-        const int t = bx + i * grid;
         const bool is_k = i < my_k;
-        const int row0 = (is_k ? t : t - a.tiles_k) * kTileRows;
+        const int row0 = tile_row0(i);
         const CUtensorMap *map = is_k ? &map_k : &map_v;
         const uint32_t fb = smem_addr(&full_bar[slot]);
         unsigned char *st = ring + slot * kTileBytes;
@@ -432,9 +435,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
 
     for (int j = 0, i = g; i < my_tiles; ++j, i += kJGroups) {
       const int slot = i % kJStages;
-      const int t = bx + i * grid;
       const bool is_k = i < my_k;
-      const int row = (is_k ? t : t - a.tiles_k) * kTileRows + r;
+      const int row = tile_row0(i) + r;
       // destination, loaded now and checked after the codes
       const bool in_range = row < a.n_rows;
       const int tok = in_range ? row / a.c.n_kv_heads : 0;
