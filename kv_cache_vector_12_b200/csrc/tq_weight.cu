@@ -12,7 +12,8 @@
 //   y[t][i] = sum_b n_ib (Pi x_tb) . c[code_ib].
 //   rotate  x_hat[b][t] = Pi x_tb per (block, token), as 16-bit fixed point
 //           (hi, lo bytes) in the decode kernel's K fragment order, with its
-//           scale factor; one CTA of d threads per (block, token).
+//           scale factor; one CTA of d threads per (block, token), which also
+//           zeroes a share of y.
 //   gemm    per CTA 128 weight rows x 8 or 16 tokens, over a range of blocks: the
 //           rows' codes, norms and the blocks' x_hat stream in by TMA bulk
 //           copies (one producer warp, mbarrier ring, bounded waits); four
@@ -21,7 +22,8 @@
 //           expanded by byte permutes into exact fixed-point centroids, four
 //           hi/lo products), scale them by n_ib and the token's factor and
 //           sum over the blocks in fp32; partial sums over block ranges meet
-//           in y by atomic adds.
+//           in y by atomic adds.  It is a programmatic dependent of the
+//           rotation: its first weight rows stream in while that still runs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -47,13 +49,25 @@ constexpr int kWStages = 4;
 // fragment position kappa (row kperm[kappa] of Pi), then the block's scale.
 // The padding tokens up to a multiple of 16 are never written: the product
 // reads them but never stores their results.
+// It also zeroes its share of y (token t, outputs b y_chunk ..), which the
+// product then accumulates into.
 __global__ void __launch_bounds__(kHeadDim) weight_rotate_kernel(DeviceParams p, const void *x, int x_dtype,
                                                                  int n_tok, int n_in, int t_pad, uint8_t *xq,
-                                                                 float *xf) {
+                                                                 float *xf, float *y, int n_out, int y_chunk) {
   __shared__ float s_x[kHeadDim];
   __shared__ float red[kHeadDim / 32];
   const int b = blockIdx.x, t = blockIdx.y, k = threadIdx.x;
   const uint16_t *prow = p.pi + (size_t)p.kperm[k] * kHeadDim;
+  // launched as a programmatic dependent: x and y are touched only once the
+  // previous kernel in the stream has completed; the product may launch
+  // from then on (it reads the packed weights, final by now, before it
+  // waits for this grid)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (t < n_tok) {
+    const int i1 = min(n_out, (b + 1) * y_chunk);
+    for (int i = b * y_chunk + k; i < i1; i += kHeadDim) y[(size_t)t * n_out + i] = 0.f;
+  }
   float xv = 0.f;
   if (t < n_tok) {
     const size_t idx = (size_t)t * n_in + (size_t)b * kHeadDim + k;
@@ -131,28 +145,42 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
 
   if (warp == kWWarps) {
     // ---------------- producer: one stage per block, the tile's rows (the
-    // capacity is a multiple of 64, so a ragged last tile copies 64 rows)
+    // capacity is a multiple of 64, so a ragged last tile copies 64 rows).
+    // The first stages' weight rows are requested before the wait for the
+    // rotation kernel (they were final before it started); their x_hat after.
     if (lane == 0) {
       const uint32_t n_rows = (uint32_t)min(kWRows, a.w.capacity - row0);
-      int issued = 0;
-      for (int it = 0; it < n_stage; ++it) {
+      const int pre = min(kWStages, n_stage);
+      auto weights = [&](int it) {
+        unsigned char *st = smem + (it % kWStages) * St::bytes;
+        const uint32_t bar = smem_u32(&full_bar[it % kWStages]);
+        const long tok = (long)(b0 + it) * a.w.capacity + row0;  // sequence 0, KV head b, position row0
+        mbar_arrive_expect_tx(bar, n_rows * (16 * BK + 2) + St::tok * (2 * kHeadDim + 4));
+        bulk_g2s(smem_u32(st + St::codes), a.w.codes_k + tok * (16 * BK), n_rows * (16 * BK), bar);
+        bulk_g2s(smem_u32(st + St::norms), a.w.norm_k + tok, n_rows * 2, bar);
+      };
+      auto activations = [&](int it) {
+        unsigned char *st = smem + (it % kWStages) * St::bytes;
+        const uint32_t bar = smem_u32(&full_bar[it % kWStages]);
+        const int b = b0 + it;
+        bulk_g2s(smem_u32(st + St::xq), a.xq + ((size_t)b * a.t_pad + (size_t)tg * St::tok) * 2 * kHeadDim,
+                 St::tok * 2 * kHeadDim, bar);
+        bulk_g2s(smem_u32(st + St::xf), a.xf + (size_t)b * a.t_pad + (size_t)tg * St::tok, St::tok * 4, bar);
+      };
+      for (int it = 0; it < pre; ++it) weights(it);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int it = 0; it < pre; ++it) activations(it);
+      int issued = pre;
+      for (int it = pre; it < n_stage; ++it) {
         const int slot = it % kWStages;
-        if (it >= kWStages && !mbar_wait(smem_u32(&empty_bar[slot]), ((it / kWStages) - 1) & 1)) {
+        if (!mbar_wait(smem_u32(&empty_bar[slot]), ((it / kWStages) - 1) & 1)) {
           atomicOr(a.p.err, kErrWaitExpired);
           abort_flag = 1;
           break;
         }
         if (*(volatile int *)&abort_flag) break;
-        unsigned char *st = smem + slot * St::bytes;
-        const uint32_t bar = smem_u32(&full_bar[slot]);
-        const int b = b0 + it;
-        const long tok = (long)b * a.w.capacity + row0;  // sequence 0, KV head b, position row0
-        mbar_arrive_expect_tx(bar, n_rows * (16 * BK + 2) + St::tok * (2 * kHeadDim + 4));
-        bulk_g2s(smem_u32(st + St::codes), a.w.codes_k + tok * (16 * BK), n_rows * (16 * BK), bar);
-        bulk_g2s(smem_u32(st + St::norms), a.w.norm_k + tok, n_rows * 2, bar);
-        bulk_g2s(smem_u32(st + St::xq), a.xq + ((size_t)b * a.t_pad + (size_t)tg * St::tok) * 2 * kHeadDim,
-                 St::tok * 2 * kHeadDim, bar);
-        bulk_g2s(smem_u32(st + St::xf), a.xf + (size_t)b * a.t_pad + (size_t)tg * St::tok, St::tok * 4, bar);
+        weights(it);
+        activations(it);
         issued = it + 1;
       }
       if (*(volatile int *)&abort_flag) {
@@ -164,6 +192,8 @@ __global__ void __launch_bounds__(kWThreads) weight_gemm_kernel(const WeightArgs
   }
 
   // ---------------- consumers: rows 32 warp + 16 rb + r (+ 8), tokens 8 nt + 2 q (+ 1)
+  // (y, zeroed by the rotation kernel, is accumulated into only after it completed)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const Lut lk = a.p.lut_k;
   float yacc[2][NT][4];
 #pragma unroll
@@ -285,10 +315,20 @@ int launch_weight_gemm(const DeviceParams &p, const tq_cache &w, int n_out, int 
   const int t_pad = (n_tok + kWTok - 1) / kWTok * kWTok;
   uint8_t *xq = reinterpret_cast<uint8_t *>(workspace);
   float *xf = reinterpret_cast<float *>(workspace + ((size_t)nb * t_pad * 2 * kHeadDim + 255) / 256 * 256);
-  cudaError_t e = cudaMemsetAsync(y, 0, (size_t)n_tok * n_out * sizeof(float), st);
-  if (e != cudaSuccess) return (int)e;
-  weight_rotate_kernel<<<dim3(nb, n_tok), kHeadDim, 0, st>>>(p, x, x_dtype, n_tok, n_in, t_pad, xq, xf);
-  e = cudaGetLastError();
+  // two launches, the second a programmatic dependent of the first: the
+  // rotation (which also zeroes y) and the product
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t rcfg = {};
+  rcfg.gridDim = dim3(nb, n_tok);
+  rcfg.blockDim = dim3(kHeadDim);
+  rcfg.stream = st;
+  rcfg.attrs = pdl;
+  rcfg.numAttrs = 1;
+  const int y_chunk = (n_out + nb - 1) / nb;
+  cudaError_t e = cudaLaunchKernelEx(&rcfg, weight_rotate_kernel, p, x, x_dtype, n_tok, n_in, t_pad, xq, xf, y, n_out,
+                                     y_chunk);
   if (e != cudaSuccess) return (int)e;
   // split the blocks so that the grid fills about four CTAs per SM
   // one n-tile of 8 tokens per CTA for up to 8 tokens, else two
@@ -315,8 +355,14 @@ int launch_weight_gemm(const DeviceParams &p, const tq_cache &w, int n_out, int 
     done.store(true, std::memory_order_release);
   }
   WeightArgs args{p, w, n_out, nb, n_tok, t_pad, per, xq, xf, y};
-  fn<<<dim3(tiles, splits, groups), kWThreads, smem, st>>>(args);
-  return (int)cudaGetLastError();
+  cudaLaunchConfig_t gcfg = {};
+  gcfg.gridDim = dim3(tiles, splits, groups);
+  gcfg.blockDim = dim3(kWThreads);
+  gcfg.dynamicSmemBytes = smem;
+  gcfg.stream = st;
+  gcfg.attrs = pdl;
+  gcfg.numAttrs = 1;
+  return (int)cudaLaunchKernelEx(&gcfg, fn, args);
 }
 
 }  // namespace tq
