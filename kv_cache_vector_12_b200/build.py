@@ -24,7 +24,7 @@ LIB = os.path.join(PKG, "libtq.so")
 # per (head dimension, K width) slice of the attention kernel's instantiations
 SOURCES = [(s, os.path.splitext(s)[0], []) for s in
            ["tq_host.cpp", "tq_fragments.cpp", "tq_api.cu", "tq_kernels.cu", "tq_quantize_tc.cu",
-            "tq_quantize_qjl_tc.cu", "tq_quantize_tc256.cu", "tq_quantize_tile.cu", "tq_decode.cu", "tq_prefill.cu", "tq_weight.cu",
+            "tq_quantize_qjl_tc.cu", "tq_quantize_tc256.cu", "tq_decode.cu", "tq_prefill.cu", "tq_weight.cu",
             "tq_noalloc.cu"]]
 SOURCES += [("tq_decode_variants.cu", f"tq_decode_variants_d{d}_k{bk}", [f"-DTQ_DECODE_DH={d}", f"-DTQ_DECODE_BK={bk}"])
             for d in (64, 128, 256) for bk in (2, 3, 4)]

@@ -115,9 +115,10 @@ int current_device();
 // --- launches (tq_kernels.cu, tq_decode.cu); return a cudaError_t as int ---
 int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                     const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
-// seq_idx and pos may both be null: token t then goes to position t of
-// sequence 0 (the row layout of tq_weight_quantize).  include_k / include_v
-// select the matrices quantized here.
+// MSE codes of K and / or V rows on tcgen05 for head dimension 128 or 64
+// (tq_quantize_tc.cu).  seq_idx and pos may both be null: token t then goes
+// to position t of sequence 0 (the row layout of tq_weight_quantize).
+// include_k / include_v select the matrices quantized here.
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                        void *stream);
@@ -126,10 +127,6 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
 int launch_quantize_tc256(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                           const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                           void *stream);
-// K (is_v false) or V rows in 64-row tiles for head dimension 64,
-// MSE codes only (tq_quantize_tile.cu).
-int launch_quantize_tile(const DeviceParams &p, const tq_cache &c, const void *x, const int32_t *seq_idx,
-                         const int32_t *pos, int n_tok, bool is_v, void *stream);
 // K rows only through the per-row kernel (batches of at most 1024 rows, or a
 // head dimension other than 128), the same index convention.
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,

@@ -204,9 +204,9 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
   const uint16_t *kk = (const uint16_t *)k, *vv = (const uint16_t *)v;
   if (p.d != kHeadDim) {
     // other head dimensions: the per-row kernel for small batches, else the
-    // tcgen05 kernel (d = 256) or the mma.sync tile kernel (d = 64) for V and
-    // for K without QJL (K with QJL keeps the per-row kernel: the QJL kernel
-    // is specialised for d = 128)
+    // tcgen05 kernels (tq_quantize_tc256.cu for d = 256, tq_quantize_tc.cu
+    // for d = 64) for V and for K without QJL (K with QJL keeps the per-row
+    // kernel: the QJL kernel is specialised for d = 128)
     if (rows <= kRowKernelMaxRows) {
       cfg.gridDim = dim3((unsigned)rows, 2);
       cfg.blockDim = dim3(p.d);
@@ -218,10 +218,9 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
       if (e != 0 || !p.qjl) return e;
       return launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream);
     }
-    int e = launch_quantize_tile(p, c, v, seq_idx, pos, n_tok, true, stream);
-    if (e != 0) return e;
-    return p.qjl ? launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream)
-                 : launch_quantize_tile(p, c, k, seq_idx, pos, n_tok, false, stream);
+    const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, !p.qjl, true, stream);
+    if (e != 0 || !p.qjl) return e;
+    return launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream);
   }
   if (rows <= kRowKernelMaxRows) {
     cfg.gridDim = dim3((unsigned)rows, 2);

@@ -3,14 +3,15 @@
 // "ステップ1: PolarQuant" (ai-accelerate.xyz TurboQuant explainer): every
 // head vector x is rotated by the random orthogonal matrix Pi and each rotated
 // coordinate is quantized with the Lloyd-Max codebook.  Here the rotation of
-// a tile of 128 head vectors is one 128x128x128 bf16 GEMM, z = X Pi^T:
+// a tile of 128 head vectors is one 128 x d x d bf16 GEMM, z = X Pi^T, for
+// head dimension d = 128 or 64 (d = 256 has its own kernel):
 //
 //   producer warp   TMA (cp.async.bulk.tensor, 128-byte swizzle) loads each
 //                   128-row tile of K or V into a 4-deep shared-memory ring;
 //                   Pi stays resident in shared memory for the CTA's lifetime.
-//   MMA warp        one thread issues 8 tcgen05.mma (kind::f16, bf16 inputs,
-//                   fp32 accumulation in tensor memory) per tile and commits
-//                   to mbarriers.
+//   MMA warp        one thread issues d / 16 tcgen05.mma (kind::f16, bf16
+//                   inputs, fp32 accumulation in tensor memory) per tile and
+//                   commits to mbarriers.
 //   4 epilogue      warpgroups, one TMEM accumulator each; every thread owns
 //   warpgroups      one row (vector): ||x|| from the shared-memory tile,
 //                   z from TMEM (tcgen05.ld 32x32b), codes against the
@@ -32,11 +33,30 @@
 namespace tq {
 namespace {
 
-constexpr int D = kHeadDim;
 constexpr int kRingStages = 4;
 constexpr int kEpiGroups = 4;
 constexpr int kQThreads = 32 * (2 + 4 * kEpiGroups);
-constexpr unsigned kTmemCols = 512;               // 4 accumulators of 128 columns
+
+// The shapes that depend on the head dimension W: a tile is W / 64 boxes of
+// 128 rows x 64 coordinates, Pi W / 64 boxes of W rows.
+template <int W>
+struct TcShape {
+  static constexpr int boxes = W / 64;
+  static constexpr int tile_bytes = kTileRows * W * 2;
+  static constexpr int pi_bytes = W * W * 2;
+  static constexpr int pi_box = W * 128;
+  static constexpr unsigned tmem_cols = kEpiGroups * W;  // one accumulator of W columns per group
+  // instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major, N = W, M = 128
+  static constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(W >> 3) << 17) | ((128u >> 4) << 24);
+  static constexpr int smem = 1024 + pi_bytes + kRingStages * tile_bytes;
+};
+
+__device__ __forceinline__ void tc_mma_n(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                   tmem_d),
+               "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
 
 struct QuantTcArgs {
   DeviceParams p;
@@ -50,15 +70,16 @@ struct QuantTcArgs {
 
 
 
-template <int BK, int BV>
+template <int W, int BK, int BV>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                        const __grid_constant__ CUtensorMap map_pi, const QuantTcArgs a) {
+  using Sh = TcShape<W>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte aligned region: Pi (32 KB) then the ring
+  // 1024-byte aligned region: Pi then the ring
   unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char *pi_tile = smem;
-  unsigned char *ring = smem + kTileBytes;
+  unsigned char *ring = smem + Sh::pi_bytes;
   __shared__ __align__(8) uint64_t full_bar[kRingStages], empty_bar[kRingStages];
   __shared__ __align__(8) uint64_t tfull_bar[kEpiGroups], tempty_bar[kEpiGroups], pi_bar;
   __shared__ uint32_t tmem_base_slot;
@@ -82,7 +103,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   }
   if (warp == 1) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base_slot)),
-                 "r"(kTmemCols)
+                 "r"(Sh::tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -92,9 +113,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const uint32_t tmem_base = tmem_base_slot;
   if (warp == 0 && lane == 0) {  // Pi belongs to the context: no earlier kernel writes it
     const uint32_t pb = smem_addr(&pi_bar);
-    bar_expect_tx(pb, kTileBytes);
-    tma_load_2d(smem_addr(pi_tile), &map_pi, 0, 0, pb);
-    tma_load_2d(smem_addr(pi_tile + kBoxBytes), &map_pi, 64, 0, pb);
+    bar_expect_tx(pb, Sh::pi_bytes);
+#pragma unroll
+    for (int b = 0; b < Sh::boxes; ++b) tma_load_2d(smem_addr(pi_tile + b * Sh::pi_box), &map_pi, 64 * b, 0, pb);
   }
   // launched as a programmatic dependent: inputs and the cache are touched
   // only once the previous kernel in the stream has completed
@@ -118,10 +139,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const CUtensorMap *map = is_k ? &map_k : &map_v;
         const int row0 = (is_k ? t : t - a.tiles_k) * kTileRows;
         const uint32_t fb = smem_addr(&full_bar[slot]);
-        unsigned char *st = ring + slot * kTileBytes;
-        bar_expect_tx(fb, kTileBytes);
-        tma_load_2d(smem_addr(st), map, 0, row0, fb);
-        tma_load_2d(smem_addr(st + kBoxBytes), map, 64, row0, fb);
+        unsigned char *st = ring + slot * Sh::tile_bytes;
+        bar_expect_tx(fb, Sh::tile_bytes);
+#pragma unroll
+        for (int b = 0; b < Sh::boxes; ++b) tma_load_2d(smem_addr(st + b * kBoxBytes), map, 64 * b, row0, fb);
         issued = i + 1;
       }
       bar_wait(pb, 0);
@@ -140,12 +161,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (ok && i >= kEpiGroups) ok = bar_wait(smem_addr(&tempty_bar[acc]), ((i / kEpiGroups) - 1) & 1);
         if (!ok || *(volatile int *)&abort_flag) break;
         tc_fence_after();
-        const uint32_t a0 = smem_addr(ring + slot * kTileBytes), b0 = smem_addr(pi_tile);
-        const uint32_t d = tmem_base + acc * 128;
+        const uint32_t a0 = smem_addr(ring + slot * Sh::tile_bytes), b0 = smem_addr(pi_tile);
+        const uint32_t d = tmem_base + acc * W;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;  // 16 bf16 along K per MMA
-          tc_mma(d, sw128_desc(a0 + off), sw128_desc(b0 + off), kk > 0);
+        for (int kk = 0; kk < W / 16; ++kk) {  // 16 bf16 along K per MMA
+          const uint32_t ao = (kk >> 2) * kBoxBytes + (kk & 3) * 32, bo = (kk >> 2) * Sh::pi_box + (kk & 3) * 32;
+          tc_mma_n(d, sw128_desc(a0 + ao), sw128_desc(b0 + bo), Sh::idesc, kk > 0);
         }
         tc_commit(smem_addr(&tfull_bar[acc]));
         tc_commit(smem_addr(&empty_bar[slot]));
@@ -189,10 +210,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // chunks permuted by r % 8; reading chunk c ^ (r % 8) keeps a warp's loads
       // conflict-free, and the order does not matter to a sum of squares.  bf16
       // squares are exact in fp32.
-      const unsigned char *st = ring + slot * kTileBytes;
+      const unsigned char *st = ring + slot * Sh::tile_bytes;
       float2 ss = make_float2(0.f, 0.f);  // sums of the squares of the low and the high halves
 #pragma unroll
-      for (int box = 0; box < 2; ++box)
+      for (int box = 0; box < Sh::boxes; ++box)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 u =
@@ -214,26 +235,27 @@ __global__ void __launch_bounds__(kQThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t trow = tmem_base + g * 128 + ((uint32_t)(32 * quarter) << 16);
-      uint32_t words[16];
+      const uint32_t trow = tmem_base + g * W + ((uint32_t)(32 * quarter) << 16);
+      constexpr int C = W / 16;  // chunks of 16 columns; C / 2 * bits words per row
+      uint32_t words[C / 2 * 4];
       if constexpr (BK == BV) {  // one copy of the epilogue code for K and V tiles
         float thr[kMaxLevels];
 #pragma unroll
         for (int e = 0; e < kMaxLevels; ++e) thr[e] = is_k ? tk[e] : tv[e];
-        uint32_t w[4 * BK];
-        epilogue_row<BK>(thr, nrm, trow, w);
+        uint32_t w[C / 2 * BK];
+        epilogue_row<BK, C>(thr, nrm, trow, w);
 #pragma unroll
-        for (int e = 0; e < 4 * BK; ++e) words[e] = w[e];
+        for (int e = 0; e < C / 2 * BK; ++e) words[e] = w[e];
       } else if (is_k) {
-        uint32_t w[4 * BK];
-        epilogue_row<BK>(tk, nrm, trow, w);
+        uint32_t w[C / 2 * BK];
+        epilogue_row<BK, C>(tk, nrm, trow, w);
 #pragma unroll
-        for (int e = 0; e < 4 * BK; ++e) words[e] = w[e];
+        for (int e = 0; e < C / 2 * BK; ++e) words[e] = w[e];
       } else {
-        uint32_t w[4 * BV];
-        epilogue_row<BV>(tv, nrm, trow, w);
+        uint32_t w[C / 2 * BV];
+        epilogue_row<BV, C>(tv, nrm, trow, w);
 #pragma unroll
-        for (int e = 0; e < 4 * BV; ++e) words[e] = w[e];
+        for (int e = 0; e < C / 2 * BV; ++e) words[e] = w[e];
       }
       tc_fence_before();
       __syncwarp();
@@ -245,11 +267,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (slot_i < 0 && tok_h == 0 && is_k) atomicOr(a.p.err, kErrTokenRange);
       }
       if (slot_i >= 0) {
-        const int bits = is_k ? BK : BV;
-        uint4 *dst = reinterpret_cast<uint4 *>((is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(16 * bits));
+        const int bits = is_k ? BK : BV;  // W / 8 * bits bytes per row
+        unsigned char *row_dst = (is_k ? a.c.codes_k : a.c.codes_v) + slot_i * (long)(W / 8 * bits);
+        if constexpr (W == 128) {
+          uint4 *dst = reinterpret_cast<uint4 *>(row_dst);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q < bits) dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+          for (int q = 0; q < 4; ++q)
+            if (q < bits) dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+        } else {
+          uint2 *dst = reinterpret_cast<uint2 *>(row_dst);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < bits) dst[q] = make_uint2(words[2 * q], words[2 * q + 1]);
+        }
         (is_k ? a.c.norm_k : a.c.norm_v)[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
       }
       if (*(volatile int *)&abort_flag) break;
@@ -261,51 +291,56 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Sh::tmem_cols)
                  : "memory");
   }
 }
 
 
-constexpr int kQuantTcSmem = 1024 + kTileBytes * (1 + kRingStages);
-
 using QuantTcFn = void (*)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
                            const __grid_constant__ CUtensorMap, const QuantTcArgs);
 
-template <int BK>
+template <int W, int BK>
 QuantTcFn pick_bv(int bv) {
-  return bv == 2 ? quantize_tc_kernel<BK, 2> : bv == 3 ? quantize_tc_kernel<BK, 3> : quantize_tc_kernel<BK, 4>;
+  return bv == 2 ? quantize_tc_kernel<W, BK, 2> : bv == 3 ? quantize_tc_kernel<W, BK, 3> : quantize_tc_kernel<W, BK, 4>;
 }
 
-QuantTcFn pick(int bk, int bv) { return bk == 2 ? pick_bv<2>(bv) : bk == 3 ? pick_bv<3>(bv) : pick_bv<4>(bv); }
+template <int W>
+QuantTcFn pick(int bk, int bv) {
+  return bk == 2 ? pick_bv<W, 2>(bv) : bk == 3 ? pick_bv<W, 3>(bv) : pick_bv<W, 4>(bv);
+}
 
 }  // namespace
 
 int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                        const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                        void *stream) {
+  if (p.d != 64 && p.d != kHeadDim) return (int)cudaErrorInvalidValue;
+  const int W = p.d;
   // cached per device (the attribute applies to the current device), and
   // atomically, as calls may come from several threads
   static std::atomic<int> cached_sm[kMaxDevices];
-  static std::atomic<bool> configured[kMaxDevices][3][3];
+  static std::atomic<bool> configured[kMaxDevices][2][3][3];
   const int dev = current_device();
   int n_sm = cached_sm[dev].load(std::memory_order_relaxed);
   if (n_sm == 0) {
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
     cached_sm[dev].store(n_sm, std::memory_order_relaxed);
   }
-  const QuantTcFn fn = pick(p.bits_k, p.bits_v);
-  std::atomic<bool> &done = configured[dev][p.bits_k - 2][p.bits_v - 2];
+  const QuantTcFn fn = W == 64 ? pick<64>(p.bits_k, p.bits_v) : pick<kHeadDim>(p.bits_k, p.bits_v);
+  const int smem = W == 64 ? TcShape<64>::smem : TcShape<kHeadDim>::smem;
+  std::atomic<bool> &done = configured[dev][W == 64 ? 0 : 1][p.bits_k - 2][p.bits_v - 2];
   if (!done.load(std::memory_order_acquire)) {
-    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantTcSmem);
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     done.store(true, std::memory_order_release);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
+  const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mk, mv, mp;
   std::memset(&mk, 0, sizeof mk);
   std::memset(&mv, 0, sizeof mv);
-  if ((include_v && !make_row_map(&mv, v, rows)) || !make_row_map(&mp, p.pi, D) ||
-      (include_k && !make_row_map(&mk, k, rows)))
+  if ((include_v && !make_row_map(&mv, v, rows, bf16, W)) || !make_row_map(&mp, p.pi, W, bf16, W, W) ||
+      (include_k && !make_row_map(&mk, k, rows, bf16, W)))
     return (int)cudaErrorInvalidValue;
   if (!include_k) mk = mv;
   if (!include_v) mv = mk;
@@ -321,7 +356,7 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kQThreads);
-  cfg.dynamicSmemBytes = kQuantTcSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = (cudaStream_t)stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;

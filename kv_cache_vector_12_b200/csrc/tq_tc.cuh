@@ -242,9 +242,8 @@ __device__ __forceinline__ uint32_t join16(uint32_t lo, uint32_t hi) {
 // nibble l % 8 of word l / 8 (l < 24), and the eight spare-column codes
 // gathered into the nibbles of one word whose bit k of every nibble then
 // moves to bit 3 of word k.
-template <int B>
-__device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const CodeConsts<B> &k,
-                                           uint32_t (&w)[4 * B]) {
+template <int B, int N>
+__device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const CodeConsts<B> &k, uint32_t (&w)[N]) {
   if constexpr (B == 3) {
     const int g = c >> 1;
     const uint32_t x0 = join16(pack16<3, 4, 4>(z, k), pack16<3, 4, 4>(z + 4, k));
@@ -265,9 +264,10 @@ __device__ __forceinline__ void code_chunk(int c, const float (&z)[16], const Co
   }
 }
 
-template <int B>
+// One row of C chunks of 16 columns (C = d / 16): its C / 2 * B code words.
+template <int B, int C = 8>
 __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], float n, uint32_t tmem_row,
-                                             uint32_t (&words)[4 * B]) {
+                                             uint32_t (&words)[C / 2 * B]) {
   constexpr int half = 1 << (B - 1);
   CodeConsts<B> k;
   const bool live = n > 0x1p-25f;  // stored fp16 norm nonzero
@@ -277,7 +277,7 @@ __device__ __forceinline__ void epilogue_row(const float (&thr)[kMaxLevels], flo
   for (int j = 0; j < half - 1; ++j) k.nt[j] = -thr[half + j] * 0x1p64f;  // positive thresholds x -2^64
   search_consts<B>(k);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < C; ++c) {
     float z[16];
     tmem_ld16(tmem_row + 16 * c, z);
     code_chunk<B>(c, z, k, words);
@@ -301,15 +301,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major [rows][128] matrix of 16-bit elements (bf16 unless
-// `type` says otherwise), boxes of 128 rows x 64 columns (128 bytes) with the 128-byte swizzle the MMA descriptors expect.
+// 2-D map over a row-major [rows][width] matrix of 16-bit elements (bf16
+// unless `type` says otherwise), boxes of box_rows rows x 64 columns (128
+// bytes) with the 128-byte swizzle the MMA descriptors expect.
 bool make_row_map(CUtensorMap *m, const void *base, long rows,
-                  CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+                  CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int width = kHeadDim,
+                  int box_rows = kTileRows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows <= 0) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kTileRows};
+  const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)width * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -47,7 +47,7 @@ def rows(n, h, d, seed, lognormal=True):
 @pytest.mark.parametrize("n_tok", [300, 700])
 def test_quantize_parity(tq, d, bits_k, bits_v, qjl, n_tok):
     """300 tokens x 2 heads: the per-row kernel; 700 x 2 (1400 rows, a ragged
-    last tile of 56): the tile kernel (V, and K without QJL)."""
+    last tile of 120): the tcgen05 kernel (V, and K without QJL)."""
     n_heads = 2
     ctx = tq.Context(d, bits_k, bits_v, qjl, 42)
     ref = params(d, bits_k, bits_v, qjl)
