@@ -1,6 +1,8 @@
 // TurboQuant quantize-on-append for sm_100a, small batches and QJL rows:
 // norm, rotation by Pi, Lloyd-Max codes, bit-pack, optional QJL residual
-// signs; and the dispatch between this kernel and the tensor-core kernel.
+// signs (one CTA per vector, or 32 vectors per CTA for batches of K rows with
+// QJL at head dimensions 64 and 256); and the dispatch between these kernels
+// and the tensor-core kernels.
 //
 // The method: ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み"
 // (rotation + per-coordinate Lloyd-Max, then the 1-bit QJL residual
@@ -181,6 +183,150 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
   }
 }
 
+// ---------------------------------------------------------------------------
+// K rows with QJL in batches, head dimension 64 or 256 (d = 128 batches run on
+// the tcgen05 QJL kernel): the per-row kernel's arithmetic for R vectors per
+// CTA.  Thread i still owns coordinate i, now of R vectors at once, so each
+// row of Pi and of S is read once per R vectors (the per-row kernel reads all
+// of S, d x d fp32, for every vector).  The R vectors sit in shared memory as
+// fp32 (x, then the residuals r in the same buffer); the norms and ||r|| are
+// warp reductions, one vector per warp in turn.  grid = ceil(rows / R).
+// ---------------------------------------------------------------------------
+template <int DH, int R>
+__global__ void __launch_bounds__(DH) quantize_qjl_rows_kernel(DeviceParams p, tq_cache c,
+                                                               const uint16_t *__restrict__ k_in,
+                                                               const int32_t *__restrict__ seq_idx,
+                                                               const int32_t *__restrict__ pos, long n_rows) {
+  constexpr int kWarps = DH / 32;
+  __shared__ __align__(16) float s_v[R][DH];  // x, then r
+  __shared__ float s_n[R], s_g[R];
+  __shared__ long s_slot[R];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long row0 = (long)blockIdx.x * R;
+  PiRow<DH> pw;
+  pw.load(p.pi + tid * DH);
+  // launched as a programmatic dependent: no input is read before the
+  // previous kernel in the stream has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#pragma unroll 4
+  for (int r = 0; r < R; ++r) {  // rows past the end are zero vectors that are never stored
+    const long row = row0 + r;
+    s_v[r][tid] = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid]) : 0.f;
+  }
+  if (tid < R) {
+    const long row = row0 + tid;
+    long slot = -1;
+    if (row < n_rows) {
+      const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
+      // (no index arrays: token t goes to position t of sequence 0)
+      slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, h, pos ? pos[t] : t);
+      if (slot < 0 && h == 0) atomicOr(p.err, kErrTokenRange);
+    }
+    s_slot[tid] = slot;
+  }
+  __syncthreads();
+  for (int r = warp; r < R; r += kWarps) {  // ||x||, fp32 over exact bf16 squares
+    float v = 0.f;
+#pragma unroll
+    for (int j = lane; j < DH; j += 32) v = fmaf(s_v[r][j], s_v[r][j], v);
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_n[r] = sqrtf(v);
+  }
+  // z_i = (Pi x)_i of the R vectors: row i of Pi against each vector
+  float acc[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll(DH <= 128 ? DH / 8 : 1)
+  for (int c8 = 0; c8 < DH / 8; ++c8) {
+    const uint4 w = pw.get(c8);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    float pf[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pf[2 * e] = __uint_as_float(u[e] << 16);
+      pf[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 x0 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8]);
+      const float4 x1 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8 + 4]);
+      acc[r] = fmaf(pf[0], x0.x, acc[r]);
+      acc[r] = fmaf(pf[1], x0.y, acc[r]);
+      acc[r] = fmaf(pf[2], x0.z, acc[r]);
+      acc[r] = fmaf(pf[3], x0.w, acc[r]);
+      acc[r] = fmaf(pf[4], x1.x, acc[r]);
+      acc[r] = fmaf(pf[5], x1.y, acc[r]);
+      acc[r] = fmaf(pf[6], x1.z, acc[r]);
+      acc[r] = fmaf(pf[7], x1.w, acc[r]);
+    }
+  }
+  __syncthreads();  // every thread is done with x: the buffer takes z, then r
+#pragma unroll
+  for (int r = 0; r < R; ++r) s_v[r][tid] = acc[r];
+  const int bits = p.bits_k, half = 1 << (bits - 1);
+  const float *thr = p.cb + 1 * kMaxLevels, *cent = p.cb;
+#pragma unroll 1
+  for (int r = 0; r < R; ++r) {
+    const float n = s_n[r];
+    // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
+    const bool live = n > 0x1p-25f;
+    const float z = live ? s_v[r][tid] : 0.f;
+    const float a = fabsf(z);
+    int m = 0;
+    for (int j = 0; j < half - 1; ++j) m += a > thr[half + j] * n ? 1 : 0;
+    const int code = z > 0.f ? half + m : half - 1 - m;
+    const long slot = s_slot[r];
+    uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + (slot < 0 ? 0 : slot) * (DH * bits / 8));
+    for (int wd = 0; wd < bits; ++wd) {  // warp w owns words w*bits .. w*bits+bits-1
+      uint32_t contrib = 0;
+      for (int kb = 0; kb < bits; ++kb) {
+        const int pbit = code_bit_pos(bits, tid, kb) - 32 * bits * warp;
+        if ((pbit >> 5) == wd) contrib |= (uint32_t)((code >> kb) & 1) << (pbit & 31);
+      }
+      const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
+      if (lane == 0 && slot >= 0) dst[warp * bits + wd] = word;
+    }
+    if (tid == 0 && slot >= 0) c.norm_k[slot] = f32_to_f16_bits_sat(n);
+    const float y = live ? z / n : 0.f;
+    s_v[r][tid] = y - cent[code];
+  }
+  __syncthreads();
+  for (int r = warp; r < R; r += kWarps) {  // ||r||
+    float v = 0.f;
+#pragma unroll
+    for (int j = lane; j < DH; j += 32) v = fmaf(s_v[r][j], s_v[r][j], v);
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_g[r] = sqrtf(v);
+  }
+  // (S r)_i of the R residuals: row i of S (fp32) against each residual
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  const float4 *srow = reinterpret_cast<const float4 *>(p.s + (size_t)tid * DH);
+#pragma unroll 2
+  for (int c4 = 0; c4 < DH / 4; ++c4) {
+    const float4 w = srow[c4];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 x = *reinterpret_cast<const float4 *>(&s_v[r][4 * c4]);
+      acc[r] = fmaf(w.x, x.x, acc[r]);
+      acc[r] = fmaf(w.y, x.y, acc[r]);
+      acc[r] = fmaf(w.z, x.z, acc[r]);
+      acc[r] = fmaf(w.w, x.w, acc[r]);
+    }
+  }
+  __syncthreads();  // s_g
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const long slot = s_slot[r];
+    const uint32_t sb = __ballot_sync(0xffffffffu, acc[r] >= 0.f);
+    if (slot >= 0) {
+      if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp] = sb;
+      if (tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(s_g[r]);
+    }
+  }
+}
+
 }  // namespace
 
 // Batches of up to kRowKernelMaxRows rows per matrix (decode-time appends) use
@@ -232,11 +378,24 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
 
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                            const int32_t *pos, int n_tok, void *stream) {
+  const long rows = (long)n_tok * c.n_kv_heads;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long)n_tok * c.n_kv_heads), 1);  // y = 0: K only
   cfg.blockDim = dim3(p.d);
   cfg.stream = (cudaStream_t)stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k;
+  if (p.d != kHeadDim && p.qjl) {  // R = 32 vectors per CTA
+    constexpr int R = 32;
+    cfg.gridDim = dim3((unsigned)((rows + R - 1) / R));
+    if (p.d == 64)
+      return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_rows_kernel<64, R>, p, c, kk, seq_idx, pos, rows);
+    return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_rows_kernel<256, R>, p, c, kk, seq_idx, pos, rows);
+  }
+  cfg.gridDim = dim3((unsigned)rows, 1);  // y = 0: K only
   if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, kk, seq_idx, pos);
   if (p.d == 256) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<256>, p, c, kk, kk, seq_idx, pos);
   return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<kHeadDim>, p, c, kk, kk, seq_idx, pos);

@@ -47,11 +47,33 @@ def rows(n, h, d, seed, lognormal=True):
 @pytest.mark.parametrize("n_tok", [300, 700])
 def test_quantize_parity(tq, d, bits_k, bits_v, qjl, n_tok):
     """300 tokens x 2 heads: the per-row kernel; 700 x 2 (1400 rows, a ragged
-    last tile of 120): the tcgen05 kernel (V, and K without QJL)."""
+    last tile of 120): the tcgen05 kernel (V, and K without QJL) and, for K
+    with QJL, the batched QJL kernel (32 vectors per CTA, the last CTA 24)."""
     n_heads = 2
+    k, v = rows(n_tok, n_heads, d, 5 + d), rows(n_tok, n_heads, d, 6 + d)
+    _quantize_and_compare(tq, d, bits_k, bits_v, qjl, k, v)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("qjl", [0, 1])
+def test_quantize_zero_and_tiny_vectors_in_batches(tq, d, qjl):
+    """700 tokens x 2 heads (the batched kernels) with rows scaled by 2^-32
+    (stored fp16 norm 0: the zero vector, whose residual is minus the centroid
+    of code 2^(b-1) - 1) and by 2^-20 (a subnormal fp16 norm: ordinary
+    codes), and exact zero rows."""
+    n_tok, n_heads = 700, 2
+    k, v = rows(n_tok, n_heads, d, 15 + d), rows(n_tok, n_heads, d, 16 + d)
+    for x in (k, v):
+        x[3:9] = (x[3:9].float() * 2.0 ** -32).to(torch.bfloat16)
+        x[9:15] = (x[9:15].float() * 2.0 ** -20).to(torch.bfloat16)
+        x[40:43] = 0
+    _quantize_and_compare(tq, d, 3, 3, qjl, k, v)
+
+
+def _quantize_and_compare(tq, d, bits_k, bits_v, qjl, k, v):
+    n_tok, n_heads = k.shape[0], k.shape[1]
     ctx = tq.Context(d, bits_k, bits_v, qjl, 42)
     ref = params(d, bits_k, bits_v, qjl)
-    k, v = rows(n_tok, n_heads, d, 5 + d), rows(n_tok, n_heads, d, 6 + d)
     cache = tq.Cache(ctx, 1, n_heads, (n_tok + 63) // 64 * 64)
     pos = torch.randperm(n_tok, generator=torch.Generator().manual_seed(d)).to(torch.int32)
     tq.quantize(ctx, cache, k.cuda(), v.cuda(), torch.zeros(n_tok, dtype=torch.int32, device="cuda"), pos.cuda())
@@ -68,6 +90,31 @@ def test_quantize_parity(tq, d, bits_k, bits_v, qjl, n_tok):
                 sc = ph.compare_signs(pl["qjl_bits"][0, h, ps], qz, skip_vectors=cc["vec_mismatch"])
                 assert sc["outside_window"] == 0, sc
                 assert ph.compare_fp16(pl["qjl_norm"][0, h, ps], qz.qjl_gamma)["worse"] == 0
+
+
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("qjl", [0, 1])
+def test_quantize_batches_flag_out_of_range_tokens(tq, d, qjl):
+    """1200 rows per matrix (the batched kernels): tokens with a bad sequence
+    or position are flagged and skipped, every other token lands."""
+    ctx = tq.Context(d, 3, 3, qjl, 42)
+    n_tok, n_heads = 600, 2
+    cache = tq.Cache(ctx, 2, n_heads, 640)
+    k = rows(n_tok, n_heads, d, 11).cuda()
+    seq_idx = torch.zeros(n_tok, dtype=torch.int32)
+    pos = torch.arange(n_tok, dtype=torch.int32)
+    seq_idx[5], pos[17], pos[599] = 2, 640, -1                         # no sequence 2; pos outside [0, 640)
+    tq.quantize(ctx, cache, k, k, seq_idx.cuda(), pos.cuda())
+    with pytest.raises(tq.TQError) as ei:
+        ctx.check_device_errors()
+    assert ei.value.status == tq.TQ_ERR_DEVICE
+    expect = torch.zeros(n_heads, 640, dtype=torch.bool)
+    expect[:, torch.tensor([t for t in range(n_tok) if t not in (5, 17, 599)])] = True
+    assert torch.equal(cache.planes["norm_k"][0].ne(0).cpu(), expect)
+    assert torch.equal(cache.planes["norm_v"][0].ne(0).cpu(), expect)
+    assert int(cache.planes["norm_k"][1].ne(0).sum()) == 0
+    if qjl:
+        assert torch.equal(cache.planes["qjl_norm"][0].ne(0).cpu(), expect)
 
 
 @pytest.mark.parametrize("d", [64, 256])
