@@ -38,6 +38,7 @@
 #include <atomic>
 #include <cmath>
 
+#include "tq_f32x2.cuh"
 #include "tq_internal.h"
 #include "tq_stream.cuh"
 
@@ -1215,19 +1216,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       tcx_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&s_empty));
+      // x' = S ||k||, two keys per instruction; the row factor fq (> 0)
+      // enters in the exponent below, so max x = fq max x'
       float mx = -INFINITY;
 #pragma unroll
       for (int j4 = 0; j4 < 16; ++j4) {
         const float4 kf = kn4[j4];
-        const float kk[4] = {kf.x, kf.y, kf.z, kf.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 4 * j4 + e;
-          uint32_t &cell = sv[j >> 4][j & 15];
-          const float x = __uint_as_float(cell) * fq * kk[e];
-          const float y = (!masked || kfirst + j <= pos) ? x : -INFINITY;
-          cell = __float_as_uint(y);
-          mx = fmaxf(mx, y);
+        for (int e = 0; e < 4; e += 2) {
+          const int j = 4 * j4 + e;  // even: keys j, j + 1 sit in one 16-column load
+          uint32_t &c0 = sv[j >> 4][j & 15], &c1 = sv[j >> 4][(j & 15) + 1];
+          float2 x = mul2(make_float2(__uint_as_float(c0), __uint_as_float(c1)),
+                          e ? make_float2(kf.z, kf.w) : make_float2(kf.x, kf.y));
+          if (masked) {
+            if (kfirst + j > pos) x.x = -INFINITY;
+            if (kfirst + j + 1 > pos) x.y = -INFINITY;
+          }
+          c0 = __float_as_uint(x.x);
+          c1 = __float_as_uint(x.y);
+          mx = max3(mx, x.x, x.y);
         }
       }
       // the row's maximum from both halves (double-buffered by tile parity)
@@ -1236,7 +1243,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       if (lane == 0) mbar_arrive(smem_u32(&mx_bar[b]));
       ok = tc_wait(&mx_bar[b], (it >> 1) & 1, err, abf);
       if (!ok) break;
-      mx = fmaxf(s_max[b][0][row], s_max[b][1][row]);
+      mx = fmaxf(s_max[b][0][row], s_max[b][1][row]) * fq;
       const float mn = fmaxf(m_run, mx);
       const float ref = fmaxf(mn, -3.0e38f);
       const float al = fast_exp2(m_run - ref);
@@ -1261,30 +1268,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
           }
         }
       }
-      float ls = 0.f;
+      // p = 2^(fq x' - ref), P' = p ||v||, two keys per instruction
+      float2 ls2 = make_float2(0.f, 0.f);
+      const float2 fq2 = make_float2(fq, fq), nref2 = make_float2(-ref, -ref);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const float4 vf = vn4[8 * c + j4];
-          const float vv[4] = {vf.x, vf.y, vf.z, vf.w};
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int j = 32 * c + 4 * j4 + 2 * e;
-            const float sa = __uint_as_float(sv[j >> 4][j & 15]), sb = __uint_as_float(sv[(j + 1) >> 4][(j + 1) & 15]);
-            const float pa = fast_exp2(sa - ref), pb = fast_exp2(sb - ref);
-            ls += pa + pb;
-            // masked keys (and keys past the copied ones, whose norms are not
-            // set) contribute 0
-            pk[2 * j4 + e] = masked ? pack_half2(sa == -INFINITY ? 0.f : pa * vv[2 * e],
-                                                 sb == -INFINITY ? 0.f : pb * vv[2 * e + 1])
-                                    : pack_half2(pa * vv[2 * e], pb * vv[2 * e + 1]);
+            const float sa = __uint_as_float(sv[j >> 4][j & 15]), sb = __uint_as_float(sv[j >> 4][(j & 15) + 1]);
+            const float2 t = fma2(make_float2(sa, sb), fq2, nref2);
+            const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            ls2 = add2(ls2, pe);
+            float2 pv = mul2(pe, e ? make_float2(vf.z, vf.w) : make_float2(vf.x, vf.y));
+            if (masked) {  // masked keys (and keys past the copied ones, whose norms are not set) contribute 0
+              if (sa == -INFINITY) pv.x = 0.f;
+              if (sb == -INFINITY) pv.y = 0.f;
+            }
+            pk[2 * j4 + e] = pack_half2(pv.x, pv.y);
           }
         }
         tmem_st16x(t_p + 16 * c, pk);
       }
-      l_run = fmaf(l_run, al, ls);
+      l_run = fmaf(l_run, al, ls2.x + ls2.y);
       tmem_wait_st();
       tcx_fence_before();
       __syncwarp();
