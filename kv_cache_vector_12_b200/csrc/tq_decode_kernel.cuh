@@ -42,6 +42,7 @@
 #include <atomic>
 #include <cmath>
 
+#include "tq_f32x2.cuh"
 #include "tq_internal.h"
 #include "tq_stream.cuh"
 
@@ -632,20 +633,43 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           float sc[4][2];  // [token u][head hd]
+          if constexpr (CTAS == 3) {
+            // the two heads of a token as one packed fp32 pair (f32x2 rounds
+            // each lane as the scalar form would)
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int hd = 0; hd < 2; ++hd) {
-              const int rb = u >> 1, e = 2 * (u & 1) + hd;
+            for (int u = 0; u < 4; ++u) {
+              const int rb = u >> 1, e = 2 * (u & 1);
               // 65536 hh + 256 mid + ll = 256 (256 hh + mid) + ll; 256 hh + mid fits int32
-              const int hm = (chh[rb][nt][e] << 8) + cmid[rb][nt][e];
-              float v = fmaf(256.f, (float)hm, (float)cll[rb][nt][e]) * fq[nt][hd];
+              const float2 hm = make_float2((float)((chh[rb][nt][e] << 8) + cmid[rb][nt][e]),
+                                            (float)((chh[rb][nt][e + 1] << 8) + cmid[rb][nt][e + 1]));
+              float2 v = mul2(fma2(make_float2(256.f, 256.f), hm,
+                                   make_float2((float)cll[rb][nt][e], (float)cll[rb][nt][e + 1])),
+                              make_float2(fq[nt][0], fq[nt][1]));
               if constexpr (QJL) {
-                const float dj = fmaf(256.f, (float)cjh[rb][nt][e], (float)cjl[rb][nt][e]);
-                v = fmaf(gm[u] * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
+                const float dj0 = fmaf(256.f, (float)cjh[rb][nt][e], (float)cjl[rb][nt][e]);
+                const float dj1 = fmaf(256.f, (float)cjh[rb][nt][e + 1], (float)cjl[rb][nt][e + 1]);
+                v.x = fmaf(gm[u] * fj[nt][0], fmaf(-2.f, dj0, -jsum[nt][0]), v.x);
+                v.y = fmaf(gm[u] * fj[nt][1], fmaf(-2.f, dj1, -jsum[nt][1]), v.y);
               }
-              sc[u][hd] = v * nk[u];
+              v = mul2(v, make_float2(nk[u], nk[u]));
+              sc[u][0] = v.x;
+              sc[u][1] = v.y;
             }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int hd = 0; hd < 2; ++hd) {
+                const int rb = u >> 1, e = 2 * (u & 1) + hd;
+                const int hm = (chh[rb][nt][e] << 8) + cmid[rb][nt][e];
+                float v = fmaf(256.f, (float)hm, (float)cll[rb][nt][e]) * fq[nt][hd];
+                if constexpr (QJL) {
+                  const float dj = fmaf(256.f, (float)cjh[rb][nt][e], (float)cjl[rb][nt][e]);
+                  v = fmaf(gm[u] * fj[nt][hd], fmaf(-2.f, dj, -jsum[nt][hd]), v);
+                }
+                sc[u][hd] = v * nk[u];
+              }
+          }
           if (partial) {  // masked tokens carry NaN norms: their scores become -inf, their weights 0
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -653,32 +677,68 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
               for (int hd = 0; hd < 2; ++hd)
                 if (isnan(nv[u])) sc[u][hd] = -INFINITY;
           }
+          if constexpr (CTAS == 3) {
+            // both heads' maxima first, then their weights as packed pairs
+            float nref[2];
 #pragma unroll
-          for (int hd = 0; hd < 2; ++hd) {
-            float mx = fmaxf(fmaxf(sc[0][hd], sc[1][hd]), fmaxf(sc[2][hd], sc[3][hd]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const float mn = fmaxf(m_run[nt][hd], mx);
-            // a finite reference keeps exp2(-inf - ref) = 0 when nothing is unmasked yet
-            const float ref = fmaxf(mn, -3.0e38f);
-            const float al = fast_exp2(m_run[nt][hd] - ref);
-            alpha[nt][hd] = al;
-            rescale |= al != 1.f;
-            m_run[nt][hd] = mn;
-            float lsum = 0.f;
+            for (int hd = 0; hd < 2; ++hd) {
+              float mx = fmaxf(max3(sc[0][hd], sc[1][hd], sc[2][hd]), sc[3][hd]);
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              const float mn = fmaxf(m_run[nt][hd], mx);
+              // a finite reference keeps exp2(-inf - ref) = 0 when nothing is unmasked yet
+              const float ref = fmaxf(mn, -3.0e38f);
+              const float al = fast_exp2(m_run[nt][hd] - ref);
+              alpha[nt][hd] = al;
+              rescale |= al != 1.f;
+              m_run[nt][hd] = mn;
+              nref[hd] = -ref;
+            }
+            float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const float pv = fast_exp2(sc[u][hd] - ref);
-              lsum += pv;
-              sc[u][hd] = pv * nv[u];
+              const float2 t = add2(make_float2(sc[u][0], sc[u][1]), make_float2(nref[0], nref[1]));
+              const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+              lsum = add2(lsum, pe);
+              const float2 pv = mul2(pe, make_float2(nv[u], nv[u]));
+              sc[u][0] = pv.x;
+              sc[u][1] = pv.y;
             }
             if (partial) {
 #pragma unroll
               for (int u = 0; u < 4; ++u)
-                if (isnan(nv[u])) sc[u][hd] = 0.f;
+                if (isnan(nv[u])) sc[u][0] = sc[u][1] = 0.f;
             }
-            l_run[nt][hd] = fmaf(l_run[nt][hd], al, lsum);
+            l_run[nt][0] = fmaf(l_run[nt][0], alpha[nt][0], lsum.x);
+            l_run[nt][1] = fmaf(l_run[nt][1], alpha[nt][1], lsum.y);
+          } else {
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+              float mx = fmaxf(fmaxf(sc[0][hd], sc[1][hd]), fmaxf(sc[2][hd], sc[3][hd]));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              const float mn = fmaxf(m_run[nt][hd], mx);
+              const float ref = fmaxf(mn, -3.0e38f);
+              const float al = fast_exp2(m_run[nt][hd] - ref);
+              alpha[nt][hd] = al;
+              rescale |= al != 1.f;
+              m_run[nt][hd] = mn;
+              float lsum = 0.f;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float pv = fast_exp2(sc[u][hd] - ref);
+                lsum += pv;
+                sc[u][hd] = pv * nv[u];
+              }
+              if (partial) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  if (isnan(nv[u])) sc[u][hd] = 0.f;
+              }
+              l_run[nt][hd] = fmaf(l_run[nt][hd], al, lsum);
+            }
           }
 #pragma unroll
           for (int rb = 0; rb < 2; ++rb) {
