@@ -1263,7 +1263,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
             tmem_wait_ld();
             reg_fence16(v);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
+            for (int e = 0; e < 16; e += 2) {
+              const float2 w = mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), make_float2(al, al));
+              v[e] = __float_as_uint(w.x);
+              v[e + 1] = __float_as_uint(w.y);
+            }
             tmem_st16x(t_o + 16 * c, v);
           }
         }
