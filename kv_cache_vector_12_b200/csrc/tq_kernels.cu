@@ -186,25 +186,29 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 // ---------------------------------------------------------------------------
 // K rows with QJL in batches, head dimension 64 or 256 (d = 128 batches run on
 // the tcgen05 QJL kernel): the per-row kernel's arithmetic for R vectors per
-// CTA.  Thread i still owns coordinate i, now of R vectors at once, so each
+// CTA.  Thread t owns coordinates t + h d / C (h < C) of all R vectors, so each
 // row of Pi and of S is read once per R vectors (the per-row kernel reads all
-// of S, d x d fp32, for every vector).  The R vectors sit in shared memory as
-// fp32 (x, then the residuals r in the same buffer); the norms and ||r|| are
-// warp reductions, one vector per warp in turn.  grid = ceil(rows / R).
+// of S, d x d fp32, for every vector), and every broadcast shared-memory load
+// of a vector's coordinates feeds C rows of Pi or S.  The R vectors sit in
+// shared memory as fp32 (x, then z, then the residuals r in the same buffer);
+// the norms and ||r|| are warp reductions, one vector per warp in turn.  A
+// coordinate block of 32 (one word of the cache layout per bit, one word of
+// sign bits) belongs to warp w = block % (d / 32 C).  grid = ceil(rows / R).
 // ---------------------------------------------------------------------------
-template <int DH, int R>
-__global__ void __launch_bounds__(DH) quantize_qjl_rows_kernel(DeviceParams p, tq_cache c,
-                                                               const uint16_t *__restrict__ k_in,
-                                                               const int32_t *__restrict__ seq_idx,
-                                                               const int32_t *__restrict__ pos, long n_rows) {
-  constexpr int kWarps = DH / 32;
-  __shared__ __align__(16) float s_v[R][DH];  // x, then r
+template <int DH, int R, int BK, int C>
+__global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams p, tq_cache c,
+                                                                   const uint16_t *__restrict__ k_in,
+                                                                   const int32_t *__restrict__ seq_idx,
+                                                                   const int32_t *__restrict__ pos, long n_rows) {
+  constexpr int kThreads = DH / C, kWarps = kThreads / 32;
+  __shared__ __align__(16) float s_v[R][DH];  // x, then z, then r
   __shared__ float s_n[R], s_g[R];
   __shared__ long s_slot[R];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long row0 = (long)blockIdx.x * R;
-  PiRow<DH> pw;
-  pw.load(p.pi + tid * DH);
+  PiRow<DH> pw[C];
+#pragma unroll
+  for (int h = 0; h < C; ++h) pw[h].load(p.pi + (tid + h * kThreads) * DH);
   // launched as a programmatic dependent: no input is read before the
   // previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -212,16 +216,18 @@ __global__ void __launch_bounds__(DH) quantize_qjl_rows_kernel(DeviceParams p, t
 #pragma unroll 4
   for (int r = 0; r < R; ++r) {  // rows past the end are zero vectors that are never stored
     const long row = row0 + r;
-    s_v[r][tid] = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid]) : 0.f;
+#pragma unroll
+    for (int h = 0; h < C; ++h)
+      s_v[r][tid + h * kThreads] = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid + h * kThreads]) : 0.f;
   }
   if (tid < R) {
     const long row = row0 + tid;
     long slot = -1;
     if (row < n_rows) {
-      const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
+      const int t = (int)(row / c.n_kv_heads), hd = (int)(row % c.n_kv_heads);
       // (no index arrays: token t goes to position t of sequence 0)
-      slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, h, pos ? pos[t] : t);
-      if (slot < 0 && h == 0) atomicOr(p.err, kErrTokenRange);
+      slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, hd, pos ? pos[t] : t);
+      if (slot < 0 && hd == 0) atomicOr(p.err, kErrTokenRange);
     }
     s_slot[tid] = slot;
   }
@@ -233,63 +239,94 @@ __global__ void __launch_bounds__(DH) quantize_qjl_rows_kernel(DeviceParams p, t
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_n[r] = sqrtf(v);
   }
-  // z_i = (Pi x)_i of the R vectors: row i of Pi against each vector
-  float acc[R];
+  // z_i = (Pi x)_i of the R vectors: rows i of Pi against each vector
+  float acc[C][R];
 #pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  for (int h = 0; h < C; ++h)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[h][r] = 0.f;
 #pragma unroll(DH <= 128 ? DH / 8 : 1)
   for (int c8 = 0; c8 < DH / 8; ++c8) {
-    const uint4 w = pw.get(c8);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-    float pf[8];
+    float pf[C][8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      pf[2 * e] = __uint_as_float(u[e] << 16);
-      pf[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+    for (int h = 0; h < C; ++h) {
+      const uint4 w = pw[h].get(c8);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pf[h][2 * e] = __uint_as_float(u[e] << 16);
+        pf[h][2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+      }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const float4 x0 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8]);
       const float4 x1 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8 + 4]);
-      acc[r] = fmaf(pf[0], x0.x, acc[r]);
-      acc[r] = fmaf(pf[1], x0.y, acc[r]);
-      acc[r] = fmaf(pf[2], x0.z, acc[r]);
-      acc[r] = fmaf(pf[3], x0.w, acc[r]);
-      acc[r] = fmaf(pf[4], x1.x, acc[r]);
-      acc[r] = fmaf(pf[5], x1.y, acc[r]);
-      acc[r] = fmaf(pf[6], x1.z, acc[r]);
-      acc[r] = fmaf(pf[7], x1.w, acc[r]);
+#pragma unroll
+      for (int h = 0; h < C; ++h) {
+        acc[h][r] = fmaf(pf[h][0], x0.x, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][1], x0.y, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][2], x0.z, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][3], x0.w, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][4], x1.x, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][5], x1.y, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][6], x1.z, acc[h][r]);
+        acc[h][r] = fmaf(pf[h][7], x1.w, acc[h][r]);
+      }
     }
   }
   __syncthreads();  // every thread is done with x: the buffer takes z, then r
 #pragma unroll
-  for (int r = 0; r < R; ++r) s_v[r][tid] = acc[r];
-  const int bits = p.bits_k, half = 1 << (bits - 1);
-  const float *thr = p.cb + 1 * kMaxLevels, *cent = p.cb;
+  for (int h = 0; h < C; ++h)
+#pragma unroll
+    for (int r = 0; r < R; ++r) s_v[r][tid + h * kThreads] = acc[h][r];
+  constexpr int half = 1 << (BK - 1);
+  const float *cent = p.cb;
+  float thr[half - 1];  // the positive thresholds
+#pragma unroll
+  for (int j = 0; j < half - 1; ++j) thr[j] = p.cb[1 * kMaxLevels + half + j];
+  // this thread's bit positions inside the BK words of its coordinate blocks
+  // (the cache layout: LSB-first for 2 and 4 bits, nibbles plus the spare
+  // column for 3 bits)
+  int wd_of[C][BK], sh_of[C][BK];
+#pragma unroll
+  for (int h = 0; h < C; ++h)
+#pragma unroll
+    for (int kb = 0; kb < BK; ++kb) {
+      const int i = tid + h * kThreads;
+      const int pbit = code_bit_pos(BK, i, kb) - 32 * BK * (i >> 5);
+      wd_of[h][kb] = pbit >> 5;
+      sh_of[h][kb] = pbit & 31;
+    }
 #pragma unroll 1
   for (int r = 0; r < R; ++r) {
     const float n = s_n[r];
     // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
     const bool live = n > 0x1p-25f;
-    const float z = live ? s_v[r][tid] : 0.f;
-    const float a = fabsf(z);
-    int m = 0;
-    for (int j = 0; j < half - 1; ++j) m += a > thr[half + j] * n ? 1 : 0;
-    const int code = z > 0.f ? half + m : half - 1 - m;
     const long slot = s_slot[r];
-    uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + (slot < 0 ? 0 : slot) * (DH * bits / 8));
-    for (int wd = 0; wd < bits; ++wd) {  // warp w owns words w*bits .. w*bits+bits-1
-      uint32_t contrib = 0;
-      for (int kb = 0; kb < bits; ++kb) {
-        const int pbit = code_bit_pos(bits, tid, kb) - 32 * bits * warp;
-        if ((pbit >> 5) == wd) contrib |= (uint32_t)((code >> kb) & 1) << (pbit & 31);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + (slot < 0 ? 0 : slot) * (DH * BK / 8));
+#pragma unroll
+    for (int h = 0; h < C; ++h) {
+      const int i = tid + h * kThreads;
+      const float z = live ? s_v[r][i] : 0.f;
+      const float a = fabsf(z);
+      int m = 0;
+#pragma unroll
+      for (int j = 0; j < half - 1; ++j) m += a > thr[j] * n ? 1 : 0;
+      const int code = z > 0.f ? half + m : half - 1 - m;
+#pragma unroll
+      for (int wd = 0; wd < BK; ++wd) {  // block i / 32 owns words BK (i / 32) ..
+        uint32_t contrib = 0;
+#pragma unroll
+        for (int kb = 0; kb < BK; ++kb)
+          if (wd_of[h][kb] == wd) contrib |= (uint32_t)((code >> kb) & 1) << sh_of[h][kb];
+        const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
+        if (lane == 0 && slot >= 0) dst[(i >> 5) * BK + wd] = word;
       }
-      const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
-      if (lane == 0 && slot >= 0) dst[warp * bits + wd] = word;
+      const float y = live ? z / n : 0.f;
+      s_v[r][i] = y - cent[code];
     }
     if (tid == 0 && slot >= 0) c.norm_k[slot] = f32_to_f16_bits_sat(n);
-    const float y = live ? z / n : 0.f;
-    s_v[r][tid] = y - cent[code];
   }
   __syncthreads();
   for (int r = warp; r < R; r += kWarps) {  // ||r||
@@ -299,31 +336,38 @@ __global__ void __launch_bounds__(DH) quantize_qjl_rows_kernel(DeviceParams p, t
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_g[r] = sqrtf(v);
   }
-  // (S r)_i of the R residuals: row i of S (fp32) against each residual
+  // (S r)_i of the R residuals: rows i of S (fp32) against each residual
 #pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = 0.f;
-  const float4 *srow = reinterpret_cast<const float4 *>(p.s + (size_t)tid * DH);
+  for (int h = 0; h < C; ++h)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[h][r] = 0.f;
 #pragma unroll 2
   for (int c4 = 0; c4 < DH / 4; ++c4) {
-    const float4 w = srow[c4];
+    float4 w[C];
+#pragma unroll
+    for (int h = 0; h < C; ++h) w[h] = reinterpret_cast<const float4 *>(p.s + (size_t)(tid + h * kThreads) * DH)[c4];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const float4 x = *reinterpret_cast<const float4 *>(&s_v[r][4 * c4]);
-      acc[r] = fmaf(w.x, x.x, acc[r]);
-      acc[r] = fmaf(w.y, x.y, acc[r]);
-      acc[r] = fmaf(w.z, x.z, acc[r]);
-      acc[r] = fmaf(w.w, x.w, acc[r]);
+#pragma unroll
+      for (int h = 0; h < C; ++h) {
+        acc[h][r] = fmaf(w[h].x, x.x, acc[h][r]);
+        acc[h][r] = fmaf(w[h].y, x.y, acc[h][r]);
+        acc[h][r] = fmaf(w[h].z, x.z, acc[h][r]);
+        acc[h][r] = fmaf(w[h].w, x.w, acc[h][r]);
+      }
     }
   }
   __syncthreads();  // s_g
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const long slot = s_slot[r];
-    const uint32_t sb = __ballot_sync(0xffffffffu, acc[r] >= 0.f);
-    if (slot >= 0) {
-      if (lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp] = sb;
-      if (tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(s_g[r]);
+#pragma unroll
+    for (int h = 0; h < C; ++h) {
+      const uint32_t sb = __ballot_sync(0xffffffffu, acc[h][r] >= 0.f);
+      if (slot >= 0 && lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp + h * kWarps] = sb;
     }
+    if (slot >= 0 && tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(s_g[r]);
   }
 }
 
@@ -388,12 +432,21 @@ int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void 
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k;
-  if (p.d != kHeadDim && p.qjl) {  // R = 32 vectors per CTA
+  if (p.d != kHeadDim && p.qjl) {  // R = 32 vectors per CTA; two coordinates per thread at d = 256
     constexpr int R = 32;
     cfg.gridDim = dim3((unsigned)((rows + R - 1) / R));
-    if (p.d == 64)
-      return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_rows_kernel<64, R>, p, c, kk, seq_idx, pos, rows);
-    return (int)cudaLaunchKernelEx(&cfg, quantize_qjl_rows_kernel<256, R>, p, c, kk, seq_idx, pos, rows);
+    cfg.blockDim = dim3(p.d == 64 ? 64 : 128);
+    using QjlRowsFn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, long);
+    const QjlRowsFn fn =
+        p.d == 64 ? (p.bits_k == 2   ? quantize_qjl_rows_kernel<64, R, 2, 1>
+                     : p.bits_k == 3 ? quantize_qjl_rows_kernel<64, R, 3, 1>
+                                     : quantize_qjl_rows_kernel<64, R, 4, 1>)
+                  : (p.bits_k == 2   ? quantize_qjl_rows_kernel<256, R, 2, 2>
+                     : p.bits_k == 3 ? quantize_qjl_rows_kernel<256, R, 3, 2>
+                                     : quantize_qjl_rows_kernel<256, R, 4, 2>);
+    // the largest shared-memory carveout: the CTAs per SM are then bounded by registers only
+    cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return (int)cudaLaunchKernelEx(&cfg, fn, p, c, kk, seq_idx, pos, rows);
   }
   cfg.gridDim = dim3((unsigned)rows, 1);  // y = 0: K only
   if (p.d == 64) return (int)cudaLaunchKernelEx(&cfg, quantize_row_kernel<64>, p, c, kk, kk, seq_idx, pos);
