@@ -127,12 +127,12 @@ int launch_quantize_tc(const DeviceParams &p, const tq_cache &c, const void *k, 
 int launch_quantize_tc256(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                           const int32_t *seq_idx, const int32_t *pos, int n_tok, bool include_k, bool include_v,
                           void *stream);
-// K rows only through the per-row kernel (batches of at most 1024 rows, or a
-// head dimension other than 128), the same index convention.
+// K rows only, the same index convention: the per-row kernel (batches of at
+// most 1024 rows), or at d = 256 with QJL the batched QJL kernel.
 int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void *k, const int32_t *seq_idx,
                            const int32_t *pos, int n_tok, void *stream);
-// K with QJL and V (MSE codes) on tcgen05 (d = 128), tiles of 128 rows, one
-// launch (tq_quantize_qjl_tc.cu).
+// K with QJL and V (MSE codes) on tcgen05 (d = 128 or 64), tiles of 128
+// rows, one launch (tq_quantize_qjl_tc.cu).
 int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void *k, const void *v,
                            const int32_t *seq_idx, const int32_t *pos, int n_tok, void *stream);
 

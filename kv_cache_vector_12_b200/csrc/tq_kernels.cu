@@ -1,8 +1,8 @@
 // TurboQuant quantize-on-append for sm_100a, small batches and QJL rows:
 // norm, rotation by Pi, Lloyd-Max codes, bit-pack, optional QJL residual
 // signs (one CTA per vector, or 32 vectors per CTA for batches of K rows with
-// QJL at head dimensions 64 and 256); and the dispatch between these kernels
-// and the tensor-core kernels.
+// QJL at head dimension 256); and the dispatch between these kernels and the
+// tensor-core kernels.
 //
 // The method: ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み"
 // (rotation + per-coordinate Lloyd-Max, then the 1-bit QJL residual
@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 }
 
 // ---------------------------------------------------------------------------
-// K rows with QJL in batches, head dimension 64 or 256 (d = 128 batches run on
-// the tcgen05 QJL kernel): the per-row kernel's arithmetic for R vectors per
+// K rows with QJL in batches at head dimension 256 (d = 64 and 128 batches run
+// on the tcgen05 QJL kernel): the per-row kernel's arithmetic for R vectors per
 // CTA.  Thread t owns coordinates t + h d / C (h < C) of all R vectors, so each
 // row of Pi and of S is read once per R vectors (the per-row kernel reads all
 // of S, d x d fp32, for every vector), and every broadcast shared-memory load
@@ -394,9 +394,11 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
   const uint16_t *kk = (const uint16_t *)k, *vv = (const uint16_t *)v;
   if (p.d != kHeadDim) {
     // other head dimensions: the per-row kernel for small batches, else the
-    // tcgen05 kernels (tq_quantize_tc256.cu for d = 256, tq_quantize_tc.cu
-    // for d = 64) for V and for K without QJL (K with QJL keeps the per-row
-    // kernel: the QJL kernel is specialised for d = 128)
+    // tcgen05 kernels: at d = 64 the MSE kernel (tq_quantize_tc.cu) or, with
+    // QJL, the QJL kernel (tq_quantize_qjl_tc.cu), both templated on d; at
+    // d = 256 the MSE kernel of tq_quantize_tc256.cu for V and for K without
+    // QJL, and the batched QJL kernel above for K with QJL (Pi, S hi and S lo
+    // at d = 256 do not fit in shared memory beside a tile ring)
     if (rows <= kRowKernelMaxRows) {
       cfg.gridDim = dim3((unsigned)rows, 2);
       cfg.blockDim = dim3(p.d);
@@ -408,9 +410,8 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
       if (e != 0 || !p.qjl) return e;
       return launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream);
     }
-    const int e = launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, !p.qjl, true, stream);
-    if (e != 0 || !p.qjl) return e;
-    return launch_quantize_rows_k(p, c, k, seq_idx, pos, n_tok, stream);
+    if (p.qjl) return launch_quantize_qjl_tc(p, c, k, v, seq_idx, pos, n_tok, stream);
+    return launch_quantize_tc(p, c, k, v, seq_idx, pos, n_tok, true, true, stream);
   }
   if (rows <= kRowKernelMaxRows) {
     cfg.gridDim = dim3((unsigned)rows, 2);
@@ -432,18 +433,14 @@ int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void 
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k;
-  if (p.d != kHeadDim && p.qjl) {  // R = 32 vectors per CTA; two coordinates per thread at d = 256
+  if (p.d == 256 && p.qjl) {  // R = 32 vectors per CTA, two coordinates per thread
     constexpr int R = 32;
     cfg.gridDim = dim3((unsigned)((rows + R - 1) / R));
-    cfg.blockDim = dim3(p.d == 64 ? 64 : 128);
+    cfg.blockDim = dim3(128);
     using QjlRowsFn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, long);
-    const QjlRowsFn fn =
-        p.d == 64 ? (p.bits_k == 2   ? quantize_qjl_rows_kernel<64, R, 2, 1>
-                     : p.bits_k == 3 ? quantize_qjl_rows_kernel<64, R, 3, 1>
-                                     : quantize_qjl_rows_kernel<64, R, 4, 1>)
-                  : (p.bits_k == 2   ? quantize_qjl_rows_kernel<256, R, 2, 2>
-                     : p.bits_k == 3 ? quantize_qjl_rows_kernel<256, R, 3, 2>
-                                     : quantize_qjl_rows_kernel<256, R, 4, 2>);
+    const QjlRowsFn fn = p.bits_k == 2   ? quantize_qjl_rows_kernel<256, R, 2, 2>
+                         : p.bits_k == 3 ? quantize_qjl_rows_kernel<256, R, 3, 2>
+                                         : quantize_qjl_rows_kernel<256, R, 4, 2>;
     // the largest shared-memory carveout: the CTAs per SM are then bounded by registers only
     cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     return (int)cudaLaunchKernelEx(&cfg, fn, p, c, kk, seq_idx, pos, rows);

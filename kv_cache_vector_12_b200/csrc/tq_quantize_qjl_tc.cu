@@ -8,10 +8,11 @@
 // each K vector (y = Pi x / ||x||) is projected by a Gaussian matrix S, and
 // only the signs of S r are kept, with ||r||.
 //
-// Per tile of 128 rows, on tcgen05 with fp32 accumulators in tensor memory:
+// Head dimension d = 128 or 64 (a template parameter W).  Per tile of 128
+// rows, on tcgen05 with fp32 accumulators in tensor memory:
 //   MMA 1   Z = X Pi^T: X by TMA (128-byte swizzle) from a 3-deep ring, Pi
 //           resident in shared memory (bf16, exact products).
-//   epilogue A (two threads per row, 64 coordinates each): ||x|| from the
+//   epilogue A (two threads per row, d / 2 coordinates each): ||x|| from the
 //           shared-memory tile, z from tensor memory, the codes against the
 //           thresholds scaled by ||x|| (the exact saturating-FMA search of
 //           the MSE kernel); for K also the residual r 2^14 = y 2^14 -
@@ -30,7 +31,7 @@
 //           K the sign bits and fp16 ||r||.
 // The K tiles come first in the tile order and the cheaper V tiles fill the
 // tail.  Two tile groups (each two warpgroups, one per half row) take
-// alternate tiles with 256 columns of tensor memory each (Z / R, then S r),
+// alternate tiles with 2 d columns of tensor memory each (Z / R, then S r),
 // so one group's MMAs run while the other computes.  One thread issues both
 // GEMMs, polling the barriers of both stages.  Every wait is bounded; on
 // expiry the kernel flags the error and stops, after waiting (bounded) for
@@ -48,19 +49,30 @@ namespace {
 constexpr int kJStages = 3;                          // X ring depth
 constexpr int kJGroups = 2;                          // tile groups (two warpgroups each)
 constexpr int kJThreads = 32 * (2 + 8 * kJGroups);   // producer, MMA issuer, epilogue
-constexpr unsigned kJTmemCols = 512;                 // per group: Z / R (128 columns), S r (128)
-constexpr int kJSmem = 1024 + kTileBytes * (3 + kJStages);  // Pi, S hi, S lo, the ring
 constexpr float kRScale = 0x1p14f;  // |r| < 1.3: r 2^14 stays below fp16's largest finite value
 
-// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both
-// K-major, N = 128, M = 128.
-constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// The shapes that depend on the head dimension W: an X tile is W / 64 boxes
+// of 128 rows x 64 coordinates; Pi, S hi and S lo are W / 64 boxes of W rows.
+template <int W>
+struct JShape {
+  static constexpr int boxes = W / 64;
+  static constexpr int tile_bytes = kTileRows * W * 2;
+  static constexpr int mat_bytes = W * W * 2;
+  static constexpr int mat_box = W * 128;
+  static constexpr unsigned tmem_cols = kJGroups * 2 * W;  // per group: Z / R (W columns), S r (W)
+  static constexpr int smem = 1024 + 3 * mat_bytes + kJStages * tile_bytes;  // Pi, S hi, S lo, the ring
+  // instruction descriptors, kind::f16, fp32 accumulator, K-major, M = 128,
+  // N = W: bf16 A and B (MMA 1), fp16 A and B (MMA 2)
+  static constexpr uint32_t idesc_bf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(W >> 3) << 17) | ((128u >> 4) << 24);
+  static constexpr uint32_t idesc_f16 = (1u << 4) | ((uint32_t)(W >> 3) << 17) | ((128u >> 4) << 24);
+};
 
 // D (tensor memory) += A (tensor memory) B (shared-memory descriptor).
-__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
                    tmem_d),
-               "r"(tmem_a), "l"(b), "r"(kIdescF16), "r"(accumulate)
+               "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
                : "memory");
 }
 
@@ -224,6 +236,27 @@ __device__ __forceinline__ void code_chunk_off(int c, const float (&off)[16], ui
   }
 }
 
+// The code words of a half row (W/2 coordinates: W/64 groups of 32, B words
+// each) at dst: 16-byte stores for W = 128 where B is even, else 8- or
+// 4-byte stores (the half row starts on a multiple of 4 B bytes).
+template <int W, int B>
+__device__ __forceinline__ void store_half_codes(unsigned char *dst, const uint32_t (&words)[4 * B]) {
+  if constexpr (W == 128 && B != 3) {
+#pragma unroll
+    for (int q = 0; q < B / 2; ++q)
+      reinterpret_cast<uint4 *>(dst)[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+  } else if constexpr (W == 128) {
+#pragma unroll
+    for (int q = 0; q < 3; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
+  } else if constexpr (B != 3) {
+#pragma unroll
+    for (int q = 0; q < B / 2; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 3; ++q) reinterpret_cast<uint32_t *>(dst)[q] = words[q];
+  }
+}
+
 // x0, x1 as two fp16 pairs hi + lo (x0 in the low halves): hi = fp16(x),
 // lo = fp16(x - hi).
 __device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -236,17 +269,18 @@ __device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, ui
 
 // 18 warps: one of the four schedulers holds five, whose registers (at most
 // 16384 per scheduler) cap a thread at 96
-template <int BK, int BV>
+template <int W, int BK, int BV>
 __global__ void __launch_bounds__(kJThreads, 1)
     quantize_qjl_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                            const __grid_constant__ CUtensorMap map_pi, const __grid_constant__ CUtensorMap map_s,
                            const QjlTcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char *pi_tile = smem;                  // Pi, bf16
-  unsigned char *s_hi = smem + kTileBytes;        // S 2^sigma, fp16 high parts
-  unsigned char *s_lo = smem + 2 * kTileBytes;    // and low parts
-  unsigned char *ring = smem + 3 * kTileBytes;
+  using Sh = JShape<W>;
+  unsigned char *pi_tile = smem;                     // Pi, bf16
+  unsigned char *s_hi = smem + Sh::mat_bytes;        // S 2^sigma, fp16 high parts
+  unsigned char *s_lo = smem + 2 * Sh::mat_bytes;    // and low parts
+  unsigned char *ring = smem + 3 * Sh::mat_bytes;
   __shared__ __align__(8) uint64_t full_bar[kJStages], empty_bar[kJStages];
   __shared__ __align__(8) uint64_t zfull[kJGroups], rfull[kJGroups], sfull[kJGroups], tfree[kJGroups];
   __shared__ __align__(8) uint64_t rr_bar[kJGroups];  // both halves' ||r||^2 written
@@ -285,7 +319,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
   }
   if (warp == 1) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_base_slot)),
-                 "r"(kJTmemCols)
+                 "r"(Sh::tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -295,13 +329,13 @@ __global__ void __launch_bounds__(kJThreads, 1)
   const uint32_t tmem_base = tmem_base_slot;
   if (warp == 0 && lane == 0) {  // Pi and S belong to the context: no earlier kernel writes them
     const uint32_t cb = smem_addr(&const_bar);
-    bar_expect_tx(cb, 3 * kTileBytes);
-    tma_load_2d(smem_addr(pi_tile), &map_pi, 0, 0, cb);
-    tma_load_2d(smem_addr(pi_tile + kBoxBytes), &map_pi, 64, 0, cb);
-    tma_load_2d(smem_addr(s_hi), &map_s, 0, 0, cb);
-    tma_load_2d(smem_addr(s_hi + kBoxBytes), &map_s, 64, 0, cb);
-    tma_load_2d(smem_addr(s_lo), &map_s, 0, 128, cb);
-    tma_load_2d(smem_addr(s_lo + kBoxBytes), &map_s, 64, 128, cb);
+    bar_expect_tx(cb, 3 * Sh::mat_bytes);
+#pragma unroll
+    for (int b = 0; b < Sh::boxes; ++b) {
+      tma_load_2d(smem_addr(pi_tile + b * Sh::mat_box), &map_pi, 64 * b, 0, cb);
+      tma_load_2d(smem_addr(s_hi + b * Sh::mat_box), &map_s, 64 * b, 0, cb);  // S rows 0 .. W - 1: hi
+      tma_load_2d(smem_addr(s_lo + b * Sh::mat_box), &map_s, 64 * b, W, cb);  // rows W .. 2 W - 1: lo
+    }
   }
   // launched as a programmatic dependent: inputs and the cache are touched
   // only once the previous kernel in the stream has completed
@@ -324,10 +358,10 @@ __global__ void __launch_bounds__(kJThreads, 1)
         const int row0 = tile_row0(i);
         const CUtensorMap *map = is_k ? &map_k : &map_v;
         const uint32_t fb = smem_addr(&full_bar[slot]);
-        unsigned char *st = ring + slot * kTileBytes;
-        bar_expect_tx(fb, kTileBytes);
-        tma_load_2d(smem_addr(st), map, 0, row0, fb);
-        tma_load_2d(smem_addr(st + kBoxBytes), map, 64, row0, fb);
+        unsigned char *st = ring + slot * Sh::tile_bytes;
+        bar_expect_tx(fb, Sh::tile_bytes);
+#pragma unroll
+        for (int b = 0; b < Sh::boxes; ++b) tma_load_2d(smem_addr(st + b * kBoxBytes), map, 64 * b, row0, fb);
         issued = i + 1;
       }
       bar_wait(smem_addr(&const_bar), 0);
@@ -351,12 +385,12 @@ __global__ void __launch_bounds__(kJThreads, 1)
           if (bar_test(smem_addr(&full_bar[slot]), (n1 / kJStages) & 1) &&
               (n1 < kJGroups || bar_test(smem_addr(&tfree[g]), ((n1 / kJGroups) - 1) & 1))) {
             tc_fence_after();
-            const uint32_t a0 = smem_addr(ring + slot * kTileBytes), b0 = smem_addr(pi_tile);
-            const uint32_t d = tmem_base + g * 256;
+            const uint32_t a0 = smem_addr(ring + slot * Sh::tile_bytes), b0 = smem_addr(pi_tile);
+            const uint32_t d = tmem_base + g * 2 * W;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;  // 16 elements along K per MMA
-              tc_mma(d, sw128_desc(a0 + off), sw128_desc(b0 + off), kk > 0);
+            for (int kk = 0; kk < W / 16; ++kk) {  // 16 elements along K per MMA
+              const uint32_t ao = (kk >> 2) * kBoxBytes + (kk & 3) * 32, bo = (kk >> 2) * Sh::mat_box + (kk & 3) * 32;
+              tc_mma_n(d, sw128_desc(a0 + ao), sw128_desc(b0 + bo), Sh::idesc_bf16, kk > 0);
             }
             tc_commit(smem_addr(&zfull[g]));
             tc_commit(smem_addr(&empty_bar[slot]));
@@ -368,14 +402,14 @@ __global__ void __launch_bounds__(kJThreads, 1)
           const int g = n2 % kJGroups;
           if (bar_test(smem_addr(&rfull[g]), (n2 / kJGroups) & 1)) {
             tc_fence_after();
-            const uint32_t ra = tmem_base + g * 256, d = ra + 128;
+            const uint32_t ra = tmem_base + g * 2 * W, d = ra + W;
             const uint32_t bh = smem_addr(s_hi), bl = smem_addr(s_lo);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-              tc_mma_ts(d, ra + 16 * kk, sw128_desc(bh + off), kk > 0);    // R_hi S_hi^T
-              tc_mma_ts(d, ra + 16 * kk, sw128_desc(bl + off), 1);         // R_hi S_lo^T
-              tc_mma_ts(d, ra + 16 * kk + 8, sw128_desc(bh + off), 1);     // R_lo S_hi^T
+            for (int kk = 0; kk < W / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * Sh::mat_box + (kk & 3) * 32;
+              tc_mma_ts(d, ra + 16 * kk, sw128_desc(bh + off), Sh::idesc_f16, kk > 0);  // R_hi S_hi^T
+              tc_mma_ts(d, ra + 16 * kk, sw128_desc(bl + off), Sh::idesc_f16, 1);       // R_hi S_lo^T
+              tc_mma_ts(d, ra + 16 * kk + 8, sw128_desc(bh + off), Sh::idesc_f16, 1);   // R_lo S_hi^T
             }
             tc_commit(smem_addr(&sfull[g]));
             ++n2;
@@ -396,12 +430,12 @@ __global__ void __launch_bounds__(kJThreads, 1)
         if (ok && i >= kJGroups) ok = bar_wait(smem_addr(&tfree[g]), ((i / kJGroups) - 1) & 1);
         if (!ok || *(volatile int *)&abort_flag) break;
         tc_fence_after();
-        const uint32_t a0 = smem_addr(ring + slot * kTileBytes), b0 = smem_addr(pi_tile);
-        const uint32_t d = tmem_base + g * 256;
+        const uint32_t a0 = smem_addr(ring + slot * Sh::tile_bytes), b0 = smem_addr(pi_tile);
+        const uint32_t d = tmem_base + g * 2 * W;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          tc_mma(d, sw128_desc(a0 + off), sw128_desc(b0 + off), kk > 0);
+        for (int kk = 0; kk < W / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * kBoxBytes + (kk & 3) * 32, bo = (kk >> 2) * Sh::mat_box + (kk & 3) * 32;
+          tc_mma_n(d, sw128_desc(a0 + ao), sw128_desc(b0 + bo), Sh::idesc_bf16, kk > 0);
         }
         tc_commit(smem_addr(&zfull[g]));
         tc_commit(smem_addr(&empty_bar[slot]));
@@ -416,7 +450,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
     }
   } else {
     // ------------------------------------------------ epilogue: tile group g,
-    // half h of every row (coordinates and projections 64 h .. 64 h + 63)
+    // half h of every row (coordinates and projections W/2 h .. W/2 h + W/2 - 1)
     const int g = (warp - 2) / 8, h = ((warp - 2) / 4) & 1;
     const int quarter = warp & 3;       // TMEM lanes 32 quarter .. + 31
     const int r = 32 * quarter + lane;  // the row this thread shares
@@ -431,7 +465,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
     for (int j = 0; j < hv - 1; ++j) kv.nt[j] = -a.p.cb[3 * kMaxLevels + hv + j] * 0x1p64f;
     search_consts<BK>(kk);
     search_consts<BV>(kv);
-    const uint32_t tz = tmem_base + g * 256 + 64 * h + ((uint32_t)(32 * quarter) << 16);
+    const uint32_t tz = tmem_base + g * 2 * W + (W / 2) * h + ((uint32_t)(32 * quarter) << 16);
+    constexpr int kHalfChunks = W / 32;  // chunks of 16 coordinates per half row
 
     for (int j = 0, i = g; i < my_tiles; ++j, i += kJGroups) {
       const int slot = i % kJStages;
@@ -449,10 +484,10 @@ __global__ void __launch_bounds__(kJThreads, 1)
       }
       // ||x|| from the swizzled tile (chunk c of row r sits at c ^ (r % 8));
       // bf16 squares are exact in fp32.  Both halves read the whole row.
-      const unsigned char *st = ring + slot * kTileBytes;
+      const unsigned char *st = ring + slot * Sh::tile_bytes;
       float2 ss = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int box = 0; box < 2; ++box)
+      for (int box = 0; box < Sh::boxes; ++box)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 u =
@@ -488,7 +523,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
         uint32_t words[4 * BK];
         float2 rr = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kHalfChunks; ++c) {
           float z[16];
           tmem_ld16(tz + 16 * c, z);
           float off[16];
@@ -530,11 +565,11 @@ __global__ void __launch_bounds__(kJThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sb[2] = {0u, 0u};  // bit n of the row = [(S r)_n >= 0], LSB first, n = 64 h ..
+        uint32_t sb[2] = {0u, 0u};  // bit n of the row = [(S r)_n >= 0], LSB first, n = W/2 h ..
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kHalfChunks; ++c) {
           float v[16];
-          tmem_ld16(tz + 128 + 16 * c, v);
+          tmem_ld16(tz + W + 16 * c, v);
           uint32_t b = 0;
 #pragma unroll
           for (int e = 0; e < 16; ++e) b |= (v[e] >= 0.f ? 1u : 0u) << e;
@@ -545,17 +580,10 @@ __global__ void __launch_bounds__(kJThreads, 1)
         if (lane == 0) bar_arrive(smem_addr(&tfree[g]));
 
         if (slot_i >= 0) {
-          // code groups 2 h and 2 h + 1: 8 BK bytes from byte 8 BK h of the row
-          uint32_t *dst = reinterpret_cast<uint32_t *>(a.c.codes_k + slot_i * (long)(16 * BK) + 8 * BK * h);
-          if constexpr (BK == 3) {
-#pragma unroll
-            for (int q = 0; q < 3; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
-          } else {
-#pragma unroll
-            for (int q = 0; q < BK / 2; ++q)
-              reinterpret_cast<uint4 *>(dst)[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-          }
-          reinterpret_cast<uint2 *>(a.c.qjl_bits + slot_i * 16)[h] = make_uint2(sb[0], sb[1]);
+          // the half row's code groups: W/16 BK bytes from byte W/16 BK h of the row
+          store_half_codes<W, BK>(a.c.codes_k + slot_i * (long)(W / 8 * BK) + W / 16 * BK * h, words);
+          if constexpr (W == 128) reinterpret_cast<uint2 *>(a.c.qjl_bits + slot_i * 16)[h] = make_uint2(sb[0], sb[1]);
+          else reinterpret_cast<uint32_t *>(a.c.qjl_bits + slot_i * (W / 8))[h] = sb[0];
           if (h == 0) {
             a.c.norm_k[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
             const float gamma = sqrtf(rr_row) * (1.f / kRScale);
@@ -568,7 +596,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
         kv.zc = live ? 0x1p127f : 0.f;
         uint32_t words[4 * BV];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kHalfChunks; ++c) {
           float z[16];
           tmem_ld16(tz + 16 * c, z);
           code_chunk<BV>(c, z, kv, words);
@@ -577,15 +605,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
         __syncwarp();
         if (lane == 0) bar_arrive(smem_addr(&tfree[g]));
         if (slot_i >= 0) {
-          uint32_t *dst = reinterpret_cast<uint32_t *>(a.c.codes_v + slot_i * (long)(16 * BV) + 8 * BV * h);
-          if constexpr (BV == 3) {
-#pragma unroll
-            for (int q = 0; q < 3; ++q) reinterpret_cast<uint2 *>(dst)[q] = make_uint2(words[2 * q], words[2 * q + 1]);
-          } else {
-#pragma unroll
-            for (int q = 0; q < BV / 2; ++q)
-              reinterpret_cast<uint4 *>(dst)[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-          }
+          store_half_codes<W, BV>(a.c.codes_v + slot_i * (long)(W / 8 * BV) + W / 16 * BV * h, words);
           if (h == 0) a.c.norm_v[slot_i] = __half_as_ushort(__float2half_rn(fminf(nrm, 65504.f)));
         }
       }
@@ -598,7 +618,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kJTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Sh::tmem_cols)
                  : "memory");
   }
 }
@@ -606,9 +626,15 @@ __global__ void __launch_bounds__(kJThreads, 1)
 using QjlTcFn = void (*)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
                          const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap, const QjlTcArgs);
 
-template <int BK>
+template <int W, int BK>
 QjlTcFn pick_bv(int bv) {
-  return bv == 2 ? quantize_qjl_tc_kernel<BK, 2> : bv == 3 ? quantize_qjl_tc_kernel<BK, 3> : quantize_qjl_tc_kernel<BK, 4>;
+  return bv == 2 ? quantize_qjl_tc_kernel<W, BK, 2> : bv == 3 ? quantize_qjl_tc_kernel<W, BK, 3>
+                                                               : quantize_qjl_tc_kernel<W, BK, 4>;
+}
+
+template <int W>
+QjlTcFn pick(int bk, int bv) {
+  return bk == 2 ? pick_bv<W, 2>(bv) : bk == 3 ? pick_bv<W, 3>(bv) : pick_bv<W, 4>(bv);
 }
 
 }  // namespace
@@ -618,24 +644,29 @@ int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void 
   // cached per device (the attribute applies to the current device), and
   // atomically, as calls may come from several threads
   static std::atomic<int> cached_sm[kMaxDevices];
-  static std::atomic<bool> configured[kMaxDevices][3][3];
+  if (p.d != 64 && p.d != kHeadDim) return (int)cudaErrorInvalidValue;
+  const int W = p.d;
+  static std::atomic<bool> configured[kMaxDevices][2][3][3];
   const int dev = current_device();
   int n_sm = cached_sm[dev].load(std::memory_order_relaxed);
   if (n_sm == 0) {
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
     cached_sm[dev].store(n_sm, std::memory_order_relaxed);
   }
-  const QjlTcFn fn = p.bits_k == 2 ? pick_bv<2>(p.bits_v) : p.bits_k == 3 ? pick_bv<3>(p.bits_v) : pick_bv<4>(p.bits_v);
-  std::atomic<bool> &done = configured[dev][p.bits_k - 2][p.bits_v - 2];
+  const QjlTcFn fn = W == 64 ? pick<64>(p.bits_k, p.bits_v) : pick<kHeadDim>(p.bits_k, p.bits_v);
+  const int smem = W == 64 ? JShape<64>::smem : JShape<kHeadDim>::smem;
+  std::atomic<bool> &done = configured[dev][W == 64 ? 0 : 1][p.bits_k - 2][p.bits_v - 2];
   if (!done.load(std::memory_order_acquire)) {
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kJSmem);
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return (int)e;
     done.store(true, std::memory_order_release);
   }
   const long rows = (long)n_tok * c.n_kv_heads;
   CUtensorMap mk, mv, mp, ms;
-  if (!make_row_map(&mk, k, rows) || !make_row_map(&mv, v, rows) || !make_row_map(&mp, p.pi, kHeadDim) ||
-      !make_row_map(&ms, p.ssplit, 2 * kHeadDim, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+  const CUtensorMapDataType bf16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_row_map(&mk, k, rows, bf16, W) || !make_row_map(&mv, v, rows, bf16, W) ||
+      !make_row_map(&mp, p.pi, W, bf16, W, W) ||
+      !make_row_map(&ms, p.ssplit, 2 * W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, W))
     return (int)cudaErrorInvalidValue;
   QjlTcArgs args{p, c, seq_idx, pos, (int)rows, (int)((rows + kTileRows - 1) / kTileRows)};
   const int n_tiles = 2 * args.tiles_k;
@@ -646,7 +677,7 @@ int launch_quantize_qjl_tc(const DeviceParams &p, const tq_cache &c, const void 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kJThreads);
-  cfg.dynamicSmemBytes = kJSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = (cudaStream_t)stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;

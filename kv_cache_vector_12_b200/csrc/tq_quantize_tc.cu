@@ -51,12 +51,6 @@ struct TcShape {
   static constexpr int smem = 1024 + pi_bytes + kRingStages * tile_bytes;
 };
 
-__device__ __forceinline__ void tc_mma_n(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
-  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-                   tmem_d),
-               "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-               : "memory");
-}
 
 struct QuantTcArgs {
   DeviceParams p;

@@ -85,6 +85,13 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
                "l"(a), "l"(b), "r"(kInstrDesc), "r"(accumulate)
                : "memory");
 }
+// The same with the instruction descriptor as an argument (other N).
+__device__ __forceinline__ void tc_mma_n(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                   tmem_d),
+               "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
