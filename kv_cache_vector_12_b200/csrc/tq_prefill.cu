@@ -665,7 +665,9 @@ int smem_of(int bk, int bv, bool qjl) {
 // At the end o = Pi^T (O / l) is one more pair of MMAs (O as bf16 hi + lo,
 // Pi^T's rows in the V fragment order as the B operand), and the lse.
 // Tensor memory: S at columns 0-127, O at 128-255, q_hat hi and lo at
-// 256-319 and 320-383, P' at 384-447.  Every mbarrier wait is bounded.
+// 256-319 and 320-383, P' at 384-447 and 448-511 (tiles alternate, so the
+// softmax of a tile does not wait for the previous tile's value MMAs unless
+// it rescales O).  Every mbarrier wait is bounded.
 // ===========================================================================
 namespace tq {
 namespace {
@@ -894,7 +896,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
-  __shared__ __align__(8) uint64_t kv_full[2], kv_empty[2], s_full, s_empty, p_full, pv_done;
+  __shared__ __align__(8) uint64_t kv_full[2], kv_empty[2], s_full, s_empty, p_full, pv_done[2];
   __shared__ __align__(8) uint64_t q_ready, scratch_done, scratch_free, o_ready, fin_bar, mma_done;
   __shared__ __align__(8) uint64_t mx_bar[2], l_bar;
   __shared__ float s_max[2][2][kTcRows], s_l[2][kTcRows];  // the half rows' maxima (by tile parity) and sums
@@ -940,7 +942,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     mbar_init(smem_u32(&s_full), 1);
     mbar_init(smem_u32(&s_empty), 8);  // the eight softmax warps
     mbar_init(smem_u32(&p_full), 8);
-    mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&pv_done[0]), 1);
+    mbar_init(smem_u32(&pv_done[1]), 1);
     mbar_init(smem_u32(&q_ready), 8);
     mbar_init(smem_u32(&scratch_done), 8);
     mbar_init(smem_u32(&scratch_free), 8);
@@ -1042,9 +1045,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kOpBox + (kk & 3) * 32;
-          tcx_mma_ts(t_o, t_p + 8 * kk, swdesc(bv + off), (it > 0 || kk > 0) ? 1u : 0u);
+          tcx_mma_ts(t_o, t_p + 64 * (it & 1) + 8 * kk, swdesc(bv + off), (it > 0 || kk > 0) ? 1u : 0u);
         }
-        tcx_commit(smem_u32(&pv_done));
+        tcx_commit(smem_u32(&pv_done[it & 1]));
         tcx_commit(smem_u32(&kv_empty[it & 1]));
       }
       // o = Pi^T (O / l): A = O as bf16 hi + lo (over K~ 0 and 1), B = Pi^T's
@@ -1248,14 +1251,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       const float ref = fmaxf(mn, -3.0e38f);
       const float al = fast_exp2(m_run - ref);
       m_run = mn;
-      // the previous tile's value MMAs read P' and write O (issued after this
-      // tile's scores, so usually finished by now): wait for them, rescale
-      // this half of O on a moved maximum, then write this half of P'
+      // P' is double-buffered in tensor memory: this tile's buffer was last
+      // read by the value MMAs of tile it - 2, while those of tile it - 1 may
+      // still be accumulating into O.  A moved maximum in the warp's rows
+      // waits for tile it - 1 and rescales this half of O; otherwise only
+      // tile it - 2 is waited for.  (Waiting on every tile's barrier phase
+      // in turn, at most one phase apart, keeps the parity waits exact.)
       if (it > 0) {
-        ok = tc_wait(&pv_done, (it - 1) & 1, err, abf);
+        const bool rescale = __any_sync(0xffffffffu, al != 1.f);
+        if (rescale) ok = tc_wait(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, err, abf);
+        else if (it >= 2) ok = tc_wait(&pv_done[it & 1], ((it - 2) >> 1) & 1, err, abf);
         if (!ok) break;
         tcx_fence_after();
-        if (__any_sync(0xffffffffu, al != 1.f)) {
+        if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t v[16];
@@ -1296,7 +1304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
             pk[2 * j4 + e] = pack_half2(pv.x, pv.y);
           }
         }
-        tmem_st16x(t_p + 16 * c, pk);
+        tmem_st16x(t_p + 64 * (it & 1) + 16 * c, pk);
       }
       l_run = fmaf(l_run, al, ls2.x + ls2.y);
       tmem_wait_st();
@@ -1305,7 +1313,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       if (lane == 0) mbar_arrive(smem_u32(&p_full));
     }
     // ---------------- o = Pi^T (O / l)
-    if (ok) ok = tc_wait(&pv_done, (n_tiles - 1) & 1, err, abf);
+    if (ok) ok = tc_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, err, abf);
     if (ok) {
       s_l[h2][row] = l_run;
       __syncwarp();
