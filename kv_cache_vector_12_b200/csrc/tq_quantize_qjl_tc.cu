@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
   __shared__ __align__(8) uint64_t full_bar[kJStages], empty_bar[kJStages];
   __shared__ __align__(8) uint64_t zfull[kJGroups], rfull[kJGroups], sfull[kJGroups], tfree[kJGroups];
   __shared__ __align__(8) uint64_t rr_bar[kJGroups];  // both halves' ||r||^2 written
-  __shared__ __align__(8) uint64_t const_bar, mma_done;
+  __shared__ __align__(8) uint64_t const_bar, s_bar, mma_done;  // Pi; S hi and lo
   __shared__ float s_rr[kJGroups][2][2][kTileRows];  // ||r||^2 of each half row, by tile parity
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
@@ -313,6 +313,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
       bar_init(smem_addr(&rr_bar[g]), 8);
     }
     bar_init(smem_addr(&const_bar), 1);
+    bar_init(smem_addr(&s_bar), 1);
     bar_init(smem_addr(&mma_done), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -329,13 +330,9 @@ __global__ void __launch_bounds__(kJThreads, 1)
   const uint32_t tmem_base = tmem_base_slot;
   if (warp == 0 && lane == 0) {  // Pi and S belong to the context: no earlier kernel writes them
     const uint32_t cb = smem_addr(&const_bar);
-    bar_expect_tx(cb, 3 * Sh::mat_bytes);
+    bar_expect_tx(cb, Sh::mat_bytes);
 #pragma unroll
-    for (int b = 0; b < Sh::boxes; ++b) {
-      tma_load_2d(smem_addr(pi_tile + b * Sh::mat_box), &map_pi, 64 * b, 0, cb);
-      tma_load_2d(smem_addr(s_hi + b * Sh::mat_box), &map_s, 64 * b, 0, cb);  // S rows 0 .. W - 1: hi
-      tma_load_2d(smem_addr(s_lo + b * Sh::mat_box), &map_s, 64 * b, W, cb);  // rows W .. 2 W - 1: lo
-    }
+    for (int b = 0; b < Sh::boxes; ++b) tma_load_2d(smem_addr(pi_tile + b * Sh::mat_box), &map_pi, 64 * b, 0, cb);
   }
   // launched as a programmatic dependent: inputs and the cache are touched
   // only once the previous kernel in the stream has completed
@@ -345,6 +342,17 @@ __global__ void __launch_bounds__(kJThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ producer (TMA)
     if (lane == 0) {
+      bool s_issued = false;
+      auto load_s = [&]() {  // S belongs to the context: no earlier kernel writes it
+        s_issued = true;
+        const uint32_t sb = smem_addr(&s_bar);
+        bar_expect_tx(sb, 2 * Sh::mat_bytes);
+#pragma unroll
+        for (int b = 0; b < Sh::boxes; ++b) {
+          tma_load_2d(smem_addr(s_hi + b * Sh::mat_box), &map_s, 64 * b, 0, sb);  // S rows 0 .. W - 1: hi
+          tma_load_2d(smem_addr(s_lo + b * Sh::mat_box), &map_s, 64 * b, W, sb);  // rows W .. 2 W - 1: lo
+        }
+      };
       int issued = 0;
       for (int i = 0; i < my_tiles; ++i) {
         const int slot = i % kJStages;
@@ -363,8 +371,13 @@ __global__ void __launch_bounds__(kJThreads, 1)
 #pragma unroll
         for (int b = 0; b < Sh::boxes; ++b) tma_load_2d(smem_addr(st + b * kBoxBytes), map, 64 * b, row0, fb);
         issued = i + 1;
+        // S (hi, lo) is needed only by the second GEMM of the first K tile:
+        // its copies queue behind the ring's first tiles
+        if (i == min(kJStages, my_tiles) - 1) load_s();
       }
+      if (!s_issued) load_s();  // (stopped early: S is still copied, and waited for below)
       bar_wait(smem_addr(&const_bar), 0);
+      bar_wait(smem_addr(&s_bar), 0);
       if (*(volatile int *)&abort_flag)  // drain: never leave copies in flight
         for (int k = (issued > kJStages ? issued - kJStages : 0); k < issued; ++k)
           bar_wait(smem_addr(&full_bar[k % kJStages]), (k / kJStages) & 1);
@@ -376,6 +389,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
     if (lane == 0) {
       bool ok = bar_wait(smem_addr(&const_bar), 0);
       int n1 = 0, n2 = 0;
+      bool s_ready = false;  // S hi and lo have landed (the second GEMM)
       unsigned long long t_last = global_ns();
       while (ok && n2 < my_k) {
         if (*(volatile int *)&abort_flag) break;
@@ -400,7 +414,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
         }
         if (n2 < n1) {
           const int g = n2 % kJGroups;
-          if (bar_test(smem_addr(&rfull[g]), (n2 / kJGroups) & 1)) {
+          if (!s_ready) s_ready = bar_test(smem_addr(&s_bar), 0);
+          if (s_ready && bar_test(smem_addr(&rfull[g]), (n2 / kJGroups) & 1)) {
             tc_fence_after();
             const uint32_t ra = tmem_base + g * 2 * W, d = ra + W;
             const uint32_t bh = smem_addr(s_hi), bl = smem_addr(s_lo);
