@@ -353,7 +353,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
     delete ctx;
     return fail(TQ_ERR_UNSUPPORTED, "internal: fragment orders or codebook tables could not be built");
   }
-  // One block: pi | pik | pivt | pif | pvf | s | sjk | sf | ssplit | codebooks | kperm | jperm | error word.
+  // One block: pi | pik | pivt | pif | pvf | s | sjkf | sf | ssplit | codebooks | kperm | jperm | error word.
   const size_t dd = (size_t)d * d;
   const size_t off_pi = 0, off_pik = off_pi + dd * 2, off_piv = off_pik + dd * 2, off_pif = off_piv + dd * 2;
   const size_t off_pvf = off_pif + dd * 2, off_s = off_pvf + dd * 2;
@@ -380,9 +380,6 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   tq::mma_b_fragments(ctx->pi_bits.data(), d, (uint32_t *)(h.data() + off_pif));
   if (qjl) {
     std::memcpy(h.data() + off_s, ctx->s.data(), dd * 4);
-    float *sjk = (float *)(h.data() + off_sjk);
-    for (int i = 0; i < d; ++i)
-      for (int j = 0; j < d; ++j) sjk[(size_t)i * d + j] = ctx->s[(size_t)jperm[i] * d + kperm[j]];
     // S 2^sigma = hi + lo with two fp16 parts (22 significant bits; only the
     // signs of S r are kept, so the power-of-two scale is free).  sigma puts
     // the largest entry at or below 2^15: hi never overflows, and lo stays in
@@ -401,6 +398,18 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
       }
       tq::mma_b_fragments(part.data(), d, (uint32_t *)(h.data() + off_sf) + (size_t)k * dd / 2);
       std::memcpy(h.data() + off_ss + (size_t)k * dd * 2, part.data(), dd * 2);
+    }
+    // the same two parts with S's rows in the QJL fragment order and its
+    // columns in the K fragment order (S'[i][j] = S[jperm i][kperm j]), as
+    // fp16 MMA B fragments: the decode kernel's q_tilde = S' q_hat
+    std::vector<uint16_t> perm_part(dd);
+    for (size_t i = 0; i < dd; ++i) rest[i] = std::ldexp((double)ctx->s[(size_t)jperm[i / d] * d + kperm[i % d]], sigma);
+    for (int k = 0; k < 2; ++k) {
+      for (size_t i = 0; i < dd; ++i) {
+        perm_part[i] = tq::double_to_half_bits(rest[i]);
+        rest[i] -= tq::half_bits_to_double(perm_part[i]);
+      }
+      tq::mma_b_fragments(perm_part.data(), d, (uint32_t *)(h.data() + off_sjk) + (size_t)k * dd / 2);
     }
   }
   uint16_t *pivt = (uint16_t *)(h.data() + off_piv);
@@ -424,7 +433,7 @@ tq_status tq_create_ex(tq_ctx **out, int32_t d, int32_t bits_k, int32_t bits_v, 
   ctx->dp.pi = (const uint16_t *)(base + off_pi);
   ctx->dp.pikf = (const uint32_t *)(base + off_pik);
   ctx->dp.s = (const float *)(base + off_s);
-  ctx->dp.sjk = (const float *)(base + off_sjk);
+  ctx->dp.sjkf = (const uint32_t *)(base + off_sjk);
   ctx->dp.pif = (const uint32_t *)(base + off_pif);
   ctx->dp.sf = (const uint32_t *)(base + off_sf);
   ctx->dp.ssplit = (const uint16_t *)(base + off_ss);

@@ -419,13 +419,14 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         if constexpr (kRows > 8) s_red[warp][r + 8] = mx1;
       }
       consumer_sync();
-      float mu[2];
+      float mu[2], qmax[2] = {0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         if (kRows <= 8 && e == 1) break;
         const int row = r + 8 * e;
         const float m = fmaxf(fmaxf(s_red[0][row], s_red[1][row]), fmaxf(s_red[2][row], s_red[3][row]));
         mu[e] = m > 0.f ? 32767.f / m : 1.f;
+        qmax[e] = m;
       }
 #pragma unroll
       for (int nt = 0; nt < NTW; ++nt) {
@@ -445,29 +446,75 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         if constexpr (kRows > 8) s_qs[r + 8][0] = a.scale * kLog2e / (mu[1] * ldexpf(1.f, a.p.k_shift));
       }
       if constexpr (QJL) {
-        // q_tilde = S q_hat: positions tid (+ 128) (QJL fragment order) of
-        // every head, from rows of S permuted into the QJL (rows) and K
-        // (columns) orders
+        // q_tilde = S' q_hat (rows of S in the QJL fragment order, columns in
+        // the K order) on the tensor cores: q_hat, scaled per head by a power
+        // of two that puts max |q_hat| in [2^13, 2^14), and S' 2^sigma as fp16
+        // hi + lo parts (hi hi + hi lo + lo hi, about 22 significant bits,
+        // fp32 sums); warp w takes the output n-tiles w NTQ .. w NTQ + NTQ - 1
+        consumer_sync();  // q_hat is complete in s_qf
+        constexpr int NTQ = D / 32, CHQ = D / 32;  // n-tiles per warp; chunks of two k-steps
+        float sc[2];  // the power-of-two scales of rows r and r + 8
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          int ex = 0;
+          if (qmax[e] > 0.f) frexpf(qmax[e], &ex);
+          sc[e] = qmax[e] > 0.f ? ldexpf(1.f, 14 - ex) : 1.f;
+        }
+        float cq[NTQ][4];
+#pragma unroll
+        for (int nt = 0; nt < NTQ; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) cq[nt][e] = 0.f;
+        const uint4 *sjf = reinterpret_cast<const uint4 *>(a.p.sjkf);
+        constexpr int kPart = (D / 8) * CHQ * 32;  // uint4 per part
+#pragma unroll 1
+        for (int j = 0; j < CHQ; ++j) {
+          uint32_t ah[2][4], al[2][4];  // A fragments of k-steps 2 j, 2 j + 1
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int row = r + 8 * (e & 1), col = 16 * (2 * j + kk) + 8 * (e >> 1) + 2 * q;
+              if (row < kRows) {
+                const float f = sc[e & 1];
+                split_f16x2(s_qf[row][col] * f, s_qf[row][col + 1] * f, ah[kk][e], al[kk][e]);
+              } else {
+                ah[kk][e] = al[kk][e] = 0u;
+              }
+            }
+#pragma unroll
+          for (int nt = 0; nt < NTQ; ++nt) {
+            const int idx = ((warp * NTQ + nt) * CHQ + j) * 32 + lane;
+            const uint4 bh = sjf[idx], bl = sjf[kPart + idx];
+            mma_f16(cq[nt], ah[0][0], ah[0][1], ah[0][2], ah[0][3], bh.x, bh.y);
+            mma_f16(cq[nt], ah[0][0], ah[0][1], ah[0][2], ah[0][3], bl.x, bl.y);
+            mma_f16(cq[nt], al[0][0], al[0][1], al[0][2], al[0][3], bh.x, bh.y);
+            mma_f16(cq[nt], ah[1][0], ah[1][1], ah[1][2], ah[1][3], bh.z, bh.w);
+            mma_f16(cq[nt], ah[1][0], ah[1][1], ah[1][2], ah[1][3], bl.z, bl.w);
+            mma_f16(cq[nt], al[1][0], al[1][1], al[1][2], al[1][3], bh.z, bh.w);
+          }
+        }
+        consumer_sync();  // every warp has read q_hat: s_qf takes q_tilde
+#pragma unroll
+        for (int nt = 0; nt < NTQ; ++nt) {
+          const int pos = 8 * (warp * NTQ + nt) + 2 * q;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int row = r + 8 * e;
+            if (row < kRows) {
+              const float u = ldexpf(1.f, -a.p.s_shift) / sc[e];  // exact: powers of two
+              *reinterpret_cast<float2 *>(&s_qf[row][pos]) = make_float2(cq[nt][2 * e] * u, cq[nt][2 * e + 1] * u);
+            }
+          }
+        }
         consumer_sync();
         constexpr int PP = D >= 128 ? D / 128 : 1;  // positions per consumer thread
         float qt[PP][kRows];
 #pragma unroll
         for (int pp = 0; pp < PP; ++pp) {
-#pragma unroll
-          for (int g = 0; g < kRows; ++g) qt[pp][g] = 0.f;
           const int pos = tid + 128 * pp;
-          if (pos < D) {
-            const float4 *srow = reinterpret_cast<const float4 *>(a.p.sjk + pos * D);
-#pragma unroll 4
-            for (int c4 = 0; c4 < D / 4; ++c4) {
-              const float4 w4 = srow[c4];
 #pragma unroll
-              for (int g = 0; g < kRows; ++g) {
-                const float4 x = *reinterpret_cast<const float4 *>(&s_qf[g][4 * c4]);
-                qt[pp][g] = fmaf(w4.x, x.x, fmaf(w4.y, x.y, fmaf(w4.z, x.z, fmaf(w4.w, x.w, qt[pp][g]))));
-              }
-            }
-          }
+          for (int g = 0; g < kRows; ++g) qt[pp][g] = pos < D ? s_qf[g][pos] : 0.f;
         }
         // nu = 32767 / max |q_tilde| per head, then the ints and their sum
 #pragma unroll

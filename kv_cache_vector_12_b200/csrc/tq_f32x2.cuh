@@ -1,8 +1,9 @@
 // Packed fp32 arithmetic of sm_100: two fp32 lanes in one 64-bit register
 // pair, one instruction for both (round to nearest, like the scalar forms),
-// and the three-input maximum.
+// the three-input maximum, and the two-part fp16 split of fp32 pairs.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace tq {
@@ -35,6 +36,16 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
 }
+// x0, x1 as two fp16 pairs hi + lo (x0 in the low halves): hi = fp16(x),
+// lo = fp16(x - hi), about 22 significant bits together.
+__device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // max(a, b, c); a NaN operand is ignored, as by fmaxf
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;

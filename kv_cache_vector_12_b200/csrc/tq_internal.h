@@ -52,7 +52,8 @@ struct DeviceParams {
   const uint32_t *pikf;   // Pi with rows in K fragment order, as the decode kernel's bf16 MMA B fragments:
                           // [warp 4][n-tile 4][chunk 4][lane 32][4 words] (16-byte aligned; see tq_api.cu)
   const float *s;         // S   [d][d] fp32 (qjl only)
-  const float *sjk;       // [d][d] fp32: sjk[kappa][kappa'] = S[jperm[kappa]][kperm[kappa']] (qjl only)
+  const uint32_t *sjkf;   // S' 2^sigma, S'[kappa][kappa'] = S[jperm[kappa]][kperm[kappa']], split into two fp16
+                          // parts (hi + lo), each as fp16 MMA B fragments laid out like pif (qjl only)
   const uint32_t *pif;    // Pi (natural row order) as bf16 MMA B fragments [n-tile 16][chunk 4][lane 32][4 words]
   const uint32_t *sf;     // S 2^sigma split into two fp16 parts (hi + lo), each as B fragments like pif:
                           // [part 2][n-tile 16][chunk 4][lane 32][4 words] (qjl only; sigma chosen on the host)

@@ -72,14 +72,6 @@ constexpr int prefill_smem_bytes() {
   return ring > scratch ? ring : scratch;
 }
 
-// fp16 pair (lo, hi) of two fp32 values as one register.
-__device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const __half2 l = __floats2half2_rn(x0 - __low2float(h), x1 - __high2float(h));
-  hi = *reinterpret_cast<const uint32_t *>(&h);
-  lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
 template <int BK, int BV, bool QJL>
 __global__ void __launch_bounds__(kPThreads, 2) prefill_attn_kernel(const PrefillArgs a) {
   using St = Stage<BK, BV, QJL, kPStageTokens>;

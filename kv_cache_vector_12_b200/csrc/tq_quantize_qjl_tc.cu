@@ -257,16 +257,6 @@ __device__ __forceinline__ void store_half_codes(unsigned char *dst, const uint3
   }
 }
 
-// x0, x1 as two fp16 pairs hi + lo (x0 in the low halves): hi = fp16(x),
-// lo = fp16(x - hi).
-__device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const float2 hf = __half22float2(h);
-  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-  hi = *reinterpret_cast<const uint32_t *>(&h);
-  lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
 // 18 warps: one of the four schedulers holds five, whose registers (at most
 // 16384 per scheduler) cap a thread at 96
 template <int W, int BK, int BV>
