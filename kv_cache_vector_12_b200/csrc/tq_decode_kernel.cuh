@@ -195,7 +195,9 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
   __shared__ int abort_flag;
   __shared__ float sm_m[kConsumerWarps][kRows], sm_l[kConsumerWarps][kRows];
   __shared__ __align__(16) uint8_t s_q8[kRows][QJL ? 4 : 2][DH];  // q_hat hi, lo; q_tilde hi, lo (fragment orders)
-  __shared__ __align__(16) float s_qf[QJL ? kRows : 1][DH];       // q_hat, fp32, K order (QJL input)
+  // this KV head's query rows (fp32), read by the rotation; then (QJL) q_hat
+  // in the K order, written once every consumer warp is past the rotation
+  __shared__ __align__(16) float s_qf[kRows][DH];
   __shared__ float s_qs[kRows][4];                                // score factor, QJL factor, sum of q_tilde ints
   __shared__ float s_red[kConsumerWarps][kRows];
 
@@ -361,6 +363,44 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     {
       const long qrow0 = (long)s * a.n_q_heads + (long)h * G;
       const bool f32 = a.q_dtype == TQ_F32;
+      // the G query rows (contiguous, 16-byte aligned) into shared memory,
+      // every load issued before any is used: one memory round trip for
+      // the prologue instead of one per k-step
+      {
+        constexpr int kMaxIt = (kRows * D / 4 + 32 * kConsumerWarps - 1) / (32 * kConsumerWarps);
+        const int n4 = G * D / 4;
+        float4 *dst = reinterpret_cast<float4 *>(&s_qf[0][0]);
+        if (f32) {
+          const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(a.q) + qrow0 * D);
+          float4 v[kMaxIt];
+#pragma unroll
+          for (int k = 0; k < kMaxIt; ++k) {
+            const int i = tid + 32 * kConsumerWarps * k;
+            if (i < n4) v[k] = src[i];
+          }
+#pragma unroll
+          for (int k = 0; k < kMaxIt; ++k) {
+            const int i = tid + 32 * kConsumerWarps * k;
+            if (i < n4) dst[i] = v[k];
+          }
+        } else {
+          const uint2 *src = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.q) + qrow0 * D);
+          uint2 v[kMaxIt];
+#pragma unroll
+          for (int k = 0; k < kMaxIt; ++k) {
+            const int i = tid + 32 * kConsumerWarps * k;
+            if (i < n4) v[k] = src[i];
+          }
+#pragma unroll
+          for (int k = 0; k < kMaxIt; ++k) {
+            const int i = tid + 32 * kConsumerWarps * k;
+            if (i < n4)
+              dst[i] = make_float4(__uint_as_float(v[k].x << 16), __uint_as_float(v[k].x & 0xffff0000u),
+                                   __uint_as_float(v[k].y << 16), __uint_as_float(v[k].y & 0xffff0000u));
+          }
+        }
+        consumer_sync();
+      }
       float c[NTW][4];
 #pragma unroll
       for (int nt = 0; nt < NTW; ++nt)
@@ -374,15 +414,9 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
           const int row = r + 8 * (e & 1), col = 16 * ks + 8 * (e >> 1) + 2 * q;
           float x0 = 0.f, x1 = 0.f;
           if (row < G) {
-            if (f32) {
-              const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(a.q) + (qrow0 + row) * D + col);
-              x0 = v.x;
-              x1 = v.y;
-            } else {
-              const uint32_t v = *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.q) + (qrow0 + row) * D + col);
-              x0 = __uint_as_float(v << 16);
-              x1 = __uint_as_float(v & 0xffff0000u);
-            }
+            const float2 v = *reinterpret_cast<const float2 *>(&s_qf[row][col]);
+            x0 = v.x;
+            x1 = v.y;
           }
           split_bf16x2(x0, x1, ahi[e], alo[e]);
         }
