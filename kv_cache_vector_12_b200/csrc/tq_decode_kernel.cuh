@@ -265,6 +265,27 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
   // launched as a programmatic dependent: the cache, q and seq_lens are final
   // once the previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the consumers' loads of this KV head's G query rows (contiguous, 16-byte
+  // aligned) go out first, beside the length's: they do not depend on it
+  constexpr int kQIt = (kRows * DH / 4 + 32 * kConsumerWarps - 1) / (32 * kConsumerWarps);
+  const int q_n4 = G * DH / 4;
+  const bool q_f32 = a.q_dtype == TQ_F32;
+  uint4 q_v[kQIt];  // raw: four fp32, or four bf16 in .x, .y (converted when stored)
+  if (warp < kConsumerWarps) {
+    const long q_off = ((long)s * a.n_q_heads + (long)h * G) * DH;
+#pragma unroll
+    for (int k = 0; k < kQIt; ++k) {
+      const int i = tid + 32 * kConsumerWarps * k;
+      if (i < q_n4) {
+        if (q_f32) {
+          q_v[k] = reinterpret_cast<const uint4 *>(static_cast<const float *>(a.q) + q_off)[i];
+        } else {
+          const uint2 u = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.q) + q_off)[i];
+          q_v[k] = make_uint4(u.x, u.y, 0u, 0u);
+        }
+      }
+    }
+  }
   int len = a.seq_lens[s];
   if (len < 0 || len > a.max_seq_len) {
     if (tid == 0 && split == 0 && h == 0) atomicOr(a.p.err, kErrSeqLen);
@@ -363,40 +384,19 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
     {
       const long qrow0 = (long)s * a.n_q_heads + (long)h * G;
       const bool f32 = a.q_dtype == TQ_F32;
-      // the G query rows (contiguous, 16-byte aligned) into shared memory,
-      // every load issued before any is used: one memory round trip for
-      // the prologue instead of one per k-step
+      // the G query rows, loaded right after the dependency wait, into
+      // shared memory
       {
-        constexpr int kMaxIt = (kRows * D / 4 + 32 * kConsumerWarps - 1) / (32 * kConsumerWarps);
-        const int n4 = G * D / 4;
         float4 *dst = reinterpret_cast<float4 *>(&s_qf[0][0]);
-        if (f32) {
-          const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(a.q) + qrow0 * D);
-          float4 v[kMaxIt];
 #pragma unroll
-          for (int k = 0; k < kMaxIt; ++k) {
-            const int i = tid + 32 * kConsumerWarps * k;
-            if (i < n4) v[k] = src[i];
-          }
-#pragma unroll
-          for (int k = 0; k < kMaxIt; ++k) {
-            const int i = tid + 32 * kConsumerWarps * k;
-            if (i < n4) dst[i] = v[k];
-          }
-        } else {
-          const uint2 *src = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.q) + qrow0 * D);
-          uint2 v[kMaxIt];
-#pragma unroll
-          for (int k = 0; k < kMaxIt; ++k) {
-            const int i = tid + 32 * kConsumerWarps * k;
-            if (i < n4) v[k] = src[i];
-          }
-#pragma unroll
-          for (int k = 0; k < kMaxIt; ++k) {
-            const int i = tid + 32 * kConsumerWarps * k;
-            if (i < n4)
-              dst[i] = make_float4(__uint_as_float(v[k].x << 16), __uint_as_float(v[k].x & 0xffff0000u),
-                                   __uint_as_float(v[k].y << 16), __uint_as_float(v[k].y & 0xffff0000u));
+        for (int k = 0; k < kQIt; ++k) {
+          const int i = tid + 32 * kConsumerWarps * k;
+          if (i < q_n4) {
+            const uint4 u = q_v[k];
+            dst[i] = q_f32 ? make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                                         __uint_as_float(u.w))
+                           : make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                         __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
           }
         }
         consumer_sync();
