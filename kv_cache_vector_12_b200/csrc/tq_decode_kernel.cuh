@@ -262,6 +262,16 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
       }
     }
   }
+  // the stage barriers (shared memory only) are set up before the wait
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), kConsumerWarps);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
   // launched as a programmatic dependent: the cache, q and seq_lens are final
   // once the previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -296,16 +306,6 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
   const int t1 = min(len, t0 + a.chunk);
   const int n_stage = (t1 - t0 + kStageTokens - 1) / kStageTokens;
   const long base = ((long)s * a.c.n_kv_heads + h) * a.c.capacity;
-
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&full_bar[i]), 1);
-      mbar_init(smem_u32(&empty_bar[i]), kConsumerWarps);
-    }
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
 
   if (warp == kConsumerWarps) {
     // ---------------- producer: one elected lane issues the bulk copies

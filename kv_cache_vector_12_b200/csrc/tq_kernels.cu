@@ -139,13 +139,14 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
   const bool qjl = !is_v && p.qjl;
   const long row = blockIdx.x;
   const int t = (int)(row / c.n_kv_heads), h = (int)(row % c.n_kv_heads);
+  // the input is loaded beside the indices, not after the destination check
+  const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * DH + tid]);
   // (no index arrays: token t goes to position t of sequence 0)
   const long slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, h, pos ? pos[t] : t);
   if (slot < 0) {
     if (tid == 0 && !is_v) atomicOr(p.err, kErrTokenRange);
     return;
   }
-  const float x = bf16_bits_to_f32((is_v ? v_in : k_in)[row * DH + tid]);
   s_x[tid] = x;
   const float n = sqrtf(block_sum<DH>(x * x, red));  // also orders s_x
   // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
