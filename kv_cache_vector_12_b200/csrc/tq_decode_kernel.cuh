@@ -501,7 +501,7 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
           for (int e = 0; e < 4; ++e) cq[nt][e] = 0.f;
         const uint4 *sjf = reinterpret_cast<const uint4 *>(a.p.sjkf);
         constexpr int kPart = (D / 8) * CHQ * 32;  // uint4 per part
-#pragma unroll 1
+#pragma unroll 2
         for (int j = 0; j < CHQ; ++j) {
           uint32_t ah[2][4], al[2][4];  // A fragments of k-steps 2 j, 2 j + 1
 #pragma unroll
