@@ -14,6 +14,7 @@
 #include <cmath>
 
 #include "tq_cache_slot.cuh"
+#include "tq_f32x2.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -191,8 +192,11 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 // row of Pi and of S is read once per R vectors (the per-row kernel reads all
 // of S, d x d fp32, for every vector), and every broadcast shared-memory load
 // of a vector's coordinates feeds C rows of Pi or S.  The R vectors sit in
-// shared memory as fp32 (x, then z, then the residuals r in the same buffer);
-// the norms and ||r|| are warp reductions, one vector per warp in turn.  A
+// shared memory as fp32 (x, then z, then the residuals r in the same buffer),
+// interleaved by pairs (vectors 2 j and 2 j + 1 alternate coordinate by
+// coordinate), so that one packed f32x2 FMA advances a row of Pi or S against
+// both vectors of a pair, each lane rounding as the scalar FMA would; the
+// norms and ||r|| are warp reductions, one vector per warp in turn.  A
 // coordinate block of 32 (one word of the cache layout per bit, one word of
 // sign bits) belongs to warp w = block % (d / 32 C).  grid = ceil(rows / R).
 // ---------------------------------------------------------------------------
@@ -202,7 +206,9 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
                                                                    const int32_t *__restrict__ seq_idx,
                                                                    const int32_t *__restrict__ pos, long n_rows) {
   constexpr int kThreads = DH / C, kWarps = kThreads / 32;
-  __shared__ __align__(16) float s_v[R][DH];  // x, then z, then r
+  static_assert(R % 2 == 0, "vectors are held in pairs");
+  __shared__ __align__(16) float s_v[R / 2][DH][2];  // x, then z, then r; vector r at [r / 2][.][r % 2]
+  auto V = [&](int r, int i) -> float & { return s_v[r >> 1][i][r & 1]; };
   __shared__ float s_n[R], s_g[R];
   __shared__ long s_slot[R];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
     const long row = row0 + r;
 #pragma unroll
     for (int h = 0; h < C; ++h)
-      s_v[r][tid + h * kThreads] = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid + h * kThreads]) : 0.f;
+      V(r, tid + h * kThreads) = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid + h * kThreads]) : 0.f;
   }
   if (tid < R) {
     const long row = row0 + tid;
@@ -236,16 +242,16 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
   for (int r = warp; r < R; r += kWarps) {  // ||x||, fp32 over exact bf16 squares
     float v = 0.f;
 #pragma unroll
-    for (int j = lane; j < DH; j += 32) v = fmaf(s_v[r][j], s_v[r][j], v);
+    for (int j = lane; j < DH; j += 32) v = fmaf(V(r, j), V(r, j), v);
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_n[r] = sqrtf(v);
   }
-  // z_i = (Pi x)_i of the R vectors: rows i of Pi against each vector
-  float acc[C][R];
+  // z_i = (Pi x)_i of the R vectors: rows i of Pi against each pair of vectors
+  float2 acc[C][R / 2];
 #pragma unroll
   for (int h = 0; h < C; ++h)
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[h][r] = 0.f;
+    for (int j = 0; j < R / 2; ++j) acc[h][j] = make_float2(0.f, 0.f);
 #pragma unroll(DH <= 128 ? DH / 8 : 1)
   for (int c8 = 0; c8 < DH / 8; ++c8) {
     float pf[C][8];
@@ -260,27 +266,27 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
       }
     }
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const float4 x0 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8]);
-      const float4 x1 = *reinterpret_cast<const float4 *>(&s_v[r][8 * c8 + 4]);
+    for (int j = 0; j < R / 2; ++j) {
+      // coordinates 8 c8 .. 8 c8 + 7 of vectors 2 j and 2 j + 1
+      const float4 *xp = reinterpret_cast<const float4 *>(&s_v[j][8 * c8][0]);
+      const float4 x[4] = {xp[0], xp[1], xp[2], xp[3]};
 #pragma unroll
-      for (int h = 0; h < C; ++h) {
-        acc[h][r] = fmaf(pf[h][0], x0.x, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][1], x0.y, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][2], x0.z, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][3], x0.w, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][4], x1.x, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][5], x1.y, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][6], x1.z, acc[h][r]);
-        acc[h][r] = fmaf(pf[h][7], x1.w, acc[h][r]);
-      }
+      for (int h = 0; h < C; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[h][j] = fma2(make_float2(pf[h][2 * e], pf[h][2 * e]), make_float2(x[e].x, x[e].y), acc[h][j]);
+          acc[h][j] = fma2(make_float2(pf[h][2 * e + 1], pf[h][2 * e + 1]), make_float2(x[e].z, x[e].w), acc[h][j]);
+        }
     }
   }
   __syncthreads();  // every thread is done with x: the buffer takes z, then r
 #pragma unroll
   for (int h = 0; h < C; ++h)
 #pragma unroll
-    for (int r = 0; r < R; ++r) s_v[r][tid + h * kThreads] = acc[h][r];
+    for (int j = 0; j < R / 2; ++j) {
+      V(2 * j, tid + h * kThreads) = acc[h][j].x;
+      V(2 * j + 1, tid + h * kThreads) = acc[h][j].y;
+    }
   constexpr int half = 1 << (BK - 1);
   const float *cent = p.cb;
   float thr[half - 1];  // the positive thresholds
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
 #pragma unroll
     for (int h = 0; h < C; ++h) {
       const int i = tid + h * kThreads;
-      const float z = live ? s_v[r][i] : 0.f;
+      const float z = live ? V(r, i) : 0.f;
       const float a = fabsf(z);
       int m = 0;
 #pragma unroll
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
         if (lane == 0 && slot >= 0) dst[(i >> 5) * BK + wd] = word;
       }
       const float y = live ? z / n : 0.f;
-      s_v[r][i] = y - cent[code];
+      V(r, i) = y - cent[code];
     }
     if (tid == 0 && slot >= 0) c.norm_k[slot] = f32_to_f16_bits_sat(n);
   }
@@ -333,29 +339,30 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
   for (int r = warp; r < R; r += kWarps) {  // ||r||
     float v = 0.f;
 #pragma unroll
-    for (int j = lane; j < DH; j += 32) v = fmaf(s_v[r][j], s_v[r][j], v);
+    for (int j = lane; j < DH; j += 32) v = fmaf(V(r, j), V(r, j), v);
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_g[r] = sqrtf(v);
   }
-  // (S r)_i of the R residuals: rows i of S (fp32) against each residual
+  // (S r)_i of the R residuals: rows i of S (fp32) against each pair of residuals
 #pragma unroll
   for (int h = 0; h < C; ++h)
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[h][r] = 0.f;
+    for (int j = 0; j < R / 2; ++j) acc[h][j] = make_float2(0.f, 0.f);
 #pragma unroll 2
   for (int c4 = 0; c4 < DH / 4; ++c4) {
     float4 w[C];
 #pragma unroll
     for (int h = 0; h < C; ++h) w[h] = reinterpret_cast<const float4 *>(p.s + (size_t)(tid + h * kThreads) * DH)[c4];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const float4 x = *reinterpret_cast<const float4 *>(&s_v[r][4 * c4]);
+    for (int j = 0; j < R / 2; ++j) {
+      const float4 *xp = reinterpret_cast<const float4 *>(&s_v[j][4 * c4][0]);
+      const float4 x0 = xp[0], x1 = xp[1];
 #pragma unroll
       for (int h = 0; h < C; ++h) {
-        acc[h][r] = fmaf(w[h].x, x.x, acc[h][r]);
-        acc[h][r] = fmaf(w[h].y, x.y, acc[h][r]);
-        acc[h][r] = fmaf(w[h].z, x.z, acc[h][r]);
-        acc[h][r] = fmaf(w[h].w, x.w, acc[h][r]);
+        acc[h][j] = fma2(make_float2(w[h].x, w[h].x), make_float2(x0.x, x0.y), acc[h][j]);
+        acc[h][j] = fma2(make_float2(w[h].y, w[h].y), make_float2(x0.z, x0.w), acc[h][j]);
+        acc[h][j] = fma2(make_float2(w[h].z, w[h].z), make_float2(x1.x, x1.y), acc[h][j]);
+        acc[h][j] = fma2(make_float2(w[h].w, w[h].w), make_float2(x1.z, x1.w), acc[h][j]);
       }
     }
   }
@@ -365,7 +372,7 @@ __global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams 
     const long slot = s_slot[r];
 #pragma unroll
     for (int h = 0; h < C; ++h) {
-      const uint32_t sb = __ballot_sync(0xffffffffu, acc[h][r] >= 0.f);
+      const uint32_t sb = __ballot_sync(0xffffffffu, ((r & 1) ? acc[h][r >> 1].y : acc[h][r >> 1].x) >= 0.f);
       if (slot >= 0 && lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp + h * kWarps] = sb;
     }
     if (slot >= 0 && tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(s_g[r]);
