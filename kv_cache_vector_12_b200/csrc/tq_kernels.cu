@@ -1,8 +1,8 @@
 // TurboQuant quantize-on-append for sm_100a, small batches and QJL rows:
 // norm, rotation by Pi, Lloyd-Max codes, bit-pack, optional QJL residual
-// signs (one CTA per vector, or 32 vectors per CTA for batches of K rows with
-// QJL at head dimension 256); and the dispatch between these kernels and the
-// tensor-core kernels.
+// signs (one CTA per vector; batches of K rows with QJL at head dimension 256
+// on mma.sync tensor cores, 64 vectors per CTA); and the dispatch between
+// these kernels and the tcgen05 kernels.
 //
 // The method: ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み"
 // (rotation + per-coordinate Lloyd-Max, then the 1-bit QJL residual
@@ -11,11 +11,13 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 
 #include "tq_cache_slot.cuh"
 #include "tq_f32x2.cuh"
 #include "tq_internal.h"
+#include "tq_stream.cuh"
 
 namespace tq {
 namespace {
@@ -186,199 +188,284 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 }
 
 // ---------------------------------------------------------------------------
-// K rows with QJL in batches at head dimension 256 (d = 64 and 128 batches run
-// on the tcgen05 QJL kernel): the per-row kernel's arithmetic for R vectors per
-// CTA.  Thread t owns coordinates t + h d / C (h < C) of all R vectors, so each
-// row of Pi and of S is read once per R vectors (the per-row kernel reads all
-// of S, d x d fp32, for every vector), and every broadcast shared-memory load
-// of a vector's coordinates feeds C rows of Pi or S.  The R vectors sit in
-// shared memory as fp32 (x, then z, then the residuals r in the same buffer),
-// interleaved by pairs (vectors 2 j and 2 j + 1 alternate coordinate by
-// coordinate), so that one packed f32x2 FMA advances a row of Pi or S against
-// both vectors of a pair, each lane rounding as the scalar FMA would; the
-// norms and ||r|| are warp reductions, one vector per warp in turn.  A
-// coordinate block of 32 (one word of the cache layout per bit, one word of
-// sign bits) belongs to warp w = block % (d / 32 C).  grid = ceil(rows / R).
+// K rows with QJL in batches at head dimension 256 on the mma.sync tensor
+// cores (Pi, S hi and S lo at d = 256 do not fit in shared memory beside a
+// tcgen05 tile ring).  A CTA takes 64 vectors (four m-tiles of 16); warp w
+// owns output coordinates 64 w .. 64 w + 63 in two chunks of 32, each one
+// coordinate block of the cache layout (BK words of codes, one word of signs).
+//   z = X Pi^T on m16n8k16 bf16 (exact products, fp32 sums): A = the bf16
+//   rows from shared memory (ldmatrix), B = Pi's bf16 fragment table;
+//   the codes, the packed words and r = z / ||x|| - c[code] come straight
+//   from the accumulator fragments (the four lanes of a quad hold a row's 32
+//   coordinates of the chunk, and OR-reduce its words);
+//   S r with r 2^14 and S 2^sigma as two-part fp16 splits, three m16n8k16
+//   f16 products (hi hi, hi lo, lo hi: about 22 significant bits, of which
+//   only the sign is kept; both scales are positive): A = the split
+//   residuals of all four warps from shared memory, B = S's fragment tables.
+// grid = ceil(rows / 64), 128 threads, two CTAs per SM.
 // ---------------------------------------------------------------------------
-template <int DH, int R, int BK, int C>
-__global__ void __launch_bounds__(DH / C) quantize_qjl_rows_kernel(DeviceParams p, tq_cache c,
-                                                                   const uint16_t *__restrict__ k_in,
-                                                                   const int32_t *__restrict__ seq_idx,
-                                                                   const int32_t *__restrict__ pos, long n_rows) {
-  constexpr int kThreads = DH / C, kWarps = kThreads / 32;
-  static_assert(R % 2 == 0, "vectors are held in pairs");
-  __shared__ __align__(16) float s_v[R / 2][DH][2];  // x, then z, then r; vector r at [r / 2][.][r % 2]
-  auto V = [&](int r, int i) -> float & { return s_v[r >> 1][i][r & 1]; };
-  __shared__ float s_n[R], s_g[R];
-  __shared__ long s_slot[R];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long row0 = (long)blockIdx.x * R;
-  PiRow<DH> pw[C];
+constexpr int kQmM = 64;        // vectors per CTA
+constexpr int kQmLd = 256 + 8;  // row stride in 16-bit elements: 528 B puts ldmatrix rows on distinct banks
+constexpr int kQmSmem = kQmM * kQmLd * 2 * 3 + kQmM * (4 + 16 + 8) + 16 * 4;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+
+// OR the code of in-block coordinate 8 jn + pe (jn < 4, pe < 8) into the BK
+// words of its 32-coordinate block (the cache layout: LSB-first for 2 and 4
+// bits; nibbles for the first 24 coordinates and the spare column of the
+// nibbles' top bits for the last 8 at 3 bits)
+template <int BK>
+__device__ __forceinline__ void or_code(uint32_t (&w)[BK], int jn, int pe, uint32_t code) {
+  if constexpr (BK == 2) {
+    w[jn >> 1] |= code << (16 * (jn & 1) + 2 * pe);
+  } else if constexpr (BK == 4) {
+    w[jn] |= code << (4 * pe);
+  } else {
+    if (jn < 3) {
+      w[jn < 3 ? jn : 0] |= code << (4 * pe);
+    } else {
 #pragma unroll
-  for (int h = 0; h < C; ++h) pw[h].load(p.pi + (tid + h * kThreads) * DH);
+      for (int k = 0; k < 3; ++k) w[k] |= ((code >> k) & 1u) << (4 * pe + 3);
+    }
+  }
+}
+
+template <int BK>
+__global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParams p, tq_cache c,
+                                                                      const uint16_t *__restrict__ k_in,
+                                                                      const int32_t *__restrict__ seq_idx,
+                                                                      const int32_t *__restrict__ pos, long n_rows) {
+  constexpr int DH = 256, M = kQmM, LD = kQmLd;
+  extern __shared__ __align__(16) unsigned char qm_smem[];
+  uint16_t *s_x = reinterpret_cast<uint16_t *>(qm_smem);   // [M][LD] bf16 rows
+  uint16_t *s_rh = s_x + M * LD;                             // [M][LD] fp16 hi of r 2^14
+  uint16_t *s_rl = s_rh + M * LD;                            // [M][LD] fp16 lo
+  float *s_n = reinterpret_cast<float *>(s_rl + M * LD);     // [M] ||x||
+  float *s_gp = s_n + M;                                     // [4][M] the warps' parts of ||r||^2
+  long *s_slot = reinterpret_cast<long *>(s_gp + 4 * M);     // [M]
+  float *s_cent = reinterpret_cast<float *>(s_slot + M);     // [16] K centroids
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  const long row0 = (long)blockIdx.x * M;
+  if (tid < 16) s_cent[tid] = p.cb[tid];
   // launched as a programmatic dependent: no input is read before the
   // previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-#pragma unroll 4
-  for (int r = 0; r < R; ++r) {  // rows past the end are zero vectors that are never stored
-    const long row = row0 + r;
+  {  // the 64 rows in 16-byte pieces (32 per row), every load issued first; rows past the end are zero
+    uint4 v[16];
 #pragma unroll
-    for (int h = 0; h < C; ++h)
-      V(r, tid + h * kThreads) = row < n_rows ? bf16_bits_to_f32(k_in[row * DH + tid + h * kThreads]) : 0.f;
+    for (int k = 0; k < 16; ++k) {
+      const int idx = tid + 128 * k;
+      const long row = row0 + (idx >> 5);
+      v[k] = row < n_rows ? reinterpret_cast<const uint4 *>(k_in + row * DH)[idx & 31] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int idx = tid + 128 * k;
+      *reinterpret_cast<uint4 *>(s_x + (idx >> 5) * LD + 8 * (idx & 31)) = v[k];
+    }
   }
-  if (tid < R) {
+  if (tid < M) {
     const long row = row0 + tid;
     long slot = -1;
     if (row < n_rows) {
-      const int t = (int)(row / c.n_kv_heads), hd = (int)(row % c.n_kv_heads);
+      const int tk = (int)(row / c.n_kv_heads), hd = (int)(row % c.n_kv_heads);
       // (no index arrays: token t goes to position t of sequence 0)
-      slot = cache_slot(c, seq_idx ? seq_idx[t] : 0, hd, pos ? pos[t] : t);
+      slot = cache_slot(c, seq_idx ? seq_idx[tk] : 0, hd, pos ? pos[tk] : tk);
       if (slot < 0 && hd == 0) atomicOr(p.err, kErrTokenRange);
     }
     s_slot[tid] = slot;
   }
   __syncthreads();
-  for (int r = warp; r < R; r += kWarps) {  // ||x||, fp32 over exact bf16 squares
+  // ||x||, fp32 over exact bf16 squares: warp w takes rows 16 w .. 16 w + 15
+  for (int rr = 0; rr < 16; ++rr) {
+    const int r = 16 * warp + rr;
+    const uint4 u = *reinterpret_cast<const uint4 *>(s_x + r * LD + 8 * lane);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
     float v = 0.f;
 #pragma unroll
-    for (int j = lane; j < DH; j += 32) v = fmaf(V(r, j), V(r, j), v);
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
+      v = fmaf(lo, lo, v);
+      v = fmaf(hi, hi, v);
+    }
+#pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_n[r] = sqrtf(v);
   }
-  // z_i = (Pi x)_i of the R vectors: rows i of Pi against each pair of vectors
-  float2 acc[C][R / 2];
-#pragma unroll
-  for (int h = 0; h < C; ++h)
-#pragma unroll
-    for (int j = 0; j < R / 2; ++j) acc[h][j] = make_float2(0.f, 0.f);
-#pragma unroll(DH <= 128 ? DH / 8 : 1)
-  for (int c8 = 0; c8 < DH / 8; ++c8) {
-    float pf[C][8];
-#pragma unroll
-    for (int h = 0; h < C; ++h) {
-      const uint4 w = pw[h].get(c8);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        pf[h][2 * e] = __uint_as_float(u[e] << 16);
-        pf[h][2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < R / 2; ++j) {
-      // coordinates 8 c8 .. 8 c8 + 7 of vectors 2 j and 2 j + 1
-      const float4 *xp = reinterpret_cast<const float4 *>(&s_v[j][8 * c8][0]);
-      const float4 x[4] = {xp[0], xp[1], xp[2], xp[3]};
-#pragma unroll
-      for (int h = 0; h < C; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc[h][j] = fma2(make_float2(pf[h][2 * e], pf[h][2 * e]), make_float2(x[e].x, x[e].y), acc[h][j]);
-          acc[h][j] = fma2(make_float2(pf[h][2 * e + 1], pf[h][2 * e + 1]), make_float2(x[e].z, x[e].w), acc[h][j]);
-        }
-    }
-  }
-  __syncthreads();  // every thread is done with x: the buffer takes z, then r
-#pragma unroll
-  for (int h = 0; h < C; ++h)
-#pragma unroll
-    for (int j = 0; j < R / 2; ++j) {
-      V(2 * j, tid + h * kThreads) = acc[h][j].x;
-      V(2 * j + 1, tid + h * kThreads) = acc[h][j].y;
-    }
+  __syncthreads();
+
   constexpr int half = 1 << (BK - 1);
-  const float *cent = p.cb;
   float thr[half - 1];  // the positive thresholds
 #pragma unroll
   for (int j = 0; j < half - 1; ++j) thr[j] = p.cb[1 * kMaxLevels + half + j];
-  // this thread's bit positions inside the BK words of its coordinate blocks
-  // (the cache layout: LSB-first for 2 and 4 bits, nibbles plus the spare
-  // column for 3 bits)
-  int wd_of[C][BK], sh_of[C][BK];
+  // this lane's ldmatrix address: row lane % 16 of an m-tile, columns 8 (lane / 16) of a k-step
+  const uint32_t a_off = (uint32_t)(((lane & 15) * LD + ((lane >> 4) << 3)) * 2);
+  const uint32_t xs = smem_u32(s_x) + a_off, rhs = smem_u32(s_rh) + a_off, rls = smem_u32(s_rl) + a_off;
+  const uint4 *pif4 = reinterpret_cast<const uint4 *>(p.pif);
+  float gs[4][2];  // this thread's part of ||r||^2 for rows 16 mt + g + 8 hf
 #pragma unroll
-  for (int h = 0; h < C; ++h)
-#pragma unroll
-    for (int kb = 0; kb < BK; ++kb) {
-      const int i = tid + h * kThreads;
-      const int pbit = code_bit_pos(BK, i, kb) - 32 * BK * (i >> 5);
-      wd_of[h][kb] = pbit >> 5;
-      sh_of[h][kb] = pbit & 31;
-    }
+  for (int mt = 0; mt < 4; ++mt) gs[mt][0] = gs[mt][1] = 0.f;
+
 #pragma unroll 1
-  for (int r = 0; r < R; ++r) {
-    const float n = s_n[r];
-    // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
-    const bool live = n > 0x1p-25f;
-    const long slot = s_slot[r];
-    uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + (slot < 0 ? 0 : slot) * (DH * BK / 8));
+  for (int cc = 0; cc < 2; ++cc) {
+    const int nt0 = 8 * warp + 4 * cc;  // first n-tile (8 coordinates each) of the chunk
+    float acc[4][4][4];
 #pragma unroll
-    for (int h = 0; h < C; ++h) {
-      const int i = tid + h * kThreads;
-      const float z = live ? V(r, i) : 0.f;
-      const float a = fabsf(z);
-      int m = 0;
+    for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int j = 0; j < half - 1; ++j) m += a > thr[j] * n ? 1 : 0;
-      const int code = z > 0.f ? half + m : half - 1 - m;
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int wd = 0; wd < BK; ++wd) {  // block i / 32 owns words BK (i / 32) ..
-        uint32_t contrib = 0;
-#pragma unroll
-        for (int kb = 0; kb < BK; ++kb)
-          if (wd_of[h][kb] == wd) contrib |= (uint32_t)((code >> kb) & 1) << sh_of[h][kb];
-        const uint32_t word = __reduce_or_sync(0xffffffffu, contrib);
-        if (lane == 0 && slot >= 0) dst[(i >> 5) * BK + wd] = word;
-      }
-      const float y = live ? z / n : 0.f;
-      V(r, i) = y - cent[code];
-    }
-    if (tid == 0 && slot >= 0) c.norm_k[slot] = f32_to_f16_bits_sat(n);
-  }
-  __syncthreads();
-  for (int r = warp; r < R; r += kWarps) {  // ||r||
-    float v = 0.f;
-#pragma unroll
-    for (int j = lane; j < DH; j += 32) v = fmaf(V(r, j), V(r, j), v);
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) s_g[r] = sqrtf(v);
-  }
-  // (S r)_i of the R residuals: rows i of S (fp32) against each pair of residuals
-#pragma unroll
-  for (int h = 0; h < C; ++h)
-#pragma unroll
-    for (int j = 0; j < R / 2; ++j) acc[h][j] = make_float2(0.f, 0.f);
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 #pragma unroll 2
-  for (int c4 = 0; c4 < DH / 4; ++c4) {
-    float4 w[C];
+    for (int j = 0; j < DH / 32; ++j) {  // k-steps 2 j and 2 j + 1: one 16-byte fragment load per n-tile
+      uint4 b[4];
 #pragma unroll
-    for (int h = 0; h < C; ++h) w[h] = reinterpret_cast<const float4 *>(p.s + (size_t)(tid + h * kThreads) * DH)[c4];
+      for (int nt = 0; nt < 4; ++nt) b[nt] = pif4[((nt0 + nt) * (DH / 32) + j) * 32 + lane];
 #pragma unroll
-    for (int j = 0; j < R / 2; ++j) {
-      const float4 *xp = reinterpret_cast<const float4 *>(&s_v[j][4 * c4][0]);
-      const float4 x0 = xp[0], x1 = xp[1];
+      for (int s2 = 0; s2 < 2; ++s2) {
+        uint32_t a[4][4];
 #pragma unroll
-      for (int h = 0; h < C; ++h) {
-        acc[h][j] = fma2(make_float2(w[h].x, w[h].x), make_float2(x0.x, x0.y), acc[h][j]);
-        acc[h][j] = fma2(make_float2(w[h].y, w[h].y), make_float2(x0.z, x0.w), acc[h][j]);
-        acc[h][j] = fma2(make_float2(w[h].z, w[h].z), make_float2(x1.x, x1.y), acc[h][j]);
-        acc[h][j] = fma2(make_float2(w[h].w, w[h].w), make_float2(x1.z, x1.w), acc[h][j]);
+        for (int mt = 0; mt < 4; ++mt) ldsm_x4(xs + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), a[mt]);
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+            mma_bf16(acc[mt][nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], s2 ? b[nt].z : b[nt].x,
+                     s2 ? b[nt].w : b[nt].y);
       }
     }
+    // codes, packed words and residuals of the chunk; fragment element e of
+    // n-tile nt0 + nt is row 16 mt + g + 8 (e / 2), coordinate 8 (nt0 + nt) + 2 t + e % 2
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = 16 * mt + g + 8 * hf;
+        const float n = s_n[r];
+        // a vector whose stored fp16 norm is zero (n <= 2^-25) is the zero vector
+        const bool live = n > 0x1p-25f;
+        const float inv = live ? 1.f / n : 0.f;
+        float tn[half - 1];
+#pragma unroll
+        for (int j = 0; j < half - 1; ++j) tn[j] = thr[j] * n;
+        uint32_t wds[BK];
+#pragma unroll
+        for (int k = 0; k < BK; ++k) wds[k] = 0u;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          float rv[2];
+#pragma unroll
+          for (int e1 = 0; e1 < 2; ++e1) {
+            const float z = live ? acc[mt][nt][2 * hf + e1] : 0.f;
+            const float a = fabsf(z);
+            int m = 0;
+#pragma unroll
+            for (int j = 0; j < half - 1; ++j) m += a > tn[j] ? 1 : 0;
+            const int code = z > 0.f ? half + m : half - 1 - m;
+            or_code<BK>(wds, nt, 2 * t + e1, (uint32_t)code);
+            rv[e1] = z * inv - s_cent[code];
+            gs[mt][hf] = fmaf(rv[e1], rv[e1], gs[mt][hf]);
+          }
+          uint32_t hi, lo;
+          split_f16x2(rv[0] * 16384.f, rv[1] * 16384.f, hi, lo);
+          const int col = 8 * (nt0 + nt) + 2 * t;
+          *reinterpret_cast<uint32_t *>(s_rh + r * LD + col) = hi;
+          *reinterpret_cast<uint32_t *>(s_rl + r * LD + col) = lo;
+        }
+#pragma unroll
+        for (int k = 0; k < BK; ++k) {
+          wds[k] |= __shfl_xor_sync(0xffffffffu, wds[k], 1);
+          wds[k] |= __shfl_xor_sync(0xffffffffu, wds[k], 2);
+        }
+        const long slot = s_slot[r];
+        if (t == 0 && slot >= 0) {
+          uint32_t *dst = reinterpret_cast<uint32_t *>(c.codes_k + slot * (DH * BK / 8)) + (2 * warp + cc) * BK;
+#pragma unroll
+          for (int k = 0; k < BK; ++k) dst[k] = wds[k];
+        }
+      }
   }
-  __syncthreads();  // s_g
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const long slot = s_slot[r];
+  for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-    for (int h = 0; h < C; ++h) {
-      const uint32_t sb = __ballot_sync(0xffffffffu, ((r & 1) ? acc[h][r >> 1].y : acc[h][r >> 1].x) >= 0.f);
-      if (slot >= 0 && lane == 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[warp + h * kWarps] = sb;
+    for (int hf = 0; hf < 2; ++hf) {
+      float v = gs[mt][hf];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if (t == 0) s_gp[warp * M + 16 * mt + g + 8 * hf] = v;
     }
-    if (slot >= 0 && tid == 0) c.qjl_norm[slot] = f32_to_f16_bits_sat(s_g[r]);
+  __syncthreads();  // every warp's residuals and ||r||^2 parts are in shared memory
+  if (tid < M) {
+    const long slot = s_slot[tid];
+    if (slot >= 0) {
+      c.norm_k[slot] = f32_to_f16_bits_sat(s_n[tid]);
+      const float g2 = (s_gp[tid] + s_gp[M + tid]) + (s_gp[2 * M + tid] + s_gp[3 * M + tid]);
+      c.qjl_norm[slot] = f32_to_f16_bits_sat(sqrtf(g2));
+    }
+  }
+  const uint4 *sf4 = reinterpret_cast<const uint4 *>(p.sf);
+  constexpr int kLoPart = DH * DH / 8;  // the lo table, in 16-byte units
+#pragma unroll 1
+  for (int cc = 0; cc < 2; ++cc) {
+    const int nt0 = 8 * warp + 4 * cc;
+    float acc[4][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < DH / 32; ++j) {
+      uint4 bh[4], bl[4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        bh[nt] = sf4[((nt0 + nt) * (DH / 32) + j) * 32 + lane];
+        bl[nt] = sf4[kLoPart + ((nt0 + nt) * (DH / 32) + j) * 32 + lane];
+      }
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        uint32_t ah[4][4], al[4][4];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          ldsm_x4(rhs + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), ah[mt]);
+          ldsm_x4(rls + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), al[mt]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const uint32_t h0 = s2 ? bh[nt].z : bh[nt].x, h1 = s2 ? bh[nt].w : bh[nt].y;
+            const uint32_t l0 = s2 ? bl[nt].z : bl[nt].x, l1 = s2 ? bl[nt].w : bl[nt].y;
+            mma_f16(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], h0, h1);
+            mma_f16(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], l0, l1);
+            mma_f16(acc[mt][nt], al[mt][0], al[mt][1], al[mt][2], al[mt][3], h0, h1);
+          }
+      }
+    }
+    // sign of (S r)_i, i = 8 (nt0 + nt) + 2 t + e % 2: bit i % 32 of word i / 32 = 2 w + cc
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sb = 0u;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e1 = 0; e1 < 2; ++e1)
+            sb |= (acc[mt][nt][2 * hf + e1] >= 0.f ? 1u : 0u) << (8 * nt + 2 * t + e1);
+        sb |= __shfl_xor_sync(0xffffffffu, sb, 1);
+        sb |= __shfl_xor_sync(0xffffffffu, sb, 2);
+        const long slot = s_slot[16 * mt + g + 8 * hf];
+        if (t == 0 && slot >= 0) reinterpret_cast<uint32_t *>(c.qjl_bits + slot * (DH / 8))[2 * warp + cc] = sb;
+      }
   }
 }
-
 }  // namespace
 
 // Batches of up to kRowKernelMaxRows rows per matrix (decode-time appends) use
@@ -405,8 +492,8 @@ int launch_quantize(const DeviceParams &p, const tq_cache &c, const void *k, con
     // tcgen05 kernels: at d = 64 the MSE kernel (tq_quantize_tc.cu) or, with
     // QJL, the QJL kernel (tq_quantize_qjl_tc.cu), both templated on d; at
     // d = 256 the MSE kernel of tq_quantize_tc256.cu for V and for K without
-    // QJL, and the batched QJL kernel above for K with QJL (Pi, S hi and S lo
-    // at d = 256 do not fit in shared memory beside a tile ring)
+    // QJL, and the mma.sync QJL kernel above for K with QJL (Pi, S hi and
+    // S lo at d = 256 do not fit in shared memory beside a tile ring)
     if (rows <= kRowKernelMaxRows) {
       cfg.gridDim = dim3((unsigned)rows, 2);
       cfg.blockDim = dim3(p.d);
@@ -441,16 +528,23 @@ int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void 
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k;
-  if (p.d == 256 && p.qjl) {  // R = 32 vectors per CTA, two coordinates per thread
-    constexpr int R = 32;
-    cfg.gridDim = dim3((unsigned)((rows + R - 1) / R));
+  if (p.d == 256 && p.qjl) {  // 64 vectors per CTA on the mma.sync tensor cores
+    cfg.gridDim = dim3((unsigned)((rows + kQmM - 1) / kQmM));
     cfg.blockDim = dim3(128);
-    using QjlRowsFn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, long);
-    const QjlRowsFn fn = p.bits_k == 2   ? quantize_qjl_rows_kernel<256, R, 2, 2>
-                         : p.bits_k == 3 ? quantize_qjl_rows_kernel<256, R, 3, 2>
-                                         : quantize_qjl_rows_kernel<256, R, 4, 2>;
-    // the largest shared-memory carveout: the CTAs per SM are then bounded by registers only
-    cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cfg.dynamicSmemBytes = kQmSmem;
+    using QjlMmaFn = void (*)(DeviceParams, tq_cache, const uint16_t *, const int32_t *, const int32_t *, long);
+    const QjlMmaFn fn = p.bits_k == 2   ? quantize_qjl_mma256_kernel<2>
+                        : p.bits_k == 3 ? quantize_qjl_mma256_kernel<3>
+                                        : quantize_qjl_mma256_kernel<4>;
+    // cached per device (the attribute applies to the current device), and
+    // atomically, as calls may come from several threads
+    static std::atomic<bool> configured[kMaxDevices][3];
+    std::atomic<bool> &done = configured[current_device()][p.bits_k - 2];
+    if (!done.load(std::memory_order_acquire)) {
+      const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kQmSmem);
+      if (e != cudaSuccess) return (int)e;
+      done.store(true, std::memory_order_release);
+    }
     return (int)cudaLaunchKernelEx(&cfg, fn, p, c, kk, seq_idx, pos, rows);
   }
   cfg.gridDim = dim3((unsigned)rows, 1);  // y = 0: K only
