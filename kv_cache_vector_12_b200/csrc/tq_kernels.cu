@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll 1
+#pragma unroll 2
     for (int j = 0; j < DH / 32; ++j) {
       uint4 bh[4], bl[4];
 #pragma unroll
