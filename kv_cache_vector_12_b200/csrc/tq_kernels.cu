@@ -1,7 +1,7 @@
 // TurboQuant quantize-on-append for sm_100a, small batches and QJL rows:
 // norm, rotation by Pi, Lloyd-Max codes, bit-pack, optional QJL residual
 // signs (one CTA per vector; batches of K rows with QJL at head dimension 256
-// on mma.sync tensor cores, 64 vectors per CTA); and the dispatch between
+// on mma.sync tensor cores, 32 vectors per CTA); and the dispatch between
 // these kernels and the tcgen05 kernels.
 //
 // The method: ai-accelerate.xyz TurboQuant explainer, "TurboQuantの仕組み"
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 // ---------------------------------------------------------------------------
 // K rows with QJL in batches at head dimension 256 on the mma.sync tensor
 // cores (Pi, S hi and S lo at d = 256 do not fit in shared memory beside a
-// tcgen05 tile ring).  A CTA takes 64 vectors (four m-tiles of 16); warp w
+// tcgen05 tile ring).  A CTA takes 32 vectors (two m-tiles of 16); warp w
 // owns output coordinates 64 w .. 64 w + 63 in two chunks of 32, each one
 // coordinate block of the cache layout (BK words of codes, one word of signs).
 //   z = X Pi^T on m16n8k16 bf16 (exact products, fp32 sums): A = the bf16
@@ -202,9 +202,13 @@ __global__ void __launch_bounds__(DH) quantize_row_kernel(DeviceParams p, tq_cac
 //   f16 products (hi hi, hi lo, lo hi: about 22 significant bits, of which
 //   only the sign is kept; both scales are positive): A = the split
 //   residuals of all four warps from shared memory, B = S's fragment tables.
-// grid = ceil(rows / 64), 128 threads, two CTAs per SM.
+// grid = ceil(rows / 32), 128 threads, four CTAs per SM (51 KB of shared
+// memory and at most 128 registers each): sixteen warps per SM hide more of
+// the MMA and L2 latency than eight warps with 64 vectors per CTA did, although
+// every fragment of Pi and S is then read once per 32 vectors instead of 64.
 // ---------------------------------------------------------------------------
-constexpr int kQmM = 64;        // vectors per CTA
+constexpr int kQmMT = 2;        // m-tiles of 16 vectors per CTA
+constexpr int kQmM = 16 * kQmMT;  // vectors per CTA
 constexpr int kQmLd = 256 + 8;  // row stride in 16-bit elements: 528 B puts ldmatrix rows on distinct banks
 constexpr int kQmSmem = kQmM * kQmLd * 2 * 3 + kQmM * (4 + 16 + 8) + 16 * 4;
 
@@ -235,7 +239,7 @@ __device__ __forceinline__ void or_code(uint32_t (&w)[BK], int jn, int pe, uint3
 }
 
 template <int BK>
-__global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParams p, tq_cache c,
+__global__ void __launch_bounds__(128, 4) quantize_qjl_mma256_kernel(DeviceParams p, tq_cache c,
                                                                       const uint16_t *__restrict__ k_in,
                                                                       const int32_t *__restrict__ seq_idx,
                                                                       const int32_t *__restrict__ pos, long n_rows) {
@@ -255,16 +259,16 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
   // previous kernel in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  {  // the 64 rows in 16-byte pieces (32 per row), every load issued first; rows past the end are zero
-    uint4 v[16];
+  {  // the M rows in 16-byte pieces (32 per row), every load issued first; rows past the end are zero
+    uint4 v[M / 4];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < M / 4; ++k) {
       const int idx = tid + 128 * k;
       const long row = row0 + (idx >> 5);
       v[k] = row < n_rows ? reinterpret_cast<const uint4 *>(k_in + row * DH)[idx & 31] : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < M / 4; ++k) {
       const int idx = tid + 128 * k;
       *reinterpret_cast<uint4 *>(s_x + (idx >> 5) * LD + 8 * (idx & 31)) = v[k];
     }
@@ -281,9 +285,9 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
     s_slot[tid] = slot;
   }
   __syncthreads();
-  // ||x||, fp32 over exact bf16 squares: warp w takes rows 16 w .. 16 w + 15
-  for (int rr = 0; rr < 16; ++rr) {
-    const int r = 16 * warp + rr;
+  // ||x||, fp32 over exact bf16 squares: warp w takes rows M w / 4 .. M (w + 1) / 4 - 1
+  for (int rr = 0; rr < M / 4; ++rr) {
+    const int r = (M / 4) * warp + rr;
     const uint4 u = *reinterpret_cast<const uint4 *>(s_x + r * LD + 8 * lane);
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
     float v = 0.f;
@@ -307,16 +311,16 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
   const uint32_t a_off = (uint32_t)(((lane & 15) * LD + ((lane >> 4) << 3)) * 2);
   const uint32_t xs = smem_u32(s_x) + a_off, rhs = smem_u32(s_rh) + a_off, rls = smem_u32(s_rl) + a_off;
   const uint4 *pif4 = reinterpret_cast<const uint4 *>(p.pif);
-  float gs[4][2];  // this thread's part of ||r||^2 for rows 16 mt + g + 8 hf
+  float gs[kQmMT][2];  // this thread's part of ||r||^2 for rows 16 mt + g + 8 hf
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) gs[mt][0] = gs[mt][1] = 0.f;
+  for (int mt = 0; mt < kQmMT; ++mt) gs[mt][0] = gs[mt][1] = 0.f;
 
 #pragma unroll 1
   for (int cc = 0; cc < 2; ++cc) {
     const int nt0 = 8 * warp + 4 * cc;  // first n-tile (8 coordinates each) of the chunk
-    float acc[4][4][4];
+    float acc[kQmMT][4][4];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -328,11 +332,11 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
       for (int nt = 0; nt < 4; ++nt) b[nt] = pif4[((nt0 + nt) * (DH / 32) + j) * 32 + lane];
 #pragma unroll
       for (int s2 = 0; s2 < 2; ++s2) {
-        uint32_t a[4][4];
+        uint32_t a[kQmMT][4];
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) ldsm_x4(xs + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), a[mt]);
+        for (int mt = 0; mt < kQmMT; ++mt) ldsm_x4(xs + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), a[mt]);
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
           for (int nt = 0; nt < 4; ++nt)
             mma_bf16(acc[mt][nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], s2 ? b[nt].z : b[nt].x,
@@ -342,7 +346,7 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
     // codes, packed words and residuals of the chunk; fragment element e of
     // n-tile nt0 + nt is row 16 mt + g + 8 (e / 2), coordinate 8 (nt0 + nt) + 2 t + e % 2
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * mt + g + 8 * hf;
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
       }
   }
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       float v = gs[mt][hf];
@@ -413,14 +417,14 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
 #pragma unroll 1
   for (int cc = 0; cc < 2; ++cc) {
     const int nt0 = 8 * warp + 4 * cc;
-    float acc[4][4][4];
+    float acc[kQmMT][4][4];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll 2
+#pragma unroll 1
     for (int j = 0; j < DH / 32; ++j) {
       uint4 bh[4], bl[4];
 #pragma unroll
@@ -430,14 +434,14 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
       }
 #pragma unroll
       for (int s2 = 0; s2 < 2; ++s2) {
-        uint32_t ah[4][4], al[4][4];
+        uint32_t ah[kQmMT][4], al[kQmMT][4];
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int mt = 0; mt < kQmMT; ++mt) {
           ldsm_x4(rhs + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), ah[mt]);
           ldsm_x4(rls + (uint32_t)((mt * 16 * LD + (2 * j + s2) * 16) * 2), al[mt]);
         }
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
           for (int nt = 0; nt < 4; ++nt) {
             const uint32_t h0 = s2 ? bh[nt].z : bh[nt].x, h1 = s2 ? bh[nt].w : bh[nt].y;
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(128, 2) quantize_qjl_mma256_kernel(DeviceParam
     }
     // sign of (S r)_i, i = 8 (nt0 + nt) + 2 t + e % 2: bit i % 32 of word i / 32 = 2 w + cc
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < kQmMT; ++mt)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t sb = 0u;
@@ -528,7 +532,7 @@ int launch_quantize_rows_k(const DeviceParams &p, const tq_cache &c, const void 
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   const uint16_t *kk = (const uint16_t *)k;
-  if (p.d == 256 && p.qjl) {  // 64 vectors per CTA on the mma.sync tensor cores
+  if (p.d == 256 && p.qjl) {  // 32 vectors per CTA on the mma.sync tensor cores
     cfg.gridDim = dim3((unsigned)((rows + kQmM - 1) / kQmM));
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = kQmSmem;
