@@ -827,10 +827,12 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
             pb[rb][nt][1] = movmatrix_trans(pack_half2(sc[2 * rb + 1][0], sc[2 * rb + 1][1]));
           }
         }
-        // the long-split build rescales unconditionally (alpha = 1 is exact):
-        // no vote, and no branch between the softmax and the value expansion
-        // to stop the scheduler from interleaving them
-        if (CTAS == 3 || __any_sync(0xffffffffu, rescale)) {
+        // the long-split build with 3-bit V rescales unconditionally (alpha =
+        // 1 is exact): no vote, and no branch between the softmax and the
+        // value expansion (longest at 3 bits, with the spare-column gather)
+        // to stop the scheduler from interleaving them; at 2 and 4 bits the
+        // vote, which skips the multiplies, measured faster
+        if ((CTAS == 3 && BV == 3) || __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
