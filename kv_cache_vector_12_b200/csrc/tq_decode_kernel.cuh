@@ -830,8 +830,9 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
         // the long-split build with 3-bit V rescales unconditionally (alpha =
         // 1 is exact): no vote, and no branch between the softmax and the
         // value expansion (longest at 3 bits, with the spare-column gather)
-        // to stop the scheduler from interleaving them; at 2 and 4 bits the
-        // vote, which skips the multiplies, measured faster
+        // to stop the scheduler from interleaving them; at 2/2 and 4/4 bits,
+        // and 4/4 with QJL, the vote, which skips the multiplies, measured
+        // faster (2/2 with QJL: 0.5 % slower, within the rule's simplicity)
         if ((CTAS == 3 && BV == 3) || __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
