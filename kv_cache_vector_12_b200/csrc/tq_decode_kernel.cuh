@@ -827,13 +827,15 @@ __global__ void __maxnreg__(CTAS == 3 ? 128 : 168) decode_mma_kernel(const Decod
             pb[rb][nt][1] = movmatrix_trans(pack_half2(sc[2 * rb + 1][0], sc[2 * rb + 1][1]));
           }
         }
-        // the long-split build with 3-bit V rescales unconditionally (alpha =
-        // 1 is exact): no vote, and no branch between the softmax and the
-        // value expansion (longest at 3 bits, with the spare-column gather)
-        // to stop the scheduler from interleaving them; at 2/2 and 4/4 bits,
-        // and 4/4 with QJL, the vote, which skips the multiplies, measured
-        // faster (2/2 with QJL: 0.5 % slower, within the rule's simplicity)
-        if ((CTAS == 3 && BV == 3) || __any_sync(0xffffffffu, rescale)) {
+        // with 3-bit V the long-split build, and the d = 256 build without
+        // QJL, rescale unconditionally (alpha = 1 is exact): no vote, and no
+        // branch between the softmax and the value expansion (longest at 3
+        // bits, with the spare-column gather) to stop the scheduler from
+        // interleaving them.  Elsewhere the vote, which skips the multiplies,
+        // measured faster: at 2/2 and 4/4 bits, 4/4 with QJL, and d = 256 with
+        // QJL (2/2 with QJL: 0.5 % slower, within the rule's simplicity)
+        constexpr bool kNoVote = BV == 3 && (CTAS == 3 || (DH == 256 && !QJL));
+        if (kNoVote || __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
